@@ -1,0 +1,472 @@
+"""Throughput of the chunkwise mLSTM forward pass on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--algo auto|simt|tc|tc_fused] [--impl ours|reference]
+
+One step = one full forward pass (gates -> chunk states -> outputs, or the
+fused kernel) over one batch of the workload, inputs resident in HBM.  At
+N > 1 (torchrun, one process per GPU) every rank runs its own batch of the same
+shape (weak scaling: the path shards over independent (batch, head) pairs, so
+there is no collective on the data path); the timing is the max over ranks.
+
+Rank 0 prints one JSON line: tokens/s over all ranks, the TFLOP/s and roofline
+of the dominant kernel (per-kernel CUDA events on the launch stream), the e2e
+throughput through the same API with pinned host buffers and the copies inside
+the timed region, the SM clocks sampled during the timed region, and (N = 1)
+the fp64 CPU oracle timed on a bounded sample of the same workload.
+
+``--impl reference`` times that oracle alone on the host cores (the only
+other place this script runs it), on the same workload and metric.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "mLSTM fw tokens/s and TFLOP/s (% bf16 TC peak) at 7B shape, T=8192"
+L2_BYTES = 126 * 2**20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                  "sm_max_mhz": 1965.0}
+# fp32 FFMA peak for the SIMT kernels: 148 SMs x 128 lanes x 2 flop x clock.
+SIMT_LANES = 148 * 128
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as fh:
+            d = json.load(fh)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def flops_per_head(T, DK, DV, L):
+    """Algorithmic tensor-core FLOPs of one (b, h): state updates, the inter-chunk
+    Q.C term, and the causal half of the intra-chunk QK^T and P.V."""
+    return {
+        "states": 2.0 * T * DK * DV,
+        "inter": 2.0 * T * DK * DV,
+        "intra": float(T) * L * (DK + DV),
+    }
+
+
+def algorithmic_bytes(w, elem):
+    BH = w.B * w.NH
+    io = BH * w.T * (2 * w.DK + 2 * w.DV) * elem + BH * w.T * 8
+    final = BH * (w.DK * w.DV + w.DK + 1) * 4
+    init = final if w.init_state else 0
+    return io + final + init
+
+
+# ----------------------------------------------------------------------------
+# clocks during the timed region (NVML reads only; no setting is changed)
+# ----------------------------------------------------------------------------
+_REASON_BITS = {
+    "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4,
+    "hw_slowdown": 0x8, "sync_boost": 0x10, "sw_thermal_slowdown": 0x20,
+    "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80,
+    "display_clock_setting": 0x100,
+}
+
+
+class ClockSampler:
+    def __init__(self, torch_dev_index):
+        self.samples = []
+        self.ok = False
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            props = torch.cuda.get_device_properties(torch_dev_index)
+            h = None
+            try:
+                bus = "%08X:%02X:%02X.0" % (props.pci_domain_id, props.pci_bus_id,
+                                             props.pci_device_id)
+                h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            except Exception:
+                h = pynvml.nvmlDeviceGetHandleByUUID("GPU-" + str(props.uuid))
+            self.h = h
+            self.nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # pragma: no cover - depends on the box
+            self.err = repr(e)
+
+    def _reasons(self):
+        nv = self.nv
+        for fn in ("nvmlDeviceGetCurrentClocksEventReasons",
+                   "nvmlDeviceGetCurrentClocksThrottleReasons"):
+            if hasattr(nv, fn):
+                return int(getattr(nv, fn)(self.h))
+        return 0
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                pw = nv.nvmlDeviceGetPowerUsage(self.h) / 1000.0
+                self.samples.append((time.perf_counter(), sm, self._reasons(), pw))
+            except Exception:
+                pass
+            time.sleep(0.05)
+
+    def start(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+
+    def stop(self):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self, t0, t1):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [],
+                    "note": "NVML unavailable: " + getattr(self, "err", "")}
+        inwin = [s for s in self.samples if t0 <= s[0] <= t1]
+        src = "timed region"
+        if not inwin:
+            inwin = [s for s in self.samples if s[0] >= t0 - 1.0]
+            src = "around the timed region (no sample fell inside it)"
+        if not inwin:
+            inwin = self.samples
+            src = "whole run"
+        bits = 0
+        for s in inwin:
+            bits |= s[2]
+        reasons = [k for k, b in _REASON_BITS.items() if bits & b and k != "gpu_idle"]
+        return {"sm_mhz": statistics.median(s[1] for s in inwin) if inwin else None,
+                "sm_max_mhz": self.max_mhz, "reasons": reasons, "samples": len(inwin),
+                "power_w_max": max((s[3] for s in inwin), default=None), "window": src}
+
+
+# ----------------------------------------------------------------------------
+# CPU baseline: the fp64 oracle on a bounded sample of the workload
+# ----------------------------------------------------------------------------
+def oracle_sample(w, x, target_s=15.0):
+    """Time the oracle on a leading block of heads x tokens of the workload,
+    sized from a short calibration run to take about `target_s` seconds.
+    Returns (tokens/s, info)."""
+    import torch
+
+    import oracle
+    cores = oracle.num_threads()
+    BH = w.B * w.NH
+
+    def sub(heads, tokens):
+        sel = [(i // w.NH, i % w.NH) for i in range(heads)]
+        out = {k: torch.stack([x[k][b, h, :tokens] for b, h in sel]).unsqueeze(0)
+               for k in ("Q", "K", "V", "i_pre", "f_pre")}
+        for k in ("C0", "n0", "m0"):
+            out[k] = None if x[k] is None else torch.stack([x[k][b, h] for b, h in sel]).unsqueeze(0)
+        return out
+
+    def timed(heads, tokens):
+        c = sub(heads, tokens)
+        t0 = time.perf_counter()
+        oracle.mlstm_recurrent(c["Q"], c["K"], c["V"], c["i_pre"], c["f_pre"], c["C0"], c["n0"],
+                               c["m0"], gate_mode=w.gate_mode)
+        return time.perf_counter() - t0
+
+    h_cal = min(BH, cores)
+    t_cal = min(w.T, 256)
+    per_unit = max(timed(h_cal, t_cal), 1e-6) / (h_cal * t_cal)  # s per head-token, all cores
+    units = target_s / per_unit
+    if units >= BH * w.T:
+        heads, tokens = BH, w.T
+    else:
+        tokens = w.T if units >= h_cal * w.T else max(t_cal, int(units // h_cal))
+        heads = min(BH, max(h_cal, int(units // tokens) // h_cal * h_cal))
+    el = timed(heads, tokens)
+    return heads * tokens / el, {"heads": heads, "tokens_per_head": tokens, "seconds": el,
+                                 "cores": cores}
+
+
+def workload_config(w, algo):
+    return {"workload": w.name, "B": w.B, "NH": w.NH, "T": w.T, "DK": w.DK, "DV": w.DV,
+            "chunk_size": w.chunk_size, "gate_mode": w.gate_mode, "dtype": w.dtype,
+            "init_state": w.init_state, "algo": algo,
+            "l2": "not flushed: each step moves %.2f GB (> %d MB L2)" % (
+                algorithmic_bytes(w, 2 if w.dtype == "bf16" else 4) / 1e9, L2_BYTES >> 20)}
+
+
+def pick_workload(name):
+    from mlstm_chunkwise_b200.inputs import WORKLOADS, sweep_workload
+    if name.startswith("sweep_"):
+        _, t, l = name.split("_")
+        return sweep_workload(int(t[1:]), int(l[1:]))
+    return WORKLOADS[name]
+
+
+# ----------------------------------------------------------------------------
+# reference arm: the oracle alone
+# ----------------------------------------------------------------------------
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return 0
+    from mlstm_chunkwise_b200.inputs import make_inputs
+    w = pick_workload(args.workload)
+    x = make_inputs(w)
+    # size one step so that the whole K + W run stays within ~2 minutes
+    budget = max(0.5, min(4.0, 120.0 / max(1, args.steps + args.warmup)))
+    _, info = oracle_sample(w, x, target_s=budget)
+    import oracle
+    heads, tokens = info["heads"], info["tokens_per_head"]
+    sel = [(i // w.NH, i % w.NH) for i in range(heads)]
+    import torch
+    c = {k: torch.stack([x[k][b, h, :tokens] for b, h in sel]).unsqueeze(0)
+         for k in ("Q", "K", "V", "i_pre", "f_pre")}
+    for k in ("C0", "n0", "m0"):
+        c[k] = None if x[k] is None else torch.stack([x[k][b, h] for b, h in sel]).unsqueeze(0)
+
+    def step():
+        oracle.mlstm_recurrent(c["Q"], c["K"], c["V"], c["i_pre"], c["f_pre"], c["C0"], c["n0"],
+                               c["m0"], gate_mode=w.gate_mode)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    el = time.perf_counter() - t0
+    value = heads * tokens * args.steps / el
+    sample = (f"{heads} heads x first {tokens} tokens of {w.name} per step "
+              f"(of {w.B * w.NH} heads x {w.T} tokens)")
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": workload_config(w, "oracle"), "impl": "reference",
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": info["cores"],
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------
+# our arm
+# ----------------------------------------------------------------------------
+def run_ours(args):
+    import ctypes
+
+    import torch
+    import torch.distributed as dist
+
+    from mlstm_chunkwise_b200 import _lib, api
+    from mlstm_chunkwise_b200 import build as libbuild
+    from mlstm_chunkwise_b200.inputs import make_inputs
+
+    if libbuild.needs_build():
+        libbuild.build()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    w = pick_workload(args.workload)
+    x = make_inputs(w, seed=w.seed + rank)
+    d = {k: (None if v is None else v.to(dev)) for k, v in x.items()}
+    B, NH, T, DK, DV, L = w.B, w.NH, w.T, w.DK, w.DV, w.chunk_size
+    elem = 2 if w.dtype == "bf16" else 4
+    ws = torch.empty(max(1, api.workspace_size(B, NH, T, DK, DV, L, w.torch_dtype, args.algo)),
+                     dtype=torch.uint8, device=dev)
+    out = {"H": torch.empty((B, NH, T, DV), dtype=w.torch_dtype, device=dev),
+           "C_T": torch.empty((B, NH, DK, DV), dtype=torch.float32, device=dev),
+           "n_T": torch.empty((B, NH, DK), dtype=torch.float32, device=dev),
+           "m_T": torch.empty((B, NH), dtype=torch.float32, device=dev)}
+
+    def step(inp):
+        api.mlstm_fw(inp["Q"], inp["K"], inp["V"], inp["i_pre"], inp["f_pre"], inp["C0"],
+                     inp["n0"], inp["m0"], chunk_size=L, gate_mode=w.gate_mode, algo=args.algo,
+                     workspace=ws, out=out)
+
+    lib = _lib.lib()
+    for _ in range(max(3, args.warmup)):
+        step(d)
+    torch.cuda.synchronize()
+    st = api.last_device_error(dev)
+    if st != _lib.OK:
+        raise SystemExit(f"device error after warm-up: {_lib.status_string(st)}")
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    stream = torch.cuda.current_stream(dev)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ms_arr = (ctypes.c_double * _lib.KERNEL_COUNT)()
+    n_arr = (ctypes.c_uint64 * _lib.KERNEL_COUNT)()
+    lib.mlstm_profile_read(ms_arr, n_arr, _lib.KERNEL_COUNT)  # clear
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    launches0 = lib.mlstm_kernel_launches()
+    lib.mlstm_profile_enable(1)
+    t_host0 = time.perf_counter()
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step(d)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    t_host1 = time.perf_counter()
+    lib.mlstm_profile_enable(0)
+    launches = lib.mlstm_kernel_launches() - launches0
+    if world > 1:
+        dist.barrier()
+    elapsed_ms = ev0.elapsed_time(ev1)
+    st = api.last_device_error(dev)
+    if st != _lib.OK:
+        raise SystemExit(f"device error in the timed region: {_lib.status_string(st)}")
+    _lib.check(lib.mlstm_profile_read(ms_arr, n_arr, _lib.KERNEL_COUNT), "mlstm_profile_read")
+    kern = {lib.mlstm_kernel_name(i).decode(): (ms_arr[i], int(n_arr[i]))
+            for i in range(_lib.KERNEL_COUNT) if n_arr[i]}
+    sampler.stop()
+    clocks = sampler.summary(t_host0, t_host1)
+
+    if world > 1:
+        t = torch.tensor([elapsed_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+
+    # --- e2e: pinned host inputs -> device -> mlstm_fw -> host outputs -------
+    hx = {k: (None if v is None else v.pin_memory()) for k, v in x.items()}
+    hout = {k: torch.empty(v.shape, dtype=v.dtype).pin_memory() for k, v in out.items()}
+    h2d = sum(v.numel() * v.element_size() for v in hx.values() if v is not None)
+    d2h = sum(v.numel() * v.element_size() for v in hout.values())
+    e2e_steps = max(1, min(args.steps, 5))
+
+    def e2e_step():
+        di = {k: (None if v is None else v.to(dev, non_blocking=True)) for k, v in hx.items()}
+        step(di)
+        for k, v in out.items():
+            hout[k].copy_(v, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    tokens_per_step = B * T * world
+    ms_per_step = elapsed_ms / args.steps
+    value = tokens_per_step / (ms_per_step / 1e3)
+    e2e_value = tokens_per_step * e2e_steps / (e2e_ms / 1e3)
+
+    # --- roofline of the dominant kernel ------------------------------------
+    peaks, peak_src = load_peaks()
+    fph = flops_per_head(T, DK, DV, L)
+    BH = B * NH
+    fam_flops = {
+        "tc_fused": BH * (fph["states"] + fph["inter"] + fph["intra"]),
+        "tc_states": BH * fph["states"], "simt_states": BH * fph["states"],
+        "tc_parallel": BH * (fph["inter"] + fph["intra"]),
+        "simt_parallel": BH * (fph["inter"] + fph["intra"]),
+    }
+    total_flops = BH * sum(fph.values())
+    top = max(kern.items(), key=lambda kv: kv[1][0])
+    top_name, (top_ms, top_n) = top
+    calls = max(1, args.steps)
+    per_launch_ms = top_ms / calls
+    sustained = elapsed_ms > 1000.0
+    if top_name.startswith("tc"):
+        peak = peaks["bf16_tflops_sustained" if sustained else "bf16_tflops"]
+        achieved = fam_flops[top_name] / (per_launch_ms / 1e3) / 1e12
+        roof = {"kernel": top_name, "bound": "tensor", "achieved": achieved, "peak": peak,
+                "unit": "TFLOP/s", "frac": achieved / peak,
+                "peak_source": f"{'bf16_tflops_sustained' if sustained else 'bf16_tflops'} "
+                               f"(of {peak_src})"}
+    elif top_name.startswith("simt"):
+        peak = SIMT_LANES * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
+        achieved = fam_flops[top_name] / (per_launch_ms / 1e3) / 1e12
+        roof = {"kernel": top_name, "bound": "alu", "achieved": achieved, "peak": peak,
+                "unit": "TFLOP/s", "frac": achieved / peak,
+                "peak_source": f"fp32 FFMA: 148 SMs x 128 lanes x 2 x sm_max_mhz (of {peak_src})"}
+    else:
+        gate_bytes = BH * T * (8 + 12)
+        achieved = gate_bytes / (per_launch_ms / 1e3) / 1e9
+        roof = {"kernel": top_name, "bound": "hbm", "achieved": achieved,
+                "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+                "peak_source": f"hbm_gbs (of {peak_src})"}
+    roof["traffic"] = None
+    roof["per_launch_ms"] = per_launch_ms
+
+    algo_used = "+".join(sorted(kern))
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
+        "data": "synthetic", "config": workload_config(w, algo_used),
+        "tflops": total_flops * world / (ms_per_step / 1e3) / 1e12,
+        "frac_bf16_peak": (total_flops / (ms_per_step / 1e3) / 1e12) / peaks["bf16_tflops"],
+        "roofline": roof,
+        "kernels_ms_per_step": {k: v[0] / calls for k, v in kern.items()},
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+        "gpu_launches": int(launches),
+        "clocks": clocks,
+    }
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        v, info = oracle_sample(w, x, target_s=args.cpu_seconds)
+        line["cpu_baseline"] = {
+            "value": v, "unit": "tokens/s", "cores": info["cores"], "kind": "oracle",
+            "sample": f"{info['heads']} heads x first {info['tokens_per_head']} tokens of "
+                      f"{w.name} ({info['seconds']:.1f} s)"}
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="xlstm7b")
+    ap.add_argument("--algo", default="auto", choices=["auto", "simt", "tc", "tc_fused"])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

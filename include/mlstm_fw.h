@@ -1,0 +1,180 @@
+/*
+ * mlstm_fw.h -- C ABI of the B200 (sm_100a) chunkwise mLSTM forward library.
+ *
+ * The operation.  For every (batch b, head h) the mLSTM ("xLSTM: the NX-AI
+ * repository behind the extended LSTM architecture", section "Exponential
+ * gating, matrix memory, and why the kernels decide everything": exponential
+ * gating with normalisation and stabilisation, a matrix memory) runs, for
+ * t = 1..T,
+ *
+ *   lf_t = logsigmoid(f~_t),   li_t = i~_t (EXP) or logsigmoid(i~_t) (SIGMOID)
+ *   m_t  = max(lf_t + m_{t-1}, li_t)
+ *   C_t  = e^{lf_t + m_{t-1} - m_t} C_{t-1} + e^{li_t - m_t} (s k_t) v_t^T
+ *   n_t  = e^{lf_t + m_{t-1} - m_t} n_{t-1} + e^{li_t - m_t} (s k_t)
+ *   h_t  = C_t^T q_t / max(|n_t^T q_t|, e^{-m_t}),     s = 1/sqrt(DK)
+ *
+ * and returns H and the final state (C_T, n_T, m_T).  It is computed
+ * chunkwise, as in "Tiled Flash Linear Attention: More Efficient Linear RNN
+ * and xLSTM Kernels" (abstract): an inter-chunk state recurrence plus an
+ * intra-chunk parallel part that is tiled a second time over query and
+ * key/value blocks, so the chunk size is not limited by the tile size.  The
+ * sigmoid input gate is that page's mLSTM variant with a sigmoid input gate.
+ * The split into a recurrent (chunk-state) call and a parallel (output) call
+ * mirrors flash-xlstm-exp 0.1.0 ("Usage": the parallel kernel takes matQ,
+ * matK, matV, vecI, vecF and matC_states, vecN_states, scaMinter_states and
+ * returns matH_out, vecN_out, vecM_out).
+ *
+ * Layouts (all row-major, contiguous, 16-byte aligned device pointers):
+ *   Q, K    [B, NH, T, DK]   dtype      V, H [B, NH, T, DV]   dtype
+ *   i_pre, f_pre [B, NH, T]  fp32       (gate pre-activations)
+ *   C0, C_T [B, NH, DK, DV]  fp32       (C stored as sum of (s k) v^T, i.e. [DK, DV])
+ *   n0, n_T [B, NH, DK]      fp32       m0, m_T [B, NH] fp32
+ * Initial states: C0, n0, m0 are all NULL (zero state, m0 = 0) or all given.
+ * Final states: each of C_T, n_T, m_T may be NULL independently.
+ *
+ * Ownership: the caller owns every buffer, including the workspace; the
+ * library allocates no device memory and keeps no state other than a 32-bit
+ * device error word.  All calls are asynchronous on `stream`; the outputs are
+ * valid once the stream has reached that point.
+ *
+ * Errors: shape/pointer problems return MLSTM_ERR_INVALID_ARG and launch
+ * nothing; shapes outside what a chosen algorithm supports return
+ * MLSTM_ERR_UNSUPPORTED and launch nothing; a failed launch returns
+ * MLSTM_ERR_CUDA.  Kernels never trap: a bounded wait that runs out sets the
+ * device error word, which mlstm_last_device_error() reports as
+ * MLSTM_ERR_TIMEOUT.  Inputs must be finite; NaN/inf inputs give unspecified
+ * (but memory-safe) results.
+ */
+#ifndef MLSTM_FW_H_
+#define MLSTM_FW_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A CUDA stream (cudaStream_t); NULL is the legacy default stream. */
+typedef struct CUstream_st* mlstm_stream_t;
+
+typedef enum {
+  MLSTM_OK = 0,
+  MLSTM_ERR_INVALID_ARG = 1,  /* bad pointer, shape or enum value          */
+  MLSTM_ERR_UNSUPPORTED = 2,  /* valid, but not supported by that algorithm */
+  MLSTM_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed       */
+  MLSTM_ERR_TIMEOUT = 4,      /* a device-side bounded wait ran out         */
+  MLSTM_ERR_DEVICE = 5        /* another device-side check failed           */
+} mlstm_status;
+
+typedef enum { MLSTM_DT_F32 = 0, MLSTM_DT_BF16 = 1 } mlstm_dtype;
+
+typedef enum { MLSTM_GATE_EXP = 0, MLSTM_GATE_SIGMOID = 1 } mlstm_gate_mode;
+
+/* Which kernels compute the path.
+ *   AUTO      the fastest algorithm that supports the arguments.
+ *   SIMT      fp32 CUDA-core kernels (the only choice for fp32 inputs).
+ *   TC        bf16 tensor-core kernels, unfused: chunk states are written to
+ *             the workspace in fp32 between the state and the output kernels.
+ *   TC_FUSED  bf16 tensor-core kernel that carries the chunk state on chip. */
+typedef enum {
+  MLSTM_ALGO_AUTO = 0,
+  MLSTM_ALGO_SIMT = 1,
+  MLSTM_ALGO_TC = 2,
+  MLSTM_ALGO_TC_FUSED = 3
+} mlstm_algo;
+
+/* Bytes of workspace mlstm_fw() needs for these arguments (written to
+ * *bytes).  Sizes: B, NH >= 1; T >= 0; DK, DV in [1, 1024]; chunk_size a
+ * multiple of 64 in [64, 4096].  Returns MLSTM_ERR_INVALID_ARG or
+ * MLSTM_ERR_UNSUPPORTED like mlstm_fw() would. */
+mlstm_status mlstm_fw_workspace_size(int B, int NH, int T, int DK, int DV, int chunk_size,
+                                     mlstm_dtype dtype, mlstm_algo algo, size_t* bytes);
+
+/* The whole forward pass: H and, where non-NULL, the final (C_T, n_T, m_T).
+ * T need not be a multiple of chunk_size (the last chunk is ragged); T = 0
+ * copies the initial state to the final state.  `workspace` must hold at
+ * least mlstm_fw_workspace_size() bytes (it may be NULL when that is 0). */
+mlstm_status mlstm_fw(const void* Q, const void* K, const void* V, const float* i_pre,
+                      const float* f_pre, const float* C0, const float* n0, const float* m0,
+                      void* H, float* C_T, float* n_T, float* m_T, int B, int NH, int T, int DK,
+                      int DV, int chunk_size, mlstm_dtype dtype, mlstm_gate_mode gate_mode,
+                      mlstm_algo algo, void* workspace, size_t workspace_bytes,
+                      mlstm_stream_t stream);
+
+/* Bytes of workspace the two calls below need (gate arrays only). */
+mlstm_status mlstm_fw_gates_workspace_size(int B, int NH, int T, int chunk_size, size_t* bytes);
+
+/* Recurrent half of the chunkwise pass: the state entering every chunk,
+ *   C_states [B, NH, NC, DK, DV], n_states [B, NH, NC, DK], m_states
+ *   [B, NH, NC + 1] (m_states[..., k] is the stabiliser entering chunk k;
+ *   index NC is the final m), NC = ceil(T / chunk_size),
+ * plus the optional final state.  Algorithm SIMT or TC (AUTO picks). */
+mlstm_status mlstm_fw_chunk_states(const void* K, const void* V, const float* i_pre,
+                                   const float* f_pre, const float* C0, const float* n0,
+                                   const float* m0, float* C_states, float* n_states,
+                                   float* m_states, float* C_T, float* n_T, float* m_T, int B,
+                                   int NH, int T, int DK, int DV, int chunk_size,
+                                   mlstm_dtype dtype, mlstm_gate_mode gate_mode, mlstm_algo algo,
+                                   void* workspace, size_t workspace_bytes,
+                                   mlstm_stream_t stream);
+
+/* Parallel half: H from Q, K, V, the gates and the chunk states produced by
+ * mlstm_fw_chunk_states (same m0 and gates).  Optional per-token outputs:
+ *   n_out [B, NH, T] = max(|n_t^T q_t|, e^{-m_t}) (the denominator), and
+ *   m_out [B, NH, T] = m_t.  Algorithm SIMT or TC (AUTO picks). */
+mlstm_status mlstm_fw_parallel(const void* Q, const void* K, const void* V, const float* i_pre,
+                               const float* f_pre, const float* m0, const float* C_states,
+                               const float* n_states, void* H, float* n_out, float* m_out, int B,
+                               int NH, int T, int DK, int DV, int chunk_size, mlstm_dtype dtype,
+                               mlstm_gate_mode gate_mode, mlstm_algo algo, void* workspace,
+                               size_t workspace_bytes, mlstm_stream_t stream);
+
+/* Synchronises `stream`, then returns and clears the device error word:
+ * MLSTM_OK, MLSTM_ERR_TIMEOUT (a bounded wait ran out) or MLSTM_ERR_DEVICE;
+ * MLSTM_ERR_CUDA if the synchronisation itself failed. */
+mlstm_status mlstm_last_device_error(mlstm_stream_t stream);
+
+/* Spin limit of every bounded device-side wait (default 2^26 polls, about a
+ * second or more).  Affects launches made after the call.  0 restores the
+ * default.  Not thread-safe with concurrent launches. */
+void mlstm_set_watchdog(uint64_t max_polls);
+
+/* Kernel families, as reported by the profiling calls below. */
+typedef enum {
+  MLSTM_KERNEL_GATES = 0,         /* gate preprocessing (2 launches per call)  */
+  MLSTM_KERNEL_SIMT_STATES = 1,   /* fp32 chunk-state recurrence               */
+  MLSTM_KERNEL_SIMT_PARALLEL = 2, /* fp32 intra-chunk + inter-chunk output     */
+  MLSTM_KERNEL_TC_STATES = 3,     /* tensor-core chunk-state recurrence        */
+  MLSTM_KERNEL_TC_PARALLEL = 4,   /* tensor-core intra-chunk TFLA kernel       */
+  MLSTM_KERNEL_TC_FUSED = 5,      /* tensor-core fused kernel                  */
+  MLSTM_KERNEL_COUNT = 6
+} mlstm_kernel_id;
+
+/* Total number of kernels this library has enqueued since it was loaded. */
+uint64_t mlstm_kernel_launches(void);
+
+/* Measurement hook, off by default.  While on, every kernel family launch is
+ * bracketed by a pair of CUDA events on the launch stream. */
+void mlstm_profile_enable(int on);
+
+/* Waits for the recorded events, then writes, per kernel family id
+ * (0 <= id < n, n <= MLSTM_KERNEL_COUNT), the summed device time in ms and the
+ * number of launches since the previous read, and clears the record.
+ * Returns MLSTM_ERR_CUDA if an event query fails. */
+mlstm_status mlstm_profile_read(double* ms, uint64_t* launches, int n);
+
+/* Static name of a kernel family id (never NULL). */
+const char* mlstm_kernel_name(int id);
+
+/* Static text for a status code (never NULL). */
+const char* mlstm_status_string(mlstm_status status);
+
+/* Library ABI version: 100 * major + minor. */
+int mlstm_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MLSTM_FW_H_ */

@@ -1,0 +1,190 @@
+"""Python binding of the C ABI (argument marshalling only).
+
+Every computation runs in the CUDA kernels of ``libmlstm_fw.so``; this module
+allocates outputs and workspace with PyTorch on the inputs' device, passes raw
+pointers and torch's current stream, and raises ``MlstmError`` on a non-OK
+status.  Inputs must be CUDA tensors: there is no CPU path.
+"""
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from . import _lib
+from ._lib import MlstmError  # noqa: F401  (re-export)
+
+_DT = {torch.float32: _lib.DT_F32, torch.bfloat16: _lib.DT_BF16}
+_GATE = {"exp": _lib.GATE_EXP, "sigmoid": _lib.GATE_SIGMOID}
+_ALGO = {"auto": _lib.ALGO_AUTO, "simt": _lib.ALGO_SIMT, "tc": _lib.ALGO_TC,
+         "tc_fused": _lib.ALGO_TC_FUSED}
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _check_tensor(name, t, dtype, shape, device):
+    if t is None:
+        return
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (the library has no CPU path)")
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def workspace_size(B, NH, T, DK, DV, chunk_size, dtype=torch.bfloat16, algo="auto") -> int:
+    n = ctypes.c_size_t(0)
+    _lib.check(_lib.lib().mlstm_fw_workspace_size(B, NH, T, DK, DV, chunk_size, _DT[dtype],
+                                                  _ALGO[algo], ctypes.byref(n)),
+               "mlstm_fw_workspace_size")
+    return int(n.value)
+
+
+def gates_workspace_size(B, NH, T, chunk_size) -> int:
+    n = ctypes.c_size_t(0)
+    _lib.check(_lib.lib().mlstm_fw_gates_workspace_size(B, NH, T, chunk_size, ctypes.byref(n)),
+               "mlstm_fw_gates_workspace_size")
+    return int(n.value)
+
+
+def _shapes(Q, V):
+    B, NH, T, DK = Q.shape
+    DV = V.shape[-1]
+    return B, NH, T, DK, DV
+
+
+def _check_common(Q, K, V, i_pre, f_pre):
+    if Q.dim() != 4:
+        raise ValueError("Q must be [B, NH, T, DK]")
+    B, NH, T, DK, DV = _shapes(Q, V)
+    dev = Q.device
+    dt = Q.dtype
+    if dt not in _DT:
+        raise ValueError(f"unsupported dtype {dt} (float32 or bfloat16)")
+    _check_tensor("Q", Q, dt, (B, NH, T, DK), dev)
+    _check_tensor("K", K, dt, (B, NH, T, DK), dev)
+    _check_tensor("V", V, dt, (B, NH, T, DV), dev)
+    _check_tensor("i_pre", i_pre, torch.float32, (B, NH, T), dev)
+    _check_tensor("f_pre", f_pre, torch.float32, (B, NH, T), dev)
+    return B, NH, T, DK, DV, dev, dt
+
+
+def _check_state(C0, n0, m0, B, NH, DK, DV, dev):
+    if (C0 is None) != (n0 is None) or (C0 is None) != (m0 is None):
+        raise ValueError("C0, n0 and m0 must be given together")
+    _check_tensor("C0", C0, torch.float32, (B, NH, DK, DV), dev)
+    _check_tensor("n0", n0, torch.float32, (B, NH, DK), dev)
+    _check_tensor("m0", m0, torch.float32, (B, NH), dev)
+
+
+def mlstm_fw(Q, K, V, i_pre, f_pre, C0=None, n0=None, m0=None, *, chunk_size: int = 64,
+             gate_mode: str = "exp", algo: str = "auto", return_last_states: bool = True,
+             workspace: torch.Tensor | None = None, out: dict | None = None):
+    """mLSTM forward pass on the GPU.
+
+    Q, K [B,NH,T,DK] and V [B,NH,T,DV] (float32 or bfloat16, same dtype);
+    i_pre, f_pre [B,NH,T] float32; optional initial state C0 [B,NH,DK,DV],
+    n0 [B,NH,DK], m0 [B,NH] float32.  Returns ``H`` or ``(H, (C_T, n_T, m_T))``.
+    ``out`` may hold preallocated ``H``/``C_T``/``n_T``/``m_T``; ``workspace``
+    a uint8 CUDA tensor of at least ``workspace_size(...)`` bytes.
+    """
+    B, NH, T, DK, DV, dev, dt = _check_common(Q, K, V, i_pre, f_pre)
+    _check_state(C0, n0, m0, B, NH, DK, DV, dev)
+    out = {} if out is None else out
+    H = out.get("H")
+    if H is None:
+        H = torch.empty((B, NH, T, DV), dtype=dt, device=dev)
+    _check_tensor("H", H, dt, (B, NH, T, DV), dev)
+    C_T = n_T = m_T = None
+    if return_last_states:
+        C_T = out.get("C_T")
+        n_T = out.get("n_T")
+        m_T = out.get("m_T")
+        if C_T is None:
+            C_T = torch.empty((B, NH, DK, DV), dtype=torch.float32, device=dev)
+        if n_T is None:
+            n_T = torch.empty((B, NH, DK), dtype=torch.float32, device=dev)
+        if m_T is None:
+            m_T = torch.empty((B, NH), dtype=torch.float32, device=dev)
+    ws_bytes = workspace_size(B, NH, T, DK, DV, chunk_size, dt, algo)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
+    elif workspace.numel() < ws_bytes or not workspace.is_cuda:
+        raise ValueError(f"workspace must be a CUDA uint8 tensor of >= {ws_bytes} bytes")
+    st = _lib.lib().mlstm_fw(
+        _ptr(Q), _ptr(K), _ptr(V), _ptr(i_pre), _ptr(f_pre), _ptr(C0), _ptr(n0), _ptr(m0),
+        _ptr(H), _ptr(C_T), _ptr(n_T), _ptr(m_T), B, NH, T, DK, DV, chunk_size, _DT[dt],
+        _GATE[gate_mode], _ALGO[algo], _ptr(workspace), workspace.numel(), _stream(dev))
+    _lib.check(st, "mlstm_fw")
+    if return_last_states:
+        return H, (C_T, n_T, m_T)
+    return H
+
+
+def mlstm_fw_chunk_states(K, V, i_pre, f_pre, C0=None, n0=None, m0=None, *, chunk_size: int = 64,
+                          gate_mode: str = "exp", algo: str = "auto"):
+    """Recurrent half: states entering every chunk and the final state.
+
+    Returns (C_states [B,NH,NC,DK,DV], n_states [B,NH,NC,DK], m_states
+    [B,NH,NC+1], (C_T, n_T, m_T)).
+    """
+    B, NH, T, DK, DV, dev, dt = _check_common(K, K, V, i_pre, f_pre)
+    _check_state(C0, n0, m0, B, NH, DK, DV, dev)
+    NC = (T + chunk_size - 1) // chunk_size
+    C_states = torch.empty((B, NH, NC, DK, DV), dtype=torch.float32, device=dev)
+    n_states = torch.empty((B, NH, NC, DK), dtype=torch.float32, device=dev)
+    m_states = torch.empty((B, NH, NC + 1), dtype=torch.float32, device=dev)
+    C_T = torch.empty((B, NH, DK, DV), dtype=torch.float32, device=dev)
+    n_T = torch.empty((B, NH, DK), dtype=torch.float32, device=dev)
+    m_T = torch.empty((B, NH), dtype=torch.float32, device=dev)
+    ws = torch.empty(max(gates_workspace_size(B, NH, T, chunk_size), 1), dtype=torch.uint8,
+                     device=dev)
+    st = _lib.lib().mlstm_fw_chunk_states(
+        _ptr(K), _ptr(V), _ptr(i_pre), _ptr(f_pre), _ptr(C0), _ptr(n0), _ptr(m0), _ptr(C_states),
+        _ptr(n_states), _ptr(m_states), _ptr(C_T), _ptr(n_T), _ptr(m_T), B, NH, T, DK, DV,
+        chunk_size, _DT[dt], _GATE[gate_mode], _ALGO[algo], _ptr(ws), ws.numel(), _stream(dev))
+    _lib.check(st, "mlstm_fw_chunk_states")
+    return C_states, n_states, m_states, (C_T, n_T, m_T)
+
+
+def mlstm_fw_parallel(Q, K, V, i_pre, f_pre, C_states, n_states, m0=None, *,
+                      chunk_size: int = 64, gate_mode: str = "exp", algo: str = "auto"):
+    """Parallel half: (H, n_out, m_out) from the chunk states."""
+    B, NH, T, DK, DV, dev, dt = _check_common(Q, K, V, i_pre, f_pre)
+    NC = (T + chunk_size - 1) // chunk_size
+    _check_tensor("C_states", C_states, torch.float32, (B, NH, NC, DK, DV), dev)
+    _check_tensor("n_states", n_states, torch.float32, (B, NH, NC, DK), dev)
+    _check_tensor("m0", m0, torch.float32, (B, NH), dev)
+    H = torch.empty((B, NH, T, DV), dtype=dt, device=dev)
+    n_out = torch.empty((B, NH, T), dtype=torch.float32, device=dev)
+    m_out = torch.empty((B, NH, T), dtype=torch.float32, device=dev)
+    ws = torch.empty(max(gates_workspace_size(B, NH, T, chunk_size), 1), dtype=torch.uint8,
+                     device=dev)
+    st = _lib.lib().mlstm_fw_parallel(
+        _ptr(Q), _ptr(K), _ptr(V), _ptr(i_pre), _ptr(f_pre), _ptr(m0), _ptr(C_states),
+        _ptr(n_states), _ptr(H), _ptr(n_out), _ptr(m_out), B, NH, T, DK, DV, chunk_size, _DT[dt],
+        _GATE[gate_mode], _ALGO[algo], _ptr(ws), ws.numel(), _stream(dev))
+    _lib.check(st, "mlstm_fw_parallel")
+    return H, n_out, m_out
+
+
+def last_device_error(device=None) -> int:
+    """Synchronises the current stream and returns (and clears) the device
+    error status (``_lib.OK``, ``_lib.ERR_TIMEOUT``, ...)."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    return int(_lib.lib().mlstm_last_device_error(_stream(dev)))
+
+
+def set_watchdog(max_polls: int) -> None:
+    _lib.lib().mlstm_set_watchdog(int(max_polls))

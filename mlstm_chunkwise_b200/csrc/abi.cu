@@ -1,0 +1,423 @@
+// C ABI of the mLSTM forward library: argument checks, workspace layout and
+// dispatch to the kernels.  Every check happens before the first launch, so an
+// error return means nothing was enqueued.
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <atomic>
+#include <mutex>
+#include <vector>
+
+#include "common.cuh"
+#include "tc.h"
+
+namespace mlstm {
+namespace {
+
+__device__ uint32_t g_error_word = 0;
+
+constexpr unsigned long long kDefaultPolls = 1ull << 26;
+unsigned long long g_max_polls = kDefaultPolls;
+
+constexpr size_t kAlign = 256;
+inline size_t round_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Largest device count this library keeps a cached error-word address for.
+constexpr int kMaxDevices = 64;
+uint32_t* g_err_ptr[kMaxDevices] = {};
+
+uint32_t* error_word_ptr() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  if (!g_err_ptr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_error_word) != cudaSuccess) return nullptr;
+    g_err_ptr[dev] = static_cast<uint32_t*>(ptr);
+  }
+  return g_err_ptr[dev];
+}
+
+struct Layout {
+  size_t gates_bytes;   // bcum, acol, amax, gtot, mchk
+  size_t states_bytes;  // C_states, n_states (unfused only)
+  size_t total;
+};
+
+mlstm_status check_sizes(int B, int NH, int T, int DK, int DV, int L) {
+  if (B < 1 || NH < 1 || T < 0 || DK < 1 || DV < 1) return MLSTM_ERR_INVALID_ARG;
+  if (L < 64 || L % 64 != 0) return MLSTM_ERR_INVALID_ARG;
+  if (L > 4096 || DK > 1024 || DV > 1024) return MLSTM_ERR_UNSUPPORTED;
+  if ((long long)B * NH > 65535) return MLSTM_ERR_UNSUPPORTED;
+  if (T > (1 << 22)) return MLSTM_ERR_UNSUPPORTED;
+  return MLSTM_OK;
+}
+
+Problem make_problem(int B, int NH, int T, int DK, int DV, int L, mlstm_gate_mode gm) {
+  Problem p{};
+  p.B = B;
+  p.NH = NH;
+  p.T = T;
+  p.DK = DK;
+  p.DV = DV;
+  p.L = L;
+  p.NC = (T + L - 1) / L;
+  p.BH = B * NH;
+  p.gate_sigmoid = gm == MLSTM_GATE_SIGMOID;
+  p.key_scale = (float)(1.0 / sqrt((double)DK));
+  p.err = nullptr;
+  p.max_polls = g_max_polls;
+  return p;
+}
+
+Layout layout_for(const Problem& p, bool with_states) {
+  Layout l{};
+  const size_t BH = (size_t)p.BH, tpad = (size_t)p.NC * p.L;
+  l.gates_bytes = 3 * round_up(BH * tpad * sizeof(float)) + round_up(BH * p.NC * sizeof(float)) +
+                  round_up(BH * (p.NC + 1) * sizeof(float));
+  if (with_states)
+    l.states_bytes = round_up(BH * p.NC * (size_t)p.DK * p.DV * sizeof(float)) +
+                     round_up(BH * p.NC * (size_t)p.DK * sizeof(float));
+  l.total = l.gates_bytes + l.states_bytes;
+  return l;
+}
+
+// Carves the gate arrays out of `ws`; returns the first byte after them.
+char* carve_gates(const Problem& p, char* ws, Gates* g, float* mchk_override) {
+  const size_t BH = (size_t)p.BH, tpad = (size_t)p.NC * p.L;
+  g->bcum = reinterpret_cast<float*>(ws);
+  ws += round_up(BH * tpad * sizeof(float));
+  g->acol = reinterpret_cast<float*>(ws);
+  ws += round_up(BH * tpad * sizeof(float));
+  g->amax = reinterpret_cast<float*>(ws);
+  ws += round_up(BH * tpad * sizeof(float));
+  g->gtot = reinterpret_cast<float*>(ws);
+  ws += round_up(BH * p.NC * sizeof(float));
+  g->mchk = mchk_override ? mchk_override : reinterpret_cast<float*>(ws);
+  ws += round_up(BH * (p.NC + 1) * sizeof(float));
+  return ws;
+}
+
+bool valid_enums(mlstm_dtype dt, mlstm_gate_mode gm, mlstm_algo algo) {
+  return (dt == MLSTM_DT_F32 || dt == MLSTM_DT_BF16) &&
+         (gm == MLSTM_GATE_EXP || gm == MLSTM_GATE_SIGMOID) &&
+         (algo == MLSTM_ALGO_AUTO || algo == MLSTM_ALGO_SIMT || algo == MLSTM_ALGO_TC ||
+          algo == MLSTM_ALGO_TC_FUSED);
+}
+
+// Resolves AUTO and checks that the chosen algorithm supports the problem.
+mlstm_status resolve_algo(const Problem& p, mlstm_dtype dt, mlstm_algo req, bool allow_fused,
+                          mlstm_algo* out) {
+  if (req == MLSTM_ALGO_AUTO) {
+    if (dt == MLSTM_DT_BF16 && p.T > 0 && allow_fused && tc_fused_supported(p)) {
+      *out = MLSTM_ALGO_TC_FUSED;
+    } else if (dt == MLSTM_DT_BF16 && p.T > 0 && tc_unfused_supported(p)) {
+      *out = MLSTM_ALGO_TC;
+    } else {
+      *out = MLSTM_ALGO_SIMT;
+    }
+    return MLSTM_OK;
+  }
+  if (req == MLSTM_ALGO_SIMT) {
+    *out = req;
+    return MLSTM_OK;
+  }
+  if (dt != MLSTM_DT_BF16 || p.T == 0) return MLSTM_ERR_UNSUPPORTED;
+  if (req == MLSTM_ALGO_TC) {
+    if (!tc_unfused_supported(p)) return MLSTM_ERR_UNSUPPORTED;
+  } else {
+    if (!allow_fused || !tc_fused_supported(p)) return MLSTM_ERR_UNSUPPORTED;
+  }
+  *out = req;
+  return MLSTM_OK;
+}
+
+inline mlstm_status from_cuda(cudaError_t e) {
+  return e == cudaSuccess ? MLSTM_OK : MLSTM_ERR_CUDA;
+}
+
+// --- launch accounting and the optional per-kernel event timing -----------
+std::atomic<uint64_t> g_launches{0};
+std::atomic<int> g_profile_on{0};
+struct Pending {
+  int id;
+  int launches;
+  cudaEvent_t start, stop;
+};
+std::mutex g_prof_mu;
+std::vector<Pending> g_pending;
+
+// Runs one launcher `fn` (which enqueues `n_launch` kernels on `st`), counting
+// the launches and, when profiling is on, bracketing them with events.
+template <typename Fn>
+cudaError_t launch_family(int id, int n_launch, cudaStream_t st, Fn&& fn) {
+  Pending pd{id, n_launch, nullptr, nullptr};
+  const bool prof = g_profile_on.load(std::memory_order_relaxed) != 0;
+  if (prof) {
+    if (cudaEventCreate(&pd.start) != cudaSuccess) return cudaGetLastError();
+    if (cudaEventCreate(&pd.stop) != cudaSuccess) return cudaGetLastError();
+    cudaEventRecord(pd.start, st);
+  }
+  cudaError_t e = fn();
+  if (e == cudaSuccess) g_launches.fetch_add((uint64_t)n_launch, std::memory_order_relaxed);
+  if (prof) {
+    cudaEventRecord(pd.stop, st);
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    g_pending.push_back(pd);
+  }
+  return e;
+}
+
+int gate_launches(const Problem& p) { return p.NC > 0 ? 2 : 1; }
+
+}  // namespace
+}  // namespace mlstm
+
+using namespace mlstm;
+
+extern "C" {
+
+int mlstm_abi_version(void) { return 100; }
+
+uint64_t mlstm_kernel_launches(void) { return g_launches.load(); }
+
+void mlstm_profile_enable(int on) { g_profile_on.store(on ? 1 : 0); }
+
+mlstm_status mlstm_profile_read(double* ms, uint64_t* launches, int n) {
+  if (n < 0 || n > MLSTM_KERNEL_COUNT || (n > 0 && (!ms || !launches)))
+    return MLSTM_ERR_INVALID_ARG;
+  std::vector<Pending> pend;
+  {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    pend.swap(g_pending);
+  }
+  for (int i = 0; i < n; ++i) {
+    ms[i] = 0.0;
+    launches[i] = 0;
+  }
+  mlstm_status st = MLSTM_OK;
+  for (Pending& pd : pend) {
+    float t = 0.f;
+    if (cudaEventSynchronize(pd.stop) != cudaSuccess ||
+        cudaEventElapsedTime(&t, pd.start, pd.stop) != cudaSuccess)
+      st = MLSTM_ERR_CUDA;
+    else if (pd.id < n) {
+      ms[pd.id] += t;
+      launches[pd.id] += (uint64_t)pd.launches;
+    }
+    cudaEventDestroy(pd.start);
+    cudaEventDestroy(pd.stop);
+  }
+  return st;
+}
+
+const char* mlstm_kernel_name(int id) {
+  switch (id) {
+    case MLSTM_KERNEL_GATES: return "gates";
+    case MLSTM_KERNEL_SIMT_STATES: return "simt_states";
+    case MLSTM_KERNEL_SIMT_PARALLEL: return "simt_parallel";
+    case MLSTM_KERNEL_TC_STATES: return "tc_states";
+    case MLSTM_KERNEL_TC_PARALLEL: return "tc_parallel";
+    case MLSTM_KERNEL_TC_FUSED: return "tc_fused";
+  }
+  return "unknown";
+}
+
+const char* mlstm_status_string(mlstm_status s) {
+  switch (s) {
+    case MLSTM_OK: return "ok";
+    case MLSTM_ERR_INVALID_ARG: return "invalid argument";
+    case MLSTM_ERR_UNSUPPORTED: return "unsupported by the selected algorithm";
+    case MLSTM_ERR_CUDA: return "CUDA error";
+    case MLSTM_ERR_TIMEOUT: return "device-side bounded wait timed out";
+    case MLSTM_ERR_DEVICE: return "device-side check failed";
+  }
+  return "unknown status";
+}
+
+void mlstm_set_watchdog(uint64_t max_polls) {
+  g_max_polls = max_polls ? (unsigned long long)max_polls : kDefaultPolls;
+}
+
+mlstm_status mlstm_fw_workspace_size(int B, int NH, int T, int DK, int DV, int chunk_size,
+                                     mlstm_dtype dtype, mlstm_algo algo, size_t* bytes) {
+  if (!bytes || !valid_enums(dtype, MLSTM_GATE_EXP, algo)) return MLSTM_ERR_INVALID_ARG;
+  mlstm_status s = check_sizes(B, NH, T, DK, DV, chunk_size);
+  if (s != MLSTM_OK) return s;
+  Problem p = make_problem(B, NH, T, DK, DV, chunk_size, MLSTM_GATE_EXP);
+  mlstm_algo a;
+  s = resolve_algo(p, dtype, algo, true, &a);
+  if (s != MLSTM_OK) return s;
+  *bytes = layout_for(p, a != MLSTM_ALGO_TC_FUSED).total;
+  return MLSTM_OK;
+}
+
+mlstm_status mlstm_fw_gates_workspace_size(int B, int NH, int T, int chunk_size, size_t* bytes) {
+  if (!bytes) return MLSTM_ERR_INVALID_ARG;
+  mlstm_status s = check_sizes(B, NH, T, 64, 64, chunk_size);
+  if (s != MLSTM_OK) return s;
+  Problem p = make_problem(B, NH, T, 64, 64, chunk_size, MLSTM_GATE_EXP);
+  *bytes = layout_for(p, false).gates_bytes;
+  return MLSTM_OK;
+}
+
+mlstm_status mlstm_fw(const void* Q, const void* K, const void* V, const float* i_pre,
+                      const float* f_pre, const float* C0, const float* n0, const float* m0,
+                      void* H, float* C_T, float* n_T, float* m_T, int B, int NH, int T, int DK,
+                      int DV, int chunk_size, mlstm_dtype dtype, mlstm_gate_mode gate_mode,
+                      mlstm_algo algo, void* workspace, size_t workspace_bytes,
+                      mlstm_stream_t stream) {
+  if (!valid_enums(dtype, gate_mode, algo)) return MLSTM_ERR_INVALID_ARG;
+  mlstm_status s = check_sizes(B, NH, T, DK, DV, chunk_size);
+  if (s != MLSTM_OK) return s;
+  if (T > 0 && (!Q || !K || !V || !i_pre || !f_pre || !H)) return MLSTM_ERR_INVALID_ARG;
+  if (!((C0 && n0 && m0) || (!C0 && !n0 && !m0))) return MLSTM_ERR_INVALID_ARG;
+  const void* ptrs[] = {Q, K, V, i_pre, f_pre, C0, n0, m0, H, C_T, n_T, m_T, workspace};
+  for (const void* q : ptrs)
+    if (!aligned16(q)) return MLSTM_ERR_INVALID_ARG;
+  Problem p = make_problem(B, NH, T, DK, DV, chunk_size, gate_mode);
+  mlstm_algo a;
+  s = resolve_algo(p, dtype, algo, true, &a);
+  if (s != MLSTM_OK) return s;
+  const Layout lay = layout_for(p, a != MLSTM_ALGO_TC_FUSED);
+  if (workspace_bytes < lay.total || (lay.total > 0 && !workspace)) return MLSTM_ERR_INVALID_ARG;
+  p.err = error_word_ptr();
+  if (!p.err) return MLSTM_ERR_CUDA;
+
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  Gates g;
+  char* rest = carve_gates(p, static_cast<char*>(workspace), &g, nullptr);
+  s = from_cuda(launch_family(MLSTM_KERNEL_GATES, gate_launches(p), st,
+                              [&] { return launch_gates(p, i_pre, f_pre, m0, g, st); }));
+  if (s != MLSTM_OK) return s;
+  if (a == MLSTM_ALGO_TC_FUSED)
+    return from_cuda(launch_family(MLSTM_KERNEL_TC_FUSED, 1, st, [&] {
+      return launch_tc_fused(p, Q, K, V, C0, n0, g, H, C_T, n_T, m_T, st);
+    }));
+
+  float* C_states = reinterpret_cast<float*>(rest);
+  float* n_states =
+      reinterpret_cast<float*>(rest + round_up((size_t)p.BH * p.NC * (size_t)DK * DV * 4));
+  if (a == MLSTM_ALGO_TC) {
+    s = from_cuda(launch_family(MLSTM_KERNEL_TC_STATES, 1, st, [&] {
+      return launch_tc_states(p, K, V, C0, n0, g, C_states, n_states, C_T, n_T, m_T, st);
+    }));
+    if (s != MLSTM_OK) return s;
+    if (T == 0) return MLSTM_OK;
+    return from_cuda(launch_family(MLSTM_KERNEL_TC_PARALLEL, 1, st, [&] {
+      return launch_tc_parallel(p, Q, K, V, g, C_states, n_states, H, nullptr, nullptr, st);
+    }));
+  }
+  s = from_cuda(launch_family(MLSTM_KERNEL_SIMT_STATES, 1, st, [&] {
+    return launch_simt_states(p, dtype, K, V, C0, n0, g, C_states, n_states, C_T, n_T, m_T, st);
+  }));
+  if (s != MLSTM_OK) return s;
+  if (T == 0) return MLSTM_OK;
+  return from_cuda(launch_family(MLSTM_KERNEL_SIMT_PARALLEL, 1, st, [&] {
+    return launch_simt_parallel(p, dtype, Q, K, V, g, C_states, n_states, H, nullptr, nullptr,
+                                st);
+  }));
+}
+
+mlstm_status mlstm_fw_chunk_states(const void* K, const void* V, const float* i_pre,
+                                   const float* f_pre, const float* C0, const float* n0,
+                                   const float* m0, float* C_states, float* n_states,
+                                   float* m_states, float* C_T, float* n_T, float* m_T, int B,
+                                   int NH, int T, int DK, int DV, int chunk_size,
+                                   mlstm_dtype dtype, mlstm_gate_mode gate_mode, mlstm_algo algo,
+                                   void* workspace, size_t workspace_bytes,
+                                   mlstm_stream_t stream) {
+  if (!valid_enums(dtype, gate_mode, algo)) return MLSTM_ERR_INVALID_ARG;
+  mlstm_status s = check_sizes(B, NH, T, DK, DV, chunk_size);
+  if (s != MLSTM_OK) return s;
+  if (T > 0 && (!K || !V || !i_pre || !f_pre || !C_states || !n_states))
+    return MLSTM_ERR_INVALID_ARG;
+  if (!m_states) return MLSTM_ERR_INVALID_ARG;
+  if (!((C0 && n0 && m0) || (!C0 && !n0 && !m0))) return MLSTM_ERR_INVALID_ARG;
+  const void* ptrs[] = {K,  V,        i_pre,    f_pre,    C0,  n0,  m0,       C_states,
+                        n_states, m_states, C_T, n_T, m_T, workspace};
+  for (const void* q : ptrs)
+    if (!aligned16(q)) return MLSTM_ERR_INVALID_ARG;
+  Problem p = make_problem(B, NH, T, DK, DV, chunk_size, gate_mode);
+  mlstm_algo a;
+  s = resolve_algo(p, dtype, algo, false, &a);
+  if (s != MLSTM_OK) return s;
+  const Layout lay = layout_for(p, false);
+  if (workspace_bytes < lay.gates_bytes || (lay.gates_bytes > 0 && !workspace))
+    return MLSTM_ERR_INVALID_ARG;
+  p.err = error_word_ptr();
+  if (!p.err) return MLSTM_ERR_CUDA;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  Gates g;
+  carve_gates(p, static_cast<char*>(workspace), &g, m_states);
+  s = from_cuda(launch_family(MLSTM_KERNEL_GATES, gate_launches(p), st,
+                              [&] { return launch_gates(p, i_pre, f_pre, m0, g, st); }));
+  if (s != MLSTM_OK) return s;
+  if (a == MLSTM_ALGO_TC)
+    return from_cuda(launch_family(MLSTM_KERNEL_TC_STATES, 1, st, [&] {
+      return launch_tc_states(p, K, V, C0, n0, g, C_states, n_states, C_T, n_T, m_T, st);
+    }));
+  return from_cuda(launch_family(MLSTM_KERNEL_SIMT_STATES, 1, st, [&] {
+    return launch_simt_states(p, dtype, K, V, C0, n0, g, C_states, n_states, C_T, n_T, m_T, st);
+  }));
+}
+
+mlstm_status mlstm_fw_parallel(const void* Q, const void* K, const void* V, const float* i_pre,
+                               const float* f_pre, const float* m0, const float* C_states,
+                               const float* n_states, void* H, float* n_out, float* m_out, int B,
+                               int NH, int T, int DK, int DV, int chunk_size, mlstm_dtype dtype,
+                               mlstm_gate_mode gate_mode, mlstm_algo algo, void* workspace,
+                               size_t workspace_bytes, mlstm_stream_t stream) {
+  if (!valid_enums(dtype, gate_mode, algo)) return MLSTM_ERR_INVALID_ARG;
+  mlstm_status s = check_sizes(B, NH, T, DK, DV, chunk_size);
+  if (s != MLSTM_OK) return s;
+  if (T > 0 && (!Q || !K || !V || !i_pre || !f_pre || !C_states || !n_states || !H))
+    return MLSTM_ERR_INVALID_ARG;
+  const void* ptrs[] = {Q, K, V, i_pre, f_pre, m0, C_states, n_states, H, n_out, m_out,
+                        workspace};
+  for (const void* q : ptrs)
+    if (!aligned16(q)) return MLSTM_ERR_INVALID_ARG;
+  Problem p = make_problem(B, NH, T, DK, DV, chunk_size, gate_mode);
+  mlstm_algo a;
+  s = resolve_algo(p, dtype, algo, false, &a);
+  if (s != MLSTM_OK) return s;
+  const Layout lay = layout_for(p, false);
+  if (workspace_bytes < lay.gates_bytes || (lay.gates_bytes > 0 && !workspace))
+    return MLSTM_ERR_INVALID_ARG;
+  if (T == 0) return MLSTM_OK;
+  p.err = error_word_ptr();
+  if (!p.err) return MLSTM_ERR_CUDA;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  Gates g;
+  carve_gates(p, static_cast<char*>(workspace), &g, nullptr);
+  s = from_cuda(launch_family(MLSTM_KERNEL_GATES, gate_launches(p), st,
+                              [&] { return launch_gates(p, i_pre, f_pre, m0, g, st); }));
+  if (s != MLSTM_OK) return s;
+  if (a == MLSTM_ALGO_TC)
+    return from_cuda(launch_family(MLSTM_KERNEL_TC_PARALLEL, 1, st, [&] {
+      return launch_tc_parallel(p, Q, K, V, g, C_states, n_states, H, n_out, m_out, st);
+    }));
+  return from_cuda(launch_family(MLSTM_KERNEL_SIMT_PARALLEL, 1, st, [&] {
+    return launch_simt_parallel(p, dtype, Q, K, V, g, C_states, n_states, H, n_out, m_out, st);
+  }));
+}
+
+mlstm_status mlstm_last_device_error(mlstm_stream_t stream) {
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return MLSTM_ERR_CUDA;
+  uint32_t* w = error_word_ptr();
+  if (!w) return MLSTM_ERR_CUDA;
+  uint32_t v = 0;
+  if (cudaMemcpy(&v, w, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return MLSTM_ERR_CUDA;
+  if (v != 0) {
+    const uint32_t zero = 0;
+    if (cudaMemcpy(w, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess)
+      return MLSTM_ERR_CUDA;
+  }
+  if (v & kErrWatchdog) return MLSTM_ERR_TIMEOUT;
+  if (v) return MLSTM_ERR_DEVICE;
+  return MLSTM_OK;
+}
+
+}  // extern "C"

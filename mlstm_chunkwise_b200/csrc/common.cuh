@@ -1,0 +1,85 @@
+// Shared device/host helpers for the mLSTM forward kernels (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "mlstm_fw.h"
+
+namespace mlstm {
+
+// ---------------------------------------------------------------------------
+// Device error word.  Kernels OR a bit in here instead of trapping; the host
+// reads and clears it in mlstm_last_device_error().
+// ---------------------------------------------------------------------------
+enum : uint32_t {
+  kErrWatchdog = 1u << 0,   // a bounded wait (mbarrier / flag) ran out
+  kErrBounds = 1u << 1,     // a debug bounds check failed
+  kErrTmem = 1u << 2,       // TMEM allocation returned an unexpected address
+};
+__device__ __forceinline__ void raise_error(uint32_t* word, uint32_t bit) {
+  if (word) atomicOr(word, bit);
+}
+
+// ---------------------------------------------------------------------------
+// Problem description passed by value to every kernel.
+// ---------------------------------------------------------------------------
+struct Problem {
+  int B, NH, T, DK, DV, L;  // L = chunk size
+  int NC;                   // number of chunks = ceil(T / L)
+  int BH;                   // B * NH
+  int gate_sigmoid;         // 0: log i = i_pre; 1: log i = logsigmoid(i_pre)
+  float key_scale;          // 1 / sqrt(DK)
+  uint32_t* err;            // device error word (see raise_error)
+  unsigned long long max_polls;  // spin limit of every bounded wait
+};
+
+// Gate workspace (all fp32, written by the gate kernels).
+//   bcum [BH, NC*L]  inclusive cumulative log forget gate inside each chunk
+//   acol [BH, NC*L]  column log-weight  a_s = log i_s - bcum_s (-inf on padding)
+//   amax [BH, NC*L]  running max of acol inside the chunk (prefix max)
+//   gtot [BH, NC]    chunk total of log forget gates (= bcum at the chunk end)
+//   mchk [BH, NC+1]  state stabiliser entering chunk k (k = NC: final m)
+struct Gates {
+  float* bcum;
+  float* acol;
+  float* amax;
+  float* gtot;
+  float* mchk;
+};
+
+__device__ __forceinline__ float to_float(float x) { return x; }
+__device__ __forceinline__ float to_float(__nv_bfloat16 x) { return __bfloat162float(x); }
+template <typename T> __device__ __forceinline__ T from_float(float x);
+template <> __device__ __forceinline__ float from_float<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_float<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+
+// log(sigmoid(x)) without overflow in either branch.
+__device__ __forceinline__ float logsigmoidf(float x) {
+  return x >= 0.f ? -log1pf(expf(-x)) : x - log1pf(expf(x));
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+}  // namespace mlstm
+
+// Launchers implemented in the individual .cu files.
+namespace mlstm {
+cudaError_t launch_gates(const Problem& p, const float* i_pre, const float* f_pre,
+                         const float* m0, Gates g, cudaStream_t st);
+cudaError_t launch_simt_states(const Problem& p, mlstm_dtype dt, const void* K, const void* V,
+                               const float* C0, const float* n0, Gates g, float* C_states,
+                               float* n_states, float* C_T, float* n_T, float* m_T,
+                               cudaStream_t st);
+cudaError_t launch_simt_parallel(const Problem& p, mlstm_dtype dt, const void* Q, const void* K,
+                                 const void* V, Gates g, const float* C_states,
+                                 const float* n_states, void* H, float* n_out, float* m_out,
+                                 cudaStream_t st);
+}  // namespace mlstm
