@@ -64,7 +64,8 @@ typedef enum {
   MLSTM_ERR_UNSUPPORTED = 2,  /* valid, but not supported by that algorithm */
   MLSTM_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed       */
   MLSTM_ERR_TIMEOUT = 4,      /* a device-side bounded wait ran out         */
-  MLSTM_ERR_DEVICE = 5        /* another device-side check failed           */
+  MLSTM_ERR_DEVICE = 5,       /* another device-side check failed           */
+  MLSTM_ERR_SCRATCH_TOO_SMALL = 6 /* needs more than the static scratch array */
 } mlstm_status;
 
 typedef enum { MLSTM_DT_F32 = 0, MLSTM_DT_BF16 = 1 } mlstm_dtype;
@@ -166,6 +167,35 @@ mlstm_status mlstm_profile_read(double* ms, uint64_t* launches, int n);
 
 /* Static name of a kernel family id (never NULL). */
 const char* mlstm_kernel_name(int id);
+
+/* The forward pass for callers that cannot allocate device memory.  The
+ * pages have no counterpart: this is a deployment variant of mlstm_fw().
+ *
+ * Some callers hold their inputs and outputs but have no way to allocate a
+ * workspace -- a plugin hook in a host framework that hands over tensors but
+ * no allocator, or a latency-critical loop that forbids cudaMalloc after
+ * start-up because it can synchronise the device.  This call takes the same
+ * arguments as mlstm_fw() minus the workspace and uses a scratch array that is
+ * part of the library's device image instead; it never allocates.
+ *
+ * Limits: the array holds mlstm_fw_static_scratch_capacity() bytes (16 MiB),
+ * which every GPU that loads the library keeps until the process exits.  A
+ * problem whose mlstm_fw_workspace_size() is larger returns
+ * MLSTM_ERR_SCRATCH_TOO_SMALL and launches nothing.  All calls share the one
+ * array, so calls that overlap on the GPU (other streams or host threads)
+ * race and must be serialised by the caller.  The first call on a device looks
+ * up the array's address with that device current; make it before any stream
+ * capture.  Other errors are those of mlstm_fw(). */
+mlstm_status mlstm_fw_static_scratch(const void* Q, const void* K, const void* V,
+                                     const float* i_pre, const float* f_pre, const float* C0,
+                                     const float* n0, const float* m0, void* H, float* C_T,
+                                     float* n_T, float* m_T, int B, int NH, int T, int DK, int DV,
+                                     int chunk_size, mlstm_dtype dtype,
+                                     mlstm_gate_mode gate_mode, mlstm_algo algo,
+                                     mlstm_stream_t stream);
+
+/* Bytes of the static scratch array used by mlstm_fw_static_scratch(). */
+size_t mlstm_fw_static_scratch_capacity(void);
 
 /* Static text for a status code (never NULL). */
 const char* mlstm_status_string(mlstm_status status);

@@ -12,6 +12,7 @@ import threading
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmlstm_fw.so")
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_DEVICE = range(6)
+ERR_SCRATCH_TOO_SMALL = 6
 DT_F32, DT_BF16 = 0, 1
 GATE_EXP, GATE_SIGMOID = 0, 1
 ALGO_AUTO, ALGO_SIMT, ALGO_TC, ALGO_TC_FUSED = 0, 1, 2, 3
@@ -28,6 +29,8 @@ SIGNATURES = {
     "mlstm_fw_gates_workspace_size": (_i, [_i, _i, _i, _i, ctypes.POINTER(_sz)]),
     "mlstm_fw_chunk_states": (_i, [_vp] * 13 + [_i] * 9 + [_vp, _sz, _vp]),
     "mlstm_fw_parallel": (_i, [_vp] * 11 + [_i] * 9 + [_vp, _sz, _vp]),
+    "mlstm_fw_static_scratch": (_i, [_vp] * 12 + [_i] * 9 + [_vp]),
+    "mlstm_fw_static_scratch_capacity": (_sz, []),
     "mlstm_last_device_error": (_i, [_vp]),
     "mlstm_set_watchdog": (None, [ctypes.c_uint64]),
     "mlstm_kernel_launches": (ctypes.c_uint64, []),

@@ -232,6 +232,8 @@ const char* mlstm_status_string(mlstm_status s) {
     case MLSTM_ERR_CUDA: return "CUDA error";
     case MLSTM_ERR_TIMEOUT: return "device-side bounded wait timed out";
     case MLSTM_ERR_DEVICE: return "device-side check failed";
+    case MLSTM_ERR_SCRATCH_TOO_SMALL:
+      return "problem needs more scratch than the library's static array holds";
   }
   return "unknown status";
 }

@@ -41,7 +41,7 @@ def test_exports_match_nm():
 
 
 def test_status_strings(L):
-    for s in range(6):
+    for s in range(7):
         assert _lib.status_string(s)
     assert _lib.status_string(99) == "unknown status"
     assert L.mlstm_abi_version() == 100
