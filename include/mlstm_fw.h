@@ -103,8 +103,11 @@ mlstm_status mlstm_fw(const void* Q, const void* K, const void* V, const float* 
                       mlstm_algo algo, void* workspace, size_t workspace_bytes,
                       mlstm_stream_t stream);
 
-/* Bytes of workspace the two calls below need (gate arrays only). */
-mlstm_status mlstm_fw_gates_workspace_size(int B, int NH, int T, int chunk_size, size_t* bytes);
+/* Bytes of workspace either of the two calls below needs for these
+ * arguments (the gate arrays, plus a bf16 copy of the chunk states for the
+ * tensor-core parallel call). */
+mlstm_status mlstm_fw_substep_workspace_size(int B, int NH, int T, int DK, int DV, int chunk_size,
+                                             mlstm_dtype dtype, mlstm_algo algo, size_t* bytes);
 
 /* Recurrent half of the chunkwise pass: the state entering every chunk,
  *   C_states [B, NH, NC, DK, DV], n_states [B, NH, NC, DK], m_states

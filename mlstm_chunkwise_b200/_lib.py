@@ -26,7 +26,8 @@ _sz = ctypes.c_size_t
 SIGNATURES = {
     "mlstm_fw_workspace_size": (_i, [_i, _i, _i, _i, _i, _i, _i, _i, ctypes.POINTER(_sz)]),
     "mlstm_fw": (_i, [_vp] * 12 + [_i] * 9 + [_vp, _sz, _vp]),
-    "mlstm_fw_gates_workspace_size": (_i, [_i, _i, _i, _i, ctypes.POINTER(_sz)]),
+    "mlstm_fw_substep_workspace_size": (_i, [_i, _i, _i, _i, _i, _i, _i, _i,
+                                             ctypes.POINTER(_sz)]),
     "mlstm_fw_chunk_states": (_i, [_vp] * 13 + [_i] * 9 + [_vp, _sz, _vp]),
     "mlstm_fw_parallel": (_i, [_vp] * 11 + [_i] * 9 + [_vp, _sz, _vp]),
     "mlstm_fw_static_scratch": (_i, [_vp] * 12 + [_i] * 9 + [_vp]),

@@ -51,10 +51,12 @@ def workspace_size(B, NH, T, DK, DV, chunk_size, dtype=torch.bfloat16, algo="aut
     return int(n.value)
 
 
-def gates_workspace_size(B, NH, T, chunk_size) -> int:
+def substep_workspace_size(B, NH, T, DK, DV, chunk_size, dtype=torch.bfloat16,
+                           algo="auto") -> int:
     n = ctypes.c_size_t(0)
-    _lib.check(_lib.lib().mlstm_fw_gates_workspace_size(B, NH, T, chunk_size, ctypes.byref(n)),
-               "mlstm_fw_gates_workspace_size")
+    _lib.check(_lib.lib().mlstm_fw_substep_workspace_size(B, NH, T, DK, DV, chunk_size, _DT[dtype],
+                                                          _ALGO[algo], ctypes.byref(n)),
+               "mlstm_fw_substep_workspace_size")
     return int(n.value)
 
 
@@ -148,8 +150,8 @@ def mlstm_fw_chunk_states(K, V, i_pre, f_pre, C0=None, n0=None, m0=None, *, chun
     C_T = torch.empty((B, NH, DK, DV), dtype=torch.float32, device=dev)
     n_T = torch.empty((B, NH, DK), dtype=torch.float32, device=dev)
     m_T = torch.empty((B, NH), dtype=torch.float32, device=dev)
-    ws = torch.empty(max(gates_workspace_size(B, NH, T, chunk_size), 1), dtype=torch.uint8,
-                     device=dev)
+    ws = torch.empty(max(substep_workspace_size(B, NH, T, DK, DV, chunk_size, dt, algo), 1),
+                     dtype=torch.uint8, device=dev)
     st = _lib.lib().mlstm_fw_chunk_states(
         _ptr(K), _ptr(V), _ptr(i_pre), _ptr(f_pre), _ptr(C0), _ptr(n0), _ptr(m0), _ptr(C_states),
         _ptr(n_states), _ptr(m_states), _ptr(C_T), _ptr(n_T), _ptr(m_T), B, NH, T, DK, DV,
@@ -169,8 +171,8 @@ def mlstm_fw_parallel(Q, K, V, i_pre, f_pre, C_states, n_states, m0=None, *,
     H = torch.empty((B, NH, T, DV), dtype=dt, device=dev)
     n_out = torch.empty((B, NH, T), dtype=torch.float32, device=dev)
     m_out = torch.empty((B, NH, T), dtype=torch.float32, device=dev)
-    ws = torch.empty(max(gates_workspace_size(B, NH, T, chunk_size), 1), dtype=torch.uint8,
-                     device=dev)
+    ws = torch.empty(max(substep_workspace_size(B, NH, T, DK, DV, chunk_size, dt, algo), 1),
+                     dtype=torch.uint8, device=dev)
     st = _lib.lib().mlstm_fw_parallel(
         _ptr(Q), _ptr(K), _ptr(V), _ptr(i_pre), _ptr(f_pre), _ptr(m0), _ptr(C_states),
         _ptr(n_states), _ptr(H), _ptr(n_out), _ptr(m_out), B, NH, T, DK, DV, chunk_size, _DT[dt],

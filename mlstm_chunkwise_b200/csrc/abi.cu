@@ -39,12 +39,6 @@ uint32_t* error_word_ptr() {
   return g_err_ptr[dev];
 }
 
-struct Layout {
-  size_t gates_bytes;   // bcum, acol, amax, gtot, mchk
-  size_t states_bytes;  // C_states, n_states (unfused only)
-  size_t total;
-};
-
 mlstm_status check_sizes(int B, int NH, int T, int DK, int DV, int L) {
   if (B < 1 || NH < 1 || T < 0 || DK < 1 || DV < 1) return MLSTM_ERR_INVALID_ARG;
   if (L < 64 || L % 64 != 0) return MLSTM_ERR_INVALID_ARG;
@@ -71,14 +65,36 @@ Problem make_problem(int B, int NH, int T, int DK, int DV, int L, mlstm_gate_mod
   return p;
 }
 
-Layout layout_for(const Problem& p, bool with_states) {
+struct Layout {
+  size_t gates_bytes;   // bcum, acol, amax, gtot, mchk
+  size_t states_bytes;  // chunk states kept between two kernels
+  size_t total;
+};
+
+// What a call needs the workspace for.
+enum class Mode { kFull, kStates, kParallel };
+
+size_t cb_bytes(const Problem& p) {
+  return round_up((size_t)p.BH * p.NC * (size_t)p.DK * p.DV * sizeof(__nv_bfloat16));
+}
+
+// Workspace layout: the gate arrays, then
+//   kFull/SIMT:     C_states fp32 [BH, NC, DK, DV], n_states fp32 [BH, NC, DK]
+//   kFull/TC:       C_states bf16 (operand copy), n_states fp32
+//   kParallel/TC:   C_states bf16 (converted from the caller's fp32 states)
+//   everything else: nothing more.
+Layout layout_for(const Problem& p, mlstm_algo a, Mode mode) {
   Layout l{};
   const size_t BH = (size_t)p.BH, tpad = (size_t)p.NC * p.L;
   l.gates_bytes = 3 * round_up(BH * tpad * sizeof(float)) + round_up(BH * p.NC * sizeof(float)) +
                   round_up(BH * (p.NC + 1) * sizeof(float));
-  if (with_states)
-    l.states_bytes = round_up(BH * p.NC * (size_t)p.DK * p.DV * sizeof(float)) +
-                     round_up(BH * p.NC * (size_t)p.DK * sizeof(float));
+  const size_t n_bytes = round_up(BH * p.NC * (size_t)p.DK * sizeof(float));
+  if (mode == Mode::kFull && a == MLSTM_ALGO_SIMT)
+    l.states_bytes = round_up(BH * p.NC * (size_t)p.DK * p.DV * sizeof(float)) + n_bytes;
+  else if (mode == Mode::kFull && a == MLSTM_ALGO_TC)
+    l.states_bytes = cb_bytes(p) + n_bytes;
+  else if (mode == Mode::kParallel && a == MLSTM_ALGO_TC)
+    l.states_bytes = cb_bytes(p);
   l.total = l.gates_bytes + l.states_bytes;
   return l;
 }
@@ -251,16 +267,22 @@ mlstm_status mlstm_fw_workspace_size(int B, int NH, int T, int DK, int DV, int c
   mlstm_algo a;
   s = resolve_algo(p, dtype, algo, true, &a);
   if (s != MLSTM_OK) return s;
-  *bytes = layout_for(p, a != MLSTM_ALGO_TC_FUSED).total;
+  *bytes = layout_for(p, a, Mode::kFull).total;
   return MLSTM_OK;
 }
 
-mlstm_status mlstm_fw_gates_workspace_size(int B, int NH, int T, int chunk_size, size_t* bytes) {
-  if (!bytes) return MLSTM_ERR_INVALID_ARG;
-  mlstm_status s = check_sizes(B, NH, T, 64, 64, chunk_size);
+mlstm_status mlstm_fw_substep_workspace_size(int B, int NH, int T, int DK, int DV, int chunk_size,
+                                             mlstm_dtype dtype, mlstm_algo algo, size_t* bytes) {
+  if (!bytes || !valid_enums(dtype, MLSTM_GATE_EXP, algo)) return MLSTM_ERR_INVALID_ARG;
+  mlstm_status s = check_sizes(B, NH, T, DK, DV, chunk_size);
   if (s != MLSTM_OK) return s;
-  Problem p = make_problem(B, NH, T, 64, 64, chunk_size, MLSTM_GATE_EXP);
-  *bytes = layout_for(p, false).gates_bytes;
+  Problem p = make_problem(B, NH, T, DK, DV, chunk_size, MLSTM_GATE_EXP);
+  mlstm_algo a;
+  s = resolve_algo(p, dtype, algo, false, &a);
+  if (s != MLSTM_OK) return s;
+  const size_t st = layout_for(p, a, Mode::kStates).total;
+  const size_t pa = layout_for(p, a, Mode::kParallel).total;
+  *bytes = st > pa ? st : pa;
   return MLSTM_OK;
 }
 
@@ -282,7 +304,7 @@ mlstm_status mlstm_fw(const void* Q, const void* K, const void* V, const float* 
   mlstm_algo a;
   s = resolve_algo(p, dtype, algo, true, &a);
   if (s != MLSTM_OK) return s;
-  const Layout lay = layout_for(p, a != MLSTM_ALGO_TC_FUSED);
+  const Layout lay = layout_for(p, a, Mode::kFull);
   if (workspace_bytes < lay.total || (lay.total > 0 && !workspace)) return MLSTM_ERR_INVALID_ARG;
   p.err = error_word_ptr();
   if (!p.err) return MLSTM_ERR_CUDA;
@@ -298,19 +320,20 @@ mlstm_status mlstm_fw(const void* Q, const void* K, const void* V, const float* 
       return launch_tc_fused(p, Q, K, V, C0, n0, g, H, C_T, n_T, m_T, st);
     }));
 
+  if (a == MLSTM_ALGO_TC) {
+    __nv_bfloat16* Cb = reinterpret_cast<__nv_bfloat16*>(rest);
+    float* n_states = reinterpret_cast<float*>(rest + cb_bytes(p));
+    s = from_cuda(launch_family(MLSTM_KERNEL_TC_STATES, 1, st, [&] {
+      return launch_tc_states(p, K, V, C0, n0, g, nullptr, Cb, n_states, C_T, n_T, m_T, st);
+    }));
+    if (s != MLSTM_OK) return s;
+    return from_cuda(launch_family(MLSTM_KERNEL_TC_PARALLEL, 1, st, [&] {
+      return launch_tc_parallel(p, Q, K, V, g, Cb, n_states, H, nullptr, nullptr, st);
+    }));
+  }
   float* C_states = reinterpret_cast<float*>(rest);
   float* n_states =
       reinterpret_cast<float*>(rest + round_up((size_t)p.BH * p.NC * (size_t)DK * DV * 4));
-  if (a == MLSTM_ALGO_TC) {
-    s = from_cuda(launch_family(MLSTM_KERNEL_TC_STATES, 1, st, [&] {
-      return launch_tc_states(p, K, V, C0, n0, g, C_states, n_states, C_T, n_T, m_T, st);
-    }));
-    if (s != MLSTM_OK) return s;
-    if (T == 0) return MLSTM_OK;
-    return from_cuda(launch_family(MLSTM_KERNEL_TC_PARALLEL, 1, st, [&] {
-      return launch_tc_parallel(p, Q, K, V, g, C_states, n_states, H, nullptr, nullptr, st);
-    }));
-  }
   s = from_cuda(launch_family(MLSTM_KERNEL_SIMT_STATES, 1, st, [&] {
     return launch_simt_states(p, dtype, K, V, C0, n0, g, C_states, n_states, C_T, n_T, m_T, st);
   }));
@@ -345,9 +368,8 @@ mlstm_status mlstm_fw_chunk_states(const void* K, const void* V, const float* i_
   mlstm_algo a;
   s = resolve_algo(p, dtype, algo, false, &a);
   if (s != MLSTM_OK) return s;
-  const Layout lay = layout_for(p, false);
-  if (workspace_bytes < lay.gates_bytes || (lay.gates_bytes > 0 && !workspace))
-    return MLSTM_ERR_INVALID_ARG;
+  const Layout lay = layout_for(p, a, Mode::kStates);
+  if (workspace_bytes < lay.total || (lay.total > 0 && !workspace)) return MLSTM_ERR_INVALID_ARG;
   p.err = error_word_ptr();
   if (!p.err) return MLSTM_ERR_CUDA;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -358,7 +380,7 @@ mlstm_status mlstm_fw_chunk_states(const void* K, const void* V, const float* i_
   if (s != MLSTM_OK) return s;
   if (a == MLSTM_ALGO_TC)
     return from_cuda(launch_family(MLSTM_KERNEL_TC_STATES, 1, st, [&] {
-      return launch_tc_states(p, K, V, C0, n0, g, C_states, n_states, C_T, n_T, m_T, st);
+      return launch_tc_states(p, K, V, C0, n0, g, C_states, nullptr, n_states, C_T, n_T, m_T, st);
     }));
   return from_cuda(launch_family(MLSTM_KERNEL_SIMT_STATES, 1, st, [&] {
     return launch_simt_states(p, dtype, K, V, C0, n0, g, C_states, n_states, C_T, n_T, m_T, st);
@@ -384,22 +406,27 @@ mlstm_status mlstm_fw_parallel(const void* Q, const void* K, const void* V, cons
   mlstm_algo a;
   s = resolve_algo(p, dtype, algo, false, &a);
   if (s != MLSTM_OK) return s;
-  const Layout lay = layout_for(p, false);
-  if (workspace_bytes < lay.gates_bytes || (lay.gates_bytes > 0 && !workspace))
-    return MLSTM_ERR_INVALID_ARG;
+  const Layout lay = layout_for(p, a, Mode::kParallel);
+  if (workspace_bytes < lay.total || (lay.total > 0 && !workspace)) return MLSTM_ERR_INVALID_ARG;
   if (T == 0) return MLSTM_OK;
   p.err = error_word_ptr();
   if (!p.err) return MLSTM_ERR_CUDA;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   Gates g;
-  carve_gates(p, static_cast<char*>(workspace), &g, nullptr);
+  char* rest = carve_gates(p, static_cast<char*>(workspace), &g, nullptr);
   s = from_cuda(launch_family(MLSTM_KERNEL_GATES, gate_launches(p), st,
                               [&] { return launch_gates(p, i_pre, f_pre, m0, g, st); }));
   if (s != MLSTM_OK) return s;
-  if (a == MLSTM_ALGO_TC)
-    return from_cuda(launch_family(MLSTM_KERNEL_TC_PARALLEL, 1, st, [&] {
-      return launch_tc_parallel(p, Q, K, V, g, C_states, n_states, H, n_out, m_out, st);
+  if (a == MLSTM_ALGO_TC) {
+    __nv_bfloat16* Cb = reinterpret_cast<__nv_bfloat16*>(rest);
+    s = from_cuda(launch_family(MLSTM_KERNEL_TC_PARALLEL, 1, st, [&] {
+      cudaError_t e =
+          launch_states_to_bf16(C_states, Cb, (size_t)p.BH * p.NC * (size_t)DK * DV, st);
+      if (e != cudaSuccess) return e;
+      return launch_tc_parallel(p, Q, K, V, g, Cb, n_states, H, n_out, m_out, st);
     }));
+    return s;
+  }
   return from_cuda(launch_family(MLSTM_KERNEL_SIMT_PARALLEL, 1, st, [&] {
     return launch_simt_parallel(p, dtype, Q, K, V, g, C_states, n_states, H, n_out, m_out, st);
   }));

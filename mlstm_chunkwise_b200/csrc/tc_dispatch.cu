@@ -1,19 +1,87 @@
-// Support predicates and launchers of the tensor-core kernels.
+// Support predicates, host-side tensor maps and launch glue of the
+// tensor-core kernels.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
 #include "tc.h"
+#include "tc_ptx.cuh"
 
 namespace mlstm {
 
-bool tc_unfused_supported(const Problem&) { return false; }
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+PFN_cuTensorMapEncodeTiled_v12000 encoder() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  return g_encode;
+}
+
+__global__ void states_to_bf16_kernel(const float4* __restrict__ src, uint2* __restrict__ dst,
+                                      size_t n4) {
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n4;
+       i += (size_t)gridDim.x * blockDim.x) {
+    const float4 v = src[i];
+    dst[i] = make_uint2(tc::pack_bf16x2(v.x, v.y), tc::pack_bf16x2(v.z, v.w));
+  }
+}
+
+}  // namespace
+
+bool encode_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1,
+                         uint64_t d2, uint32_t b0, uint32_t b1) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = encoder();
+  if (!enc || b0 * 2 != 128) return false;
+  const cuuint64_t dims[3] = {d0, d1, d2};
+  const cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
+  const cuuint32_t box[3] = {b0, b1, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool tc_unfused_supported(const Problem& p) {
+  return tc_states_supported(p) && tc_parallel_supported(p);
+}
+
 bool tc_fused_supported(const Problem&) { return false; }
 
-cudaError_t launch_tc_states(const Problem&, const void*, const void*, const float*, const float*,
-                             Gates, float*, float*, float*, float*, float*, cudaStream_t) {
-  return cudaErrorNotSupported;
+cudaError_t launch_tc_states(const Problem& p, const void* K, const void* V, const float* C0,
+                             const float* n0, Gates g, float* C_states, __nv_bfloat16* Cb,
+                             float* n_states, float* C_T, float* n_T, float* m_T,
+                             cudaStream_t st) {
+  return launch_tc_states_impl(p, K, V, C0, n0, g, C_states, Cb, n_states, C_T, n_T, m_T, st);
 }
-cudaError_t launch_tc_parallel(const Problem&, const void*, const void*, const void*, Gates,
-                               const float*, const float*, void*, float*, float*, cudaStream_t) {
-  return cudaErrorNotSupported;
+
+cudaError_t launch_tc_parallel(const Problem& p, const void* Q, const void* K, const void* V,
+                               Gates g, const __nv_bfloat16* Cb, const float* n_states, void* H,
+                               float* n_out, float* m_out, cudaStream_t st) {
+  return launch_tc_parallel_bf16states(p, Q, K, V, g, Cb, n_states, H, n_out, m_out, st);
 }
+
+cudaError_t launch_states_to_bf16(const float* src, __nv_bfloat16* dst, size_t n,
+                                  cudaStream_t st) {
+  const size_t n4 = n / 4;  // DK * DV is a multiple of 4 for every supported shape
+  if (n4 == 0) return cudaSuccess;
+  const int blocks = (int)((n4 + 255) / 256 < 148 * 16 ? (n4 + 255) / 256 : 148 * 16);
+  states_to_bf16_kernel<<<blocks, 256, 0, st>>>(reinterpret_cast<const float4*>(src),
+                                                reinterpret_cast<uint2*>(dst), n4);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_tc_fused(const Problem&, const void*, const void*, const void*, const float*,
                             const float*, Gates, void*, float*, float*, float*, cudaStream_t) {
   return cudaErrorNotSupported;

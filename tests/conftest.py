@@ -27,3 +27,16 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+@pytest.fixture(autouse=True)
+def _short_device_watchdog(request):
+    """GPU tests run with a short bounded-wait limit (~67 ms per wait) so that
+    a pipeline bug surfaces as MLSTM_ERR_TIMEOUT quickly instead of slowly."""
+    if "gpu" not in request.keywords:
+        yield
+        return
+    from mlstm_chunkwise_b200 import api
+    api.set_watchdog(1 << 22)
+    yield
+    api.set_watchdog(0)
