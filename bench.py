@@ -287,6 +287,8 @@ def run_ours(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
     w = pick_workload(args.workload)
+    if args.batch:
+        w = w.replace(name=f"{w.name}_B{args.batch}", B=args.batch)
     x = make_inputs(w, seed=w.seed + rank)
     d = {k: (None if v is None else v.to(dev)) for k, v in x.items()}
     B, NH, T, DK, DV, L = w.B, w.NH, w.T, w.DK, w.DV, w.chunk_size
@@ -362,17 +364,20 @@ def run_ours(args):
         for k, v in out.items():
             hout[k].copy_(v, non_blocking=True)
 
-    e2e_step()
-    torch.cuda.synchronize()
+    e2e_ms = float("nan")
+    if not args.no_e2e:
+        e2e_step()
+        torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
+    if not args.no_e2e:
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = e0.elapsed_time(e1)
     if world > 1:
         t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -381,7 +386,7 @@ def run_ours(args):
     tokens_per_step = B * T * world
     ms_per_step = elapsed_ms / args.steps
     value = tokens_per_step / (ms_per_step / 1e3)
-    e2e_value = tokens_per_step * e2e_steps / (e2e_ms / 1e3)
+    e2e_value = None if args.no_e2e else tokens_per_step * e2e_steps / (e2e_ms / 1e3)
 
     # --- roofline of the dominant kernel ------------------------------------
     peaks, peak_src = load_peaks()
@@ -431,8 +436,9 @@ def run_ours(args):
         "frac_bf16_peak": (total_flops / (ms_per_step / 1e3) / 1e12) / peaks["bf16_tflops"],
         "roofline": roof,
         "kernels_ms_per_step": {k: v[0] / calls for k, v in kern.items()},
-        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+        "e2e": None if args.no_e2e else {
+            "value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "steps": e2e_steps},
         "gpu_launches": int(launches),
         "clocks": clocks,
     }
@@ -460,6 +466,10 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true",
+                    help="skip the host-buffer end-to-end loop (profiling runs)")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="override the workload's batch size (smaller profiling captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
