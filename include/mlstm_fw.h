@@ -139,6 +139,12 @@ mlstm_status mlstm_fw_parallel(const void* Q, const void* K, const void* V, cons
  * MLSTM_ERR_CUDA if the synchronisation itself failed. */
 mlstm_status mlstm_last_device_error(mlstm_stream_t stream);
 
+/* The raw device error word read by the last mlstm_last_device_error() call:
+ * bit 0 a bounded wait ran out, bit 1 a bounds check failed, bit 2 a TMEM
+ * allocation check failed; bits 8..15 identify the first wait that ran out
+ * (a kernel-specific site number, for diagnosis). */
+uint32_t mlstm_last_device_error_word(void);
+
 /* Spin limit of every bounded device-side wait (default 2^26 polls, about a
  * second or more).  Affects launches made after the call.  0 restores the
  * default.  Not thread-safe with concurrent launches. */

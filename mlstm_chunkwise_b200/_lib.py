@@ -33,6 +33,7 @@ SIGNATURES = {
     "mlstm_fw_static_scratch": (_i, [_vp] * 12 + [_i] * 9 + [_vp]),
     "mlstm_fw_static_scratch_capacity": (_sz, []),
     "mlstm_last_device_error": (_i, [_vp]),
+    "mlstm_last_device_error_word": (ctypes.c_uint32, []),
     "mlstm_set_watchdog": (None, [ctypes.c_uint64]),
     "mlstm_kernel_launches": (ctypes.c_uint64, []),
     "mlstm_profile_enable": (None, [_i]),

@@ -18,6 +18,7 @@ namespace {
 __device__ uint32_t g_error_word = 0;
 
 constexpr unsigned long long kDefaultPolls = 1ull << 26;
+uint32_t g_last_error_word = 0;
 unsigned long long g_max_polls = kDefaultPolls;
 
 constexpr size_t kAlign = 256;
@@ -195,6 +196,8 @@ using namespace mlstm;
 extern "C" {
 
 int mlstm_abi_version(void) { return 100; }
+
+uint32_t mlstm_last_device_error_word(void) { return g_last_error_word; }
 
 uint64_t mlstm_kernel_launches(void) { return g_launches.load(); }
 
@@ -439,6 +442,7 @@ mlstm_status mlstm_last_device_error(mlstm_stream_t stream) {
   if (!w) return MLSTM_ERR_CUDA;
   uint32_t v = 0;
   if (cudaMemcpy(&v, w, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return MLSTM_ERR_CUDA;
+  g_last_error_word = v;
   if (v != 0) {
     const uint32_t zero = 0;
     if (cudaMemcpy(w, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess)

@@ -36,6 +36,10 @@ cudaError_t launch_tc_states_impl(const Problem& p, const void* K, const void* V
                                   const float* n0, Gates g, float* C_states, __nv_bfloat16* Cb,
                                   float* n_states, float* C_T, float* n_T, float* m_T,
                                   cudaStream_t st);
+bool tc_parallel_wide_supported(const Problem& p);
+cudaError_t launch_tc_parallel_wide(const Problem& p, const void* Q, const void* K, const void* V,
+                                    Gates g, const __nv_bfloat16* Cb, const float* n_states,
+                                    void* H, float* n_out, float* m_out, cudaStream_t st);
 cudaError_t launch_tc_parallel_bf16states(const Problem& p, const void* Q, const void* K,
                                           const void* V, Gates g, const __nv_bfloat16* Cb,
                                           const float* n_states, void* H, float* n_out,

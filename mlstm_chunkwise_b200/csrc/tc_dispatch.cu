@@ -69,6 +69,11 @@ cudaError_t launch_tc_states(const Problem& p, const void* K, const void* V, con
 cudaError_t launch_tc_parallel(const Problem& p, const void* Q, const void* K, const void* V,
                                Gates g, const __nv_bfloat16* Cb, const float* n_states, void* H,
                                float* n_out, float* m_out, cudaStream_t st) {
+  // Chunks of at most 256 tokens: one item per query tile covering every value
+  // column (S computed once).  Longer chunks: one item per query tile and
+  // value tile.
+  if (tc_parallel_wide_supported(p))
+    return launch_tc_parallel_wide(p, Q, K, V, g, Cb, n_states, H, n_out, m_out, st);
   return launch_tc_parallel_bf16states(p, Q, K, V, g, Cb, n_states, H, n_out, m_out, st);
 }
 

@@ -1,10 +1,10 @@
 // G3: intra-chunk TFLA kernel on tcgen05 (the parallel half of the chunkwise
-// mLSTM forward pass).
+// mLSTM forward pass), persistent.
 //
 // "Tiled Flash Linear Attention: More Efficient Linear RNN and xLSTM Kernels"
 // (abstract): the intra-chunk part is tiled a second time, over query and
-// key/value blocks, so the chunk size is not tied to the tile size.  Here one
-// CTA owns 128 query rows (one L_Q tile) of one chunk and DVT value columns of
+// key/value blocks, so the chunk size is not tied to the tile size.  A work
+// item is 128 query rows (one L_Q tile) of one chunk and DVT value columns of
 // one (b, h); it walks the L_KV = 128 key/value tiles of the chunk up to the
 // diagonal.  For row r (token t) of chunk k with mu_r = max(m_k, amax_r):
 //
@@ -13,15 +13,27 @@
 //   den_r = e^{m_k - mu_r} n_k.q_r    +  sum_{s<=r} P_rs
 //   h_r   = O_r / max(|den_r|, e^{-(bcum_r + mu_r)})
 //
-// Roles (192 threads):
-//   warp 0      TMA producer: Q tile once, then K / C / V slabs through a ring
+// The grid is at most one CTA per SM; each CTA takes items
+// blockIdx.x, blockIdx.x + gridDim.x, ...  Items are numbered with the value
+// tile fastest, then the query tile, then (b, h), so the CTAs running at the
+// same time share chunks (K, V and the chunk state stay in L2).  The TMA
+// producer runs ahead across item boundaries, so the next item's loads overlap
+// the current item's P.V and epilogue.
+//
+// Roles (320 threads):
+//   warp 0      TMA producer: Q tile per item, K / C / V slabs through a ring
 //   warp 1      TMEM owner and single-thread MMA issuer
-//   warps 2..5  one thread per query row (= TMEM lane): gating of S into P,
-//               rescaling of the inter-chunk term, row sums, epilogue.
-// TMEM (512 columns): O accumulator [128 x DVT] at column 0, two S buffers
-// [128 x 128] at columns 256 and 384.  Shared memory: Q tile (DK/64 swizzled
-// slabs), a ring of NSTAGE slabs, the bf16 P tile (A operand of P.V).
-// MMA order: S_0, Q.C, { S_i, P_{i-1}.V_{i-1} }, P_last.V_last.
+//   warps 2..9  two threads per query row (= TMEM lane), each owning half of
+//               the columns: gating of S into P, rescaling of the inter-chunk
+//               term, row sums, epilogue.
+// TMEM (512 columns): the O accumulator at column 0 -- for DVT <= 128 a second
+// one at column 128, used by alternate items so that one item's epilogue
+// overlaps the next item's MMAs -- and two S buffers [128 x 128] at columns
+// 256 and 384.  Shared
+// memory: the Q tile (DK/64 swizzled slabs), a ring of 16 KB slabs as deep as
+// the remaining space allows (7 stages at DK = 256), the bf16 P tile (A
+// operand of P.V), the per-item column weights and n_k.
+// MMA order per item: S_0, Q.C, { S_i, P_{i-1}.V_{i-1} }, P_last.V_last.
 #include <cuda.h>
 
 #include "tc.h"
@@ -32,54 +44,78 @@ namespace {
 
 using namespace tc;
 
-constexpr int kThreads = 192;
-constexpr int kQT = 128;  // query rows per CTA
+constexpr int kThreads = 320;
+constexpr int kQT = 128;  // query rows per item
 constexpr int kKT = 128;  // key/value rows per intra tile
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColO = 0, kColS0 = 256, kColS1 = 384;
+constexpr uint32_t kColS0 = 256, kColS1 = 384;  // O buffer(s) at columns 0 (and 128)
 constexpr int kMaxL = 1024;  // largest chunk this kernel handles
 
 template <int DK, int DVT>
 struct Cfg {
+  static_assert(DVT == 64 || DVT == 128 || DVT == 256, "value tile of 64, 128 or 256 columns");
+  // Two O accumulators (alternating between items) fit next to the two S
+  // buffers only for value tiles of at most 128 columns.
+  static constexpr int kOBufs = DVT <= 128 ? 2 : 1;
   static constexpr int kSlabsK = DK / 64;
   static constexpr uint32_t kQBytes = kQT * DK * 2;
-  static constexpr uint32_t kKSlabBytes = kKT * 128;        // 128 rows x 64 bf16
+  static constexpr uint32_t kKSlabBytes = kKT * 128;           // 128 rows x 64 bf16
   static constexpr uint32_t kMNSlabBytes = (DVT / 64) * 8192;  // 64 rows x DVT bf16
   static constexpr uint32_t kStageBytes = kKSlabBytes > kMNSlabBytes ? kKSlabBytes : kMNSlabBytes;
-  static constexpr int kStages = kStageBytes >= 32768 ? 3 : 4;
   static constexpr uint32_t kPBytes = kQT * kKT * 2;
+  static constexpr uint32_t kMiscBytes = 2 * kMaxL * 4 + 2 * DK * 4 + 256 * 4 + 512;
+  static constexpr uint32_t kBudget = 227 * 1024 - 1024;  // minus alignment slack
+  static constexpr int kStagesFit = (int)((kBudget - kQBytes - kPBytes - kMiscBytes) / kStageBytes);
+  static constexpr int kStages = kStagesFit > 12 ? 12 : kStagesFit;
+  static_assert(kStages >= 3, "ring too shallow");
   static constexpr uint32_t kOffQ = 0;
   static constexpr uint32_t kOffStage = kOffQ + kQBytes;
   static constexpr uint32_t kOffP = kOffStage + kStages * kStageBytes;
-  static constexpr uint32_t kOffAcol = kOffP + kPBytes;          // float[kMaxL]
-  static constexpr uint32_t kOffN = kOffAcol + kMaxL * 4;        // float[DK]
-  static constexpr uint32_t kOffBar = kOffN + DK * 4;            // barriers
-  static constexpr int kNumBars = 2 * 4 + 1 + 2 + 2 + 1 + 1 + 1 + 1;
-  static constexpr uint32_t kOffTmemSlot = kOffBar + kNumBars * 8;
+  static constexpr uint32_t kOffAcol = kOffP + kPBytes;      // float[2][kMaxL]
+  static constexpr uint32_t kOffN = kOffAcol + 2 * kMaxL * 4;  // float[2][DK]
+  static constexpr uint32_t kOffRed = kOffN + 2 * DK * 4;      // float[256]
+  static constexpr uint32_t kOffBar = kOffRed + 256 * 4;       // barriers
+  static constexpr uint32_t kOffTmemSlot = kOffBar + 360;
   static constexpr uint32_t kBytes = kOffTmemSlot + 16;
   static constexpr uint32_t kSmem = kBytes + 1024;  // slack for 1024-byte alignment
+  static_assert(kSmem <= 227 * 1024, "shared memory");
 };
 
+// Barrier addresses, computed from one base (no arrays: a runtime-indexed
+// array would live in local memory).
 struct Bars {
-  uint32_t full[4], empty[4], q_full, s_full[2], s_empty[2], inter_done, p_full, p_empty, o_done;
+  uint32_t a;
+  __device__ __forceinline__ uint32_t full(int i) const { return a + 8 * i; }
+  __device__ __forceinline__ uint32_t empty(int i) const { return a + 128 + 8 * i; }
+  __device__ __forceinline__ uint32_t q_full() const { return a + 256; }
+  __device__ __forceinline__ uint32_t q_empty() const { return a + 264; }
+  __device__ __forceinline__ uint32_t s_full(int b) const { return a + 272 + 8 * b; }
+  __device__ __forceinline__ uint32_t s_empty(int b) const { return a + 288 + 8 * b; }
+  __device__ __forceinline__ uint32_t inter_done() const { return a + 304; }
+  __device__ __forceinline__ uint32_t p_full() const { return a + 312; }
+  __device__ __forceinline__ uint32_t p_empty() const { return a + 320; }
+  __device__ __forceinline__ uint32_t o_done() const { return a + 328; }
+  __device__ __forceinline__ uint32_t o_empty(int b) const { return a + 336 + 8 * b; }
+  __device__ __forceinline__ uint32_t mma_idle() const { return a + 352; }
 };
 
-template <int DK, int DVT>
-__device__ __forceinline__ Bars make_bars(uint32_t base) {
-  Bars b;
-  uint32_t a = base + Cfg<DK, DVT>::kOffBar;
-  for (int i = 0; i < 4; ++i) b.full[i] = a + 8 * i;
-  for (int i = 0; i < 4; ++i) b.empty[i] = a + 32 + 8 * i;
-  b.q_full = a + 64;
-  b.s_full[0] = a + 72;
-  b.s_full[1] = a + 80;
-  b.s_empty[0] = a + 88;
-  b.s_empty[1] = a + 96;
-  b.inter_done = a + 104;
-  b.p_full = a + 112;
-  b.p_empty = a + 120;
-  b.o_done = a + 128;
-  return b;
+// Work item -> (b*h, query tile, value tile).
+struct Item {
+  int bh, t0, dv0, k, c0, n_kv;
+};
+
+__device__ __forceinline__ Item decode_item(int it, const Problem& p, int n_dv, int n_q) {
+  Item x;
+  const int d = it % n_dv;
+  const int rest = it / n_dv;
+  const int qt = rest % n_q;
+  x.bh = rest / n_q;
+  x.t0 = qt * kQT;
+  x.dv0 = d * (p.DV / n_dv);
+  x.k = x.t0 / p.L;
+  x.c0 = x.k * p.L;
+  x.n_kv = (x.t0 - x.c0) / kKT + 1;
+  return x;
 }
 
 template <int DK, int DVT>
@@ -88,53 +124,47 @@ tc_parallel_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_c,
                    Problem p, Gates g, const float* __restrict__ n_states,
                    __nv_bfloat16* __restrict__ H, float* __restrict__ n_out,
-                   float* __restrict__ m_out) {
+                   float* __restrict__ m_out, int n_items) {
   using C = Cfg<DK, DVT>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
-  const Bars bar = make_bars<DK, DVT>(sbase);
+  const Bars bar{sbase + C::kOffBar};
   float* acol_s = reinterpret_cast<float*>(smem + C::kOffAcol);
   float* n_s = reinterpret_cast<float*>(smem + C::kOffN);
+  float* red_s = reinterpret_cast<float*>(smem + C::kOffRed);
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + C::kOffTmemSlot);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int dv0 = blockIdx.x * DVT;
-  const int t0 = blockIdx.y * kQT;
-  const int bh = blockIdx.z;
-  const int L = p.L;
-  const int k = t0 / L;
-  const int c0 = k * L;                    // first token of the chunk
-  const int n_kv = (t0 - c0) / kKT + 1;    // key/value tiles up to the diagonal
-  const long tpad = (long)p.NC * L;
-  const float m_in = g.mchk[(long)bh * (p.NC + 1) + k];
+  const int n_dv = p.DV / DVT;
+  const int n_q = (p.T + kQT - 1) / kQT;
+  const long tpad = (long)p.NC * p.L;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::kStages; ++i) {
-      mbar_init(bar.full[i], 1);
-      mbar_init(bar.empty[i], 1);
+      mbar_init(bar.full(i), 1);
+      mbar_init(bar.empty(i), 1);
     }
-    mbar_init(bar.q_full, 1);
+    mbar_init(bar.q_full(), 1);
+    mbar_init(bar.q_empty(), 1 + 256);  // MMA commit + the row threads' reads of Q
     for (int i = 0; i < 2; ++i) {
-      mbar_init(bar.s_full[i], 1);
-      mbar_init(bar.s_empty[i], 128);
+      mbar_init(bar.s_full(i), 1);
+      mbar_init(bar.s_empty(i), 256);
     }
-    mbar_init(bar.inter_done, 1);
-    mbar_init(bar.p_full, 128);
-    mbar_init(bar.p_empty, 1);
-    mbar_init(bar.o_done, 1);
+    mbar_init(bar.inter_done(), 1);
+    mbar_init(bar.p_full(), 256);
+    mbar_init(bar.p_empty(), 1);
+    mbar_init(bar.o_done(), 1);
+    mbar_init(bar.o_empty(0), 256);
+    mbar_init(bar.o_empty(1), 256);
+    mbar_init(bar.mma_idle(), 1);
     fence_barrier_init();
   }
   if (warp == 1) {
     tmem_alloc(smem_u32((const void*)tmem_slot), kTmemCols);
     tmem_relinquish();
   }
-  // Column weights of the chunk prefix [c0, t0 + 128), pre-multiplied by log2(e).
-  for (int j = threadIdx.x; j < n_kv * kKT; j += kThreads)
-    acol_s[j] = g.acol[(long)bh * tpad + c0 + j] * 1.4426950408889634f;
-  for (int j = threadIdx.x; j < DK; j += kThreads)
-    n_s[j] = n_states[((long)bh * p.NC + k) * DK + j];
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -147,66 +177,78 @@ tc_parallel_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
       tma_prefetch_desc(&tm_c);
-      mbar_expect_tx(bar.q_full, C::kQBytes);
-      for (int c = 0; c < C::kSlabsK; ++c)
-        tma_load_3d(sbase + C::kOffQ + c * 16384, &tm_q, c * 64, t0, bh, bar.q_full);
       int slab = 0;
       bool ok = true;
       auto next_stage = [&](uint32_t bytes) -> uint32_t {
         const int s = slab % C::kStages, u = slab / C::kStages;
-        if (u > 0) ok = ok && mbar_wait(bar.empty[s], (u - 1) & 1, p);
-        mbar_expect_tx(bar.full[s], bytes);
+        if (u > 0) ok = ok && mbar_wait(bar.empty(s), (u - 1) & 1, p, 1);
+        mbar_expect_tx(bar.full(s), bytes);
         ++slab;
         return (uint32_t)s;
       };
-      auto load_k = [&](int i) {
+      int n = 0;
+      for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++n) {
+        const Item x = decode_item(it, p, n_dv, n_q);
+        auto load_k = [&](int i) {
+          for (int c = 0; c < C::kSlabsK && ok; ++c) {
+            const uint32_t s = next_stage(C::kKSlabBytes);
+            tma_load_3d(sbase + C::kOffStage + s * C::kStageBytes, &tm_k, c * 64, x.c0 + i * kKT,
+                        x.bh, bar.full(s));
+          }
+        };
+        auto load_v = [&](int i) {
+          for (int v = 0; v < 2 && ok; ++v) {
+            const uint32_t s = next_stage(C::kMNSlabBytes);
+            for (int b = 0; b < DVT / 64; ++b)
+              tma_load_3d(sbase + C::kOffStage + s * C::kStageBytes + b * 8192, &tm_v,
+                          x.dv0 + b * 64, x.c0 + i * kKT + v * 64, x.bh, bar.full(s));
+          }
+        };
+        // Q before any ring slab of this item: the MMA consumes nothing of the
+        // item until Q has landed, so a ring slab issued first could wait for
+        // a stage that only frees after Q arrives.
+        if (n > 0) ok = mbar_wait(bar.q_empty(), (n - 1) & 1, p, 2);
+        if (!ok) break;
+        mbar_expect_tx(bar.q_full(), C::kQBytes);
+        for (int c = 0; c < C::kSlabsK; ++c)
+          tma_load_3d(sbase + C::kOffQ + c * 16384, &tm_q, c * 64, x.t0, x.bh, bar.q_full());
+        load_k(0);
         for (int c = 0; c < C::kSlabsK && ok; ++c) {
-          const uint32_t s = next_stage(C::kKSlabBytes);
-          tma_load_3d(sbase + C::kOffStage + s * C::kStageBytes, &tm_k, c * 64, c0 + i * kKT, bh,
-                      bar.full[s]);
-        }
-      };
-      auto load_v = [&](int i) {
-        for (int v = 0; v < 2 && ok; ++v) {
           const uint32_t s = next_stage(C::kMNSlabBytes);
           for (int b = 0; b < DVT / 64; ++b)
-            tma_load_3d(sbase + C::kOffStage + s * C::kStageBytes + b * 8192, &tm_v, dv0 + b * 64,
-                        c0 + i * kKT + v * 64, bh, bar.full[s]);
+            tma_load_3d(sbase + C::kOffStage + s * C::kStageBytes + b * 8192, &tm_c, x.dv0 + b * 64,
+                        c * 64, x.bh * p.NC + x.k, bar.full(s));
         }
-      };
-      load_k(0);
-      for (int c = 0; c < C::kSlabsK && ok; ++c) {
-        const uint32_t s = next_stage(C::kMNSlabBytes);
-        for (int b = 0; b < DVT / 64; ++b)
-          tma_load_3d(sbase + C::kOffStage + s * C::kStageBytes + b * 8192, &tm_c, dv0 + b * 64,
-                      c * 64, bh * p.NC + k, bar.full[s]);
+        for (int i = 1; i < x.n_kv && ok; ++i) {
+          load_k(i);
+          load_v(i - 1);
+        }
+        load_v(x.n_kv - 1);
       }
-      for (int i = 1; i < n_kv && ok; ++i) {
-        load_k(i);
-        load_v(i - 1);
-      }
-      load_v(n_kv - 1);
-      // Drain: every issued stage must have landed before the CTA may exit.
+      // Drain: every issued load must have landed before the CTA may exit.
       for (int q = (slab > C::kStages ? slab - C::kStages : 0); q < slab; ++q)
-        mbar_wait(bar.full[q % C::kStages], (q / C::kStages) & 1, p);
+        mbar_wait(bar.full(q % C::kStages), (q / C::kStages) & 1, p, 13);
+      if (n > 0) mbar_wait(bar.q_full(), (n - 1) & 1, p, 14);
     }
   } else if (warp == 1) {
     // ---------------------------- MMA issuer ------------------------------
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16(128, kKT, 0, 0);
       constexpr uint32_t idO = idesc_bf16(128, DVT, 0, 1);
-      bool ok = mbar_wait(bar.q_full, 0, p);
-      int slab = 0;
+      bool ok = true;
+      int slab = 0;   // ring position
+      int tile = 0;   // S tiles issued so far (all items)
+      int ptile = 0;  // P.V tiles issued so far
       auto take = [&]() -> uint32_t {
         const int s = slab % C::kStages, u = slab / C::kStages;
-        ok = ok && mbar_wait(bar.full[s], u & 1, p);
+        ok = ok && mbar_wait(bar.full(s), u & 1, p, 5);
         tc_fence_after();
         ++slab;
         return (uint32_t)s;
       };
-      auto mma_s = [&](int i) {
-        const int buf = i & 1;
-        if (i >= 2) ok = ok && mbar_wait(bar.s_empty[buf], ((i >> 1) - 1) & 1, p);
+      auto mma_s = [&]() {
+        const int buf = tile & 1;
+        if (tile >= 2) ok = ok && mbar_wait(bar.s_empty(buf), ((tile >> 1) - 1) & 1, p, 4);
         tc_fence_after();
         const uint32_t d = tmem + (buf ? kColS1 : kColS0);
         for (int c = 0; c < C::kSlabsK; ++c) {
@@ -218,12 +260,14 @@ tc_parallel_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
           for (int kk = 0; kk < 4; ++kk)
             mma_bf16_ss(d, sdesc_sw128(a0 + kk * 32, 16, 1024), sdesc_sw128(b0 + kk * 32, 16, 1024),
                         idS, (c | kk) != 0);
-          mma_commit(bar.empty[s]);
+          mma_commit(bar.empty(s));
         }
-        mma_commit(bar.s_full[buf]);
+        mma_commit(bar.s_full(buf));
+        ++tile;
       };
-      auto mma_pv = [&](int i) {
-        ok = ok && mbar_wait(bar.p_full, i & 1, p);
+      int ob = 0;  // output buffer of the current item
+      auto mma_pv = [&]() {
+        ok = ok && mbar_wait(bar.p_full(), ptile & 1, p, 7);
         tc_fence_after();
         for (int v = 0; v < 2; ++v) {
           const uint32_t s = take();
@@ -232,148 +276,231 @@ tc_parallel_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
           const uint32_t b0 = sbase + C::kOffStage + s * C::kStageBytes;
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            mma_bf16_ss(tmem + kColO, sdesc_sw128(a0 + kk * 32, 16, 1024),
+            mma_bf16_ss(tmem + ob * 128u, sdesc_sw128(a0 + kk * 32, 16, 1024),
                         sdesc_sw128(b0 + kk * 2048, 8192, 1024), idO, 1);
-          mma_commit(bar.empty[s]);
+          mma_commit(bar.empty(s));
         }
-        mma_commit(bar.p_empty);
+        mma_commit(bar.p_empty());
+        ++ptile;
       };
-      if (ok) mma_s(0);
-      for (int c = 0; c < C::kSlabsK && ok; ++c) {  // inter-chunk term Q.C_k
-        const uint32_t s = take();
-        if (!ok) break;
-        const uint32_t a0 = sbase + C::kOffQ + c * 16384;
-        const uint32_t b0 = sbase + C::kOffStage + s * C::kStageBytes;
+      int n = 0;
+      for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++n) {
+        const Item x = decode_item(it, p, n_dv, n_q);
+        ok = mbar_wait(bar.q_full(), n & 1, p, 3);
+        if (ok) mma_s();
+        // O buffers alternate between items (when there are two): the epilogue
+        // of item n - kOBufs must have drained this one.
+        ob = n % C::kOBufs;
+        if (n >= C::kOBufs)
+          ok = ok && mbar_wait(bar.o_empty(ob), ((n / C::kOBufs) - 1) & 1, p, 6);
+        tc_fence_after();
+        for (int c = 0; c < C::kSlabsK && ok; ++c) {  // inter-chunk term Q.C_k
+          const uint32_t s = take();
+          if (!ok) break;
+          const uint32_t a0 = sbase + C::kOffQ + c * 16384;
+          const uint32_t b0 = sbase + C::kOffStage + s * C::kStageBytes;
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_bf16_ss(tmem + kColO, sdesc_sw128(a0 + kk * 32, 16, 1024),
-                      sdesc_sw128(b0 + kk * 2048, 8192, 1024), idO, (c | kk) != 0);
-        mma_commit(bar.empty[s]);
+          for (int kk = 0; kk < 4; ++kk)
+            mma_bf16_ss(tmem + ob * 128u, sdesc_sw128(a0 + kk * 32, 16, 1024),
+                        sdesc_sw128(b0 + kk * 2048, 8192, 1024), idO, (c | kk) != 0);
+          mma_commit(bar.empty(s));
+        }
+        if (!ok) break;
+        mma_commit(bar.inter_done());
+        for (int i = 1; i < x.n_kv && ok; ++i) {
+          mma_s();
+          if (ok) mma_pv();
+        }
+        if (!ok) break;
+        mma_commit(bar.q_empty());  // every MMA that reads Q has been issued
+        mma_pv();
+        if (!ok) break;
+        mma_commit(bar.o_done());
       }
-      if (ok) mma_commit(bar.inter_done);
-      for (int i = 1; i < n_kv && ok; ++i) {
-        mma_s(i);
-        if (ok) mma_pv(i - 1);
-      }
-      if (ok) mma_pv(n_kv - 1);
-      mma_commit(bar.o_done);  // also orders every MMA above before teardown
-      mbar_wait(bar.o_done, 0, p);
+      mma_commit(bar.mma_idle());  // completes once every MMA above has finished
+      mbar_wait(bar.mma_idle(), 0, p, 15);
     }
   } else {
     // ------------------- gating / softmax / epilogue ----------------------
+    // 256 row threads: half h = 0 (warps 2..5) owns S columns [0, 64), the
+    // first DVT/2 output columns and the first half of the Q.n dot product;
+    // half h = 1 (warps 6..9) owns the other halves.  Both halves of a row
+    // combine their partial denominators once, in the epilogue.
     const int q = warp & 3;              // TMEM lane quadrant of this warp
     const int r = q * 32 + lane;         // query row in the tile = TMEM lane
-    const int t = t0 + r;
+    const int rt = threadIdx.x - 64;     // 0..255 among the row threads
+    const int h = rt >> 7;               // column half
     const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16);
-    const float amax = g.amax[(long)bh * tpad + t];
-    const float bc = g.bcum[(long)bh * tpad + t];
-    const float mu = fmaxf(m_in, amax);
-    const float mu2 = mu * 1.4426950408889634f;
-    const float f_inter = expf(m_in - mu);
     const float ks = p.key_scale;
+    constexpr int kHalfO = DVT / 2;
+    constexpr int kSlabsPerHalf = (C::kSlabsK + 1) / 2;
     bool ok = true;
+    int tile = 0;
+    int n = 0;
 
-    // den_inter = q_r . n_k from the swizzled Q tile.
-    ok = mbar_wait(bar.q_full, 0, p);
-    float dn = 0.f;
-    for (int c = 0; c < C::kSlabsK; ++c) {
-      const uint8_t* slab_ptr = smem + C::kOffQ + c * 16384;
+    // Per-item values, fetched one item ahead.
+    auto fetch_rows = [&](const Item& x, float& m_in, float& amax, float& bc) {
+      const int t = x.t0 + r;
+      m_in = g.mchk[(long)x.bh * (p.NC + 1) + x.k];
+      amax = g.amax[(long)x.bh * tpad + t];
+      bc = g.bcum[(long)x.bh * tpad + t];
+    };
+    auto fetch_cols = [&](const Item& x, int buf) {
+      float* ac = acol_s + buf * kMaxL;
+      float* nn = n_s + buf * DK;
+      for (int j = rt; j < x.n_kv * kKT; j += 256)
+        ac[j] = g.acol[(long)x.bh * tpad + x.c0 + j] * 1.4426950408889634f;
+      for (int j = rt; j < DK; j += 256) nn[j] = n_states[((long)x.bh * p.NC + x.k) * DK + j];
+    };
+    float nx_m_in = 0.f, nx_amax = 0.f, nx_bc = 0.f;
+    if (blockIdx.x < n_items) {
+      const Item x0 = decode_item(blockIdx.x, p, n_dv, n_q);
+      fetch_rows(x0, nx_m_in, nx_amax, nx_bc);
+      fetch_cols(x0, 0);
+    }
+    for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++n) {
+      const Item x = decode_item(it, p, n_dv, n_q);
+      const int t = x.t0 + r;
+      const float m_in = nx_m_in, amax = nx_amax, bc = nx_bc;
+      const float* ac = acol_s + (n & 1) * kMaxL;
+      const uint32_t colO = (uint32_t)(n % C::kOBufs) * 128u;
+      const float* nn = n_s + (n & 1) * DK;
+      const float mu = fmaxf(m_in, amax);
+      const float mu2 = mu * 1.4426950408889634f;
+      const float f_inter = expf(m_in - mu);
+      named_bar_sync(1, 256);  // this item's column data is in shared memory
+
+      // Partial den_inter = q_r . n_k over this half's slabs; then release Q.
+      ok = mbar_wait(bar.q_full(), n & 1, p, 8);
+      float dn = 0.f;
+      for (int c = h * kSlabsPerHalf; c < C::kSlabsK && c < (h + 1) * kSlabsPerHalf && ok; ++c) {
+        const uint8_t* slab_ptr = smem + C::kOffQ + c * 16384;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const uint4 v = *reinterpret_cast<const uint4*>(slab_ptr + sw128_offset(r, j));
-        const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&v);
+        for (int j = 0; j < 8; ++j) {
+          const uint4 v = *reinterpret_cast<const uint4*>(slab_ptr + sw128_offset(r, j));
+          const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&v);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 f2 = __bfloat1622float2(h2[e]);
-          dn = fmaf(f2.x, n_s[c * 64 + j * 8 + 2 * e], dn);
-          dn = fmaf(f2.y, n_s[c * 64 + j * 8 + 2 * e + 1], dn);
+          for (int e = 0; e < 4; ++e) {
+            const float2 f2 = __bfloat1622float2(h2[e]);
+            dn = fmaf(f2.x, nn[c * 64 + j * 8 + 2 * e], dn);
+            dn = fmaf(f2.y, nn[c * 64 + j * 8 + 2 * e + 1], dn);
+          }
         }
       }
-    }
-    float den = f_inter * dn;
+      mbar_arrive(bar.q_empty());
+      float den = f_inter * dn;
 
-    // Rescale the inter-chunk term of the accumulator to the row frame mu_r.
-    ok = ok && mbar_wait(bar.inter_done, 0, p);
-    tc_fence_after();
-    if (ok) {
-      for (int c = 0; c < DVT; c += 32) {
-        uint32_t v[32];
-        tmem_ld32(trow + kColO + c, v);
-        tmem_wait_ld();
-#pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * f_inter);
-        tmem_st32(trow + kColO + c, v);
-      }
-      tmem_wait_st();
-    }
-
-    for (int i = 0; i < n_kv; ++i) {
-      const int buf = i & 1;
-      ok = ok && mbar_wait(bar.s_full[buf], (i >> 1) & 1, p);
-      if (i >= 1) ok = ok && mbar_wait(bar.p_empty, (i - 1) & 1, p);
+      // Rescale this half of the inter-chunk term to the row frame mu_r.
+      ok = ok && mbar_wait(bar.inter_done(), n & 1, p, 9);
       tc_fence_after();
-      const bool diag = (i == n_kv - 1);
-      const uint32_t scol = buf ? kColS1 : kColS0;
-      float rs = 0.f;
       if (ok) {
-#pragma unroll 1
-        for (int c = 0; c < kKT; c += 32) {
-          uint32_t v[32];
-          tmem_ld32(trow + scol + c, v);
+        for (int c = h * kHalfO; c < (h + 1) * kHalfO; c += 64) {
+          uint32_t v0[32], v1[32];
+          tmem_ld32(trow + colO + c, v0);
+          if (kHalfO >= 64) tmem_ld32(trow + colO + c + 32, v1);
           tmem_wait_ld();
-          uint32_t pk[16];
 #pragma unroll
-          for (int j = 0; j < 32; j += 2) {
-            const int s0 = c + j;
-            float pa = __uint_as_float(v[j]) * ks * ex2_approx(acol_s[i * kKT + s0] - mu2);
-            float pb = __uint_as_float(v[j + 1]) * ks * ex2_approx(acol_s[i * kKT + s0 + 1] - mu2);
+          for (int j = 0; j < 32; ++j) v0[j] = __float_as_uint(__uint_as_float(v0[j]) * f_inter);
+          tmem_st32(trow + colO + c, v0);
+          if (kHalfO >= 64) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v1[j] = __float_as_uint(__uint_as_float(v1[j]) * f_inter);
+            tmem_st32(trow + colO + c + 32, v1);
+          }
+        }
+        tmem_wait_st();
+      }
+
+      for (int i = 0; i < x.n_kv; ++i, ++tile) {
+        const int buf = tile & 1;
+        ok = ok && mbar_wait(bar.s_full(buf), (tile >> 1) & 1, p, 10);
+        if (tile >= 1) ok = ok && mbar_wait(bar.p_empty(), (tile - 1) & 1, p, 11);
+        tc_fence_after();
+        const bool diag = (i == x.n_kv - 1);
+        const uint32_t scol = (buf ? kColS1 : kColS0) + h * 64;
+        float rs = 0.f;
+        if (ok) {
+          uint32_t v[64];
+          tmem_ld32(trow + scol, *reinterpret_cast<uint32_t(*)[32]>(v));
+          tmem_ld32(trow + scol + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+          tmem_wait_ld();
+          uint32_t pk[32];
+          const float* acl = ac + i * kKT + h * 64;
+#pragma unroll
+          for (int j = 0; j < 64; j += 2) {
+            const int s0 = h * 64 + j;  // key/value index within the tile
+            float pa = __uint_as_float(v[j]) * ks * ex2_approx(acl[j] - mu2);
+            float pb = __uint_as_float(v[j + 1]) * ks * ex2_approx(acl[j + 1] - mu2);
             if (diag && s0 > r) pa = 0.f;
             if (diag && s0 + 1 > r) pb = 0.f;
             rs += pa + pb;
             pk[j >> 1] = pack_bf16x2(pa, pb);
           }
-          // 32 columns = 64 bytes = 4 chunks of the swizzled 128-byte row.
-          uint8_t* prow = smem + C::kOffP + (c >> 6) * 16384;
-          const int cb = (c & 63) >> 3;  // first 16-byte chunk within the row
+          // This half's 64 columns are exactly atom column h of the P tile.
+          uint8_t* prow = smem + C::kOffP + h * 16384;
 #pragma unroll
-          for (int j = 0; j < 4; ++j)
-            *reinterpret_cast<uint4*>(prow + sw128_offset(r, cb + j)) =
+          for (int j = 0; j < 8; ++j)
+            *reinterpret_cast<uint4*>(prow + sw128_offset(r, j)) =
                 make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
         }
+        den += rs;
+        tc_fence_before();
+        mbar_arrive(bar.s_empty(buf));
+        fence_proxy_async_smem();
+        mbar_arrive(bar.p_full());
       }
-      den += rs;
-      tc_fence_before();
-      mbar_arrive(bar.s_empty[buf]);
-      fence_proxy_async_smem();
-      mbar_arrive(bar.p_full);
-    }
 
-    // Epilogue: h = O / max(|den|, e^{-m_r}).
-    ok = ok && mbar_wait(bar.o_done, 0, p);
-    tc_fence_after();
-    const float mr = bc + mu;
-    const float denom = fmaxf(fabsf(den), expf(-mr));
-    const float inv = 1.f / denom;
-    if (ok) {
-      for (int c = 0; c < DVT; c += 32) {
-        uint32_t v[32];
-        tmem_ld32(trow + kColO + c, v);
-        tmem_wait_ld();
-        if (t < p.T) {
-          uint32_t pk[16];
+      // Fetch the next item's row values and column data while P.V finishes.
+      const int it_next = it + gridDim.x;
+      if (it_next < n_items) {
+        const Item xn = decode_item(it_next, p, n_dv, n_q);
+        fetch_rows(xn, nx_m_in, nx_amax, nx_bc);
+        fetch_cols(xn, (n + 1) & 1);
+      }
+
+      // Epilogue: combine the two halves' denominators, h = O / max(|den|, e^{-m_r}).
+      red_s[rt] = den;
+      named_bar_sync(1, 256);
+      den += red_s[rt ^ 128];
+      ok = ok && mbar_wait(bar.o_done(), n & 1, p, 12);
+      tc_fence_after();
+      const float mr = bc + mu;
+      const float denom = fmaxf(fabsf(den), expf(-mr));
+      const float inv = 1.f / denom;
+      if (ok) {
+        for (int c = h * kHalfO; c < (h + 1) * kHalfO; c += 64) {
+          uint32_t v0[32], v1[32];
+          tmem_ld32(trow + colO + c, v0);
+          if (kHalfO >= 64) tmem_ld32(trow + colO + c + 32, v1);
+          tmem_wait_ld();
+          if (t < p.T) {
+            uint32_t pk[16];
 #pragma unroll
-          for (int j = 0; j < 32; j += 2)
-            pk[j >> 1] = pack_bf16x2(__uint_as_float(v[j]) * inv, __uint_as_float(v[j + 1]) * inv);
-          uint4* dst = reinterpret_cast<uint4*>(H + ((long)bh * p.T + t) * p.DV + dv0 + c);
+            for (int j = 0; j < 32; j += 2)
+              pk[j >> 1] =
+                  pack_bf16x2(__uint_as_float(v0[j]) * inv, __uint_as_float(v0[j + 1]) * inv);
+            uint4* dst = reinterpret_cast<uint4*>(H + ((long)x.bh * p.T + t) * p.DV + x.dv0 + c);
 #pragma unroll
-          for (int j = 0; j < 4; ++j)
-            dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+            for (int j = 0; j < 4; ++j)
+              dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+            if (kHalfO >= 64) {
+#pragma unroll
+              for (int j = 0; j < 32; j += 2)
+                pk[j >> 1] =
+                    pack_bf16x2(__uint_as_float(v1[j]) * inv, __uint_as_float(v1[j + 1]) * inv);
+#pragma unroll
+              for (int j = 0; j < 4; ++j)
+                dst[4 + j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+            }
+          }
         }
       }
-    }
-    if (t < p.T && blockIdx.x == 0) {
-      if (n_out) n_out[(long)bh * p.T + t] = denom;
-      if (m_out) m_out[(long)bh * p.T + t] = mr;
+      tc_fence_before();
+      mbar_arrive(bar.o_empty(n % C::kOBufs));
+      if (t < p.T && x.dv0 == 0 && h == 0) {
+        if (n_out) n_out[(long)x.bh * p.T + t] = denom;
+        if (m_out) m_out[(long)x.bh * p.T + t] = mr;
+      }
     }
   }
 
@@ -399,9 +526,16 @@ cudaError_t launch_parallel_t(const Problem& p, const void* Q, const void* K, co
   auto kern = tc_parallel_kernel<DK, DVT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   if (e != cudaSuccess) return e;
-  dim3 grid(p.DV / DVT, (p.T + kQT - 1) / kQT, p.BH);
+  int dev = 0, sms = 0;
+  e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  const long items = (long)p.BH * ((p.T + kQT - 1) / kQT) * (p.DV / DVT);
+  if (items > (1L << 30)) return cudaErrorInvalidValue;
+  const int grid = (int)(items < sms ? items : sms);
   kern<<<grid, kThreads, C::kSmem, st>>>(tq, tk, tv, tcm, p, g, n_states,
-                                         static_cast<__nv_bfloat16*>(H), n_out, m_out);
+                                         static_cast<__nv_bfloat16*>(H), n_out, m_out, (int)items);
   return cudaGetLastError();
 }
 
@@ -417,7 +551,7 @@ cudaError_t launch_tc_parallel_bf16states(const Problem& p, const void* Q, const
                                           const void* V, Gates g, const __nv_bfloat16* Cb,
                                           const float* n_states, void* H, float* n_out,
                                           float* m_out, cudaStream_t st) {
-  const int dvt = p.DV >= 256 ? 256 : p.DV;
+  const int dvt = p.DV % 256 == 0 ? 256 : (p.DV >= 128 ? 128 : p.DV);
 #define MLSTM_PAR_CASE(dk, dvt_)                                                                \
   if (p.DK == dk && dvt == dvt_)                                                                \
     return launch_parallel_t<dk, dvt_>(p, Q, K, V, g, Cb, n_states, H, n_out, m_out, st);

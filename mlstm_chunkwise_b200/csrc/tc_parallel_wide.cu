@@ -1,0 +1,549 @@
+// G3 for chunks of at most 256 tokens: one work item per (b, h) and 128-row
+// query tile, covering every value column of the head.
+//
+// Same per-row mathematics as tc_parallel.cu ("Tiled Flash Linear Attention:
+// More Efficient Linear RNN and xLSTM Kernels", abstract: the intra-chunk part
+// tiled over query and key/value blocks):
+//
+//   O_r   = e^{m_k - mu_r} C_k^T q_r  +  sum_{s<=r} P_rs v_s
+//   P_rs  = (s q_r.k_s) e^{acol_s - mu_r}                (0 above the diagonal)
+//   den_r = e^{m_k - mu_r} n_k.q_r    +  sum_{s<=r} P_rs
+//   h_r   = O_r / max(|den_r|, e^{-(bcum_r + mu_r)})
+//
+// What differs is the work decomposition.  With at most two 128-token
+// key/value tiles per query tile, the gated P tiles of an item fit in shared
+// memory, so an item computes S and P once and then sweeps the value columns
+// in 128-wide tiles d: O_d = Q~ C_k[:, d] + sum_i P_i V_i[:, d], where Q~ is
+// the query tile with row r scaled by e^{m_k - mu_r} (in place, once the S
+// MMAs have read Q).  The Q tile is loaded once per item, S is never
+// recomputed per value tile, and the MMAs of consecutive value tiles need no
+// hand-off from the row threads.  The two TMEM output accumulators alternate
+// between value tiles; the epilogue of tile d (bf16 rows into a swizzled
+// staging tile, then a TMA store) overlaps the MMAs of tile d + 1.
+//
+// Roles (320 threads): warp 0 TMA producer; warp 1 TMEM owner and MMA issuer;
+// warps 2..9 two threads per query row (each owning half of the columns):
+// gating of S into P, the in-place scaling of Q, row sums, epilogue.
+// TMEM (512 columns): O at 0 and 128, S at 256 and 384.
+// MMA order per item: S_0 [, S_1], (wait for the scaled Q), then for every
+// value tile d: Q~.C_k[:, d], P_0.V_0[:, d] [, P_1.V_1[:, d]].
+#include <cuda.h>
+
+#include "tc.h"
+#include "tc_ptx.cuh"
+
+namespace mlstm {
+namespace {
+
+using namespace tc;
+
+constexpr int kThreads = 320;
+constexpr int kQT = 128;
+constexpr int kKT = 128;
+constexpr int kPSlots = 2;  // key/value tiles per item (chunks of at most 256)
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColS0 = 256, kColS1 = 384;
+
+template <int DK, int DVT>
+struct WCfg {
+  static_assert(DVT == 64 || DVT == 128, "value tile of 64 or 128 columns");
+  static constexpr int kSlabsK = DK / 64;
+  static constexpr uint32_t kQBytes = kQT * DK * 2;
+  static constexpr uint32_t kKSlabBytes = kKT * 128;
+  static constexpr uint32_t kMNSlabBytes = (DVT / 64) * 8192;
+  static constexpr uint32_t kStageBytes = 16384;
+  static_assert(kKSlabBytes <= kStageBytes && kMNSlabBytes <= kStageBytes, "stage size");
+  static constexpr uint32_t kPBytes = kQT * kKT * 2;  // one slot
+  static constexpr uint32_t kOutBytes = kQT * DVT * 2;  // output staging tile
+  static constexpr uint32_t kMiscBytes = 2 * kPSlots * kKT * 4 + 2 * DK * 4 + 256 * 4 + 512;
+  static constexpr uint32_t kBudget = 227 * 1024 - 1024;
+  static constexpr int kStagesFit =
+      (int)((kBudget - kQBytes - kPSlots * kPBytes - kOutBytes - kMiscBytes) / kStageBytes);
+  static constexpr int kStages = kStagesFit > 12 ? 12 : kStagesFit;
+  static_assert(kStages >= 3, "ring too shallow");
+  static constexpr uint32_t kOffQ = 0;
+  static constexpr uint32_t kOffP = kOffQ + kQBytes;
+  static constexpr uint32_t kOffOut = kOffP + kPSlots * kPBytes;
+  static constexpr uint32_t kOffStage = kOffOut + kOutBytes;
+  static constexpr uint32_t kOffAcol = kOffStage + kStages * kStageBytes;  // float[2][256]
+  static constexpr uint32_t kOffN = kOffAcol + 2 * kPSlots * kKT * 4;       // float[2][DK]
+  static constexpr uint32_t kOffRed = kOffN + 2 * DK * 4;                   // float[256]
+  static constexpr uint32_t kOffBar = kOffRed + 256 * 4;
+  static constexpr uint32_t kOffTmemSlot = kOffBar + 384;
+  static constexpr uint32_t kBytes = kOffTmemSlot + 16;
+  static constexpr uint32_t kSmem = kBytes + 1024;
+  static_assert(kSmem <= 227 * 1024, "shared memory");
+};
+
+struct WBars {
+  uint32_t a;
+  __device__ __forceinline__ uint32_t full(int i) const { return a + 8 * i; }
+  __device__ __forceinline__ uint32_t empty(int i) const { return a + 128 + 8 * i; }
+  __device__ __forceinline__ uint32_t q_full() const { return a + 256; }
+  __device__ __forceinline__ uint32_t q_empty() const { return a + 264; }
+  __device__ __forceinline__ uint32_t s_full(int b) const { return a + 272 + 8 * b; }
+  __device__ __forceinline__ uint32_t s_empty(int b) const { return a + 288 + 8 * b; }
+  __device__ __forceinline__ uint32_t p_full(int i) const { return a + 304 + 8 * i; }
+  __device__ __forceinline__ uint32_t p_empty(int i) const { return a + 320 + 8 * i; }
+  __device__ __forceinline__ uint32_t q_scaled() const { return a + 336; }
+  __device__ __forceinline__ uint32_t o_done() const { return a + 352; }
+  __device__ __forceinline__ uint32_t o_empty(int b) const { return a + 360 + 8 * b; }
+  __device__ __forceinline__ uint32_t mma_idle() const { return a + 376; }
+};
+
+struct WItem {
+  int bh, t0, k, c0, n_kv;
+};
+
+__device__ __forceinline__ WItem decode_witem(int it, const Problem& p, int n_q) {
+  WItem x;
+  x.bh = it / n_q;
+  x.t0 = (it % n_q) * kQT;
+  x.k = x.t0 / p.L;
+  x.c0 = x.k * p.L;
+  x.n_kv = (x.t0 - x.c0) / kKT + 1;
+  return x;
+}
+
+template <int DK, int DVT>
+__global__ void __launch_bounds__(kThreads, 1)
+tc_parallel_wide_kernel(const __grid_constant__ CUtensorMap tm_q,
+                        const __grid_constant__ CUtensorMap tm_k,
+                        const __grid_constant__ CUtensorMap tm_v,
+                        const __grid_constant__ CUtensorMap tm_c,
+                        const __grid_constant__ CUtensorMap tm_h, Problem p, Gates g,
+                        const float* __restrict__ n_states,
+                        float* __restrict__ n_out, float* __restrict__ m_out, int n_items) {
+  using C = WCfg<DK, DVT>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const WBars bar{sbase + C::kOffBar};
+  float* acol_s = reinterpret_cast<float*>(smem + C::kOffAcol);
+  float* n_s = reinterpret_cast<float*>(smem + C::kOffN);
+  float* red_s = reinterpret_cast<float*>(smem + C::kOffRed);
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + C::kOffTmemSlot);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_dv = p.DV / DVT;
+  const int n_q = (p.T + kQT - 1) / kQT;
+  const long tpad = (long)p.NC * p.L;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::kStages; ++i) {
+      mbar_init(bar.full(i), 1);
+      mbar_init(bar.empty(i), 1);
+    }
+    mbar_init(bar.q_full(), 1);
+    mbar_init(bar.q_empty(), 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar.s_full(i), 1);
+      mbar_init(bar.s_empty(i), 256);
+      mbar_init(bar.p_full(i), 256);
+      mbar_init(bar.p_empty(i), 1);
+      mbar_init(bar.o_empty(i), 256);
+    }
+    mbar_init(bar.q_scaled(), 256);
+    mbar_init(bar.o_done(), 1);
+    mbar_init(bar.mma_idle(), 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32((const void*)tmem_slot), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ---------------------------- TMA producer ----------------------------
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      tma_prefetch_desc(&tm_c);
+      int slab = 0;
+      bool ok = true;
+      auto next_stage = [&](uint32_t bytes) -> uint32_t {
+        const int s = slab % C::kStages, u = slab / C::kStages;
+        if (u > 0) ok = ok && mbar_wait(bar.empty(s), (u - 1) & 1, p, 1);
+        mbar_expect_tx(bar.full(s), bytes);
+        ++slab;
+        return sbase + C::kOffStage + (uint32_t)s * C::kStageBytes;
+      };
+      int n = 0;
+      for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++n) {
+        const WItem x = decode_witem(it, p, n_q);
+        if (n > 0) ok = mbar_wait(bar.q_empty(), (n - 1) & 1, p, 2);
+        if (!ok) break;
+        mbar_expect_tx(bar.q_full(), C::kQBytes);
+        for (int c = 0; c < C::kSlabsK; ++c)
+          tma_load_3d(sbase + C::kOffQ + c * 16384, &tm_q, c * 64, x.t0, x.bh, bar.q_full());
+        for (int i = 0; i < x.n_kv && ok; ++i)
+          for (int c = 0; c < C::kSlabsK && ok; ++c) {
+            const uint32_t dst = next_stage(C::kKSlabBytes);
+            tma_load_3d(dst, &tm_k, c * 64, x.c0 + i * kKT, x.bh,
+                        bar.full((slab - 1) % C::kStages));
+          }
+        for (int d = 0; d < n_dv && ok; ++d) {
+          const int dv0 = d * DVT;
+          for (int c = 0; c < C::kSlabsK && ok; ++c) {
+            const uint32_t dst = next_stage(C::kMNSlabBytes);
+            for (int b = 0; b < DVT / 64; ++b)
+              tma_load_3d(dst + b * 8192, &tm_c, dv0 + b * 64, c * 64, x.bh * p.NC + x.k,
+                          bar.full((slab - 1) % C::kStages));
+          }
+          for (int i = 0; i < x.n_kv && ok; ++i)
+            for (int v = 0; v < 2 && ok; ++v) {
+              const uint32_t dst = next_stage(C::kMNSlabBytes);
+              for (int b = 0; b < DVT / 64; ++b)
+                tma_load_3d(dst + b * 8192, &tm_v, dv0 + b * 64, x.c0 + i * kKT + v * 64, x.bh,
+                            bar.full((slab - 1) % C::kStages));
+            }
+        }
+      }
+      for (int q = (slab > C::kStages ? slab - C::kStages : 0); q < slab; ++q)
+        mbar_wait(bar.full(q % C::kStages), (q / C::kStages) & 1, p, 13);
+      if (n > 0) mbar_wait(bar.q_full(), (n - 1) & 1, p, 14);
+    }
+  } else if (warp == 1) {
+    // ---------------------------- MMA issuer ------------------------------
+    if (lane == 0) {
+      constexpr uint32_t idS = idesc_bf16(128, kKT, 0, 0);
+      constexpr uint32_t idO = idesc_bf16(128, DVT, 0, 1);
+      bool ok = true;
+      int slab = 0, tile = 0, dcount = 0;
+      int pc0 = 0, pc1 = 0;  // times P slot 0 / 1 has been filled (no arrays: registers)
+      auto take = [&]() -> uint32_t {
+        const int s = slab % C::kStages, u = slab / C::kStages;
+        ok = ok && mbar_wait(bar.full(s), u & 1, p, 5);
+        tc_fence_after();
+        ++slab;
+        return (uint32_t)s;
+      };
+      int n = 0;
+      for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++n) {
+        const WItem x = decode_witem(it, p, n_q);
+        ok = mbar_wait(bar.q_full(), n & 1, p, 3);
+        for (int i = 0; i < x.n_kv && ok; ++i, ++tile) {  // S_i
+          const int buf = tile & 1;
+          if (tile >= 2) ok = ok && mbar_wait(bar.s_empty(buf), ((tile >> 1) - 1) & 1, p, 4);
+          tc_fence_after();
+          const uint32_t dS = tmem + (buf ? kColS1 : kColS0);
+          for (int c = 0; c < C::kSlabsK && ok; ++c) {
+            const uint32_t s = take();
+            if (!ok) break;
+            const uint32_t a0 = sbase + C::kOffQ + c * 16384;
+            const uint32_t b0 = sbase + C::kOffStage + s * C::kStageBytes;
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              mma_bf16_ss(dS, sdesc_sw128(a0 + kk * 32, 16, 1024),
+                          sdesc_sw128(b0 + kk * 32, 16, 1024), idS, (c | kk) != 0);
+            mma_commit(bar.empty(s));
+          }
+          mma_commit(bar.s_full(buf));
+        }
+        ok = ok && mbar_wait(bar.q_scaled(), n & 1, p, 7);  // Q rows scaled in place
+        tc_fence_after();
+        for (int d = 0; d < n_dv && ok; ++d, ++dcount) {
+          const int ob = dcount & 1;
+          const uint32_t dO = tmem + (uint32_t)ob * 128u;
+          if (dcount >= 2) ok = ok && mbar_wait(bar.o_empty(ob), ((dcount >> 1) - 1) & 1, p, 6);
+          tc_fence_after();
+          for (int c = 0; c < C::kSlabsK && ok; ++c) {  // Q . C_k[:, d]
+            const uint32_t s = take();
+            if (!ok) break;
+            const uint32_t a0 = sbase + C::kOffQ + c * 16384;
+            const uint32_t b0 = sbase + C::kOffStage + s * C::kStageBytes;
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              mma_bf16_ss(dO, sdesc_sw128(a0 + kk * 32, 16, 1024),
+                          sdesc_sw128(b0 + kk * 2048, 8192, 1024), idO, (c | kk) != 0);
+            mma_commit(bar.empty(s));
+          }
+          if (!ok) break;
+          if (d == n_dv - 1) mma_commit(bar.q_empty());  // last reader of Q issued
+          for (int i = 0; i < x.n_kv && ok; ++i) {
+            if (d == 0) ok = mbar_wait(bar.p_full(i), (i ? pc1 : pc0) & 1, p, 8);
+            tc_fence_after();
+            for (int v = 0; v < 2 && ok; ++v) {
+              const uint32_t s = take();
+              if (!ok) break;
+              const uint32_t a0 = sbase + C::kOffP + i * C::kPBytes + v * 16384;
+              const uint32_t b0 = sbase + C::kOffStage + s * C::kStageBytes;
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk)
+                mma_bf16_ss(dO, sdesc_sw128(a0 + kk * 32, 16, 1024),
+                            sdesc_sw128(b0 + kk * 2048, 8192, 1024), idO, 1);
+              mma_commit(bar.empty(s));
+            }
+            if (d == n_dv - 1) {
+              mma_commit(bar.p_empty(i));
+              if (i) ++pc1; else ++pc0;
+            }
+          }
+          if (!ok) break;
+          mma_commit(bar.o_done());
+        }
+      }
+      mma_commit(bar.mma_idle());
+      mbar_wait(bar.mma_idle(), 0, p, 15);
+    }
+  } else {
+    // ------------------- gating / softmax / epilogue ----------------------
+    const int q = warp & 3;
+    const int r = q * 32 + lane;
+    const int rt = threadIdx.x - 64;
+    const int h = rt >> 7;
+    const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16);
+    const float ks = p.key_scale;
+    constexpr int kHalfO = DVT / 2;
+    constexpr int kSlabsPerHalf = (C::kSlabsK + 1) / 2;
+    bool ok = true;
+    int tile = 0, dcount = 0;
+    int pc0 = 0, pc1 = 0;
+    auto fetch_rows = [&](const WItem& x, float& m_in, float& amax, float& bc) {
+      const int t = x.t0 + r;
+      m_in = g.mchk[(long)x.bh * (p.NC + 1) + x.k];
+      amax = g.amax[(long)x.bh * tpad + t];
+      bc = g.bcum[(long)x.bh * tpad + t];
+    };
+    auto fetch_cols = [&](const WItem& x, int buf) {
+      float* ac = acol_s + buf * kPSlots * kKT;
+      float* nn = n_s + buf * DK;
+      for (int j = rt; j < x.n_kv * kKT; j += 256)
+        ac[j] = g.acol[(long)x.bh * tpad + x.c0 + j] * 1.4426950408889634f;
+      for (int j = rt; j < DK; j += 256) nn[j] = n_states[((long)x.bh * p.NC + x.k) * DK + j];
+    };
+    float nx_m_in = 0.f, nx_amax = 0.f, nx_bc = 0.f;
+    if (blockIdx.x < n_items) {
+      const WItem x0 = decode_witem(blockIdx.x, p, n_q);
+      fetch_rows(x0, nx_m_in, nx_amax, nx_bc);
+      fetch_cols(x0, 0);
+    }
+    int n = 0;
+    for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++n) {
+      const WItem x = decode_witem(it, p, n_q);
+      const int t = x.t0 + r;
+      const float m_in = nx_m_in, amax = nx_amax, bc = nx_bc;
+      const float* ac = acol_s + (n & 1) * kPSlots * kKT;
+      const float* nn = n_s + (n & 1) * DK;
+      const float mu = fmaxf(m_in, amax);
+      const float mu2 = mu * 1.4426950408889634f;
+      const float f_inter = expf(m_in - mu);
+      named_bar_sync(1, 256);
+
+      // Partial den_inter = q_r . n_k over this half's slabs; then release Q.
+      ok = mbar_wait(bar.q_full(), n & 1, p, 9);
+      float dn = 0.f;
+      for (int c = h * kSlabsPerHalf; c < C::kSlabsK && c < (h + 1) * kSlabsPerHalf && ok; ++c) {
+        const uint8_t* slab_ptr = smem + C::kOffQ + c * 16384;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const uint4 v = *reinterpret_cast<const uint4*>(slab_ptr + sw128_offset(r, j));
+          const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f2 = __bfloat1622float2(h2[e]);
+            dn = fmaf(f2.x, nn[c * 64 + j * 8 + 2 * e], dn);
+            dn = fmaf(f2.y, nn[c * 64 + j * 8 + 2 * e + 1], dn);
+          }
+        }
+      }
+      float den = f_inter * dn;
+
+      // Gated P tiles, once per item.
+      for (int i = 0; i < x.n_kv; ++i, ++tile) {
+        const int buf = tile & 1;
+        ok = ok && mbar_wait(bar.s_full(buf), (tile >> 1) & 1, p, 10);
+        const int pc = i ? pc1 : pc0;
+        if (pc >= 1) ok = ok && mbar_wait(bar.p_empty(i), (pc - 1) & 1, p, 11);
+        tc_fence_after();
+        const bool diag = (i == x.n_kv - 1);
+        const uint32_t scol = (buf ? kColS1 : kColS0) + h * 64;
+        float rs = 0.f;
+        if (ok) {
+          uint32_t v[64];
+          tmem_ld32(trow + scol, *reinterpret_cast<uint32_t(*)[32]>(v));
+          tmem_ld32(trow + scol + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+          tmem_wait_ld();
+          uint32_t pk[32];
+          const float* acl = ac + i * kKT + h * 64;
+#pragma unroll
+          for (int j = 0; j < 64; j += 2) {
+            const int s0 = h * 64 + j;
+            float pa = __uint_as_float(v[j]) * ks * ex2_approx(acl[j] - mu2);
+            float pb = __uint_as_float(v[j + 1]) * ks * ex2_approx(acl[j + 1] - mu2);
+            if (diag && s0 > r) pa = 0.f;
+            if (diag && s0 + 1 > r) pb = 0.f;
+            rs += pa + pb;
+            pk[j >> 1] = pack_bf16x2(pa, pb);
+          }
+          uint8_t* prow = smem + C::kOffP + i * C::kPBytes + h * 16384;
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            *reinterpret_cast<uint4*>(prow + sw128_offset(r, j)) =
+                make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+        }
+        den += rs;
+        tc_fence_before();
+        mbar_arrive(bar.s_empty(buf));
+        fence_proxy_async_smem();
+        mbar_arrive(bar.p_full(i));
+        if (i) ++pc1; else ++pc0;
+      }
+
+      // Every S MMA of this item has completed (the waits above): scale this
+      // half of the Q row by e^{m_k - mu_r} in place for the inter-chunk MMAs.
+      if (ok) {
+        for (int c = h * kSlabsPerHalf; c < C::kSlabsK && c < (h + 1) * kSlabsPerHalf; ++c) {
+          uint8_t* slab_ptr = smem + C::kOffQ + c * 16384;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            uint4* ptr = reinterpret_cast<uint4*>(slab_ptr + sw128_offset(r, j));
+            uint4 u = *ptr;
+            __nv_bfloat162* h2 = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 f2 = __bfloat1622float2(h2[e]);
+              h2[e] = __floats2bfloat162_rn(f2.x * f_inter, f2.y * f_inter);
+            }
+            *ptr = u;
+          }
+        }
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(bar.q_scaled());
+
+      // The next item's row values and column data (other buffer).
+      const int it_next = it + gridDim.x;
+      if (it_next < n_items) {
+        const WItem xn = decode_witem(it_next, p, n_q);
+        fetch_rows(xn, nx_m_in, nx_amax, nx_bc);
+        fetch_cols(xn, (n + 1) & 1);
+      }
+
+      // Both halves' partial denominators -> the row's denominator.
+      red_s[rt] = den;
+      named_bar_sync(1, 256);
+      den += red_s[rt ^ 128];
+      const float mr = bc + mu;
+      const float denom = fmaxf(fabsf(den), expf(-mr));
+      const float inv = 1.f / denom;
+      if (t < p.T && h == 0) {
+        if (n_out) n_out[(long)x.bh * p.T + t] = denom;
+        if (m_out) m_out[(long)x.bh * p.T + t] = mr;
+      }
+
+      for (int d = 0; d < n_dv; ++d, ++dcount) {
+        const uint32_t colO = (uint32_t)(dcount & 1) * 128u + h * kHalfO;
+        ok = ok && mbar_wait(bar.o_done(), dcount & 1, p, 14);
+        tc_fence_after();
+        if (rt == 0) tma_store_wait_read_all();  // the staging tile is free again
+        named_bar_sync(1, 256);
+        if (ok) {
+          uint32_t v0[32], v1[32];
+          tmem_ld32(trow + colO, v0);
+          if (kHalfO >= 64) tmem_ld32(trow + colO + 32, v1);
+          tmem_wait_ld();
+          // this half's columns: box (h * kHalfO) / 64, 16-byte chunks from cb
+          uint8_t* box = smem + C::kOffOut + ((h * kHalfO) >> 6) * 16384;
+          const int cb = ((h * kHalfO) & 63) >> 3;
+          uint32_t pk[16];
+#pragma unroll
+          for (int j = 0; j < 32; j += 2)
+            pk[j >> 1] = pack_bf16x2(__uint_as_float(v0[j]) * inv, __uint_as_float(v0[j + 1]) * inv);
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            *reinterpret_cast<uint4*>(box + sw128_offset(r, cb + j)) =
+                make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+          if (kHalfO >= 64) {
+#pragma unroll
+            for (int j = 0; j < 32; j += 2)
+              pk[j >> 1] =
+                  pack_bf16x2(__uint_as_float(v1[j]) * inv, __uint_as_float(v1[j + 1]) * inv);
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              *reinterpret_cast<uint4*>(box + sw128_offset(r, cb + 4 + j)) =
+                  make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(bar.o_empty(dcount & 1));
+        fence_proxy_async_smem();
+        named_bar_sync(1, 256);
+        if (rt == 0 && ok) {
+          for (int b = 0; b < DVT / 64; ++b)
+            tma_store_3d(&tm_h, sbase + C::kOffOut + b * 16384, d * DVT + b * 64, x.t0, x.bh);
+          tma_store_commit();
+        }
+      }
+    }
+    if (rt == 0) tma_store_wait_all();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+template <int DK, int DVT>
+cudaError_t launch_wide_t(const Problem& p, const void* Q, const void* K, const void* V, Gates g,
+                          const __nv_bfloat16* Cb, const float* n_states, void* H, float* n_out,
+                          float* m_out, cudaStream_t st) {
+  using C = WCfg<DK, DVT>;
+  CUtensorMap tq, tk, tv, tcm, th;
+  if (!encode_tmap_bf16_3d(&tq, Q, p.DK, p.T, p.BH, 64, kQT) ||
+      !encode_tmap_bf16_3d(&tk, K, p.DK, p.T, p.BH, 64, kKT) ||
+      !encode_tmap_bf16_3d(&tv, V, p.DV, p.T, p.BH, 64, 64) ||
+      !encode_tmap_bf16_3d(&tcm, Cb, p.DV, p.DK, (uint64_t)p.BH * p.NC, 64, 64) ||
+      !encode_tmap_bf16_3d(&th, H, p.DV, p.T, p.BH, 64, kQT))
+    return cudaErrorInvalidValue;
+  auto kern = tc_parallel_wide_kernel<DK, DVT>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+  if (e != cudaSuccess) return e;
+  int dev = 0, sms = 0;
+  e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  const long items = (long)p.BH * ((p.T + kQT - 1) / kQT);
+  if (items > (1L << 30)) return cudaErrorInvalidValue;
+  const int grid = (int)(items < sms ? items : sms);
+  kern<<<grid, kThreads, C::kSmem, st>>>(tq, tk, tv, tcm, th, p, g, n_states, n_out, m_out,
+                                         (int)items);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool tc_parallel_wide_supported(const Problem& p) {
+  const bool dk_ok = p.DK == 64 || p.DK == 128 || p.DK == 256;
+  const bool dv_ok = p.DV == 64 || p.DV % 128 == 0;
+  return dk_ok && dv_ok && p.DV <= 1024 && p.L % kKT == 0 && p.L <= kPSlots * kKT && p.T > 0;
+}
+
+cudaError_t launch_tc_parallel_wide(const Problem& p, const void* Q, const void* K, const void* V,
+                                    Gates g, const __nv_bfloat16* Cb, const float* n_states,
+                                    void* H, float* n_out, float* m_out, cudaStream_t st) {
+  const int dvt = p.DV >= 128 ? 128 : 64;
+#define MLSTM_WIDE_CASE(dk, dvt_)                                                             \
+  if (p.DK == dk && dvt == dvt_)                                                              \
+    return launch_wide_t<dk, dvt_>(p, Q, K, V, g, Cb, n_states, H, n_out, m_out, st);
+  MLSTM_WIDE_CASE(64, 64)
+  MLSTM_WIDE_CASE(64, 128)
+  MLSTM_WIDE_CASE(128, 64)
+  MLSTM_WIDE_CASE(128, 128)
+  MLSTM_WIDE_CASE(256, 64)
+  MLSTM_WIDE_CASE(256, 128)
+#undef MLSTM_WIDE_CASE
+  return cudaErrorNotSupported;
+}
+
+}  // namespace mlstm

@@ -58,16 +58,19 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 }
 
 // Waits for the phase with the given parity to complete.  Gives up after
-// about max_polls * 16 ns (wall time on the global timer), sets the watchdog
-// bit in the error word and returns false.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const Problem& p) {
+// about max_polls * 16 ns (wall time on the global timer), records the
+// watchdog bit -- and, for the first wait that gives up, `site` in bits 8..15
+// of the error word -- and returns false.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const Problem& p,
+                                          uint32_t site = 0) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t limit = p.max_polls * 16ull;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (globaltimer_ns() - t0 > limit) {
-      raise_error(p.err, kErrWatchdog);
+      if (p.err && atomicCAS(p.err, 0u, kErrWatchdog | (site << 8)) != 0u)
+        atomicOr(p.err, kErrWatchdog);
       return false;
     }
   }
@@ -87,6 +90,28 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* m, 
       " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(m)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
       : "memory");
+}
+
+// TMA tile store from shared memory (bulk-group completion).  Rows or columns
+// past the tensor's extent are not written.
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* m, uint32_t src, int c0, int c1,
+                                             int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+          reinterpret_cast<uint64_t>(m)),
+      "r"(src), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+__device__ __forceinline__ void tma_store_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// Waits until every committed store has finished reading shared memory.
+__device__ __forceinline__ void tma_store_wait_read_all() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// Waits until every committed store has completed.
+__device__ __forceinline__ void tma_store_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
 // Makes generic-proxy writes to shared memory visible to the async proxy

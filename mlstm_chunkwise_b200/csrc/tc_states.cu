@@ -8,18 +8,20 @@
 //   C_{k+1} = e^{g_k + m_k - m_{k+1}} C_k + K_k^T diag(w) V_k,
 //   w_s     = s e^{g_k + acol_s - m_{k+1}},   n likewise with V -> 1,
 //
-// a dense rank-L update of the [DK, DV] state.  One CTA owns 128 rows of DK
-// (TMEM lanes) and DVT columns of DV of one (b, h); the fp32 master state
-// lives in TMEM for the whole sequence and the MMA accumulates each chunk's
-// update straight into it.  Before each chunk the row threads read the master
-// (the state entering the chunk), write it out (fp32 and/or bf16 operand
-// copy), and scale it by the decay.
+// a dense rank-L update of the [DK, DV] state.  One CTA owns the whole DK
+// extent (one or two 128-row halves, each a TMEM accumulator) and DVT columns
+// of DV of one (b, h), for the whole sequence; the fp32 master state lives in
+// TMEM and the MMA accumulates each chunk's update straight into it.  K and V
+// stream in 64-token stages through a ring deep enough to keep ~190 KB of
+// loads in flight.  Before each chunk the worker threads read the master (the
+// state entering the chunk), write it out (fp32 and/or bf16 operand copy) and
+// scale it by the decay.
 //
-// Roles (192 threads): warp 0 TMA producer (one 128-token K/V tile at a time),
-// warp 1 TMEM owner + MMA issuer, warps 2..5 one thread per state row: the
-// decay pass, the n-vector column sums (fp32, from the unrounded products
-// w_s k_s), the per-token weights (applied to the K tile in place, row by row)
-// and the stores.
+// Roles (320 threads): warp 0 TMA producer, warp 1 TMEM owner + MMA issuer,
+// warps 2..9 workers: per chunk, the token weights and the store and decay of
+// the master state; per stage, one pass that accumulates the n-vector partial
+// sums (fp32, from the unrounded products w_s k_s) and weights the K rows in
+// place.
 #include <cuda.h>
 
 #include "tc.h"
@@ -30,55 +32,81 @@ namespace {
 
 using namespace tc;
 
-constexpr int kThreads = 192;
-constexpr int kRows = 128;  // DK rows per CTA
-constexpr int kKT = 128;    // tokens per tile
+constexpr int kThreads = 320;
+constexpr int kWorkers = 256;
+constexpr int kStageTok = 64;  // tokens per ring stage
 
-template <int DVT>
+template <int DK, int DVT>
 struct SCfg {
-  static constexpr uint32_t kKBytes = kKT * kRows * 2;     // 2 boxes of [128 tokens x 64 dk]
-  static constexpr uint32_t kVBytes = kKT * DVT * 2;       // DVT/64 boxes of [128 x 64 dv]
-  static constexpr uint32_t kOffK = 0;
-  static constexpr uint32_t kOffV = kKBytes;
-  static constexpr uint32_t kOffW = kOffV + kVBytes;       // float[128] token weights
-  static constexpr uint32_t kOffBar = kOffW + kKT * 4;
-  static constexpr uint32_t kOffSlot = kOffBar + 8 * 8;
+  static_assert(DK == 128 || DK == 256, "DK of 128 or 256");
+  static_assert(DVT == 64 || DVT == 128 || DVT == 256, "value tile");
+  static constexpr int kHalves = DK / 128;
+  static constexpr uint32_t kKBytes = kStageTok * DK * 2;   // DK/64 boxes of [64 tok x 64 dk]
+  static constexpr uint32_t kVBytes = kStageTok * DVT * 2;  // DVT/64 boxes of [64 tok x 64 dv]
+  static constexpr uint32_t kStageBytes = kKBytes + kVBytes;
+  static constexpr int kMaxL = 1024;
+  static constexpr int kCC = DK / 8;             // 16-byte column chunks per token row
+  static constexpr int kRowsPer = kStageTok * kCC / 256;  // rows per worker per stage
+  static constexpr uint32_t kWBytes = kMaxL * 4;           // token weights of one chunk
+  static constexpr uint32_t kRedBytes = (256 / kCC) * DK * 4;  // n partials [row group][dk]
+  static constexpr uint32_t kBudget = 227 * 1024 - 1024 - 512 - kWBytes - kRedBytes;
+  static constexpr int kStagesFit = (int)(kBudget / kStageBytes);
+  static constexpr int kStages = kStagesFit > 8 ? 8 : kStagesFit;
+  static_assert(kStages >= 2, "ring too shallow");
+  static constexpr uint32_t kOffStage = 0;
+  static constexpr uint32_t kOffW = kStages * kStageBytes;  // float[kMaxL]
+  static constexpr uint32_t kOffRed = kOffW + kWBytes;      // float[256 / kCC][DK]
+  static constexpr uint32_t kOffBar = kOffRed + kRedBytes;
+  static constexpr uint32_t kOffSlot = kOffBar + 8 * 32;
   static constexpr uint32_t kBytes = kOffSlot + 16;
   static constexpr uint32_t kSmem = kBytes + 1024;
-  static constexpr uint32_t kTmemCols = DVT < 32 ? 32 : DVT;
+  static_assert(kSmem <= 227 * 1024, "shared memory");
+  static constexpr uint32_t kTmemCols = (kHalves * DVT) < 32 ? 32 : kHalves * DVT;
 };
 
-template <int DVT>
-__global__ void __launch_bounds__(kThreads)
+struct SBars {
+  uint32_t a;
+  __device__ __forceinline__ uint32_t full(int i) const { return a + 8 * i; }
+  __device__ __forceinline__ uint32_t empty(int i) const { return a + 64 + 8 * i; }
+  __device__ __forceinline__ uint32_t kready(int i) const { return a + 128 + 8 * i; }
+  __device__ __forceinline__ uint32_t master() const { return a + 192; }
+  __device__ __forceinline__ uint32_t chunk() const { return a + 200; }
+  __device__ __forceinline__ uint32_t done() const { return a + 208; }
+};
+
+template <int DK, int DVT>
+__global__ void __launch_bounds__(kThreads, 1)
 tc_states_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                  Problem p, Gates g, const float* __restrict__ C0, const float* __restrict__ n0,
                  float* __restrict__ C_states, __nv_bfloat16* __restrict__ Cb,
                  float* __restrict__ n_states, float* __restrict__ C_T, float* __restrict__ n_T,
                  float* __restrict__ m_T) {
-  using S = SCfg<DVT>;
+  using S = SCfg<DK, DVT>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
-  const uint32_t b_full = sbase + S::kOffBar, b_kready = b_full + 8, b_empty = b_full + 16,
-                 b_master = b_full + 24, b_chunk = b_full + 32, b_done = b_full + 40;
+  const SBars bar{sbase + S::kOffBar};
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + S::kOffSlot);
   float* w_s = reinterpret_cast<float*>(smem + S::kOffW);
+  float* red_s = reinterpret_cast<float*>(smem + S::kOffRed);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int dv0 = blockIdx.x * DVT, dk0 = blockIdx.y * kRows, bh = blockIdx.z;
-  const int L = p.L, NC = p.NC, T = p.T, DK = p.DK, DV = p.DV;
-  const int tiles = L / kKT;
+  const int dv0 = blockIdx.x * DVT, bh = blockIdx.y;
+  const int L = p.L, NC = p.NC, T = p.T, DV = p.DV;
+  const int stages_per_chunk = L / kStageTok;
   const long tpad = (long)NC * L;
   const bool n_owner = blockIdx.x == 0;
 
   if (threadIdx.x == 0) {
-    mbar_init(b_full, 1);
-    mbar_init(b_kready, 128);
-    mbar_init(b_empty, 1);
-    mbar_init(b_master, 128);
-    mbar_init(b_chunk, 1);
-    mbar_init(b_done, 1);
+    for (int i = 0; i < S::kStages; ++i) {
+      mbar_init(bar.full(i), 1);
+      mbar_init(bar.empty(i), 1);
+      mbar_init(bar.kready(i), kWorkers);
+    }
+    mbar_init(bar.master(), kWorkers);
+    mbar_init(bar.chunk(), 1);
+    mbar_init(bar.done(), 1);
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -91,194 +119,259 @@ tc_states_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
+    // ---------------------------- TMA producer ----------------------------
     if (lane == 0) {
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
       bool ok = true;
-      int n = 0;
-      for (int k = 0; k < NC && ok; ++k) {
-        for (int i = 0; i < tiles && ok; ++i, ++n) {
-          if (n > 0) ok = mbar_wait(b_empty, (n - 1) & 1, p);
-          if (!ok) break;
-          const int kv0 = k * L + i * kKT;
-          mbar_expect_tx(b_full, S::kKBytes + S::kVBytes);
-          for (int b = 0; b < 2; ++b)
-            tma_load_3d(sbase + S::kOffK + b * 16384, &tm_k, dk0 + b * 64, kv0, bh, b_full);
-          for (int b = 0; b < DVT / 64; ++b)
-            tma_load_3d(sbase + S::kOffV + b * 16384, &tm_v, dv0 + b * 64, kv0, bh, b_full);
-        }
+      const int total = NC * stages_per_chunk;
+      int issued = 0;
+      for (int n = 0; n < total && ok; ++n) {
+        const int s = n % S::kStages, u = n / S::kStages;
+        if (u > 0) ok = mbar_wait(bar.empty(s), (u - 1) & 1, p, 1);
+        if (!ok) break;
+        const int tok0 = n * kStageTok;  // chunks are whole stages: k * L + j * 64
+        const uint32_t st = sbase + S::kOffStage + (uint32_t)s * S::kStageBytes;
+        mbar_expect_tx(bar.full(s), S::kStageBytes);
+        for (int b = 0; b < DK / 64; ++b)
+          tma_load_3d(st + b * 8192, &tm_k, b * 64, tok0, bh, bar.full(s));
+        for (int b = 0; b < DVT / 64; ++b)
+          tma_load_3d(st + S::kKBytes + b * 8192, &tm_v, dv0 + b * 64, tok0, bh, bar.full(s));
+        issued = n + 1;
       }
-      if (n > 0) mbar_wait(b_full, (n - 1) & 1, p);  // last load landed before exit
+      for (int q = (issued > S::kStages ? issued - S::kStages : 0); q < issued; ++q)
+        mbar_wait(bar.full(q % S::kStages), (q / S::kStages) & 1, p, 13);
     }
   } else if (warp == 1) {
+    // ---------------------------- MMA issuer ------------------------------
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16(128, DVT, 1, 1);
       bool ok = true;
       int n = 0;
       for (int k = 0; k < NC && ok; ++k) {
-        ok = mbar_wait(b_master, k & 1, p);
-        for (int i = 0; i < tiles && ok; ++i, ++n) {
-          ok = mbar_wait(b_kready, n & 1, p);
+        ok = mbar_wait(bar.master(), k & 1, p, 2);
+        for (int j = 0; j < stages_per_chunk && ok; ++j, ++n) {
+          const int s = n % S::kStages;
+          ok = mbar_wait(bar.kready(s), (n / S::kStages) & 1, p, 3);
           if (!ok) break;
           tc_fence_after();
+          const uint32_t st = sbase + S::kOffStage + (uint32_t)s * S::kStageBytes;
 #pragma unroll
-          for (int kk = 0; kk < kKT / 16; ++kk)
-            mma_bf16_ss(tmem, sdesc_sw128(sbase + S::kOffK + kk * 2048, 16384, 1024),
-                        sdesc_sw128(sbase + S::kOffV + kk * 2048, 16384, 1024), idesc, 1);
-          mma_commit(b_empty);
+          for (int hf = 0; hf < S::kHalves; ++hf) {
+            // A = (w K)^T: M = the 128 dk rows of this half (two 64-dk boxes,
+            // MN-major), K = tokens.  B = V: N = the value columns (MN-major).
+            const uint32_t a0 = st + hf * 16384;
+#pragma unroll
+            for (int kk = 0; kk < kStageTok / 16; ++kk)
+              mma_bf16_ss(tmem + hf * DVT, sdesc_sw128(a0 + kk * 2048, 8192, 1024),
+                          sdesc_sw128(st + S::kKBytes + kk * 2048, 8192, 1024), idesc, 1);
+          }
+          mma_commit(bar.empty(s));
         }
-        if (ok) mma_commit(b_chunk);
+        if (ok) mma_commit(bar.chunk());
       }
-      mma_commit(b_done);  // completes once every MMA above has finished
+      mma_commit(bar.done());
     }
   } else {
+    // ------------------------------ workers -------------------------------
+    const int wt = threadIdx.x - 64;  // 0..255
     const int q = warp & 3;
-    const int r = q * 32 + lane;  // state row within the CTA = TMEM lane
-    const int dk = dk0 + r;
+    const int r = q * 32 + lane;      // TMEM lane = state row within a half
+    const int ch = wt >> 7;           // which half of the value columns
+    constexpr int kColsPer = DVT / 2;  // value columns per worker in the state passes
     const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16);
     const float* mchk = g.mchk + (long)bh * (NC + 1);
+    // n-vector: worker wt owns dk column wt (DK <= 256) for the running n.
+    const bool n_mine = n_owner && wt < DK;
+    float nval = (n_mine && n0) ? n0[(long)bh * DK + wt] : 0.f;
+    // Stage pass mapping: 16-byte column chunk cc (8 dk columns) of token rows
+    // rg * kRowsPer .. + kRowsPer - 1.
+    const int cc = wt % S::kCC;
+    const int rg = wt / S::kCC;
+    float part[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // n partials, this chunk
     bool ok = true;
-    float nval = (n_owner && n0) ? n0[(long)bh * DK + dk] : 0.f;
 
-    // master <- C0 (or zero)
-    for (int c = 0; c < DVT; c += 32) {
-      uint32_t v[32];
+    // master <- C0 (or zero): row r of each half, this worker's column half
+    for (int hf = 0; hf < S::kHalves; ++hf) {
+      const int dk = hf * 128 + r;
+      for (int c = 0; c < kColsPer; c += 32) {
+        const int col = ch * kColsPer + c;
+        uint32_t v[32];
 #pragma unroll
-      for (int j = 0; j < 32; ++j)
-        v[j] = __float_as_uint(C0 ? C0[((long)bh * DK + dk) * DV + dv0 + c + j] : 0.f);
-      tmem_st32(trow + c, v);
+        for (int j = 0; j < 32; ++j)
+          v[j] = __float_as_uint(C0 ? C0[((long)bh * DK + dk) * DV + dv0 + col + j] : 0.f);
+        tmem_st32(trow + hf * DVT + col, v);
+      }
     }
     tmem_wait_st();
+
+    // Column weights of the first chunk, prefetched (<= 4 per worker).
+    float acol_next[S::kMaxL / 256];
+#pragma unroll
+    for (int i = 0; i < S::kMaxL / 256; ++i) {
+      const int j = wt + 256 * i;
+      acol_next[i] = (j < L && j < T) ? g.acol[(long)bh * tpad + j] : -INFINITY;
+    }
 
     int n = 0;
     for (int k = 0; k < NC && ok; ++k) {
       if (k > 0) {
-        ok = mbar_wait(b_chunk, (k - 1) & 1, p);
+        ok = mbar_wait(bar.chunk(), (k - 1) & 1, p, 4);
         tc_fence_after();
+        if (n_owner) {
+          // fold the previous chunk's n partials into the running n
+#pragma unroll
+          for (int e = 0; e < 8; ++e) red_s[rg * DK + cc * 8 + e] = part[e];
+        }
+        named_bar_sync(1, kWorkers);
+        if (n_mine) {
+          float acc = 0.f;
+          for (int q2 = 0; q2 < 256 / S::kCC; ++q2) acc += red_s[q2 * DK + wt];
+          nval += acc;
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) part[e] = 0.f;
       }
       const float m_in = mchk[k], m_out = mchk[k + 1];
       const float gk = g.gtot[(long)bh * NC + k];
       const float decay = expf(gk + m_in - m_out);
       // state entering chunk k: store, then decay in place
-      const long row_off = (((long)bh * NC + k) * DK + dk) * DV + dv0;
-      for (int c = 0; c < DVT && ok; c += 32) {
-        uint32_t v[32];
-        tmem_ld32(trow + c, v);
-        tmem_wait_ld();
-        if (C_states) {
-          float4* dst = reinterpret_cast<float4*>(C_states + row_off + c);
+      for (int hf = 0; hf < S::kHalves && ok; ++hf) {
+        const int dk = hf * 128 + r;
+        const long row_off = (((long)bh * NC + k) * DK + dk) * DV + dv0;
+        for (int c = 0; c < kColsPer; c += 32) {
+          const int col = ch * kColsPer + c;
+          uint32_t v[32];
+          tmem_ld32(trow + hf * DVT + col, v);
+          tmem_wait_ld();
+          if (C_states) {
+            float4* dst = reinterpret_cast<float4*>(C_states + row_off + col);
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              dst[j] = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
+                                   __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
+          }
+          if (Cb) {
+            uint4* dst = reinterpret_cast<uint4*>(Cb + row_off + col);
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              dst[j] = make_uint4(
+                  pack_bf16x2(__uint_as_float(v[8 * j]), __uint_as_float(v[8 * j + 1])),
+                  pack_bf16x2(__uint_as_float(v[8 * j + 2]), __uint_as_float(v[8 * j + 3])),
+                  pack_bf16x2(__uint_as_float(v[8 * j + 4]), __uint_as_float(v[8 * j + 5])),
+                  pack_bf16x2(__uint_as_float(v[8 * j + 6]), __uint_as_float(v[8 * j + 7])));
+          }
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * decay);
+          tmem_st32(trow + hf * DVT + col, v);
+        }
+      }
+      tmem_wait_st();
+      if (n_mine) n_states[((long)bh * NC + k) * DK + wt] = nval;
+      nval *= decay;
+      tc_fence_before();
+      mbar_arrive(bar.master());
+
+      // Token weights of chunk k (from the prefetched column weights), then
+      // prefetch chunk k + 1's.
+#pragma unroll
+      for (int i = 0; i < S::kMaxL / 256; ++i) {
+        const int j = wt + 256 * i;
+        if (j < L) w_s[j] = p.key_scale * expf(gk + acol_next[i] - m_out);  // -inf -> 0
+      }
+#pragma unroll
+      for (int i = 0; i < S::kMaxL / 256; ++i) {
+        const int j = wt + 256 * i;
+        const long t = (long)(k + 1) * L + j;
+        acol_next[i] = (k + 1 < NC && j < L && t < T) ? g.acol[(long)bh * tpad + t] : -INFINITY;
+      }
+      named_bar_sync(1, kWorkers);
+
+      for (int j = 0; j < stages_per_chunk && ok; ++j, ++n) {
+        const int s = n % S::kStages;
+        ok = mbar_wait(bar.full(s), (n / S::kStages) & 1, p, 5);
+        uint8_t* box = smem + S::kOffStage + (uint32_t)s * S::kStageBytes + (cc >> 3) * 8192;
+        const float* ws = w_s + j * kStageTok;
+        // One pass: accumulate the unrounded products w_s k_s into the n
+        // partials (the normaliser enters h through |n^T q|, which can cancel,
+        // so it must not see the bf16 rounding), and weight the K rows in
+        // place for the rank-64 update.
+#pragma unroll
+        for (int rr = 0; rr < S::kRowsPer; ++rr) {
+          const int row = rg * S::kRowsPer + rr;
+          const float w = ws[row];
+          uint4* ptr = reinterpret_cast<uint4*>(box + sw128_offset(row, cc & 7));
+          uint4 u = *ptr;
+          __nv_bfloat162* h2 = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = __bfloat1622float2(h2[e]);
+            part[2 * e] = fmaf(f.x, w, part[2 * e]);
+            part[2 * e + 1] = fmaf(f.y, w, part[2 * e + 1]);
+            h2[e] = __floats2bfloat162_rn(f.x * w, f.y * w);
+          }
+          *ptr = u;
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(bar.kready(s));
+      }
+    }
+    // final state (fold the last chunk's n partials first)
+    if (ok) ok = mbar_wait(bar.chunk(), (NC - 1) & 1, p, 6);
+    tc_fence_after();
+    if (n_owner) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) red_s[rg * DK + cc * 8 + e] = part[e];
+    }
+    named_bar_sync(1, kWorkers);
+    if (n_mine) {
+      float acc = 0.f;
+      for (int q2 = 0; q2 < 256 / S::kCC; ++q2) acc += red_s[q2 * DK + wt];
+      nval += acc;
+    }
+    if (ok && C_T) {
+      for (int hf = 0; hf < S::kHalves; ++hf) {
+        const int dk = hf * 128 + r;
+        for (int c = 0; c < kColsPer; c += 32) {
+          const int col = ch * kColsPer + c;
+          uint32_t v[32];
+          tmem_ld32(trow + hf * DVT + col, v);
+          tmem_wait_ld();
+          float4* dst = reinterpret_cast<float4*>(C_T + ((long)bh * DK + dk) * DV + dv0 + col);
 #pragma unroll
           for (int j = 0; j < 8; ++j)
             dst[j] = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
                                  __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
         }
-        if (Cb) {
-          uint4* dst = reinterpret_cast<uint4*>(Cb + row_off + c);
-#pragma unroll
-          for (int j = 0; j < 4; ++j)
-            dst[j] = make_uint4(
-                pack_bf16x2(__uint_as_float(v[8 * j]), __uint_as_float(v[8 * j + 1])),
-                pack_bf16x2(__uint_as_float(v[8 * j + 2]), __uint_as_float(v[8 * j + 3])),
-                pack_bf16x2(__uint_as_float(v[8 * j + 4]), __uint_as_float(v[8 * j + 5])),
-                pack_bf16x2(__uint_as_float(v[8 * j + 6]), __uint_as_float(v[8 * j + 7])));
-        }
-#pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * decay);
-        tmem_st32(trow + c, v);
-      }
-      tmem_wait_st();
-      if (n_owner) n_states[((long)bh * NC + k) * DK + dk] = nval;
-      nval *= decay;
-      tc_fence_before();
-      mbar_arrive(b_master);
-
-      for (int i = 0; i < tiles && ok; ++i, ++n) {
-        ok = mbar_wait(b_full, n & 1, p);
-        // Token weights of this tile: thread r owns token row r.
-        const long t = (long)k * L + i * kKT + r;
-        const float w = (t < T) ? p.key_scale * expf(gk + g.acol[(long)bh * tpad + t] - m_out) : 0.f;
-        w_s[r] = w;
-        named_bar_sync(1, 128);
-        if (n_owner) {
-          // n update in fp32 from the unrounded products w_s k_s (thread r owns
-          // dk column r).  The normaliser enters h through |n^T q|, which can
-          // cancel, so it must not see the bf16 rounding of w_s k_s.
-          const uint8_t* box = smem + S::kOffK + (r >> 6) * 16384;
-          const int cc = r & 63;
-          float acc = 0.f;
-#pragma unroll 8
-          for (int s = 0; s < kKT; ++s) {
-            const __nv_bfloat16 x = *reinterpret_cast<const __nv_bfloat16*>(
-                box + sw128_offset(s, cc >> 3) + (cc & 7) * 2);
-            acc = fmaf(__bfloat162float(x), w_s[s], acc);
-          }
-          nval += acc;
-          named_bar_sync(1, 128);  // every column read done before the rows are rescaled
-        }
-        // Thread r scales token row r of the K tile by its weight, in place
-        // (bf16 operand of the rank-128 update).
-#pragma unroll
-        for (int b = 0; b < 2; ++b) {
-          uint8_t* box = smem + S::kOffK + b * 16384;
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            uint4* ptr = reinterpret_cast<uint4*>(box + sw128_offset(r, j));
-            uint4 u = *ptr;
-            __nv_bfloat162* h2 = reinterpret_cast<__nv_bfloat162*>(&u);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              float2 f = __bfloat1622float2(h2[e]);
-              h2[e] = __floats2bfloat162_rn(f.x * w, f.y * w);
-            }
-            *ptr = u;
-          }
-        }
-        fence_proxy_async_smem();
-        mbar_arrive(b_kready);
       }
     }
-    // final state
-    if (ok) ok = mbar_wait(b_chunk, (NC - 1) & 1, p);
-    tc_fence_after();
-    if (ok && C_T) {
-      for (int c = 0; c < DVT; c += 32) {
-        uint32_t v[32];
-        tmem_ld32(trow + c, v);
-        tmem_wait_ld();
-        float4* dst = reinterpret_cast<float4*>(C_T + ((long)bh * DK + dk) * DV + dv0 + c);
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-          dst[j] = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
-                               __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
-      }
-    }
-    if (n_owner && n_T) n_T[(long)bh * DK + dk] = nval;
-    if (m_T && blockIdx.x == 0 && blockIdx.y == 0 && r == 0) m_T[bh] = mchk[NC];
+    if (n_mine && n_T) n_T[(long)bh * DK + wt] = nval;
+    if (m_T && blockIdx.x == 0 && wt == 0) m_T[bh] = mchk[NC];
   }
 
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
-    if (lane == 0) mbar_wait(b_done, 0, p);
+    if (lane == 0) mbar_wait(bar.done(), 0, p, 15);
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, S::kTmemCols);
   }
 }
 
-template <int DVT>
+template <int DK, int DVT>
 cudaError_t launch_states_t(const Problem& p, const void* K, const void* V, const float* C0,
                             const float* n0, Gates g, float* C_states, __nv_bfloat16* Cb,
                             float* n_states, float* C_T, float* n_T, float* m_T, cudaStream_t st) {
-  using S = SCfg<DVT>;
+  using S = SCfg<DK, DVT>;
   CUtensorMap tk, tv;
-  if (!encode_tmap_bf16_3d(&tk, K, p.DK, p.T, p.BH, 64, kKT) ||
-      !encode_tmap_bf16_3d(&tv, V, p.DV, p.T, p.BH, 64, kKT))
+  if (!encode_tmap_bf16_3d(&tk, K, p.DK, p.T, p.BH, 64, kStageTok) ||
+      !encode_tmap_bf16_3d(&tv, V, p.DV, p.T, p.BH, 64, kStageTok))
     return cudaErrorInvalidValue;
-  auto kern = tc_states_kernel<DVT>;
+  auto kern = tc_states_kernel<DK, DVT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kSmem);
   if (e != cudaSuccess) return e;
-  dim3 grid(p.DV / DVT, p.DK / kRows, p.BH);
+  dim3 grid(p.DV / DVT, p.BH);
   kern<<<grid, kThreads, S::kSmem, st>>>(tk, tv, p, g, C0, n0, C_states, Cb, n_states, C_T, n_T,
                                          m_T);
   return cudaGetLastError();
@@ -288,7 +381,8 @@ cudaError_t launch_states_t(const Problem& p, const void* K, const void* V, cons
 
 bool tc_states_supported(const Problem& p) {
   const bool dv_ok = p.DV == 64 || p.DV == 128 || p.DV % 256 == 0;
-  return (p.DK == 128 || p.DK == 256) && dv_ok && p.DV <= 1024 && p.L % kKT == 0 && p.T > 0;
+  return (p.DK == 128 || p.DK == 256) && dv_ok && p.DV <= 1024 && p.L % 128 == 0 &&
+         p.L <= 1024 && p.T > 0;
 }
 
 cudaError_t launch_tc_states_impl(const Problem& p, const void* K, const void* V, const float* C0,
@@ -296,11 +390,17 @@ cudaError_t launch_tc_states_impl(const Problem& p, const void* K, const void* V
                                   float* n_states, float* C_T, float* n_T, float* m_T,
                                   cudaStream_t st) {
   const int dvt = p.DV >= 256 ? 256 : p.DV;
-  switch (dvt) {
-    case 64: return launch_states_t<64>(p, K, V, C0, n0, g, C_states, Cb, n_states, C_T, n_T, m_T, st);
-    case 128: return launch_states_t<128>(p, K, V, C0, n0, g, C_states, Cb, n_states, C_T, n_T, m_T, st);
-    case 256: return launch_states_t<256>(p, K, V, C0, n0, g, C_states, Cb, n_states, C_T, n_T, m_T, st);
-  }
+#define MLSTM_ST_CASE(dk, dvt_)                                                                  \
+  if (p.DK == dk && dvt == dvt_)                                                                 \
+    return launch_states_t<dk, dvt_>(p, K, V, C0, n0, g, C_states, Cb, n_states, C_T, n_T, m_T, \
+                                     st);
+  MLSTM_ST_CASE(128, 64)
+  MLSTM_ST_CASE(128, 128)
+  MLSTM_ST_CASE(128, 256)
+  MLSTM_ST_CASE(256, 64)
+  MLSTM_ST_CASE(256, 128)
+  MLSTM_ST_CASE(256, 256)
+#undef MLSTM_ST_CASE
   return cudaErrorNotSupported;
 }
 

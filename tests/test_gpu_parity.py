@@ -32,7 +32,9 @@ def run(w, x, algo="auto"):
     H, fin = api.mlstm_fw(d["Q"], d["K"], d["V"], d["i_pre"], d["f_pre"], d["C0"], d["n0"],
                           d["m0"], chunk_size=w.chunk_size, gate_mode=w.gate_mode, algo=algo)
     torch.cuda.synchronize()
-    assert api.last_device_error() == _lib.OK
+    st = api.last_device_error()
+    assert st == _lib.OK, \
+        f"device status {st}, error word 0x{_lib.lib().mlstm_last_device_error_word():08x}"
     return H, fin
 
 
