@@ -11,22 +11,33 @@
 //   h_r   = O_r / max(|den_r|, e^{-(bcum_r + mu_r)})
 //
 // What differs is the work decomposition.  With at most two 128-token
-// key/value tiles per query tile, the gated P tiles of an item fit in shared
-// memory, so an item computes S and P once and then sweeps the value columns
-// in 128-wide tiles d: O_d = Q~ C_k[:, d] + sum_i P_i V_i[:, d], where Q~ is
-// the query tile with row r scaled by e^{m_k - mu_r} (in place, once the S
-// MMAs have read Q).  The Q tile is loaded once per item, S is never
-// recomputed per value tile, and the MMAs of consecutive value tiles need no
-// hand-off from the row threads.  The two TMEM output accumulators alternate
-// between value tiles; the epilogue of tile d (bf16 rows into a swizzled
-// staging tile, then a TMA store) overlaps the MMAs of tile d + 1.
+// key/value tiles per query tile, the gated P tiles of an item stay on chip,
+// so an item computes S and P once and then sweeps the value columns in
+// 128-wide tiles d: O_d = sum_i P_i V_i[:, d] + Q~ C_k[:, d], where Q~ is the
+// query tile with row r scaled by e^{m_k - mu_r} (in place, once the S MMAs
+// have read Q).  The Q tile is loaded once per item, S is never recomputed per
+// value tile, and the MMAs of consecutive value tiles need no hand-off from
+// the row threads.  The two TMEM output accumulators alternate between value
+// tiles; the epilogue of tile d (bf16 rows into a swizzled staging tile, then
+// a TMA store) overlaps the MMAs of tile d + 1.
+//
+// P never touches shared memory: the row threads write it back as packed bf16
+// over the TMEM columns of the S tile it came from, and the P.V MMAs take
+// their A operand from TMEM.  The shared memory this saves deepens the TMA
+// ring, which is what bounds this kernel (each item streams C_k and V through
+// the ring once per value tile).
 //
 // Roles (320 threads): warp 0 TMA producer; warp 1 TMEM owner and MMA issuer;
 // warps 2..9 two threads per query row (each owning half of the columns):
 // gating of S into P, the in-place scaling of Q, row sums, epilogue.
-// TMEM (512 columns): O at 0 and 128, S at 256 and 384.
-// MMA order per item: S_0 [, S_1], (wait for the scaled Q), then for every
-// value tile d: Q~.C_k[:, d], P_0.V_0[:, d] [, P_1.V_1[:, d]].
+// TMEM (512 columns): O at 0 and 128, S_0 / P_0 at 256, S_1 / P_1 at 384.
+// The half of the row threads that owns S columns [64h, 64h + 64) writes its
+// 64 bf16 P values (32 packed columns) to columns [64h, 64h + 32), which only
+// it has read, so the halves never race.
+// MMA order per item: S_0 [, S_1], then for every value tile d:
+// P_0.V_0[:, d] [, P_1.V_1[:, d]], (first tile: wait for the scaled Q),
+// Q~.C_k[:, d].  S_i of the next item waits until the last P_i.V_i MMA of
+// this one has completed; the Q~.C_k MMAs issued after it hide that wait.
 #include <cuda.h>
 
 #include "tc.h"
@@ -41,6 +52,7 @@ constexpr int kThreads = 320;
 constexpr int kQT = 128;
 constexpr int kKT = 128;
 constexpr int kPSlots = 2;  // key/value tiles per item (chunks of at most 256)
+constexpr uint32_t kColPHalf = 64;  // P columns of the upper half within an S tile
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS0 = 256, kColS1 = 384;
 
@@ -53,17 +65,15 @@ struct WCfg {
   static constexpr uint32_t kMNSlabBytes = (DVT / 64) * 8192;
   static constexpr uint32_t kStageBytes = 16384;
   static_assert(kKSlabBytes <= kStageBytes && kMNSlabBytes <= kStageBytes, "stage size");
-  static constexpr uint32_t kPBytes = kQT * kKT * 2;  // one slot
   static constexpr uint32_t kOutBytes = kQT * DVT * 2;  // output staging tile
   static constexpr uint32_t kMiscBytes = 2 * kPSlots * kKT * 4 + 2 * DK * 4 + 256 * 4 + 512;
   static constexpr uint32_t kBudget = 227 * 1024 - 1024;
   static constexpr int kStagesFit =
-      (int)((kBudget - kQBytes - kPSlots * kPBytes - kOutBytes - kMiscBytes) / kStageBytes);
+      (int)((kBudget - kQBytes - kOutBytes - kMiscBytes) / kStageBytes);
   static constexpr int kStages = kStagesFit > 12 ? 12 : kStagesFit;
   static_assert(kStages >= 3, "ring too shallow");
   static constexpr uint32_t kOffQ = 0;
-  static constexpr uint32_t kOffP = kOffQ + kQBytes;
-  static constexpr uint32_t kOffOut = kOffP + kPSlots * kPBytes;
+  static constexpr uint32_t kOffOut = kOffQ + kQBytes;
   static constexpr uint32_t kOffStage = kOffOut + kOutBytes;
   static constexpr uint32_t kOffAcol = kOffStage + kStages * kStageBytes;  // float[2][256]
   static constexpr uint32_t kOffN = kOffAcol + 2 * kPSlots * kKT * 4;       // float[2][DK]
@@ -81,12 +91,14 @@ struct WBars {
   __device__ __forceinline__ uint32_t empty(int i) const { return a + 128 + 8 * i; }
   __device__ __forceinline__ uint32_t q_full() const { return a + 256; }
   __device__ __forceinline__ uint32_t q_empty() const { return a + 264; }
-  __device__ __forceinline__ uint32_t s_full(int b) const { return a + 272 + 8 * b; }
-  __device__ __forceinline__ uint32_t s_empty(int b) const { return a + 288 + 8 * b; }
+  __device__ __forceinline__ uint32_t s_full(int i) const { return a + 272 + 8 * i; }
+  // One "accumulator ready" barrier per O buffer: consecutive value tiles need
+  // no hand-off from the row threads, so a single barrier could complete twice
+  // before they wait on it and its parity would no longer tell the tiles apart.
+  __device__ __forceinline__ uint32_t o_full(int b) const { return a + 288 + 8 * b; }
   __device__ __forceinline__ uint32_t p_full(int i) const { return a + 304 + 8 * i; }
-  __device__ __forceinline__ uint32_t p_empty(int i) const { return a + 320 + 8 * i; }
+  __device__ __forceinline__ uint32_t pv_done(int i) const { return a + 320 + 8 * i; }
   __device__ __forceinline__ uint32_t q_scaled() const { return a + 336; }
-  __device__ __forceinline__ uint32_t o_done() const { return a + 352; }
   __device__ __forceinline__ uint32_t o_empty(int b) const { return a + 360 + 8 * b; }
   __device__ __forceinline__ uint32_t mma_idle() const { return a + 376; }
 };
@@ -139,13 +151,12 @@ tc_parallel_wide_kernel(const __grid_constant__ CUtensorMap tm_q,
     mbar_init(bar.q_empty(), 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar.s_full(i), 1);
-      mbar_init(bar.s_empty(i), 256);
       mbar_init(bar.p_full(i), 256);
-      mbar_init(bar.p_empty(i), 1);
+      mbar_init(bar.pv_done(i), 1);
+      mbar_init(bar.o_full(i), 1);
       mbar_init(bar.o_empty(i), 256);
     }
     mbar_init(bar.q_scaled(), 256);
-    mbar_init(bar.o_done(), 1);
     mbar_init(bar.mma_idle(), 1);
     fence_barrier_init();
   }
@@ -190,12 +201,6 @@ tc_parallel_wide_kernel(const __grid_constant__ CUtensorMap tm_q,
           }
         for (int d = 0; d < n_dv && ok; ++d) {
           const int dv0 = d * DVT;
-          for (int c = 0; c < C::kSlabsK && ok; ++c) {
-            const uint32_t dst = next_stage(C::kMNSlabBytes);
-            for (int b = 0; b < DVT / 64; ++b)
-              tma_load_3d(dst + b * 8192, &tm_c, dv0 + b * 64, c * 64, x.bh * p.NC + x.k,
-                          bar.full((slab - 1) % C::kStages));
-          }
           for (int i = 0; i < x.n_kv && ok; ++i)
             for (int v = 0; v < 2 && ok; ++v) {
               const uint32_t dst = next_stage(C::kMNSlabBytes);
@@ -203,6 +208,12 @@ tc_parallel_wide_kernel(const __grid_constant__ CUtensorMap tm_q,
                 tma_load_3d(dst + b * 8192, &tm_v, dv0 + b * 64, x.c0 + i * kKT + v * 64, x.bh,
                             bar.full((slab - 1) % C::kStages));
             }
+          for (int c = 0; c < C::kSlabsK && ok; ++c) {
+            const uint32_t dst = next_stage(C::kMNSlabBytes);
+            for (int b = 0; b < DVT / 64; ++b)
+              tma_load_3d(dst + b * 8192, &tm_c, dv0 + b * 64, c * 64, x.bh * p.NC + x.k,
+                          bar.full((slab - 1) % C::kStages));
+          }
         }
       }
       for (int q = (slab > C::kStages ? slab - C::kStages : 0); q < slab; ++q)
@@ -215,8 +226,8 @@ tc_parallel_wide_kernel(const __grid_constant__ CUtensorMap tm_q,
       constexpr uint32_t idS = idesc_bf16(128, kKT, 0, 0);
       constexpr uint32_t idO = idesc_bf16(128, DVT, 0, 1);
       bool ok = true;
-      int slab = 0, tile = 0, dcount = 0;
-      int pc0 = 0, pc1 = 0;  // times P slot 0 / 1 has been filled (no arrays: registers)
+      int slab = 0, dcount = 0;
+      int sc0 = 0, sc1 = 0;  // times S tile 0 / 1 has been filled (no arrays: registers)
       auto take = [&]() -> uint32_t {
         const int s = slab % C::kStages, u = slab / C::kStages;
         ok = ok && mbar_wait(bar.full(s), u & 1, p, 5);
@@ -228,11 +239,11 @@ tc_parallel_wide_kernel(const __grid_constant__ CUtensorMap tm_q,
       for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++n) {
         const WItem x = decode_witem(it, p, n_q);
         ok = mbar_wait(bar.q_full(), n & 1, p, 3);
-        for (int i = 0; i < x.n_kv && ok; ++i, ++tile) {  // S_i
-          const int buf = tile & 1;
-          if (tile >= 2) ok = ok && mbar_wait(bar.s_empty(buf), ((tile >> 1) - 1) & 1, p, 4);
+        for (int i = 0; i < x.n_kv && ok; ++i) {  // S_i
+          const int fills = i ? sc1 : sc0;
+          if (fills >= 1) ok = ok && mbar_wait(bar.pv_done(i), (fills - 1) & 1, p, 4);
           tc_fence_after();
-          const uint32_t dS = tmem + (buf ? kColS1 : kColS0);
+          const uint32_t dS = tmem + (i ? kColS1 : kColS0);
           for (int c = 0; c < C::kSlabsK && ok; ++c) {
             const uint32_t s = take();
             if (!ok) break;
@@ -244,16 +255,36 @@ tc_parallel_wide_kernel(const __grid_constant__ CUtensorMap tm_q,
                           sdesc_sw128(b0 + kk * 32, 16, 1024), idS, (c | kk) != 0);
             mma_commit(bar.empty(s));
           }
-          mma_commit(bar.s_full(buf));
+          mma_commit(bar.s_full(i));
+          if (i) ++sc1; else ++sc0;
         }
-        ok = ok && mbar_wait(bar.q_scaled(), n & 1, p, 7);  // Q rows scaled in place
-        tc_fence_after();
         for (int d = 0; d < n_dv && ok; ++d, ++dcount) {
           const int ob = dcount & 1;
           const uint32_t dO = tmem + (uint32_t)ob * 128u;
           if (dcount >= 2) ok = ok && mbar_wait(bar.o_empty(ob), ((dcount >> 1) - 1) & 1, p, 6);
           tc_fence_after();
-          for (int c = 0; c < C::kSlabsK && ok; ++c) {  // Q . C_k[:, d]
+          for (int i = 0; i < x.n_kv && ok; ++i) {  // P_i . V_i[:, d], A from TMEM
+            if (d == 0) ok = mbar_wait(bar.p_full(i), ((i ? sc1 : sc0) - 1) & 1, p, 8);
+            tc_fence_after();
+            const uint32_t aP = tmem + (i ? kColS1 : kColS0);
+            for (int v = 0; v < 2 && ok; ++v) {
+              const uint32_t s = take();
+              if (!ok) break;
+              const uint32_t b0 = sbase + C::kOffStage + s * C::kStageBytes;
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk)
+                mma_bf16_ts(dO, aP + (uint32_t)v * kColPHalf + (uint32_t)kk * 8u,
+                            sdesc_sw128(b0 + kk * 2048, 8192, 1024), idO, (i | v | kk) != 0);
+              mma_commit(bar.empty(s));
+            }
+            if (d == n_dv - 1) mma_commit(bar.pv_done(i));
+          }
+          if (!ok) break;
+          if (d == 0) {
+            ok = mbar_wait(bar.q_scaled(), n & 1, p, 7);  // Q rows scaled in place
+            tc_fence_after();
+          }
+          for (int c = 0; c < C::kSlabsK && ok; ++c) {  // Q~ . C_k[:, d]
             const uint32_t s = take();
             if (!ok) break;
             const uint32_t a0 = sbase + C::kOffQ + c * 16384;
@@ -261,32 +292,12 @@ tc_parallel_wide_kernel(const __grid_constant__ CUtensorMap tm_q,
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
               mma_bf16_ss(dO, sdesc_sw128(a0 + kk * 32, 16, 1024),
-                          sdesc_sw128(b0 + kk * 2048, 8192, 1024), idO, (c | kk) != 0);
+                          sdesc_sw128(b0 + kk * 2048, 8192, 1024), idO, 1);
             mma_commit(bar.empty(s));
           }
           if (!ok) break;
           if (d == n_dv - 1) mma_commit(bar.q_empty());  // last reader of Q issued
-          for (int i = 0; i < x.n_kv && ok; ++i) {
-            if (d == 0) ok = mbar_wait(bar.p_full(i), (i ? pc1 : pc0) & 1, p, 8);
-            tc_fence_after();
-            for (int v = 0; v < 2 && ok; ++v) {
-              const uint32_t s = take();
-              if (!ok) break;
-              const uint32_t a0 = sbase + C::kOffP + i * C::kPBytes + v * 16384;
-              const uint32_t b0 = sbase + C::kOffStage + s * C::kStageBytes;
-#pragma unroll
-              for (int kk = 0; kk < 4; ++kk)
-                mma_bf16_ss(dO, sdesc_sw128(a0 + kk * 32, 16, 1024),
-                            sdesc_sw128(b0 + kk * 2048, 8192, 1024), idO, 1);
-              mma_commit(bar.empty(s));
-            }
-            if (d == n_dv - 1) {
-              mma_commit(bar.p_empty(i));
-              if (i) ++pc1; else ++pc0;
-            }
-          }
-          if (!ok) break;
-          mma_commit(bar.o_done());
+          mma_commit(bar.o_full(ob));
         }
       }
       mma_commit(bar.mma_idle());
@@ -303,8 +314,8 @@ tc_parallel_wide_kernel(const __grid_constant__ CUtensorMap tm_q,
     constexpr int kHalfO = DVT / 2;
     constexpr int kSlabsPerHalf = (C::kSlabsK + 1) / 2;
     bool ok = true;
-    int tile = 0, dcount = 0;
-    int pc0 = 0, pc1 = 0;
+    int dcount = 0;
+    int pc0 = 0, pc1 = 0;  // times S tile 0 / 1 has been turned into P
     auto fetch_rows = [&](const WItem& x, float& m_in, float& amax, float& bc) {
       const int t = x.t0 + r;
       m_in = g.mchk[(long)x.bh * (p.NC + 1) + x.k];
@@ -355,15 +366,13 @@ tc_parallel_wide_kernel(const __grid_constant__ CUtensorMap tm_q,
       }
       float den = f_inter * dn;
 
-      // Gated P tiles, once per item.
-      for (int i = 0; i < x.n_kv; ++i, ++tile) {
-        const int buf = tile & 1;
-        ok = ok && mbar_wait(bar.s_full(buf), (tile >> 1) & 1, p, 10);
+      // Gated P tiles, once per item, written back over their S tiles in TMEM.
+      for (int i = 0; i < x.n_kv; ++i) {
         const int pc = i ? pc1 : pc0;
-        if (pc >= 1) ok = ok && mbar_wait(bar.p_empty(i), (pc - 1) & 1, p, 11);
+        ok = ok && mbar_wait(bar.s_full(i), pc & 1, p, 10);
         tc_fence_after();
         const bool diag = (i == x.n_kv - 1);
-        const uint32_t scol = (buf ? kColS1 : kColS0) + h * 64;
+        const uint32_t scol = (i ? kColS1 : kColS0) + h * kColPHalf;
         float rs = 0.f;
         if (ok) {
           uint32_t v[64];
@@ -382,16 +391,11 @@ tc_parallel_wide_kernel(const __grid_constant__ CUtensorMap tm_q,
             rs += pa + pb;
             pk[j >> 1] = pack_bf16x2(pa, pb);
           }
-          uint8_t* prow = smem + C::kOffP + i * C::kPBytes + h * 16384;
-#pragma unroll
-          for (int j = 0; j < 8; ++j)
-            *reinterpret_cast<uint4*>(prow + sw128_offset(r, j)) =
-                make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+          tmem_st32(trow + scol, pk);
+          tmem_wait_st();
         }
         den += rs;
         tc_fence_before();
-        mbar_arrive(bar.s_empty(buf));
-        fence_proxy_async_smem();
         mbar_arrive(bar.p_full(i));
         if (i) ++pc1; else ++pc0;
       }
@@ -440,7 +444,7 @@ tc_parallel_wide_kernel(const __grid_constant__ CUtensorMap tm_q,
 
       for (int d = 0; d < n_dv; ++d, ++dcount) {
         const uint32_t colO = (uint32_t)(dcount & 1) * 128u + h * kHalfO;
-        ok = ok && mbar_wait(bar.o_done(), dcount & 1, p, 14);
+        ok = ok && mbar_wait(bar.o_full(dcount & 1), (dcount >> 1) & 1, p, 12);
         tc_fence_after();
         if (rt == 0) tma_store_wait_read_all();  // the staging tile is free again
         named_bar_sync(1, 256);
