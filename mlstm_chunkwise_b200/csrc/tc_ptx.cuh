@@ -248,6 +248,13 @@ __device__ __forceinline__ uint32_t sw128_offset(uint32_t r, uint32_t c) {
   return r * 128u + ((c ^ (r & 7u)) << 4);
 }
 
+// Byte offset of 16-byte chunk c (0..3) of row r in a tile of 64-byte rows
+// laid out with the 64-byte swizzle (chunk bits 4..5 XOR address bits 7..8);
+// the tile must start on a 512-byte boundary.
+__device__ __forceinline__ uint32_t sw64_offset(int r, int c) {
+  return (uint32_t)(r * 64 + ((c ^ ((r >> 1) & 3)) << 4));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
@@ -273,5 +280,11 @@ __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
 // Out-of-range elements of a box read as zero.  Returns false on failure.
 bool encode_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1,
                          uint64_t d2, uint32_t b0, uint32_t b1);
+
+// General form: elements of `elem_bytes` (2 = bf16, 4 = fp32) and a swizzle
+// span of `swizzle_bytes` (32, 64 or 128), which must equal the box's inner
+// extent in bytes (b0 * elem_bytes).  Returns false on failure.
+bool encode_tmap_3d(CUtensorMap* map, const void* base, int elem_bytes, uint64_t d0, uint64_t d1,
+                    uint64_t d2, uint32_t b0, uint32_t b1, int swizzle_bytes);
 
 }  // namespace mlstm

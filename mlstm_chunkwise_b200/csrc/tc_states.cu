@@ -15,7 +15,10 @@
 // stream in 64-token stages through a ring deep enough to keep ~190 KB of
 // loads in flight.  Before each chunk the worker threads read the master (the
 // state entering the chunk), write it out (fp32 and/or bf16 operand copy) and
-// scale it by the decay.
+// scale it by the decay.  The write-out goes through a 2 KB shared-memory tile
+// per warp (32 state rows x 64 bytes) and a TMA store: a warp whose lanes each
+// stored their own state row would touch 32 rows per instruction, and those
+// scattered stores, not the MMAs, would then set the pace of the recurrence.
 //
 // Roles (320 threads): warp 0 TMA producer, warp 1 TMEM owner + MMA issuer,
 // warps 2..9 workers: per chunk, the token weights and the store and decay of
@@ -23,6 +26,8 @@
 // sums (fp32, from the unrounded products w_s k_s) and weights the K rows in
 // place.
 #include <cuda.h>
+
+#include <cstring>
 
 #include "tc.h"
 #include "tc_ptx.cuh"
@@ -49,14 +54,17 @@ struct SCfg {
   static constexpr int kRowsPer = kStageTok * kCC / 256;  // rows per worker per stage
   static constexpr uint32_t kWBytes = kMaxL * 4;           // token weights of one chunk
   static constexpr uint32_t kRedBytes = (256 / kCC) * DK * 4;  // n partials [row group][dk]
-  static constexpr uint32_t kBudget = 227 * 1024 - 1024 - 512 - kWBytes - kRedBytes;
+  static constexpr uint32_t kStgBytes = 8 * 2048;  // one 32 x 64-byte store tile per worker warp
+  static constexpr uint32_t kBudget = 227 * 1024 - 1024 - 512 - kWBytes - kRedBytes - kStgBytes;
   static constexpr int kStagesFit = (int)(kBudget / kStageBytes);
   static constexpr int kStages = kStagesFit > 8 ? 8 : kStagesFit;
   static_assert(kStages >= 2, "ring too shallow");
   static constexpr uint32_t kOffStage = 0;
   static constexpr uint32_t kOffW = kStages * kStageBytes;  // float[kMaxL]
   static constexpr uint32_t kOffRed = kOffW + kWBytes;      // float[256 / kCC][DK]
-  static constexpr uint32_t kOffBar = kOffRed + kRedBytes;
+  static constexpr uint32_t kOffStg = kOffRed + kRedBytes;  // [8 warps][32 rows][64 B], 64 B swizzle
+  static_assert(kOffStg % 1024 == 0, "store tiles must sit on a swizzle-atom boundary");
+  static constexpr uint32_t kOffBar = kOffStg + kStgBytes;
   static constexpr uint32_t kOffSlot = kOffBar + 8 * 32;
   static constexpr uint32_t kBytes = kOffSlot + 16;
   static constexpr uint32_t kSmem = kBytes + 1024;
@@ -77,6 +85,7 @@ struct SBars {
 template <int DK, int DVT>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_states_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                 const __grid_constant__ CUtensorMap tm_cs, const __grid_constant__ CUtensorMap tm_cb,
                  Problem p, Gates g, const float* __restrict__ C0, const float* __restrict__ n0,
                  float* __restrict__ C_states, __nv_bfloat16* __restrict__ Cb,
                  float* __restrict__ n_states, float* __restrict__ C_T, float* __restrict__ n_T,
@@ -181,6 +190,8 @@ tc_states_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
     constexpr int kColsPer = DVT / 2;  // value columns per worker in the state passes
     const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16);
     const float* mchk = g.mchk + (long)bh * (NC + 1);
+    uint8_t* stg = smem + S::kOffStg + (warp - 2) * 2048;  // this warp's store tile
+    const uint32_t stg_u = sbase + S::kOffStg + (uint32_t)(warp - 2) * 2048u;
     // n-vector: worker wt owns dk column wt (DK <= 256) for the running n.
     const bool n_mine = n_owner && wt < DK;
     float nval = (n_mine && n0) ? n0[(long)bh * DK + wt] : 0.f;
@@ -235,31 +246,48 @@ tc_states_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
       const float m_in = mchk[k], m_out = mchk[k + 1];
       const float gk = g.gtot[(long)bh * NC + k];
       const float decay = expf(gk + m_in - m_out);
-      // state entering chunk k: store, then decay in place
+      // state entering chunk k: store (TMA, from this warp's tile), then decay in place
       for (int hf = 0; hf < S::kHalves && ok; ++hf) {
-        const int dk = hf * 128 + r;
-        const long row_off = (((long)bh * NC + k) * DK + dk) * DV + dv0;
+        const int dk0 = hf * 128 + q * 32;  // first state row of this warp's lanes
         for (int c = 0; c < kColsPer; c += 32) {
           const int col = ch * kColsPer + c;
           uint32_t v[32];
           tmem_ld32(trow + hf * DVT + col, v);
           tmem_wait_ld();
-          if (C_states) {
-            float4* dst = reinterpret_cast<float4*>(C_states + row_off + col);
+          if (C_states) {  // fp32: two 16-column boxes
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
-              dst[j] = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
-                                   __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
+            for (int half = 0; half < 2; ++half) {
+              if (lane == 0) tma_store_wait_read_all();
+              __syncwarp();
+#pragma unroll
+              for (int j = 0; j < 4; ++j)
+                *reinterpret_cast<uint4*>(stg + sw64_offset(lane, j)) =
+                    make_uint4(v[16 * half + 4 * j], v[16 * half + 4 * j + 1],
+                               v[16 * half + 4 * j + 2], v[16 * half + 4 * j + 3]);
+              fence_proxy_async_smem();
+              __syncwarp();
+              if (lane == 0) {
+                tma_store_3d(&tm_cs, stg_u, dv0 + col + 16 * half, dk0, bh * NC + k);
+                tma_store_commit();
+              }
+            }
           }
           if (Cb) {
-            uint4* dst = reinterpret_cast<uint4*>(Cb + row_off + col);
+            if (lane == 0) tma_store_wait_read_all();
+            __syncwarp();
 #pragma unroll
             for (int j = 0; j < 4; ++j)
-              dst[j] = make_uint4(
+              *reinterpret_cast<uint4*>(stg + sw64_offset(lane, j)) = make_uint4(
                   pack_bf16x2(__uint_as_float(v[8 * j]), __uint_as_float(v[8 * j + 1])),
                   pack_bf16x2(__uint_as_float(v[8 * j + 2]), __uint_as_float(v[8 * j + 3])),
                   pack_bf16x2(__uint_as_float(v[8 * j + 4]), __uint_as_float(v[8 * j + 5])),
                   pack_bf16x2(__uint_as_float(v[8 * j + 6]), __uint_as_float(v[8 * j + 7])));
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_3d(&tm_cb, stg_u, dv0 + col, dk0, bh * NC + k);
+              tma_store_commit();
+            }
           }
 #pragma unroll
           for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * decay);
@@ -347,6 +375,7 @@ tc_states_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
     }
     if (n_mine && n_T) n_T[(long)bh * DK + wt] = nval;
     if (m_T && blockIdx.x == 0 && wt == 0) m_T[bh] = mchk[NC];
+    if (lane == 0) tma_store_wait_all();  // the state stores have landed
   }
 
   tc_fence_before();
@@ -364,16 +393,21 @@ cudaError_t launch_states_t(const Problem& p, const void* K, const void* V, cons
                             const float* n0, Gates g, float* C_states, __nv_bfloat16* Cb,
                             float* n_states, float* C_T, float* n_T, float* m_T, cudaStream_t st) {
   using S = SCfg<DK, DVT>;
-  CUtensorMap tk, tv;
+  CUtensorMap tk, tv, tcs, tcb;
+  memset(&tcs, 0, sizeof(tcs));
+  memset(&tcb, 0, sizeof(tcb));
+  const uint64_t n_boxes = (uint64_t)p.BH * p.NC;  // state tiles [DK][DV] per (b, h, chunk)
   if (!encode_tmap_bf16_3d(&tk, K, p.DK, p.T, p.BH, 64, kStageTok) ||
-      !encode_tmap_bf16_3d(&tv, V, p.DV, p.T, p.BH, 64, kStageTok))
+      !encode_tmap_bf16_3d(&tv, V, p.DV, p.T, p.BH, 64, kStageTok) ||
+      (C_states && !encode_tmap_3d(&tcs, C_states, 4, p.DV, p.DK, n_boxes, 16, 32, 64)) ||
+      (Cb && !encode_tmap_3d(&tcb, Cb, 2, p.DV, p.DK, n_boxes, 32, 32, 64)))
     return cudaErrorInvalidValue;
   auto kern = tc_states_kernel<DK, DVT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kSmem);
   if (e != cudaSuccess) return e;
   dim3 grid(p.DV / DVT, p.BH);
-  kern<<<grid, kThreads, S::kSmem, st>>>(tk, tv, p, g, C0, n0, C_states, Cb, n_states, C_T, n_T,
-                                         m_T);
+  kern<<<grid, kThreads, S::kSmem, st>>>(tk, tv, tcs, tcb, p, g, C0, n0, C_states, Cb, n_states,
+                                         C_T, n_T, m_T);
   return cudaGetLastError();
 }
 
