@@ -423,8 +423,7 @@ mlstm_status mlstm_fw_parallel(const void* Q, const void* K, const void* V, cons
   if (a == MLSTM_ALGO_TC) {
     __nv_bfloat16* Cb = reinterpret_cast<__nv_bfloat16*>(rest);
     s = from_cuda(launch_family(MLSTM_KERNEL_TC_PARALLEL, 1, st, [&] {
-      cudaError_t e =
-          launch_states_to_bf16(C_states, Cb, (size_t)p.BH * p.NC * (size_t)DK * DV, st);
+      cudaError_t e = launch_states_to_operand(C_states, Cb, (long)p.BH * p.NC, DK, DV, st);
       if (e != cudaSuccess) return e;
       return launch_tc_parallel(p, Q, K, V, g, Cb, n_states, H, n_out, m_out, st);
     }));

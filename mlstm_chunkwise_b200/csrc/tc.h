@@ -5,6 +5,17 @@
 
 namespace mlstm {
 
+// Layout of the bf16 operand copy of the chunk states (internal to the
+// tensor-core path).  For every (b, h, chunk) index bhk and every 64-column
+// block vb of DV there is a [DK][64] block of 128-byte rows, and row dk holds
+// its 16-byte chunk j at position j ^ (dk & 7): byte for byte the shared-memory
+// image of an MN-major operand tile with the 128-byte swizzle.  A run of rows
+// that starts at a multiple of 8 therefore moves between global and shared
+// memory with one untiled bulk copy, in either direction.
+__host__ __device__ inline size_t cb_block_row(long bhk, int vb, int dk, int DK, int n_vb) {
+  return (((size_t)bhk * n_vb + vb) * DK + dk) * 64;  // element offset of row dk of the block
+}
+
 // Support predicates (bf16 inputs assumed).
 bool tc_states_supported(const Problem& p);
 bool tc_parallel_supported(const Problem& p);
@@ -23,8 +34,10 @@ cudaError_t launch_tc_parallel(const Problem& p, const void* Q, const void* K, c
                                Gates g, const __nv_bfloat16* Cb, const float* n_states, void* H,
                                float* n_out, float* m_out, cudaStream_t st);
 
-// fp32 -> bf16 copy of caller-provided chunk states (n elements).
-cudaError_t launch_states_to_bf16(const float* src, __nv_bfloat16* dst, size_t n, cudaStream_t st);
+// Caller-provided fp32 chunk states [BH * NC][DK][DV] -> the bf16 operand copy
+// in the swizzled block layout above (DV a multiple of 64).
+cudaError_t launch_states_to_operand(const float* src, __nv_bfloat16* dst, long n_bhk, int DK,
+                                     int DV, cudaStream_t st);
 
 // Fused kernel: chunk state carried on chip; H and the final state.
 cudaError_t launch_tc_fused(const Problem& p, const void* Q, const void* K, const void* V,

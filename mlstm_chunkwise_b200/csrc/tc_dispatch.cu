@@ -27,12 +27,24 @@ PFN_cuTensorMapEncodeTiled_v12000 encoder() {
   return g_encode;
 }
 
-__global__ void states_to_bf16_kernel(const float4* __restrict__ src, uint2* __restrict__ dst,
-                                      size_t n4) {
-  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n4;
+// One thread per 16-byte chunk (8 values) of the destination: reads 8
+// consecutive fp32 values of a state row and writes them as one bf16 chunk at
+// its swizzled position.
+__global__ void states_to_operand_kernel(const float4* __restrict__ src, uint4* __restrict__ dst,
+                                         long n_bhk, int DK, int DV) {
+  const int n_vb = DV / 64;
+  const size_t n_chunks = (size_t)n_bhk * DK * (DV / 8);
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n_chunks;
        i += (size_t)gridDim.x * blockDim.x) {
-    const float4 v = src[i];
-    dst[i] = make_uint2(tc::pack_bf16x2(v.x, v.y), tc::pack_bf16x2(v.z, v.w));
+    const int cj = (int)(i % (DV / 8));  // 8-column chunk of the state row
+    const size_t row = i / (DV / 8);      // bhk * DK + dk
+    const int dk = (int)(row % DK);
+    const long bhk = (long)(row / DK);
+    const float4 a = src[2 * i], b = src[2 * i + 1];
+    const int vb = cj >> 3, j = cj & 7;
+    uint4 v = make_uint4(tc::pack_bf16x2(a.x, a.y), tc::pack_bf16x2(a.z, a.w),
+                         tc::pack_bf16x2(b.x, b.y), tc::pack_bf16x2(b.z, b.w));
+    dst[cb_block_row(bhk, vb, dk, DK, n_vb) / 8 + (j ^ (dk & 7))] = v;
   }
 }
 
@@ -67,7 +79,9 @@ bool encode_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64
 }
 
 bool tc_unfused_supported(const Problem& p) {
-  return tc_states_supported(p) && tc_parallel_supported(p);
+  // The chunk-state kernel writes the operand copy in 64-column blocks, one
+  // warp per 32 x 64 tile, which needs at least 128 value columns per CTA.
+  return tc_states_supported(p) && tc_parallel_supported(p) && p.DV % 128 == 0;
 }
 
 bool tc_fused_supported(const Problem&) { return false; }
@@ -90,13 +104,15 @@ cudaError_t launch_tc_parallel(const Problem& p, const void* Q, const void* K, c
   return launch_tc_parallel_bf16states(p, Q, K, V, g, Cb, n_states, H, n_out, m_out, st);
 }
 
-cudaError_t launch_states_to_bf16(const float* src, __nv_bfloat16* dst, size_t n,
-                                  cudaStream_t st) {
-  const size_t n4 = n / 4;  // DK * DV is a multiple of 4 for every supported shape
-  if (n4 == 0) return cudaSuccess;
-  const int blocks = (int)((n4 + 255) / 256 < 148 * 16 ? (n4 + 255) / 256 : 148 * 16);
-  states_to_bf16_kernel<<<blocks, 256, 0, st>>>(reinterpret_cast<const float4*>(src),
-                                                reinterpret_cast<uint2*>(dst), n4);
+cudaError_t launch_states_to_operand(const float* src, __nv_bfloat16* dst, long n_bhk, int DK,
+                                     int DV, cudaStream_t st) {
+  if (DV % 64 != 0) return cudaErrorNotSupported;
+  const size_t n_chunks = (size_t)n_bhk * DK * (DV / 8);
+  if (n_chunks == 0) return cudaSuccess;
+  const size_t want = (n_chunks + 255) / 256;
+  const int blocks = (int)(want < 148 * 16 ? want : 148 * 16);
+  states_to_operand_kernel<<<blocks, 256, 0, st>>>(reinterpret_cast<const float4*>(src),
+                                                   reinterpret_cast<uint4*>(dst), n_bhk, DK, DV);
   return cudaGetLastError();
 }
 

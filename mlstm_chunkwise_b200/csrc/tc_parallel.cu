@@ -121,7 +121,7 @@ __device__ __forceinline__ Item decode_item(int it, const Problem& p, int n_dv, 
 template <int DK, int DVT>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_parallel_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_c,
+                   const __grid_constant__ CUtensorMap tm_v, const __nv_bfloat16* __restrict__ Cb,
                    Problem p, Gates g, const float* __restrict__ n_states,
                    __nv_bfloat16* __restrict__ H, float* __restrict__ n_out,
                    float* __restrict__ m_out, int n_items) {
@@ -176,7 +176,6 @@ tc_parallel_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
-      tma_prefetch_desc(&tm_c);
       int slab = 0;
       bool ok = true;
       auto next_stage = [&](uint32_t bytes) -> uint32_t {
@@ -215,9 +214,11 @@ tc_parallel_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         load_k(0);
         for (int c = 0; c < C::kSlabsK && ok; ++c) {
           const uint32_t s = next_stage(C::kMNSlabBytes);
-          for (int b = 0; b < DVT / 64; ++b)
-            tma_load_3d(sbase + C::kOffStage + s * C::kStageBytes + b * 8192, &tm_c, x.dv0 + b * 64,
-                        c * 64, x.bh * p.NC + x.k, bar.full(s));
+          for (int b = 0; b < DVT / 64; ++b)  // C_k rows [64c, 64c + 64) of block dv0 / 64 + b
+            bulk_load(sbase + C::kOffStage + s * C::kStageBytes + b * 8192,
+                      Cb + cb_block_row((long)x.bh * p.NC + x.k, x.dv0 / 64 + b, c * 64, DK,
+                                        p.DV / 64),
+                      8192, bar.full(s));
         }
         for (int i = 1; i < x.n_kv && ok; ++i) {
           load_k(i);
@@ -517,11 +518,10 @@ cudaError_t launch_parallel_t(const Problem& p, const void* Q, const void* K, co
                               Gates g, const __nv_bfloat16* Cb, const float* n_states, void* H,
                               float* n_out, float* m_out, cudaStream_t st) {
   using C = Cfg<DK, DVT>;
-  CUtensorMap tq, tk, tv, tcm;
+  CUtensorMap tq, tk, tv;
   if (!encode_tmap_bf16_3d(&tq, Q, p.DK, p.T, p.BH, 64, kQT) ||
       !encode_tmap_bf16_3d(&tk, K, p.DK, p.T, p.BH, 64, kKT) ||
-      !encode_tmap_bf16_3d(&tv, V, p.DV, p.T, p.BH, 64, 64) ||
-      !encode_tmap_bf16_3d(&tcm, Cb, p.DV, p.DK, (uint64_t)p.BH * p.NC, 64, 64))
+      !encode_tmap_bf16_3d(&tv, V, p.DV, p.T, p.BH, 64, 64))
     return cudaErrorInvalidValue;
   auto kern = tc_parallel_kernel<DK, DVT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
@@ -534,7 +534,7 @@ cudaError_t launch_parallel_t(const Problem& p, const void* Q, const void* K, co
   const long items = (long)p.BH * ((p.T + kQT - 1) / kQT) * (p.DV / DVT);
   if (items > (1L << 30)) return cudaErrorInvalidValue;
   const int grid = (int)(items < sms ? items : sms);
-  kern<<<grid, kThreads, C::kSmem, st>>>(tq, tk, tv, tcm, p, g, n_states,
+  kern<<<grid, kThreads, C::kSmem, st>>>(tq, tk, tv, Cb, p, g, n_states,
                                          static_cast<__nv_bfloat16*>(H), n_out, m_out, (int)items);
   return cudaGetLastError();
 }

@@ -122,7 +122,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 tc_parallel_wide_kernel(const __grid_constant__ CUtensorMap tm_q,
                         const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v,
-                        const __grid_constant__ CUtensorMap tm_c,
+                        const __nv_bfloat16* __restrict__ Cb,
                         const __grid_constant__ CUtensorMap tm_h, Problem p, Gates g,
                         const float* __restrict__ n_states,
                         float* __restrict__ n_out, float* __restrict__ m_out, int n_items) {
@@ -175,7 +175,6 @@ tc_parallel_wide_kernel(const __grid_constant__ CUtensorMap tm_q,
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
-      tma_prefetch_desc(&tm_c);
       int slab = 0;
       bool ok = true;
       auto next_stage = [&](uint32_t bytes) -> uint32_t {
@@ -208,11 +207,13 @@ tc_parallel_wide_kernel(const __grid_constant__ CUtensorMap tm_q,
                 tma_load_3d(dst + b * 8192, &tm_v, dv0 + b * 64, x.c0 + i * kKT + v * 64, x.bh,
                             bar.full((slab - 1) % C::kStages));
             }
-          for (int c = 0; c < C::kSlabsK && ok; ++c) {
+          for (int c = 0; c < C::kSlabsK && ok; ++c) {  // C_k rows [64c, 64c + 64)
             const uint32_t dst = next_stage(C::kMNSlabBytes);
             for (int b = 0; b < DVT / 64; ++b)
-              tma_load_3d(dst + b * 8192, &tm_c, dv0 + b * 64, c * 64, x.bh * p.NC + x.k,
-                          bar.full((slab - 1) % C::kStages));
+              bulk_load(dst + b * 8192,
+                        Cb + cb_block_row((long)x.bh * p.NC + x.k, dv0 / 64 + b, c * 64, DK,
+                                          p.DV / 64),
+                        8192, bar.full((slab - 1) % C::kStages));
           }
         }
       }
@@ -502,11 +503,10 @@ cudaError_t launch_wide_t(const Problem& p, const void* Q, const void* K, const 
                           const __nv_bfloat16* Cb, const float* n_states, void* H, float* n_out,
                           float* m_out, cudaStream_t st) {
   using C = WCfg<DK, DVT>;
-  CUtensorMap tq, tk, tv, tcm, th;
+  CUtensorMap tq, tk, tv, th;
   if (!encode_tmap_bf16_3d(&tq, Q, p.DK, p.T, p.BH, 64, kQT) ||
       !encode_tmap_bf16_3d(&tk, K, p.DK, p.T, p.BH, 64, kKT) ||
       !encode_tmap_bf16_3d(&tv, V, p.DV, p.T, p.BH, 64, 64) ||
-      !encode_tmap_bf16_3d(&tcm, Cb, p.DV, p.DK, (uint64_t)p.BH * p.NC, 64, 64) ||
       !encode_tmap_bf16_3d(&th, H, p.DV, p.T, p.BH, 64, kQT))
     return cudaErrorInvalidValue;
   auto kern = tc_parallel_wide_kernel<DK, DVT>;
@@ -520,7 +520,7 @@ cudaError_t launch_wide_t(const Problem& p, const void* Q, const void* K, const 
   const long items = (long)p.BH * ((p.T + kQT - 1) / kQT);
   if (items > (1L << 30)) return cudaErrorInvalidValue;
   const int grid = (int)(items < sms ? items : sms);
-  kern<<<grid, kThreads, C::kSmem, st>>>(tq, tk, tv, tcm, th, p, g, n_states, n_out, m_out,
+  kern<<<grid, kThreads, C::kSmem, st>>>(tq, tk, tv, Cb, th, p, g, n_states, n_out, m_out,
                                          (int)items);
   return cudaGetLastError();
 }

@@ -21,10 +21,12 @@
 // scattered stores, not the MMAs, would then set the pace of the recurrence.
 //
 // Roles (320 threads): warp 0 TMA producer, warp 1 TMEM owner + MMA issuer,
-// warps 2..9 workers: per chunk, the token weights and the store and decay of
-// the master state; per stage, one pass that accumulates the n-vector partial
-// sums (fp32, from the unrounded products w_s k_s) and weights the K rows in
-// place.
+// warps 2..9 workers: per chunk, the store and decay of the master state; per
+// stage, one pass that computes its token weights, accumulates the n-vector
+// partial sums (fp32, from the unrounded products w_s k_s) and weights the K
+// rows in place.  The first stage of chunk k is weighted before the workers
+// wait for chunk k - 1's MMAs to drain, so that work leaves the critical path;
+// the n-vector needs no MMA and is carried by the workers alone.
 #include <cuda.h>
 
 #include <cstring>
@@ -49,20 +51,19 @@ struct SCfg {
   static constexpr uint32_t kKBytes = kStageTok * DK * 2;   // DK/64 boxes of [64 tok x 64 dk]
   static constexpr uint32_t kVBytes = kStageTok * DVT * 2;  // DVT/64 boxes of [64 tok x 64 dv]
   static constexpr uint32_t kStageBytes = kKBytes + kVBytes;
-  static constexpr int kMaxL = 1024;
   static constexpr int kCC = DK / 8;             // 16-byte column chunks per token row
   static constexpr int kRowsPer = kStageTok * kCC / 256;  // rows per worker per stage
-  static constexpr uint32_t kWBytes = kMaxL * 4;           // token weights of one chunk
   static constexpr uint32_t kRedBytes = (256 / kCC) * DK * 4;  // n partials [row group][dk]
-  static constexpr uint32_t kStgBytes = 8 * 2048;  // one 32 x 64-byte store tile per worker warp
-  static constexpr uint32_t kBudget = 227 * 1024 - 1024 - 512 - kWBytes - kRedBytes - kStgBytes;
+  // Two 32 x 64-byte store tiles per worker warp; the n-partial exchange
+  // reuses the same bytes (it never overlaps a state store).
+  static constexpr uint32_t kStgBytes = 8 * 2 * 2048;
+  static_assert(kRedBytes <= kStgBytes, "n partials must fit in the store tiles");
+  static constexpr uint32_t kBudget = 227 * 1024 - 1024 - 512 - kStgBytes;
   static constexpr int kStagesFit = (int)(kBudget / kStageBytes);
   static constexpr int kStages = kStagesFit > 8 ? 8 : kStagesFit;
   static_assert(kStages >= 2, "ring too shallow");
   static constexpr uint32_t kOffStage = 0;
-  static constexpr uint32_t kOffW = kStages * kStageBytes;  // float[kMaxL]
-  static constexpr uint32_t kOffRed = kOffW + kWBytes;      // float[256 / kCC][DK]
-  static constexpr uint32_t kOffStg = kOffRed + kRedBytes;  // [8 warps][32 rows][64 B], 64 B swizzle
+  static constexpr uint32_t kOffStg = kStages * kStageBytes;  // [8 warps][2][32 rows][64 B], 64 B swizzle
   static_assert(kOffStg % 1024 == 0, "store tiles must sit on a swizzle-atom boundary");
   static constexpr uint32_t kOffBar = kOffStg + kStgBytes;
   static constexpr uint32_t kOffSlot = kOffBar + 8 * 32;
@@ -85,8 +86,7 @@ struct SBars {
 template <int DK, int DVT>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_states_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                 const __grid_constant__ CUtensorMap tm_cs, const __grid_constant__ CUtensorMap tm_cb,
-                 Problem p, Gates g, const float* __restrict__ C0, const float* __restrict__ n0,
+                 const __grid_constant__ CUtensorMap tm_cs, Problem p, Gates g, const float* __restrict__ C0, const float* __restrict__ n0,
                  float* __restrict__ C_states, __nv_bfloat16* __restrict__ Cb,
                  float* __restrict__ n_states, float* __restrict__ C_T, float* __restrict__ n_T,
                  float* __restrict__ m_T) {
@@ -97,12 +97,11 @@ tc_states_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
   const uint32_t sbase = smem_u32(smem);
   const SBars bar{sbase + S::kOffBar};
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + S::kOffSlot);
-  float* w_s = reinterpret_cast<float*>(smem + S::kOffW);
-  float* red_s = reinterpret_cast<float*>(smem + S::kOffRed);
+  float* red_s = reinterpret_cast<float*>(smem + S::kOffStg);  // aliases the store tiles
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int dv0 = blockIdx.x * DVT, bh = blockIdx.y;
-  const int L = p.L, NC = p.NC, T = p.T, DV = p.DV;
+  const int L = p.L, NC = p.NC, DV = p.DV;
   const int stages_per_chunk = L / kStageTok;
   const long tpad = (long)NC * L;
   const bool n_owner = blockIdx.x == 0;
@@ -190,8 +189,11 @@ tc_states_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
     constexpr int kColsPer = DVT / 2;  // value columns per worker in the state passes
     const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16);
     const float* mchk = g.mchk + (long)bh * (NC + 1);
-    uint8_t* stg = smem + S::kOffStg + (warp - 2) * 2048;  // this warp's store tile
-    const uint32_t stg_u = sbase + S::kOffStg + (uint32_t)(warp - 2) * 2048u;
+    const float* acol = g.acol + (long)bh * tpad;  // -inf on padding: weight 0
+    // this warp's two store tiles
+    uint8_t* stg = smem + S::kOffStg + (warp - 2) * 4096;
+    const uint32_t stg_u = sbase + S::kOffStg + (uint32_t)(warp - 2) * 4096u;
+    int n_st = 0;  // state stores issued by this warp (selects the tile)
     // n-vector: worker wt owns dk column wt (DK <= 256) for the running n.
     const bool n_mine = n_owner && wt < DK;
     float nval = (n_mine && n0) ? n0[(long)bh * DK + wt] : 0.f;
@@ -216,147 +218,178 @@ tc_states_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
     }
     tmem_wait_st();
 
-    // Column weights of the first chunk, prefetched (<= 4 per worker).
-    float acol_next[S::kMaxL / 256];
+    // Adds this chunk's n partials into the running n (all workers take part).
+    // red_s spans several warps' store tiles, so every warp's stores must have
+    // read them first (n_owner is uniform over the CTA, so are the barriers).
+    auto fold_n = [&]() {
+      if (n_owner) {
+        if (lane == 0) tma_store_wait_read_all();
+        named_bar_sync(1, kWorkers);
 #pragma unroll
-    for (int i = 0; i < S::kMaxL / 256; ++i) {
-      const int j = wt + 256 * i;
-      acol_next[i] = (j < L && j < T) ? g.acol[(long)bh * tpad + j] : -INFINITY;
-    }
-
-    int n = 0;
-    for (int k = 0; k < NC && ok; ++k) {
-      if (k > 0) {
-        ok = mbar_wait(bar.chunk(), (k - 1) & 1, p, 4);
-        tc_fence_after();
-        if (n_owner) {
-          // fold the previous chunk's n partials into the running n
-#pragma unroll
-          for (int e = 0; e < 8; ++e) red_s[rg * DK + cc * 8 + e] = part[e];
-        }
+        for (int e = 0; e < 8; ++e) red_s[rg * DK + cc * 8 + e] = part[e];
         named_bar_sync(1, kWorkers);
         if (n_mine) {
           float acc = 0.f;
           for (int q2 = 0; q2 < 256 / S::kCC; ++q2) acc += red_s[q2 * DK + wt];
           nval += acc;
         }
-#pragma unroll
-        for (int e = 0; e < 8; ++e) part[e] = 0.f;
       }
+#pragma unroll
+      for (int e = 0; e < 8; ++e) part[e] = 0.f;
+    };
+
+    // Column weights of this worker's rows, one stage ahead.
+    constexpr int kRP = S::kRowsPer;
+    static_assert(kRP % 4 == 0, "rows per worker in float4 groups");
+    float4 a_nxt[kRP / 4];
+    auto load_acol = [&](int stage_idx) {
+#pragma unroll
+      for (int i = 0; i < kRP / 4; ++i)
+        a_nxt[i] = *reinterpret_cast<const float4*>(acol + (long)stage_idx * kStageTok +
+                                                    rg * kRP + 4 * i);
+    };
+    load_acol(0);
+
+    // One pass over ring stage n: weights w = s e^{g_k + acol - m_{k+1}} of its
+    // rows, the n partials from the unrounded products w k (the normaliser
+    // enters h through |n^T q|, which can cancel, so it must not see the bf16
+    // rounding), and the K rows weighted in place for the rank-64 update.
+    auto stage_pass = [&](int n, float gk, float m_out) {
+      const int s = n % S::kStages;
+      float a_cur[kRP];
+#pragma unroll
+      for (int i = 0; i < kRP / 4; ++i) {
+        a_cur[4 * i] = a_nxt[i].x;
+        a_cur[4 * i + 1] = a_nxt[i].y;
+        a_cur[4 * i + 2] = a_nxt[i].z;
+        a_cur[4 * i + 3] = a_nxt[i].w;
+      }
+      if (n + 1 < NC * stages_per_chunk) load_acol(n + 1);
+      ok = ok && mbar_wait(bar.full(s), (n / S::kStages) & 1, p, 5);
+      uint8_t* box = smem + S::kOffStage + (uint32_t)s * S::kStageBytes + (cc >> 3) * 8192;
+#pragma unroll
+      for (int rr = 0; rr < kRP; ++rr) {
+        const int row = rg * kRP + rr;
+        const float w = p.key_scale * expf(gk + a_cur[rr] - m_out);  // -inf -> 0
+        uint4* ptr = reinterpret_cast<uint4*>(box + sw128_offset(row, cc & 7));
+        uint4 u = *ptr;
+        __nv_bfloat162* h2 = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __bfloat1622float2(h2[e]);
+          part[2 * e] = fmaf(f.x, w, part[2 * e]);
+          part[2 * e + 1] = fmaf(f.y, w, part[2 * e + 1]);
+          h2[e] = __floats2bfloat162_rn(f.x * w, f.y * w);
+        }
+        *ptr = u;
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(bar.kready(s));
+    };
+
+    // Packs 16 words into this warp's next store tile and stores it with TMA
+    // at (x, y, z) of `map`; the tile used two stores ago must have been read.
+    auto store_tile = [&](const CUtensorMap* map, const uint32_t (&w16)[16], int x, int y, int z) {
+      const uint32_t t = (uint32_t)(n_st & 1) * 2048u;
+      if (lane == 0) tma_store_wait_read_1();
+      __syncwarp();
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        *reinterpret_cast<uint4*>(stg + t + sw64_offset(lane, j)) =
+            make_uint4(w16[4 * j], w16[4 * j + 1], w16[4 * j + 2], w16[4 * j + 3]);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        tma_store_3d(map, stg_u + t, x, y, z);
+        tma_store_commit();
+      }
+      ++n_st;
+    };
+
+    int n = 0;
+    for (int k = 0; k < NC && ok; ++k) {
+      if (k > 0) fold_n();  // chunk k - 1's partials: every worker has passed its stages
       const float m_in = mchk[k], m_out = mchk[k + 1];
       const float gk = g.gtot[(long)bh * NC + k];
       const float decay = expf(gk + m_in - m_out);
-      // state entering chunk k: store (TMA, from this warp's tile), then decay in place
-      for (int hf = 0; hf < S::kHalves && ok; ++hf) {
-        const int dk0 = hf * 128 + q * 32;  // first state row of this warp's lanes
-        for (int c = 0; c < kColsPer; c += 32) {
-          const int col = ch * kColsPer + c;
-          uint32_t v[32];
-          tmem_ld32(trow + hf * DVT + col, v);
-          tmem_wait_ld();
-          if (C_states) {  // fp32: two 16-column boxes
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-              if (lane == 0) tma_store_wait_read_all();
-              __syncwarp();
+      if (n_mine) n_states[((long)bh * NC + k) * DK + wt] = nval;
+      nval *= decay;
+
+      // The first stage of chunk k needs nothing from the MMAs.
+      stage_pass(n++, gk, m_out);
+      if (k > 0) {
+        ok = ok && mbar_wait(bar.chunk(), (k - 1) & 1, p, 4);
+        tc_fence_after();
+      }
+      named_bar_sync(1, kWorkers);  // the n-partial reads are done: store tiles free
+
+      // state entering chunk k: store (from this warp's tiles), then decay in place
+      if (Cb) {
+        // bf16 operand copy: one 32-row x 64-column tile per warp, already in
+        // the swizzled block layout, leaves with one 4 KB bulk store.
+        for (int hf = 0; hf < S::kHalves && ok; ++hf) {
+          const int dk0 = hf * 128 + q * 32;  // first state row of this warp's lanes
+          for (int c = 0; c < kColsPer; c += 64) {
+            const int col = ch * kColsPer + c;
+            if (lane == 0) tma_store_wait_read_all();  // the previous tile has been read
+            __syncwarp();
+#pragma unroll 1
+            for (int hh = 0; hh < 2; ++hh) {
+              uint32_t v[32];
+              tmem_ld32(trow + hf * DVT + col + 32 * hh, v);
+              tmem_wait_ld();
 #pragma unroll
               for (int j = 0; j < 4; ++j)
-                *reinterpret_cast<uint4*>(stg + sw64_offset(lane, j)) =
-                    make_uint4(v[16 * half + 4 * j], v[16 * half + 4 * j + 1],
-                               v[16 * half + 4 * j + 2], v[16 * half + 4 * j + 3]);
-              fence_proxy_async_smem();
-              __syncwarp();
-              if (lane == 0) {
-                tma_store_3d(&tm_cs, stg_u, dv0 + col + 16 * half, dk0, bh * NC + k);
-                tma_store_commit();
-              }
-            }
-          }
-          if (Cb) {
-            if (lane == 0) tma_store_wait_read_all();
-            __syncwarp();
+                *reinterpret_cast<uint4*>(stg + lane * 128 + (((4 * hh + j) ^ (lane & 7)) << 4)) =
+                    make_uint4(
+                        pack_bf16x2(__uint_as_float(v[8 * j]), __uint_as_float(v[8 * j + 1])),
+                        pack_bf16x2(__uint_as_float(v[8 * j + 2]), __uint_as_float(v[8 * j + 3])),
+                        pack_bf16x2(__uint_as_float(v[8 * j + 4]), __uint_as_float(v[8 * j + 5])),
+                        pack_bf16x2(__uint_as_float(v[8 * j + 6]), __uint_as_float(v[8 * j + 7])));
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-              *reinterpret_cast<uint4*>(stg + sw64_offset(lane, j)) = make_uint4(
-                  pack_bf16x2(__uint_as_float(v[8 * j]), __uint_as_float(v[8 * j + 1])),
-                  pack_bf16x2(__uint_as_float(v[8 * j + 2]), __uint_as_float(v[8 * j + 3])),
-                  pack_bf16x2(__uint_as_float(v[8 * j + 4]), __uint_as_float(v[8 * j + 5])),
-                  pack_bf16x2(__uint_as_float(v[8 * j + 6]), __uint_as_float(v[8 * j + 7])));
+              for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * decay);
+              tmem_st32(trow + hf * DVT + col + 32 * hh, v);
+            }
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
-              tma_store_3d(&tm_cb, stg_u, dv0 + col, dk0, bh * NC + k);
+              bulk_store(Cb + cb_block_row((long)bh * NC + k, (dv0 + col) / 64, dk0, DK, DV / 64),
+                         stg_u, 4096);
               tma_store_commit();
             }
           }
+        }
+      } else {
+        // fp32 states (or none): 16-column tiles through the tensor map
+        for (int hf = 0; hf < S::kHalves && ok; ++hf) {
+          const int dk0 = hf * 128 + q * 32;
+          for (int c = 0; c < kColsPer; c += 32) {
+            const int col = ch * kColsPer + c;
+            uint32_t v[32];
+            tmem_ld32(trow + hf * DVT + col, v);
+            tmem_wait_ld();
+            if (C_states) {
+              store_tile(&tm_cs, *reinterpret_cast<const uint32_t(*)[16]>(v), dv0 + col, dk0,
+                         bh * NC + k);
+              store_tile(&tm_cs, *reinterpret_cast<const uint32_t(*)[16]>(v + 16), dv0 + col + 16,
+                         dk0, bh * NC + k);
+            }
 #pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * decay);
-          tmem_st32(trow + hf * DVT + col, v);
+            for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * decay);
+            tmem_st32(trow + hf * DVT + col, v);
+          }
         }
       }
       tmem_wait_st();
-      if (n_mine) n_states[((long)bh * NC + k) * DK + wt] = nval;
-      nval *= decay;
       tc_fence_before();
       mbar_arrive(bar.master());
 
-      // Token weights of chunk k (from the prefetched column weights), then
-      // prefetch chunk k + 1's.
-#pragma unroll
-      for (int i = 0; i < S::kMaxL / 256; ++i) {
-        const int j = wt + 256 * i;
-        if (j < L) w_s[j] = p.key_scale * expf(gk + acol_next[i] - m_out);  // -inf -> 0
-      }
-#pragma unroll
-      for (int i = 0; i < S::kMaxL / 256; ++i) {
-        const int j = wt + 256 * i;
-        const long t = (long)(k + 1) * L + j;
-        acol_next[i] = (k + 1 < NC && j < L && t < T) ? g.acol[(long)bh * tpad + t] : -INFINITY;
-      }
-      named_bar_sync(1, kWorkers);
-
-      for (int j = 0; j < stages_per_chunk && ok; ++j, ++n) {
-        const int s = n % S::kStages;
-        ok = mbar_wait(bar.full(s), (n / S::kStages) & 1, p, 5);
-        uint8_t* box = smem + S::kOffStage + (uint32_t)s * S::kStageBytes + (cc >> 3) * 8192;
-        const float* ws = w_s + j * kStageTok;
-        // One pass: accumulate the unrounded products w_s k_s into the n
-        // partials (the normaliser enters h through |n^T q|, which can cancel,
-        // so it must not see the bf16 rounding), and weight the K rows in
-        // place for the rank-64 update.
-#pragma unroll
-        for (int rr = 0; rr < S::kRowsPer; ++rr) {
-          const int row = rg * S::kRowsPer + rr;
-          const float w = ws[row];
-          uint4* ptr = reinterpret_cast<uint4*>(box + sw128_offset(row, cc & 7));
-          uint4 u = *ptr;
-          __nv_bfloat162* h2 = reinterpret_cast<__nv_bfloat162*>(&u);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 f = __bfloat1622float2(h2[e]);
-            part[2 * e] = fmaf(f.x, w, part[2 * e]);
-            part[2 * e + 1] = fmaf(f.y, w, part[2 * e + 1]);
-            h2[e] = __floats2bfloat162_rn(f.x * w, f.y * w);
-          }
-          *ptr = u;
-        }
-        fence_proxy_async_smem();
-        mbar_arrive(bar.kready(s));
-      }
+      for (int j = 1; j < stages_per_chunk && ok; ++j) stage_pass(n++, gk, m_out);
     }
     // final state (fold the last chunk's n partials first)
     if (ok) ok = mbar_wait(bar.chunk(), (NC - 1) & 1, p, 6);
     tc_fence_after();
-    if (n_owner) {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) red_s[rg * DK + cc * 8 + e] = part[e];
-    }
-    named_bar_sync(1, kWorkers);
-    if (n_mine) {
-      float acc = 0.f;
-      for (int q2 = 0; q2 < 256 / S::kCC; ++q2) acc += red_s[q2 * DK + wt];
-      nval += acc;
-    }
+    fold_n();
     if (ok && C_T) {
       for (int hf = 0; hf < S::kHalves; ++hf) {
         const int dk = hf * 128 + r;
@@ -393,21 +426,23 @@ cudaError_t launch_states_t(const Problem& p, const void* K, const void* V, cons
                             const float* n0, Gates g, float* C_states, __nv_bfloat16* Cb,
                             float* n_states, float* C_T, float* n_T, float* m_T, cudaStream_t st) {
   using S = SCfg<DK, DVT>;
-  CUtensorMap tk, tv, tcs, tcb;
+  CUtensorMap tk, tv, tcs;
   memset(&tcs, 0, sizeof(tcs));
-  memset(&tcb, 0, sizeof(tcb));
+  // One of the two state copies per launch (they share the store tiles); the
+  // operand copy is written in 64-column tiles, two per worker row at least.
+  if (C_states && Cb) return cudaErrorInvalidValue;
+  if (Cb && (DVT < 128 || p.DV % 64 != 0)) return cudaErrorNotSupported;
   const uint64_t n_boxes = (uint64_t)p.BH * p.NC;  // state tiles [DK][DV] per (b, h, chunk)
   if (!encode_tmap_bf16_3d(&tk, K, p.DK, p.T, p.BH, 64, kStageTok) ||
       !encode_tmap_bf16_3d(&tv, V, p.DV, p.T, p.BH, 64, kStageTok) ||
-      (C_states && !encode_tmap_3d(&tcs, C_states, 4, p.DV, p.DK, n_boxes, 16, 32, 64)) ||
-      (Cb && !encode_tmap_3d(&tcb, Cb, 2, p.DV, p.DK, n_boxes, 32, 32, 64)))
+      (C_states && !encode_tmap_3d(&tcs, C_states, 4, p.DV, p.DK, n_boxes, 16, 32, 64)))
     return cudaErrorInvalidValue;
   auto kern = tc_states_kernel<DK, DVT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kSmem);
   if (e != cudaSuccess) return e;
   dim3 grid(p.DV / DVT, p.BH);
-  kern<<<grid, kThreads, S::kSmem, st>>>(tk, tv, tcs, tcb, p, g, C0, n0, C_states, Cb, n_states,
-                                         C_T, n_T, m_T);
+  kern<<<grid, kThreads, S::kSmem, st>>>(tk, tv, tcs, p, g, C0, n0, C_states, Cb, n_states, C_T,
+                                         n_T, m_T);
   return cudaGetLastError();
 }
 
