@@ -117,6 +117,18 @@ __device__ __forceinline__ WItem decode_witem(int it, const Problem& p, int n_q)
   return x;
 }
 
+// The k-th item of this CTA.  Items alternate between the first and the
+// second query tile of a chunk, and the second has twice the intra-chunk work;
+// a plain stride of an even grid would give each CTA only one kind (and the
+// kernel the time of the slower half).  With an even grid the lowest index bit
+// is therefore flipped on odd rounds: every CTA takes both kinds, and the two
+// tiles of a chunk still run side by side in neighbouring CTAs (their C_k and
+// V tiles are shared through L2).
+__device__ __forceinline__ int item_at(int k) {
+  const int G = (int)gridDim.x, c = (int)blockIdx.x;
+  return k * G + ((G & 1) ? c : (c ^ (k & 1)));
+}
+
 template <int DK, int DVT>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_parallel_wide_kernel(const __grid_constant__ CUtensorMap tm_q,
@@ -185,7 +197,7 @@ tc_parallel_wide_kernel(const __grid_constant__ CUtensorMap tm_q,
         return sbase + C::kOffStage + (uint32_t)s * C::kStageBytes;
       };
       int n = 0;
-      for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++n) {
+      for (int it = item_at(0); it < n_items && ok; it = item_at(n + 1), ++n) {
         const WItem x = decode_witem(it, p, n_q);
         if (n > 0) ok = mbar_wait(bar.q_empty(), (n - 1) & 1, p, 2);
         if (!ok) break;
@@ -237,7 +249,7 @@ tc_parallel_wide_kernel(const __grid_constant__ CUtensorMap tm_q,
         return (uint32_t)s;
       };
       int n = 0;
-      for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++n) {
+      for (int it = item_at(0); it < n_items && ok; it = item_at(n + 1), ++n) {
         const WItem x = decode_witem(it, p, n_q);
         ok = mbar_wait(bar.q_full(), n & 1, p, 3);
         for (int i = 0; i < x.n_kv && ok; ++i) {  // S_i
@@ -337,7 +349,7 @@ tc_parallel_wide_kernel(const __grid_constant__ CUtensorMap tm_q,
       fetch_cols(x0, 0);
     }
     int n = 0;
-    for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++n) {
+    for (int it = item_at(0); it < n_items && ok; it = item_at(n + 1), ++n) {
       const WItem x = decode_witem(it, p, n_q);
       const int t = x.t0 + r;
       const float m_in = nx_m_in, amax = nx_amax, bc = nx_bc;
@@ -424,7 +436,7 @@ tc_parallel_wide_kernel(const __grid_constant__ CUtensorMap tm_q,
       mbar_arrive(bar.q_scaled());
 
       // The next item's row values and column data (other buffer).
-      const int it_next = it + gridDim.x;
+      const int it_next = item_at(n + 1);
       if (it_next < n_items) {
         const WItem xn = decode_witem(it_next, p, n_q);
         fetch_rows(xn, nx_m_in, nx_amax, nx_bc);
