@@ -41,6 +41,28 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 SIMT_LANES = 148 * 128
 
 
+def rank_seed(w, rank):
+    """Every rank draws its own batch of the same workload shape."""
+    return w.seed + rank
+
+
+def max_over_ranks(value, device, world):
+    """The largest per-rank value over all ranks (the slowest rank times the
+    job).  Every rank must call it, in the same order."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(tokens_per_rank_step, world, ms_per_step):
+    """Whole-job tokens/s: all ranks' tokens over the max-over-ranks step time."""
+    return tokens_per_rank_step * world / (ms_per_step / 1e3)
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -372,7 +394,7 @@ def run_ours(args):
     w = pick_workload(args.workload)
     if args.batch:
         w = w.replace(name=f"{w.name}_B{args.batch}", B=args.batch)
-    x = make_inputs(w, seed=w.seed + rank)
+    x = make_inputs(w, seed=rank_seed(w, rank))
     d = {k: (None if v is None else v.to(dev)) for k, v in x.items()}
     B, NH, T, DK, DV, L = w.B, w.NH, w.T, w.DK, w.DV, w.chunk_size
     elem = 2 if w.dtype == "bf16" else 4
@@ -429,10 +451,7 @@ def run_ours(args):
     sampler.stop()
     clocks = sampler.summary(t_host0, t_host1)
 
-    if world > 1:
-        t = torch.tensor([elapsed_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    elapsed_ms = max_over_ranks(elapsed_ms, dev, world)
 
     # --- e2e: pinned host inputs -> device -> mlstm_fw -> host outputs -------
     hx = {k: (None if v is None else v.pin_memory()) for k, v in x.items()}
@@ -461,15 +480,12 @@ def run_ours(args):
         e1.record(stream)
         torch.cuda.synchronize()
         e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e2e_ms, dev, world)
 
     tokens_per_step = B * T * world
     ms_per_step = elapsed_ms / args.steps
-    value = tokens_per_step / (ms_per_step / 1e3)
-    e2e_value = None if args.no_e2e else tokens_per_step * e2e_steps / (e2e_ms / 1e3)
+    value = job_throughput(B * T, world, ms_per_step)
+    e2e_value = None if args.no_e2e else job_throughput(B * T, world, e2e_ms / e2e_steps)
 
     # --- roofline of the dominant kernel ------------------------------------
     peaks, peak_src = load_peaks()

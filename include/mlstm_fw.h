@@ -150,6 +150,18 @@ uint32_t mlstm_last_device_error_word(void);
  * default.  Not thread-safe with concurrent launches. */
 void mlstm_set_watchdog(uint64_t max_polls);
 
+/* Failure-detection self-test.  Enqueues on `stream` one tiny kernel whose
+ * only waiting thread waits on an mbarrier that nothing ever completes,
+ * through the same bounded wait that every kernel of the library uses.  After
+ * the watchdog limit (mlstm_set_watchdog) the wait gives up, sets bit 0 of the
+ * device error word and the site 0xF7 in bits 8..15, and the kernel returns
+ * normally: the next mlstm_last_device_error() on the stream reports
+ * MLSTM_ERR_TIMEOUT and the CUDA context stays usable.  Nothing traps or
+ * faults.  Returns MLSTM_OK once enqueued, MLSTM_ERR_CUDA if the launch
+ * fails.  The pages have no counterpart: it exists to exercise the watchdog
+ * that backs every wait of the forward pass. */
+mlstm_status mlstm_watchdog_selftest(mlstm_stream_t stream);
+
 /* Kernel families, as reported by the profiling calls below. */
 typedef enum {
   MLSTM_KERNEL_GATES = 0,         /* gate preprocessing (2 launches per call)  */

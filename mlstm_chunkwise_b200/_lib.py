@@ -35,6 +35,7 @@ SIGNATURES = {
     "mlstm_last_device_error": (_i, [_vp]),
     "mlstm_last_device_error_word": (ctypes.c_uint32, []),
     "mlstm_set_watchdog": (None, [ctypes.c_uint64]),
+    "mlstm_watchdog_selftest": (_i, [_vp]),
     "mlstm_kernel_launches": (ctypes.c_uint64, []),
     "mlstm_profile_enable": (None, [_i]),
     "mlstm_profile_read": (_i, [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_uint64),

@@ -190,3 +190,11 @@ def last_device_error(device=None) -> int:
 
 def set_watchdog(max_polls: int) -> None:
     _lib.lib().mlstm_set_watchdog(int(max_polls))
+
+
+def watchdog_selftest(device=None) -> None:
+    """Enqueues the failure-detection self-test (one bounded wait that nothing
+    satisfies) on the current stream; the next ``last_device_error`` returns
+    ``_lib.ERR_TIMEOUT``."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    _lib.check(_lib.lib().mlstm_watchdog_selftest(_stream(dev)), "mlstm_watchdog_selftest")

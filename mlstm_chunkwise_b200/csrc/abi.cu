@@ -261,6 +261,13 @@ void mlstm_set_watchdog(uint64_t max_polls) {
   g_max_polls = max_polls ? (unsigned long long)max_polls : kDefaultPolls;
 }
 
+mlstm_status mlstm_watchdog_selftest(mlstm_stream_t stream) {
+  uint32_t* w = error_word_ptr();
+  if (!w) return MLSTM_ERR_CUDA;
+  return from_cuda(
+      launch_watchdog_selftest(w, g_max_polls, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 mlstm_status mlstm_fw_workspace_size(int B, int NH, int T, int DK, int DV, int chunk_size,
                                      mlstm_dtype dtype, mlstm_algo algo, size_t* bytes) {
   if (!bytes || !valid_enums(dtype, MLSTM_GATE_EXP, algo)) return MLSTM_ERR_INVALID_ARG;

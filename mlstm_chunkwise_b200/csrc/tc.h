@@ -44,6 +44,11 @@ cudaError_t launch_tc_fused(const Problem& p, const void* Q, const void* K, cons
                             const float* C0, const float* n0, Gates g, void* H, float* C_T,
                             float* n_T, float* m_T, cudaStream_t st);
 
+// Failure-detection self-test (selftest.cu): one bounded wait that nothing
+// satisfies; it sets the watchdog bit and its site in *err and returns.
+cudaError_t launch_watchdog_selftest(uint32_t* err, unsigned long long max_polls,
+                                     cudaStream_t st);
+
 // Implementations (one per kernel file).
 cudaError_t launch_tc_states_impl(const Problem& p, const void* K, const void* V, const float* C0,
                                   const float* n0, Gates g, float* C_states, __nv_bfloat16* Cb,
