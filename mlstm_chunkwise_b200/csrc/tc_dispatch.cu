@@ -84,8 +84,6 @@ bool tc_unfused_supported(const Problem& p) {
   return tc_states_supported(p) && tc_parallel_supported(p) && p.DV % 128 == 0;
 }
 
-bool tc_fused_supported(const Problem&) { return false; }
-
 cudaError_t launch_tc_states(const Problem& p, const void* K, const void* V, const float* C0,
                              const float* n0, Gates g, float* C_states, __nv_bfloat16* Cb,
                              float* n_states, float* C_T, float* n_T, float* m_T,
@@ -114,11 +112,6 @@ cudaError_t launch_states_to_operand(const float* src, __nv_bfloat16* dst, long 
   states_to_operand_kernel<<<blocks, 256, 0, st>>>(reinterpret_cast<const float4*>(src),
                                                    reinterpret_cast<uint4*>(dst), n_bhk, DK, DV);
   return cudaGetLastError();
-}
-
-cudaError_t launch_tc_fused(const Problem&, const void*, const void*, const void*, const float*,
-                            const float*, Gates, void*, float*, float*, float*, cudaStream_t) {
-  return cudaErrorNotSupported;
 }
 
 }  // namespace mlstm

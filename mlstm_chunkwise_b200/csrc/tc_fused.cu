@@ -1,0 +1,618 @@
+// G4: the fused chunkwise forward pass -- chunk state carried on chip.
+//
+// "flash-xlstm-exp 0.1.0", "Upgrade roadmap" item 2 plans a kernel that fuses
+// the recurrent (chunk state) and parallel (output) halves so that the chunk
+// states never go through HBM.  This is that kernel for heads that fit one SM:
+// d_qk = 128, d_v of 64 or 128, chunks of 128 tokens.  Per (b, h) the chunks
+// are processed in order by one CTA; for chunk k (same quantities as the
+// unfused kernels, "Tiled Flash Linear Attention", abstract):
+//
+//   S       = Q_k K_k^T                                   (tcgen05, TMEM)
+//   P_rs    = s S_rs e^{acol_s - mu_r}  (s <= r)           (row threads, TMEM)
+//   O       = P V_k + Q~ C_k,  Q~ = diag(e^{m_k - mu_r}) Q_k
+//   h_r     = O_r / max(|den_r|, e^{-(bcum_r + mu_r)}),  den_r = e^{m_k - mu_r} n_k.q_r + sum_s P_rs
+//   C_{k+1} = e^{g_k + m_k - m_{k+1}} C_k + (w K_k)^T V_k,  w_s = s e^{g_k + acol_s - m_{k+1}}
+//   n_{k+1} = the same with V -> 1 (fp32, from the unrounded products w_s k_s)
+//
+// The fp32 master state C lives in TMEM for the whole sequence of a head; the
+// Q~ C_k MMA reads a bf16 copy of it that the row threads write into shared
+// memory once per chunk (together with the decay of the master).  The n
+// vector is carried in shared memory by the row threads.
+//
+// Roles (320 threads): warp 0 TMA producer; warp 1 TMEM owner and MMA issuer;
+// warps 2..9 two threads per row (each owning half of the columns).  One
+// persistent CTA per SM walks its heads; the chunk counter runs on across
+// heads, so the next head's first chunk is prefetched like any other.
+// MMA order per chunk j:  [ready(j)]  P.V(j)  S(j+1)  Q~.C(j)  C += (wK)^T V(j)
+// Row order per chunk j:  prep(j+1) (den_inter, P, Q~, wK, n)  epilogue(j)
+//                         [master ready] operand copy of C_{j+1}, decay -> ready(j+1)
+// TMEM (512 columns): master C [0, 128), S/P buffers [128, 256) and
+// [256, 384), O [384, 512).
+#include <cuda.h>
+
+#include "tc.h"
+#include "tc_ptx.cuh"
+
+namespace mlstm {
+namespace {
+
+using namespace tc;
+
+constexpr int kThreads = 320;
+constexpr int kL = 128;   // chunk = query tile = key tile
+constexpr int kDK = 128;  // key width handled by this kernel
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColC = 0, kColS0 = 128, kColS1 = 256, kColO = 384;
+
+template <int DV>
+struct FCfg {
+  static_assert(DV == 64 || DV == 128, "d_v of 64 or 128");
+  static constexpr uint32_t kQBytes = kL * kDK * 2;   // 2 slabs [128 rows x 64] (16 KB each)
+  static constexpr uint32_t kKBytes = kL * kDK * 2;
+  static constexpr uint32_t kVBytes = kL * DV * 2;    // [2 key halves][DV / 64 blocks][64 x 64]
+  static constexpr uint32_t kCBytes = kDK * DV * 2;   // [2 dk slabs][DV / 64 blocks][64 x 64]
+  static constexpr int kVBufs = DV <= 64 ? 2 : 1;
+  static constexpr int kRG = 256 / (kDK / 8);         // row groups of the K pass (16)
+  static constexpr uint32_t kOffQ = 0;                                   // 2 buffers
+  static constexpr uint32_t kOffK = kOffQ + 2 * kQBytes;                 // 2 buffers
+  static constexpr uint32_t kOffV = kOffK + 2 * kKBytes;                 // kVBufs buffers
+  static constexpr uint32_t kOffC = kOffV + kVBufs * kVBytes;
+  static constexpr uint32_t kOffRedN = kOffC + kCBytes;                  // float[kRG][kDK]
+  static constexpr uint32_t kOffN = kOffRedN + kRG * kDK * 4;            // float[kDK]
+  static constexpr uint32_t kOffAcol = kOffN + kDK * 4;                  // float[2][kL]
+  static constexpr uint32_t kOffRed = kOffAcol + 2 * kL * 4;             // float[256]
+  static constexpr uint32_t kOffBar = kOffRed + 256 * 4;
+  static constexpr uint32_t kOffTmemSlot = kOffBar + 256;
+  static constexpr uint32_t kBytes = kOffTmemSlot + 16;
+  static constexpr uint32_t kSmem = kBytes + 1024;
+  static_assert(kSmem <= 227 * 1024, "shared memory");
+};
+
+struct FBars {
+  uint32_t a;
+  __device__ __forceinline__ uint32_t q_full(int b) const { return a + 8 * b; }
+  __device__ __forceinline__ uint32_t q_free(int b) const { return a + 16 + 8 * b; }
+  __device__ __forceinline__ uint32_t k_full(int b) const { return a + 32 + 8 * b; }
+  __device__ __forceinline__ uint32_t k_free(int b) const { return a + 48 + 8 * b; }
+  __device__ __forceinline__ uint32_t v_full(int b) const { return a + 64 + 8 * b; }
+  __device__ __forceinline__ uint32_t v_free(int b) const { return a + 80 + 8 * b; }
+  __device__ __forceinline__ uint32_t s_full(int b) const { return a + 96 + 8 * b; }
+  __device__ __forceinline__ uint32_t ready() const { return a + 112; }
+  __device__ __forceinline__ uint32_t o_full() const { return a + 120; }
+  __device__ __forceinline__ uint32_t upd_done() const { return a + 128; }
+  __device__ __forceinline__ uint32_t mma_idle() const { return a + 136; }
+};
+
+// The j-th chunk of this CTA (over its heads in turn): head and chunk index.
+struct FChunk {
+  int bh, k;
+};
+__device__ __forceinline__ FChunk chunk_at(int j, int NC) {
+  FChunk c;
+  c.bh = (int)blockIdx.x + (j / NC) * (int)gridDim.x;
+  c.k = j % NC;
+  return c;
+}
+
+template <int DV>
+__global__ void __launch_bounds__(kThreads, 1)
+tc_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_h,
+                Problem p, Gates g, const float* __restrict__ C0, const float* __restrict__ n0,
+                float* __restrict__ C_T, float* __restrict__ n_T, float* __restrict__ m_T) {
+  using F = FCfg<DV>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const FBars bar{sbase + F::kOffBar};
+  float* redn_s = reinterpret_cast<float*>(smem + F::kOffRedN);
+  float* n_s = reinterpret_cast<float*>(smem + F::kOffN);
+  float* acol_s = reinterpret_cast<float*>(smem + F::kOffAcol);
+  float* red_s = reinterpret_cast<float*>(smem + F::kOffRed);
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + F::kOffTmemSlot);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int NC = p.NC;
+  const int my_heads = p.BH > (int)blockIdx.x
+                           ? (p.BH - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x
+                           : 0;
+  const int total = my_heads * NC;  // chunks of this CTA
+  const long tpad = (long)NC * p.L;
+
+  if (threadIdx.x == 0) {
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar.q_full(b), 1);
+      mbar_init(bar.q_free(b), 1);
+      mbar_init(bar.k_full(b), 1);
+      mbar_init(bar.k_free(b), 1);
+      mbar_init(bar.v_full(b), 1);
+      mbar_init(bar.v_free(b), 1);
+      mbar_init(bar.s_full(b), 1);
+    }
+    mbar_init(bar.ready(), 256);
+    mbar_init(bar.o_full(), 1);
+    mbar_init(bar.upd_done(), 1);
+    mbar_init(bar.mma_idle(), 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32((const void*)tmem_slot), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ---------------------------- TMA producer ----------------------------
+    // Order: Q(0), K(0), then per chunk j: V(j), Q(j+1), K(j+1).  Each load
+    // waits for the release of its buffer by the chunk two (Q, K) or
+    // kVBufs (V) before; every release completes once per chunk of its
+    // buffer and the next load of that buffer is issued only after the wait.
+    if (lane == 0 && total > 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      bool ok = true;
+      auto load_qk = [&](int j) {
+        const FChunk c = chunk_at(j, NC);
+        const int b = j & 1, t0 = c.k * kL;
+        if (j >= 2) ok = ok && mbar_wait(bar.q_free(b), ((j >> 1) - 1) & 1, p, 1);
+        if (!ok) return;
+        mbar_expect_tx(bar.q_full(b), F::kQBytes);
+        for (int s = 0; s < 2; ++s)
+          tma_load_3d(sbase + F::kOffQ + b * F::kQBytes + s * 16384, &tm_q, s * 64, t0, c.bh,
+                      bar.q_full(b));
+        if (j >= 2) ok = ok && mbar_wait(bar.k_free(b), ((j >> 1) - 1) & 1, p, 2);
+        if (!ok) return;
+        mbar_expect_tx(bar.k_full(b), F::kKBytes);
+        for (int s = 0; s < 2; ++s)
+          tma_load_3d(sbase + F::kOffK + b * F::kKBytes + s * 16384, &tm_k, s * 64, t0, c.bh,
+                      bar.k_full(b));
+      };
+      auto load_v = [&](int j) {
+        const FChunk c = chunk_at(j, NC);
+        const int b = j % F::kVBufs, t0 = c.k * kL;
+        if (j >= F::kVBufs) ok = ok && mbar_wait(bar.v_free(b), ((j / F::kVBufs) - 1) & 1, p, 3);
+        if (!ok) return;
+        mbar_expect_tx(bar.v_full(b), F::kVBytes);
+        for (int v = 0; v < 2; ++v)
+          for (int blk = 0; blk < DV / 64; ++blk)
+            tma_load_3d(sbase + F::kOffV + b * F::kVBytes + (v * (DV / 64) + blk) * 8192, &tm_v,
+                        blk * 64, t0 + v * 64, c.bh, bar.v_full(b));
+      };
+      load_qk(0);
+      for (int j = 0; j < total && ok; ++j) {
+        load_v(j);
+        if (j + 1 < total) load_qk(j + 1);
+      }
+      // Drain: the last loads of every buffer must land before the CTA exits.
+      for (int j = (total > 2 ? total - 2 : 0); j < total; ++j) {
+        mbar_wait(bar.q_full(j & 1), (j >> 1) & 1, p, 12);
+        mbar_wait(bar.k_full(j & 1), (j >> 1) & 1, p, 12);
+      }
+      for (int j = (total > F::kVBufs ? total - F::kVBufs : 0); j < total; ++j)
+        mbar_wait(bar.v_full(j % F::kVBufs), (j / F::kVBufs) & 1, p, 12);
+    }
+  } else if (warp == 1) {
+    // ---------------------------- MMA issuer ------------------------------
+    if (lane == 0 && total > 0) {
+      constexpr uint32_t idS = idesc_bf16(128, kL, 0, 0);
+      constexpr uint32_t idO = idesc_bf16(128, DV, 0, 1);
+      constexpr uint32_t idU = idesc_bf16(128, DV, 1, 1);
+      bool ok = true;
+      // S(j) = Q K^T into S buffer j & 1.  That buffer held P(j - 2), read by
+      // P.V(j - 2), which precedes Q~.C(j - 2): o_full of chunk j - 2 (waited
+      // by the caller) means it has been read.
+      auto issue_s = [&](int j) {
+        const int b = j & 1;
+        ok = ok && mbar_wait(bar.q_full(b), (j >> 1) & 1, p, 4);
+        ok = ok && mbar_wait(bar.k_full(b), (j >> 1) & 1, p, 4);
+        tc_fence_after();
+        if (!ok) return;
+        const uint32_t qa = sbase + F::kOffQ + b * F::kQBytes;
+        const uint32_t ka = sbase + F::kOffK + b * F::kKBytes;
+        const uint32_t dS = tmem + (b ? kColS1 : kColS0);
+#pragma unroll
+        for (int s = 0; s < 2; ++s)
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_bf16_ss(dS, sdesc_sw128(qa + s * 16384 + kk * 32, 16, 1024),
+                        sdesc_sw128(ka + s * 16384 + kk * 32, 16, 1024), idS, (s | kk) != 0);
+        mma_commit(bar.s_full(b));
+      };
+      issue_s(0);
+      for (int j = 0; j < total && ok; ++j) {
+        const int b = j & 1, vb = j % F::kVBufs;
+        // ready(j): P(j), Q~(j), w K(j) in place, the operand copy of C_j and
+        // the decayed master; it also follows the epilogue of chunk j - 1, so
+        // the single O accumulator is free.  (Completes once per chunk; the
+        // next completion needs this chunk's MMAs.)
+        ok = ok && mbar_wait(bar.ready(), j & 1, p, 5);
+        ok = ok && mbar_wait(bar.v_full(vb), (j / F::kVBufs) & 1, p, 6);
+        tc_fence_after();
+        if (!ok) break;
+        const uint32_t qa = sbase + F::kOffQ + b * F::kQBytes;
+        const uint32_t ka = sbase + F::kOffK + b * F::kKBytes;
+        const uint32_t va = sbase + F::kOffV + vb * F::kVBytes;
+        const uint32_t ca = sbase + F::kOffC;
+        const uint32_t aP = tmem + (b ? kColS1 : kColS0);
+        // P . V, A = P from TMEM (key half v: columns [64 v, 64 v + 32))
+#pragma unroll
+        for (int v = 0; v < 2; ++v)
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_bf16_ts(tmem + kColO, aP + v * 64 + kk * 8,
+                        sdesc_sw128(va + v * (DV / 64) * 8192 + kk * 2048, 8192, 1024), idO,
+                        (v | kk) != 0);
+        if (j + 1 < total) {
+          if (j >= 1) ok = ok && mbar_wait(bar.o_full(), (j - 1) & 1, p, 7);
+          issue_s(j + 1);
+          if (!ok) break;
+        }
+        // Q~ . C_j (operand copy in shared memory, MN-major)
+#pragma unroll
+        for (int s = 0; s < 2; ++s)
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_bf16_ss(tmem + kColO, sdesc_sw128(qa + s * 16384 + kk * 32, 16, 1024),
+                        sdesc_sw128(ca + s * (DV / 64) * 8192 + kk * 2048, 8192, 1024), idO, 1);
+        mma_commit(bar.o_full());
+        // master += (w K)^T V: A = K^T MN-major (dk halves 16 KB apart), B = V
+#pragma unroll
+        for (int kk = 0; kk < kL / 16; ++kk)
+          mma_bf16_ss(tmem + kColC, sdesc_sw128(ka + kk * 2048, 16384, 1024),
+                      sdesc_sw128(va + (kk >> 2) * (DV / 64) * 8192 + (kk & 3) * 2048, 8192, 1024),
+                      idU, 1);
+        mma_commit(bar.upd_done());
+        mma_commit(bar.k_free(b));
+        mma_commit(bar.v_free(vb));
+      }
+      mma_commit(bar.mma_idle());
+      mbar_wait(bar.mma_idle(), 0, p, 15);
+    }
+  } else {
+    // ------------------------------ row threads ---------------------------
+    const int q = warp & 3;
+    const int r = q * 32 + lane;   // query row / TMEM lane / dk row of the master
+    const int rt = threadIdx.x - 64;
+    const int h = rt >> 7;         // half of the columns
+    const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16);
+    const float ks = p.key_scale;
+    constexpr float kLog2e = 1.4426950408889634f;
+    constexpr int kHalfV = DV / 2;
+    // K pass mapping: 16-byte chunk cc (8 dk columns) of rows rg * 8 .. + 7
+    const int cc = rt % (kDK / 8);
+    const int rg = rt / (kDK / 8);
+    bool ok = true;
+
+    struct Rows {
+      float m_in, m_out, mu, bc, gk, decay;
+    };
+    auto fetch = [&](const FChunk& c, int buf) -> Rows {
+      Rows v;
+      const long base = (long)c.bh * tpad + (long)c.k * kL;
+      v.m_in = g.mchk[(long)c.bh * (NC + 1) + c.k];
+      v.m_out = g.mchk[(long)c.bh * (NC + 1) + c.k + 1];
+      v.mu = fmaxf(v.m_in, g.amax[base + r]);
+      v.bc = g.bcum[base + r];
+      v.gk = g.gtot[(long)c.bh * NC + c.k];
+      v.decay = expf(v.gk + v.m_in - v.m_out);
+      float* ac = acol_s + buf * kL;
+      if (rt < kL) ac[rt] = g.acol[base + rt];
+      return v;
+    };
+    // master <- C0 of head bh (or zero)
+    auto init_master = [&](int bh) {
+      for (int c = 0; c < kHalfV; c += 32) {
+        uint32_t v[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e)
+          v[e] = __float_as_uint(C0 ? C0[((long)bh * kDK + r) * DV + h * kHalfV + c + e] : 0.f);
+        tmem_st32(trow + kColC + h * kHalfV + c, v);
+      }
+      tmem_wait_st();
+    };
+    // C_T and m_T of head bh from the master (all its updates completed);
+    // n_T is written where the n vector of the head ends (see the loop).
+    auto write_final = [&](int bh) {
+      for (int c = 0; c < kHalfV; c += 32) {
+        uint32_t v[32];
+        tmem_ld32(trow + kColC + h * kHalfV + c, v);
+        tmem_wait_ld();
+        if (C_T) {
+          float4* dst = reinterpret_cast<float4*>(C_T + ((long)bh * kDK + r) * DV + h * kHalfV + c);
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            dst[e] = make_float4(__uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1]),
+                                 __uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3]));
+        }
+      }
+      if (rt == 0 && m_T) m_T[bh] = g.mchk[(long)bh * (NC + 1) + NC];
+    };
+    // Operand copy of the master (C of the chunk about to start) into shared
+    // memory as bf16 (MN-major, 128-byte swizzle), then the decay of the
+    // master in place.  Called once every MMA of the previous chunk has
+    // completed (its Q~.C read the old copy; its update wrote the master).
+    auto copy_and_decay = [&](float decay) {
+      const int sl = r >> 6, rr = r & 63;
+      uint8_t* crow = smem + F::kOffC + sl * (DV / 64) * 8192 + rr * 128;
+      for (int c = 0; c < kHalfV; c += 32) {
+        uint32_t v[32];
+        tmem_ld32(trow + kColC + h * kHalfV + c, v);
+        tmem_wait_ld();
+        const int col0 = h * kHalfV + c;  // first d_v column of these 32
+        uint8_t* blk = crow + (col0 >> 6) * 8192;
+        const int ch0 = (col0 & 63) >> 3;
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          *reinterpret_cast<uint4*>(blk + (((ch0 + e) ^ (rr & 7)) << 4)) = make_uint4(
+              pack_bf16x2(__uint_as_float(v[8 * e]), __uint_as_float(v[8 * e + 1])),
+              pack_bf16x2(__uint_as_float(v[8 * e + 2]), __uint_as_float(v[8 * e + 3])),
+              pack_bf16x2(__uint_as_float(v[8 * e + 4]), __uint_as_float(v[8 * e + 5])),
+              pack_bf16x2(__uint_as_float(v[8 * e + 6]), __uint_as_float(v[8 * e + 7])));
+#pragma unroll
+        for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * decay);
+        tmem_st32(trow + kColC + h * kHalfV + c, v);
+      }
+      tmem_wait_st();
+    };
+    // Everything of chunk j that needs S(j) but not the MMAs of chunk j - 1:
+    // den_inter from the unscaled Q and n_j, P into TMEM, the scaled Q~ and
+    // the weighted K in place, and n_{j+1}.  Returns this half's partial
+    // denominator.
+    auto prep = [&](int j, const Rows& rv) -> float {
+      const int b = j & 1;
+      uint8_t* qbuf = smem + F::kOffQ + b * F::kQBytes;
+      uint8_t* kbuf = smem + F::kOffK + b * F::kKBytes;
+      const float* ac = acol_s + b * kL;
+      const float f_inter = expf(rv.m_in - rv.mu);
+      const float mu2 = rv.mu * kLog2e;
+      ok = ok && mbar_wait(bar.s_full(b), (j >> 1) & 1, p, 8);  // S(j) done: Q, K read
+      tc_fence_after();
+      // den_inter over this half's 64 dk columns (slab h of Q)
+      float dn = 0.f;
+      {
+        const uint8_t* slab = qbuf + h * 16384;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const uint4 u = *reinterpret_cast<const uint4*>(slab + sw128_offset(r, c));
+          const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f2 = __bfloat1622float2(h2[e]);
+            dn = fmaf(f2.x, n_s[h * 64 + c * 8 + 2 * e], dn);
+            dn = fmaf(f2.y, n_s[h * 64 + c * 8 + 2 * e + 1], dn);
+          }
+        }
+      }
+      float den = f_inter * dn;
+      // P = gated S over this half's 64 keys, back into the S columns it read
+      // (in two passes of 32 keys: the packed 16 columns of the first pass
+      // land on columns that pass has already read).
+      {
+        const uint32_t scol = (b ? kColS1 : kColS0) + h * 64;
+        float rs = 0.f;
+#pragma unroll
+        for (int hp = 0; hp < 2; ++hp) {
+          uint32_t v[32];
+          tmem_ld32(trow + scol + hp * 32, v);
+          tmem_wait_ld();
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const int s0 = h * 64 + hp * 32 + e;
+            float pa = __uint_as_float(v[e]) * ks * ex2_approx(ac[s0] * kLog2e - mu2);
+            float pb = __uint_as_float(v[e + 1]) * ks * ex2_approx(ac[s0 + 1] * kLog2e - mu2);
+            if (s0 > r) pa = 0.f;
+            if (s0 + 1 > r) pb = 0.f;
+            rs += pa + pb;
+            pk[e >> 1] = pack_bf16x2(pa, pb);
+          }
+          tmem_st16(trow + scol + hp * 16, pk);
+        }
+        den += rs;
+      }
+      // Q~ = e^{m_k - mu_r} q_r in place (slab h)
+      {
+        uint8_t* slab = qbuf + h * 16384;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          uint4* ptr = reinterpret_cast<uint4*>(slab + sw128_offset(r, c));
+          uint4 u = *ptr;
+          __nv_bfloat162* h2 = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f2 = __bfloat1622float2(h2[e]);
+            h2[e] = __floats2bfloat162_rn(f2.x * f_inter, f2.y * f_inter);
+          }
+          *ptr = u;
+        }
+      }
+      // w K in place and the n partials from the unrounded products
+      float part[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      {
+        uint8_t* slab = kbuf + (cc >> 3) * 16384;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int row = rg * 8 + i;
+          const float w = ks * expf(rv.gk + ac[row] - rv.m_out);  // -inf -> 0
+          uint4* ptr = reinterpret_cast<uint4*>(slab + sw128_offset(row, cc & 7));
+          uint4 u = *ptr;
+          __nv_bfloat162* h2 = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f2 = __bfloat1622float2(h2[e]);
+            part[2 * e] = fmaf(f2.x, w, part[2 * e]);
+            part[2 * e + 1] = fmaf(f2.y, w, part[2 * e + 1]);
+            h2[e] = __floats2bfloat162_rn(f2.x * w, f2.y * w);
+          }
+          *ptr = u;
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < 8; ++e) redn_s[rg * kDK + cc * 8 + e] = part[e];
+      tmem_wait_st();
+      named_bar_sync(1, 256);  // n_j reads done, partials in place
+      if (rt < kDK) {
+        float acc = 0.f;
+#pragma unroll
+        for (int i = 0; i < F::kRG; ++i) acc += redn_s[i * kDK + rt];
+        n_s[rt] = rv.decay * n_s[rt] + acc;  // n_{j+1}
+      }
+      fence_proxy_async_smem();  // Q~ and w K for the MMAs
+      named_bar_sync(1, 256);  // n_{j+1} visible; redn_s free
+      return den;
+    };
+
+    // Epilogue of chunk j: the row's denominator from both halves, then
+    // O / den as bf16 through the chunk's (now free) Q buffer and TMA stores.
+    auto epilogue = [&](int j, const FChunk& c, const Rows& rv, float den_part) {
+      const int b = j & 1;
+      red_s[rt] = den_part;
+      named_bar_sync(1, 256);
+      const float den = den_part + red_s[rt ^ 128];
+      const float denom = fmaxf(fabsf(den), expf(-(rv.bc + rv.mu)));
+      const float inv = 1.f / denom;
+      ok = ok && mbar_wait(bar.o_full(), j & 1, p, 9);  // Q~.C(j) done: Q(j) free
+      tc_fence_after();
+      uint32_t v0[32], v1[32];
+      tmem_ld32(trow + kColO + h * kHalfV, v0);
+      if (kHalfV >= 64) tmem_ld32(trow + kColO + h * kHalfV + 32, v1);
+      tmem_wait_ld();
+      uint8_t* stg = smem + F::kOffQ + b * F::kQBytes;  // [DV / 64 boxes][128 rows][128 B]
+      const int col0 = h * kHalfV;
+      uint8_t* box = stg + (col0 >> 6) * 16384;
+      const int ch0 = (col0 & 63) >> 3;
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        *reinterpret_cast<uint4*>(box + sw128_offset(r, ch0 + e)) = make_uint4(
+            pack_bf16x2(__uint_as_float(v0[8 * e]) * inv, __uint_as_float(v0[8 * e + 1]) * inv),
+            pack_bf16x2(__uint_as_float(v0[8 * e + 2]) * inv, __uint_as_float(v0[8 * e + 3]) * inv),
+            pack_bf16x2(__uint_as_float(v0[8 * e + 4]) * inv, __uint_as_float(v0[8 * e + 5]) * inv),
+            pack_bf16x2(__uint_as_float(v0[8 * e + 6]) * inv, __uint_as_float(v0[8 * e + 7]) * inv));
+      if (kHalfV >= 64) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          *reinterpret_cast<uint4*>(box + sw128_offset(r, ch0 + 4 + e)) = make_uint4(
+              pack_bf16x2(__uint_as_float(v1[8 * e]) * inv, __uint_as_float(v1[8 * e + 1]) * inv),
+              pack_bf16x2(__uint_as_float(v1[8 * e + 2]) * inv,
+                          __uint_as_float(v1[8 * e + 3]) * inv),
+              pack_bf16x2(__uint_as_float(v1[8 * e + 4]) * inv,
+                          __uint_as_float(v1[8 * e + 5]) * inv),
+              pack_bf16x2(__uint_as_float(v1[8 * e + 6]) * inv,
+                          __uint_as_float(v1[8 * e + 7]) * inv));
+      }
+      fence_proxy_async_smem();
+      named_bar_sync(1, 256);
+      if (rt == 0) {
+        if (ok)
+          for (int bx = 0; bx < DV / 64; ++bx)
+            tma_store_3d(&tm_h, sbase + F::kOffQ + b * F::kQBytes + bx * 16384, bx * 64,
+                         c.k * kL, c.bh);
+        tma_store_commit();
+        tma_store_wait_read_all();  // the Q buffer may take chunk j + 2's Q
+        mbar_arrive(bar.q_free(b));
+      }
+    };
+
+    if (total > 0) {
+      const FChunk c0 = chunk_at(0, NC);
+      init_master(c0.bh);
+      if (rt < kDK) n_s[rt] = n0 ? n0[(long)c0.bh * kDK + rt] : 0.f;
+      Rows cur = fetch(c0, 0);
+      named_bar_sync(1, 256);  // acol, n visible
+      float den_cur = prep(0, cur);
+      copy_and_decay(cur.decay);
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(bar.ready());
+      for (int j = 0; j < total && ok; ++j) {
+        const FChunk c = chunk_at(j, NC);
+        const bool last_of_head = (c.k == NC - 1);
+        Rows nxt = cur;
+        float den_nxt = 0.f;
+        FChunk cn{};
+        if (j + 1 < total) {
+          cn = chunk_at(j + 1, NC);
+          nxt = fetch(cn, (j + 1) & 1);
+          if (last_of_head) {
+            // n_T of this head before the next head's n0 replaces it
+            named_bar_sync(1, 256);
+            if (rt < kDK && n_T) n_T[(long)c.bh * kDK + rt] = n_s[rt];
+            if (rt < kDK) n_s[rt] = n0 ? n0[(long)cn.bh * kDK + rt] : 0.f;
+          }
+          named_bar_sync(1, 256);  // acol of chunk j + 1 and n visible
+          den_nxt = prep(j + 1, nxt);
+        } else if (last_of_head) {
+          named_bar_sync(1, 256);
+          if (rt < kDK && n_T) n_T[(long)c.bh * kDK + rt] = n_s[rt];
+        }
+        epilogue(j, c, cur, den_cur);
+        // Every MMA of chunk j has completed (upd_done is committed last).
+        ok = ok && mbar_wait(bar.upd_done(), j & 1, p, 10);
+        tc_fence_after();
+        if (last_of_head) write_final(c.bh);
+        if (j + 1 < total) {
+          if (last_of_head) init_master(cn.bh);  // master <- C0 of the next head
+          copy_and_decay(nxt.decay);
+          fence_proxy_async_smem();
+          tc_fence_before();
+          mbar_arrive(bar.ready());
+        }
+        cur = nxt;
+        den_cur = den_nxt;
+      }
+      if (rt == 0) tma_store_wait_all();
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+template <int DV>
+cudaError_t launch_fused_t(const Problem& p, const void* Q, const void* K, const void* V,
+                           const float* C0, const float* n0, Gates g, void* H, float* C_T,
+                           float* n_T, float* m_T, cudaStream_t st) {
+  using F = FCfg<DV>;
+  CUtensorMap tq, tk, tv, th;
+  if (!encode_tmap_bf16_3d(&tq, Q, p.DK, p.T, p.BH, 64, kL) ||
+      !encode_tmap_bf16_3d(&tk, K, p.DK, p.T, p.BH, 64, kL) ||
+      !encode_tmap_bf16_3d(&tv, V, p.DV, p.T, p.BH, 64, 64) ||
+      !encode_tmap_bf16_3d(&th, H, p.DV, p.T, p.BH, 64, kL))
+    return cudaErrorInvalidValue;
+  auto kern = tc_fused_kernel<DV>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, F::kSmem);
+  if (e != cudaSuccess) return e;
+  int dev = 0, sms = 0;
+  e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  const int grid = p.BH < sms ? p.BH : sms;
+  kern<<<grid, kThreads, F::kSmem, st>>>(tq, tk, tv, th, p, g, C0, n0, C_T, n_T, m_T);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool tc_fused_supported(const Problem& p) {
+  return p.DK == kDK && (p.DV == 64 || p.DV == 128) && p.L == kL && p.T > 0;
+}
+
+cudaError_t launch_tc_fused(const Problem& p, const void* Q, const void* K, const void* V,
+                            const float* C0, const float* n0, Gates g, void* H, float* C_T,
+                            float* n_T, float* m_T, cudaStream_t st) {
+  if (p.DV == 64) return launch_fused_t<64>(p, Q, K, V, C0, n0, g, H, C_T, n_T, m_T, st);
+  if (p.DV == 128) return launch_fused_t<128>(p, Q, K, V, C0, n0, g, H, C_T, n_T, m_T, st);
+  return cudaErrorNotSupported;
+}
+
+}  // namespace mlstm
