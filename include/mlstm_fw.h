@@ -73,11 +73,19 @@ typedef enum { MLSTM_DT_F32 = 0, MLSTM_DT_BF16 = 1 } mlstm_dtype;
 typedef enum { MLSTM_GATE_EXP = 0, MLSTM_GATE_SIGMOID = 1 } mlstm_gate_mode;
 
 /* Which kernels compute the path.
- *   AUTO      the fastest algorithm that supports the arguments.
+ *   AUTO      TC_FUSED where it is supported and there are at least 592
+ *             (b, h) pairs (4 per SM of a 148-SM B200), else TC where it is
+ *             supported, else SIMT.  A fixed rule, so workspace sizes computed
+ *             for AUTO always match the algorithm the call picks.
  *   SIMT      fp32 CUDA-core kernels (the only choice for fp32 inputs).
- *   TC        bf16 tensor-core kernels, unfused: chunk states are written to
- *             the workspace in fp32 between the state and the output kernels.
- *   TC_FUSED  bf16 tensor-core kernel that carries the chunk state on chip. */
+ *   TC        bf16 tensor-core kernels, unfused: the state entering every
+ *             chunk goes to the workspace (as a bf16 operand copy plus fp32
+ *             n) between the state and the output kernels.  Needs d_qk of
+ *             128 or 256, d_v of 128 or a multiple of 256 (up to 1024), and a
+ *             chunk size that is a multiple of 128 up to 1024.
+ *   TC_FUSED  bf16 tensor-core kernel that carries the chunk state on chip
+ *             ("Upgrade roadmap" item 2 of the flash-xlstm-exp page): d_qk =
+ *             128, d_v of 64 or 128, chunk size 128. */
 typedef enum {
   MLSTM_ALGO_AUTO = 0,
   MLSTM_ALGO_SIMT = 1,

@@ -127,7 +127,14 @@ bool valid_enums(mlstm_dtype dt, mlstm_gate_mode gm, mlstm_algo algo) {
 mlstm_status resolve_algo(const Problem& p, mlstm_dtype dt, mlstm_algo req, bool allow_fused,
                           mlstm_algo* out) {
   if (req == MLSTM_ALGO_AUTO) {
-    if (dt == MLSTM_DT_BF16 && p.T > 0 && allow_fused && tc_fused_supported(p)) {
+    // The fused kernel walks each head's chunks in order on one SM, so it
+    // wins only with several heads per SM (measured: 1024 heads of 8 chunks
+    // faster than the unfused path, 256 heads slower).  The threshold is a
+    // constant (4 heads per SM of a 148-SM B200) so that the workspace size
+    // computed on the host always matches the algorithm a call picks.
+    constexpr int kFusedMinHeads = 4 * 148;
+    if (dt == MLSTM_DT_BF16 && p.T > 0 && allow_fused && tc_fused_supported(p) &&
+        p.BH >= kFusedMinHeads) {
       *out = MLSTM_ALGO_TC_FUSED;
     } else if (dt == MLSTM_DT_BF16 && p.T > 0 && tc_unfused_supported(p)) {
       *out = MLSTM_ALGO_TC;

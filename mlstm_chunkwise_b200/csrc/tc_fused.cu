@@ -19,11 +19,13 @@
 // memory once per chunk (together with the decay of the master).  The n
 // vector is carried in shared memory by the row threads.
 //
-// Roles (320 threads): warp 0 TMA producer; warp 1 TMEM owner and MMA issuer;
-// warps 2..9 two threads per row (each owning half of the columns).  One
+// Roles (352 threads): warp 0 TMA producer; warp 1 TMEM owner and MMA issuer;
+// warp 2 stores H (a TMA store per chunk, then it releases the Q buffer the
+// rows were staged in); warps 3..10 two threads per row (each owning half of
+// the columns).  One
 // persistent CTA per SM walks its heads; the chunk counter runs on across
 // heads, so the next head's first chunk is prefetched like any other.
-// MMA order per chunk j:  [ready(j)]  P.V(j)  S(j+1)  Q~.C(j)  C += (wK)^T V(j)
+// MMA order per chunk j:  [ready(j)]  S(j+1)  [V(j)]  P.V(j)  Q~.C(j)  C += (wK)^T V(j)
 // Row order per chunk j:  prep(j+1) (den_inter, P, Q~, wK, n)  epilogue(j)
 //                         [master ready] operand copy of C_{j+1}, decay -> ready(j+1)
 // TMEM (512 columns): master C [0, 128), S/P buffers [128, 256) and
@@ -38,7 +40,7 @@ namespace {
 
 using namespace tc;
 
-constexpr int kThreads = 320;
+constexpr int kThreads = 352;
 constexpr int kL = 128;   // chunk = query tile = key tile
 constexpr int kDK = 128;  // key width handled by this kernel
 constexpr uint32_t kTmemCols = 512;
@@ -59,8 +61,9 @@ struct FCfg {
   static constexpr uint32_t kOffC = kOffV + kVBufs * kVBytes;
   static constexpr uint32_t kOffRedN = kOffC + kCBytes;                  // float[kRG][kDK]
   static constexpr uint32_t kOffN = kOffRedN + kRG * kDK * 4;            // float[kDK]
-  static constexpr uint32_t kOffAcol = kOffN + kDK * 4;                  // float[2][kL]
-  static constexpr uint32_t kOffRed = kOffAcol + 2 * kL * 4;             // float[256]
+  // per chunk (2 buffers) and key column: acol, e^{acol - c}, the weight w
+  static constexpr uint32_t kOffAcol = kOffN + kDK * 4;                  // float[2][3][kL]
+  static constexpr uint32_t kOffRed = kOffAcol + 2 * 3 * kL * 4;         // float[256]
   static constexpr uint32_t kOffBar = kOffRed + 256 * 4;
   static constexpr uint32_t kOffTmemSlot = kOffBar + 256;
   static constexpr uint32_t kBytes = kOffTmemSlot + 16;
@@ -81,6 +84,8 @@ struct FBars {
   __device__ __forceinline__ uint32_t o_full() const { return a + 120; }
   __device__ __forceinline__ uint32_t upd_done() const { return a + 128; }
   __device__ __forceinline__ uint32_t mma_idle() const { return a + 136; }
+  // H rows of the chunk staged in Q buffer b by all 256 row threads
+  __device__ __forceinline__ uint32_t stg_full(int b) const { return a + 144 + 8 * b; }
 };
 
 // The j-th chunk of this CTA (over its heads in turn): head and chunk index.
@@ -134,6 +139,8 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     mbar_init(bar.o_full(), 1);
     mbar_init(bar.upd_done(), 1);
     mbar_init(bar.mma_idle(), 1);
+    mbar_init(bar.stg_full(0), 256);
+    mbar_init(bar.stg_full(1), 256);
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -231,6 +238,12 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         // the single O accumulator is free.  (Completes once per chunk; the
         // next completion needs this chunk's MMAs.)
         ok = ok && mbar_wait(bar.ready(), j & 1, p, 5);
+        tc_fence_after();
+        // S(j + 1) first: the row threads turn it into P while V(j) arrives.
+        if (j + 1 < total) {
+          if (j >= 1) ok = ok && mbar_wait(bar.o_full(), (j - 1) & 1, p, 7);
+          issue_s(j + 1);
+        }
         ok = ok && mbar_wait(bar.v_full(vb), (j / F::kVBufs) & 1, p, 6);
         tc_fence_after();
         if (!ok) break;
@@ -247,11 +260,6 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             mma_bf16_ts(tmem + kColO, aP + v * 64 + kk * 8,
                         sdesc_sw128(va + v * (DV / 64) * 8192 + kk * 2048, 8192, 1024), idO,
                         (v | kk) != 0);
-        if (j + 1 < total) {
-          if (j >= 1) ok = ok && mbar_wait(bar.o_full(), (j - 1) & 1, p, 7);
-          issue_s(j + 1);
-          if (!ok) break;
-        }
         // Q~ . C_j (operand copy in shared memory, MN-major)
 #pragma unroll
         for (int s = 0; s < 2; ++s)
@@ -273,11 +281,32 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       mma_commit(bar.mma_idle());
       mbar_wait(bar.mma_idle(), 0, p, 15);
     }
+  } else if (warp == 2) {
+    // ------------------------------ H stores ------------------------------
+    // stg_full(b) completes once per chunk staged in buffer b; the next chunk
+    // of that buffer is staged only after its Q has been loaded, which waits
+    // for the q_free this thread arrives on.
+    if (lane == 0 && total > 0) {
+      bool ok = true;
+      for (int j = 0; j < total && ok; ++j) {
+        const int b = j & 1;
+        const FChunk c = chunk_at(j, NC);
+        ok = mbar_wait(bar.stg_full(b), (j >> 1) & 1, p, 11);
+        if (!ok) break;
+        for (int bx = 0; bx < DV / 64; ++bx)
+          tma_store_3d(&tm_h, sbase + F::kOffQ + b * F::kQBytes + bx * 16384, bx * 64, c.k * kL,
+                       c.bh);
+        tma_store_commit();
+        tma_store_wait_read_all();  // the Q buffer may take chunk j + 2's Q
+        mbar_arrive(bar.q_free(b));
+      }
+      tma_store_wait_all();
+    }
   } else {
     // ------------------------------ row threads ---------------------------
     const int q = warp & 3;
     const int r = q * 32 + lane;   // query row / TMEM lane / dk row of the master
-    const int rt = threadIdx.x - 64;
+    const int rt = threadIdx.x - 96;
     const int h = rt >> 7;         // half of the columns
     const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16);
     const float ks = p.key_scale;
@@ -288,20 +317,50 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const int rg = rt / (kDK / 8);
     bool ok = true;
 
+    // Per-chunk row values.  When sep is set the exponent of P splits into a
+    // column factor e^{acol_s - c} (c = the chunk's largest acol, factor
+    // <= 1) and a row factor e^{c - mu_r} that stays below e^60, so P costs
+    // two multiplies per element instead of an exponential.
     struct Rows {
-      float m_in, m_out, mu, bc, gk, decay;
+      float m_in, m_out, mu, bc, gk, decay, rowf;
+      bool sep;
     };
-    auto fetch = [&](const FChunk& c, int buf) -> Rows {
-      Rows v;
+    // Gate values of a chunk, loaded two chunks ahead of their use (the
+    // loads stay in flight while the chunk in between is processed).
+    struct Raw {
+      float m_in, m_out, amax, bc, gk, acol, amax0, amax_last;
+    };
+    auto load_raw = [&](const FChunk& c) -> Raw {
+      Raw v;
       const long base = (long)c.bh * tpad + (long)c.k * kL;
       v.m_in = g.mchk[(long)c.bh * (NC + 1) + c.k];
       v.m_out = g.mchk[(long)c.bh * (NC + 1) + c.k + 1];
-      v.mu = fmaxf(v.m_in, g.amax[base + r]);
+      v.amax = g.amax[base + r];
       v.bc = g.bcum[base + r];
       v.gk = g.gtot[(long)c.bh * NC + c.k];
-      v.decay = expf(v.gk + v.m_in - v.m_out);
-      float* ac = acol_s + buf * kL;
-      if (rt < kL) ac[rt] = g.acol[base + rt];
+      v.acol = rt < kL ? g.acol[base + rt] : 0.f;
+      v.amax0 = g.amax[base];
+      v.amax_last = g.amax[base + kL - 1];
+      return v;
+    };
+    auto finish = [&](const Raw& w, int buf) -> Rows {
+      Rows v;
+      v.m_in = w.m_in;
+      v.m_out = w.m_out;
+      v.mu = fmaxf(w.m_in, w.amax);
+      v.bc = w.bc;
+      v.gk = w.gk;
+      v.decay = expf(w.gk + w.m_in - w.m_out);
+      const float cmax = w.amax_last;               // max over the chunk (amax is a running max)
+      const float mu0 = fmaxf(w.m_in, w.amax0);     // the smallest mu_r of the chunk
+      v.sep = (cmax - mu0) <= 60.f;
+      v.rowf = v.sep ? ks * expf(cmax - v.mu) : 0.f;
+      if (rt < kL) {
+        float* col = acol_s + buf * 3 * kL;
+        col[rt] = w.acol;
+        col[kL + rt] = expf(w.acol - cmax);                         // -inf -> 0
+        col[2 * kL + rt] = ks * expf(w.gk + w.acol - w.m_out);      // -inf -> 0
+      }
       return v;
     };
     // master <- C0 of head bh (or zero)
@@ -367,11 +426,15 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const int b = j & 1;
       uint8_t* qbuf = smem + F::kOffQ + b * F::kQBytes;
       uint8_t* kbuf = smem + F::kOffK + b * F::kKBytes;
-      const float* ac = acol_s + b * kL;
+      const float* ac = acol_s + b * 3 * kL;   // acol
+      const float* cf = ac + kL;                // e^{acol - c}
+      const float* wc = ac + 2 * kL;            // s e^{g + acol - m_out}
       const float f_inter = expf(rv.m_in - rv.mu);
       const float mu2 = rv.mu * kLog2e;
-      ok = ok && mbar_wait(bar.s_full(b), (j >> 1) & 1, p, 8);  // S(j) done: Q, K read
-      tc_fence_after();
+      // den_inter needs Q(j) and n_j only: it overlaps the S MMA.  (q_full of
+      // a buffer completes once per load; the next load of the buffer needs
+      // this chunk's Q released, after this wait.)
+      ok = ok && mbar_wait(bar.q_full(b), (j >> 1) & 1, p, 8);
       // den_inter over this half's 64 dk columns (slab h of Q)
       float dn = 0.f;
       {
@@ -381,14 +444,20 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           const uint4 u = *reinterpret_cast<const uint4*>(slab + sw128_offset(r, c));
           const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u);
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 f2 = __bfloat1622float2(h2[e]);
-            dn = fmaf(f2.x, n_s[h * 64 + c * 8 + 2 * e], dn);
-            dn = fmaf(f2.y, n_s[h * 64 + c * 8 + 2 * e + 1], dn);
+          for (int e = 0; e < 4; e += 2) {
+            const float4 nv = *reinterpret_cast<const float4*>(n_s + h * 64 + c * 8 + 2 * e);
+            const float2 fa = __bfloat1622float2(h2[e]);
+            const float2 fb = __bfloat1622float2(h2[e + 1]);
+            dn = fmaf(fa.x, nv.x, dn);
+            dn = fmaf(fa.y, nv.y, dn);
+            dn = fmaf(fb.x, nv.z, dn);
+            dn = fmaf(fb.y, nv.w, dn);
           }
         }
       }
       float den = f_inter * dn;
+      ok = ok && mbar_wait(bar.s_full(b), (j >> 1) & 1, p, 8);  // S(j) done: Q, K read
+      tc_fence_after();
       // P = gated S over this half's 64 keys, back into the S columns it read
       // (in two passes of 32 keys: the packed 16 columns of the first pass
       // land on columns that pass has already read).
@@ -404,8 +473,14 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
             const int s0 = h * 64 + hp * 32 + e;
-            float pa = __uint_as_float(v[e]) * ks * ex2_approx(ac[s0] * kLog2e - mu2);
-            float pb = __uint_as_float(v[e + 1]) * ks * ex2_approx(ac[s0 + 1] * kLog2e - mu2);
+            float pa, pb;
+            if (rv.sep) {
+              pa = __uint_as_float(v[e]) * cf[s0] * rv.rowf;
+              pb = __uint_as_float(v[e + 1]) * cf[s0 + 1] * rv.rowf;
+            } else {
+              pa = __uint_as_float(v[e]) * ks * ex2_approx(ac[s0] * kLog2e - mu2);
+              pb = __uint_as_float(v[e + 1]) * ks * ex2_approx(ac[s0 + 1] * kLog2e - mu2);
+            }
             if (s0 > r) pa = 0.f;
             if (s0 + 1 > r) pb = 0.f;
             rs += pa + pb;
@@ -438,7 +513,7 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           const int row = rg * 8 + i;
-          const float w = ks * expf(rv.gk + ac[row] - rv.m_out);  // -inf -> 0
+          const float w = wc[row];
           uint4* ptr = reinterpret_cast<uint4*>(slab + sw128_offset(row, cc & 7));
           uint4 u = *ptr;
           __nv_bfloat162* h2 = reinterpret_cast<__nv_bfloat162*>(&u);
@@ -506,23 +581,16 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                           __uint_as_float(v1[8 * e + 7]) * inv));
       }
       fence_proxy_async_smem();
-      named_bar_sync(1, 256);
-      if (rt == 0) {
-        if (ok)
-          for (int bx = 0; bx < DV / 64; ++bx)
-            tma_store_3d(&tm_h, sbase + F::kOffQ + b * F::kQBytes + bx * 16384, bx * 64,
-                         c.k * kL, c.bh);
-        tma_store_commit();
-        tma_store_wait_read_all();  // the Q buffer may take chunk j + 2's Q
-        mbar_arrive(bar.q_free(b));
-      }
+      mbar_arrive(bar.stg_full(b));  // the store warp takes it from here
     };
 
     if (total > 0) {
       const FChunk c0 = chunk_at(0, NC);
+      Raw pending = load_raw(c0);
       init_master(c0.bh);
       if (rt < kDK) n_s[rt] = n0 ? n0[(long)c0.bh * kDK + rt] : 0.f;
-      Rows cur = fetch(c0, 0);
+      Rows cur = finish(pending, 0);
+      if (total > 1) pending = load_raw(chunk_at(1, NC));
       named_bar_sync(1, 256);  // acol, n visible
       float den_cur = prep(0, cur);
       copy_and_decay(cur.decay);
@@ -537,7 +605,8 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         FChunk cn{};
         if (j + 1 < total) {
           cn = chunk_at(j + 1, NC);
-          nxt = fetch(cn, (j + 1) & 1);
+          nxt = finish(pending, (j + 1) & 1);
+          if (j + 2 < total) pending = load_raw(chunk_at(j + 2, NC));
           if (last_of_head) {
             // n_T of this head before the next head's n0 replaces it
             named_bar_sync(1, 256);
@@ -565,7 +634,6 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         cur = nxt;
         den_cur = den_nxt;
       }
-      if (rt == 0) tma_store_wait_all();
     }
   }
 
