@@ -82,6 +82,19 @@ def flops_per_head(T, DK, DV, L):
     }
 
 
+def chunk_state_bytes_written(algo_families, B, NH, T, DK, DV, L):
+    """HBM bytes of chunk states written per step (the states entering every
+    chunk, excluding the final state): the bf16 operand copy plus fp32 n on
+    the unfused tensor-core path, fp32 C and n on the SIMT path, none in the
+    fused kernel."""
+    BH, NC = B * NH, -(-T // L)
+    if "tc_states" in algo_families:
+        return BH * NC * (DK * DV * 2 + DK * 4)
+    if "simt_states" in algo_families:
+        return BH * NC * (DK * DV * 4 + DK * 4)
+    return 0
+
+
 def kernel_bytes(fam, B, NH, T, DK, DV, L, elem):
     """Algorithmic DRAM bytes of one launch of a kernel family on the unfused
     or fused path: every input read once, every output written once (the
@@ -518,6 +531,7 @@ def run_ours(args):
         "frac_bf16_peak": (total_flops / (ms_per_step / 1e3) / 1e12) / peaks["bf16_tflops"],
         "roofline": roof,
         "kernels_ms_per_step": {k: v[0] / calls for k, v in kern.items()},
+        "chunk_state_bytes_written": chunk_state_bytes_written(set(kern), B, NH, T, DK, DV, L),
         "e2e": None if args.no_e2e else {
             "value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "steps": e2e_steps},

@@ -75,3 +75,14 @@ def test_recorded_traffic_entries_name_existing_profiles_and_sources(bench):
         for f in e["sources"]:
             assert os.path.exists(os.path.join(ROOT, "mlstm_chunkwise_b200", "csrc", f)), f
         assert len(e["sha1"]) == 40
+
+
+def test_chunk_state_bytes_by_path(bench):
+    s = SHAPE_7B
+    args = (s["B"], s["NH"], s["T"], s["DK"], s["DV"], s["L"])
+    BH, NC = s["B"] * s["NH"], s["T"] // s["L"]
+    assert bench.chunk_state_bytes_written({"gates", "tc_fused"}, *args) == 0
+    tc = bench.chunk_state_bytes_written({"gates", "tc_states", "tc_parallel"}, *args)
+    simt = bench.chunk_state_bytes_written({"gates", "simt_states", "simt_parallel"}, *args)
+    assert tc == BH * NC * (s["DK"] * s["DV"] * 2 + s["DK"] * 4)
+    assert simt > tc  # fp32 states on the SIMT path
