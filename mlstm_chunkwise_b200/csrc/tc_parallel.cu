@@ -13,10 +13,12 @@
 //   den_r = e^{m_k - mu_r} n_k.q_r    +  sum_{s<=r} P_rs
 //   h_r   = O_r / max(|den_r|, e^{-(bcum_r + mu_r)})
 //
-// The grid is at most one CTA per SM; each CTA takes items
-// blockIdx.x, blockIdx.x + gridDim.x, ...  Items are numbered with the value
-// tile fastest, then the query tile, then (b, h), so the CTAs running at the
-// same time share chunks (K, V and the chunk state stay in L2).  The TMA
+// The grid is at most one CTA per SM.  Items are numbered with the value tile
+// fastest, then the query tile, then (b, h), and taken in rounds of gridDim.x
+// consecutive items, so the CTAs running at the same time share chunks (K, V
+// and the chunk state stay in L2).  Within a round the CTAs take the items in
+// snake order (see item_at): an item's work grows with its query tile's
+// position in the chunk, and the snake pairs heavy with light items.  The TMA
 // producer runs ahead across item boundaries, so the next item's loads overlap
 // the current item's P.V and epilogue.
 //
@@ -118,6 +120,16 @@ __device__ __forceinline__ Item decode_item(int it, const Problem& p, int n_dv, 
   return x;
 }
 
+// The k-th item of this CTA: round k, position c on even rounds and G - 1 - c
+// on odd ones.  Item costs repeat with the period P = (query tiles per chunk)
+// x (value tiles); when P divides 2G every CTA's pair of rounds sums to the
+// same work (a plain stride gave each CTA the same position every round, and
+// the kernel the time of the heaviest position).
+__device__ __forceinline__ int item_at(int k) {
+  const int G = (int)gridDim.x, c = (int)blockIdx.x;
+  return k * G + ((k & 1) ? (G - 1 - c) : c);
+}
+
 template <int DK, int DVT>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_parallel_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -186,7 +198,7 @@ tc_parallel_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         return (uint32_t)s;
       };
       int n = 0;
-      for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++n) {
+      for (int it = item_at(0); it < n_items && ok; it = item_at(n + 1), ++n) {
         const Item x = decode_item(it, p, n_dv, n_q);
         auto load_k = [&](int i) {
           for (int c = 0; c < C::kSlabsK && ok; ++c) {
@@ -285,7 +297,7 @@ tc_parallel_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         ++ptile;
       };
       int n = 0;
-      for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++n) {
+      for (int it = item_at(0); it < n_items && ok; it = item_at(n + 1), ++n) {
         const Item x = decode_item(it, p, n_dv, n_q);
         ok = mbar_wait(bar.q_full(), n & 1, p, 3);
         if (ok) mma_s();
@@ -359,7 +371,7 @@ tc_parallel_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       fetch_rows(x0, nx_m_in, nx_amax, nx_bc);
       fetch_cols(x0, 0);
     }
-    for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++n) {
+    for (int it = item_at(0); it < n_items && ok; it = item_at(n + 1), ++n) {
       const Item x = decode_item(it, p, n_dv, n_q);
       const int t = x.t0 + r;
       const float m_in = nx_m_in, amax = nx_amax, bc = nx_bc;
@@ -452,7 +464,7 @@ tc_parallel_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       }
 
       // Fetch the next item's row values and column data while P.V finishes.
-      const int it_next = it + gridDim.x;
+      const int it_next = item_at(n + 1);
       if (it_next < n_items) {
         const Item xn = decode_item(it_next, p, n_dv, n_q);
         fetch_rows(xn, nx_m_in, nx_amax, nx_bc);
