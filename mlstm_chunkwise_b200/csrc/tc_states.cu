@@ -78,9 +78,11 @@ struct SBars {
   __device__ __forceinline__ uint32_t full(int i) const { return a + 8 * i; }
   __device__ __forceinline__ uint32_t empty(int i) const { return a + 64 + 8 * i; }
   __device__ __forceinline__ uint32_t kready(int i) const { return a + 128 + 8 * i; }
-  __device__ __forceinline__ uint32_t master() const { return a + 192; }
-  __device__ __forceinline__ uint32_t chunk() const { return a + 200; }
-  __device__ __forceinline__ uint32_t done() const { return a + 208; }
+  // per d_qk half: the state entering the chunk is ready (workers) / the
+  // half's MMAs of the chunk have completed (commit)
+  __device__ __forceinline__ uint32_t master(int hf) const { return a + 192 + 8 * hf; }
+  __device__ __forceinline__ uint32_t chunk(int hf) const { return a + 208 + 8 * hf; }
+  __device__ __forceinline__ uint32_t done() const { return a + 224; }
 };
 
 template <int DK, int DVT>
@@ -112,8 +114,10 @@ tc_states_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
       mbar_init(bar.empty(i), 1);
       mbar_init(bar.kready(i), kWorkers);
     }
-    mbar_init(bar.master(), kWorkers);
-    mbar_init(bar.chunk(), 1);
+    for (int hf = 0; hf < 2; ++hf) {
+      mbar_init(bar.master(hf), kWorkers);
+      mbar_init(bar.chunk(hf), 1);
+    }
     mbar_init(bar.done(), 1);
     fence_barrier_init();
   }
@@ -157,7 +161,6 @@ tc_states_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
       bool ok = true;
       int n = 0;
       for (int k = 0; k < NC && ok; ++k) {
-        ok = mbar_wait(bar.master(), k & 1, p, 2);
         for (int j = 0; j < stages_per_chunk && ok; ++j, ++n) {
           const int s = n % S::kStages;
           ok = mbar_wait(bar.kready(s), (n / S::kStages) & 1, p, 3);
@@ -166,6 +169,12 @@ tc_states_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
           const uint32_t st = sbase + S::kOffStage + (uint32_t)s * S::kStageBytes;
 #pragma unroll
           for (int hf = 0; hf < S::kHalves; ++hf) {
+            // master(hf) completes once per chunk; its next completion needs
+            // this half's MMAs of the chunk (chunk(hf), committed below).
+            if (j == 0) {
+              ok = ok && mbar_wait(bar.master(hf), k & 1, p, 2);
+              tc_fence_after();
+            }
             // A = (w K)^T: M = the 128 dk rows of this half (two 64-dk boxes,
             // MN-major), K = tokens.  B = V: N = the value columns (MN-major).
             const uint32_t a0 = st + hf * 16384;
@@ -173,10 +182,11 @@ tc_states_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
             for (int kk = 0; kk < kStageTok / 16; ++kk)
               mma_bf16_ss(tmem + hf * DVT, sdesc_sw128(a0 + kk * 2048, 8192, 1024),
                           sdesc_sw128(st + S::kKBytes + kk * 2048, 8192, 1024), idesc, 1);
+            // the half's last MMAs of the chunk: its boundary pass may start
+            if (j == stages_per_chunk - 1) mma_commit(bar.chunk(hf));
           }
           mma_commit(bar.empty(s));
         }
-        if (ok) mma_commit(bar.chunk());
       }
       mma_commit(bar.done());
     }
@@ -317,18 +327,21 @@ tc_states_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
 
       // The first stage of chunk k needs nothing from the MMAs.
       stage_pass(n++, gk, m_out);
-      if (k > 0) {
-        ok = ok && mbar_wait(bar.chunk(), (k - 1) & 1, p, 4);
-        tc_fence_after();
-      }
       named_bar_sync(1, kWorkers);  // the n-partial reads are done: store tiles free
 
-      // state entering chunk k: store (from this warp's tiles), then decay in place
-      if (Cb) {
-        // bf16 operand copy: one 32-row x 64-column tile per warp, already in
-        // the swizzled block layout, leaves with one 4 KB bulk store.
-        for (int hf = 0; hf < S::kHalves && ok; ++hf) {
-          const int dk0 = hf * 128 + q * 32;  // first state row of this warp's lanes
+      // The state entering chunk k, half by half (row halves of d_qk): store it
+      // (from this warp's tiles), then decay it in place.  Half hf waits only
+      // for its own MMAs of chunk k - 1 and releases itself to the MMAs of
+      // chunk k, so one half's MMAs overlap the other half's pass.
+      for (int hf = 0; hf < S::kHalves && ok; ++hf) {
+        if (k > 0) {
+          ok = ok && mbar_wait(bar.chunk(hf), (k - 1) & 1, p, 4);
+          tc_fence_after();
+        }
+        const int dk0 = hf * 128 + q * 32;  // first state row of this warp's lanes
+        if (Cb) {
+          // bf16 operand copy: one 32-row x 64-column tile per warp, already in
+          // the swizzled block layout, leaves with one 4 KB bulk store.
           for (int c = 0; c < kColsPer; c += 64) {
             const int col = ch * kColsPer + c;
             if (lane == 0) tma_store_wait_read_all();  // the previous tile has been read
@@ -358,11 +371,8 @@ tc_states_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
               tma_store_commit();
             }
           }
-        }
-      } else {
-        // fp32 states (or none): 16-column tiles through the tensor map
-        for (int hf = 0; hf < S::kHalves && ok; ++hf) {
-          const int dk0 = hf * 128 + q * 32;
+        } else {
+          // fp32 states (or none): 16-column tiles through the tensor map
           for (int c = 0; c < kColsPer; c += 32) {
             const int col = ch * kColsPer + c;
             uint32_t v[32];
@@ -379,15 +389,15 @@ tc_states_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
             tmem_st32(trow + hf * DVT + col, v);
           }
         }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar.master(hf));
       }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(bar.master());
 
       for (int j = 1; j < stages_per_chunk && ok; ++j) stage_pass(n++, gk, m_out);
     }
     // final state (fold the last chunk's n partials first)
-    if (ok) ok = mbar_wait(bar.chunk(), (NC - 1) & 1, p, 6);
+    for (int hf = 0; hf < S::kHalves && ok; ++hf) ok = mbar_wait(bar.chunk(hf), (NC - 1) & 1, p, 6);
     tc_fence_after();
     fold_n();
     if (ok && C_T) {
