@@ -79,9 +79,12 @@ size_t cb_bytes(const Problem& p) {
   return round_up((size_t)p.BH * p.NC * (size_t)p.DK * p.DV * sizeof(__nv_bfloat16));
 }
 
+size_t seg_bytes(const Problem& p) { return round_up(tc_states_segment_floats(p) * sizeof(float)); }
+
 // Workspace layout: the gate arrays, then
 //   kFull/SIMT:     C_states fp32 [BH, NC, DK, DV], n_states fp32 [BH, NC, DK]
-//   kFull/TC:       C_states bf16 (operand copy), n_states fp32
+//   kFull/TC:       C_states bf16 (operand copy), n_states fp32, segment end states
+//   kStates/TC:     segment end states
 //   kParallel/TC:   C_states bf16 (converted from the caller's fp32 states)
 //   everything else: nothing more.
 Layout layout_for(const Problem& p, mlstm_algo a, Mode mode) {
@@ -93,7 +96,9 @@ Layout layout_for(const Problem& p, mlstm_algo a, Mode mode) {
   if (mode == Mode::kFull && a == MLSTM_ALGO_SIMT)
     l.states_bytes = round_up(BH * p.NC * (size_t)p.DK * p.DV * sizeof(float)) + n_bytes;
   else if (mode == Mode::kFull && a == MLSTM_ALGO_TC)
-    l.states_bytes = cb_bytes(p) + n_bytes;
+    l.states_bytes = cb_bytes(p) + n_bytes + seg_bytes(p);
+  else if (mode == Mode::kStates && a == MLSTM_ALGO_TC)
+    l.states_bytes = seg_bytes(p);
   else if (mode == Mode::kParallel && a == MLSTM_ALGO_TC)
     l.states_bytes = cb_bytes(p);
   l.total = l.gates_bytes + l.states_bytes;
@@ -340,8 +345,11 @@ mlstm_status mlstm_fw(const void* Q, const void* K, const void* V, const float* 
   if (a == MLSTM_ALGO_TC) {
     __nv_bfloat16* Cb = reinterpret_cast<__nv_bfloat16*>(rest);
     float* n_states = reinterpret_cast<float*>(rest + cb_bytes(p));
-    s = from_cuda(launch_family(MLSTM_KERNEL_TC_STATES, 1, st, [&] {
-      return launch_tc_states(p, K, V, C0, n0, g, nullptr, Cb, n_states, C_T, n_T, m_T, st);
+    float* seg_ws = reinterpret_cast<float*>(
+        rest + cb_bytes(p) + round_up((size_t)p.BH * p.NC * (size_t)DK * sizeof(float)));
+    s = from_cuda(launch_family(MLSTM_KERNEL_TC_STATES, tc_states_launches(p), st, [&] {
+      return launch_tc_states(p, K, V, C0, n0, g, nullptr, Cb, n_states, C_T, n_T, m_T, seg_ws,
+                              st);
     }));
     if (s != MLSTM_OK) return s;
     return from_cuda(launch_family(MLSTM_KERNEL_TC_PARALLEL, 1, st, [&] {
@@ -391,13 +399,14 @@ mlstm_status mlstm_fw_chunk_states(const void* K, const void* V, const float* i_
   if (!p.err) return MLSTM_ERR_CUDA;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   Gates g;
-  carve_gates(p, static_cast<char*>(workspace), &g, m_states);
+  float* seg_ws = reinterpret_cast<float*>(carve_gates(p, static_cast<char*>(workspace), &g, m_states));
   s = from_cuda(launch_family(MLSTM_KERNEL_GATES, gate_launches(p), st,
                               [&] { return launch_gates(p, i_pre, f_pre, m0, g, st); }));
   if (s != MLSTM_OK) return s;
   if (a == MLSTM_ALGO_TC)
-    return from_cuda(launch_family(MLSTM_KERNEL_TC_STATES, 1, st, [&] {
-      return launch_tc_states(p, K, V, C0, n0, g, C_states, nullptr, n_states, C_T, n_T, m_T, st);
+    return from_cuda(launch_family(MLSTM_KERNEL_TC_STATES, tc_states_launches(p), st, [&] {
+      return launch_tc_states(p, K, V, C0, n0, g, C_states, nullptr, n_states, C_T, n_T, m_T,
+                              seg_ws, st);
     }));
   return from_cuda(launch_family(MLSTM_KERNEL_SIMT_STATES, 1, st, [&] {
     return launch_simt_states(p, dtype, K, V, C0, n0, g, C_states, n_states, C_T, n_T, m_T, st);

@@ -25,9 +25,18 @@ bool tc_fused_supported(const Problem& p);
 // Chunk states on tensor cores.  Writes the state entering every chunk as fp32
 // (C_states, nullable) and/or as the bf16 operand copy read by the parallel
 // kernel (Cb, nullable), the fp32 n states, and the optional final state.
+// With too few (b, h, d_v tile) units to fill the GPU the chunk sequences are
+// split into tc_states_segments(p) segments; seg_ws (tc_states_segment_floats(p)
+// floats, nullable when that is 0) holds the segments' end states between the
+// recurrence and the fix-up launch.
 cudaError_t launch_tc_states(const Problem& p, const void* K, const void* V, const float* C0,
                              const float* n0, Gates g, float* C_states, __nv_bfloat16* Cb,
-                             float* n_states, float* C_T, float* n_T, float* m_T, cudaStream_t st);
+                             float* n_states, float* C_T, float* n_T, float* m_T, float* seg_ws,
+                             cudaStream_t st);
+int tc_states_dvt(const Problem& p);
+int tc_states_segments(const Problem& p);
+size_t tc_states_segment_floats(const Problem& p);
+inline int tc_states_launches(const Problem& p) { return tc_states_segments(p) > 1 ? 2 : 1; }
 
 // Intra-chunk TFLA kernel + inter-chunk term, reading bf16 chunk states.
 cudaError_t launch_tc_parallel(const Problem& p, const void* Q, const void* K, const void* V,
@@ -53,7 +62,7 @@ cudaError_t launch_watchdog_selftest(uint32_t* err, unsigned long long max_polls
 cudaError_t launch_tc_states_impl(const Problem& p, const void* K, const void* V, const float* C0,
                                   const float* n0, Gates g, float* C_states, __nv_bfloat16* Cb,
                                   float* n_states, float* C_T, float* n_T, float* m_T,
-                                  cudaStream_t st);
+                                  float* seg_ws, cudaStream_t st);
 bool tc_parallel_wide_supported(const Problem& p);
 cudaError_t launch_tc_parallel_wide(const Problem& p, const void* Q, const void* K, const void* V,
                                     Gates g, const __nv_bfloat16* Cb, const float* n_states,

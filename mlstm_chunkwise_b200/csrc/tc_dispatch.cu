@@ -86,9 +86,10 @@ bool tc_unfused_supported(const Problem& p) {
 
 cudaError_t launch_tc_states(const Problem& p, const void* K, const void* V, const float* C0,
                              const float* n0, Gates g, float* C_states, __nv_bfloat16* Cb,
-                             float* n_states, float* C_T, float* n_T, float* m_T,
+                             float* n_states, float* C_T, float* n_T, float* m_T, float* seg_ws,
                              cudaStream_t st) {
-  return launch_tc_states_impl(p, K, V, C0, n0, g, C_states, Cb, n_states, C_T, n_T, m_T, st);
+  return launch_tc_states_impl(p, K, V, C0, n0, g, C_states, Cb, n_states, C_T, n_T, m_T, seg_ws,
+                               st);
 }
 
 cudaError_t launch_tc_parallel(const Problem& p, const void* Q, const void* K, const void* V,

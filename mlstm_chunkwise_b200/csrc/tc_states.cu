@@ -20,6 +20,14 @@
 // stored their own state row would touch 32 rows per instruction, and those
 // scattered stores, not the MMAs, would then set the pace of the recurrence.
 //
+// When there are too few (b, h, d_v tile) units to fill the GPU, each one's
+// chunk sequence is split into segments that run side by side (grid z).  A
+// segment after the first starts from a zero state; since the recurrence is
+// linear in the state, the state entering chunk k of segment s is
+//   C_k = C_k(local) + e^{G(k0, k) + m_{k0} - m_k} C_{k0},   G = sum of g_j, j in [k0, k)
+// and tc_states_fixup_kernel adds that term, with the states C_{k0} entering
+// each segment obtained by a short scan over the segments' end states.
+//
 // Roles (320 threads): warp 0 TMA producer, warp 1 TMEM owner + MMA issuer,
 // warps 2..9 workers: per chunk, the store and decay of the master state; per
 // stage, one pass that computes its token weights, accumulates the n-vector
@@ -91,7 +99,7 @@ tc_states_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                  const __grid_constant__ CUtensorMap tm_cs, Problem p, Gates g, const float* __restrict__ C0, const float* __restrict__ n0,
                  float* __restrict__ C_states, __nv_bfloat16* __restrict__ Cb,
                  float* __restrict__ n_states, float* __restrict__ C_T, float* __restrict__ n_T,
-                 float* __restrict__ m_T) {
+                 float* __restrict__ m_T, float* __restrict__ seg_C, float* __restrict__ seg_n) {
   using S = SCfg<DK, DVT>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -107,6 +115,12 @@ tc_states_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
   const int stages_per_chunk = L / kStageTok;
   const long tpad = (long)NC * L;
   const bool n_owner = blockIdx.x == 0;
+  // this CTA's segment of chunks [k0, k1)
+  const int seg = blockIdx.z, n_seg = gridDim.z;
+  const int ncs = (NC + n_seg - 1) / n_seg;
+  const int k0 = seg * ncs, k1 = (k0 + ncs < NC) ? k0 + ncs : NC;
+  const int nk = k1 - k0;  // >= 1 (the host picks n_seg so)
+  const int s0 = k0 * stages_per_chunk;  // first ring stage, counted from token 0
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < S::kStages; ++i) {
@@ -136,13 +150,13 @@ tc_states_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
       bool ok = true;
-      const int total = NC * stages_per_chunk;
+      const int total = nk * stages_per_chunk;
       int issued = 0;
       for (int n = 0; n < total && ok; ++n) {
         const int s = n % S::kStages, u = n / S::kStages;
         if (u > 0) ok = mbar_wait(bar.empty(s), (u - 1) & 1, p, 1);
         if (!ok) break;
-        const int tok0 = n * kStageTok;  // chunks are whole stages: k * L + j * 64
+        const int tok0 = (s0 + n) * kStageTok;  // chunks are whole stages: k * L + j * 64
         const uint32_t st = sbase + S::kOffStage + (uint32_t)s * S::kStageBytes;
         mbar_expect_tx(bar.full(s), S::kStageBytes);
         for (int b = 0; b < DK / 64; ++b)
@@ -160,7 +174,7 @@ tc_states_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
       constexpr uint32_t idesc = idesc_bf16(128, DVT, 1, 1);
       bool ok = true;
       int n = 0;
-      for (int k = 0; k < NC && ok; ++k) {
+      for (int k = 0; k < nk && ok; ++k) {
         for (int j = 0; j < stages_per_chunk && ok; ++j, ++n) {
           const int s = n % S::kStages;
           ok = mbar_wait(bar.kready(s), (n / S::kStages) & 1, p, 3);
@@ -199,14 +213,14 @@ tc_states_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
     constexpr int kColsPer = DVT / 2;  // value columns per worker in the state passes
     const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16);
     const float* mchk = g.mchk + (long)bh * (NC + 1);
-    const float* acol = g.acol + (long)bh * tpad;  // -inf on padding: weight 0
+    const float* acol = g.acol + (long)bh * tpad + (long)s0 * kStageTok;  // -inf on padding
     // this warp's two store tiles
     uint8_t* stg = smem + S::kOffStg + (warp - 2) * 4096;
     const uint32_t stg_u = sbase + S::kOffStg + (uint32_t)(warp - 2) * 4096u;
     int n_st = 0;  // state stores issued by this warp (selects the tile)
     // n-vector: worker wt owns dk column wt (DK <= 256) for the running n.
     const bool n_mine = n_owner && wt < DK;
-    float nval = (n_mine && n0) ? n0[(long)bh * DK + wt] : 0.f;
+    float nval = (n_mine && n0 && seg == 0) ? n0[(long)bh * DK + wt] : 0.f;
     // Stage pass mapping: 16-byte column chunk cc (8 dk columns) of token rows
     // rg * kRowsPer .. + kRowsPer - 1.
     const int cc = wt % S::kCC;
@@ -222,7 +236,8 @@ tc_states_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         uint32_t v[32];
 #pragma unroll
         for (int j = 0; j < 32; ++j)
-          v[j] = __float_as_uint(C0 ? C0[((long)bh * DK + dk) * DV + dv0 + col + j] : 0.f);
+          v[j] = __float_as_uint((C0 && seg == 0) ? C0[((long)bh * DK + dk) * DV + dv0 + col + j]
+                                                  : 0.f);
         tmem_st32(trow + hf * DVT + col, v);
       }
     }
@@ -274,7 +289,7 @@ tc_states_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         a_cur[4 * i + 2] = a_nxt[i].z;
         a_cur[4 * i + 3] = a_nxt[i].w;
       }
-      if (n + 1 < NC * stages_per_chunk) load_acol(n + 1);
+      if (n + 1 < nk * stages_per_chunk) load_acol(n + 1);
       ok = ok && mbar_wait(bar.full(s), (n / S::kStages) & 1, p, 5);
       uint8_t* box = smem + S::kOffStage + (uint32_t)s * S::kStageBytes + (cc >> 3) * 8192;
 #pragma unroll
@@ -317,8 +332,8 @@ tc_states_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
     };
 
     int n = 0;
-    for (int k = 0; k < NC && ok; ++k) {
-      if (k > 0) fold_n();  // chunk k - 1's partials: every worker has passed its stages
+    for (int k = k0; k < k1 && ok; ++k) {
+      if (k > k0) fold_n();  // chunk k - 1's partials: every worker has passed its stages
       const float m_in = mchk[k], m_out = mchk[k + 1];
       const float gk = g.gtot[(long)bh * NC + k];
       const float decay = expf(gk + m_in - m_out);
@@ -334,8 +349,8 @@ tc_states_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
       // for its own MMAs of chunk k - 1 and releases itself to the MMAs of
       // chunk k, so one half's MMAs overlap the other half's pass.
       for (int hf = 0; hf < S::kHalves && ok; ++hf) {
-        if (k > 0) {
-          ok = ok && mbar_wait(bar.chunk(hf), (k - 1) & 1, p, 4);
+        if (k > k0) {
+          ok = ok && mbar_wait(bar.chunk(hf), (k - k0 - 1) & 1, p, 4);
           tc_fence_after();
         }
         const int dk0 = hf * 128 + q * 32;  // first state row of this warp's lanes
@@ -397,10 +412,13 @@ tc_states_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
       for (int j = 1; j < stages_per_chunk && ok; ++j) stage_pass(n++, gk, m_out);
     }
     // final state (fold the last chunk's n partials first)
-    for (int hf = 0; hf < S::kHalves && ok; ++hf) ok = mbar_wait(bar.chunk(hf), (NC - 1) & 1, p, 6);
+    for (int hf = 0; hf < S::kHalves && ok; ++hf) ok = mbar_wait(bar.chunk(hf), (nk - 1) & 1, p, 6);
     tc_fence_after();
     fold_n();
-    if (ok && C_T) {
+    // The last segment's end state is C_T (local when segmented: the fix-up
+    // adds the rest); an earlier segment's goes to its slot of seg_C / seg_n.
+    const bool last_seg = seg == n_seg - 1;
+    if (ok && (C_T || !last_seg)) {
       for (int hf = 0; hf < S::kHalves; ++hf) {
         const int dk = hf * 128 + r;
         for (int c = 0; c < kColsPer; c += 32) {
@@ -408,7 +426,11 @@ tc_states_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
           uint32_t v[32];
           tmem_ld32(trow + hf * DVT + col, v);
           tmem_wait_ld();
-          float4* dst = reinterpret_cast<float4*>(C_T + ((long)bh * DK + dk) * DV + dv0 + col);
+          float* row_dst =
+              last_seg ? C_T + ((long)bh * DK + dk) * DV + dv0 + col
+                       : seg_C + ((((long)bh * gridDim.x + blockIdx.x) * (n_seg - 1) + seg) * DK + dk) *
+                                     DVT + col;
+          float4* dst = reinterpret_cast<float4*>(row_dst);
 #pragma unroll
           for (int j = 0; j < 8; ++j)
             dst[j] = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
@@ -416,8 +438,9 @@ tc_states_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         }
       }
     }
-    if (n_mine && n_T) n_T[(long)bh * DK + wt] = nval;
-    if (m_T && blockIdx.x == 0 && wt == 0) m_T[bh] = mchk[NC];
+    if (n_mine && last_seg && n_T) n_T[(long)bh * DK + wt] = nval;
+    if (n_mine && !last_seg) seg_n[((long)bh * (n_seg - 1) + seg) * DK + wt] = nval;
+    if (m_T && last_seg && blockIdx.x == 0 && wt == 0) m_T[bh] = mchk[NC];
     if (lane == 0) tma_store_wait_all();  // the state stores have landed
   }
 
@@ -431,10 +454,161 @@ tc_states_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
   }
 }
 
+// Segment fix-up (see the top of this file).  A thread owns 8 consecutive
+// value columns of one state row in one segment s >= 1 (grid z = s - 1): it
+// forms the state entering the segment from the earlier segments' end states,
+// then walks the segment's chunks adding a_k times it to each stored state,
+//   a_k = e^{sum of e_j, j in [k0, k)},   e_j = g_j + m_j - m_{j+1} <= 0,
+// the same per-chunk decay factors the recurrence applies.  kOperand: the
+// states are the bf16 operand copy (block layout of cb_block_row), else fp32
+// [b h k][DK][DV].
+template <bool kOperand>
+__global__ void __launch_bounds__(256)
+tc_states_fixup_kernel(Problem p, Gates g, int DVT, const float* __restrict__ seg_C,
+                       const float* __restrict__ seg_n, float* __restrict__ C_states,
+                       __nv_bfloat16* __restrict__ Cb, float* __restrict__ n_states,
+                       float* __restrict__ C_T, float* __restrict__ n_T) {
+  const int DK = p.DK, DV = p.DV, NC = p.NC;
+  const int bh = blockIdx.y, seg = blockIdx.z + 1, n_seg = gridDim.z + 1;
+  const int ncs = (NC + n_seg - 1) / n_seg;
+  const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x * blockDim.x + threadIdx.x;  // < DK * DV / 8 (exact grid)
+  int dk, col, vb = 0, jp = 0;
+  if (kOperand) {
+    jp = t & 7;  // 16-byte position within the 128-byte row
+    dk = (t >> 3) % DK;
+    vb = (t >> 3) / DK;
+    col = vb * 64 + ((jp ^ (dk & 7)) << 3);
+  } else {
+    dk = t / (DV / 8);
+    col = (t % (DV / 8)) * 8;
+  }
+  const bool n_thread = col == 0;  // one thread per state row carries n
+  const float* gt = g.gtot + (long)bh * NC;
+  const float* mc = g.mchk + (long)bh * (NC + 1);
+  auto e_of = [&](int k) { return gt[k] + mc[k] - mc[k + 1]; };
+
+  // The state entering segment seg: C_{k0(s+1)} = E_s + A_s C_{k0(s)}, with E_s
+  // segment s's end state from a zero start (segment 0 started from C0).
+  const int n_dvt = DV / DVT, dvt = col / DVT, cin = col % DVT;
+  float cs[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  float ns = 0.f;
+  for (int s = 0; s < seg; ++s) {
+    float A = 0.f;  // multiplies a zero state when s == 0
+    if (s > 0) {
+      const int a0 = s * ncs, a1 = min(a0 + ncs, NC);
+      float acc = 0.f;
+      for (int k = a0 + lane; k < a1; k += 32) acc += e_of(k);
+#pragma unroll
+      for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+      A = expf(acc);
+    }
+    const float4* e = reinterpret_cast<const float4*>(
+        seg_C + ((((long)bh * n_dvt + dvt) * (n_seg - 1) + s) * DK + dk) * DVT + cin);
+    const float4 e0 = e[0], e1 = e[1];
+    const float ev[8] = {e0.x, e0.y, e0.z, e0.w, e1.x, e1.y, e1.z, e1.w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) cs[i] = fmaf(A, cs[i], ev[i]);
+    if (n_thread) ns = fmaf(A, ns, seg_n[((long)bh * (n_seg - 1) + s) * DK + dk]);
+  }
+
+  const int k0 = seg * ncs, k1 = min(k0 + ncs, NC);
+  float lg = 0.f;  // sum of e_j over [k0, kb)
+  for (int kb = k0; kb < k1; kb += 32) {
+    // coefficients of chunks kb .. kb + 31: an exclusive warp scan of e
+    const int kl = kb + lane;
+    const float x = kl < k1 ? e_of(kl) : 0.f;
+    float inc = x;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const float y = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += y;
+    }
+    float exc = __shfl_up_sync(0xffffffffu, inc, 1);
+    if (lane == 0) exc = 0.f;
+    const float a_lane = expf(lg + exc);
+    lg += __shfl_sync(0xffffffffu, inc, 31);
+    const int nb = min(32, k1 - kb);
+    for (int c0 = 0; c0 < nb; c0 += 4) {
+      // four chunks at a time: loads first, so that they overlap
+      constexpr int kB = 4;
+      float a[kB];
+#pragma unroll
+      for (int u = 0; u < kB; ++u) a[u] = __shfl_sync(0xffffffffu, a_lane, (c0 + u) & 31);
+      if (kOperand) {
+        uint4 v[kB];
+        __nv_bfloat16* ptr[kB];
+#pragma unroll
+        for (int u = 0; u < kB; ++u) {
+          if (c0 + u < nb) {
+            ptr[u] = Cb + cb_block_row((long)bh * NC + kb + c0 + u, vb, dk, DK, DV / 64) + jp * 8;
+            v[u] = *reinterpret_cast<const uint4*>(ptr[u]);
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < kB; ++u) {
+          if (c0 + u < nb) {
+            __nv_bfloat162* h2 = reinterpret_cast<__nv_bfloat162*>(&v[u]);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 f = __bfloat1622float2(h2[e]);
+              h2[e] = __floats2bfloat162_rn(fmaf(a[u], cs[2 * e], f.x),
+                                            fmaf(a[u], cs[2 * e + 1], f.y));
+            }
+            *reinterpret_cast<uint4*>(ptr[u]) = v[u];
+          }
+        }
+      } else {
+        float4 v[kB][2];
+        float* ptr[kB];
+#pragma unroll
+        for (int u = 0; u < kB; ++u) {
+          if (c0 + u < nb) {
+            ptr[u] = C_states + (((long)bh * NC + kb + c0 + u) * DK + dk) * DV + col;
+            v[u][0] = reinterpret_cast<const float4*>(ptr[u])[0];
+            v[u][1] = reinterpret_cast<const float4*>(ptr[u])[1];
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < kB; ++u) {
+          if (c0 + u < nb) {
+            float* f = reinterpret_cast<float*>(&v[u][0]);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) f[i] = fmaf(a[u], cs[i], f[i]);
+            reinterpret_cast<float4*>(ptr[u])[0] = v[u][0];
+            reinterpret_cast<float4*>(ptr[u])[1] = v[u][1];
+          }
+        }
+      }
+      if (n_thread) {
+#pragma unroll
+        for (int u = 0; u < kB; ++u)
+          if (c0 + u < nb) n_states[((long)bh * NC + kb + c0 + u) * DK + dk] += a[u] * ns;
+      }
+    }
+  }
+  // the last segment's end state is the final state
+  if (seg == n_seg - 1) {
+    const float aT = expf(lg);
+    if (C_T) {
+      float4* d = reinterpret_cast<float4*>(C_T + ((long)bh * DK + dk) * DV + col);
+      float4 d0 = d[0], d1 = d[1];
+      d0 = make_float4(fmaf(aT, cs[0], d0.x), fmaf(aT, cs[1], d0.y), fmaf(aT, cs[2], d0.z),
+                       fmaf(aT, cs[3], d0.w));
+      d1 = make_float4(fmaf(aT, cs[4], d1.x), fmaf(aT, cs[5], d1.y), fmaf(aT, cs[6], d1.z),
+                       fmaf(aT, cs[7], d1.w));
+      d[0] = d0;
+      d[1] = d1;
+    }
+    if (n_thread && n_T) n_T[(long)bh * DK + dk] += aT * ns;
+  }
+}
+
 template <int DK, int DVT>
 cudaError_t launch_states_t(const Problem& p, const void* K, const void* V, const float* C0,
                             const float* n0, Gates g, float* C_states, __nv_bfloat16* Cb,
-                            float* n_states, float* C_T, float* n_T, float* m_T, cudaStream_t st) {
+                            float* n_states, float* C_T, float* n_T, float* m_T, float* seg_ws,
+                            cudaStream_t st) {
   using S = SCfg<DK, DVT>;
   CUtensorMap tk, tv, tcs;
   memset(&tcs, 0, sizeof(tcs));
@@ -450,9 +624,22 @@ cudaError_t launch_states_t(const Problem& p, const void* K, const void* V, cons
   auto kern = tc_states_kernel<DK, DVT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kSmem);
   if (e != cudaSuccess) return e;
-  dim3 grid(p.DV / DVT, p.BH);
+  const int n_seg = tc_states_segments(p);
+  if (n_seg > 1 && !seg_ws) return cudaErrorInvalidValue;
+  float* seg_C = seg_ws;
+  float* seg_n = n_seg > 1 ? seg_ws + (size_t)p.BH * (n_seg - 1) * p.DK * p.DV : nullptr;
+  dim3 grid(p.DV / DVT, p.BH, n_seg);
   kern<<<grid, kThreads, S::kSmem, st>>>(tk, tv, tcs, p, g, C0, n0, C_states, Cb, n_states, C_T,
-                                         n_T, m_T);
+                                         n_T, m_T, seg_C, seg_n);
+  e = cudaGetLastError();
+  if (e != cudaSuccess || n_seg == 1) return e;
+  dim3 fgrid(p.DK * p.DV / 8 / 256, p.BH, n_seg - 1);
+  if (Cb)
+    tc_states_fixup_kernel<true><<<fgrid, 256, 0, st>>>(p, g, DVT, seg_C, seg_n, C_states, Cb,
+                                                        n_states, C_T, n_T);
+  else
+    tc_states_fixup_kernel<false><<<fgrid, 256, 0, st>>>(p, g, DVT, seg_C, seg_n, C_states, Cb,
+                                                         n_states, C_T, n_T);
   return cudaGetLastError();
 }
 
@@ -464,15 +651,37 @@ bool tc_states_supported(const Problem& p) {
          p.L <= 1024 && p.T > 0;
 }
 
+int tc_states_dvt(const Problem& p) { return p.DV >= 256 ? 256 : p.DV; }
+
+int tc_states_segments(const Problem& p) {
+  // Split chunk sequences only while the (b, h, d_v tile) units leave SMs of a
+  // 148-SM B200 idle; at most 8 segments, each at least 2 chunks long.  A
+  // function of the shape alone, so the workspace the host sizes always fits.
+  constexpr int kSMs = 148, kMaxSegments = 8;
+  const int units = p.BH * (p.DV / tc_states_dvt(p));
+  int s = kSMs / units;
+  if (s > kMaxSegments) s = kMaxSegments;
+  if (s > p.NC / 2) s = p.NC / 2;
+  // segment s covers chunks [s * ncs, min((s + 1) * ncs, NC)), ncs = ceil(NC / n):
+  // none may be empty
+  while (s > 1 && (s - 1) * ((p.NC + s - 1) / s) >= p.NC) --s;
+  return s < 1 ? 1 : s;
+}
+
+size_t tc_states_segment_floats(const Problem& p) {
+  const size_t extra = (size_t)tc_states_segments(p) - 1;
+  return extra * p.BH * p.DK * ((size_t)p.DV + 1);
+}
+
 cudaError_t launch_tc_states_impl(const Problem& p, const void* K, const void* V, const float* C0,
                                   const float* n0, Gates g, float* C_states, __nv_bfloat16* Cb,
                                   float* n_states, float* C_T, float* n_T, float* m_T,
-                                  cudaStream_t st) {
-  const int dvt = p.DV >= 256 ? 256 : p.DV;
+                                  float* seg_ws, cudaStream_t st) {
+  const int dvt = tc_states_dvt(p);
 #define MLSTM_ST_CASE(dk, dvt_)                                                                  \
   if (p.DK == dk && dvt == dvt_)                                                                 \
     return launch_states_t<dk, dvt_>(p, K, V, C0, n0, g, C_states, Cb, n_states, C_T, n_T, m_T, \
-                                     st);
+                                     seg_ws, st);
   MLSTM_ST_CASE(128, 64)
   MLSTM_ST_CASE(128, 128)
   MLSTM_ST_CASE(128, 256)
