@@ -31,11 +31,18 @@
 // TMEM (512 columns): the O accumulator at column 0 -- for DVT <= 128 a second
 // one at column 128, used by alternate items so that one item's epilogue
 // overlaps the next item's MMAs -- and two S buffers [128 x 128] at columns
-// 256 and 384.  Shared
-// memory: the Q tile (DK/64 swizzled slabs), a ring of 16 KB slabs as deep as
-// the remaining space allows (7 stages at DK = 256), the bf16 P tile (A
-// operand of P.V), the per-item column weights and n_k.
-// MMA order per item: S_0, Q.C, { S_i, P_{i-1}.V_{i-1} }, P_last.V_last.
+// 256 and 384.  The row threads write each gated P tile back as packed bf16
+// over the S buffer it came from (the half that owns S columns [64h, 64h + 64)
+// writes its 32 packed columns at [64h, 64h + 32), which only it has read), and
+// the P.V MMAs take their A operand from TMEM, so the two S buffers also double
+// buffer P: the gating of key tile i + 1 overlaps the P.V MMA of tile i.  An S
+// buffer is refilled only once the P.V MMA reading it has completed.  Shared
+// memory: the Q tile (DK/64 swizzled slabs), a ring of slabs as deep as the
+// remaining space allows (at DK = 256: 9 stages of 16 KB for value tiles of up
+// to 128 columns, 4 of 32 KB for 256), the per-item column weights and n_k.
+// MMA order per item: S_0, Q.C, { S_i, P_{i-1}.V_{i-1} }, P_last.V_last.  The
+// row threads gate S_0 while Q.C runs, then rescale Q.C to the row frame
+// before releasing P_0, so P_0.V_0 accumulates on the rescaled term.
 #include <cuda.h>
 
 #include "tc.h"
@@ -51,6 +58,7 @@ constexpr int kQT = 128;  // query rows per item
 constexpr int kKT = 128;  // key/value rows per intra tile
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS0 = 256, kColS1 = 384;  // O buffer(s) at columns 0 (and 128)
+constexpr uint32_t kColPHalf = 64;  // P columns of the upper half within an S tile
 constexpr int kMaxL = 1024;  // largest chunk this kernel handles
 
 template <int DK, int DVT>
@@ -64,20 +72,18 @@ struct Cfg {
   static constexpr uint32_t kKSlabBytes = kKT * 128;           // 128 rows x 64 bf16
   static constexpr uint32_t kMNSlabBytes = (DVT / 64) * 8192;  // 64 rows x DVT bf16
   static constexpr uint32_t kStageBytes = kKSlabBytes > kMNSlabBytes ? kKSlabBytes : kMNSlabBytes;
-  static constexpr uint32_t kPBytes = kQT * kKT * 2;
   static constexpr uint32_t kMiscBytes = 2 * kMaxL * 4 + 2 * DK * 4 + 256 * 4 + 512;
   static constexpr uint32_t kBudget = 227 * 1024 - 1024;  // minus alignment slack
-  static constexpr int kStagesFit = (int)((kBudget - kQBytes - kPBytes - kMiscBytes) / kStageBytes);
+  static constexpr int kStagesFit = (int)((kBudget - kQBytes - kMiscBytes) / kStageBytes);
   static constexpr int kStages = kStagesFit > 12 ? 12 : kStagesFit;
   static_assert(kStages >= 3, "ring too shallow");
   static constexpr uint32_t kOffQ = 0;
   static constexpr uint32_t kOffStage = kOffQ + kQBytes;
-  static constexpr uint32_t kOffP = kOffStage + kStages * kStageBytes;
-  static constexpr uint32_t kOffAcol = kOffP + kPBytes;      // float[2][kMaxL]
+  static constexpr uint32_t kOffAcol = kOffStage + kStages * kStageBytes;  // float[2][kMaxL]
   static constexpr uint32_t kOffN = kOffAcol + 2 * kMaxL * 4;  // float[2][DK]
   static constexpr uint32_t kOffRed = kOffN + 2 * DK * 4;      // float[256]
   static constexpr uint32_t kOffBar = kOffRed + 256 * 4;       // barriers
-  static constexpr uint32_t kOffTmemSlot = kOffBar + 360;
+  static constexpr uint32_t kOffTmemSlot = kOffBar + 368;
   static constexpr uint32_t kBytes = kOffTmemSlot + 16;
   static constexpr uint32_t kSmem = kBytes + 1024;  // slack for 1024-byte alignment
   static_assert(kSmem <= 227 * 1024, "shared memory");
@@ -91,14 +97,15 @@ struct Bars {
   __device__ __forceinline__ uint32_t empty(int i) const { return a + 128 + 8 * i; }
   __device__ __forceinline__ uint32_t q_full() const { return a + 256; }
   __device__ __forceinline__ uint32_t q_empty() const { return a + 264; }
+  // per S buffer: S landed, P written over it, P.V read it
   __device__ __forceinline__ uint32_t s_full(int b) const { return a + 272 + 8 * b; }
-  __device__ __forceinline__ uint32_t s_empty(int b) const { return a + 288 + 8 * b; }
-  __device__ __forceinline__ uint32_t inter_done() const { return a + 304; }
-  __device__ __forceinline__ uint32_t p_full() const { return a + 312; }
-  __device__ __forceinline__ uint32_t p_empty() const { return a + 320; }
-  __device__ __forceinline__ uint32_t o_done() const { return a + 328; }
-  __device__ __forceinline__ uint32_t o_empty(int b) const { return a + 336 + 8 * b; }
-  __device__ __forceinline__ uint32_t mma_idle() const { return a + 352; }
+  __device__ __forceinline__ uint32_t p_full(int b) const { return a + 288 + 8 * b; }
+  __device__ __forceinline__ uint32_t pv_done(int b) const { return a + 304 + 8 * b; }
+  __device__ __forceinline__ uint32_t inter_done() const { return a + 320; }
+  // per O buffer: accumulator complete, drained by the epilogue
+  __device__ __forceinline__ uint32_t o_full(int b) const { return a + 328 + 8 * b; }
+  __device__ __forceinline__ uint32_t o_empty(int b) const { return a + 344 + 8 * b; }
+  __device__ __forceinline__ uint32_t mma_idle() const { return a + 360; }
 };
 
 // Work item -> (b*h, query tile, value tile).
@@ -162,14 +169,12 @@ tc_parallel_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     mbar_init(bar.q_empty(), 1 + 256);  // MMA commit + the row threads' reads of Q
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar.s_full(i), 1);
-      mbar_init(bar.s_empty(i), 256);
+      mbar_init(bar.p_full(i), 256);
+      mbar_init(bar.pv_done(i), 1);
+      mbar_init(bar.o_full(i), 1);
+      mbar_init(bar.o_empty(i), 256);
     }
     mbar_init(bar.inter_done(), 1);
-    mbar_init(bar.p_full(), 256);
-    mbar_init(bar.p_empty(), 1);
-    mbar_init(bar.o_done(), 1);
-    mbar_init(bar.o_empty(0), 256);
-    mbar_init(bar.o_empty(1), 256);
     mbar_init(bar.mma_idle(), 1);
     fence_barrier_init();
   }
@@ -251,7 +256,6 @@ tc_parallel_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       bool ok = true;
       int slab = 0;   // ring position
       int tile = 0;   // S tiles issued so far (all items)
-      int ptile = 0;  // P.V tiles issued so far
       auto take = [&]() -> uint32_t {
         const int s = slab % C::kStages, u = slab / C::kStages;
         ok = ok && mbar_wait(bar.full(s), u & 1, p, 5);
@@ -259,9 +263,11 @@ tc_parallel_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         ++slab;
         return (uint32_t)s;
       };
+      // S tile j goes to buffer j & 1, whose previous P (tile j - 2) must have
+      // been read by its P.V MMAs.
       auto mma_s = [&]() {
         const int buf = tile & 1;
-        if (tile >= 2) ok = ok && mbar_wait(bar.s_empty(buf), ((tile >> 1) - 1) & 1, p, 4);
+        if (tile >= 2) ok = ok && mbar_wait(bar.pv_done(buf), ((tile >> 1) - 1) & 1, p, 4);
         tc_fence_after();
         const uint32_t d = tmem + (buf ? kColS1 : kColS0);
         for (int c = 0; c < C::kSlabsK; ++c) {
@@ -279,27 +285,29 @@ tc_parallel_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         ++tile;
       };
       int ob = 0;  // output buffer of the current item
-      auto mma_pv = [&]() {
-        ok = ok && mbar_wait(bar.p_full(), ptile & 1, p, 7);
+      // P_j . V_j with P_j (S tile j, gated) from TMEM.
+      auto mma_pv = [&](int j) {
+        const int buf = j & 1;
+        ok = ok && mbar_wait(bar.p_full(buf), (j >> 1) & 1, p, 7);
         tc_fence_after();
+        const uint32_t aP = tmem + (buf ? kColS1 : kColS0);
         for (int v = 0; v < 2; ++v) {
           const uint32_t s = take();
           if (!ok) return;
-          const uint32_t a0 = sbase + C::kOffP + v * 16384;
           const uint32_t b0 = sbase + C::kOffStage + s * C::kStageBytes;
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            mma_bf16_ss(tmem + ob * 128u, sdesc_sw128(a0 + kk * 32, 16, 1024),
+            mma_bf16_ts(tmem + ob * 128u, aP + (uint32_t)v * kColPHalf + (uint32_t)kk * 8u,
                         sdesc_sw128(b0 + kk * 2048, 8192, 1024), idO, 1);
           mma_commit(bar.empty(s));
         }
-        mma_commit(bar.p_empty());
-        ++ptile;
+        mma_commit(bar.pv_done(buf));
       };
       int n = 0;
       for (int it = item_at(0); it < n_items && ok; it = item_at(n + 1), ++n) {
         const Item x = decode_item(it, p, n_dv, n_q);
         ok = mbar_wait(bar.q_full(), n & 1, p, 3);
+        const int j0 = tile;  // this item's S_0
         if (ok) mma_s();
         // O buffers alternate between items (when there are two): the epilogue
         // of item n - kOBufs must have drained this one.
@@ -322,13 +330,13 @@ tc_parallel_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         mma_commit(bar.inter_done());
         for (int i = 1; i < x.n_kv && ok; ++i) {
           mma_s();
-          if (ok) mma_pv();
+          if (ok) mma_pv(j0 + i - 1);
         }
         if (!ok) break;
         mma_commit(bar.q_empty());  // every MMA that reads Q has been issued
-        mma_pv();
+        mma_pv(j0 + x.n_kv - 1);
         if (!ok) break;
-        mma_commit(bar.o_done());
+        mma_commit(bar.o_full(ob));
       }
       mma_commit(bar.mma_idle());  // completes once every MMA above has finished
       mbar_wait(bar.mma_idle(), 0, p, 15);
@@ -403,34 +411,16 @@ tc_parallel_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       mbar_arrive(bar.q_empty());
       float den = f_inter * dn;
 
-      // Rescale this half of the inter-chunk term to the row frame mu_r.
-      ok = ok && mbar_wait(bar.inter_done(), n & 1, p, 9);
-      tc_fence_after();
-      if (ok) {
-        for (int c = h * kHalfO; c < (h + 1) * kHalfO; c += 64) {
-          uint32_t v0[32], v1[32];
-          tmem_ld32(trow + colO + c, v0);
-          if (kHalfO >= 64) tmem_ld32(trow + colO + c + 32, v1);
-          tmem_wait_ld();
-#pragma unroll
-          for (int j = 0; j < 32; ++j) v0[j] = __float_as_uint(__uint_as_float(v0[j]) * f_inter);
-          tmem_st32(trow + colO + c, v0);
-          if (kHalfO >= 64) {
-#pragma unroll
-            for (int j = 0; j < 32; ++j) v1[j] = __float_as_uint(__uint_as_float(v1[j]) * f_inter);
-            tmem_st32(trow + colO + c + 32, v1);
-          }
-        }
-        tmem_wait_st();
-      }
-
+      // Gated P tiles, written back over their S tiles in TMEM.  P_0 is
+      // released only after this half of the inter-chunk term (Q.C, issued
+      // after S_0) has been rescaled to the row frame mu_r, since P_0.V_0
+      // accumulates on top of it.
       for (int i = 0; i < x.n_kv; ++i, ++tile) {
         const int buf = tile & 1;
         ok = ok && mbar_wait(bar.s_full(buf), (tile >> 1) & 1, p, 10);
-        if (tile >= 1) ok = ok && mbar_wait(bar.p_empty(), (tile - 1) & 1, p, 11);
         tc_fence_after();
         const bool diag = (i == x.n_kv - 1);
-        const uint32_t scol = (buf ? kColS1 : kColS0) + h * 64;
+        const uint32_t scol = (buf ? kColS1 : kColS0) + h * kColPHalf;
         float rs = 0.f;
         if (ok) {
           uint32_t v[64];
@@ -449,18 +439,34 @@ tc_parallel_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             rs += pa + pb;
             pk[j >> 1] = pack_bf16x2(pa, pb);
           }
-          // This half's 64 columns are exactly atom column h of the P tile.
-          uint8_t* prow = smem + C::kOffP + h * 16384;
-#pragma unroll
-          for (int j = 0; j < 8; ++j)
-            *reinterpret_cast<uint4*>(prow + sw128_offset(r, j)) =
-                make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+          tmem_st32(trow + scol, pk);
         }
         den += rs;
+        if (i == 0) {
+          ok = ok && mbar_wait(bar.inter_done(), n & 1, p, 9);
+          tc_fence_after();
+          if (ok) {
+            for (int c = h * kHalfO; c < (h + 1) * kHalfO; c += 64) {
+              uint32_t v0[32], v1[32];
+              tmem_ld32(trow + colO + c, v0);
+              if (kHalfO >= 64) tmem_ld32(trow + colO + c + 32, v1);
+              tmem_wait_ld();
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                v0[j] = __float_as_uint(__uint_as_float(v0[j]) * f_inter);
+              tmem_st32(trow + colO + c, v0);
+              if (kHalfO >= 64) {
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                  v1[j] = __float_as_uint(__uint_as_float(v1[j]) * f_inter);
+                tmem_st32(trow + colO + c + 32, v1);
+              }
+            }
+          }
+        }
+        tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(bar.s_empty(buf));
-        fence_proxy_async_smem();
-        mbar_arrive(bar.p_full());
+        mbar_arrive(bar.p_full(buf));
       }
 
       // Fetch the next item's row values and column data while P.V finishes.
@@ -475,7 +481,7 @@ tc_parallel_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       red_s[rt] = den;
       named_bar_sync(1, 256);
       den += red_s[rt ^ 128];
-      ok = ok && mbar_wait(bar.o_done(), n & 1, p, 12);
+      ok = ok && mbar_wait(bar.o_full(n % C::kOBufs), (n / C::kOBufs) & 1, p, 12);
       tc_fence_after();
       const float mr = bc + mu;
       const float denom = fmaxf(fabsf(den), expf(-mr));
