@@ -30,13 +30,14 @@
 //               term, row sums, epilogue.
 // TMEM (512 columns): the O accumulator at column 0 -- for DVT <= 128 a second
 // one at column 128, used by alternate items so that one item's epilogue
-// overlaps the next item's MMAs -- and two S buffers [128 x 128] at columns
-// 256 and 384.  The row threads write each gated P tile back as packed bf16
-// over the S buffer it came from (the half that owns S columns [64h, 64h + 64)
-// writes its 32 packed columns at [64h, 64h + 32), which only it has read), and
-// the P.V MMAs take their A operand from TMEM, so the two S buffers also double
-// buffer P: the gating of key tile i + 1 overlaps the P.V MMA of tile i.  An S
-// buffer is refilled only once the P.V MMA reading it has completed.  Shared
+// overlaps the next item's MMAs -- one S tile [128 x 128] at column 256 and two
+// P buffers of 64 columns at 384 and 448.  The row threads load S_i, release
+// the S buffer at once (so S_{i+1} is computed while they gate S_i), and write
+// the gated tile as packed bf16 into P buffer i mod 2 (the half that owns keys
+// [64h, 64h + 64) writes 32 packed columns at 32h), once the P.V MMA that read
+// that buffer two tiles earlier has completed.  The P.V MMAs take their A
+// operand from TMEM, so the gating of key tile i + 1 overlaps the P.V MMA of
+// tile i and no MMA waits for another to complete.  Shared
 // memory: the Q tile (DK/64 swizzled slabs), a ring of slabs as deep as the
 // remaining space allows (at DK = 256: 9 stages of 16 KB for value tiles of up
 // to 128 columns, 4 of 32 KB for 256), the per-item column weights and n_k.
@@ -57,8 +58,9 @@ constexpr int kThreads = 320;
 constexpr int kQT = 128;  // query rows per item
 constexpr int kKT = 128;  // key/value rows per intra tile
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS0 = 256, kColS1 = 384;  // O buffer(s) at columns 0 (and 128)
-constexpr uint32_t kColPHalf = 64;  // P columns of the upper half within an S tile
+constexpr uint32_t kColS = 256;                 // O buffer(s) at columns 0 (and 128)
+constexpr uint32_t kColP0 = 384, kColP1 = 448;  // two P buffers of 64 packed columns
+constexpr uint32_t kColPHalf = 32;              // P columns of the upper key half
 constexpr int kMaxL = 1024;  // largest chunk this kernel handles
 
 template <int DK, int DVT>
@@ -97,8 +99,9 @@ struct Bars {
   __device__ __forceinline__ uint32_t empty(int i) const { return a + 128 + 8 * i; }
   __device__ __forceinline__ uint32_t q_full() const { return a + 256; }
   __device__ __forceinline__ uint32_t q_empty() const { return a + 264; }
-  // per S buffer: S landed, P written over it, P.V read it
-  __device__ __forceinline__ uint32_t s_full(int b) const { return a + 272 + 8 * b; }
+  // the S tile landed / was read; per P buffer: P written, P.V read it
+  __device__ __forceinline__ uint32_t s_full() const { return a + 272; }
+  __device__ __forceinline__ uint32_t s_empty() const { return a + 280; }
   __device__ __forceinline__ uint32_t p_full(int b) const { return a + 288 + 8 * b; }
   __device__ __forceinline__ uint32_t pv_done(int b) const { return a + 304 + 8 * b; }
   __device__ __forceinline__ uint32_t inter_done() const { return a + 320; }
@@ -167,8 +170,9 @@ tc_parallel_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     }
     mbar_init(bar.q_full(), 1);
     mbar_init(bar.q_empty(), 1 + 256);  // MMA commit + the row threads' reads of Q
+    mbar_init(bar.s_full(), 1);
+    mbar_init(bar.s_empty(), 256);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(bar.s_full(i), 1);
       mbar_init(bar.p_full(i), 256);
       mbar_init(bar.pv_done(i), 1);
       mbar_init(bar.o_full(i), 1);
@@ -263,13 +267,11 @@ tc_parallel_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         ++slab;
         return (uint32_t)s;
       };
-      // S tile j goes to buffer j & 1, whose previous P (tile j - 2) must have
-      // been read by its P.V MMAs.
+      // S tile j overwrites tile j - 1, which the row threads must have loaded.
       auto mma_s = [&]() {
-        const int buf = tile & 1;
-        if (tile >= 2) ok = ok && mbar_wait(bar.pv_done(buf), ((tile >> 1) - 1) & 1, p, 4);
+        if (tile >= 1) ok = ok && mbar_wait(bar.s_empty(), (tile - 1) & 1, p, 4);
         tc_fence_after();
-        const uint32_t d = tmem + (buf ? kColS1 : kColS0);
+        const uint32_t d = tmem + kColS;
         for (int c = 0; c < C::kSlabsK; ++c) {
           const uint32_t s = take();
           if (!ok) return;
@@ -281,16 +283,16 @@ tc_parallel_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                         idS, (c | kk) != 0);
           mma_commit(bar.empty(s));
         }
-        mma_commit(bar.s_full(buf));
+        mma_commit(bar.s_full());
         ++tile;
       };
       int ob = 0;  // output buffer of the current item
-      // P_j . V_j with P_j (S tile j, gated) from TMEM.
+      // P_j . V_j with P_j (S tile j, gated) from P buffer j mod 2.
       auto mma_pv = [&](int j) {
         const int buf = j & 1;
         ok = ok && mbar_wait(bar.p_full(buf), (j >> 1) & 1, p, 7);
         tc_fence_after();
-        const uint32_t aP = tmem + (buf ? kColS1 : kColS0);
+        const uint32_t aP = tmem + (buf ? kColP1 : kColP0);
         for (int v = 0; v < 2; ++v) {
           const uint32_t s = take();
           if (!ok) return;
@@ -359,36 +361,54 @@ tc_parallel_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     int tile = 0;
     int n = 0;
 
-    // Per-item values, fetched one item ahead.
-    auto fetch_rows = [&](const Item& x, float& m_in, float& amax, float& bc) {
-      const int t = x.t0 + r;
-      m_in = g.mchk[(long)x.bh * (p.NC + 1) + x.k];
-      amax = g.amax[(long)x.bh * tpad + t];
-      bc = g.bcum[(long)x.bh * tpad + t];
+    // Per-item values, fetched one item ahead.  The exponent of P splits as
+    //   e^{acol_s - mu_r} = e^{acol_s - c} e^{c - mu_r},
+    // c = the largest column weight of the item's keys (amax of its last row,
+    // amax being a running maximum), so the column factor is at most 1.  When
+    // the row factor stays below e^60 for every row of the tile (sep), P costs
+    // two multiplies per element; otherwise the column data holds acol log2(e)
+    // and each element takes its own exponential.
+    struct RowVals {
+      float m_in, amax, bc, c;
+      bool sep;
     };
-    auto fetch_cols = [&](const Item& x, int buf) {
+    auto fetch_rows = [&](const Item& x) -> RowVals {
+      RowVals v;
+      const long base = (long)x.bh * tpad;
+      v.m_in = g.mchk[(long)x.bh * (p.NC + 1) + x.k];
+      v.amax = g.amax[base + x.t0 + r];
+      v.bc = g.bcum[base + x.t0 + r];
+      v.c = g.amax[base + x.t0 + kQT - 1];
+      v.sep = v.c - fmaxf(v.m_in, g.amax[base + x.t0]) <= 60.f;  // uniform over the CTA
+      return v;
+    };
+    auto fetch_cols = [&](const Item& x, int buf, const RowVals& v) {
       float* ac = acol_s + buf * kMaxL;
       float* nn = n_s + buf * DK;
-      for (int j = rt; j < x.n_kv * kKT; j += 256)
-        ac[j] = g.acol[(long)x.bh * tpad + x.c0 + j] * 1.4426950408889634f;
+      for (int j = rt; j < x.n_kv * kKT; j += 256) {
+        const float a = g.acol[(long)x.bh * tpad + x.c0 + j];
+        ac[j] = v.sep ? expf(a - v.c) : a * 1.4426950408889634f;  // -inf -> 0 / -inf
+      }
       for (int j = rt; j < DK; j += 256) nn[j] = n_states[((long)x.bh * p.NC + x.k) * DK + j];
     };
-    float nx_m_in = 0.f, nx_amax = 0.f, nx_bc = 0.f;
+    RowVals nx{0.f, 0.f, 0.f, 0.f, false};
     if (blockIdx.x < n_items) {
       const Item x0 = decode_item(blockIdx.x, p, n_dv, n_q);
-      fetch_rows(x0, nx_m_in, nx_amax, nx_bc);
-      fetch_cols(x0, 0);
+      nx = fetch_rows(x0);
+      fetch_cols(x0, 0, nx);
     }
     for (int it = item_at(0); it < n_items && ok; it = item_at(n + 1), ++n) {
       const Item x = decode_item(it, p, n_dv, n_q);
       const int t = x.t0 + r;
-      const float m_in = nx_m_in, amax = nx_amax, bc = nx_bc;
+      const RowVals rv = nx;
+      const float bc = rv.bc;
       const float* ac = acol_s + (n & 1) * kMaxL;
       const uint32_t colO = (uint32_t)(n % C::kOBufs) * 128u;
       const float* nn = n_s + (n & 1) * DK;
-      const float mu = fmaxf(m_in, amax);
+      const float mu = fmaxf(rv.m_in, rv.amax);
       const float mu2 = mu * 1.4426950408889634f;
-      const float f_inter = expf(m_in - mu);
+      const float f_inter = expf(rv.m_in - mu);
+      const float rowf = rv.sep ? ks * expf(rv.c - mu) : 0.f;
       named_bar_sync(1, 256);  // this item's column data is in shared memory
 
       // Partial den_inter = q_r . n_k over this half's slabs; then release Q.
@@ -417,29 +437,48 @@ tc_parallel_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       // accumulates on top of it.
       for (int i = 0; i < x.n_kv; ++i, ++tile) {
         const int buf = tile & 1;
-        ok = ok && mbar_wait(bar.s_full(buf), (tile >> 1) & 1, p, 10);
+        ok = ok && mbar_wait(bar.s_full(), tile & 1, p, 10);
         tc_fence_after();
         const bool diag = (i == x.n_kv - 1);
-        const uint32_t scol = (buf ? kColS1 : kColS0) + h * kColPHalf;
+        const uint32_t scol = kColS + h * 64;
+        const uint32_t pcol = (buf ? kColP1 : kColP0) + h * kColPHalf;
         float rs = 0.f;
-        if (ok) {
+        {
           uint32_t v[64];
           tmem_ld32(trow + scol, *reinterpret_cast<uint32_t(*)[32]>(v));
           tmem_ld32(trow + scol + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
           tmem_wait_ld();
+          tc_fence_before();
+          mbar_arrive(bar.s_empty());  // S is in registers: the next S may land
           uint32_t pk[32];
           const float* acl = ac + i * kKT + h * 64;
+          if (rv.sep) {
 #pragma unroll
-          for (int j = 0; j < 64; j += 2) {
-            const int s0 = h * 64 + j;  // key/value index within the tile
-            float pa = __uint_as_float(v[j]) * ks * ex2_approx(acl[j] - mu2);
-            float pb = __uint_as_float(v[j + 1]) * ks * ex2_approx(acl[j + 1] - mu2);
-            if (diag && s0 > r) pa = 0.f;
-            if (diag && s0 + 1 > r) pb = 0.f;
-            rs += pa + pb;
-            pk[j >> 1] = pack_bf16x2(pa, pb);
+            for (int j = 0; j < 64; j += 2) {
+              const int s0 = h * 64 + j;  // key/value index within the tile
+              float pa = __uint_as_float(v[j]) * acl[j] * rowf;
+              float pb = __uint_as_float(v[j + 1]) * acl[j + 1] * rowf;
+              if (diag && s0 > r) pa = 0.f;
+              if (diag && s0 + 1 > r) pb = 0.f;
+              rs += pa + pb;
+              pk[j >> 1] = pack_bf16x2(pa, pb);
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 64; j += 2) {
+              const int s0 = h * 64 + j;
+              float pa = __uint_as_float(v[j]) * ks * ex2_approx(acl[j] - mu2);
+              float pb = __uint_as_float(v[j + 1]) * ks * ex2_approx(acl[j + 1] - mu2);
+              if (diag && s0 > r) pa = 0.f;
+              if (diag && s0 + 1 > r) pb = 0.f;
+              rs += pa + pb;
+              pk[j >> 1] = pack_bf16x2(pa, pb);
+            }
           }
-          tmem_st32(trow + scol, pk);
+          // P buffer buf was last read by the P.V MMAs of tile - 2
+          if (tile >= 2) ok = ok && mbar_wait(bar.pv_done(buf), ((tile >> 1) - 1) & 1, p, 11);
+          tc_fence_after();
+          tmem_st32(trow + pcol, pk);
         }
         den += rs;
         if (i == 0) {
@@ -473,8 +512,8 @@ tc_parallel_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       const int it_next = item_at(n + 1);
       if (it_next < n_items) {
         const Item xn = decode_item(it_next, p, n_dv, n_q);
-        fetch_rows(xn, nx_m_in, nx_amax, nx_bc);
-        fetch_cols(xn, (n + 1) & 1);
+        nx = fetch_rows(xn);
+        fetch_cols(xn, (n + 1) & 1, nx);
       }
 
       // Epilogue: combine the two halves' denominators, h = O / max(|den|, e^{-m_r}).

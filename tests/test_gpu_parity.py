@@ -227,3 +227,28 @@ def test_fp32_path_is_tight():
         H, fin = run(w, x, "auto")
         ref = parity.oracle_run(x, w.gate_mode)
         parity.compare(H, fin, ref, 1e-4, label=f"f32 T{T} L{L}")
+
+
+@pytest.mark.parametrize("T,L,spikes", [(512, 128, (400, 470)), (512, 256, (300, 470)),
+                                        (1536, 512, (1100, 1300))])
+def test_input_gate_spikes(T, L, spikes):
+    """Input-gate spikes (+70) inside a query tile push the row stabilisers of
+    the later rows some e^70 above the first row's, past the range where the
+    gate exponent splits into a column and a row factor: the kernels fall back
+    to one exponential per element there and must still match the oracle.
+
+    The spikes sit in the last chunk.  A spike in an earlier chunk leaves every
+    later chunk state dominated by one token (rank one), and then
+    h = C q / |n.q| is ill-conditioned on the rows where q.k is small: the bf16
+    operand copy of C that the inter-chunk tensor-core product reads rounds
+    each entry by up to 2^-9 of |k_j v_d|, which such rows amplify by
+    |q||k| / |q.k| (measured: 7.5% on the worst row at T=512, L=128)."""
+    w = WORKLOADS["mid"].replace(name="spikes", B=1, NH=2, T=T, chunk_size=L)
+    x = make_inputs(w)
+    for t in spikes:
+        x["i_pre"][:, :, t] = 70.0
+    ref = parity.oracle_run(x, w.gate_mode)
+    for algo in ALGOS:
+        if supported(w, algo):
+            H, fin = run(w, x, algo)
+            parity.compare(H, fin, ref, parity.TOL[w.dtype], label=f"spikes L{L}/{algo}")
