@@ -82,7 +82,11 @@ typedef enum { MLSTM_GATE_EXP = 0, MLSTM_GATE_SIGMOID = 1 } mlstm_gate_mode;
  *             chunk goes to the workspace (as a bf16 operand copy plus fp32
  *             n) between the state and the output kernels.  Needs d_qk of
  *             128 or 256, d_v of 128 or a multiple of 256 (up to 1024), and a
- *             chunk size that is a multiple of 128 up to 1024.
+ *             chunk size that is a multiple of 128 up to 1024, or 64 with
+ *             d_qk = 128 (two chunks per 128-row query tile).  With few
+ *             (b, h) pairs the state kernel splits each sequence into
+ *             segments and adds a fix-up launch; the workspace then also
+ *             holds the segments' end states.
  *   TC_FUSED  bf16 tensor-core kernel that carries the chunk state on chip
  *             ("Upgrade roadmap" item 2 of the flash-xlstm-exp page): d_qk =
  *             128, d_v of 64 or 128, chunk size 128. */

@@ -81,7 +81,8 @@ bool encode_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64
 bool tc_unfused_supported(const Problem& p) {
   // The chunk-state kernel writes the operand copy in 64-column blocks, one
   // warp per 32 x 64 tile, which needs at least 128 value columns per CTA.
-  return tc_states_supported(p) && tc_parallel_supported(p) && p.DV % 128 == 0;
+  return tc_states_supported(p) && (tc_parallel_supported(p) || tc_parallel_wide_supported(p)) &&
+         p.DV % 128 == 0;
 }
 
 cudaError_t launch_tc_states(const Problem& p, const void* K, const void* V, const float* C0,

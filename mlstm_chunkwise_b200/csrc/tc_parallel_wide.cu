@@ -34,6 +34,15 @@
 // The half of the row threads that owns S columns [64h, 64h + 64) writes its
 // 64 bf16 P values (32 packed columns) to columns [64h, 64h + 32), which only
 // it has read, so the halves never race.
+// Chunks of 64 tokens (kPair): a 128-row query tile holds two chunks, 2j and
+// 2j + 1.  S covers both, and P is masked to the causal pairs within each chunk
+// (block diagonal).  The two halves of the tile need different chunk states,
+// so the inter-chunk product runs over a K-stacked operand,
+//   [Q~ masked to chunk 2j | Q~ masked to chunk 2j + 1] . [C_2j ; C_2j+1],
+// which is one accumulation into the same O: the row threads write their
+// scaled Q row into its chunk's half of a double-width Q buffer and zeros into
+// the other half.
+//
 // MMA order per item: S_0 [, S_1], then for every value tile d:
 // P_0.V_0[:, d] [, P_1.V_1[:, d]], (first tile: wait for the scaled Q),
 // Q~.C_k[:, d].  S_i of the next item waits until the last P_i.V_i MMA of
@@ -56,17 +65,21 @@ constexpr uint32_t kColPHalf = 64;  // P columns of the upper half within an S t
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS0 = 256, kColS1 = 384;
 
-template <int DK, int DVT>
+template <int DK, int DVT, bool kPair>
 struct WCfg {
   static_assert(DVT == 64 || DVT == 128, "value tile of 64 or 128 columns");
+  static_assert(!kPair || DK <= 128, "pairs of 64-token chunks: d_qk up to 128");
+  static constexpr int kChunks = kPair ? 2 : 1;  // chunks per query tile
   static constexpr int kSlabsK = DK / 64;
-  static constexpr uint32_t kQBytes = kQT * DK * 2;
+  static constexpr uint32_t kQLoadBytes = kQT * DK * 2;
+  static constexpr uint32_t kQBytes = kChunks * kQLoadBytes;  // kPair: the stacked Q~ operand
   static constexpr uint32_t kKSlabBytes = kKT * 128;
   static constexpr uint32_t kMNSlabBytes = (DVT / 64) * 8192;
   static constexpr uint32_t kStageBytes = 16384;
   static_assert(kKSlabBytes <= kStageBytes && kMNSlabBytes <= kStageBytes, "stage size");
   static constexpr uint32_t kOutBytes = kQT * DVT * 2;  // output staging tile
-  static constexpr uint32_t kMiscBytes = 2 * kPSlots * kKT * 4 + 2 * DK * 4 + 256 * 4 + 512;
+  static constexpr uint32_t kMiscBytes =
+      2 * kPSlots * kKT * 4 + 2 * kChunks * DK * 4 + 256 * 4 + 512;
   static constexpr uint32_t kBudget = 227 * 1024 - 1024;
   static constexpr int kStagesFit =
       (int)((kBudget - kQBytes - kOutBytes - kMiscBytes) / kStageBytes);
@@ -76,8 +89,8 @@ struct WCfg {
   static constexpr uint32_t kOffOut = kOffQ + kQBytes;
   static constexpr uint32_t kOffStage = kOffOut + kOutBytes;
   static constexpr uint32_t kOffAcol = kOffStage + kStages * kStageBytes;  // float[2][256]
-  static constexpr uint32_t kOffN = kOffAcol + 2 * kPSlots * kKT * 4;       // float[2][DK]
-  static constexpr uint32_t kOffRed = kOffN + 2 * DK * 4;                   // float[256]
+  static constexpr uint32_t kOffN = kOffAcol + 2 * kPSlots * kKT * 4;  // float[2][kChunks][DK]
+  static constexpr uint32_t kOffRed = kOffN + 2 * kChunks * DK * 4;    // float[256]
   static constexpr uint32_t kOffBar = kOffRed + 256 * 4;
   static constexpr uint32_t kOffTmemSlot = kOffBar + 384;
   static constexpr uint32_t kBytes = kOffTmemSlot + 16;
@@ -129,7 +142,7 @@ __device__ __forceinline__ int item_at(int k) {
   return k * G + ((G & 1) ? c : (c ^ (k & 1)));
 }
 
-template <int DK, int DVT>
+template <int DK, int DVT, bool kPair>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_parallel_wide_kernel(const __grid_constant__ CUtensorMap tm_q,
                         const __grid_constant__ CUtensorMap tm_k,
@@ -138,7 +151,7 @@ tc_parallel_wide_kernel(const __grid_constant__ CUtensorMap tm_q,
                         const __grid_constant__ CUtensorMap tm_h, Problem p, Gates g,
                         const float* __restrict__ n_states,
                         float* __restrict__ n_out, float* __restrict__ m_out, int n_items) {
-  using C = WCfg<DK, DVT>;
+  using C = WCfg<DK, DVT, kPair>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -201,7 +214,7 @@ tc_parallel_wide_kernel(const __grid_constant__ CUtensorMap tm_q,
         const WItem x = decode_witem(it, p, n_q);
         if (n > 0) ok = mbar_wait(bar.q_empty(), (n - 1) & 1, p, 2);
         if (!ok) break;
-        mbar_expect_tx(bar.q_full(), C::kQBytes);
+        mbar_expect_tx(bar.q_full(), C::kQLoadBytes);
         for (int c = 0; c < C::kSlabsK; ++c)
           tma_load_3d(sbase + C::kOffQ + c * 16384, &tm_q, c * 64, x.t0, x.bh, bar.q_full());
         for (int i = 0; i < x.n_kv && ok; ++i)
@@ -219,12 +232,16 @@ tc_parallel_wide_kernel(const __grid_constant__ CUtensorMap tm_q,
                 tma_load_3d(dst + b * 8192, &tm_v, dv0 + b * 64, x.c0 + i * kKT + v * 64, x.bh,
                             bar.full((slab - 1) % C::kStages));
             }
-          for (int c = 0; c < C::kSlabsK && ok; ++c) {  // C_k rows [64c, 64c + 64)
+          // C_k rows [64c, 64c + 64) (kPair: then those of chunk k + 1, or of
+          // chunk k again past the last chunk, where the zero half of the
+          // stacked Q~ operand meets them)
+          for (int c = 0; c < C::kChunks * C::kSlabsK && ok; ++c) {
+            const int kc = x.k + c / C::kSlabsK < p.NC ? x.k + c / C::kSlabsK : p.NC - 1;
             const uint32_t dst = next_stage(C::kMNSlabBytes);
             for (int b = 0; b < DVT / 64; ++b)
               bulk_load(dst + b * 8192,
-                        Cb + cb_block_row((long)x.bh * p.NC + x.k, dv0 / 64 + b, c * 64, DK,
-                                          p.DV / 64),
+                        Cb + cb_block_row((long)x.bh * p.NC + kc, dv0 / 64 + b,
+                                          (c % C::kSlabsK) * 64, DK, p.DV / 64),
                         8192, bar.full((slab - 1) % C::kStages));
           }
         }
@@ -297,7 +314,7 @@ tc_parallel_wide_kernel(const __grid_constant__ CUtensorMap tm_q,
             ok = mbar_wait(bar.q_scaled(), n & 1, p, 7);  // Q rows scaled in place
             tc_fence_after();
           }
-          for (int c = 0; c < C::kSlabsK && ok; ++c) {  // Q~ . C_k[:, d]
+          for (int c = 0; c < C::kChunks * C::kSlabsK && ok; ++c) {  // Q~ . C_k[:, d]
             const uint32_t s = take();
             if (!ok) break;
             const uint32_t a0 = sbase + C::kOffQ + c * 16384;
@@ -329,18 +346,25 @@ tc_parallel_wide_kernel(const __grid_constant__ CUtensorMap tm_q,
     bool ok = true;
     int dcount = 0;
     int pc0 = 0, pc1 = 0;  // times S tile 0 / 1 has been turned into P
+    // kPair: rows 64..127 belong to chunk k + 1 (past the last chunk they are
+    // past T, and chunk k stands in)
+    const int rchunk = kPair && r >= 64 ? 1 : 0;
+    auto chunk_of = [&](const WItem& x, int part) {
+      return x.k + part < p.NC ? x.k + part : p.NC - 1;
+    };
     auto fetch_rows = [&](const WItem& x, float& m_in, float& amax, float& bc) {
       const int t = x.t0 + r;
-      m_in = g.mchk[(long)x.bh * (p.NC + 1) + x.k];
+      m_in = g.mchk[(long)x.bh * (p.NC + 1) + chunk_of(x, rchunk)];
       amax = g.amax[(long)x.bh * tpad + t];
       bc = g.bcum[(long)x.bh * tpad + t];
     };
     auto fetch_cols = [&](const WItem& x, int buf) {
       float* ac = acol_s + buf * kPSlots * kKT;
-      float* nn = n_s + buf * DK;
+      float* nn = n_s + buf * C::kChunks * DK;
       for (int j = rt; j < x.n_kv * kKT; j += 256)
         ac[j] = g.acol[(long)x.bh * tpad + x.c0 + j] * 1.4426950408889634f;
-      for (int j = rt; j < DK; j += 256) nn[j] = n_states[((long)x.bh * p.NC + x.k) * DK + j];
+      for (int j = rt; j < C::kChunks * DK; j += 256)
+        nn[j] = n_states[((long)x.bh * p.NC + chunk_of(x, j / DK)) * DK + j % DK];
     };
     float nx_m_in = 0.f, nx_amax = 0.f, nx_bc = 0.f;
     if (blockIdx.x < n_items) {
@@ -354,7 +378,7 @@ tc_parallel_wide_kernel(const __grid_constant__ CUtensorMap tm_q,
       const int t = x.t0 + r;
       const float m_in = nx_m_in, amax = nx_amax, bc = nx_bc;
       const float* ac = acol_s + (n & 1) * kPSlots * kKT;
-      const float* nn = n_s + (n & 1) * DK;
+      const float* nn = n_s + ((n & 1) * C::kChunks + rchunk) * DK;
       const float mu = fmaxf(m_in, amax);
       const float mu2 = mu * 1.4426950408889634f;
       const float f_inter = expf(m_in - mu);
@@ -401,6 +425,7 @@ tc_parallel_wide_kernel(const __grid_constant__ CUtensorMap tm_q,
             float pb = __uint_as_float(v[j + 1]) * ks * ex2_approx(acl[j + 1] - mu2);
             if (diag && s0 > r) pa = 0.f;
             if (diag && s0 + 1 > r) pb = 0.f;
+            if (kPair && ((s0 ^ r) & 64)) pa = pb = 0.f;  // key and query in different chunks
             rs += pa + pb;
             pk[j >> 1] = pack_bf16x2(pa, pb);
           }
@@ -414,21 +439,25 @@ tc_parallel_wide_kernel(const __grid_constant__ CUtensorMap tm_q,
       }
 
       // Every S MMA of this item has completed (the waits above): scale this
-      // half of the Q row by e^{m_k - mu_r} in place for the inter-chunk MMAs.
+      // half of the Q row by e^{m_k - mu_r} in place for the inter-chunk MMAs
+      // (kPair: into the row's chunk half of the stacked operand, zeros into
+      // the other half).
       if (ok) {
         for (int c = h * kSlabsPerHalf; c < C::kSlabsK && c < (h + 1) * kSlabsPerHalf; ++c) {
           uint8_t* slab_ptr = smem + C::kOffQ + c * 16384;
+          uint8_t* dst_ptr = slab_ptr + rchunk * C::kSlabsK * 16384;
+          uint8_t* zero_ptr = slab_ptr + (1 - rchunk) * C::kSlabsK * 16384;
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
-            uint4* ptr = reinterpret_cast<uint4*>(slab_ptr + sw128_offset(r, j));
-            uint4 u = *ptr;
+            uint4 u = *reinterpret_cast<const uint4*>(slab_ptr + sw128_offset(r, j));
             __nv_bfloat162* h2 = reinterpret_cast<__nv_bfloat162*>(&u);
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               const float2 f2 = __bfloat1622float2(h2[e]);
               h2[e] = __floats2bfloat162_rn(f2.x * f_inter, f2.y * f_inter);
             }
-            *ptr = u;
+            *reinterpret_cast<uint4*>(dst_ptr + sw128_offset(r, j)) = u;
+            if (kPair) *reinterpret_cast<uint4*>(zero_ptr + sw128_offset(r, j)) = make_uint4(0, 0, 0, 0);
           }
         }
       }
@@ -510,18 +539,18 @@ tc_parallel_wide_kernel(const __grid_constant__ CUtensorMap tm_q,
   }
 }
 
-template <int DK, int DVT>
+template <int DK, int DVT, bool kPair>
 cudaError_t launch_wide_t(const Problem& p, const void* Q, const void* K, const void* V, Gates g,
                           const __nv_bfloat16* Cb, const float* n_states, void* H, float* n_out,
                           float* m_out, cudaStream_t st) {
-  using C = WCfg<DK, DVT>;
+  using C = WCfg<DK, DVT, kPair>;
   CUtensorMap tq, tk, tv, th;
   if (!encode_tmap_bf16_3d(&tq, Q, p.DK, p.T, p.BH, 64, kQT) ||
       !encode_tmap_bf16_3d(&tk, K, p.DK, p.T, p.BH, 64, kKT) ||
       !encode_tmap_bf16_3d(&tv, V, p.DV, p.T, p.BH, 64, 64) ||
       !encode_tmap_bf16_3d(&th, H, p.DV, p.T, p.BH, 64, kQT))
     return cudaErrorInvalidValue;
-  auto kern = tc_parallel_wide_kernel<DK, DVT>;
+  auto kern = tc_parallel_wide_kernel<DK, DVT, kPair>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 0;
@@ -542,22 +571,28 @@ cudaError_t launch_wide_t(const Problem& p, const void* Q, const void* K, const 
 bool tc_parallel_wide_supported(const Problem& p) {
   const bool dk_ok = p.DK == 64 || p.DK == 128 || p.DK == 256;
   const bool dv_ok = p.DV == 64 || p.DV % 128 == 0;
-  return dk_ok && dv_ok && p.DV <= 1024 && p.L % kKT == 0 && p.L <= kPSlots * kKT && p.T > 0;
+  const bool l_ok = (p.L % kKT == 0 && p.L <= kPSlots * kKT) || (p.L == 64 && p.DK <= 128);
+  return dk_ok && dv_ok && p.DV <= 1024 && l_ok && p.T > 0;
 }
 
 cudaError_t launch_tc_parallel_wide(const Problem& p, const void* Q, const void* K, const void* V,
                                     Gates g, const __nv_bfloat16* Cb, const float* n_states,
                                     void* H, float* n_out, float* m_out, cudaStream_t st) {
   const int dvt = p.DV >= 128 ? 128 : 64;
-#define MLSTM_WIDE_CASE(dk, dvt_)                                                             \
-  if (p.DK == dk && dvt == dvt_)                                                              \
-    return launch_wide_t<dk, dvt_>(p, Q, K, V, g, Cb, n_states, H, n_out, m_out, st);
-  MLSTM_WIDE_CASE(64, 64)
-  MLSTM_WIDE_CASE(64, 128)
-  MLSTM_WIDE_CASE(128, 64)
-  MLSTM_WIDE_CASE(128, 128)
-  MLSTM_WIDE_CASE(256, 64)
-  MLSTM_WIDE_CASE(256, 128)
+  const bool pair = p.L == 64;
+#define MLSTM_WIDE_CASE(dk, dvt_, pair_)                                                      \
+  if (p.DK == dk && dvt == dvt_ && pair == pair_)                                             \
+    return launch_wide_t<dk, dvt_, pair_>(p, Q, K, V, g, Cb, n_states, H, n_out, m_out, st);
+  MLSTM_WIDE_CASE(64, 64, false)
+  MLSTM_WIDE_CASE(64, 128, false)
+  MLSTM_WIDE_CASE(128, 64, false)
+  MLSTM_WIDE_CASE(128, 128, false)
+  MLSTM_WIDE_CASE(256, 64, false)
+  MLSTM_WIDE_CASE(256, 128, false)
+  MLSTM_WIDE_CASE(64, 64, true)
+  MLSTM_WIDE_CASE(64, 128, true)
+  MLSTM_WIDE_CASE(128, 64, true)
+  MLSTM_WIDE_CASE(128, 128, true)
 #undef MLSTM_WIDE_CASE
   return cudaErrorNotSupported;
 }

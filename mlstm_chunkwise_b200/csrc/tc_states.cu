@@ -647,7 +647,7 @@ cudaError_t launch_states_t(const Problem& p, const void* K, const void* V, cons
 
 bool tc_states_supported(const Problem& p) {
   const bool dv_ok = p.DV == 64 || p.DV == 128 || p.DV % 256 == 0;
-  return (p.DK == 128 || p.DK == 256) && dv_ok && p.DV <= 1024 && p.L % 128 == 0 &&
+  return (p.DK == 128 || p.DK == 256) && dv_ok && p.DV <= 1024 && p.L % kStageTok == 0 &&
          p.L <= 1024 && p.T > 0;
 }
 

@@ -91,9 +91,9 @@ def test_workload_full_size_sampled_heads(name):
     assert torch.isfinite(H).all()
 
 
-@pytest.mark.parametrize("T", [1024, 65536])
-def test_sweep_full_size_sampled_heads(T):
-    w = sweep_workload(T, 256)
+@pytest.mark.parametrize("T,L", [(1024, 256), (65536, 256), (1024, 64), (65536, 64)])
+def test_sweep_full_size_sampled_heads(T, L):
+    w = sweep_workload(T, L)
     x = make_inputs(w)
     H, fin = run(w, x, "auto")
     heads = [(0, 0), (w.B - 1, w.NH - 1)]
@@ -252,3 +252,19 @@ def test_input_gate_spikes(T, L, spikes):
         if supported(w, algo):
             H, fin = run(w, x, algo)
             parity.compare(H, fin, ref, parity.TOL[w.dtype], label=f"spikes L{L}/{algo}")
+
+
+@pytest.mark.parametrize("T,DK,DV,init", [(960, 128, 128, False), (1000, 128, 128, True),
+                                         (300, 128, 256, True), (64, 128, 128, False)])
+def test_chunk64_pairs(T, DK, DV, init):
+    """64-token chunks on the tensor-core path: two chunks per 128-row query
+    tile with a block-diagonal causal mask and a K-stacked inter-chunk operand;
+    odd chunk counts (the last tile's second chunk past T), ragged tails and an
+    initial state."""
+    w = WORKLOADS["mid"].replace(name="chunk64", B=1, NH=2, T=T, DK=DK, DV=DV, chunk_size=64,
+                                 init_state=init)
+    assert supported(w, "tc")
+    x = make_inputs(w)
+    ref = parity.oracle_run(x, w.gate_mode)
+    H, fin = run(w, x, "tc")
+    parity.compare(H, fin, ref, parity.TOL[w.dtype], label=f"chunk64 T{T} d{DK}/{DV}")
