@@ -582,6 +582,124 @@ def run_ours(args):
     return 0
 
 
+# ----------------------------------------------------------------------------
+# single-token step (decode) at a workload's B, NH, d_qk, d_v
+# ----------------------------------------------------------------------------
+STEP_METRIC = "mLSTM single-token step tokens/s (one token per sequence per step)"
+
+
+def step_bytes(B, NH, DK, DV, elem):
+    """Algorithmic bytes of one step: the fp32 state (C, n, m) read and written
+    once, q, k, v, h and the two gate pre-activations moved once."""
+    state = B * NH * (DK * DV + DK + 1) * 4
+    return 2 * state + B * NH * ((2 * DK + 2 * DV) * elem + 2 * 4)
+
+
+def run_step(args):
+    import ctypes
+
+    import torch
+
+    import oracle
+    from mlstm_chunkwise_b200 import _lib, api
+    from mlstm_chunkwise_b200 import build as libbuild
+
+    if libbuild.needs_build():
+        libbuild.build()
+    if int(os.environ.get("WORLD_SIZE", "1")) != 1 or args.gpus != 1:
+        raise SystemExit("--op step runs on one GPU")
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    w = pick_workload(args.workload)
+    B = args.batch or w.B
+    NH, DK, DV, dt = w.NH, w.DK, w.DV, w.torch_dtype
+    elem = 2 if w.dtype == "bf16" else 4
+    g = torch.Generator().manual_seed(rank_seed(w, 0))
+    n_tok = args.steps + max(3, args.warmup)
+    tok = {"q": torch.randn((n_tok, B, NH, DK), generator=g).to(dt),
+           "k": torch.randn((n_tok, B, NH, DK), generator=g).to(dt),
+           "v": torch.randn((n_tok, B, NH, DV), generator=g).to(dt),
+           "i": torch.randn((n_tok, B, NH), generator=g) + w.i_mean,
+           "f": torch.rand((n_tok, B, NH), generator=g) * (w.f_high - w.f_low) + w.f_low}
+    dtok = {k: v.to(dev) for k, v in tok.items()}
+    C = torch.zeros((B, NH, DK, DV), device=dev)
+    n = torch.zeros((B, NH, DK), device=dev)
+    m = torch.zeros((B, NH), device=dev)
+    h = torch.empty((B, NH, DV), dtype=dt, device=dev)
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+
+    def step(i):
+        api.mlstm_step(dtok["q"][i], dtok["k"][i], dtok["v"][i], dtok["i"][i], dtok["f"][i],
+                       C, n, m, gate_mode=w.gate_mode, h=h)
+
+    warm = max(3, args.warmup)
+    for i in range(warm):
+        flush.zero_()
+        step(i)
+    torch.cuda.synchronize()
+    lib = _lib.lib()
+    ms_arr = (ctypes.c_double * _lib.KERNEL_COUNT)()
+    n_arr = (ctypes.c_uint64 * _lib.KERNEL_COUNT)()
+    lib.mlstm_profile_read(ms_arr, n_arr, _lib.KERNEL_COUNT)
+    sampler = ClockSampler(0)
+    sampler.start()
+    stream = torch.cuda.current_stream(dev)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    launches0 = lib.mlstm_kernel_launches()
+    t_host0 = time.perf_counter()
+    for j, (e0, e1) in enumerate(evs):
+        flush.zero_()  # the state does not stay in L2 between steps
+        e0.record(stream)
+        step(warm + j)
+        e1.record(stream)
+    torch.cuda.synchronize()
+    t_host1 = time.perf_counter()
+    launches = lib.mlstm_kernel_launches() - launches0
+    sampler.stop()
+    st = api.last_device_error(dev)
+    if st != _lib.OK:
+        raise SystemExit(f"device error in the timed region: {_lib.status_string(st)}")
+    ms = sum(e0.elapsed_time(e1) for e0, e1 in evs) / args.steps
+    peaks, peak_src = load_peaks()
+    nbytes = step_bytes(B, NH, DK, DV, elem)
+    achieved = nbytes / (ms / 1e3) / 1e9
+    line = {
+        "metric": STEP_METRIC, "value": B / (ms / 1e3), "unit": "tokens/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": warm, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+        "config": {"workload": f"step_{w.name}", "B": B, "NH": NH, "DK": DK, "DV": DV,
+                   "gate_mode": w.gate_mode, "dtype": w.dtype,
+                   "l2": "flushed before every step (a %d MB write outside the events)"
+                         % (2 * L2_BYTES >> 20)},
+        "roofline": {"kernel": "step", "bound": "hbm", "achieved": achieved,
+                     "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / peaks["hbm_gbs"],
+                     "peak_source": f"hbm_gbs (of {peak_src})", "algorithmic_bytes": nbytes,
+                     "traffic": None, "per_launch_ms": ms},
+        "gpu_launches": int(launches), "e2e": None,
+        "clocks": sampler.summary(t_host0, t_host1),
+    }
+    if not args.no_cpu_baseline:
+        # the oracle's recurrence over one token from the state, for every (b, h)
+        Ch, nh, mh = C.cpu(), n.cpu(), m.cpu()
+        t0 = time.perf_counter()
+        reps = 0
+        while True:
+            oracle.mlstm_recurrent(tok["q"][0][:, :, None], tok["k"][0][:, :, None],
+                                   tok["v"][0][:, :, None], tok["i"][0][:, :, None],
+                                   tok["f"][0][:, :, None], Ch, nh, mh, gate_mode=w.gate_mode)
+            reps += 1
+            el = time.perf_counter() - t0
+            if el > min(args.cpu_seconds, 5.0):
+                break
+        line["cpu_baseline"] = {"value": B * reps / el, "unit": "tokens/s",
+                                "cores": oracle.num_threads(), "kind": "oracle",
+                                "sample": f"{reps} steps of all {B * NH} heads ({el:.1f} s)"}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -596,11 +714,15 @@ def main():
                     help="skip the host-buffer end-to-end loop (profiling runs)")
     ap.add_argument("--batch", type=int, default=0,
                     help="override the workload's batch size (smaller profiling captures)")
+    ap.add_argument("--op", default="fw", choices=["fw", "step"],
+                    help="fw: the forward pass (default); step: the single-token step")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":
         return run_reference(args)
+    if args.op == "step":
+        return run_step(args)
     return run_ours(args)
 
 

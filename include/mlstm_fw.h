@@ -146,6 +146,26 @@ mlstm_status mlstm_fw_parallel(const void* Q, const void* K, const void* V, cons
                                mlstm_gate_mode gate_mode, mlstm_algo algo, void* workspace,
                                size_t workspace_bytes, mlstm_stream_t stream);
 
+/* Single-token step (decode), the recurrence of mlstm_fw for T = 1: advances
+ * the state of every (b, h) by one token in place and writes that token's
+ * output ("xLSTM: the NX-AI repository behind the extended LSTM
+ * architecture", section "Exponential gating, matrix memory, and why the
+ * kernels decide everything": the step kernel is a separate choice from the
+ * chunkwise one).
+ *   q, k [B, NH, DK] and v, h [B, NH, DV] in `dtype` (device, contiguous);
+ *   i_pre, f_pre [B, NH] fp32;
+ *   C [B, NH, DK, DV], n [B, NH, DK], m [B, NH] fp32: the state before the
+ *   token on entry, after it on return (a zero state is C = n = 0, m = 0).
+ *   m' = max(logsigmoid(f~) + m, li), C' = fa C + ia (s k) v^T,
+ *   n' = fa n + ia s k, h = C'^T q / max(|n'^T q|, e^{-m'}), s = 1/sqrt(DK).
+ * Sizes: B, NH >= 1, DK, DV in [1, 1024].  No workspace; two launches on
+ * `stream`, asynchronous.  All pointers 16-byte aligned and non-null, else
+ * MLSTM_ERR_INVALID_ARG before any launch. */
+mlstm_status mlstm_step(const void* q, const void* k, const void* v, const float* i_pre,
+                        const float* f_pre, float* C, float* n, float* m, void* h, int B, int NH,
+                        int DK, int DV, mlstm_dtype dtype, mlstm_gate_mode gate_mode,
+                        mlstm_stream_t stream);
+
 /* Synchronises `stream`, then returns and clears the device error word:
  * MLSTM_OK, MLSTM_ERR_TIMEOUT (a bounded wait ran out) or MLSTM_ERR_DEVICE;
  * MLSTM_ERR_CUDA if the synchronisation itself failed. */
@@ -182,7 +202,8 @@ typedef enum {
   MLSTM_KERNEL_TC_STATES = 3,     /* tensor-core chunk-state recurrence        */
   MLSTM_KERNEL_TC_PARALLEL = 4,   /* tensor-core intra-chunk TFLA kernel       */
   MLSTM_KERNEL_TC_FUSED = 5,      /* tensor-core fused kernel                  */
-  MLSTM_KERNEL_COUNT = 6
+  MLSTM_KERNEL_STEP = 6,          /* single-token step (2 launches per call)   */
+  MLSTM_KERNEL_COUNT = 7
 } mlstm_kernel_id;
 
 /* Total number of kernels this library has enqueued since it was loaded. */

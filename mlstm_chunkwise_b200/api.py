@@ -134,6 +134,37 @@ def mlstm_fw(Q, K, V, i_pre, f_pre, C0=None, n0=None, m0=None, *, chunk_size: in
     return H
 
 
+def mlstm_step(q, k, v, i_pre, f_pre, C, n, m, *, gate_mode: str = "exp", h=None):
+    """One token of the recurrence for every (b, h), in place on the state.
+
+    q, k [B,NH,DK] and v [B,NH,DV] (float32 or bfloat16, same dtype); i_pre,
+    f_pre [B,NH] float32; C [B,NH,DK,DV], n [B,NH,DK], m [B,NH] float32 CUDA
+    tensors holding the state before the token, overwritten with the state
+    after it.  Returns h [B,NH,DV] in the input dtype (``h`` may be given).
+    """
+    if q.dim() != 3 or k.shape != q.shape or v.dim() != 3 or v.shape[:2] != q.shape[:2]:
+        raise ValueError("q, k must be [B,NH,DK] and v [B,NH,DV] with the same B, NH")
+    B, NH, DK = q.shape
+    DV = v.shape[2]
+    dt, dev = q.dtype, q.device
+    if dt not in _DT or k.dtype != dt or v.dtype != dt:
+        raise ValueError("q, k, v must share a dtype of float32 or bfloat16")
+    for name, t in (("i_pre", i_pre), ("f_pre", f_pre), ("m", m)):
+        _check_tensor(name, t, torch.float32, (B, NH), dev)
+    _check_tensor("C", C, torch.float32, (B, NH, DK, DV), dev)
+    _check_tensor("n", n, torch.float32, (B, NH, DK), dev)
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _check_tensor(name, t, dt, tuple(t.shape), dev)
+    if h is None:
+        h = torch.empty((B, NH, DV), dtype=dt, device=dev)
+    _check_tensor("h", h, dt, (B, NH, DV), dev)
+    st = _lib.lib().mlstm_step(_ptr(q), _ptr(k), _ptr(v), _ptr(i_pre), _ptr(f_pre), _ptr(C),
+                               _ptr(n), _ptr(m), _ptr(h), B, NH, DK, DV, _DT[dt],
+                               _GATE[gate_mode], _stream(dev))
+    _lib.check(st, "mlstm_step")
+    return h
+
+
 def mlstm_fw_chunk_states(K, V, i_pre, f_pre, C0=None, n0=None, m0=None, *, chunk_size: int = 64,
                           gate_mode: str = "exp", algo: str = "auto"):
     """Recurrent half: states entering every chunk and the final state.

@@ -251,6 +251,7 @@ const char* mlstm_kernel_name(int id) {
     case MLSTM_KERNEL_TC_STATES: return "tc_states";
     case MLSTM_KERNEL_TC_PARALLEL: return "tc_parallel";
     case MLSTM_KERNEL_TC_FUSED: return "tc_fused";
+    case MLSTM_KERNEL_STEP: return "step";
   }
   return "unknown";
 }
@@ -454,6 +455,23 @@ mlstm_status mlstm_fw_parallel(const void* Q, const void* K, const void* V, cons
   }
   return from_cuda(launch_family(MLSTM_KERNEL_SIMT_PARALLEL, 1, st, [&] {
     return launch_simt_parallel(p, dtype, Q, K, V, g, C_states, n_states, H, n_out, m_out, st);
+  }));
+}
+
+mlstm_status mlstm_step(const void* q, const void* k, const void* v, const float* i_pre,
+                        const float* f_pre, float* C, float* n, float* m, void* h, int B, int NH,
+                        int DK, int DV, mlstm_dtype dtype, mlstm_gate_mode gate_mode,
+                        mlstm_stream_t stream) {
+  if (!valid_enums(dtype, gate_mode, MLSTM_ALGO_AUTO)) return MLSTM_ERR_INVALID_ARG;
+  if (B < 1 || NH < 1 || DK < 1 || DV < 1) return MLSTM_ERR_INVALID_ARG;
+  if (DK > 1024 || DV > 1024 || (long long)B * NH > 65535) return MLSTM_ERR_UNSUPPORTED;
+  const void* ptrs[] = {q, k, v, i_pre, f_pre, C, n, m, h};
+  for (const void* ptr : ptrs)
+    if (!ptr || !aligned16(ptr)) return MLSTM_ERR_INVALID_ARG;
+  Problem p = make_problem(B, NH, 1, DK, DV, 64, gate_mode);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  return from_cuda(launch_family(MLSTM_KERNEL_STEP, 2, st, [&] {
+    return launch_step(p, dtype, q, k, v, i_pre, f_pre, C, n, m, h, st);
   }));
 }
 

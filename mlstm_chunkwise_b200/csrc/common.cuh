@@ -74,6 +74,9 @@ __device__ __forceinline__ float warp_sum(float v) {
 namespace mlstm {
 cudaError_t launch_gates(const Problem& p, const float* i_pre, const float* f_pre,
                          const float* m0, Gates g, cudaStream_t st);
+cudaError_t launch_step(const Problem& p, mlstm_dtype dt, const void* q, const void* k,
+                        const void* v, const float* i_pre, const float* f_pre, float* C,
+                        float* n, float* m, void* h, cudaStream_t st);
 cudaError_t launch_simt_states(const Problem& p, mlstm_dtype dt, const void* K, const void* V,
                                const float* C0, const float* n0, Gates g, float* C_states,
                                float* n_states, float* C_T, float* n_T, float* m_T,
