@@ -700,6 +700,96 @@ def run_step(args):
     return 0
 
 
+# ----------------------------------------------------------------------------
+# backward pass (fp32 CUDA-core kernels) at a workload's shape
+# ----------------------------------------------------------------------------
+BW_METRIC = "mLSTM backward tokens/s (gradients of a loss on H, forward recomputed)"
+
+
+def bw_flops_per_head(T, DK, DV, L):
+    """Algorithmic FLOPs of the gradient kernels for one (b, h), causal halves
+    counted once: the reverse state recurrence and the three inter-chunk terms
+    (2 T DK DV each), and six intra-chunk contractions (T L d each: dP and P.K
+    for dq, dP and P.Q for dk, S and P.dU for dv).  The recomputed forward is
+    counted separately (flops_per_head)."""
+    return 8.0 * T * DK * DV + 3.0 * T * L * (DK + DV)
+
+
+def run_bw(args):
+    import ctypes
+
+    import torch
+
+    from mlstm_chunkwise_b200 import _lib, api
+    from mlstm_chunkwise_b200 import build as libbuild
+    from mlstm_chunkwise_b200.inputs import make_inputs
+
+    if libbuild.needs_build():
+        libbuild.build()
+    if int(os.environ.get("WORLD_SIZE", "1")) != 1 or args.gpus != 1:
+        raise SystemExit("--op bw runs on one GPU")
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    w = pick_workload(args.workload)
+    if args.batch:
+        w = w.replace(name=f"{w.name}_B{args.batch}", B=args.batch)
+    x = make_inputs(w, seed=rank_seed(w, 0))
+    g = torch.Generator().manual_seed(rank_seed(w, 0) + 1)
+    d = {k: (None if v is None else v.to(dev)) for k, v in x.items()}
+    dH = torch.randn((w.B, w.NH, w.T, w.DV), generator=g).to(w.torch_dtype).to(dev)
+    B, NH, T, DK, DV, L = w.B, w.NH, w.T, w.DK, w.DV, w.chunk_size
+
+    def step():
+        api.mlstm_bw(d["Q"], d["K"], d["V"], d["i_pre"], d["f_pre"], dH, d["C0"], d["n0"],
+                     d["m0"], chunk_size=L, gate_mode=w.gate_mode)
+
+    warm = max(3, args.warmup)
+    for _ in range(warm):
+        step()
+    torch.cuda.synchronize()
+    lib = _lib.lib()
+    sampler = ClockSampler(0)
+    sampler.start()
+    stream = torch.cuda.current_stream(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    launches0 = lib.mlstm_kernel_launches()
+    t_host0 = time.perf_counter()
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    t_host1 = time.perf_counter()
+    launches = lib.mlstm_kernel_launches() - launches0
+    sampler.stop()
+    st = api.last_device_error(dev)
+    if st != _lib.OK:
+        raise SystemExit(f"device error in the timed region: {_lib.status_string(st)}")
+    ms = e0.elapsed_time(e1) / args.steps
+    peaks, peak_src = load_peaks()
+    fph = flops_per_head(T, DK, DV, L)
+    fw_flops = B * NH * (fph["states"] + fph["inter"] + fph["intra"])
+    bw_flops = B * NH * bw_flops_per_head(T, DK, DV, L)
+    peak = SIMT_LANES * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
+    achieved = (fw_flops + bw_flops) / (ms / 1e3) / 1e12
+    line = {
+        "metric": BW_METRIC, "value": B * T / (ms / 1e3), "unit": "tokens/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": warm, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+        "config": workload_config(w, "bw (fp32 CUDA-core kernels)"),
+        "tflops": achieved,
+        "roofline": {"kernel": "bw", "bound": "alu", "achieved": achieved, "peak": peak,
+                     "unit": "TFLOP/s", "frac": achieved / peak,
+                     "peak_source": f"fp32 FFMA: 148 SMs x 128 lanes x 2 x sm_max_mhz (of {peak_src})",
+                     "algorithmic_flops": fw_flops + bw_flops, "traffic": None,
+                     "per_launch_ms": ms},
+        "gpu_launches": int(launches), "e2e": None,
+        "clocks": sampler.summary(t_host0, t_host1),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -714,8 +804,9 @@ def main():
                     help="skip the host-buffer end-to-end loop (profiling runs)")
     ap.add_argument("--batch", type=int, default=0,
                     help="override the workload's batch size (smaller profiling captures)")
-    ap.add_argument("--op", default="fw", choices=["fw", "step"],
-                    help="fw: the forward pass (default); step: the single-token step")
+    ap.add_argument("--op", default="fw", choices=["fw", "step", "bw"],
+                    help="fw: the forward pass (default); step: the single-token step; "
+                         "bw: the backward pass")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -723,6 +814,8 @@ def main():
         return run_reference(args)
     if args.op == "step":
         return run_step(args)
+    if args.op == "bw":
+        return run_bw(args)
     return run_ours(args)
 
 

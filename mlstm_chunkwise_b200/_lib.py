@@ -16,7 +16,7 @@ ERR_SCRATCH_TOO_SMALL = 6
 DT_F32, DT_BF16 = 0, 1
 GATE_EXP, GATE_SIGMOID = 0, 1
 ALGO_AUTO, ALGO_SIMT, ALGO_TC, ALGO_TC_FUSED = 0, 1, 2, 3
-KERNEL_COUNT = 7
+KERNEL_COUNT = 8
 
 _vp = ctypes.c_void_p
 _i = ctypes.c_int
@@ -32,6 +32,8 @@ SIGNATURES = {
     "mlstm_fw_parallel": (_i, [_vp] * 11 + [_i] * 9 + [_vp, _sz, _vp]),
     "mlstm_fw_static_scratch": (_i, [_vp] * 12 + [_i] * 9 + [_vp]),
     "mlstm_fw_static_scratch_capacity": (_sz, []),
+    "mlstm_bw_workspace_size": (_i, [_i] * 6 + [ctypes.POINTER(_sz)]),
+    "mlstm_bw": (_i, [_vp] * 17 + [_i] * 8 + [_vp, _sz, _vp]),
     "mlstm_step": (_i, [_vp] * 9 + [_i] * 6 + [_vp]),
     "mlstm_last_device_error": (_i, [_vp]),
     "mlstm_last_device_error_word": (ctypes.c_uint32, []),

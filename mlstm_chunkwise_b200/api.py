@@ -134,6 +134,35 @@ def mlstm_fw(Q, K, V, i_pre, f_pre, C0=None, n0=None, m0=None, *, chunk_size: in
     return H
 
 
+def mlstm_bw(Q, K, V, i_pre, f_pre, dH, C0=None, n0=None, m0=None, *, chunk_size: int = 64,
+             gate_mode: str = "exp"):
+    """Gradients of a loss L(H) of the forward output, given dH = dL/dH.
+
+    Inputs as ``mlstm_fw``.  Returns a dict with dQ, dK, dV (input dtype),
+    di_pre, df_pre [B,NH,T] and, when an initial state is given, dC0, dn0,
+    dm0 (float32).
+    """
+    B, NH, T, DK, DV, dev, dt = _check_common(Q, K, V, i_pre, f_pre)
+    _check_state(C0, n0, m0, B, NH, DK, DV, dev)
+    _check_tensor("dH", dH, dt, (B, NH, T, DV), dev)
+    out = {"dQ": torch.empty_like(Q), "dK": torch.empty_like(K), "dV": torch.empty_like(V),
+           "di_pre": torch.empty_like(i_pre), "df_pre": torch.empty_like(f_pre)}
+    if C0 is not None:
+        out.update(dC0=torch.empty_like(C0), dn0=torch.empty_like(n0), dm0=torch.empty_like(m0))
+    n = ctypes.c_size_t(0)
+    _lib.check(_lib.lib().mlstm_bw_workspace_size(B, NH, T, DK, DV, chunk_size, ctypes.byref(n)),
+               "mlstm_bw_workspace_size")
+    ws = torch.empty(max(n.value, 1), dtype=torch.uint8, device=dev)
+    st = _lib.lib().mlstm_bw(
+        _ptr(Q), _ptr(K), _ptr(V), _ptr(i_pre), _ptr(f_pre), _ptr(C0), _ptr(n0), _ptr(m0),
+        _ptr(dH), _ptr(out["dQ"]), _ptr(out["dK"]), _ptr(out["dV"]), _ptr(out["di_pre"]),
+        _ptr(out["df_pre"]), _ptr(out.get("dC0")), _ptr(out.get("dn0")), _ptr(out.get("dm0")),
+        B, NH, T, DK, DV, chunk_size, _DT[dt], _GATE[gate_mode], _ptr(ws), ws.numel(),
+        _stream(dev))
+    _lib.check(st, "mlstm_bw")
+    return out
+
+
 def mlstm_step(q, k, v, i_pre, f_pre, C, n, m, *, gate_mode: str = "exp", h=None):
     """One token of the recurrence for every (b, h), in place on the state.
 

@@ -252,6 +252,7 @@ const char* mlstm_kernel_name(int id) {
     case MLSTM_KERNEL_TC_PARALLEL: return "tc_parallel";
     case MLSTM_KERNEL_TC_FUSED: return "tc_fused";
     case MLSTM_KERNEL_STEP: return "step";
+    case MLSTM_KERNEL_BW: return "bw";
   }
   return "unknown";
 }
@@ -455,6 +456,53 @@ mlstm_status mlstm_fw_parallel(const void* Q, const void* K, const void* V, cons
   }
   return from_cuda(launch_family(MLSTM_KERNEL_SIMT_PARALLEL, 1, st, [&] {
     return launch_simt_parallel(p, dtype, Q, K, V, g, C_states, n_states, H, n_out, m_out, st);
+  }));
+}
+
+mlstm_status mlstm_bw_workspace_size(int B, int NH, int T, int DK, int DV, int chunk_size,
+                                     size_t* bytes) {
+  if (!bytes) return MLSTM_ERR_INVALID_ARG;
+  mlstm_status s = check_sizes(B, NH, T, DK, DV, chunk_size);
+  if (s != MLSTM_OK) return s;
+  *bytes = bwd_workspace_bytes(make_problem(B, NH, T, DK, DV, chunk_size, MLSTM_GATE_EXP));
+  return MLSTM_OK;
+}
+
+mlstm_status mlstm_bw(const void* Q, const void* K, const void* V, const float* i_pre,
+                      const float* f_pre, const float* C0, const float* n0, const float* m0,
+                      const void* dH, void* dQ, void* dK, void* dV, float* di_pre, float* df_pre,
+                      float* dC0, float* dn0, float* dm0, int B, int NH, int T, int DK, int DV,
+                      int chunk_size, mlstm_dtype dtype, mlstm_gate_mode gate_mode,
+                      void* workspace, size_t workspace_bytes, mlstm_stream_t stream) {
+  if (!valid_enums(dtype, gate_mode, MLSTM_ALGO_AUTO)) return MLSTM_ERR_INVALID_ARG;
+  mlstm_status s = check_sizes(B, NH, T, DK, DV, chunk_size);
+  if (s != MLSTM_OK) return s;
+  if (!((C0 && n0 && m0) || (!C0 && !n0 && !m0))) return MLSTM_ERR_INVALID_ARG;
+  if (T > 0 && (!Q || !K || !V || !i_pre || !f_pre || !dH || !dQ || !dK || !dV || !di_pre ||
+                !df_pre))
+    return MLSTM_ERR_INVALID_ARG;
+  const void* ptrs[] = {Q,  K,      V,      i_pre, f_pre, C0,  n0,  m0, dH,
+                        dQ, dK,     dV,     di_pre, df_pre, dC0, dn0, dm0, workspace};
+  for (const void* q : ptrs)
+    if (!aligned16(q)) return MLSTM_ERR_INVALID_ARG;
+  Problem p = make_problem(B, NH, T, DK, DV, chunk_size, gate_mode);
+  const size_t need = bwd_workspace_bytes(p);
+  if (workspace_bytes < need || !workspace) return MLSTM_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (T == 0) {  // no output token: the initial state gets no gradient
+    if (dC0 && cudaMemsetAsync(dC0, 0, sizeof(float) * p.BH * DK * DV, st) != cudaSuccess)
+      return MLSTM_ERR_CUDA;
+    if (dn0 && cudaMemsetAsync(dn0, 0, sizeof(float) * p.BH * DK, st) != cudaSuccess)
+      return MLSTM_ERR_CUDA;
+    if (dm0 && cudaMemsetAsync(dm0, 0, sizeof(float) * p.BH, st) != cudaSuccess)
+      return MLSTM_ERR_CUDA;
+    return MLSTM_OK;
+  }
+  p.err = error_word_ptr();
+  if (!p.err) return MLSTM_ERR_CUDA;
+  return from_cuda(launch_family(MLSTM_KERNEL_BW, 10, st, [&] {
+    return launch_backward(p, dtype, Q, K, V, i_pre, f_pre, C0, n0, m0, dH, dQ, dK, dV, di_pre,
+                           df_pre, dC0, dn0, dm0, workspace, st);
   }));
 }
 

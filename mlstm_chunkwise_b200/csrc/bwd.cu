@@ -1,0 +1,683 @@
+// Backward pass of the chunkwise mLSTM (fp32 CUDA-core kernels).
+//
+// The forward ("Tiled Flash Linear Attention: More Efficient Linear RNN and
+// xLSTM Kernels", abstract: the mLSTM as an inter-chunk recurrence plus an
+// intra-chunk parallel part) is h_t = C-bar_t^T q_t / max(|n-bar_t . q_t|, 1)
+// in the unstabilised frame, where C-bar_t = sum_{s<=t} W_ts (s k_s) v_s^T
+// (plus the decayed initial state) and W_ts = e^{log i_s + sum_{s<l<=t} log f_l}.
+// For a loss L(H) with dh_t = dL/dh_t, writing D_t = max(|a_t|, 1),
+// a_t = n-bar_t . q_t, du_t = dh_t / D_t and
+// da_t = -(dh_t . h_t) / D_t sign(a_t) [|a_t| > 1]:
+//
+//   dq_t  = sum_{s<=t} W_ts (v_s . du_t + da_t) k^_s      (k^ = s k)
+//   dk^_s = sum_{t>=s} W_ts (du_t . v_s + da_t) q_t
+//   dv_s  = sum_{t>=s} W_ts (q_t . k^_s) du_t
+//   dL/d log i_s = k_s . dk_s,   dL/d log f_l = sum_{t>=l} (q_t . dq_t - k_t . dk_t)
+//
+// (the last two identities, and these three sums, are checked against an
+// fp64 autograd oracle).  In the stabilised frame of the forward every weight
+// becomes a factor <= 1 that the forward already uses:
+//   intra-chunk   W_ts e^{-m_t} = e^{acol_s - mu_t}            (the gate factor of P)
+//   query side    e^{m_k + bcum_t - m_t} = e^{m_k - mu_t}       (the Q~ scaling)
+//   key side      e^{g_k + acol_s - m_{k+1}}                    (the state-update weight)
+// and with du~_t = dh_t / den_t, da~_t = -(dh_t . h_t) / den_t sign(a_t)
+// [|a_t| > e^{-m_t}] (den_t = max(|a_t|, e^{-m_t}) in the stabilised frame):
+//
+//   G~_k = e^{g_k + m_k - m_{k+1}} G~_{k+1} + sum_{t in k} e^{m_k - mu_t} q_t du~_t^T
+//   g~_k = (the same with du~ -> da~)                      G~_NC = 0, g~_NC = 0
+//   dq_t  = e^{m_k - mu_t} (C_k du~_t + da~_t n_k) + sum_{s<=t in k} e^{acol_s - mu_t} dP_ts k^_s
+//   dk^_s = w_s (G~_{k+1} v_s + g~_{k+1}) + sum_{t>=s in k} e^{acol_s - mu_t} dP_ts q_t
+//   dv_s  = w_s G~_{k+1}^T k^_s + sum_{t>=s in k} e^{acol_s - mu_t} S_ts du~_t
+//   dP_ts = du~_t . v_s + da~_t,  S_ts = q_t . k^_s,  w_s = e^{g_k + acol_s - m_{k+1}}
+//
+// G~_k is the gradient with respect to the state entering chunk k, in that
+// state's frame, so dC0 = G~_0, dn0 = g~_0 and dm0 = <C0, dC0> + n0 . dn0.
+//
+// Launches: the forward's gates, chunk states and outputs (fp32 h and the
+// signed denominator kept), a per-token pass forming du~ and da~, the reverse
+// state recurrence, dq, dk, dv, and the gate gradients (dot products and a
+// reverse scan).  Every kernel tiles 64 x 64 outputs over 256 threads (4 x 4
+// per thread), like the fp32 forward kernels.
+#include <math.h>
+
+#include "common.cuh"
+
+namespace mlstm {
+namespace {
+
+constexpr int kT = 64;        // tile edge
+constexpr int kS = 32;        // contraction slab
+constexpr int kThr = 256;
+
+template <typename TIn>
+__device__ __forceinline__ float ld(const TIn* base, long idx, bool ok) {
+  return ok ? to_float(base[idx]) : 0.f;
+}
+
+__device__ __forceinline__ float sum16(float v) {
+#pragma unroll
+  for (int o = 8; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// acc[i][j] += sum_c A[ty*4+i][c] * B[c][tx*4+j] over one slab
+__device__ __forceinline__ void mac_slab(float (&acc)[4][4], const float (*A)[kS + 1],
+                                         const float (*B)[kT], int ty, int tx) {
+#pragma unroll 4
+  for (int c = 0; c < kS; ++c) {
+    float a[4], b[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) a[i] = A[ty * 4 + i][c];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) b[j] = B[c][tx * 4 + j];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+  }
+}
+
+// acc[i][j] += sum_s P[ty*4+i][s] * B[s][tx*4+j] over a 64-long contraction
+__device__ __forceinline__ void mac_tile(float (&acc)[4][4], const float (*P)[kT + 1],
+                                         const float (*B)[kT], int ty, int tx) {
+#pragma unroll 4
+  for (int s = 0; s < kT; ++s) {
+    float a[4], b[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) a[i] = P[ty * 4 + i][s];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) b[j] = B[s][tx * 4 + j];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// du~ [BH, T, DV] and da~ [BH, T]: one warp per token.
+// ---------------------------------------------------------------------------
+template <typename TIn>
+__global__ void __launch_bounds__(kThr)
+bwd_prep_kernel(Problem p, const TIn* __restrict__ dH, const float* __restrict__ H32,
+                const float* __restrict__ a_sig, const float* __restrict__ den,
+                const float* __restrict__ mr, float* __restrict__ dU, float* __restrict__ dA) {
+  const long tok = (long)blockIdx.x * (kThr / 32) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (tok >= (long)p.BH * p.T) return;
+  const float inv = 1.f / den[tok];
+  float dot = 0.f;
+  for (int c = lane; c < p.DV; c += 32) {
+    const float g = to_float(dH[tok * p.DV + c]);
+    dU[tok * p.DV + c] = g * inv;
+    dot = fmaf(g, H32[tok * p.DV + c], dot);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+  if (lane == 0) {
+    const float a = a_sig[tok];
+    const bool on_n = fabsf(a) > expf(-mr[tok]);  // the max picked |n.q|
+    dA[tok] = on_n ? -dot * inv * (a >= 0.f ? 1.f : -1.f) : 0.f;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Reverse recurrence: G~_k [BH, NC+1, DK, DV], g~_k [BH, NC+1, DK].  One block
+// per (b, h, 64 x 64 tile of [DK, DV]); blocks with blockIdx.x == 0 carry g~.
+// ---------------------------------------------------------------------------
+template <typename TIn>
+__global__ void __launch_bounds__(kThr)
+bwd_states_kernel(Problem p, const TIn* __restrict__ Q, const float* __restrict__ dU,
+                  const float* __restrict__ dA, Gates g, float* __restrict__ G_states,
+                  float* __restrict__ g_states, float* __restrict__ dC0,
+                  float* __restrict__ dn0) {
+  __shared__ float Qs[kT][kT + 1];
+  __shared__ float Us[kT][kT + 1];
+  __shared__ float das[kT];
+  const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
+  const int dv0 = blockIdx.x * kT, dk0 = blockIdx.y * kT, bh = blockIdx.z;
+  const int DK = p.DK, DV = p.DV, T = p.T, L = p.L, NC = p.NC;
+  const bool g_owner = blockIdx.x == 0 && tid < kT && dk0 + tid < DK;
+  const long tpad = (long)NC * L;
+  float acc[4][4] = {};
+  float gacc = 0.f;
+  auto store = [&](int k) {
+    float* Gk = G_states + ((long)bh * (NC + 1) + k) * DK * DV;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int a = dk0 + ty * 4 + i, c = dv0 + tx * 4 + j;
+        if (a < DK && c < DV) Gk[(long)a * DV + c] = acc[i][j];
+      }
+    if (g_owner) g_states[((long)bh * (NC + 1) + k) * DK + dk0 + tid] = gacc;
+  };
+  store(NC);
+  for (int k = NC - 1; k >= 0; --k) {
+    const float m_in = g.mchk[(long)bh * (NC + 1) + k];
+    const float m_out = g.mchk[(long)bh * (NC + 1) + k + 1];
+    const float decay = expf(g.gtot[(long)bh * NC + k] + m_in - m_out);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[i][j] *= decay;
+    gacc *= decay;
+    for (int r0 = 0; r0 < L; r0 += kT) {
+      for (int e = tid; e < kT * kT; e += kThr) {
+        const int r = e / kT, c = e % kT;
+        const long t = (long)k * L + r0 + r;
+        const bool tok = t < T;
+        float f = 0.f;
+        if (tok) f = expf(m_in - fmaxf(m_in, g.amax[(long)bh * tpad + t]));  // e^{m_k - mu_t}
+        Qs[r][c] = f * ld(Q, ((long)bh * T + t) * DK + dk0 + c, tok && dk0 + c < DK);
+        Us[r][c] = (tok && dv0 + c < DV) ? dU[((long)bh * T + t) * DV + dv0 + c] : 0.f;
+      }
+      if (tid < kT) {
+        const long t = (long)k * L + r0 + tid;
+        das[tid] = t < T ? dA[(long)bh * T + t] : 0.f;
+      }
+      __syncthreads();
+#pragma unroll 4
+      for (int r = 0; r < kT; ++r) {
+        float a[4], b[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) a[i] = Qs[r][ty * 4 + i];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) b[j] = Us[r][tx * 4 + j];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+        if (g_owner) gacc = fmaf(Qs[r][tid], das[r], gacc);
+      }
+      __syncthreads();
+    }
+    store(k);
+  }
+  if (dC0) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int a = dk0 + ty * 4 + i, c = dv0 + tx * 4 + j;
+        if (a < DK && c < DV) dC0[((long)bh * DK + a) * DV + c] = acc[i][j];
+      }
+  }
+  if (dn0 && g_owner) dn0[(long)bh * DK + dk0 + tid] = gacc;
+}
+
+// ---------------------------------------------------------------------------
+// dq: one block per (b, h, 64 queries, 64 columns of d_qk).  Also adds the
+// block's part of q_t . dq_t into qdq (zeroed beforehand).
+// ---------------------------------------------------------------------------
+template <typename TIn>
+__global__ void __launch_bounds__(kThr)
+bwd_dq_kernel(Problem p, const TIn* __restrict__ Q, const TIn* __restrict__ K,
+              const TIn* __restrict__ V, Gates g, const float* __restrict__ C_states,
+              const float* __restrict__ n_states, const float* __restrict__ dU,
+              const float* __restrict__ dA, TIn* __restrict__ dQ, float* __restrict__ qdq) {
+  __shared__ float As[kT][kS + 1];
+  __shared__ float Bs[kT][kT];   // a slab [kS][kT], or a whole [kT][kT] tile
+  __shared__ float Ps[kT][kT + 1];
+  __shared__ float mu_s[kT], das[kT], acol_s[kT];
+  const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
+  const int dk0 = blockIdx.x * kT, bh = blockIdx.z;
+  const long t0 = (long)blockIdx.y * kT;
+  const int DK = p.DK, DV = p.DV, T = p.T, L = p.L, NC = p.NC;
+  const int k = (int)(t0 / L);
+  const long tpad = (long)NC * L;
+  const float m_in = g.mchk[(long)bh * (NC + 1) + k];
+  if (tid < kT) {
+    const long t = t0 + tid;
+    mu_s[tid] = fmaxf(m_in, g.amax[(long)bh * tpad + t]);
+    das[tid] = t < T ? dA[(long)bh * T + t] : 0.f;
+  }
+  __syncthreads();
+  float acc[4][4] = {};
+  // inter: X[t][d] = sum_c du~[t][c] C_k[d][c]
+  const float* Ck = C_states + ((long)bh * NC + k) * DK * DV;
+  for (int c0 = 0; c0 < DV; c0 += kS) {
+    for (int e = tid; e < kT * kS; e += kThr) {
+      const int r = e / kS, c = e % kS;
+      const long t = t0 + r;
+      As[r][c] = (t < T && c0 + c < DV) ? dU[((long)bh * T + t) * DV + c0 + c] : 0.f;
+    }
+    for (int e = tid; e < kS * kT; e += kThr) {
+      const int c = e / kT, j = e % kT;
+      Bs[c][j] = (c0 + c < DV && dk0 + j < DK) ? Ck[(long)(dk0 + j) * DV + c0 + c] : 0.f;
+    }
+    __syncthreads();
+    mac_slab(acc, As, Bs, ty, tx);
+    __syncthreads();
+  }
+  const float* nk = n_states + ((long)bh * NC + k) * DK;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int r = ty * 4 + i;
+    const float f = expf(m_in - mu_s[r]);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int d = dk0 + tx * 4 + j;
+      acc[i][j] = f * (acc[i][j] + das[r] * (d < DK ? nk[d] : 0.f));
+    }
+  }
+  // intra: key tiles of the chunk up to the diagonal
+  for (long s0 = (long)k * L; s0 <= t0; s0 += kT) {
+    float dP[4][4] = {};
+    for (int c0 = 0; c0 < DV; c0 += kS) {
+      for (int e = tid; e < kT * kS; e += kThr) {
+        const int r = e / kS, c = e % kS;
+        const long t = t0 + r;
+        As[r][c] = (t < T && c0 + c < DV) ? dU[((long)bh * T + t) * DV + c0 + c] : 0.f;
+      }
+      for (int e = tid; e < kS * kT; e += kThr) {
+        const int c = e / kT, j = e % kT;
+        Bs[c][j] = ld(V, ((long)bh * T + s0 + j) * DV + c0 + c, s0 + j < T && c0 + c < DV);
+      }
+      __syncthreads();
+      mac_slab(dP, As, Bs, ty, tx);
+      __syncthreads();
+    }
+    if (tid < kT) acol_s[tid] = g.acol[(long)bh * tpad + s0 + tid];
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int r = ty * 4 + i, s = tx * 4 + j;
+        const bool ok = s0 + s <= t0 + r && t0 + r < T;
+        Ps[r][s] = ok ? expf(acol_s[s] - mu_s[r]) * (dP[i][j] + das[r]) : 0.f;
+      }
+    for (int e = tid; e < kT * kT; e += kThr) {
+      const int s = e / kT, j = e % kT;
+      Bs[s][j] = p.key_scale * ld(K, ((long)bh * T + s0 + s) * DK + dk0 + j,
+                                  s0 + s < T && dk0 + j < DK);
+    }
+    __syncthreads();
+    mac_tile(acc, Ps, Bs, ty, tx);
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const long t = t0 + ty * 4 + i;
+    float part = 0.f;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int d = dk0 + tx * 4 + j;
+      if (t < T && d < DK) {
+        dQ[((long)bh * T + t) * DK + d] = from_float<TIn>(acc[i][j]);
+        part = fmaf(to_float(Q[((long)bh * T + t) * DK + d]), acc[i][j], part);
+      }
+    }
+    part = sum16(part);
+    if (tx == 0 && t < T) atomicAdd(&qdq[(long)bh * T + t], part);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// dk: one block per (b, h, 64 keys, 64 columns of d_qk).  Adds k_s . dk_s
+// into kdk (zeroed beforehand).
+// ---------------------------------------------------------------------------
+template <typename TIn>
+__global__ void __launch_bounds__(kThr)
+bwd_dk_kernel(Problem p, const TIn* __restrict__ Q, const TIn* __restrict__ K,
+              const TIn* __restrict__ V, Gates g, const float* __restrict__ G_states,
+              const float* __restrict__ g_states, const float* __restrict__ dU,
+              const float* __restrict__ dA, TIn* __restrict__ dK, float* __restrict__ kdk) {
+  __shared__ float As[kT][kS + 1];
+  __shared__ float Bs[kT][kT];
+  __shared__ float Ps[kT][kT + 1];
+  __shared__ float mu_s[kT], das[kT], acol_s[kT];
+  const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
+  const int dk0 = blockIdx.x * kT, bh = blockIdx.z;
+  const long s0 = (long)blockIdx.y * kT;
+  const int DK = p.DK, DV = p.DV, T = p.T, L = p.L, NC = p.NC;
+  const int k = (int)(s0 / L);
+  const long tpad = (long)NC * L;
+  const float m_in = g.mchk[(long)bh * (NC + 1) + k];
+  const float m_out = g.mchk[(long)bh * (NC + 1) + k + 1];
+  const float gk = g.gtot[(long)bh * NC + k];
+  if (tid < kT) acol_s[tid] = g.acol[(long)bh * tpad + s0 + tid];
+  __syncthreads();
+  float acc[4][4] = {};
+  // inter: Y[s][d] = sum_c v_s[c] G~_{k+1}[d][c] + g~_{k+1}[d], times w_s
+  const float* Gk = G_states + ((long)bh * (NC + 1) + k + 1) * DK * DV;
+  const float* gk1 = g_states + ((long)bh * (NC + 1) + k + 1) * DK;
+  for (int c0 = 0; c0 < DV; c0 += kS) {
+    for (int e = tid; e < kT * kS; e += kThr) {
+      const int r = e / kS, c = e % kS;
+      As[r][c] = ld(V, ((long)bh * T + s0 + r) * DV + c0 + c, s0 + r < T && c0 + c < DV);
+    }
+    for (int e = tid; e < kS * kT; e += kThr) {
+      const int c = e / kT, j = e % kT;
+      Bs[c][j] = (c0 + c < DV && dk0 + j < DK) ? Gk[(long)(dk0 + j) * DV + c0 + c] : 0.f;
+    }
+    __syncthreads();
+    mac_slab(acc, As, Bs, ty, tx);
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int r = ty * 4 + i;
+    const float w = expf(gk + acol_s[r] - m_out);  // 0 on padding (acol = -inf)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int d = dk0 + tx * 4 + j;
+      acc[i][j] = w * (acc[i][j] + (d < DK ? gk1[d] : 0.f));
+    }
+  }
+  // intra: query tiles of the chunk from the diagonal on
+  const long chunk_end = (long)(k + 1) * L;
+  for (long q0 = s0; q0 < chunk_end && q0 < T; q0 += kT) {
+    if (tid < kT) {
+      const long t = q0 + tid;
+      mu_s[tid] = fmaxf(m_in, g.amax[(long)bh * tpad + t]);
+      das[tid] = t < T ? dA[(long)bh * T + t] : 0.f;
+    }
+    float dP[4][4] = {};  // [s][t]
+    for (int c0 = 0; c0 < DV; c0 += kS) {
+      for (int e = tid; e < kT * kS; e += kThr) {
+        const int r = e / kS, c = e % kS;
+        As[r][c] = ld(V, ((long)bh * T + s0 + r) * DV + c0 + c, s0 + r < T && c0 + c < DV);
+      }
+      for (int e = tid; e < kS * kT; e += kThr) {
+        const int c = e / kT, j = e % kT;
+        const long t = q0 + j;
+        Bs[c][j] = (t < T && c0 + c < DV) ? dU[((long)bh * T + t) * DV + c0 + c] : 0.f;
+      }
+      __syncthreads();
+      mac_slab(dP, As, Bs, ty, tx);
+      __syncthreads();
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int s = ty * 4 + i, r = tx * 4 + j;  // key s, query r
+        const bool ok = q0 + r >= s0 + s && q0 + r < T;
+        Ps[s][r] = ok ? expf(acol_s[s] - mu_s[r]) * (dP[i][j] + das[r]) : 0.f;
+      }
+    for (int e = tid; e < kT * kT; e += kThr) {
+      const int r = e / kT, j = e % kT;
+      Bs[r][j] = ld(Q, ((long)bh * T + q0 + r) * DK + dk0 + j, q0 + r < T && dk0 + j < DK);
+    }
+    __syncthreads();
+    mac_tile(acc, Ps, Bs, ty, tx);
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const long s = s0 + ty * 4 + i;
+    float part = 0.f;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int d = dk0 + tx * 4 + j;
+      if (s < T && d < DK) {
+        const float dk = p.key_scale * acc[i][j];
+        dK[((long)bh * T + s) * DK + d] = from_float<TIn>(dk);
+        part = fmaf(to_float(K[((long)bh * T + s) * DK + d]), dk, part);
+      }
+    }
+    part = sum16(part);
+    if (tx == 0 && s < T) atomicAdd(&kdk[(long)bh * T + s], part);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// dv: one block per (b, h, 64 keys, 64 columns of d_v).
+// ---------------------------------------------------------------------------
+template <typename TIn>
+__global__ void __launch_bounds__(kThr)
+bwd_dv_kernel(Problem p, const TIn* __restrict__ Q, const TIn* __restrict__ K, Gates g,
+              const float* __restrict__ G_states, const float* __restrict__ dU,
+              TIn* __restrict__ dV) {
+  __shared__ float As[kT][kS + 1];
+  __shared__ float Bs[kT][kT];
+  __shared__ float Ps[kT][kT + 1];
+  __shared__ float mu_s[kT], acol_s[kT];
+  const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
+  const int dv0 = blockIdx.x * kT, bh = blockIdx.z;
+  const long s0 = (long)blockIdx.y * kT;
+  const int DK = p.DK, DV = p.DV, T = p.T, L = p.L, NC = p.NC;
+  const int k = (int)(s0 / L);
+  const long tpad = (long)NC * L;
+  const float m_in = g.mchk[(long)bh * (NC + 1) + k];
+  const float m_out = g.mchk[(long)bh * (NC + 1) + k + 1];
+  const float gk = g.gtot[(long)bh * NC + k];
+  if (tid < kT) acol_s[tid] = g.acol[(long)bh * tpad + s0 + tid];
+  __syncthreads();
+  float acc[4][4] = {};
+  // inter: Z[s][c] = sum_d k^_s[d] G~_{k+1}[d][c], times w_s
+  const float* Gk = G_states + ((long)bh * (NC + 1) + k + 1) * DK * DV;
+  for (int d0 = 0; d0 < DK; d0 += kS) {
+    for (int e = tid; e < kT * kS; e += kThr) {
+      const int r = e / kS, c = e % kS;
+      As[r][c] = p.key_scale * ld(K, ((long)bh * T + s0 + r) * DK + d0 + c,
+                                  s0 + r < T && d0 + c < DK);
+    }
+    for (int e = tid; e < kS * kT; e += kThr) {
+      const int c = e / kT, j = e % kT;
+      Bs[c][j] = (d0 + c < DK && dv0 + j < DV) ? Gk[(long)(d0 + c) * DV + dv0 + j] : 0.f;
+    }
+    __syncthreads();
+    mac_slab(acc, As, Bs, ty, tx);
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float w = expf(gk + acol_s[ty * 4 + i] - m_out);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[i][j] *= w;
+  }
+  const long chunk_end = (long)(k + 1) * L;
+  for (long q0 = s0; q0 < chunk_end && q0 < T; q0 += kT) {
+    if (tid < kT) mu_s[tid] = fmaxf(m_in, g.amax[(long)bh * tpad + q0 + tid]);
+    float S[4][4] = {};  // [s][t] = k^_s . q_t
+    for (int d0 = 0; d0 < DK; d0 += kS) {
+      for (int e = tid; e < kT * kS; e += kThr) {
+        const int r = e / kS, c = e % kS;
+        As[r][c] = p.key_scale * ld(K, ((long)bh * T + s0 + r) * DK + d0 + c,
+                                    s0 + r < T && d0 + c < DK);
+      }
+      for (int e = tid; e < kS * kT; e += kThr) {
+        const int c = e / kT, j = e % kT;
+        Bs[c][j] = ld(Q, ((long)bh * T + q0 + j) * DK + d0 + c, q0 + j < T && d0 + c < DK);
+      }
+      __syncthreads();
+      mac_slab(S, As, Bs, ty, tx);
+      __syncthreads();
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int s = ty * 4 + i, r = tx * 4 + j;
+        const bool ok = q0 + r >= s0 + s && q0 + r < T;
+        Ps[s][r] = ok ? expf(acol_s[s] - mu_s[r]) * S[i][j] : 0.f;
+      }
+    for (int e = tid; e < kT * kT; e += kThr) {
+      const int r = e / kT, j = e % kT;
+      const long t = q0 + r;
+      Bs[r][j] = (t < T && dv0 + j < DV) ? dU[((long)bh * T + t) * DV + dv0 + j] : 0.f;
+    }
+    __syncthreads();
+    mac_tile(acc, Ps, Bs, ty, tx);
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const long s = s0 + ty * 4 + i;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int c = dv0 + tx * 4 + j;
+      if (s < T && c < DV) dV[((long)bh * T + s) * DV + c] = from_float<TIn>(acc[i][j]);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Gate gradients, one block per (b, h): di from k.dk, df from the reverse
+// scan of q.dq - k.dk, and dm0 = <C0, dC0> + n0 . dn0.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kThr)
+bwd_gates_kernel(Problem p, const float* __restrict__ i_pre, const float* __restrict__ f_pre,
+                 const float* __restrict__ qdq, const float* __restrict__ kdk,
+                 float* __restrict__ di, float* __restrict__ df, const float* __restrict__ C0,
+                 const float* __restrict__ n0, const float* __restrict__ dC0,
+                 const float* __restrict__ dn0, float* __restrict__ dm0) {
+  __shared__ float seg[kThr];
+  const int bh = blockIdx.x, tid = threadIdx.x;
+  const long T = p.T, base = (long)bh * T;
+  // thread tid owns tokens [lo, hi)
+  const long per = (T + kThr - 1) / kThr;
+  const long lo = tid * per < T ? tid * per : T, hi = lo + per < T ? lo + per : T;
+  float sum = 0.f;
+  for (long t = lo; t < hi; ++t) {
+    const float i = i_pre[base + t];
+    const float dli = kdk[base + t];
+    di[base + t] = p.gate_sigmoid ? dli / (1.f + expf(i)) : dli;  // 1 - sigmoid(i) = 1/(1+e^i)
+    sum += qdq[base + t] - kdk[base + t];
+  }
+  seg[tid] = sum;
+  __syncthreads();
+  // suffix sums of the segment totals (inclusive, from the right)
+  for (int o = 1; o < kThr; o <<= 1) {
+    const float add = tid + o < kThr ? seg[tid + o] : 0.f;
+    __syncthreads();
+    seg[tid] += add;
+    __syncthreads();
+  }
+  float run = tid + 1 < kThr ? seg[tid + 1] : 0.f;  // everything right of this segment
+  for (long t = hi - 1; t >= lo; --t) {
+    run += qdq[base + t] - kdk[base + t];
+    df[base + t] = run / (1.f + expf(f_pre[base + t]));  // d log f / d f~ = 1 - sigmoid(f~)
+  }
+  if (dm0) {
+    float acc = 0.f;
+    if (C0) {
+      const long n = (long)p.DK * p.DV;
+      for (long e = tid; e < n; e += kThr) acc = fmaf(C0[bh * n + e], dC0[bh * n + e], acc);
+      for (int e = tid; e < p.DK; e += kThr)
+        acc = fmaf(n0[(long)bh * p.DK + e], dn0[(long)bh * p.DK + e], acc);
+    }
+    __syncthreads();
+    seg[tid] = acc;
+    __syncthreads();
+    for (int o = kThr / 2; o > 0; o >>= 1) {
+      if (tid < o) seg[tid] += seg[tid + o];
+      __syncthreads();
+    }
+    if (tid == 0) dm0[bh] = seg[0];
+  }
+}
+
+// Workspace carve (all fp32): see bwd_workspace_bytes.
+struct BwdWs {
+  Gates g;
+  float *C_states, *n_states, *H32, *a_sig, *den, *mr, *dU, *dA, *G_states, *g_states, *qdq,
+      *kdk, *dC0, *dn0;
+};
+
+constexpr size_t kAlign = 256;
+inline size_t al(size_t b) { return (b + kAlign - 1) / kAlign * kAlign; }
+
+size_t carve(const Problem& p, char* base, BwdWs* w) {
+  const size_t BH = p.BH, T = p.T, NC = p.NC, tpad = NC * p.L, DK = p.DK, DV = p.DV;
+  size_t off = 0;
+  auto take = [&](size_t n) -> float* {
+    float* ptr = base ? reinterpret_cast<float*>(base + off) : nullptr;
+    off += al(n * sizeof(float));
+    return ptr;
+  };
+  Gates g;
+  g.bcum = take(BH * tpad);
+  g.acol = take(BH * tpad);
+  g.amax = take(BH * tpad);
+  g.gtot = take(BH * NC);
+  g.mchk = take(BH * (NC + 1));
+  BwdWs x;
+  x.g = g;
+  x.C_states = take(BH * NC * DK * DV);
+  x.n_states = take(BH * NC * DK);
+  x.H32 = take(BH * T * DV);
+  x.a_sig = take(BH * T);
+  x.den = take(BH * T);
+  x.mr = take(BH * T);
+  x.dU = take(BH * T * DV);
+  x.dA = take(BH * T);
+  x.G_states = take(BH * (NC + 1) * DK * DV);
+  x.g_states = take(BH * (NC + 1) * DK);
+  x.qdq = take(BH * T);
+  x.kdk = take(BH * T);
+  x.dC0 = take(BH * DK * DV);
+  x.dn0 = take(BH * DK);
+  if (w) *w = x;
+  return off;
+}
+
+template <typename TIn>
+cudaError_t launch_bwd_t(const Problem& p, mlstm_dtype dt, const void* Q, const void* K,
+                         const void* V, const float* i_pre, const float* f_pre, const float* C0,
+                         const float* n0, const float* m0, const void* dH, void* dQ, void* dK,
+                         void* dV, float* di, float* df, float* dC0, float* dn0, float* dm0,
+                         void* ws, cudaStream_t st) {
+  BwdWs w;
+  carve(p, static_cast<char*>(ws), &w);
+  const TIn* q = static_cast<const TIn*>(Q);
+  const TIn* k = static_cast<const TIn*>(K);
+  const TIn* v = static_cast<const TIn*>(V);
+  cudaError_t e = launch_gates(p, i_pre, f_pre, m0, w.g, st);
+  if (e != cudaSuccess) return e;
+  e = launch_simt_states(p, dt, K, V, C0, n0, w.g, w.C_states, w.n_states, nullptr, nullptr,
+                         nullptr, st);
+  if (e != cudaSuccess) return e;
+  e = launch_simt_parallel(p, dt, Q, K, V, w.g, w.C_states, w.n_states, nullptr, w.den, w.mr, st,
+                           w.H32, w.a_sig);
+  if (e != cudaSuccess) return e;
+  const long toks = (long)p.BH * p.T;
+  bwd_prep_kernel<TIn><<<(unsigned)((toks + 7) / 8), kThr, 0, st>>>(
+      p, static_cast<const TIn*>(dH), w.H32, w.a_sig, w.den, w.mr, w.dU, w.dA);
+  const int nk = (p.DK + kT - 1) / kT, nv = (p.DV + kT - 1) / kT, nt = (p.T + kT - 1) / kT;
+  bwd_states_kernel<TIn><<<dim3(nv, nk, p.BH), kThr, 0, st>>>(p, q, w.dU, w.dA, w.g, w.G_states,
+                                                              w.g_states, w.dC0, w.dn0);
+  e = cudaMemsetAsync(w.qdq, 0, sizeof(float) * toks, st);
+  if (e != cudaSuccess) return e;
+  e = cudaMemsetAsync(w.kdk, 0, sizeof(float) * toks, st);
+  if (e != cudaSuccess) return e;
+  bwd_dq_kernel<TIn><<<dim3(nk, nt, p.BH), kThr, 0, st>>>(
+      p, q, k, v, w.g, w.C_states, w.n_states, w.dU, w.dA, static_cast<TIn*>(dQ), w.qdq);
+  bwd_dk_kernel<TIn><<<dim3(nk, nt, p.BH), kThr, 0, st>>>(
+      p, q, k, v, w.g, w.G_states, w.g_states, w.dU, w.dA, static_cast<TIn*>(dK), w.kdk);
+  bwd_dv_kernel<TIn><<<dim3(nv, nt, p.BH), kThr, 0, st>>>(p, q, k, w.g, w.G_states, w.dU,
+                                                          static_cast<TIn*>(dV));
+  bwd_gates_kernel<<<p.BH, kThr, 0, st>>>(p, i_pre, f_pre, w.qdq, w.kdk, di, df, C0, n0, w.dC0,
+                                          w.dn0, dm0);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  if (dC0) {
+    e = cudaMemcpyAsync(dC0, w.dC0, sizeof(float) * p.BH * p.DK * p.DV,
+                        cudaMemcpyDeviceToDevice, st);
+    if (e != cudaSuccess) return e;
+  }
+  if (dn0)
+    e = cudaMemcpyAsync(dn0, w.dn0, sizeof(float) * p.BH * p.DK, cudaMemcpyDeviceToDevice, st);
+  return e;
+}
+
+}  // namespace
+
+size_t bwd_workspace_bytes(const Problem& p) { return carve(p, nullptr, nullptr); }
+
+cudaError_t launch_backward(const Problem& p, mlstm_dtype dt, const void* Q, const void* K,
+                            const void* V, const float* i_pre, const float* f_pre,
+                            const float* C0, const float* n0, const float* m0, const void* dH,
+                            void* dQ, void* dK, void* dV, float* di, float* df, float* dC0,
+                            float* dn0, float* dm0, void* ws, cudaStream_t st) {
+  if (dt == MLSTM_DT_BF16)
+    return launch_bwd_t<__nv_bfloat16>(p, dt, Q, K, V, i_pre, f_pre, C0, n0, m0, dH, dQ, dK, dV,
+                                       di, df, dC0, dn0, dm0, ws, st);
+  return launch_bwd_t<float>(p, dt, Q, K, V, i_pre, f_pre, C0, n0, m0, dH, dQ, dK, dV, di, df,
+                             dC0, dn0, dm0, ws, st);
+}
+
+}  // namespace mlstm

@@ -74,6 +74,15 @@ __device__ __forceinline__ float warp_sum(float v) {
 namespace mlstm {
 cudaError_t launch_gates(const Problem& p, const float* i_pre, const float* f_pre,
                          const float* m0, Gates g, cudaStream_t st);
+// Backward pass (bwd.cu).  dH in the input dtype; dQ, dK, dV in the input
+// dtype; di, df [BH, T], dC0 [BH, DK, DV], dn0 [BH, DK], dm0 [BH] fp32
+// (the last three nullable).  `ws` holds bwd_workspace_bytes(p) bytes.
+size_t bwd_workspace_bytes(const Problem& p);
+cudaError_t launch_backward(const Problem& p, mlstm_dtype dt, const void* Q, const void* K,
+                            const void* V, const float* i_pre, const float* f_pre,
+                            const float* C0, const float* n0, const float* m0, const void* dH,
+                            void* dQ, void* dK, void* dV, float* di, float* df, float* dC0,
+                            float* dn0, float* dm0, void* ws, cudaStream_t st);
 cudaError_t launch_step(const Problem& p, mlstm_dtype dt, const void* q, const void* k,
                         const void* v, const float* i_pre, const float* f_pre, float* C,
                         float* n, float* m, void* h, cudaStream_t st);
@@ -84,5 +93,5 @@ cudaError_t launch_simt_states(const Problem& p, mlstm_dtype dt, const void* K, 
 cudaError_t launch_simt_parallel(const Problem& p, mlstm_dtype dt, const void* Q, const void* K,
                                  const void* V, Gates g, const float* C_states,
                                  const float* n_states, void* H, float* n_out, float* m_out,
-                                 cudaStream_t st);
+                                 cudaStream_t st, float* H32 = nullptr, float* a_out = nullptr);
 }  // namespace mlstm

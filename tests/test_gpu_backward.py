@@ -1,0 +1,75 @@
+"""Backward pass (mlstm_bw) against the fp64 autograd oracle.
+
+Same seeded inputs on both sides; the upstream gradient dH is drawn in the
+input dtype.  Metric as the forward's: per (b, h) slice, max|x - y| / max|y|.
+"""
+import pytest
+import torch
+
+import parity
+from oracle import backward as ob
+from mlstm_chunkwise_b200 import _lib, api
+from mlstm_chunkwise_b200.inputs import WORKLOADS, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+# tolerance of the gradients: as the forward's for bf16 inputs; fp32 inputs
+# accumulate the suffix sums of the forget-gate gradient over T tokens in fp32
+TOL = {"f32": 1e-4, "bf16": 2e-2}
+
+CASES = [
+    # B, NH, T, DK, DV, chunk, dtype, gate, initial state
+    (1, 2, 256, 64, 64, 64, "f32", "exp", False),
+    (1, 2, 256, 64, 64, 64, "bf16", "exp", False),
+    (2, 1, 200, 64, 64, 64, "f32", "exp", True),        # ragged tail, initial state
+    (1, 2, 512, 128, 128, 128, "bf16", "exp", False),
+    (1, 2, 512, 128, 128, 256, "f32", "sigmoid", True),
+    (1, 1, 130, 100, 72, 64, "f32", "exp", True),       # dims that are not tile multiples
+    (1, 2, 1, 64, 64, 64, "f32", "exp", True),          # single token
+]
+
+
+def _grad_case(B, NH, T, DK, DV, L, dtype, gate, init, seed=11):
+    w = WORKLOADS["mid"].replace(name="bw", B=B, NH=NH, T=T, DK=DK, DV=DV, chunk_size=L,
+                                 dtype=dtype, gate_mode=gate, init_state=init, i_mean=0.0)
+    x = make_inputs(w, seed=seed)
+    g = torch.Generator().manual_seed(seed + 1)
+    dH = torch.randn((B, NH, T, DV), generator=g).to(w.torch_dtype)
+    ref = ob.gradients(x, dH, gate)
+    d = parity.to_dev(x)
+    got = api.mlstm_bw(d["Q"], d["K"], d["V"], d["i_pre"], d["f_pre"], dH.cuda(), d["C0"],
+                       d["n0"], d["m0"], chunk_size=L, gate_mode=gate)
+    torch.cuda.synchronize()
+    assert api.last_device_error() == _lib.OK
+    return w, ref, got
+
+
+def _errors(ref, got):
+    names = [("dQ", "dQ"), ("dK", "dK"), ("dV", "dV"), ("di_pre", "di_pre"), ("df_pre", "df_pre")]
+    if "dC0" in got:
+        names += [("dC0", "dC0"), ("dn0", "dn0")]
+    errs = {k: parity.worst_rel(got[g].double().cpu().numpy(), ref[k].numpy()) for g, k in names}
+    if "dm0" in got:
+        errs["dm0"] = float((got["dm0"].double().cpu() - ref["dm0"]).abs().max()
+                            / max(1.0, float(ref["dm0"].abs().max())))
+    return errs
+
+
+@pytest.mark.parametrize("case", CASES, ids=lambda c: "-".join(map(str, c)))
+def test_backward_matches_autograd_oracle(case):
+    w, ref, got = _grad_case(*case)
+    errs = _errors(ref, got)
+    bad = {k: v for k, v in errs.items() if not v <= TOL[w.dtype]}
+    assert not bad, f"{case}: {errs}"
+
+
+def test_backward_chunk_size_invariance():
+    """The gradients do not depend on the chunk size (64, 128, 256)."""
+    outs = []
+    for L in (64, 128, 256):
+        _, _, got = _grad_case(1, 2, 512, 64, 64, L, "f32", "exp", True)
+        outs.append(got)
+    for o in outs[1:]:
+        for k in ("dQ", "dK", "dV", "di_pre", "df_pre", "dC0"):
+            assert parity.worst_rel(o[k].double().cpu().numpy(),
+                                    outs[0][k].double().cpu().numpy()) < 1e-4, k
