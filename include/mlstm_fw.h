@@ -146,9 +146,10 @@ mlstm_status mlstm_fw_parallel(const void* Q, const void* K, const void* V, cons
                                mlstm_gate_mode gate_mode, mlstm_algo algo, void* workspace,
                                size_t workspace_bytes, mlstm_stream_t stream);
 
-/* Workspace bytes of mlstm_bw() for these sizes (sizes as mlstm_fw). */
+/* Workspace bytes of mlstm_bw() for these sizes and input type (sizes as
+ * mlstm_fw). */
 mlstm_status mlstm_bw_workspace_size(int B, int NH, int T, int DK, int DV, int chunk_size,
-                                     size_t* bytes);
+                                     mlstm_dtype dtype, size_t* bytes);
 
 /* Backward pass: the gradients of a loss L(H) of the forward's output, given
  * dH = dL/dH, with respect to every input of mlstm_fw.  It recomputes the
@@ -158,16 +159,18 @@ mlstm_status mlstm_bw_workspace_size(int B, int NH, int T, int DK, int DV, int c
  * inter-chunk terms, and the gate gradients from the identities
  * dL/d log i_s = k_s . dk_s and dL/d log f_l = sum_{t >= l} (q_t . dq_t -
  * k_t . dk_t) ("Tiled Flash Linear Attention: More Efficient Linear RNN and
- * xLSTM Kernels": the chunkwise split applied to the gradient).  fp32
- * CUDA-core kernels for both input types; the derivation and its
- * stabilisation are in the header of the implementation file.
+ * xLSTM Kernels": the chunkwise split applied to the gradient).  The
+ * recomputed forward runs on the tensor cores for bf16 inputs where the TC
+ * algorithm supports the shape (else on the fp32 kernels); the gradient
+ * kernels are fp32 CUDA-core kernels for both input types.  The derivation
+ * and its stabilisation are in the header of the implementation file.
  *   Q, K, V, dH in `dtype` as in mlstm_fw; dQ, dK, dV out, same shapes and
  *   dtype; di_pre, df_pre [B, NH, T] fp32 out; C0/n0/m0 all given or all
  *   null; dC0 [B, NH, DK, DV], dn0 [B, NH, DK], dm0 [B, NH] fp32 out
  *   (nullable; zero-state calls get the gradient a zero initial state would
  *   have).  The loss is on H only (no gradient arrives through C_T/n_T/m_T).
  * Errors as mlstm_fw; the workspace must hold mlstm_bw_workspace_size bytes.
- * Ten launches, asynchronous on `stream`. */
+ * 10 to 12 launches, asynchronous on `stream`. */
 mlstm_status mlstm_bw(const void* Q, const void* K, const void* V, const float* i_pre,
                       const float* f_pre, const float* C0, const float* n0, const float* m0,
                       const void* dH, void* dQ, void* dK, void* dV, float* di_pre, float* df_pre,
@@ -232,7 +235,7 @@ typedef enum {
   MLSTM_KERNEL_TC_PARALLEL = 4,   /* tensor-core intra-chunk TFLA kernel       */
   MLSTM_KERNEL_TC_FUSED = 5,      /* tensor-core fused kernel                  */
   MLSTM_KERNEL_STEP = 6,          /* single-token step (2 launches per call)   */
-  MLSTM_KERNEL_BW = 7,            /* backward pass (10 launches per call)      */
+  MLSTM_KERNEL_BW = 7,            /* backward pass (10 to 12 launches per call) */
   MLSTM_KERNEL_COUNT = 8
 } mlstm_kernel_id;
 

@@ -32,7 +32,7 @@ SIGNATURES = {
     "mlstm_fw_parallel": (_i, [_vp] * 11 + [_i] * 9 + [_vp, _sz, _vp]),
     "mlstm_fw_static_scratch": (_i, [_vp] * 12 + [_i] * 9 + [_vp]),
     "mlstm_fw_static_scratch_capacity": (_sz, []),
-    "mlstm_bw_workspace_size": (_i, [_i] * 6 + [ctypes.POINTER(_sz)]),
+    "mlstm_bw_workspace_size": (_i, [_i] * 7 + [ctypes.POINTER(_sz)]),
     "mlstm_bw": (_i, [_vp] * 17 + [_i] * 8 + [_vp, _sz, _vp]),
     "mlstm_step": (_i, [_vp] * 9 + [_i] * 6 + [_vp]),
     "mlstm_last_device_error": (_i, [_vp]),

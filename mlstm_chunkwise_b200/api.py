@@ -150,8 +150,8 @@ def mlstm_bw(Q, K, V, i_pre, f_pre, dH, C0=None, n0=None, m0=None, *, chunk_size
     if C0 is not None:
         out.update(dC0=torch.empty_like(C0), dn0=torch.empty_like(n0), dm0=torch.empty_like(m0))
     n = ctypes.c_size_t(0)
-    _lib.check(_lib.lib().mlstm_bw_workspace_size(B, NH, T, DK, DV, chunk_size, ctypes.byref(n)),
-               "mlstm_bw_workspace_size")
+    _lib.check(_lib.lib().mlstm_bw_workspace_size(B, NH, T, DK, DV, chunk_size, _DT[dt],
+                                                  ctypes.byref(n)), "mlstm_bw_workspace_size")
     ws = torch.empty(max(n.value, 1), dtype=torch.uint8, device=dev)
     st = _lib.lib().mlstm_bw(
         _ptr(Q), _ptr(K), _ptr(V), _ptr(i_pre), _ptr(f_pre), _ptr(C0), _ptr(n0), _ptr(m0),

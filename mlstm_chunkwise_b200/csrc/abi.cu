@@ -61,6 +61,7 @@ Problem make_problem(int B, int NH, int T, int DK, int DV, int L, mlstm_gate_mod
   p.BH = B * NH;
   p.gate_sigmoid = gm == MLSTM_GATE_SIGMOID;
   p.key_scale = (float)(1.0 / sqrt((double)DK));
+  p.signed_den = 0;
   p.err = nullptr;
   p.max_polls = g_max_polls;
   return p;
@@ -460,11 +461,11 @@ mlstm_status mlstm_fw_parallel(const void* Q, const void* K, const void* V, cons
 }
 
 mlstm_status mlstm_bw_workspace_size(int B, int NH, int T, int DK, int DV, int chunk_size,
-                                     size_t* bytes) {
-  if (!bytes) return MLSTM_ERR_INVALID_ARG;
+                                     mlstm_dtype dtype, size_t* bytes) {
+  if (!bytes || !valid_enums(dtype, MLSTM_GATE_EXP, MLSTM_ALGO_AUTO)) return MLSTM_ERR_INVALID_ARG;
   mlstm_status s = check_sizes(B, NH, T, DK, DV, chunk_size);
   if (s != MLSTM_OK) return s;
-  *bytes = bwd_workspace_bytes(make_problem(B, NH, T, DK, DV, chunk_size, MLSTM_GATE_EXP));
+  *bytes = bwd_workspace_bytes(make_problem(B, NH, T, DK, DV, chunk_size, MLSTM_GATE_EXP), dtype);
   return MLSTM_OK;
 }
 
@@ -486,7 +487,7 @@ mlstm_status mlstm_bw(const void* Q, const void* K, const void* V, const float* 
   for (const void* q : ptrs)
     if (!aligned16(q)) return MLSTM_ERR_INVALID_ARG;
   Problem p = make_problem(B, NH, T, DK, DV, chunk_size, gate_mode);
-  const size_t need = bwd_workspace_bytes(p);
+  const size_t need = bwd_workspace_bytes(p, dtype);
   if (workspace_bytes < need || !workspace) return MLSTM_ERR_INVALID_ARG;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (T == 0) {  // no output token: the initial state gets no gradient
@@ -500,7 +501,7 @@ mlstm_status mlstm_bw(const void* Q, const void* K, const void* V, const float* 
   }
   p.err = error_word_ptr();
   if (!p.err) return MLSTM_ERR_CUDA;
-  return from_cuda(launch_family(MLSTM_KERNEL_BW, 10, st, [&] {
+  return from_cuda(launch_family(MLSTM_KERNEL_BW, bwd_launches(p, dtype), st, [&] {
     return launch_backward(p, dtype, Q, K, V, i_pre, f_pre, C0, n0, m0, dH, dQ, dK, dV, di_pre,
                            df_pre, dC0, dn0, dm0, workspace, st);
   }));

@@ -1,4 +1,4 @@
-// Backward pass of the chunkwise mLSTM (fp32 CUDA-core kernels).
+// Backward pass of the chunkwise mLSTM (fp32 CUDA-core gradient kernels).
 //
 // The forward ("Tiled Flash Linear Attention: More Efficient Linear RNN and
 // xLSTM Kernels", abstract: the mLSTM as an inter-chunk recurrence plus an
@@ -33,14 +33,18 @@
 // G~_k is the gradient with respect to the state entering chunk k, in that
 // state's frame, so dC0 = G~_0, dn0 = g~_0 and dm0 = <C0, dC0> + n0 . dn0.
 //
-// Launches: the forward's gates, chunk states and outputs (fp32 h and the
-// signed denominator kept), a per-token pass forming du~ and da~, the reverse
-// state recurrence, dq, dk, dv, and the gate gradients (dot products and a
-// reverse scan).  Every kernel tiles 64 x 64 outputs over 256 threads (4 x 4
-// per thread), like the fp32 forward kernels.
+// Launches: the forward's gates, chunk states and outputs (h and the signed
+// denominator kept), a per-token pass forming du~ and da~, the reverse state
+// recurrence, dq, dk, dv, and the gate gradients (dot products and a reverse
+// scan).  The forward is recomputed on the tensor cores for bf16 inputs where
+// the unfused tensor-core path supports the shape (fp32 chunk states, then
+// their bf16 operand copy for the output kernel, h in bf16), else on the fp32
+// kernels (h in fp32).  The gradient kernels tile 64 x 64 outputs over 256
+// threads (4 x 4 per thread), like the fp32 forward kernels.
 #include <math.h>
 
 #include "common.cuh"
+#include "tc.h"
 
 namespace mlstm {
 namespace {
@@ -97,27 +101,28 @@ __device__ __forceinline__ void mac_tile(float (&acc)[4][4], const float (*P)[kT
 // ---------------------------------------------------------------------------
 // du~ [BH, T, DV] and da~ [BH, T]: one warp per token.
 // ---------------------------------------------------------------------------
-template <typename TIn>
+// den_s holds copysign(max(|a|, e^{-m}), a) of the forward (signed_den mode).
+template <typename TIn, typename TH>
 __global__ void __launch_bounds__(kThr)
-bwd_prep_kernel(Problem p, const TIn* __restrict__ dH, const float* __restrict__ H32,
-                const float* __restrict__ a_sig, const float* __restrict__ den,
-                const float* __restrict__ mr, float* __restrict__ dU, float* __restrict__ dA) {
+bwd_prep_kernel(Problem p, const TIn* __restrict__ dH, const TH* __restrict__ Hf,
+                const float* __restrict__ den_s, const float* __restrict__ mr,
+                float* __restrict__ dU, float* __restrict__ dA) {
   const long tok = (long)blockIdx.x * (kThr / 32) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (tok >= (long)p.BH * p.T) return;
-  const float inv = 1.f / den[tok];
+  const float ds = den_s[tok];
+  const float inv = 1.f / fabsf(ds);
   float dot = 0.f;
   for (int c = lane; c < p.DV; c += 32) {
     const float g = to_float(dH[tok * p.DV + c]);
     dU[tok * p.DV + c] = g * inv;
-    dot = fmaf(g, H32[tok * p.DV + c], dot);
+    dot = fmaf(g, to_float(Hf[tok * p.DV + c]), dot);
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
   if (lane == 0) {
-    const float a = a_sig[tok];
-    const bool on_n = fabsf(a) > expf(-mr[tok]);  // the max picked |n.q|
-    dA[tok] = on_n ? -dot * inv * (a >= 0.f ? 1.f : -1.f) : 0.f;
+    const bool on_n = fabsf(ds) > expf(-mr[tok]);  // the max picked |n.q|
+    dA[tok] = on_n ? -dot * inv * (ds >= 0.f ? 1.f : -1.f) : 0.f;
   }
 }
 
@@ -574,19 +579,31 @@ bwd_gates_kernel(Problem p, const float* __restrict__ i_pre, const float* __rest
 // Workspace carve (all fp32): see bwd_workspace_bytes.
 struct BwdWs {
   Gates g;
-  float *C_states, *n_states, *H32, *a_sig, *den, *mr, *dU, *dA, *G_states, *g_states, *qdq,
-      *kdk, *dC0, *dn0;
+  float *C_states, *n_states, *H32, *den, *mr, *dU, *dA, *G_states, *g_states, *qdq, *kdk, *dC0,
+      *dn0, *seg;
+  __nv_bfloat16 *Cb, *H16;  // tensor-core recompute: operand copy of the states, bf16 h
 };
+
+// Whether the forward is recomputed on the tensor cores.
+bool tc_recompute(const Problem& p, mlstm_dtype dt) {
+  return dt == MLSTM_DT_BF16 && tc_unfused_supported(p);
+}
 
 constexpr size_t kAlign = 256;
 inline size_t al(size_t b) { return (b + kAlign - 1) / kAlign * kAlign; }
 
-size_t carve(const Problem& p, char* base, BwdWs* w) {
+size_t carve(const Problem& p, mlstm_dtype dt, char* base, BwdWs* w) {
   const size_t BH = p.BH, T = p.T, NC = p.NC, tpad = NC * p.L, DK = p.DK, DV = p.DV;
+  const bool tc = tc_recompute(p, dt);
   size_t off = 0;
   auto take = [&](size_t n) -> float* {
     float* ptr = base ? reinterpret_cast<float*>(base + off) : nullptr;
     off += al(n * sizeof(float));
+    return ptr;
+  };
+  auto take16 = [&](size_t n) -> __nv_bfloat16* {
+    __nv_bfloat16* ptr = base ? reinterpret_cast<__nv_bfloat16*>(base + off) : nullptr;
+    off += al(n * sizeof(__nv_bfloat16));
     return ptr;
   };
   Gates g;
@@ -599,8 +616,10 @@ size_t carve(const Problem& p, char* base, BwdWs* w) {
   x.g = g;
   x.C_states = take(BH * NC * DK * DV);
   x.n_states = take(BH * NC * DK);
-  x.H32 = take(BH * T * DV);
-  x.a_sig = take(BH * T);
+  x.H32 = tc ? nullptr : take(BH * T * DV);
+  x.Cb = tc ? take16(BH * NC * DK * DV) : nullptr;
+  x.H16 = tc ? take16(BH * T * DV) : nullptr;
+  x.seg = tc ? take(tc_states_segment_floats(p)) : nullptr;
   x.den = take(BH * T);
   x.mr = take(BH * T);
   x.dU = take(BH * T * DV);
@@ -622,21 +641,38 @@ cudaError_t launch_bwd_t(const Problem& p, mlstm_dtype dt, const void* Q, const 
                          void* dV, float* di, float* df, float* dC0, float* dn0, float* dm0,
                          void* ws, cudaStream_t st) {
   BwdWs w;
-  carve(p, static_cast<char*>(ws), &w);
+  carve(p, dt, static_cast<char*>(ws), &w);
   const TIn* q = static_cast<const TIn*>(Q);
   const TIn* k = static_cast<const TIn*>(K);
   const TIn* v = static_cast<const TIn*>(V);
+  Problem ps = p;
+  ps.signed_den = 1;  // the forward outputs keep the sign of the denominator
+  const bool tc = tc_recompute(p, dt);
   cudaError_t e = launch_gates(p, i_pre, f_pre, m0, w.g, st);
   if (e != cudaSuccess) return e;
-  e = launch_simt_states(p, dt, K, V, C0, n0, w.g, w.C_states, w.n_states, nullptr, nullptr,
-                         nullptr, st);
-  if (e != cudaSuccess) return e;
-  e = launch_simt_parallel(p, dt, Q, K, V, w.g, w.C_states, w.n_states, nullptr, w.den, w.mr, st,
-                           w.H32, w.a_sig);
+  if (tc) {
+    e = launch_tc_states(p, K, V, C0, n0, w.g, w.C_states, nullptr, w.n_states, nullptr, nullptr,
+                         nullptr, w.seg, st);
+    if (e != cudaSuccess) return e;
+    e = launch_states_to_operand(w.C_states, w.Cb, (long)p.BH * p.NC, p.DK, p.DV, st);
+    if (e != cudaSuccess) return e;
+    e = launch_tc_parallel(ps, Q, K, V, w.g, w.Cb, w.n_states, w.H16, w.den, w.mr, st);
+  } else {
+    e = launch_simt_states(p, dt, K, V, C0, n0, w.g, w.C_states, w.n_states, nullptr, nullptr,
+                           nullptr, st);
+    if (e != cudaSuccess) return e;
+    e = launch_simt_parallel(ps, dt, Q, K, V, w.g, w.C_states, w.n_states, nullptr, w.den, w.mr,
+                             st, w.H32);
+  }
   if (e != cudaSuccess) return e;
   const long toks = (long)p.BH * p.T;
-  bwd_prep_kernel<TIn><<<(unsigned)((toks + 7) / 8), kThr, 0, st>>>(
-      p, static_cast<const TIn*>(dH), w.H32, w.a_sig, w.den, w.mr, w.dU, w.dA);
+  const unsigned prep_blocks = (unsigned)((toks + 7) / 8);
+  if (tc)
+    bwd_prep_kernel<TIn, __nv_bfloat16><<<prep_blocks, kThr, 0, st>>>(
+        p, static_cast<const TIn*>(dH), w.H16, w.den, w.mr, w.dU, w.dA);
+  else
+    bwd_prep_kernel<TIn, float><<<prep_blocks, kThr, 0, st>>>(
+        p, static_cast<const TIn*>(dH), w.H32, w.den, w.mr, w.dU, w.dA);
   const int nk = (p.DK + kT - 1) / kT, nv = (p.DV + kT - 1) / kT, nt = (p.T + kT - 1) / kT;
   bwd_states_kernel<TIn><<<dim3(nv, nk, p.BH), kThr, 0, st>>>(p, q, w.dU, w.dA, w.g, w.G_states,
                                                               w.g_states, w.dC0, w.dn0);
@@ -666,7 +702,13 @@ cudaError_t launch_bwd_t(const Problem& p, mlstm_dtype dt, const void* Q, const 
 
 }  // namespace
 
-size_t bwd_workspace_bytes(const Problem& p) { return carve(p, nullptr, nullptr); }
+size_t bwd_workspace_bytes(const Problem& p, mlstm_dtype dt) { return carve(p, dt, nullptr, nullptr); }
+
+int bwd_launches(const Problem& p, mlstm_dtype dt) {
+  // gates (2) + recompute (simt: 2; tensor cores: states [+ fix-up] + operand copy + outputs)
+  // + prep, reverse states, dq, dk, dv, gate gradients (6)
+  return 2 + (tc_recompute(p, dt) ? 2 + tc_states_launches(p) : 2) + 6;
+}
 
 cudaError_t launch_backward(const Problem& p, mlstm_dtype dt, const void* Q, const void* K,
                             const void* V, const float* i_pre, const float* f_pre,

@@ -31,6 +31,7 @@ struct Problem {
   int BH;                   // B * NH
   int gate_sigmoid;         // 0: log i = i_pre; 1: log i = logsigmoid(i_pre)
   float key_scale;          // 1 / sqrt(DK)
+  int signed_den;           // output kernels: n_out = copysign(max(|den|, e^{-m}), den)
   uint32_t* err;            // device error word (see raise_error)
   unsigned long long max_polls;  // spin limit of every bounded wait
 };
@@ -77,7 +78,8 @@ cudaError_t launch_gates(const Problem& p, const float* i_pre, const float* f_pr
 // Backward pass (bwd.cu).  dH in the input dtype; dQ, dK, dV in the input
 // dtype; di, df [BH, T], dC0 [BH, DK, DV], dn0 [BH, DK], dm0 [BH] fp32
 // (the last three nullable).  `ws` holds bwd_workspace_bytes(p) bytes.
-size_t bwd_workspace_bytes(const Problem& p);
+size_t bwd_workspace_bytes(const Problem& p, mlstm_dtype dt);
+int bwd_launches(const Problem& p, mlstm_dtype dt);
 cudaError_t launch_backward(const Problem& p, mlstm_dtype dt, const void* Q, const void* K,
                             const void* V, const float* i_pre, const float* f_pre,
                             const float* C0, const float* n0, const float* m0, const void* dH,
@@ -93,5 +95,5 @@ cudaError_t launch_simt_states(const Problem& p, mlstm_dtype dt, const void* K, 
 cudaError_t launch_simt_parallel(const Problem& p, mlstm_dtype dt, const void* Q, const void* K,
                                  const void* V, Gates g, const float* C_states,
                                  const float* n_states, void* H, float* n_out, float* m_out,
-                                 cudaStream_t st, float* H32 = nullptr, float* a_out = nullptr);
+                                 cudaStream_t st, float* H32 = nullptr);
 }  // namespace mlstm

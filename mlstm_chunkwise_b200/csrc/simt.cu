@@ -135,7 +135,7 @@ simt_parallel_kernel(Problem p, const TIn* __restrict__ Q, const TIn* __restrict
                      const TIn* __restrict__ V, Gates g, const float* __restrict__ C_states,
                      const float* __restrict__ n_states, TIn* __restrict__ H,
                      float* __restrict__ n_out, float* __restrict__ m_out,
-                     float* __restrict__ H32, float* __restrict__ a_out) {
+                     float* __restrict__ H32) {
   constexpr int kSlab = 32;
   // Phase buffers alias one another: {Qs, Ks} or {Qs, Cs} during the
   // contractions over DK, {Ps, Vs} during P.V.
@@ -285,9 +285,8 @@ simt_parallel_kernel(Problem p, const TIn* __restrict__ Q, const TIn* __restrict
       else H[((long)bh * T + t) * DV + c] = from_float<TIn>(acc[i][j] * inv);
     }
     if (blockIdx.x == 0 && tx == 0) {
-      if (n_out) n_out[(long)bh * T + t] = denom;
+      if (n_out) n_out[(long)bh * T + t] = p.signed_den ? copysignf(denom, den[i]) : denom;
       if (m_out) m_out[(long)bh * T + t] = mr;
-      if (a_out) a_out[(long)bh * T + t] = den[i];  // signed, before the max
     }
   }
 }
@@ -312,18 +311,18 @@ cudaError_t launch_simt_states(const Problem& p, mlstm_dtype dt, const void* K, 
 cudaError_t launch_simt_parallel(const Problem& p, mlstm_dtype dt, const void* Q, const void* K,
                                  const void* V, Gates g, const float* C_states,
                                  const float* n_states, void* H, float* n_out, float* m_out,
-                                 cudaStream_t st, float* H32, float* a_out) {
+                                 cudaStream_t st, float* H32) {
   if (p.T == 0) return cudaSuccess;
   const int qblocks = (p.T + kTile - 1) / kTile;
   dim3 grid((p.DV + kTile - 1) / kTile, qblocks, p.BH);
   if (dt == MLSTM_DT_F32)
     simt_parallel_kernel<float><<<grid, kThreads, 0, st>>>(
         p, (const float*)Q, (const float*)K, (const float*)V, g, C_states, n_states, (float*)H,
-        n_out, m_out, H32, a_out);
+        n_out, m_out, H32);
   else
     simt_parallel_kernel<__nv_bfloat16><<<grid, kThreads, 0, st>>>(
         p, (const __nv_bfloat16*)Q, (const __nv_bfloat16*)K, (const __nv_bfloat16*)V, g,
-        C_states, n_states, (__nv_bfloat16*)H, n_out, m_out, H32, a_out);
+        C_states, n_states, (__nv_bfloat16*)H, n_out, m_out, H32);
   return cudaGetLastError();
 }
 

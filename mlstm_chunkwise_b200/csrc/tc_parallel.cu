@@ -556,7 +556,7 @@ tc_parallel_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       tc_fence_before();
       mbar_arrive(bar.o_empty(n % C::kOBufs));
       if (t < p.T && x.dv0 == 0 && h == 0) {
-        if (n_out) n_out[(long)x.bh * p.T + t] = denom;
+        if (n_out) n_out[(long)x.bh * p.T + t] = p.signed_den ? copysignf(denom, den) : denom;
         if (m_out) m_out[(long)x.bh * p.T + t] = mr;
       }
     }

@@ -480,7 +480,7 @@ tc_parallel_wide_kernel(const __grid_constant__ CUtensorMap tm_q,
       const float denom = fmaxf(fabsf(den), expf(-mr));
       const float inv = 1.f / denom;
       if (t < p.T && h == 0) {
-        if (n_out) n_out[(long)x.bh * p.T + t] = denom;
+        if (n_out) n_out[(long)x.bh * p.T + t] = p.signed_den ? copysignf(denom, den) : denom;
         if (m_out) m_out[(long)x.bh * p.T + t] = mr;
       }
 

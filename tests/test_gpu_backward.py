@@ -26,6 +26,8 @@ CASES = [
     (1, 2, 512, 128, 128, 256, "f32", "sigmoid", True),
     (1, 1, 130, 100, 72, 64, "f32", "exp", True),       # dims that are not tile multiples
     (1, 2, 1, 64, 64, 64, "f32", "exp", True),          # single token
+    (1, 2, 640, 256, 512, 256, "bf16", "exp", True),    # 7B head shape: forward recomputed on TC
+    (1, 2, 384, 128, 128, 64, "bf16", "sigmoid", False),  # chunk 64 on TC (pair mode)
 ]
 
 
