@@ -43,6 +43,8 @@
 // threads (4 x 4 per thread), like the fp32 forward kernels.
 #include <math.h>
 
+#include <type_traits>
+
 #include "common.cuh"
 #include "tc.h"
 
@@ -212,163 +214,241 @@ bwd_states_kernel(Problem p, const TIn* __restrict__ Q, const float* __restrict_
 }
 
 // ---------------------------------------------------------------------------
-// dq: one block per (b, h, 64 queries, 64 columns of d_qk).  Also adds the
-// block's part of q_t . dq_t into qdq (zeroed beforehand).
+// dq, dk, dv.  A block owns 64 rows (queries for dq, keys for dk and dv) and a
+// range of kW <= 256 output columns, so the 64 x 64 products it needs per
+// pair of row tiles (dP = dU V^T, or S = K^ Q^T) are formed once for the whole
+// range rather than once per 64 columns.  Layouts (all in shared memory,
+// contraction index first so that every inner-loop read is a float4):
+//   At[c][r]  A operand: 64 rows, slab of 32 along the contraction
+//   Bw[c][j]  B operand: kW columns (or 64 for the square products)
+//   Pt[s][r]  the gated 64 x 64 tile, contraction index (s or t) first
+// Square products use a 16 x 16 thread grid with 4 x 4 outputs per thread;
+// the wide accumulators a grid of 8 row groups (warps) x 32 lanes with 8 rows x
+// kW/32 columns per thread (columns 4 lane + {0..3} and 128 + 4 lane + {0..3}
+// for kW = 256, so every float4 read of a warp is contiguous).
 // ---------------------------------------------------------------------------
-template <typename TIn>
+constexpr int kTP = kT + 4;  // row stride of At and Pt (keeps float4 alignment)
+
+template <int kW>
+struct WideSmem {
+  float At[kS][kTP];
+  float Bw[kS][kW];
+  float Pt[kT][kTP];
+  float mu[kT], da[kT], acol[kT], fw[kT];
+};
+
+template <int kW>
+__device__ __forceinline__ int wide_col(int lane, int j) {
+  constexpr int kC = kW / 32;
+  return kC >= 4 ? (j >> 2) * 128 + 4 * lane + (j & 3) : kC * lane + j;
+}
+
+// acc[i][j] += sum_{c < kS} A[c][wy*8 + i] * B[c][wide_col(wx, j)]
+template <int kW>
+__device__ __forceinline__ void mac_wide(float (&acc)[8][kW / 32], const float (*A)[kTP],
+                                         const float (*B)[kW], int wy, int wx) {
+  constexpr int kC = kW / 32;
+#pragma unroll 4
+  for (int c = 0; c < kS; ++c) {
+    const float4 a0 = *reinterpret_cast<const float4*>(&A[c][wy * 8]);
+    const float4 a1 = *reinterpret_cast<const float4*>(&A[c][wy * 8 + 4]);
+    const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+    float b[kC];
+    if (kC >= 4) {
+#pragma unroll
+      for (int h = 0; h < kC / 4; ++h) {
+        const float4 bv = *reinterpret_cast<const float4*>(&B[c][h * 128 + 4 * wx]);
+        b[4 * h] = bv.x; b[4 * h + 1] = bv.y; b[4 * h + 2] = bv.z; b[4 * h + 3] = bv.w;
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < kC; ++j) b[j] = B[c][kC * wx + j];
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+      for (int j = 0; j < kC; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+  }
+}
+
+// acc[i][j] += sum_{c < kS} A[c][ty*4 + i] * B[c][tx*4 + j]   (64 x 64 product)
+template <int kW>
+__device__ __forceinline__ void mac_square(float (&acc)[4][4], const float (*A)[kTP],
+                                           const float (*B)[kW], int ty, int tx) {
+#pragma unroll 4
+  for (int c = 0; c < kS; ++c) {
+    const float4 av = *reinterpret_cast<const float4*>(&A[c][ty * 4]);
+    const float4 bv = *reinterpret_cast<const float4*>(&B[c][tx * 4]);
+    const float a[4] = {av.x, av.y, av.z, av.w}, b[4] = {bv.x, bv.y, bv.z, bv.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+  }
+}
+
+// dst[c][r] = scale * X[(row0 + r) * ld + c0 + c] for r < nrows (<= width of
+// dst rows), c < kS; zero outside [0, rows_valid) x [0, cols_valid).  Lanes
+// take consecutive rows (conflict-free shared stores).
+template <typename TX, int kLd>
+__device__ __forceinline__ void load_cmajor(float (*dst)[kLd], const TX* X, long row0, int nrows,
+                                            long rows_valid, long ld, int c0, int cols_valid,
+                                            float scale) {
+  for (int e = threadIdx.x; e < nrows * (kS / 4); e += kThr) {
+    const int r = e % nrows, grp = e / nrows;
+    const long row = row0 + r;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int c = c0 + grp * 4 + q;
+      dst[grp * 4 + q][r] = (row < rows_valid && c < cols_valid) ? scale * to_float(X[row * ld + c]) : 0.f;
+    }
+  }
+}
+
+// dst[s][j] = scale * X[(row0 + s) * ld + col0 + j] for s < kS, j < kW: the
+// contraction runs along X's rows, the wide index along its columns.
+template <typename TX, int kW>
+__device__ __forceinline__ void load_rmajor(float (*dst)[kW], const TX* X, long row0,
+                                            long rows_valid, long ld, int col0, int cols_valid,
+                                            float scale) {
+  for (int e = threadIdx.x; e < kS * (kW / 4); e += kThr) {
+    const int j4 = e % (kW / 4), s = e / (kW / 4);
+    const long row = row0 + s;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int col = col0 + 4 * j4 + q;
+      dst[s][4 * j4 + q] = (row < rows_valid && col < cols_valid) ? scale * to_float(X[row * ld + col]) : 0.f;
+    }
+  }
+}
+
+// dq for 64 queries and kW columns of d_qk; adds q_t . dq_t into qdq.
+template <typename TIn, int kW>
 __global__ void __launch_bounds__(kThr)
 bwd_dq_kernel(Problem p, const TIn* __restrict__ Q, const TIn* __restrict__ K,
               const TIn* __restrict__ V, Gates g, const float* __restrict__ C_states,
               const float* __restrict__ n_states, const float* __restrict__ dU,
               const float* __restrict__ dA, TIn* __restrict__ dQ, float* __restrict__ qdq) {
-  __shared__ float As[kT][kS + 1];
-  __shared__ float Bs[kT][kT];   // a slab [kS][kT], or a whole [kT][kT] tile
-  __shared__ float Ps[kT][kT + 1];
-  __shared__ float mu_s[kT], das[kT], acol_s[kT];
-  const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
-  const int dk0 = blockIdx.x * kT, bh = blockIdx.z;
+  constexpr int kC = kW / 32;
+  extern __shared__ __align__(16) unsigned char dsm[];
+  WideSmem<kW>& sm = *reinterpret_cast<WideSmem<kW>*>(dsm);
+  const int tid = threadIdx.x, wy = tid >> 5, wx = tid & 31, ty = tid >> 4, tx = tid & 15;
+  const int d0 = blockIdx.x * kW, bh = blockIdx.z;
   const long t0 = (long)blockIdx.y * kT;
   const int DK = p.DK, DV = p.DV, T = p.T, L = p.L, NC = p.NC;
   const int k = (int)(t0 / L);
-  const long tpad = (long)NC * L;
+  const long tpad = (long)NC * L, base = (long)bh * T;
   const float m_in = g.mchk[(long)bh * (NC + 1) + k];
   if (tid < kT) {
     const long t = t0 + tid;
-    mu_s[tid] = fmaxf(m_in, g.amax[(long)bh * tpad + t]);
-    das[tid] = t < T ? dA[(long)bh * T + t] : 0.f;
+    sm.mu[tid] = fmaxf(m_in, g.amax[(long)bh * tpad + t]);
+    sm.da[tid] = t < T ? dA[base + t] : 0.f;
+    sm.fw[tid] = expf(m_in - sm.mu[tid]);
   }
-  __syncthreads();
-  float acc[4][4] = {};
-  // inter: X[t][d] = sum_c du~[t][c] C_k[d][c]
+  float acc[8][kC] = {};
+  // inter: sum_c du~[t][c] C_k[d][c]
   const float* Ck = C_states + ((long)bh * NC + k) * DK * DV;
   for (int c0 = 0; c0 < DV; c0 += kS) {
-    for (int e = tid; e < kT * kS; e += kThr) {
-      const int r = e / kS, c = e % kS;
-      const long t = t0 + r;
-      As[r][c] = (t < T && c0 + c < DV) ? dU[((long)bh * T + t) * DV + c0 + c] : 0.f;
-    }
-    for (int e = tid; e < kS * kT; e += kThr) {
-      const int c = e / kT, j = e % kT;
-      Bs[c][j] = (c0 + c < DV && dk0 + j < DK) ? Ck[(long)(dk0 + j) * DV + c0 + c] : 0.f;
-    }
+    load_cmajor<float, kTP>(sm.At, dU + base * DV, t0, kT, T, DV, c0, DV, 1.f);
+    load_cmajor<float, kW>(sm.Bw, Ck, d0, kW, DK, DV, c0, DV, 1.f);
     __syncthreads();
-    mac_slab(acc, As, Bs, ty, tx);
+    mac_wide<kW>(acc, sm.At, sm.Bw, wy, wx);
     __syncthreads();
   }
   const float* nk = n_states + ((long)bh * NC + k) * DK;
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int r = ty * 4 + i;
-    const float f = expf(m_in - mu_s[r]);
+  for (int i = 0; i < 8; ++i) {
+    const int r = wy * 8 + i;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int d = dk0 + tx * 4 + j;
-      acc[i][j] = f * (acc[i][j] + das[r] * (d < DK ? nk[d] : 0.f));
+    for (int j = 0; j < kC; ++j) {
+      const int d = d0 + wide_col<kW>(wx, j);
+      acc[i][j] = sm.fw[r] * (acc[i][j] + sm.da[r] * (d < DK ? nk[d] : 0.f));
     }
   }
   // intra: key tiles of the chunk up to the diagonal
   for (long s0 = (long)k * L; s0 <= t0; s0 += kT) {
+    if (tid < kT) sm.acol[tid] = g.acol[(long)bh * tpad + s0 + tid];
     float dP[4][4] = {};
     for (int c0 = 0; c0 < DV; c0 += kS) {
-      for (int e = tid; e < kT * kS; e += kThr) {
-        const int r = e / kS, c = e % kS;
-        const long t = t0 + r;
-        As[r][c] = (t < T && c0 + c < DV) ? dU[((long)bh * T + t) * DV + c0 + c] : 0.f;
-      }
-      for (int e = tid; e < kS * kT; e += kThr) {
-        const int c = e / kT, j = e % kT;
-        Bs[c][j] = ld(V, ((long)bh * T + s0 + j) * DV + c0 + c, s0 + j < T && c0 + c < DV);
-      }
+      load_cmajor<float, kTP>(sm.At, dU + base * DV, t0, kT, T, DV, c0, DV, 1.f);
+      load_cmajor<TIn, kW>(sm.Bw, V + base * DV, s0, kT, T, DV, c0, DV, 1.f);
       __syncthreads();
-      mac_slab(dP, As, Bs, ty, tx);
+      mac_square<kW>(dP, sm.At, sm.Bw, ty, tx);
       __syncthreads();
     }
-    if (tid < kT) acol_s[tid] = g.acol[(long)bh * tpad + s0 + tid];
-    __syncthreads();
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const int r = ty * 4 + i, s = tx * 4 + j;
-        const bool ok = s0 + s <= t0 + r && t0 + r < T;
-        Ps[r][s] = ok ? expf(acol_s[s] - mu_s[r]) * (dP[i][j] + das[r]) : 0.f;
+        const int r = ty * 4 + i, sc = tx * 4 + j;
+        const bool ok = s0 + sc <= t0 + r && t0 + r < T;
+        sm.Pt[sc][r] = ok ? expf(sm.acol[sc] - sm.mu[r]) * (dP[i][j] + sm.da[r]) : 0.f;
       }
-    for (int e = tid; e < kT * kT; e += kThr) {
-      const int s = e / kT, j = e % kT;
-      Bs[s][j] = p.key_scale * ld(K, ((long)bh * T + s0 + s) * DK + dk0 + j,
-                                  s0 + s < T && dk0 + j < DK);
+    for (int half = 0; half < 2; ++half) {
+      load_rmajor<TIn, kW>(sm.Bw, K + base * DK, s0 + half * kS, T, DK, d0, DK, p.key_scale);
+      __syncthreads();
+      mac_wide<kW>(acc, sm.Pt + half * kS, sm.Bw, wy, wx);
+      __syncthreads();
     }
-    __syncthreads();
-    mac_tile(acc, Ps, Bs, ty, tx);
-    __syncthreads();
   }
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const long t = t0 + ty * 4 + i;
+  for (int i = 0; i < 8; ++i) {
+    const long t = t0 + wy * 8 + i;
     float part = 0.f;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int d = dk0 + tx * 4 + j;
+    for (int j = 0; j < kC; ++j) {
+      const int d = d0 + wide_col<kW>(wx, j);
       if (t < T && d < DK) {
-        dQ[((long)bh * T + t) * DK + d] = from_float<TIn>(acc[i][j]);
-        part = fmaf(to_float(Q[((long)bh * T + t) * DK + d]), acc[i][j], part);
+        dQ[(base + t) * DK + d] = from_float<TIn>(acc[i][j]);
+        part = fmaf(to_float(Q[(base + t) * DK + d]), acc[i][j], part);
       }
     }
-    part = sum16(part);
-    if (tx == 0 && t < T) atomicAdd(&qdq[(long)bh * T + t], part);
+    part = warp_sum(part);
+    if (wx == 0 && t < T) atomicAdd(&qdq[base + t], part);
   }
 }
 
-// ---------------------------------------------------------------------------
-// dk: one block per (b, h, 64 keys, 64 columns of d_qk).  Adds k_s . dk_s
-// into kdk (zeroed beforehand).
-// ---------------------------------------------------------------------------
-template <typename TIn>
+// dk for 64 keys and kW columns of d_qk; adds k_s . dk_s into kdk.
+template <typename TIn, int kW>
 __global__ void __launch_bounds__(kThr)
 bwd_dk_kernel(Problem p, const TIn* __restrict__ Q, const TIn* __restrict__ K,
               const TIn* __restrict__ V, Gates g, const float* __restrict__ G_states,
               const float* __restrict__ g_states, const float* __restrict__ dU,
               const float* __restrict__ dA, TIn* __restrict__ dK, float* __restrict__ kdk) {
-  __shared__ float As[kT][kS + 1];
-  __shared__ float Bs[kT][kT];
-  __shared__ float Ps[kT][kT + 1];
-  __shared__ float mu_s[kT], das[kT], acol_s[kT];
-  const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
-  const int dk0 = blockIdx.x * kT, bh = blockIdx.z;
+  constexpr int kC = kW / 32;
+  extern __shared__ __align__(16) unsigned char dsm[];
+  WideSmem<kW>& sm = *reinterpret_cast<WideSmem<kW>*>(dsm);
+  const int tid = threadIdx.x, wy = tid >> 5, wx = tid & 31, ty = tid >> 4, tx = tid & 15;
+  const int d0 = blockIdx.x * kW, bh = blockIdx.z;
   const long s0 = (long)blockIdx.y * kT;
   const int DK = p.DK, DV = p.DV, T = p.T, L = p.L, NC = p.NC;
   const int k = (int)(s0 / L);
-  const long tpad = (long)NC * L;
+  const long tpad = (long)NC * L, base = (long)bh * T;
   const float m_in = g.mchk[(long)bh * (NC + 1) + k];
   const float m_out = g.mchk[(long)bh * (NC + 1) + k + 1];
   const float gk = g.gtot[(long)bh * NC + k];
-  if (tid < kT) acol_s[tid] = g.acol[(long)bh * tpad + s0 + tid];
-  __syncthreads();
-  float acc[4][4] = {};
-  // inter: Y[s][d] = sum_c v_s[c] G~_{k+1}[d][c] + g~_{k+1}[d], times w_s
+  if (tid < kT) {
+    sm.acol[tid] = g.acol[(long)bh * tpad + s0 + tid];
+    sm.fw[tid] = expf(gk + sm.acol[tid] - m_out);  // 0 on padding (acol = -inf)
+  }
+  float acc[8][kC] = {};
+  // inter: sum_c v_s[c] G~_{k+1}[d][c] + g~_{k+1}[d], times w_s
   const float* Gk = G_states + ((long)bh * (NC + 1) + k + 1) * DK * DV;
   const float* gk1 = g_states + ((long)bh * (NC + 1) + k + 1) * DK;
   for (int c0 = 0; c0 < DV; c0 += kS) {
-    for (int e = tid; e < kT * kS; e += kThr) {
-      const int r = e / kS, c = e % kS;
-      As[r][c] = ld(V, ((long)bh * T + s0 + r) * DV + c0 + c, s0 + r < T && c0 + c < DV);
-    }
-    for (int e = tid; e < kS * kT; e += kThr) {
-      const int c = e / kT, j = e % kT;
-      Bs[c][j] = (c0 + c < DV && dk0 + j < DK) ? Gk[(long)(dk0 + j) * DV + c0 + c] : 0.f;
-    }
+    load_cmajor<TIn, kTP>(sm.At, V + base * DV, s0, kT, T, DV, c0, DV, 1.f);
+    load_cmajor<float, kW>(sm.Bw, Gk, d0, kW, DK, DV, c0, DV, 1.f);
     __syncthreads();
-    mac_slab(acc, As, Bs, ty, tx);
+    mac_wide<kW>(acc, sm.At, sm.Bw, wy, wx);
     __syncthreads();
   }
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int r = ty * 4 + i;
-    const float w = expf(gk + acol_s[r] - m_out);  // 0 on padding (acol = -inf)
+  for (int i = 0; i < 8; ++i) {
+    const int r = wy * 8 + i;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int d = dk0 + tx * 4 + j;
-      acc[i][j] = w * (acc[i][j] + (d < DK ? gk1[d] : 0.f));
+    for (int j = 0; j < kC; ++j) {
+      const int d = d0 + wide_col<kW>(wx, j);
+      acc[i][j] = sm.fw[r] * (acc[i][j] + (d < DK ? gk1[d] : 0.f));
     }
   }
   // intra: query tiles of the chunk from the diagonal on
@@ -376,146 +456,119 @@ bwd_dk_kernel(Problem p, const TIn* __restrict__ Q, const TIn* __restrict__ K,
   for (long q0 = s0; q0 < chunk_end && q0 < T; q0 += kT) {
     if (tid < kT) {
       const long t = q0 + tid;
-      mu_s[tid] = fmaxf(m_in, g.amax[(long)bh * tpad + t]);
-      das[tid] = t < T ? dA[(long)bh * T + t] : 0.f;
+      sm.mu[tid] = fmaxf(m_in, g.amax[(long)bh * tpad + t]);
+      sm.da[tid] = t < T ? dA[base + t] : 0.f;
     }
-    float dP[4][4] = {};  // [s][t]
+    float dP[4][4] = {};  // [key s][query t]
     for (int c0 = 0; c0 < DV; c0 += kS) {
-      for (int e = tid; e < kT * kS; e += kThr) {
-        const int r = e / kS, c = e % kS;
-        As[r][c] = ld(V, ((long)bh * T + s0 + r) * DV + c0 + c, s0 + r < T && c0 + c < DV);
-      }
-      for (int e = tid; e < kS * kT; e += kThr) {
-        const int c = e / kT, j = e % kT;
-        const long t = q0 + j;
-        Bs[c][j] = (t < T && c0 + c < DV) ? dU[((long)bh * T + t) * DV + c0 + c] : 0.f;
-      }
+      load_cmajor<TIn, kTP>(sm.At, V + base * DV, s0, kT, T, DV, c0, DV, 1.f);
+      load_cmajor<float, kW>(sm.Bw, dU + base * DV, q0, kT, T, DV, c0, DV, 1.f);
       __syncthreads();
-      mac_slab(dP, As, Bs, ty, tx);
+      mac_square<kW>(dP, sm.At, sm.Bw, ty, tx);
       __syncthreads();
     }
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const int s = ty * 4 + i, r = tx * 4 + j;  // key s, query r
-        const bool ok = q0 + r >= s0 + s && q0 + r < T;
-        Ps[s][r] = ok ? expf(acol_s[s] - mu_s[r]) * (dP[i][j] + das[r]) : 0.f;
+        const int sr = ty * 4 + i, tq = tx * 4 + j;
+        const bool ok = q0 + tq >= s0 + sr && q0 + tq < T;
+        sm.Pt[tq][sr] = ok ? expf(sm.acol[sr] - sm.mu[tq]) * (dP[i][j] + sm.da[tq]) : 0.f;
       }
-    for (int e = tid; e < kT * kT; e += kThr) {
-      const int r = e / kT, j = e % kT;
-      Bs[r][j] = ld(Q, ((long)bh * T + q0 + r) * DK + dk0 + j, q0 + r < T && dk0 + j < DK);
+    for (int half = 0; half < 2; ++half) {
+      load_rmajor<TIn, kW>(sm.Bw, Q + base * DK, q0 + half * kS, T, DK, d0, DK, 1.f);
+      __syncthreads();
+      mac_wide<kW>(acc, sm.Pt + half * kS, sm.Bw, wy, wx);
+      __syncthreads();
     }
-    __syncthreads();
-    mac_tile(acc, Ps, Bs, ty, tx);
-    __syncthreads();
   }
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const long s = s0 + ty * 4 + i;
+  for (int i = 0; i < 8; ++i) {
+    const long sr = s0 + wy * 8 + i;
     float part = 0.f;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int d = dk0 + tx * 4 + j;
-      if (s < T && d < DK) {
-        const float dk = p.key_scale * acc[i][j];
-        dK[((long)bh * T + s) * DK + d] = from_float<TIn>(dk);
-        part = fmaf(to_float(K[((long)bh * T + s) * DK + d]), dk, part);
+    for (int j = 0; j < kC; ++j) {
+      const int d = d0 + wide_col<kW>(wx, j);
+      if (sr < T && d < DK) {
+        const float v = p.key_scale * acc[i][j];
+        dK[(base + sr) * DK + d] = from_float<TIn>(v);
+        part = fmaf(to_float(K[(base + sr) * DK + d]), v, part);
       }
     }
-    part = sum16(part);
-    if (tx == 0 && s < T) atomicAdd(&kdk[(long)bh * T + s], part);
+    part = warp_sum(part);
+    if (wx == 0 && sr < T) atomicAdd(&kdk[base + sr], part);
   }
 }
 
-// ---------------------------------------------------------------------------
-// dv: one block per (b, h, 64 keys, 64 columns of d_v).
-// ---------------------------------------------------------------------------
-template <typename TIn>
+// dv for 64 keys and kW columns of d_v.
+template <typename TIn, int kW>
 __global__ void __launch_bounds__(kThr)
 bwd_dv_kernel(Problem p, const TIn* __restrict__ Q, const TIn* __restrict__ K, Gates g,
               const float* __restrict__ G_states, const float* __restrict__ dU,
               TIn* __restrict__ dV) {
-  __shared__ float As[kT][kS + 1];
-  __shared__ float Bs[kT][kT];
-  __shared__ float Ps[kT][kT + 1];
-  __shared__ float mu_s[kT], acol_s[kT];
-  const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
-  const int dv0 = blockIdx.x * kT, bh = blockIdx.z;
+  constexpr int kC = kW / 32;
+  extern __shared__ __align__(16) unsigned char dsm[];
+  WideSmem<kW>& sm = *reinterpret_cast<WideSmem<kW>*>(dsm);
+  const int tid = threadIdx.x, wy = tid >> 5, wx = tid & 31, ty = tid >> 4, tx = tid & 15;
+  const int c0w = blockIdx.x * kW, bh = blockIdx.z;
   const long s0 = (long)blockIdx.y * kT;
   const int DK = p.DK, DV = p.DV, T = p.T, L = p.L, NC = p.NC;
   const int k = (int)(s0 / L);
-  const long tpad = (long)NC * L;
+  const long tpad = (long)NC * L, base = (long)bh * T;
   const float m_in = g.mchk[(long)bh * (NC + 1) + k];
   const float m_out = g.mchk[(long)bh * (NC + 1) + k + 1];
   const float gk = g.gtot[(long)bh * NC + k];
-  if (tid < kT) acol_s[tid] = g.acol[(long)bh * tpad + s0 + tid];
-  __syncthreads();
-  float acc[4][4] = {};
-  // inter: Z[s][c] = sum_d k^_s[d] G~_{k+1}[d][c], times w_s
+  if (tid < kT) {
+    sm.acol[tid] = g.acol[(long)bh * tpad + s0 + tid];
+    sm.fw[tid] = expf(gk + sm.acol[tid] - m_out);
+  }
+  float acc[8][kC] = {};
+  // inter: sum_d k^_s[d] G~_{k+1}[d][c], times w_s
   const float* Gk = G_states + ((long)bh * (NC + 1) + k + 1) * DK * DV;
-  for (int d0 = 0; d0 < DK; d0 += kS) {
-    for (int e = tid; e < kT * kS; e += kThr) {
-      const int r = e / kS, c = e % kS;
-      As[r][c] = p.key_scale * ld(K, ((long)bh * T + s0 + r) * DK + d0 + c,
-                                  s0 + r < T && d0 + c < DK);
-    }
-    for (int e = tid; e < kS * kT; e += kThr) {
-      const int c = e / kT, j = e % kT;
-      Bs[c][j] = (d0 + c < DK && dv0 + j < DV) ? Gk[(long)(d0 + c) * DV + dv0 + j] : 0.f;
-    }
+  for (int dd = 0; dd < DK; dd += kS) {
+    load_cmajor<TIn, kTP>(sm.At, K + base * DK, s0, kT, T, DK, dd, DK, p.key_scale);
+    load_rmajor<float, kW>(sm.Bw, Gk, dd, DK, DV, c0w, DV, 1.f);
     __syncthreads();
-    mac_slab(acc, As, Bs, ty, tx);
+    mac_wide<kW>(acc, sm.At, sm.Bw, wy, wx);
     __syncthreads();
   }
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float w = expf(gk + acol_s[ty * 4 + i] - m_out);
+  for (int i = 0; i < 8; ++i)
 #pragma unroll
-    for (int j = 0; j < 4; ++j) acc[i][j] *= w;
-  }
+    for (int j = 0; j < kC; ++j) acc[i][j] *= sm.fw[wy * 8 + i];
   const long chunk_end = (long)(k + 1) * L;
   for (long q0 = s0; q0 < chunk_end && q0 < T; q0 += kT) {
-    if (tid < kT) mu_s[tid] = fmaxf(m_in, g.amax[(long)bh * tpad + q0 + tid]);
-    float S[4][4] = {};  // [s][t] = k^_s . q_t
-    for (int d0 = 0; d0 < DK; d0 += kS) {
-      for (int e = tid; e < kT * kS; e += kThr) {
-        const int r = e / kS, c = e % kS;
-        As[r][c] = p.key_scale * ld(K, ((long)bh * T + s0 + r) * DK + d0 + c,
-                                    s0 + r < T && d0 + c < DK);
-      }
-      for (int e = tid; e < kS * kT; e += kThr) {
-        const int c = e / kT, j = e % kT;
-        Bs[c][j] = ld(Q, ((long)bh * T + q0 + j) * DK + d0 + c, q0 + j < T && d0 + c < DK);
-      }
+    if (tid < kT) sm.mu[tid] = fmaxf(m_in, g.amax[(long)bh * tpad + q0 + tid]);
+    float S[4][4] = {};  // [key s][query t] = k^_s . q_t
+    for (int dd = 0; dd < DK; dd += kS) {
+      load_cmajor<TIn, kTP>(sm.At, K + base * DK, s0, kT, T, DK, dd, DK, p.key_scale);
+      load_cmajor<TIn, kW>(sm.Bw, Q + base * DK, q0, kT, T, DK, dd, DK, 1.f);
       __syncthreads();
-      mac_slab(S, As, Bs, ty, tx);
+      mac_square<kW>(S, sm.At, sm.Bw, ty, tx);
       __syncthreads();
     }
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const int s = ty * 4 + i, r = tx * 4 + j;
-        const bool ok = q0 + r >= s0 + s && q0 + r < T;
-        Ps[s][r] = ok ? expf(acol_s[s] - mu_s[r]) * S[i][j] : 0.f;
+        const int sr = ty * 4 + i, tq = tx * 4 + j;
+        const bool ok = q0 + tq >= s0 + sr && q0 + tq < T;
+        sm.Pt[tq][sr] = ok ? expf(sm.acol[sr] - sm.mu[tq]) * S[i][j] : 0.f;
       }
-    for (int e = tid; e < kT * kT; e += kThr) {
-      const int r = e / kT, j = e % kT;
-      const long t = q0 + r;
-      Bs[r][j] = (t < T && dv0 + j < DV) ? dU[((long)bh * T + t) * DV + dv0 + j] : 0.f;
+    for (int half = 0; half < 2; ++half) {
+      load_rmajor<float, kW>(sm.Bw, dU + base * DV, q0 + half * kS, T, DV, c0w, DV, 1.f);
+      __syncthreads();
+      mac_wide<kW>(acc, sm.Pt + half * kS, sm.Bw, wy, wx);
+      __syncthreads();
     }
-    __syncthreads();
-    mac_tile(acc, Ps, Bs, ty, tx);
-    __syncthreads();
   }
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const long s = s0 + ty * 4 + i;
+  for (int i = 0; i < 8; ++i) {
+    const long sr = s0 + wy * 8 + i;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int c = dv0 + tx * 4 + j;
-      if (s < T && c < DV) dV[((long)bh * T + s) * DV + c] = from_float<TIn>(acc[i][j]);
+    for (int j = 0; j < kC; ++j) {
+      const int c = c0w + wide_col<kW>(wx, j);
+      if (sr < T && c < DV) dV[(base + sr) * DV + c] = from_float<TIn>(acc[i][j]);
     }
   }
 }
@@ -574,6 +627,17 @@ bwd_gates_kernel(Problem p, const float* __restrict__ i_pre, const float* __rest
     }
     if (tid == 0) dm0[bh] = seg[0];
   }
+}
+
+// Picks the column range of the wide gradient kernels for an output of D
+// columns and calls fn(std::integral_constant<int, W>, grid, shared bytes).
+template <typename TIn, typename Fn>
+cudaError_t launch_wide(const Problem& p, int D, Fn&& fn) {
+  const dim3 g64((D + 63) / 64, (p.T + kT - 1) / kT, p.BH);
+  const dim3 g128((D + 127) / 128, g64.y, p.BH), g256((D + 255) / 256, g64.y, p.BH);
+  if (D > 128) return fn(std::integral_constant<int, 256>{}, g256, sizeof(WideSmem<256>));
+  if (D > 64) return fn(std::integral_constant<int, 128>{}, g128, sizeof(WideSmem<128>));
+  return fn(std::integral_constant<int, 64>{}, g64, sizeof(WideSmem<64>));
 }
 
 // Workspace carve (all fp32): see bwd_workspace_bytes.
@@ -680,12 +744,39 @@ cudaError_t launch_bwd_t(const Problem& p, mlstm_dtype dt, const void* Q, const 
   if (e != cudaSuccess) return e;
   e = cudaMemsetAsync(w.kdk, 0, sizeof(float) * toks, st);
   if (e != cudaSuccess) return e;
-  bwd_dq_kernel<TIn><<<dim3(nk, nt, p.BH), kThr, 0, st>>>(
-      p, q, k, v, w.g, w.C_states, w.n_states, w.dU, w.dA, static_cast<TIn*>(dQ), w.qdq);
-  bwd_dk_kernel<TIn><<<dim3(nk, nt, p.BH), kThr, 0, st>>>(
-      p, q, k, v, w.g, w.G_states, w.g_states, w.dU, w.dA, static_cast<TIn*>(dK), w.kdk);
-  bwd_dv_kernel<TIn><<<dim3(nv, nt, p.BH), kThr, 0, st>>>(p, q, k, w.g, w.G_states, w.dU,
-                                                          static_cast<TIn*>(dV));
+  e = launch_wide<TIn>(p, p.DK, [&](auto wtag, dim3 grid, size_t smem) {
+    constexpr int W = decltype(wtag)::value;
+    const cudaError_t ea = cudaFuncSetAttribute(bwd_dq_kernel<TIn, W>,
+                                                cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                (int)smem);
+    if (ea != cudaSuccess) return ea;
+    bwd_dq_kernel<TIn, W><<<grid, kThr, smem, st>>>(p, q, k, v, w.g, w.C_states, w.n_states,
+                                                    w.dU, w.dA, static_cast<TIn*>(dQ), w.qdq);
+    return cudaGetLastError();
+  });
+  if (e != cudaSuccess) return e;
+  e = launch_wide<TIn>(p, p.DK, [&](auto wtag, dim3 grid, size_t smem) {
+    constexpr int W = decltype(wtag)::value;
+    const cudaError_t ea = cudaFuncSetAttribute(bwd_dk_kernel<TIn, W>,
+                                                cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                (int)smem);
+    if (ea != cudaSuccess) return ea;
+    bwd_dk_kernel<TIn, W><<<grid, kThr, smem, st>>>(p, q, k, v, w.g, w.G_states, w.g_states,
+                                                    w.dU, w.dA, static_cast<TIn*>(dK), w.kdk);
+    return cudaGetLastError();
+  });
+  if (e != cudaSuccess) return e;
+  e = launch_wide<TIn>(p, p.DV, [&](auto wtag, dim3 grid, size_t smem) {
+    constexpr int W = decltype(wtag)::value;
+    const cudaError_t ea = cudaFuncSetAttribute(bwd_dv_kernel<TIn, W>,
+                                                cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                (int)smem);
+    if (ea != cudaSuccess) return ea;
+    bwd_dv_kernel<TIn, W><<<grid, kThr, smem, st>>>(p, q, k, w.g, w.G_states, w.dU,
+                                                    static_cast<TIn*>(dV));
+    return cudaGetLastError();
+  });
+  if (e != cudaSuccess) return e;
   bwd_gates_kernel<<<p.BH, kThr, 0, st>>>(p, i_pre, f_pre, w.qdq, w.kdk, di, df, C0, n0, w.dC0,
                                           w.dn0, dm0);
   e = cudaGetLastError();
