@@ -170,7 +170,7 @@ mlstm_status mlstm_bw_workspace_size(int B, int NH, int T, int DK, int DV, int c
  *   (nullable; zero-state calls get the gradient a zero initial state would
  *   have).  The loss is on H only (no gradient arrives through C_T/n_T/m_T).
  * Errors as mlstm_fw; the workspace must hold mlstm_bw_workspace_size bytes.
- * 10 to 12 launches, asynchronous on `stream`. */
+ * 10 to 13 launches, asynchronous on `stream`. */
 mlstm_status mlstm_bw(const void* Q, const void* K, const void* V, const float* i_pre,
                       const float* f_pre, const float* C0, const float* n0, const float* m0,
                       const void* dH, void* dQ, void* dK, void* dV, float* di_pre, float* df_pre,
@@ -235,7 +235,7 @@ typedef enum {
   MLSTM_KERNEL_TC_PARALLEL = 4,   /* tensor-core intra-chunk TFLA kernel       */
   MLSTM_KERNEL_TC_FUSED = 5,      /* tensor-core fused kernel                  */
   MLSTM_KERNEL_STEP = 6,          /* single-token step (2 launches per call)   */
-  MLSTM_KERNEL_BW = 7,            /* backward pass (10 to 12 launches per call) */
+  MLSTM_KERNEL_BW = 7,            /* backward pass (10 to 13 launches per call) */
   MLSTM_KERNEL_COUNT = 8
 } mlstm_kernel_id;
 

@@ -130,20 +130,26 @@ bwd_prep_kernel(Problem p, const TIn* __restrict__ dH, const TH* __restrict__ Hf
 
 // ---------------------------------------------------------------------------
 // Reverse recurrence: G~_k [BH, NC+1, DK, DV], g~_k [BH, NC+1, DK].  One block
-// per (b, h, 64 x 64 tile of [DK, DV]); blocks with blockIdx.x == 0 carry g~.
+// per (b, h, 64 x 64 tile of [DK, DV], segment); blocks with blockIdx.x == 0
+// carry g~.  With n_seg > 1 the chunks are cut into segments (as the forward
+// state kernel does) that each run from a zero state at their end;
+// bwd_states_fixup_kernel then adds the state carried in from the segments
+// after them: G~_k += e^{sum_{j in [k, k1)} (g_j + m_j - m_{j+1})} G~_{k1}.
 // ---------------------------------------------------------------------------
 template <typename TIn>
 __global__ void __launch_bounds__(kThr)
 bwd_states_kernel(Problem p, const TIn* __restrict__ Q, const float* __restrict__ dU,
                   const float* __restrict__ dA, Gates g, float* __restrict__ G_states,
-                  float* __restrict__ g_states, float* __restrict__ dC0,
-                  float* __restrict__ dn0) {
+                  float* __restrict__ g_states, int n_seg) {
   __shared__ float Qs[kT][kT + 1];
   __shared__ float Us[kT][kT + 1];
   __shared__ float das[kT];
   const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
-  const int dv0 = blockIdx.x * kT, dk0 = blockIdx.y * kT, bh = blockIdx.z;
+  const int dv0 = blockIdx.x * kT, dk0 = blockIdx.y * kT;
+  const int bh = blockIdx.z / n_seg, seg = blockIdx.z % n_seg;
   const int DK = p.DK, DV = p.DV, T = p.T, L = p.L, NC = p.NC;
+  const int ncs = (NC + n_seg - 1) / n_seg;
+  const int k0 = seg * ncs, k1 = k0 + ncs < NC ? k0 + ncs : NC;
   const bool g_owner = blockIdx.x == 0 && tid < kT && dk0 + tid < DK;
   const long tpad = (long)NC * L;
   float acc[4][4] = {};
@@ -159,8 +165,8 @@ bwd_states_kernel(Problem p, const TIn* __restrict__ Q, const float* __restrict_
       }
     if (g_owner) g_states[((long)bh * (NC + 1) + k) * DK + dk0 + tid] = gacc;
   };
-  store(NC);
-  for (int k = NC - 1; k >= 0; --k) {
+  if (seg == n_seg - 1) store(NC);  // G~_NC = 0; other segment ends belong to the next segment
+  for (int k = k1 - 1; k >= k0; --k) {
     const float m_in = g.mchk[(long)bh * (NC + 1) + k];
     const float m_out = g.mchk[(long)bh * (NC + 1) + k + 1];
     const float decay = expf(g.gtot[(long)bh * NC + k] + m_in - m_out);
@@ -201,16 +207,39 @@ bwd_states_kernel(Problem p, const TIn* __restrict__ Q, const float* __restrict_
     }
     store(k);
   }
-  if (dC0) {
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int a = dk0 + ty * 4 + i, c = dv0 + tx * 4 + j;
-        if (a < DK && c < DV) dC0[((long)bh * DK + a) * DV + c] = acc[i][j];
-      }
+}
+
+// Adds the carried-in state to the segments before the last one.  One thread
+// per element of [DK, DV] (then of g~'s DK) and (b, h); walks the segments
+// from the end, so each segment's end value is final when it is used.
+__global__ void __launch_bounds__(kThr)
+bwd_states_fixup_kernel(Problem p, Gates g, float* __restrict__ G_states,
+                        float* __restrict__ g_states, int n_seg) {
+  const long per = (long)p.DK * p.DV;
+  const long e = (long)blockIdx.x * kThr + threadIdx.x;
+  const int bh = blockIdx.y, NC = p.NC;
+  if (e >= per + p.DK) return;
+  float* base;
+  long stride;
+  if (e < per) {
+    base = G_states + (long)bh * (NC + 1) * per + e;
+    stride = per;
+  } else {
+    base = g_states + (long)bh * (NC + 1) * p.DK + (e - per);
+    stride = p.DK;
   }
-  if (dn0 && g_owner) dn0[(long)bh * DK + dk0 + tid] = gacc;
+  const float* gt = g.gtot + (long)bh * NC;
+  const float* mc = g.mchk + (long)bh * (NC + 1);
+  const int ncs = (NC + n_seg - 1) / n_seg;
+  for (int s = n_seg - 2; s >= 0; --s) {
+    const int k0 = s * ncs, k1 = k0 + ncs < NC ? k0 + ncs : NC;
+    const float carried = base[(long)k1 * stride];  // final: its segment was fixed before
+    float lg = 0.f;
+    for (int k = k1 - 1; k >= k0; --k) {
+      lg += gt[k] + mc[k] - mc[k + 1];
+      base[(long)k * stride] = fmaf(expf(lg), carried, base[(long)k * stride]);
+    }
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -629,6 +658,18 @@ bwd_gates_kernel(Problem p, const float* __restrict__ i_pre, const float* __rest
   }
 }
 
+// Segments of the reverse recurrence: enough (b, h, tile, segment) blocks
+// for about four per SM of a 148-SM B200, at most 8 segments, each at least
+// two chunks and none empty.
+int bwd_segments(const Problem& p) {
+  const int units = p.BH * ((p.DK + kT - 1) / kT) * ((p.DV + kT - 1) / kT);
+  int s = 4 * 148 / units;
+  if (s > 8) s = 8;
+  if (s > p.NC / 2) s = p.NC / 2;
+  while (s > 1 && (s - 1) * ((p.NC + s - 1) / s) >= p.NC) --s;
+  return s < 1 ? 1 : s;
+}
+
 // Picks the column range of the wide gradient kernels for an output of D
 // columns and calls fn(std::integral_constant<int, W>, grid, shared bytes).
 template <typename TIn, typename Fn>
@@ -738,8 +779,22 @@ cudaError_t launch_bwd_t(const Problem& p, mlstm_dtype dt, const void* Q, const 
     bwd_prep_kernel<TIn, float><<<prep_blocks, kThr, 0, st>>>(
         p, static_cast<const TIn*>(dH), w.H32, w.den, w.mr, w.dU, w.dA);
   const int nk = (p.DK + kT - 1) / kT, nv = (p.DV + kT - 1) / kT, nt = (p.T + kT - 1) / kT;
-  bwd_states_kernel<TIn><<<dim3(nv, nk, p.BH), kThr, 0, st>>>(p, q, w.dU, w.dA, w.g, w.G_states,
-                                                              w.g_states, w.dC0, w.dn0);
+  const int n_seg = bwd_segments(p);
+  bwd_states_kernel<TIn><<<dim3(nv, nk, p.BH * n_seg), kThr, 0, st>>>(p, q, w.dU, w.dA, w.g,
+                                                                     w.G_states, w.g_states, n_seg);
+  if (n_seg > 1) {
+    const long n_el = (long)p.DK * p.DV + p.DK;
+    bwd_states_fixup_kernel<<<dim3((unsigned)((n_el + kThr - 1) / kThr), p.BH), kThr, 0, st>>>(
+        p, w.g, w.G_states, w.g_states, n_seg);
+  }
+  // dC0 = G~_0, dn0 = g~_0 (index 0 of every head's states)
+  e = cudaMemcpy2DAsync(w.dC0, sizeof(float) * p.DK * p.DV, w.G_states,
+                        sizeof(float) * (p.NC + 1) * p.DK * p.DV, sizeof(float) * p.DK * p.DV,
+                        p.BH, cudaMemcpyDeviceToDevice, st);
+  if (e != cudaSuccess) return e;
+  e = cudaMemcpy2DAsync(w.dn0, sizeof(float) * p.DK, w.g_states, sizeof(float) * (p.NC + 1) * p.DK,
+                        sizeof(float) * p.DK, p.BH, cudaMemcpyDeviceToDevice, st);
+  if (e != cudaSuccess) return e;
   e = cudaMemsetAsync(w.qdq, 0, sizeof(float) * toks, st);
   if (e != cudaSuccess) return e;
   e = cudaMemsetAsync(w.kdk, 0, sizeof(float) * toks, st);
@@ -797,8 +852,9 @@ size_t bwd_workspace_bytes(const Problem& p, mlstm_dtype dt) { return carve(p, d
 
 int bwd_launches(const Problem& p, mlstm_dtype dt) {
   // gates (2) + recompute (simt: 2; tensor cores: states [+ fix-up] + operand copy + outputs)
-  // + prep, reverse states, dq, dk, dv, gate gradients (6)
-  return 2 + (tc_recompute(p, dt) ? 2 + tc_states_launches(p) : 2) + 6;
+  // + prep, reverse states [+ fix-up], dq, dk, dv, gate gradients (6 or 7)
+  return 2 + (tc_recompute(p, dt) ? 2 + tc_states_launches(p) : 2) + 6 +
+         (bwd_segments(p) > 1 ? 1 : 0);
 }
 
 cudaError_t launch_backward(const Problem& p, mlstm_dtype dt, const void* Q, const void* K,
