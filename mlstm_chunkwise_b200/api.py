@@ -258,3 +258,40 @@ def watchdog_selftest(device=None) -> None:
     ``_lib.ERR_TIMEOUT``."""
     dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
     _lib.check(_lib.lib().mlstm_watchdog_selftest(_stream(dev)), "mlstm_watchdog_selftest")
+
+
+class _MlstmChunkwise(torch.autograd.Function):
+    """Differentiable mLSTM: the forward is ``mlstm_fw``, the backward
+    ``mlstm_bw`` (which recomputes what it needs from the inputs).  Gradients
+    flow from H only; the returned final state carries none."""
+
+    @staticmethod
+    def forward(ctx, Q, K, V, i_pre, f_pre, C0, n0, m0, chunk_size, gate_mode, algo):
+        H, (C_T, n_T, m_T) = mlstm_fw(Q, K, V, i_pre, f_pre, C0, n0, m0, chunk_size=chunk_size,
+                                      gate_mode=gate_mode, algo=algo)
+        ctx.save_for_backward(Q, K, V, i_pre, f_pre, C0, n0, m0)
+        ctx.cfg = (chunk_size, gate_mode)
+        ctx.mark_non_differentiable(C_T, n_T, m_T)
+        return H, C_T, n_T, m_T
+
+    @staticmethod
+    def backward(ctx, dH, dC_T, dn_T, dm_T):
+        Q, K, V, i_pre, f_pre, C0, n0, m0 = ctx.saved_tensors
+        chunk_size, gate_mode = ctx.cfg
+        g = mlstm_bw(Q, K, V, i_pre, f_pre, dH.contiguous(), C0, n0, m0, chunk_size=chunk_size,
+                     gate_mode=gate_mode)
+        return (g["dQ"], g["dK"], g["dV"], g["di_pre"], g["df_pre"], g.get("dC0"), g.get("dn0"),
+                g.get("dm0"), None, None, None)
+
+
+def mlstm_chunkwise(Q, K, V, i_pre, f_pre, C0=None, n0=None, m0=None, *, chunk_size: int = 64,
+                    gate_mode: str = "exp", algo: str = "auto"):
+    """mLSTM forward pass that autograd can differentiate (through ``mlstm_bw``).
+
+    Same arguments and shapes as ``mlstm_fw``; returns ``(H, (C_T, n_T, m_T))``.
+    The gradient of a loss on H reaches Q, K, V, both gate pre-activations and
+    the initial state; the final state is returned without a gradient path.
+    """
+    H, C_T, n_T, m_T = _MlstmChunkwise.apply(Q, K, V, i_pre, f_pre, C0, n0, m0, chunk_size,
+                                             gate_mode, algo)
+    return H, (C_T, n_T, m_T)

@@ -75,3 +75,23 @@ def test_backward_chunk_size_invariance():
         for k in ("dQ", "dK", "dV", "di_pre", "df_pre", "dC0"):
             assert parity.worst_rel(o[k].double().cpu().numpy(),
                                     outs[0][k].double().cpu().numpy()) < 1e-4, k
+
+
+def test_autograd_function_matches_the_oracle():
+    """mlstm_chunkwise under torch.autograd: loss.backward() fills the inputs'
+    .grad with the oracle's gradients (bf16 inputs, initial state)."""
+    w = WORKLOADS["mid"].replace(name="ag", B=1, NH=2, T=384, chunk_size=128, init_state=True)
+    x = make_inputs(w, seed=21)
+    g = torch.Generator().manual_seed(22)
+    dH = torch.randn((w.B, w.NH, w.T, w.DV), generator=g).to(w.torch_dtype)
+    ref = ob.gradients(x, dH, w.gate_mode)
+    leaves = {k: v.cuda().requires_grad_(True) for k, v in x.items() if v is not None}
+    H, _ = api.mlstm_chunkwise(leaves["Q"], leaves["K"], leaves["V"], leaves["i_pre"],
+                               leaves["f_pre"], leaves["C0"], leaves["n0"], leaves["m0"],
+                               chunk_size=w.chunk_size)
+    (H.float() * dH.cuda().float()).sum().backward()
+    torch.cuda.synchronize()
+    assert api.last_device_error() == _lib.OK
+    for name in ("Q", "K", "V", "i_pre", "f_pre", "C0", "n0"):
+        err = parity.worst_rel(leaves[name].grad.double().cpu().numpy(), ref["d" + name].numpy())
+        assert err < TOL[w.dtype], (name, err)
