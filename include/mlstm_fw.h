@@ -190,8 +190,10 @@ mlstm_status mlstm_bw(const void* Q, const void* K, const void* V, const float* 
  *   token on entry, after it on return (a zero state is C = n = 0, m = 0).
  *   m' = max(logsigmoid(f~) + m, li), C' = fa C + ia (s k) v^T,
  *   n' = fa n + ia s k, h = C'^T q / max(|n'^T q|, e^{-m'}), s = 1/sqrt(DK).
- * Sizes: B, NH >= 1, DK, DV in [1, 1024].  No workspace; two launches on
- * `stream`, asynchronous.  All pointers 16-byte aligned and non-null, else
+ * Sizes: B, NH >= 1, DK, DV in [1, 1024].  No workspace; asynchronous on
+ * `stream`: one launch (a thread-block cluster per head), or two when d_v is
+ * not a multiple of 4 and above 256 (a head then spans more column tiles
+ * than one cluster holds).  All pointers 16-byte aligned and non-null, else
  * MLSTM_ERR_INVALID_ARG before any launch. */
 mlstm_status mlstm_step(const void* q, const void* k, const void* v, const float* i_pre,
                         const float* f_pre, float* C, float* n, float* m, void* h, int B, int NH,
@@ -234,7 +236,7 @@ typedef enum {
   MLSTM_KERNEL_TC_STATES = 3,     /* tensor-core chunk-state recurrence        */
   MLSTM_KERNEL_TC_PARALLEL = 4,   /* tensor-core intra-chunk TFLA kernel       */
   MLSTM_KERNEL_TC_FUSED = 5,      /* tensor-core fused kernel                  */
-  MLSTM_KERNEL_STEP = 6,          /* single-token step (2 launches per call)   */
+  MLSTM_KERNEL_STEP = 6,          /* single-token step (1 or 2 launches)       */
   MLSTM_KERNEL_BW = 7,            /* backward pass (10 to 13 launches per call) */
   MLSTM_KERNEL_COUNT = 8
 } mlstm_kernel_id;

@@ -519,7 +519,7 @@ mlstm_status mlstm_step(const void* q, const void* k, const void* v, const float
     if (!ptr || !aligned16(ptr)) return MLSTM_ERR_INVALID_ARG;
   Problem p = make_problem(B, NH, 1, DK, DV, 64, gate_mode);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  return from_cuda(launch_family(MLSTM_KERNEL_STEP, 2, st, [&] {
+  return from_cuda(launch_family(MLSTM_KERNEL_STEP, step_launches(p), st, [&] {
     return launch_step(p, dtype, q, k, v, i_pre, f_pre, C, n, m, h, st);
   }));
 }

@@ -85,6 +85,7 @@ cudaError_t launch_backward(const Problem& p, mlstm_dtype dt, const void* Q, con
                             const float* C0, const float* n0, const float* m0, const void* dH,
                             void* dQ, void* dK, void* dV, float* di, float* df, float* dC0,
                             float* dn0, float* dm0, void* ws, cudaStream_t st);
+int step_launches(const Problem& p);
 cudaError_t launch_step(const Problem& p, mlstm_dtype dt, const void* q, const void* k,
                         const void* v, const float* i_pre, const float* f_pre, float* C,
                         float* n, float* m, void* h, cudaStream_t st);

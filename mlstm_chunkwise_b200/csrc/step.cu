@@ -18,9 +18,12 @@
 // rows with eight rows in flight per thread, and h of the tile comes out of
 // the same pass (a shared-memory reduction over the warps).
 // The denominator only needs n'.q = fa (n.q) + ia (s k.q), which every block
-// forms from the old n, so no block depends on another; step_norm_kernel then
-// writes n' and m' in place (stream order puts it after every read of the old
-// values).
+// forms from the old n.  The blocks of one (b, h) are launched as one thread-
+// block cluster (at most 8 column tiles): once every block of the cluster has
+// read the old n and m, a cluster barrier lets block 0 write n' and m' in
+// place.  Where the tiles of a head do not fit one cluster, step_norm_kernel
+// writes them in a second launch instead (stream order puts it after every
+// read of the old values).
 #include "common.cuh"
 
 namespace mlstm {
@@ -65,8 +68,8 @@ template <typename T, int kVec>
 __global__ void __launch_bounds__(kStepWarps * 32)
 step_state_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                   const float* __restrict__ i_pre, const float* __restrict__ f_pre,
-                  float* __restrict__ C, const float* __restrict__ n, const float* __restrict__ m,
-                  T* __restrict__ h, int DK, int DV, int sig, float key_scale) {
+                  float* __restrict__ C, float* __restrict__ n, float* __restrict__ m,
+                  T* __restrict__ h, int DK, int DV, int sig, float key_scale, int cluster_nm) {
   constexpr int kCols = 32 * kVec;       // value columns per block
   extern __shared__ float sh[];
   float* sk = sh;                        // s k   [DK]
@@ -93,6 +96,16 @@ step_state_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __r
     dots[2 * ty + 1] = kq;
   }
   __syncthreads();
+  if (cluster_nm) {
+    // every block of this head's cluster has read the old n and m
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                     : "memory");
+    if (blockIdx.x == 0) {
+      for (int i = threadIdx.x; i < DK; i += blockDim.x)
+        n[(long)bh * DK + i] = fmaf(gt.fa, n[(long)bh * DK + i], gt.ia * sk[i]);
+      if (threadIdx.x == 0) m[bh] = gt.m_new;
+    }
+  }
 
   // columns col .. col + kVec - 1 (kVec == 4 needs DV % 4 == 0, so all or none are valid)
   const int col = blockIdx.x * kCols + tx * kVec;
@@ -178,15 +191,39 @@ size_t step_smem_bytes(int DK, int cols) {
   return (2 * (size_t)DK + kStepWarps * (size_t)cols + 2 * kStepWarps) * sizeof(float);
 }
 
+constexpr int kMaxCluster = 8;  // portable cluster size
+
+// Launches the state kernel; with one cluster per head (the tiles of a head
+// fit one cluster) it also writes n' and m' and returns true.
 template <typename T, int kVec>
-void launch_state(const Problem& p, const void* q, const void* k, const void* v,
-                  const float* i_pre, const float* f_pre, float* C, const float* n,
-                  const float* m, void* h, cudaStream_t st) {
+cudaError_t launch_state(const Problem& p, const void* q, const void* k, const void* v,
+                         const float* i_pre, const float* f_pre, float* C, float* n, float* m,
+                         void* h, cudaStream_t st, bool* nm_done) {
   constexpr int kCols = 32 * kVec;
-  const dim3 grid((p.DV + kCols - 1) / kCols, p.BH);
-  step_state_kernel<T, kVec><<<grid, kStepWarps * 32, step_smem_bytes(p.DK, kCols), st>>>(
-      static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), i_pre, f_pre,
-      C, n, m, static_cast<T*>(h), p.DK, p.DV, p.gate_sigmoid, p.key_scale);
+  const int gx = (p.DV + kCols - 1) / kCols;
+  const int cluster = gx <= kMaxCluster ? 1 : 0;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(gx, p.BH);
+  cfg.blockDim = dim3(kStepWarps * 32);
+  cfg.dynamicSmemBytes = step_smem_bytes(p.DK, kCols);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = cluster ? gx : 1;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  *nm_done = cluster != 0;
+  return cudaLaunchKernelEx(&cfg, step_state_kernel<T, kVec>, static_cast<const T*>(q),
+                            static_cast<const T*>(k), static_cast<const T*>(v), i_pre, f_pre, C, n,
+                            m, static_cast<T*>(h), p.DK, p.DV, p.gate_sigmoid, p.key_scale,
+                            cluster);
+}
+
+int step_launches(const Problem& p) {
+  const int cols = p.DV % 4 == 0 ? 128 : 32;
+  return (p.DV + cols - 1) / cols <= kMaxCluster ? 1 : 2;
 }
 
 cudaError_t launch_step(const Problem& p, mlstm_dtype dt, const void* q, const void* k,
@@ -195,15 +232,15 @@ cudaError_t launch_step(const Problem& p, mlstm_dtype dt, const void* q, const v
   if (step_smem_bytes(p.DK, 128) > 48 * 1024) return cudaErrorNotSupported;
   // 16-byte state accesses when every row starts on a 16-byte boundary
   const bool vec = p.DV % 4 == 0;
-  if (dt == MLSTM_DT_BF16) {
-    if (vec) launch_state<__nv_bfloat16, 4>(p, q, k, v, i_pre, f_pre, C, n, m, h, st);
-    else launch_state<__nv_bfloat16, 1>(p, q, k, v, i_pre, f_pre, C, n, m, h, st);
-  } else {
-    if (vec) launch_state<float, 4>(p, q, k, v, i_pre, f_pre, C, n, m, h, st);
-    else launch_state<float, 1>(p, q, k, v, i_pre, f_pre, C, n, m, h, st);
-  }
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+  bool nm_done = false;
+  cudaError_t e;
+  if (dt == MLSTM_DT_BF16)
+    e = vec ? launch_state<__nv_bfloat16, 4>(p, q, k, v, i_pre, f_pre, C, n, m, h, st, &nm_done)
+            : launch_state<__nv_bfloat16, 1>(p, q, k, v, i_pre, f_pre, C, n, m, h, st, &nm_done);
+  else
+    e = vec ? launch_state<float, 4>(p, q, k, v, i_pre, f_pre, C, n, m, h, st, &nm_done)
+            : launch_state<float, 1>(p, q, k, v, i_pre, f_pre, C, n, m, h, st, &nm_done);
+  if (e != cudaSuccess || nm_done) return e;
   step_norm_kernel<<<p.BH, 256, 0, st>>>(k, dt == MLSTM_DT_BF16, i_pre, f_pre, n, m, p.DK,
                                          p.gate_sigmoid, p.key_scale);
   return cudaGetLastError();

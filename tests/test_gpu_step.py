@@ -16,7 +16,8 @@ from mlstm_chunkwise_b200.inputs import WORKLOADS, make_inputs
 
 pytestmark = pytest.mark.gpu
 
-SHAPES = [(2, 3, 64, 64), (1, 4, 128, 128), (2, 2, 256, 512), (1, 2, 100, 72), (1, 1, 1, 1)]
+SHAPES = [(2, 3, 64, 64), (1, 4, 128, 128), (2, 2, 256, 512), (1, 2, 100, 72), (1, 1, 1, 1),
+          (1, 2, 64, 1024), (1, 2, 32, 262)]  # d_v 1024: 8 tiles per cluster; 262: two launches
 
 
 def _state(B, NH, DK, DV, seed):
