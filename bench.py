@@ -120,13 +120,13 @@ def kernel_bytes(fam, B, NH, T, DK, DV, L, elem):
 # the entry records a SHA-1 over those files and is ignored when it differs.
 MEASURED_TRAFFIC = {
     ("tc_parallel", "xlstm7b"): {
-        "bytes": 2.128e9, "profile": "profiles/tc_unfused_xlstm7b.md",
+        "bytes": 2.127e9, "profile": "profiles/tc_unfused_xlstm7b.md",
         "sources": ["tc_parallel_wide.cu", "tc_ptx.cuh", "tc.h", "common.cuh"],
-        "sha1": "2cf1359c5e387e0a5008c3e01626af1c9a1ca7fb"},
+        "sha1": "75dbcbcf74df5f0115693d98aa5a7105832df9fd"},
     ("tc_states", "xlstm7b"): {
-        "bytes": 1.327e9, "profile": "profiles/tc_unfused_xlstm7b.md",
+        "bytes": 1.326e9, "profile": "profiles/tc_unfused_xlstm7b.md",
         "sources": ["tc_states.cu", "tc_ptx.cuh", "tc.h", "common.cuh"],
-        "sha1": "df123dfd099a8fed8c8d17fdbaf9802284e7d3ef"},
+        "sha1": "64f549befc01d79047227790c36aa26b5ebd9b82"},
 }
 
 
