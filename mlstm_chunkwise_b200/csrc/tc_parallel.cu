@@ -431,10 +431,10 @@ tc_parallel_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       mbar_arrive(bar.q_empty());
       float den = f_inter * dn;
 
-      // Gated P tiles, written back over their S tiles in TMEM.  P_0 is
-      // released only after this half of the inter-chunk term (Q.C, issued
-      // after S_0) has been rescaled to the row frame mu_r, since P_0.V_0
-      // accumulates on top of it.
+      // Gated P tiles into the two TMEM P buffers (tile i into buffer i mod
+      // 2).  P_0 is released only after this half of the inter-chunk term
+      // (Q.C, issued after S_0) has been rescaled to the row frame mu_r, since
+      // P_0.V_0 accumulates on top of it.
       for (int i = 0; i < x.n_kv; ++i, ++tile) {
         const int buf = tile & 1;
         ok = ok && mbar_wait(bar.s_full(), tile & 1, p, 10);
