@@ -16,8 +16,11 @@ from mlstm_chunkwise_b200.inputs import WORKLOADS, make_inputs
 
 pytestmark = pytest.mark.gpu
 
+# d_v 1024: 8 tiles per cluster; 262: two launches; 97 x 33 two 32-column
+# tiles (4-byte accesses), the last one ragged; 300 and 200 rows are not a
+# multiple of the eight rows a batch keeps in flight per warp.
 SHAPES = [(2, 3, 64, 64), (1, 4, 128, 128), (2, 2, 256, 512), (1, 2, 100, 72), (1, 1, 1, 1),
-          (1, 2, 64, 1024), (1, 2, 32, 262)]  # d_v 1024: 8 tiles per cluster; 262: two launches
+          (1, 2, 64, 1024), (1, 2, 32, 262), (1, 2, 300, 96), (1, 1, 200, 40), (3, 1, 97, 33)]
 
 
 def _state(B, NH, DK, DV, seed):
