@@ -701,7 +701,8 @@ def run_step(args):
 
 
 # ----------------------------------------------------------------------------
-# backward pass (fp32 CUDA-core kernels) at a workload's shape
+# backward pass at a workload's shape (bf16 with d_qk 128 or 256: tensor-core
+# kernels on 128-token chunks; otherwise the fp32 CUDA-core kernels)
 # ----------------------------------------------------------------------------
 BW_METRIC = "mLSTM backward tokens/s (gradients of a loss on H, forward recomputed)"
 
@@ -767,20 +768,29 @@ def run_bw(args):
         raise SystemExit(f"device error in the timed region: {_lib.status_string(st)}")
     ms = e0.elapsed_time(e1) / args.steps
     peaks, peak_src = load_peaks()
-    fph = flops_per_head(T, DK, DV, L)
+    # the tensor-core backward runs on 128-token chunks whatever chunk_size is
+    tc_bw = (w.dtype == "bf16" and DK in (128, 256) and (DV == 128 or DV % 256 == 0) and DV <= 1024
+             and T >= 128)
+    Lb = 128 if tc_bw else L
+    fph = flops_per_head(T, DK, DV, Lb)
     fw_flops = B * NH * (fph["states"] + fph["inter"] + fph["intra"])
-    bw_flops = B * NH * bw_flops_per_head(T, DK, DV, L)
-    peak = SIMT_LANES * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
+    bw_flops = B * NH * bw_flops_per_head(T, DK, DV, Lb)
     achieved = (fw_flops + bw_flops) / (ms / 1e3) / 1e12
+    if tc_bw:
+        algo, bound, peak = "bw (tensor cores, 128-token chunks)", "tensor", peaks["bf16_tflops"]
+        peak_source = f"bf16_tflops (of {peak_src})"
+    else:
+        algo, bound = "bw (fp32 CUDA-core kernels)", "alu"
+        peak = SIMT_LANES * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
+        peak_source = f"fp32 FFMA: 148 SMs x 128 lanes x 2 x sm_max_mhz (of {peak_src})"
     line = {
         "metric": BW_METRIC, "value": B * T / (ms / 1e3), "unit": "tokens/s", "n_gpus": 1,
         "steps": args.steps, "warmup": warm, "ms_per_step": ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
-        "config": workload_config(w, "bw (fp32 CUDA-core kernels)"),
+        "config": workload_config(w, algo),
         "tflops": achieved,
-        "roofline": {"kernel": "bw", "bound": "alu", "achieved": achieved, "peak": peak,
-                     "unit": "TFLOP/s", "frac": achieved / peak,
-                     "peak_source": f"fp32 FFMA: 148 SMs x 128 lanes x 2 x sm_max_mhz (of {peak_src})",
+        "roofline": {"kernel": "bw", "bound": bound, "achieved": achieved, "peak": peak,
+                     "unit": "TFLOP/s", "frac": achieved / peak, "peak_source": peak_source,
                      "algorithmic_flops": fw_flops + bw_flops, "traffic": None,
                      "per_launch_ms": ms},
         "gpu_launches": int(launches), "e2e": None,

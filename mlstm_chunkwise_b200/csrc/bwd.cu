@@ -101,23 +101,35 @@ __device__ __forceinline__ void mac_tile(float (&acc)[4][4], const float (*P)[kT
 }
 
 // ---------------------------------------------------------------------------
-// du~ [BH, T, DV] and da~ [BH, T]: one warp per token.
+// du~ [BH, T, DV] (fp32 when dU is set; in bf16 for the tensor-core
+// gradients when dU16 is set, and with rows scaled by e^{m_k - mu_t} when dUr16
+// is set) and da~ [BH, T]: one warp per token.
 // ---------------------------------------------------------------------------
 // den_s holds copysign(max(|a|, e^{-m}), a) of the forward (signed_den mode).
 template <typename TIn, typename TH>
 __global__ void __launch_bounds__(kThr)
 bwd_prep_kernel(Problem p, const TIn* __restrict__ dH, const TH* __restrict__ Hf,
                 const float* __restrict__ den_s, const float* __restrict__ mr,
-                float* __restrict__ dU, float* __restrict__ dA) {
+                float* __restrict__ dU, float* __restrict__ dA,
+                __nv_bfloat16* __restrict__ dU16 = nullptr,
+                __nv_bfloat16* __restrict__ dUr16 = nullptr, Gates gt = {}) {
   const long tok = (long)blockIdx.x * (kThr / 32) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (tok >= (long)p.BH * p.T) return;
   const float ds = den_s[tok];
   const float inv = 1.f / fabsf(ds);
+  float r = 0.f;  // e^{m_k - mu_t}, the row factor of the reverse-state update
+  if (dUr16) {
+    const long bh = tok / p.T, t = tok % p.T;
+    const float m_in = gt.mchk[bh * (p.NC + 1) + t / p.L];
+    r = expf(m_in - fmaxf(m_in, gt.amax[bh * (long)p.NC * p.L + t]));
+  }
   float dot = 0.f;
   for (int c = lane; c < p.DV; c += 32) {
     const float g = to_float(dH[tok * p.DV + c]);
-    dU[tok * p.DV + c] = g * inv;
+    if (dU) dU[tok * p.DV + c] = g * inv;
+    if (dU16) dU16[tok * p.DV + c] = __float2bfloat16_rn(g * inv);
+    if (dUr16) dUr16[tok * p.DV + c] = __float2bfloat16_rn(r * g * inv);
     dot = fmaf(g, to_float(Hf[tok * p.DV + c]), dot);
   }
 #pragma unroll
@@ -687,6 +699,10 @@ struct BwdWs {
   float *C_states, *n_states, *H32, *den, *mr, *dU, *dA, *G_states, *g_states, *qdq, *kdk, *dC0,
       *dn0, *seg;
   __nv_bfloat16 *Cb, *H16;  // tensor-core recompute: operand copy of the states, bf16 h
+  // tensor-core gradients: du~ (plain and row-scaled), reverse states, squares,
+  // per-chunk updates of the reverse states and of g~
+  __nv_bfloat16 *dU16, *dUr16, *Gb, *sq;
+  float *U, *uvec;
 };
 
 // Whether the forward is recomputed on the tensor cores.
@@ -694,12 +710,31 @@ bool tc_recompute(const Problem& p, mlstm_dtype dt) {
   return dt == MLSTM_DT_BF16 && tc_unfused_supported(p);
 }
 
+// The tensor-core gradients work in chunks of 128 tokens (one MMA tile of
+// rows) whatever the caller's chunk size: the gradients do not depend on the
+// chunking (up to rounding), and the whole backward, recomputed forward
+// included, then runs on that chunking.
+Problem tc_bwd_problem(const Problem& p) {
+  Problem pb = p;
+  pb.L = 128;
+  pb.NC = (p.T + 127) / 128;
+  return pb;
+}
+// Sequences shorter than one such chunk stay on the fp32 kernels: they cost
+// nothing there, and with a handful of tokens the terms of the forget-gate
+// gradient (sums of q.dq - k.dk) cancel far below the bf16 operands' rounding.
+bool tc_backward(const Problem& p, mlstm_dtype dt) {
+  return dt == MLSTM_DT_BF16 && p.T >= 128 && tc_bwd_supported(tc_bwd_problem(p));
+}
+
 constexpr size_t kAlign = 256;
 inline size_t al(size_t b) { return (b + kAlign - 1) / kAlign * kAlign; }
 
-size_t carve(const Problem& p, mlstm_dtype dt, char* base, BwdWs* w) {
+size_t carve(const Problem& p_in, mlstm_dtype dt, char* base, BwdWs* w) {
+  const bool tcb = tc_backward(p_in, dt);
+  const Problem p = tcb ? tc_bwd_problem(p_in) : p_in;
   const size_t BH = p.BH, T = p.T, NC = p.NC, tpad = NC * p.L, DK = p.DK, DV = p.DV;
-  const bool tc = tc_recompute(p, dt);
+  const bool tc = tcb || tc_recompute(p, dt);
   size_t off = 0;
   auto take = [&](size_t n) -> float* {
     float* ptr = base ? reinterpret_cast<float*>(base + off) : nullptr;
@@ -717,9 +752,9 @@ size_t carve(const Problem& p, mlstm_dtype dt, char* base, BwdWs* w) {
   g.amax = take(BH * tpad);
   g.gtot = take(BH * NC);
   g.mchk = take(BH * (NC + 1));
-  BwdWs x;
+  BwdWs x = {};
   x.g = g;
-  x.C_states = take(BH * NC * DK * DV);
+  x.C_states = tcb ? nullptr : take(BH * NC * DK * DV);
   x.n_states = take(BH * NC * DK);
   x.H32 = tc ? nullptr : take(BH * T * DV);
   x.Cb = tc ? take16(BH * NC * DK * DV) : nullptr;
@@ -727,16 +762,79 @@ size_t carve(const Problem& p, mlstm_dtype dt, char* base, BwdWs* w) {
   x.seg = tc ? take(tc_states_segment_floats(p)) : nullptr;
   x.den = take(BH * T);
   x.mr = take(BH * T);
-  x.dU = take(BH * T * DV);
+  x.dU = tcb ? nullptr : take(BH * T * DV);
   x.dA = take(BH * T);
-  x.G_states = take(BH * (NC + 1) * DK * DV);
+  x.G_states = tcb ? nullptr : take(BH * (NC + 1) * DK * DV);
   x.g_states = take(BH * (NC + 1) * DK);
   x.qdq = take(BH * T);
   x.kdk = take(BH * T);
   x.dC0 = take(BH * DK * DV);
   x.dn0 = take(BH * DK);
+  if (tcb) {
+    x.dU16 = take16(BH * T * DV);
+    x.dUr16 = take16(BH * T * DV);
+    x.Gb = take16(BH * (NC + 1) * DK * DV);
+    x.sq = take16(tc_bwd_square_elems(p));
+    x.U = take(BH * NC * DK * DV);
+    x.uvec = take(BH * NC * DK);
+  }
   if (w) *w = x;
   return off;
+}
+
+// The backward on the tensor cores (bf16, 128-token chunks): the forward
+// recomputed on the tensor cores (gates, chunk states as the bf16 operand
+// copy, h and the signed denominator), the per-token pass (du~ in bf16, plain
+// and row-scaled), the reverse states (per-chunk updates on the tensor cores,
+// then a reverse scan), the squares and dq, dk, dv (tc_bwd.cu), and the gate
+// gradients.
+cudaError_t launch_bwd_tc(const Problem& p_in, const void* Q, const void* K, const void* V,
+                          const float* i_pre, const float* f_pre, const float* C0,
+                          const float* n0, const float* m0, const void* dH, void* dQ, void* dK,
+                          void* dV, float* di, float* df, float* dC0, float* dn0, float* dm0,
+                          void* ws, cudaStream_t st) {
+  const Problem p = tc_bwd_problem(p_in);
+  BwdWs w;
+  carve(p_in, MLSTM_DT_BF16, static_cast<char*>(ws), &w);
+  cudaError_t e = launch_gates(p, i_pre, f_pre, m0, w.g, st);
+  if (e != cudaSuccess) return e;
+  e = launch_tc_states(p, K, V, C0, n0, w.g, nullptr, w.Cb, w.n_states, nullptr, nullptr, nullptr,
+                       w.seg, st);
+  if (e != cudaSuccess) return e;
+  Problem ps = p;
+  ps.signed_den = 1;  // the forward outputs keep the sign of the denominator
+  e = launch_tc_parallel(ps, Q, K, V, w.g, w.Cb, w.n_states, w.H16, w.den, w.mr, st);
+  if (e != cudaSuccess) return e;
+  const long toks = (long)p.BH * p.T;
+  bwd_prep_kernel<__nv_bfloat16, __nv_bfloat16><<<(unsigned)((toks + 7) / 8), kThr, 0, st>>>(
+      p, static_cast<const __nv_bfloat16*>(dH), w.H16, w.den, w.mr, nullptr, w.dA, w.dU16,
+      w.dUr16, w.g);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  e = launch_tc_bwd_states(p, Q, w.dUr16, w.g, w.dA, w.U, w.uvec, w.Gb, w.g_states, w.dC0, st);
+  if (e != cudaSuccess) return e;
+  e = cudaMemcpy2DAsync(w.dn0, sizeof(float) * p.DK, w.g_states, sizeof(float) * (p.NC + 1) * p.DK,
+                        sizeof(float) * p.DK, p.BH, cudaMemcpyDeviceToDevice, st);
+  if (e != cudaSuccess) return e;
+  e = cudaMemsetAsync(w.qdq, 0, sizeof(float) * toks, st);
+  if (e != cudaSuccess) return e;
+  e = cudaMemsetAsync(w.kdk, 0, sizeof(float) * toks, st);
+  if (e != cudaSuccess) return e;
+  e = launch_tc_bwd(p, Q, K, V, w.dU16, w.g, w.dA, w.n_states, w.g_states, w.Cb, w.Gb, w.sq, dQ,
+                    dK, dV, w.qdq, w.kdk, st);
+  if (e != cudaSuccess) return e;
+  bwd_gates_kernel<<<p.BH, kThr, 0, st>>>(p, i_pre, f_pre, w.qdq, w.kdk, di, df, C0, n0, w.dC0,
+                                          w.dn0, dm0);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  if (dC0) {
+    e = cudaMemcpyAsync(dC0, w.dC0, sizeof(float) * p.BH * p.DK * p.DV,
+                        cudaMemcpyDeviceToDevice, st);
+    if (e != cudaSuccess) return e;
+  }
+  if (dn0)
+    e = cudaMemcpyAsync(dn0, w.dn0, sizeof(float) * p.BH * p.DK, cudaMemcpyDeviceToDevice, st);
+  return e;
 }
 
 template <typename TIn>
@@ -853,6 +951,12 @@ size_t bwd_workspace_bytes(const Problem& p, mlstm_dtype dt) { return carve(p, d
 int bwd_launches(const Problem& p, mlstm_dtype dt) {
   // gates (2) + recompute (simt: 2; tensor cores: states [+ fix-up] + operand copy + outputs)
   // + prep, reverse states [+ fix-up], dq, dk, dv, gate gradients (6 or 7)
+  if (tc_backward(p, dt)) {
+    // gates (2), chunk states [+ fix-up], outputs, prep, reverse states
+    // (updates, g~ increments, scan), squares + dq + dk + dv, gate gradients
+    const Problem pb = tc_bwd_problem(p);
+    return 2 + tc_states_launches(pb) + 1 + 1 + kTcBwdStateLaunches + kTcBwdLaunches + 1;
+  }
   return 2 + (tc_recompute(p, dt) ? 2 + tc_states_launches(p) : 2) + 6 +
          (bwd_segments(p) > 1 ? 1 : 0);
 }
@@ -862,6 +966,9 @@ cudaError_t launch_backward(const Problem& p, mlstm_dtype dt, const void* Q, con
                             const float* C0, const float* n0, const float* m0, const void* dH,
                             void* dQ, void* dK, void* dV, float* di, float* df, float* dC0,
                             float* dn0, float* dm0, void* ws, cudaStream_t st) {
+  if (tc_backward(p, dt))
+    return launch_bwd_tc(p, Q, K, V, i_pre, f_pre, C0, n0, m0, dH, dQ, dK, dV, di, df, dC0, dn0,
+                         dm0, ws, st);
   if (dt == MLSTM_DT_BF16)
     return launch_bwd_t<__nv_bfloat16>(p, dt, Q, K, V, i_pre, f_pre, C0, n0, m0, dH, dQ, dK, dV,
                                        di, df, dC0, dn0, dm0, ws, st);

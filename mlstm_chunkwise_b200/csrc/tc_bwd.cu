@@ -1,0 +1,549 @@
+// Backward pass of the chunkwise mLSTM on tcgen05: the gradients dq, dk, dv
+// of 128-token chunks ("Tiled Flash Linear Attention: More Efficient Linear
+// RNN and xLSTM Kernels", abstract: the mLSTM as an inter-chunk recurrence
+// plus an intra-chunk parallel part; its backward has the same two parts).
+//
+// In the stabilised frame of the forward (mu_t = max(m_k, amax_t) for token t
+// of chunk k, k^ = s k with s = 1/sqrt(d_qk)) the per-chunk gradients are
+//
+//   dP_ts = (du~_t . v_s + da~_t) e^{acol_s - mu_t} [s <= t]
+//   Sg_ts = (q_t . k^_s) e^{acol_s - mu_t} [s <= t]
+//   dq_t  = sum_s dP_ts k^_s + e^{m_k - mu_t} (C_k du~_t + da~_t n_k)
+//   dk^_s = sum_t dP_ts q_t  + w_s (G~_{k+1} v_s + g~_{k+1})
+//   dv_s  = sum_t Sg_ts du~_t + w_s G~_{k+1}^T k^_s,     w_s = e^{g_k + acol_s - m_{k+1}}
+//
+// (the SIMT kernels of bwd.cu state the same sums; G~, g~ come from the
+// reverse state recurrence).  Every gradient is two GEMMs with 128 rows: an
+// intra-chunk term (a gated 128 x 128 square times a token-major operand) and
+// a state term (a token-major operand times a [d_qk, d_v] state), each in its
+// own TMEM accumulator because the state term carries a per-row factor the
+// intra term does not; the epilogue combines them.
+//
+// The reverse states come from the same machinery: G~_k = e^{g_k + m_k -
+// m_{k+1}} G~_{k+1} + U_k with U_k = Q_k^T diag(e^{m_k - mu_t}) dU~_k, a
+// [d_qk, d_v] product over the chunk's tokens (one more job of the kernel,
+// from a bf16 copy of du~ whose rows carry e^{m_k - mu_t}), then a reverse
+// scan over the chunks, elementwise, that writes every G~_k as the bf16
+// operand copy (and G~_0 in fp32: the gradient of the initial state); g~ the
+// same way from the per-chunk sums of e^{m_k - mu_t} da~_t q_t.
+//
+// Launches: one for both squares (dP and Sg, written as bf16 in the block
+// layout of cb_block_row, so that the gradient kernels can read them as K- or
+// MN-major operand tiles with single bulk copies), then one each for dq, dk
+// and dv.  Token-major operands (Q, K, V, du~ in bf16) arrive by TMA in
+// 64 x 64 boxes with the 128-byte swizzle; the states (the forward's bf16
+// operand copy C_k and the reverse states G~ in the same block layout) and the
+// squares by untiled bulk copies.
+//
+// Roles (192 threads): warp 0 producer (TMA and bulk copies through a
+// 3-stage ring of 32 KB stages), warp 1 TMEM owner and MMA issuer, warps 2..5
+// the epilogue (TMEM lane = chunk row).  About 100 KB of shared memory and 256
+// TMEM columns per CTA: two CTAs share an SM, so one's epilogue overlaps the
+// other's loads.
+#include <cuda.h>
+
+#include "tc.h"
+#include "tc_ptx.cuh"
+
+namespace mlstm {
+namespace {
+
+using namespace tc;
+
+constexpr int kBT = 128;  // tokens per chunk = MMA rows
+constexpr int kThreads = 192;
+constexpr int kStages = 3;
+constexpr uint32_t kTileBytes = 16384;               // 128 rows x 128 bytes
+constexpr uint32_t kStageBytes = 2 * kTileBytes;      // A + B
+constexpr uint32_t kOffBar = kStages * kStageBytes;   // full[3], empty[3], acc
+constexpr uint32_t kOffSlot = kOffBar + 8 * 8;
+constexpr uint32_t kOffVec = kOffSlot + 16;           // 128 floats
+constexpr uint32_t kBytes = kOffVec + kBT * 4;
+constexpr uint32_t kSmem = kBytes + 1024;             // + alignment slack
+constexpr uint32_t kTmemCols = 256;                   // acc1 at 0, acc2 at 128
+
+enum Job : int { kSquares = 0, kDQ = 1, kDK = 2, kDV = 3, kU = 4 };
+
+struct TcBwdArgs {
+  Problem p;                       // chunking of 128 tokens
+  Gates g;
+  const float* dA;                 // da~ [BH, T]
+  const float* n_states;           // n_k [BH, NC, DK]
+  const float* g_states;           // g~_k [BH, NC + 1, DK]
+  const __nv_bfloat16* Cb;         // C_k, block layout, index bh NC + k
+  const __nv_bfloat16* Gb;         // G~_k, block layout, index bh (NC + 1) + k
+  __nv_bfloat16* sq;               // squares [BH NC][dP, Sg][2 s blocks][128 t][64]
+  const __nv_bfloat16* X;          // dq: Q, dk: K (for q.dq and k.dk)
+  __nv_bfloat16* out;              // dQ, dK or dV [BH, T, D]
+  float* dot;                      // q.dq or k.dk [BH, T] (accumulated)
+  float* U;                        // kU: U_k [BH, NC, DK, DV]
+};
+
+// Element offset of row r of s-block sb of square `which` of chunk bhk.
+__device__ __forceinline__ size_t sq_row(long bhk, int which, int sb, int r) {
+  return (((size_t)bhk * 2 + which) * 2 + sb) * (size_t)(kBT * 64) + (size_t)r * 64;
+}
+
+template <int kJob, int NT>
+__global__ void __launch_bounds__(kThreads, 2)
+tc_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+              const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_du,
+              const TcBwdArgs a) {
+  static_assert(NT == 64 || NT == 128, "output tile");
+  const Problem& p = a.p;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar_full = sbase + kOffBar, bar_empty = bar_full + 8 * kStages;
+  const uint32_t bar_acc = bar_full + 16 * kStages;
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + kOffSlot);
+  float* vec = reinterpret_cast<float*>(smem + kOffVec);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int k = blockIdx.y, bh = blockIdx.z;
+  const int NC = p.NC, T = p.T, DK = p.DK, DV = p.DV;
+  const int t0 = k * kBT;
+  // kU: blockIdx.x = column tile + (DV / 128) row tile; rows m0.. of DK
+  const int n0 = kJob == kSquares ? 0
+                 : kJob == kU     ? (blockIdx.x % (DV / 128)) * 128
+                                  : blockIdx.x * NT;
+  const int m0 = kJob == kU ? (blockIdx.x / (DV / 128)) * 128 : 0;
+  const int which = kJob == kSquares ? blockIdx.x : 0;  // squares: 0 = dP, 1 = Sg
+  const long bhk = (long)bh * NC + k;
+  const long bhk1 = (long)bh * (NC + 1) + k + 1;  // G~_{k+1}
+  const int n_vb = DV / 64;
+  // slabs of 64 along the contraction: term 1, then term 2
+  const int n1 = kJob == kSquares ? (which == 0 ? DV : DK) / 64 : 2;  // kU: 128 tokens
+  const int n2 = kJob == kDQ || kJob == kDK ? DV / 64 : (kJob == kDV ? DK / 64 : 0);
+  const int nS = n1 + n2;
+  constexpr int kN = kJob == kSquares ? kBT : NT;  // MMA N
+  constexpr uint32_t kBBytes = kN * 128;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(bar_full + 8 * i, 1);
+      mbar_init(bar_empty + 8 * i, 1);
+    }
+    mbar_init(bar_acc, 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32((const void*)tmem_slot), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------ producer ------------------------------
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      tma_prefetch_desc(&tm_du);
+      bool ok = true;
+      int issued = 0;
+      for (int i = 0; i < nS && ok; ++i) {
+        const int s = i % kStages, u = i / kStages;
+        if (u > 0) ok = mbar_wait(bar_empty + 8 * s, (u - 1) & 1, p, 1);
+        if (!ok) break;
+        const uint32_t sa = sbase + (uint32_t)s * kStageBytes, sb = sa + kTileBytes;
+        const uint32_t fb = bar_full + 8 * s;
+        mbar_expect_tx(fb, kTileBytes + kBBytes);
+        // token-major K-major tile: 128 rows of the chunk, contraction columns x0..x0+63
+        auto tok_rows = [&](const CUtensorMap* m, uint32_t dst, int x0) {
+          tma_load_3d(dst, m, x0, t0, bh, fb);
+          tma_load_3d(dst + 8192, m, x0, t0 + 64, bh, fb);
+        };
+        // token-major MN-major tile: columns n0.., contraction tokens t0 + 64 i..
+        auto tok_cols = [&](const CUtensorMap* m, uint32_t dst, int i1) {
+#pragma unroll
+          for (int b = 0; b < NT / 64; ++b)
+            tma_load_3d(dst + b * 8192, m, n0 + b * 64, t0 + i1 * 64, bh, fb);
+        };
+        // square as an MN-major A: rows s (two 64-blocks), contraction tokens 64 i..
+        auto sq_cols = [&](int w, uint32_t dst, int i1) {
+          bulk_load(dst, a.sq + sq_row(bhk, w, 0, i1 * 64), 8192, fb);
+          bulk_load(dst + 8192, a.sq + sq_row(bhk, w, 1, i1 * 64), 8192, fb);
+        };
+        if constexpr (kJob == kSquares) {
+          const CUtensorMap* ma = which == 0 ? &tm_du : &tm_q;
+          const CUtensorMap* mb = which == 0 ? &tm_v : &tm_k;
+          tok_rows(ma, sa, i * 64);
+          tok_rows(mb, sb, i * 64);
+        } else if constexpr (kJob == kDQ) {
+          if (i < n1) {
+            bulk_load(sa, a.sq + sq_row(bhk, 0, i, 0), kTileBytes, fb);  // dP, K-major
+            tok_cols(&tm_k, sb, i);
+          } else {
+            const int j = i - n1;
+            tok_rows(&tm_du, sa, j * 64);
+            bulk_load(sb, a.Cb + cb_block_row(bhk, j, n0, DK, n_vb), kBBytes, fb);
+          }
+        } else if constexpr (kJob == kDK) {
+          if (i < n1) {
+            sq_cols(0, sa, i);  // dP^T
+            tok_cols(&tm_q, sb, i);
+          } else {
+            const int j = i - n1;
+            tok_rows(&tm_v, sa, j * 64);
+            bulk_load(sb, a.Gb + cb_block_row(bhk1, j, n0, DK, n_vb), kBBytes, fb);
+          }
+        } else if constexpr (kJob == kU) {
+          // A = Q^T: rows d = m0.. (two 64-blocks), contraction tokens; B = r dU~
+          tma_load_3d(sa, &tm_q, m0, t0 + i * 64, bh, fb);
+          tma_load_3d(sa + 8192, &tm_q, m0 + 64, t0 + i * 64, bh, fb);
+          tok_cols(&tm_du, sb, i);
+        } else {
+          if (i < n1) {
+            sq_cols(1, sa, i);  // Sg^T
+            tok_cols(&tm_du, sb, i);
+          } else {
+            const int j = i - n1;
+            tok_rows(&tm_k, sa, j * 64);
+#pragma unroll
+            for (int b = 0; b < NT / 64; ++b)
+              bulk_load(sb + b * 8192, a.Gb + cb_block_row(bhk1, n0 / 64 + b, j * 64, DK, n_vb),
+                        8192, fb);
+          }
+        }
+        issued = i + 1;
+      }
+      // every copy issued has landed before the CTA may exit
+      for (int q = (issued > kStages ? issued - kStages : 0); q < issued; ++q)
+        mbar_wait(bar_full + 8 * (q % kStages), (q / kStages) & 1, p, 2);
+    }
+  } else if (warp == 1) {
+    // ------------------------------ MMA issuer ----------------------------
+    if (lane == 0) {
+      // operand majors per term: 1 = MN-major
+      constexpr int a1 = (kJob == kDK || kJob == kDV || kJob == kU) ? 1 : 0;
+      constexpr int b1 = kJob == kSquares ? 0 : 1;
+      constexpr int b2 = kJob == kDV ? 1 : 0;
+      constexpr uint32_t id1 = idesc_bf16(128, kN, a1, b1);
+      constexpr uint32_t id2 = idesc_bf16(128, kN, 0, b2);
+      bool ok = true;
+      for (int i = 0; i < nS && ok; ++i) {
+        const int s = i % kStages;
+        ok = mbar_wait(bar_full + 8 * s, (i / kStages) & 1, p, 3);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t sa = sbase + (uint32_t)s * kStageBytes, sb = sa + kTileBytes;
+        const bool t2 = i >= n1;
+        const bool first = i == 0 || i == n1;
+        const uint32_t d = tmem + (t2 ? 128u : 0u);
+        const int am = t2 ? 0 : a1, bm = t2 ? b2 : b1;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t ad = am ? sdesc_sw128(sa + kk * 2048, 8192, 1024)
+                                 : sdesc_sw128(sa + kk * 32, 16, 1024);
+          const uint64_t bd = bm ? sdesc_sw128(sb + kk * 2048, 8192, 1024)
+                                 : sdesc_sw128(sb + kk * 32, 16, 1024);
+          mma_bf16_ss(d, ad, bd, t2 ? id2 : id1, (first && kk == 0) ? 0u : 1u);
+        }
+        mma_commit(bar_empty + 8 * s);
+      }
+      mma_commit(bar_acc);
+    }
+  } else {
+    // ------------------------------ epilogue ------------------------------
+    const int q4 = warp & 3;
+    const int r = q4 * 32 + lane;  // chunk row = TMEM lane
+    const uint32_t trow = tmem + ((uint32_t)(q4 * 32) << 16);
+    const long tpad = (long)NC * kBT;
+    const int t = t0 + r;
+    const bool valid = t < T;
+    const float m_in = a.g.mchk[(long)bh * (NC + 1) + k];
+    const float m_out = a.g.mchk[(long)bh * (NC + 1) + k + 1];
+    const float acol_r = a.g.acol[(long)bh * tpad + t];  // -inf on padding
+    const float mu = fmaxf(m_in, a.g.amax[(long)bh * tpad + t]);
+    if constexpr (kJob == kSquares) {
+      vec[r] = acol_r;
+      named_bar_sync(1, 128);
+    }
+    const bool ok = mbar_wait(bar_acc, 0, p, 4);
+    tc_fence_after();
+    if (ok) {
+      if constexpr (kJob == kSquares) {
+        const float da = (which == 0 && valid) ? a.dA[(long)bh * T + t] : 0.f;
+#pragma unroll 1
+        for (int c = 0; c < kBT / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32(trow + c * 32, v);
+          tmem_wait_ld();
+          uint32_t w[16];
+#pragma unroll
+          for (int j = 0; j < 32; j += 2) {
+            float f[2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int s = c * 32 + j + e;
+              const float x = __uint_as_float(v[j + e]);
+              const float val = which == 0 ? x + da : p.key_scale * x;
+              f[e] = (valid && s <= r) ? val * expf(vec[s] - mu) : 0.f;
+            }
+            w[j / 2] = pack_bf16x2(f[0], f[1]);
+          }
+          __nv_bfloat16* row = a.sq + sq_row(bhk, which, c >> 1, r);
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int cc = (c & 1) * 4 + u;  // 16-byte chunk of the 128-byte row
+            *reinterpret_cast<uint4*>(row + ((cc ^ (r & 7)) * 8)) =
+                make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+          }
+        }
+      } else if constexpr (kJob == kU) {
+        float* dst = a.U + (bhk * DK + m0 + r) * (long)DV + n0;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t v[32];
+          tmem_ld32(trow + c * 32, v);
+          tmem_wait_ld();
+          float4* d4 = reinterpret_cast<float4*>(dst + c * 32);
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            d4[u] = make_float4(__uint_as_float(v[4 * u]), __uint_as_float(v[4 * u + 1]),
+                                __uint_as_float(v[4 * u + 2]), __uint_as_float(v[4 * u + 3]));
+        }
+      } else {
+        const int D = kJob == kDV ? DV : DK;
+        float rs, alpha = 0.f, s1, s2;
+        const float* beta = nullptr;
+        if constexpr (kJob == kDQ) {
+          rs = expf(m_in - mu);
+          alpha = valid ? a.dA[(long)bh * T + t] : 0.f;
+          beta = a.n_states + bhk * DK;
+          s1 = p.key_scale;
+          s2 = 1.f;
+        } else {
+          const float gk = a.g.gtot[(long)bh * NC + k];
+          rs = expf(gk + acol_r - m_out);  // w_s, 0 on padding
+          if constexpr (kJob == kDK) {
+            alpha = 1.f;
+            beta = a.g_states + bhk1 * DK;
+            s1 = p.key_scale;
+            s2 = p.key_scale;
+          } else {
+            s1 = 1.f;
+            s2 = p.key_scale;
+          }
+        }
+        float dot = 0.f;
+        const long orow = ((long)bh * T + t) * D + n0;
+#pragma unroll 1
+        for (int c = 0; c < NT / 32; ++c) {
+          uint32_t v1[32], v2[32];
+          tmem_ld32(trow + c * 32, v1);
+          tmem_ld32(trow + 128 + c * 32, v2);
+          tmem_wait_ld();
+          float o[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            float x2 = __uint_as_float(v2[j]);
+            if (kJob != kDV) x2 = fmaf(alpha, beta[n0 + c * 32 + j], x2);
+            // dq: s acc1 + rs (acc2 + da n);  dk: s (acc1 + w (acc2 + g~));  dv: acc1 + s w acc2
+            o[j] = kJob == kDK ? s1 * fmaf(rs, x2, __uint_as_float(v1[j]))
+                               : fmaf(s1, __uint_as_float(v1[j]), s2 * rs * x2);
+          }
+          if (valid) {
+            uint4* dst = reinterpret_cast<uint4*>(a.out + orow + c * 32);
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+              dst[u] = make_uint4(pack_bf16x2(o[8 * u], o[8 * u + 1]),
+                                  pack_bf16x2(o[8 * u + 2], o[8 * u + 3]),
+                                  pack_bf16x2(o[8 * u + 4], o[8 * u + 5]),
+                                  pack_bf16x2(o[8 * u + 6], o[8 * u + 7]));
+            if constexpr (kJob != kDV) {
+              const uint4* xs = reinterpret_cast<const uint4*>(a.X + orow + c * 32);
+#pragma unroll
+              for (int u = 0; u < 4; ++u) {
+                const uint4 xv = xs[u];
+                const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  const float2 f = __bfloat1622float2(
+                      *reinterpret_cast<const __nv_bfloat162*>(&xw[e]));
+                  dot = fmaf(f.x, o[8 * u + 2 * e], dot);
+                  dot = fmaf(f.y, o[8 * u + 2 * e + 1], dot);
+                }
+              }
+            }
+          }
+        }
+        if (kJob != kDV && valid) atomicAdd(&a.dot[(long)bh * T + t], dot);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    if (lane == 0) mbar_wait(bar_acc, 0, p, 5);  // every MMA has completed
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// Per-chunk increments of g~: u_k[d] = sum_{t in k, t < T} e^{m_k - mu_t} da~_t q_t[d].
+// One block per (chunk, b h), one thread per d.
+__global__ void __launch_bounds__(256)
+tc_bwd_gvec_kernel(Problem p, Gates g, const __nv_bfloat16* __restrict__ Q,
+                   const float* __restrict__ dA, float* __restrict__ u) {
+  const int k = blockIdx.x, bh = blockIdx.y, d = threadIdx.x;
+  const int NC = p.NC, T = p.T, DK = p.DK;
+  if (d >= DK) return;
+  const long tpad = (long)NC * kBT;
+  const float m_in = g.mchk[(long)bh * (NC + 1) + k];
+  const int t1 = min(T, (k + 1) * kBT);
+  float acc = 0.f;
+#pragma unroll 4
+  for (int t = k * kBT; t < t1; ++t) {
+    const float w = expf(m_in - fmaxf(m_in, g.amax[(long)bh * tpad + t])) * dA[(long)bh * T + t];
+    acc = fmaf(w, __bfloat162float(Q[((long)bh * T + t) * DK + d]), acc);
+  }
+  u[((long)bh * NC + k) * DK + d] = acc;
+}
+
+// Reverse scan G~_k = e^{g_k + m_k - m_{k+1}} G~_{k+1} + U_k from G~_NC = 0:
+// every G~_k as the bf16 operand copy (block layout of cb_block_row, index
+// bh (NC + 1) + k), G~_0 in fp32 into dC0; threads past the state do g~ into
+// g_states [BH, NC + 1, DK] from the increments u.  A state thread owns 8
+// consecutive columns of one row (one 16-byte chunk of the copy).
+__global__ void __launch_bounds__(256)
+tc_bwd_scan_kernel(Problem p, Gates g, const float* __restrict__ U, const float* __restrict__ u,
+                   __nv_bfloat16* __restrict__ Gb, float* __restrict__ g_states,
+                   float* __restrict__ dC0) {
+  const int bh = blockIdx.y, NC = p.NC, DK = p.DK, DV = p.DV;
+  const long idx = (long)blockIdx.x * blockDim.x + threadIdx.x;
+  const long n_st = (long)DK * DV / 8;
+  const float* gt = g.gtot + (long)bh * NC;
+  const float* mc = g.mchk + (long)bh * (NC + 1);
+  if (idx < n_st) {
+    const int dk = (int)(idx * 8 / DV), c = (int)(idx * 8 % DV);
+    const int vb = c / 64, j = (c % 64) / 8, n_vb = DV / 64;
+    const size_t pos = (size_t)((j ^ (dk & 7)) * 8);
+    float G[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    *reinterpret_cast<uint4*>(Gb + cb_block_row((long)bh * (NC + 1) + NC, vb, dk, DK, n_vb) + pos) =
+        make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll 2
+    for (int k = NC - 1; k >= 0; --k) {
+      const float decay = expf(gt[k] + mc[k] - mc[k + 1]);
+      const float4* src = reinterpret_cast<const float4*>(U + (((long)bh * NC + k) * DK + dk) * DV + c);
+      const float4 x0 = src[0], x1 = src[1];
+      G[0] = fmaf(decay, G[0], x0.x);
+      G[1] = fmaf(decay, G[1], x0.y);
+      G[2] = fmaf(decay, G[2], x0.z);
+      G[3] = fmaf(decay, G[3], x0.w);
+      G[4] = fmaf(decay, G[4], x1.x);
+      G[5] = fmaf(decay, G[5], x1.y);
+      G[6] = fmaf(decay, G[6], x1.z);
+      G[7] = fmaf(decay, G[7], x1.w);
+      *reinterpret_cast<uint4*>(Gb + cb_block_row((long)bh * (NC + 1) + k, vb, dk, DK, n_vb) + pos) =
+          make_uint4(pack_bf16x2(G[0], G[1]), pack_bf16x2(G[2], G[3]), pack_bf16x2(G[4], G[5]),
+                     pack_bf16x2(G[6], G[7]));
+    }
+    float4* d4 = reinterpret_cast<float4*>(dC0 + ((long)bh * DK + dk) * DV + c);
+    d4[0] = make_float4(G[0], G[1], G[2], G[3]);
+    d4[1] = make_float4(G[4], G[5], G[6], G[7]);
+  } else if (idx < n_st + DK) {
+    const int d = (int)(idx - n_st);
+    float gv = 0.f;
+    g_states[((long)bh * (NC + 1) + NC) * DK + d] = 0.f;
+    for (int k = NC - 1; k >= 0; --k) {
+      gv = fmaf(expf(gt[k] + mc[k] - mc[k + 1]), gv, u[((long)bh * NC + k) * DK + d]);
+      g_states[((long)bh * (NC + 1) + k) * DK + d] = gv;
+    }
+  }
+}
+
+template <int kJob, int NT>
+cudaError_t launch_job(const CUtensorMap* m, const TcBwdArgs& a, dim3 grid, cudaStream_t st) {
+  auto kern = tc_bwd_kernel<kJob, NT>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, kThreads, kSmem, st>>>(m[0], m[1], m[2], m[3], a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool tc_bwd_supported(const Problem& pb) {
+  return pb.L == kBT && (pb.DK == 128 || pb.DK == 256) && pb.DV % 128 == 0 && pb.DV <= 1024 &&
+         pb.T > 0 && tc_unfused_supported(pb);
+}
+
+size_t tc_bwd_square_elems(const Problem& pb) { return (size_t)pb.BH * pb.NC * 2 * kBT * kBT; }
+
+cudaError_t launch_tc_bwd_states(const Problem& pb, const void* Q, const __nv_bfloat16* dUr16,
+                                 Gates g, const float* dA, float* U, float* u,
+                                 __nv_bfloat16* Gb, float* g_states, float* dC0,
+                                 cudaStream_t st) {
+  if (!tc_bwd_supported(pb)) return cudaErrorNotSupported;
+  CUtensorMap m[4];
+  if (!encode_tmap_3d(&m[0], Q, 2, pb.DK, pb.T, pb.BH, 64, 64, 128) ||
+      !encode_tmap_3d(&m[3], dUr16, 2, pb.DV, pb.T, pb.BH, 64, 64, 128))
+    return cudaErrorInvalidValue;
+  m[1] = m[0];
+  m[2] = m[0];
+  TcBwdArgs a = {};
+  a.p = pb;
+  a.g = g;
+  a.U = U;
+  cudaError_t e =
+      launch_job<kU, 128>(m, a, dim3((pb.DK / 128) * (pb.DV / 128), pb.NC, pb.BH), st);
+  if (e != cudaSuccess) return e;
+  tc_bwd_gvec_kernel<<<dim3(pb.NC, pb.BH), pb.DK, 0, st>>>(
+      pb, g, static_cast<const __nv_bfloat16*>(Q), dA, u);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const long n = (long)pb.DK * pb.DV / 8 + pb.DK;
+  tc_bwd_scan_kernel<<<dim3((unsigned)((n + 255) / 256), pb.BH), 256, 0, st>>>(pb, g, U, u, Gb,
+                                                                              g_states, dC0);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_tc_bwd(const Problem& pb, const void* Q, const void* K, const void* V,
+                          const __nv_bfloat16* dU16, Gates g, const float* dA,
+                          const float* n_states, const float* g_states, const __nv_bfloat16* Cb,
+                          const __nv_bfloat16* Gb, __nv_bfloat16* sq, void* dQ, void* dK,
+                          void* dV, float* qdq, float* kdk, cudaStream_t st) {
+  if (!tc_bwd_supported(pb)) return cudaErrorNotSupported;
+  CUtensorMap m[4];
+  if (!encode_tmap_3d(&m[0], Q, 2, pb.DK, pb.T, pb.BH, 64, 64, 128) ||
+      !encode_tmap_3d(&m[1], K, 2, pb.DK, pb.T, pb.BH, 64, 64, 128) ||
+      !encode_tmap_3d(&m[2], V, 2, pb.DV, pb.T, pb.BH, 64, 64, 128) ||
+      !encode_tmap_3d(&m[3], dU16, 2, pb.DV, pb.T, pb.BH, 64, 64, 128))
+    return cudaErrorInvalidValue;
+  TcBwdArgs a = {};
+  a.p = pb;
+  a.g = g;
+  a.dA = dA;
+  a.n_states = n_states;
+  a.g_states = g_states;
+  a.Cb = Cb;
+  a.Gb = Gb;
+  a.sq = sq;
+  cudaError_t e = launch_job<kSquares, 128>(m, a, dim3(2, pb.NC, pb.BH), st);
+  if (e != cudaSuccess) return e;
+  // 128 output columns per CTA (DK and DV are multiples of 128)
+  a.X = static_cast<const __nv_bfloat16*>(Q);
+  a.out = static_cast<__nv_bfloat16*>(dQ);
+  a.dot = qdq;
+  e = launch_job<kDQ, 128>(m, a, dim3(pb.DK / 128, pb.NC, pb.BH), st);
+  if (e != cudaSuccess) return e;
+  a.X = static_cast<const __nv_bfloat16*>(K);
+  a.out = static_cast<__nv_bfloat16*>(dK);
+  a.dot = kdk;
+  e = launch_job<kDK, 128>(m, a, dim3(pb.DK / 128, pb.NC, pb.BH), st);
+  if (e != cudaSuccess) return e;
+  a.X = nullptr;
+  a.out = static_cast<__nv_bfloat16*>(dV);
+  a.dot = nullptr;
+  return launch_job<kDV, 128>(m, a, dim3(pb.DV / 128, pb.NC, pb.BH), st);
+}
+
+}  // namespace mlstm

@@ -28,6 +28,11 @@ CASES = [
     (1, 2, 1, 64, 64, 64, "f32", "exp", True),          # single token
     (1, 2, 640, 256, 512, 256, "bf16", "exp", True),    # 7B head shape: forward recomputed on TC
     (1, 2, 384, 128, 128, 64, "bf16", "sigmoid", False),  # chunk 64 on TC (pair mode)
+    # bf16 with d_qk 128 or 256: tensor-core gradients on 128-token chunks
+    (2, 2, 200, 128, 256, 64, "bf16", "exp", True),     # ragged last chunk, 2 value tiles
+    (1, 1, 2048, 128, 128, 256, "bf16", "sigmoid", True),  # one head: segmented recurrences
+    (1, 2, 130, 128, 128, 128, "bf16", "exp", True),    # a 2-token last chunk
+    (2, 1, 100, 128, 128, 128, "bf16", "exp", True),    # shorter than a chunk: fp32 kernels
 ]
 
 
