@@ -1,4 +1,5 @@
-// Backward pass of the chunkwise mLSTM (fp32 CUDA-core gradient kernels).
+// Backward pass of the chunkwise mLSTM: host orchestration and the fp32
+// CUDA-core gradient kernels.
 //
 // The forward ("Tiled Flash Linear Attention: More Efficient Linear RNN and
 // xLSTM Kernels", abstract: the mLSTM as an inter-chunk recurrence plus an
@@ -33,14 +34,17 @@
 // G~_k is the gradient with respect to the state entering chunk k, in that
 // state's frame, so dC0 = G~_0, dn0 = g~_0 and dm0 = <C0, dC0> + n0 . dn0.
 //
-// Launches: the forward's gates, chunk states and outputs (h and the signed
-// denominator kept), a per-token pass forming du~ and da~, the reverse state
-// recurrence, dq, dk, dv, and the gate gradients (dot products and a reverse
-// scan).  The forward is recomputed on the tensor cores for bf16 inputs where
-// the unfused tensor-core path supports the shape (fp32 chunk states, then
-// their bf16 operand copy for the output kernel, h in bf16), else on the fp32
-// kernels (h in fp32).  The gradient kernels tile 64 x 64 outputs over 256
-// threads (4 x 4 per thread), like the fp32 forward kernels.
+// Two paths.  bf16 inputs with d_qk of 128 or 256 (and a d_v the tensor-core
+// forward takes), at least 128 tokens: everything on 128-token chunks, the
+// forward recomputed on the tensor cores, the reverse states and dq, dk, dv as
+// tcgen05 GEMMs (tc_bwd.cu; launch_bwd_tc below).  Otherwise, in this file:
+// the forward's gates, chunk states and outputs (h and the signed denominator
+// kept), a per-token pass forming du~ and da~, the reverse state recurrence,
+// dq, dk, dv, and the gate gradients (dot products and a reverse scan), on
+// fp32 CUDA-core kernels (the forward recomputed on the tensor cores for bf16
+// shapes the unfused tensor-core forward supports: fp32 chunk states, their
+// bf16 operand copy, h in bf16).  The gradient kernels own 64 rows and up to
+// 256 output columns (8 x 8 accumulators per thread).
 #include <math.h>
 
 #include <type_traits>
@@ -58,46 +62,6 @@ constexpr int kThr = 256;
 template <typename TIn>
 __device__ __forceinline__ float ld(const TIn* base, long idx, bool ok) {
   return ok ? to_float(base[idx]) : 0.f;
-}
-
-__device__ __forceinline__ float sum16(float v) {
-#pragma unroll
-  for (int o = 8; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  return v;
-}
-
-// acc[i][j] += sum_c A[ty*4+i][c] * B[c][tx*4+j] over one slab
-__device__ __forceinline__ void mac_slab(float (&acc)[4][4], const float (*A)[kS + 1],
-                                         const float (*B)[kT], int ty, int tx) {
-#pragma unroll 4
-  for (int c = 0; c < kS; ++c) {
-    float a[4], b[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) a[i] = A[ty * 4 + i][c];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) b[j] = B[c][tx * 4 + j];
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
-  }
-}
-
-// acc[i][j] += sum_s P[ty*4+i][s] * B[s][tx*4+j] over a 64-long contraction
-__device__ __forceinline__ void mac_tile(float (&acc)[4][4], const float (*P)[kT + 1],
-                                         const float (*B)[kT], int ty, int tx) {
-#pragma unroll 4
-  for (int s = 0; s < kT; ++s) {
-    float a[4], b[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) a[i] = P[ty * 4 + i][s];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) b[j] = B[s][tx * 4 + j];
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
-  }
 }
 
 // ---------------------------------------------------------------------------
@@ -700,9 +664,9 @@ struct BwdWs {
       *dn0, *seg;
   __nv_bfloat16 *Cb, *H16;  // tensor-core recompute: operand copy of the states, bf16 h
   // tensor-core gradients: du~ (plain and row-scaled), reverse states, squares,
-  // per-chunk updates of the reverse states and of g~
+  // per-chunk increments of g~
   __nv_bfloat16 *dU16, *dUr16, *Gb, *sq;
-  float *U, *uvec;
+  float* uvec;
 };
 
 // Whether the forward is recomputed on the tensor cores.
@@ -775,7 +739,6 @@ size_t carve(const Problem& p_in, mlstm_dtype dt, char* base, BwdWs* w) {
     x.dUr16 = take16(BH * T * DV);
     x.Gb = take16(BH * (NC + 1) * DK * DV);
     x.sq = take16(tc_bwd_square_elems(p));
-    x.U = take(BH * NC * DK * DV);
     x.uvec = take(BH * NC * DK);
   }
   if (w) *w = x;
@@ -811,7 +774,7 @@ cudaError_t launch_bwd_tc(const Problem& p_in, const void* Q, const void* K, con
       w.dUr16, w.g);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  e = launch_tc_bwd_states(p, Q, w.dUr16, w.g, w.dA, w.U, w.uvec, w.Gb, w.g_states, w.dC0, st);
+  e = launch_tc_bwd_states(p, Q, w.dUr16, w.g, w.dA, w.uvec, w.Gb, w.g_states, w.dC0, st);
   if (e != cudaSuccess) return e;
   e = cudaMemcpy2DAsync(w.dn0, sizeof(float) * p.DK, w.g_states, sizeof(float) * (p.NC + 1) * p.DK,
                         sizeof(float) * p.DK, p.BH, cudaMemcpyDeviceToDevice, st);
@@ -876,7 +839,7 @@ cudaError_t launch_bwd_t(const Problem& p, mlstm_dtype dt, const void* Q, const 
   else
     bwd_prep_kernel<TIn, float><<<prep_blocks, kThr, 0, st>>>(
         p, static_cast<const TIn*>(dH), w.H32, w.den, w.mr, w.dU, w.dA);
-  const int nk = (p.DK + kT - 1) / kT, nv = (p.DV + kT - 1) / kT, nt = (p.T + kT - 1) / kT;
+  const int nk = (p.DK + kT - 1) / kT, nv = (p.DV + kT - 1) / kT;
   const int n_seg = bwd_segments(p);
   bwd_states_kernel<TIn><<<dim3(nv, nk, p.BH * n_seg), kThr, 0, st>>>(p, q, w.dU, w.dA, w.g,
                                                                      w.G_states, w.g_states, n_seg);
@@ -953,7 +916,7 @@ int bwd_launches(const Problem& p, mlstm_dtype dt) {
   // + prep, reverse states [+ fix-up], dq, dk, dv, gate gradients (6 or 7)
   if (tc_backward(p, dt)) {
     // gates (2), chunk states [+ fix-up], outputs, prep, reverse states
-    // (updates, g~ increments, scan), squares + dq + dk + dv, gate gradients
+    // (g~ increments, recurrence), squares + dq + dk + dv, gate gradients
     const Problem pb = tc_bwd_problem(p);
     return 2 + tc_states_launches(pb) + 1 + 1 + kTcBwdStateLaunches + kTcBwdLaunches + 1;
   }

@@ -67,16 +67,15 @@ cudaError_t launch_tc_bwd(const Problem& pb, const void* Q, const void* K, const
                           const __nv_bfloat16* Gb, __nv_bfloat16* sq, void* dQ, void* dK,
                           void* dV, float* qdq, float* kdk, cudaStream_t st);
 constexpr int kTcBwdLaunches = 4;
-// Reverse states on tensor cores (tc_bwd.cu): U_k = Q_k^T dUr_k per chunk
-// (dUr16: du~ with rows scaled by e^{m_k - mu_t}, bf16), the per-chunk g~
-// increments u, and the reverse scan writing Gb (bf16 operand copy of every
-// G~_k, NC + 1 per head), g_states (fp32) and dC0 = G~_0 (fp32).  Scratch: U
-// [BH, NC, DK, DV] and u [BH, NC, DK] fp32.
+// Reverse states on tensor cores (tc_bwd.cu): the per-chunk g~ increments u
+// (scratch [BH, NC, DK] fp32), then the recurrence G~_k = decay_k G~_{k+1} +
+// Q_k^T dUr_k (dUr16: du~ with rows scaled by e^{m_k - mu_t}, bf16) writing Gb
+// (bf16 operand copy of every G~_k, NC + 1 per head), g_states (fp32) and
+// dC0 = G~_0 (fp32).
 cudaError_t launch_tc_bwd_states(const Problem& pb, const void* Q, const __nv_bfloat16* dUr16,
-                                 Gates g, const float* dA, float* U, float* u,
-                                 __nv_bfloat16* Gb, float* g_states, float* dC0,
-                                 cudaStream_t st);
-constexpr int kTcBwdStateLaunches = 3;
+                                 Gates g, const float* dA, float* u, __nv_bfloat16* Gb,
+                                 float* g_states, float* dC0, cudaStream_t st);
+constexpr int kTcBwdStateLaunches = 2;
 
 // Failure-detection self-test (selftest.cu): one bounded wait that nothing
 // satisfies; it sets the watchdog bit and its site in *err and returns.

@@ -19,13 +19,12 @@
 // own TMEM accumulator because the state term carries a per-row factor the
 // intra term does not; the epilogue combines them.
 //
-// The reverse states come from the same machinery: G~_k = e^{g_k + m_k -
-// m_{k+1}} G~_{k+1} + U_k with U_k = Q_k^T diag(e^{m_k - mu_t}) dU~_k, a
-// [d_qk, d_v] product over the chunk's tokens (one more job of the kernel,
-// from a bf16 copy of du~ whose rows carry e^{m_k - mu_t}), then a reverse
-// scan over the chunks, elementwise, that writes every G~_k as the bf16
-// operand copy (and G~_0 in fp32: the gradient of the initial state); g~ the
-// same way from the per-chunk sums of e^{m_k - mu_t} da~_t q_t.
+// The reverse states G~_k = e^{g_k + m_k - m_{k+1}} G~_{k+1} + Q_k^T dUr_k
+// (dUr: a bf16 copy of du~ whose rows carry e^{m_k - mu_t}) run in
+// tc_bwd_rev_kernel: a CTA per 128 x 128 tile of the state keeps the running
+// G~ in TMEM and walks the chunks from the last, writing every G~_k as the
+// bf16 operand copy (and G~_0 in fp32: the gradient of the initial state);
+// g~ follows from the per-chunk sums of e^{m_k - mu_t} da~_t q_t.
 //
 // Launches: one for both squares (dP and Sg, written as bf16 in the block
 // layout of cb_block_row, so that the gradient kernels can read them as K- or
@@ -62,7 +61,7 @@ constexpr uint32_t kBytes = kOffVec + kBT * 4;
 constexpr uint32_t kSmem = kBytes + 1024;             // + alignment slack
 constexpr uint32_t kTmemCols = 256;                   // acc1 at 0, acc2 at 128
 
-enum Job : int { kSquares = 0, kDQ = 1, kDK = 2, kDV = 3, kU = 4 };
+enum Job : int { kSquares = 0, kDQ = 1, kDK = 2, kDV = 3 };
 
 struct TcBwdArgs {
   Problem p;                       // chunking of 128 tokens
@@ -76,7 +75,6 @@ struct TcBwdArgs {
   const __nv_bfloat16* X;          // dq: Q, dk: K (for q.dq and k.dk)
   __nv_bfloat16* out;              // dQ, dK or dV [BH, T, D]
   float* dot;                      // q.dq or k.dk [BH, T] (accumulated)
-  float* U;                        // kU: U_k [BH, NC, DK, DV]
 };
 
 // Element offset of row r of s-block sb of square `which` of chunk bhk.
@@ -104,17 +102,13 @@ tc_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
   const int k = blockIdx.y, bh = blockIdx.z;
   const int NC = p.NC, T = p.T, DK = p.DK, DV = p.DV;
   const int t0 = k * kBT;
-  // kU: blockIdx.x = column tile + (DV / 128) row tile; rows m0.. of DK
-  const int n0 = kJob == kSquares ? 0
-                 : kJob == kU     ? (blockIdx.x % (DV / 128)) * 128
-                                  : blockIdx.x * NT;
-  const int m0 = kJob == kU ? (blockIdx.x / (DV / 128)) * 128 : 0;
+  const int n0 = kJob == kSquares ? 0 : blockIdx.x * NT;
   const int which = kJob == kSquares ? blockIdx.x : 0;  // squares: 0 = dP, 1 = Sg
   const long bhk = (long)bh * NC + k;
   const long bhk1 = (long)bh * (NC + 1) + k + 1;  // G~_{k+1}
   const int n_vb = DV / 64;
   // slabs of 64 along the contraction: term 1, then term 2
-  const int n1 = kJob == kSquares ? (which == 0 ? DV : DK) / 64 : 2;  // kU: 128 tokens
+  const int n1 = kJob == kSquares ? (which == 0 ? DV : DK) / 64 : 2;
   const int n2 = kJob == kDQ || kJob == kDK ? DV / 64 : (kJob == kDV ? DK / 64 : 0);
   const int nS = n1 + n2;
   constexpr int kN = kJob == kSquares ? kBT : NT;  // MMA N
@@ -192,11 +186,6 @@ tc_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             tok_rows(&tm_v, sa, j * 64);
             bulk_load(sb, a.Gb + cb_block_row(bhk1, j, n0, DK, n_vb), kBBytes, fb);
           }
-        } else if constexpr (kJob == kU) {
-          // A = Q^T: rows d = m0.. (two 64-blocks), contraction tokens; B = r dU~
-          tma_load_3d(sa, &tm_q, m0, t0 + i * 64, bh, fb);
-          tma_load_3d(sa + 8192, &tm_q, m0 + 64, t0 + i * 64, bh, fb);
-          tok_cols(&tm_du, sb, i);
         } else {
           if (i < n1) {
             sq_cols(1, sa, i);  // Sg^T
@@ -220,7 +209,7 @@ tc_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     // ------------------------------ MMA issuer ----------------------------
     if (lane == 0) {
       // operand majors per term: 1 = MN-major
-      constexpr int a1 = (kJob == kDK || kJob == kDV || kJob == kU) ? 1 : 0;
+      constexpr int a1 = (kJob == kDK || kJob == kDV) ? 1 : 0;
       constexpr int b1 = kJob == kSquares ? 0 : 1;
       constexpr int b2 = kJob == kDV ? 1 : 0;
       constexpr uint32_t id1 = idesc_bf16(128, kN, a1, b1);
@@ -294,19 +283,6 @@ tc_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             *reinterpret_cast<uint4*>(row + ((cc ^ (r & 7)) * 8)) =
                 make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
           }
-        }
-      } else if constexpr (kJob == kU) {
-        float* dst = a.U + (bhk * DK + m0 + r) * (long)DV + n0;
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t v[32];
-          tmem_ld32(trow + c * 32, v);
-          tmem_wait_ld();
-          float4* d4 = reinterpret_cast<float4*>(dst + c * 32);
-#pragma unroll
-          for (int u = 0; u < 8; ++u)
-            d4[u] = make_float4(__uint_as_float(v[4 * u]), __uint_as_float(v[4 * u + 1]),
-                                __uint_as_float(v[4 * u + 2]), __uint_as_float(v[4 * u + 3]));
         }
       } else {
         const int D = kJob == kDV ? DV : DK;
@@ -389,74 +365,221 @@ tc_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 }
 
 // Per-chunk increments of g~: u_k[d] = sum_{t in k, t < T} e^{m_k - mu_t} da~_t q_t[d].
-// One block per (chunk, b h), one thread per d.
+// One block of 256 threads per (chunk, b h): a thread sums 8 consecutive d
+// (16-byte loads of q) over every (256 / (DK / 8))-th token of the chunk, and
+// the token groups are added up in shared memory.
 __global__ void __launch_bounds__(256)
 tc_bwd_gvec_kernel(Problem p, Gates g, const __nv_bfloat16* __restrict__ Q,
                    const float* __restrict__ dA, float* __restrict__ u) {
-  const int k = blockIdx.x, bh = blockIdx.y, d = threadIdx.x;
-  const int NC = p.NC, T = p.T, DK = p.DK;
-  if (d >= DK) return;
+  __shared__ float red[256 * 8];
+  const int k = blockIdx.x, bh = blockIdx.y, NC = p.NC, T = p.T, DK = p.DK;
+  const int n_dg = DK / 8, n_tg = 256 / n_dg;
+  const int dg = threadIdx.x % n_dg, tg = threadIdx.x / n_dg;
   const long tpad = (long)NC * kBT;
   const float m_in = g.mchk[(long)bh * (NC + 1) + k];
   const int t1 = min(T, (k + 1) * kBT);
-  float acc = 0.f;
-#pragma unroll 4
-  for (int t = k * kBT; t < t1; ++t) {
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  for (int t = k * kBT + tg; t < t1; t += n_tg) {
     const float w = expf(m_in - fmaxf(m_in, g.amax[(long)bh * tpad + t])) * dA[(long)bh * T + t];
-    acc = fmaf(w, __bfloat162float(Q[((long)bh * T + t) * DK + d]), acc);
+    const uint4 qv = *reinterpret_cast<const uint4*>(Q + ((long)bh * T + t) * DK + dg * 8);
+    const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&qw[e]));
+      acc[2 * e] = fmaf(w, f.x, acc[2 * e]);
+      acc[2 * e + 1] = fmaf(w, f.y, acc[2 * e + 1]);
+    }
   }
-  u[((long)bh * NC + k) * DK + d] = acc;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) red[threadIdx.x * 8 + e] = acc[e];
+  __syncthreads();
+  for (int d = threadIdx.x; d < DK; d += blockDim.x) {
+    float sum = 0.f;
+    for (int q = 0; q < n_tg; ++q) sum += red[(q * n_dg + d / 8) * 8 + d % 8];
+    u[((long)bh * NC + k) * DK + d] = sum;
+  }
 }
 
-// Reverse scan G~_k = e^{g_k + m_k - m_{k+1}} G~_{k+1} + U_k from G~_NC = 0:
-// every G~_k as the bf16 operand copy (block layout of cb_block_row, index
-// bh (NC + 1) + k), G~_0 in fp32 into dC0; threads past the state do g~ into
-// g_states [BH, NC + 1, DK] from the increments u.  A state thread owns 8
-// consecutive columns of one row (one 16-byte chunk of the copy).
-__global__ void __launch_bounds__(256)
-tc_bwd_scan_kernel(Problem p, Gates g, const float* __restrict__ U, const float* __restrict__ u,
-                   __nv_bfloat16* __restrict__ Gb, float* __restrict__ g_states,
-                   float* __restrict__ dC0) {
-  const int bh = blockIdx.y, NC = p.NC, DK = p.DK, DV = p.DV;
-  const long idx = (long)blockIdx.x * blockDim.x + threadIdx.x;
-  const long n_st = (long)DK * DV / 8;
-  const float* gt = g.gtot + (long)bh * NC;
-  const float* mc = g.mchk + (long)bh * (NC + 1);
-  if (idx < n_st) {
-    const int dk = (int)(idx * 8 / DV), c = (int)(idx * 8 % DV);
-    const int vb = c / 64, j = (c % 64) / 8, n_vb = DV / 64;
-    const size_t pos = (size_t)((j ^ (dk & 7)) * 8);
-    float G[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    *reinterpret_cast<uint4*>(Gb + cb_block_row((long)bh * (NC + 1) + NC, vb, dk, DK, n_vb) + pos) =
-        make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll 2
-    for (int k = NC - 1; k >= 0; --k) {
-      const float decay = expf(gt[k] + mc[k] - mc[k + 1]);
-      const float4* src = reinterpret_cast<const float4*>(U + (((long)bh * NC + k) * DK + dk) * DV + c);
-      const float4 x0 = src[0], x1 = src[1];
-      G[0] = fmaf(decay, G[0], x0.x);
-      G[1] = fmaf(decay, G[1], x0.y);
-      G[2] = fmaf(decay, G[2], x0.z);
-      G[3] = fmaf(decay, G[3], x0.w);
-      G[4] = fmaf(decay, G[4], x1.x);
-      G[5] = fmaf(decay, G[5], x1.y);
-      G[6] = fmaf(decay, G[6], x1.z);
-      G[7] = fmaf(decay, G[7], x1.w);
-      *reinterpret_cast<uint4*>(Gb + cb_block_row((long)bh * (NC + 1) + k, vb, dk, DK, n_vb) + pos) =
-          make_uint4(pack_bf16x2(G[0], G[1]), pack_bf16x2(G[2], G[3]), pack_bf16x2(G[4], G[5]),
-                     pack_bf16x2(G[6], G[7]));
+// Reverse recurrence on tcgen05: one CTA per (b, h) and 128 x 128 tile of
+// the [d_qk, d_v] gradient state, walking the chunks from the last,
+//
+//   G~_k = e^{g_k + m_k - m_{k+1}} G~_{k+1} + Q_k^T dUr_k,   G~_NC = 0,
+//
+// with the running G~ as a TMEM accumulator (dUr: du~ with rows scaled by
+// e^{m_k - mu_t}).  Per chunk the epilogue warps read G~_{k+1}, store it as
+// the bf16 operand copy Gb (block layout of cb_block_row, index
+// bh (NC + 1) + k + 1) and write it back times the decay; the chunk's two
+// MMAs then accumulate onto it.  G~_0 also goes to dC0 in fp32.
+// The CTAs of the first column tile carry g~ along (one row per thread) from
+// the increments u.  Roles and ring as tc_bwd_kernel.
+__global__ void __launch_bounds__(kThreads, 2)
+tc_bwd_rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_dur,
+                  Problem p, Gates g, const float* __restrict__ u, __nv_bfloat16* __restrict__ Gb,
+                  float* __restrict__ g_states, float* __restrict__ dC0) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar_full = sbase + kOffBar, bar_empty = bar_full + 8 * kStages;
+  const uint32_t bar_acc = bar_full + 16 * kStages, bar_master = bar_acc + 8;
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + kOffSlot);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int NC = p.NC, DK = p.DK, DV = p.DV, bh = blockIdx.y;
+  const int n_ct = DV / 128;
+  const int m0 = (blockIdx.x / n_ct) * 128, n0 = (blockIdx.x % n_ct) * 128;
+  const int nS = 2 * NC;  // two 64-token slabs per chunk, chunks from the last
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(bar_full + 8 * i, 1);
+      mbar_init(bar_empty + 8 * i, 1);
     }
-    float4* d4 = reinterpret_cast<float4*>(dC0 + ((long)bh * DK + dk) * DV + c);
-    d4[0] = make_float4(G[0], G[1], G[2], G[3]);
-    d4[1] = make_float4(G[4], G[5], G[6], G[7]);
-  } else if (idx < n_st + DK) {
-    const int d = (int)(idx - n_st);
+    mbar_init(bar_acc, 1);
+    mbar_init(bar_master, 128);
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32((const void*)tmem_slot), 128);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_dur);
+      bool ok = true;
+      int issued = 0;
+      for (int i = 0; i < nS && ok; ++i) {
+        const int s = i % kStages, uu = i / kStages;
+        if (uu > 0) ok = mbar_wait(bar_empty + 8 * s, (uu - 1) & 1, p, 6);
+        if (!ok) break;
+        const int t = (NC - 1 - i / 2) * kBT + (i & 1) * 64;
+        const uint32_t sa = sbase + (uint32_t)s * kStageBytes, sb = sa + kTileBytes;
+        const uint32_t fb = bar_full + 8 * s;
+        mbar_expect_tx(fb, 2 * kTileBytes);
+        // A = Q^T (rows d, MN-major), B = dUr (columns c, MN-major); K = tokens
+        tma_load_3d(sa, &tm_q, m0, t, bh, fb);
+        tma_load_3d(sa + 8192, &tm_q, m0 + 64, t, bh, fb);
+        tma_load_3d(sb, &tm_dur, n0, t, bh, fb);
+        tma_load_3d(sb + 8192, &tm_dur, n0 + 64, t, bh, fb);
+        issued = i + 1;
+      }
+      for (int q = (issued > kStages ? issued - kStages : 0); q < issued; ++q)
+        mbar_wait(bar_full + 8 * (q % kStages), (q / kStages) & 1, p, 7);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16(128, 128, 1, 1);
+      bool ok = true;
+      for (int kk = 0; kk < NC && ok; ++kk) {
+        // the epilogue has scaled the running state by this chunk's decay
+        ok = mbar_wait(bar_master, kk & 1, p, 8);
+        if (!ok) break;
+        tc_fence_after();
+        for (int h = 0; h < 2 && ok; ++h) {
+          const int i = 2 * kk + h, s = i % kStages;
+          ok = mbar_wait(bar_full + 8 * s, (i / kStages) & 1, p, 9);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t sa = sbase + (uint32_t)s * kStageBytes, sb = sa + kTileBytes;
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            mma_bf16_ss(tmem, sdesc_sw128(sa + q * 2048, 8192, 1024),
+                        sdesc_sw128(sb + q * 2048, 8192, 1024), idesc,
+                        (kk == 0 && h == 0 && q == 0) ? 0u : 1u);
+          mma_commit(bar_empty + 8 * s);
+        }
+        mma_commit(bar_acc);
+      }
+    }
+  } else {
+    const int q4 = warp & 3, r = q4 * 32 + lane, d = m0 + r;
+    const uint32_t trow = tmem + ((uint32_t)(q4 * 32) << 16);
+    const float* gt = g.gtot + (long)bh * NC;
+    const float* mc = g.mchk + (long)bh * (NC + 1);
+    const int n_vb = DV / 64;
+    const bool g_owner = n0 == 0;
     float gv = 0.f;
-    g_states[((long)bh * (NC + 1) + NC) * DK + d] = 0.f;
-    for (int k = NC - 1; k >= 0; --k) {
-      gv = fmaf(expf(gt[k] + mc[k] - mc[k + 1]), gv, u[((long)bh * NC + k) * DK + d]);
-      g_states[((long)bh * (NC + 1) + k) * DK + d] = gv;
+    // row d, columns n0 + c*32 .. +31 of G~ (index kidx) as bf16
+    auto store_b16 = [&](long kidx, int c, const uint32_t (&v)[32]) {
+      const int col = n0 + c * 32;
+      __nv_bfloat16* row = Gb + cb_block_row((long)bh * (NC + 1) + kidx, col / 64, d, DK, n_vb);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int j = (col % 64) / 8 + q;
+        *reinterpret_cast<uint4*>(row + ((j ^ (d & 7)) * 8)) = make_uint4(
+            pack_bf16x2(__uint_as_float(v[8 * q]), __uint_as_float(v[8 * q + 1])),
+            pack_bf16x2(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3])),
+            pack_bf16x2(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5])),
+            pack_bf16x2(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7])));
+      }
+    };
+    bool ok = true;
+    for (int kk = 0; kk < NC; ++kk) {
+      const int k = NC - 1 - kk;
+      const float decay = expf(gt[k] + mc[k] - mc[k + 1]);
+      if (kk == 0) {
+        // G~_NC = 0: nothing in TMEM yet (the first MMA overwrites)
+        uint32_t z[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) z[j] = 0u;
+        tc_fence_before();
+        mbar_arrive(bar_master);
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) store_b16(NC, c, z);
+      } else {
+        ok = ok && mbar_wait(bar_acc, (kk - 1) & 1, p, 10);
+        tc_fence_after();
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t v[32];
+          tmem_ld32(trow + c * 32, v);
+          tmem_wait_ld();
+          store_b16(k + 1, c, v);  // G~_{k+1}
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(decay * __uint_as_float(v[j]));
+          tmem_st32(trow + c * 32, v);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar_master);
+      }
+      if (g_owner) {
+        g_states[((long)bh * (NC + 1) + k + 1) * DK + d] = gv;
+        gv = fmaf(decay, gv, u[((long)bh * NC + k) * DK + d]);
+      }
     }
+    // G~_0
+    ok = ok && mbar_wait(bar_acc, (NC - 1) & 1, p, 11);
+    tc_fence_after();
+    if (g_owner) g_states[(long)bh * (NC + 1) * DK + d] = gv;
+#pragma unroll 1
+    for (int c = 0; c < 4; ++c) {
+      uint32_t v[32];
+      tmem_ld32(trow + c * 32, v);
+      tmem_wait_ld();
+      store_b16(0, c, v);
+      float4* dst = reinterpret_cast<float4*>(dC0 + ((long)bh * DK + d) * DV + n0 + c * 32);
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        dst[q] = make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
+                             __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3]));
+    }
+    (void)ok;
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    if (lane == 0) mbar_wait(bar_acc, (NC - 1) & 1, p, 12);
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 128);
   }
 }
 
@@ -479,30 +602,21 @@ bool tc_bwd_supported(const Problem& pb) {
 size_t tc_bwd_square_elems(const Problem& pb) { return (size_t)pb.BH * pb.NC * 2 * kBT * kBT; }
 
 cudaError_t launch_tc_bwd_states(const Problem& pb, const void* Q, const __nv_bfloat16* dUr16,
-                                 Gates g, const float* dA, float* U, float* u,
-                                 __nv_bfloat16* Gb, float* g_states, float* dC0,
-                                 cudaStream_t st) {
+                                 Gates g, const float* dA, float* u, __nv_bfloat16* Gb,
+                                 float* g_states, float* dC0, cudaStream_t st) {
   if (!tc_bwd_supported(pb)) return cudaErrorNotSupported;
-  CUtensorMap m[4];
-  if (!encode_tmap_3d(&m[0], Q, 2, pb.DK, pb.T, pb.BH, 64, 64, 128) ||
-      !encode_tmap_3d(&m[3], dUr16, 2, pb.DV, pb.T, pb.BH, 64, 64, 128))
+  CUtensorMap mq, mu;
+  if (!encode_tmap_3d(&mq, Q, 2, pb.DK, pb.T, pb.BH, 64, 64, 128) ||
+      !encode_tmap_3d(&mu, dUr16, 2, pb.DV, pb.T, pb.BH, 64, 64, 128))
     return cudaErrorInvalidValue;
-  m[1] = m[0];
-  m[2] = m[0];
-  TcBwdArgs a = {};
-  a.p = pb;
-  a.g = g;
-  a.U = U;
-  cudaError_t e =
-      launch_job<kU, 128>(m, a, dim3((pb.DK / 128) * (pb.DV / 128), pb.NC, pb.BH), st);
+  tc_bwd_gvec_kernel<<<dim3(pb.NC, pb.BH), 256, 0, st>>>(pb, g, static_cast<const __nv_bfloat16*>(Q),
+                                                         dA, u);
+  cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  tc_bwd_gvec_kernel<<<dim3(pb.NC, pb.BH), pb.DK, 0, st>>>(
-      pb, g, static_cast<const __nv_bfloat16*>(Q), dA, u);
-  e = cudaGetLastError();
+  e = cudaFuncSetAttribute(tc_bwd_rev_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
   if (e != cudaSuccess) return e;
-  const long n = (long)pb.DK * pb.DV / 8 + pb.DK;
-  tc_bwd_scan_kernel<<<dim3((unsigned)((n + 255) / 256), pb.BH), 256, 0, st>>>(pb, g, U, u, Gb,
-                                                                              g_states, dC0);
+  tc_bwd_rev_kernel<<<dim3((pb.DK / 128) * (pb.DV / 128), pb.BH), kThreads, kSmem, st>>>(
+      mq, mu, pb, g, u, Gb, g_states, dC0);
   return cudaGetLastError();
 }
 
