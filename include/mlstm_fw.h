@@ -159,18 +159,24 @@ mlstm_status mlstm_bw_workspace_size(int B, int NH, int T, int DK, int DV, int c
  * inter-chunk terms, and the gate gradients from the identities
  * dL/d log i_s = k_s . dk_s and dL/d log f_l = sum_{t >= l} (q_t . dq_t -
  * k_t . dk_t) ("Tiled Flash Linear Attention: More Efficient Linear RNN and
- * xLSTM Kernels": the chunkwise split applied to the gradient).  The
- * recomputed forward runs on the tensor cores for bf16 inputs where the TC
- * algorithm supports the shape (else on the fp32 kernels); the gradient
- * kernels are fp32 CUDA-core kernels for both input types.  The derivation
- * and its stabilisation are in the header of the implementation file.
+ * xLSTM Kernels": the chunkwise split applied to the gradient).
+ * Two paths.  bf16 inputs with DK of 128 or 256, a DV the tensor-core forward
+ * takes (128, or a multiple of 256 up to 1024) and T >= 128: the whole
+ * backward runs on tensor cores in 128-token chunks whatever chunk_size says
+ * (the gradients do not depend on the chunking, up to rounding); the
+ * recomputed forward, the reverse state recurrence and the gradient GEMMs
+ * use bf16 operands with fp32 accumulation.  Everything else: fp32 CUDA-core
+ * gradient kernels on chunk_size (the forward recomputed on the tensor cores
+ * for bf16 shapes the TC algorithm supports).  The derivation and its
+ * stabilisation are in the header of the implementation files (bwd.cu,
+ * tc_bwd.cu).
  *   Q, K, V, dH in `dtype` as in mlstm_fw; dQ, dK, dV out, same shapes and
  *   dtype; di_pre, df_pre [B, NH, T] fp32 out; C0/n0/m0 all given or all
  *   null; dC0 [B, NH, DK, DV], dn0 [B, NH, DK], dm0 [B, NH] fp32 out
  *   (nullable; zero-state calls get the gradient a zero initial state would
  *   have).  The loss is on H only (no gradient arrives through C_T/n_T/m_T).
  * Errors as mlstm_fw; the workspace must hold mlstm_bw_workspace_size bytes.
- * 10 to 13 launches, asynchronous on `stream`. */
+ * 10 to 14 launches, asynchronous on `stream`. */
 mlstm_status mlstm_bw(const void* Q, const void* K, const void* V, const float* i_pre,
                       const float* f_pre, const float* C0, const float* n0, const float* m0,
                       const void* dH, void* dQ, void* dK, void* dV, float* di_pre, float* df_pre,

@@ -21,7 +21,7 @@
 //
 // The reverse states G~_k = e^{g_k + m_k - m_{k+1}} G~_{k+1} + Q_k^T dUr_k
 // (dUr: a bf16 copy of du~ whose rows carry e^{m_k - mu_t}) run in
-// tc_bwd_rev_kernel: a CTA per 128 x 128 tile of the state keeps the running
+// tc_bwd_rev_kernel: a CTA per 128 x 256 (or 128) tile of the state keeps the running
 // G~ in TMEM and walks the chunks from the last, writing every G~_k as the
 // bf16 operand copy (and G~_0 in fp32: the gradient of the initial state);
 // g~ follows from the per-chunk sums of e^{m_k - mu_t} da~_t q_t.
@@ -400,47 +400,70 @@ tc_bwd_gvec_kernel(Problem p, Gates g, const __nv_bfloat16* __restrict__ Q,
   }
 }
 
-// Reverse recurrence on tcgen05: one CTA per (b, h) and 128 x 128 tile of
-// the [d_qk, d_v] gradient state, walking the chunks from the last,
+// Reverse recurrence on tcgen05: one CTA per (b, h) and 128 x NT tile of
+// the [d_qk, d_v] gradient state (NT = 256 where d_v allows, else 128),
+// walking the chunks from the last,
 //
 //   G~_k = e^{g_k + m_k - m_{k+1}} G~_{k+1} + Q_k^T dUr_k,   G~_NC = 0,
 //
 // with the running G~ as a TMEM accumulator (dUr: du~ with rows scaled by
-// e^{m_k - mu_t}).  Per chunk the epilogue warps read G~_{k+1}, store it as
-// the bf16 operand copy Gb (block layout of cb_block_row, index
-// bh (NC + 1) + k + 1) and write it back times the decay; the chunk's two
-// MMAs then accumulate onto it.  G~_0 also goes to dC0 in fp32.
-// The CTAs of the first column tile carry g~ along (one row per thread) from
-// the increments u.  Roles and ring as tc_bwd_kernel.
-__global__ void __launch_bounds__(kThreads, 2)
+// e^{m_k - mu_t}).  Per chunk the epilogue warps read G~_{k+1} 32 columns at
+// a time, store it as the bf16 operand copy Gb (block layout of
+// cb_block_row, index bh (NC + 1) + k + 1) and write it back times the
+// decay; the chunk's two MMAs then accumulate onto it.  G~_0 also goes to
+// dC0 in fp32.  The chunk
+// steps are sequential, so each CTA takes a wide tile and eight epilogue
+// warps (two per TMEM lane quadrant, each half of the columns) to spread the
+// fixed cost of a step (the TMEM round trip and the MMA hand-off) over more
+// of the state.  The CTAs of the first column tile carry g~ along (one row
+// per thread of the first column half) from the increments u.
+// Roles (320 threads): warp 0 producer, warp 1 TMEM owner and MMA issuer,
+// warps 2..9 epilogue; ring of 64-token stages (A = Q^T 16 KB, B = dUr
+// NT x 128 bytes), 96 KB in all, two CTAs per SM.
+constexpr int kRevThreads = 320;
+template <int NT>
+struct RevCfg {
+  static constexpr uint32_t kBBytes = NT * 128;
+  static constexpr uint32_t kStageBytes = kTileBytes + kBBytes;
+  static constexpr int kStages = NT == 256 ? 2 : 3;
+  static constexpr uint32_t kOffBar = kStages * kStageBytes;
+  static constexpr uint32_t kOffSlot = kOffBar + 8 * 8;
+  static constexpr uint32_t kSmem = kOffSlot + 16 + 1024;
+  static constexpr int kCols = NT / 2;  // columns per epilogue thread
+};
+
+template <int NT>
+__global__ void __launch_bounds__(kRevThreads, 2)
 tc_bwd_rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_dur,
                   Problem p, Gates g, const float* __restrict__ u, __nv_bfloat16* __restrict__ Gb,
                   float* __restrict__ g_states, float* __restrict__ dC0) {
+  using R = RevCfg<NT>;
+  constexpr int kSt = R::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
-  const uint32_t bar_full = sbase + kOffBar, bar_empty = bar_full + 8 * kStages;
-  const uint32_t bar_acc = bar_full + 16 * kStages, bar_master = bar_acc + 8;
-  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + kOffSlot);
+  const uint32_t bar_full = sbase + R::kOffBar, bar_empty = bar_full + 8 * kSt;
+  const uint32_t bar_acc = bar_full + 16 * kSt, bar_master = bar_acc + 8;
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + R::kOffSlot);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int NC = p.NC, DK = p.DK, DV = p.DV, bh = blockIdx.y;
-  const int n_ct = DV / 128;
-  const int m0 = (blockIdx.x / n_ct) * 128, n0 = (blockIdx.x % n_ct) * 128;
+  const int n_ct = DV / NT;
+  const int m0 = (blockIdx.x / n_ct) * 128, n0 = (blockIdx.x % n_ct) * NT;
   const int nS = 2 * NC;  // two 64-token slabs per chunk, chunks from the last
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kStages; ++i) {
+    for (int i = 0; i < kSt; ++i) {
       mbar_init(bar_full + 8 * i, 1);
       mbar_init(bar_empty + 8 * i, 1);
     }
     mbar_init(bar_acc, 1);
-    mbar_init(bar_master, 128);
+    mbar_init(bar_master, kRevThreads - 64);
     fence_barrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32((const void*)tmem_slot), 128);
+    tmem_alloc(smem_u32((const void*)tmem_slot), NT);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -455,26 +478,26 @@ tc_bwd_rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       bool ok = true;
       int issued = 0;
       for (int i = 0; i < nS && ok; ++i) {
-        const int s = i % kStages, uu = i / kStages;
+        const int s = i % kSt, uu = i / kSt;
         if (uu > 0) ok = mbar_wait(bar_empty + 8 * s, (uu - 1) & 1, p, 6);
         if (!ok) break;
         const int t = (NC - 1 - i / 2) * kBT + (i & 1) * 64;
-        const uint32_t sa = sbase + (uint32_t)s * kStageBytes, sb = sa + kTileBytes;
+        const uint32_t sa = sbase + (uint32_t)s * R::kStageBytes, sb = sa + kTileBytes;
         const uint32_t fb = bar_full + 8 * s;
-        mbar_expect_tx(fb, 2 * kTileBytes);
+        mbar_expect_tx(fb, R::kStageBytes);
         // A = Q^T (rows d, MN-major), B = dUr (columns c, MN-major); K = tokens
         tma_load_3d(sa, &tm_q, m0, t, bh, fb);
         tma_load_3d(sa + 8192, &tm_q, m0 + 64, t, bh, fb);
-        tma_load_3d(sb, &tm_dur, n0, t, bh, fb);
-        tma_load_3d(sb + 8192, &tm_dur, n0 + 64, t, bh, fb);
+#pragma unroll
+        for (int b = 0; b < NT / 64; ++b) tma_load_3d(sb + b * 8192, &tm_dur, n0 + b * 64, t, bh, fb);
         issued = i + 1;
       }
-      for (int q = (issued > kStages ? issued - kStages : 0); q < issued; ++q)
-        mbar_wait(bar_full + 8 * (q % kStages), (q / kStages) & 1, p, 7);
+      for (int q = (issued > kSt ? issued - kSt : 0); q < issued; ++q)
+        mbar_wait(bar_full + 8 * (q % kSt), (q / kSt) & 1, p, 7);
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16(128, 128, 1, 1);
+      constexpr uint32_t idesc = idesc_bf16(128, NT, 1, 1);
       bool ok = true;
       for (int kk = 0; kk < NC && ok; ++kk) {
         // the epilogue has scaled the running state by this chunk's decay
@@ -482,11 +505,11 @@ tc_bwd_rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         if (!ok) break;
         tc_fence_after();
         for (int h = 0; h < 2 && ok; ++h) {
-          const int i = 2 * kk + h, s = i % kStages;
-          ok = mbar_wait(bar_full + 8 * s, (i / kStages) & 1, p, 9);
+          const int i = 2 * kk + h, s = i % kSt;
+          ok = mbar_wait(bar_full + 8 * s, (i / kSt) & 1, p, 9);
           if (!ok) break;
           tc_fence_after();
-          const uint32_t sa = sbase + (uint32_t)s * kStageBytes, sb = sa + kTileBytes;
+          const uint32_t sa = sbase + (uint32_t)s * R::kStageBytes, sb = sa + kTileBytes;
 #pragma unroll
           for (int q = 0; q < 4; ++q)
             mma_bf16_ss(tmem, sdesc_sw128(sa + q * 2048, 8192, 1024),
@@ -499,15 +522,17 @@ tc_bwd_rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     }
   } else {
     const int q4 = warp & 3, r = q4 * 32 + lane, d = m0 + r;
-    const uint32_t trow = tmem + ((uint32_t)(q4 * 32) << 16);
+    const int ch = (warp - 2) >> 2;  // column half
+    const int c0 = ch * R::kCols;    // first column of this thread within the tile
+    const uint32_t trow = tmem + ((uint32_t)(q4 * 32) << 16) + (uint32_t)c0;
     const float* gt = g.gtot + (long)bh * NC;
     const float* mc = g.mchk + (long)bh * (NC + 1);
     const int n_vb = DV / 64;
-    const bool g_owner = n0 == 0;
+    const bool g_owner = n0 == 0 && ch == 0;
     float gv = 0.f;
-    // row d, columns n0 + c*32 .. +31 of G~ (index kidx) as bf16
+    // row d, tile columns c0 + c*32 .. +31 of G~ (index kidx) as bf16
     auto store_b16 = [&](long kidx, int c, const uint32_t (&v)[32]) {
-      const int col = n0 + c * 32;
+      const int col = n0 + c0 + c * 32;
       __nv_bfloat16* row = Gb + cb_block_row((long)bh * (NC + 1) + kidx, col / 64, d, DK, n_vb);
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
@@ -519,24 +544,28 @@ tc_bwd_rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             pack_bf16x2(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7])));
       }
     };
+    constexpr int kG = R::kCols / 32;  // 32-column groups per thread
     bool ok = true;
+    float decay = expf(gt[NC - 1] + mc[NC - 1] - mc[NC]);
     for (int kk = 0; kk < NC; ++kk) {
       const int k = NC - 1 - kk;
-      const float decay = expf(gt[k] + mc[k] - mc[k + 1]);
+      // next chunk's decay and this chunk's g~ increment, loaded ahead of the wait
+      const float decay_next = k > 0 ? expf(gt[k - 1] + mc[k - 1] - mc[k]) : 0.f;
+      const float uk = g_owner ? u[((long)bh * NC + k) * DK + d] : 0.f;
       if (kk == 0) {
         // G~_NC = 0: nothing in TMEM yet (the first MMA overwrites)
+        tc_fence_before();
+        mbar_arrive(bar_master);
         uint32_t z[32];
 #pragma unroll
         for (int j = 0; j < 32; ++j) z[j] = 0u;
-        tc_fence_before();
-        mbar_arrive(bar_master);
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) store_b16(NC, c, z);
+#pragma unroll
+        for (int c = 0; c < kG; ++c) store_b16(NC, c, z);
       } else {
         ok = ok && mbar_wait(bar_acc, (kk - 1) & 1, p, 10);
         tc_fence_after();
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < kG; ++c) {
           uint32_t v[32];
           tmem_ld32(trow + c * 32, v);
           tmem_wait_ld();
@@ -551,20 +580,21 @@ tc_bwd_rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       }
       if (g_owner) {
         g_states[((long)bh * (NC + 1) + k + 1) * DK + d] = gv;
-        gv = fmaf(decay, gv, u[((long)bh * NC + k) * DK + d]);
+        gv = fmaf(decay, gv, uk);
       }
+      decay = decay_next;
     }
     // G~_0
     ok = ok && mbar_wait(bar_acc, (NC - 1) & 1, p, 11);
     tc_fence_after();
     if (g_owner) g_states[(long)bh * (NC + 1) * DK + d] = gv;
 #pragma unroll 1
-    for (int c = 0; c < 4; ++c) {
+    for (int c = 0; c < kG; ++c) {
       uint32_t v[32];
       tmem_ld32(trow + c * 32, v);
       tmem_wait_ld();
       store_b16(0, c, v);
-      float4* dst = reinterpret_cast<float4*>(dC0 + ((long)bh * DK + d) * DV + n0 + c * 32);
+      float4* dst = reinterpret_cast<float4*>(dC0 + ((long)bh * DK + d) * DV + n0 + c0 + c * 32);
 #pragma unroll
       for (int q = 0; q < 8; ++q)
         dst[q] = make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
@@ -579,8 +609,21 @@ tc_bwd_rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     if (lane == 0) mbar_wait(bar_acc, (NC - 1) & 1, p, 12);
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem, 128);
+    tmem_dealloc(tmem, NT);
   }
+}
+
+template <int NT>
+cudaError_t launch_rev(const CUtensorMap& mq, const CUtensorMap& mu, const Problem& pb, Gates g,
+                       const float* u, __nv_bfloat16* Gb, float* g_states, float* dC0,
+                       cudaStream_t st) {
+  using R = RevCfg<NT>;
+  cudaError_t e = cudaFuncSetAttribute(tc_bwd_rev_kernel<NT>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, R::kSmem);
+  if (e != cudaSuccess) return e;
+  tc_bwd_rev_kernel<NT><<<dim3((pb.DK / 128) * (pb.DV / NT), pb.BH), kRevThreads, R::kSmem, st>>>(
+      mq, mu, pb, g, u, Gb, g_states, dC0);
+  return cudaGetLastError();
 }
 
 template <int kJob, int NT>
@@ -613,11 +656,7 @@ cudaError_t launch_tc_bwd_states(const Problem& pb, const void* Q, const __nv_bf
                                                          dA, u);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(tc_bwd_rev_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
-  if (e != cudaSuccess) return e;
-  tc_bwd_rev_kernel<<<dim3((pb.DK / 128) * (pb.DV / 128), pb.BH), kThreads, kSmem, st>>>(
-      mq, mu, pb, g, u, Gb, g_states, dC0);
-  return cudaGetLastError();
+  return launch_rev<128>(mq, mu, pb, g, u, Gb, g_states, dC0, st);
 }
 
 cudaError_t launch_tc_bwd(const Problem& pb, const void* Q, const void* K, const void* V,
