@@ -51,6 +51,7 @@
 
 #include "common.cuh"
 #include "tc.h"
+#include "tc_bwd.h"
 
 namespace mlstm {
 namespace {

@@ -42,6 +42,7 @@
 #include <cuda.h>
 
 #include "tc.h"
+#include "tc_bwd.h"
 #include "tc_ptx.cuh"
 
 namespace mlstm {
