@@ -33,6 +33,7 @@ CASES = [
     (1, 1, 2048, 128, 128, 256, "bf16", "sigmoid", True),  # one head: segmented recurrences
     (1, 2, 130, 128, 128, 128, "bf16", "exp", True),    # a 2-token last chunk
     (2, 1, 100, 128, 128, 128, "bf16", "exp", True),    # shorter than a chunk: fp32 kernels
+    (1, 2, 300, 256, 256, 512, "bf16", "sigmoid", True),  # d_qk 256 x d_v 256, ragged
 ]
 
 
@@ -68,6 +69,31 @@ def test_backward_matches_autograd_oracle(case):
     errs = _errors(ref, got)
     bad = {k: v for k, v in errs.items() if not v <= TOL[w.dtype]}
     assert not bad, f"{case}: {errs}"
+
+
+@pytest.mark.parametrize("gates", [(4.0, -3.0, 6.0), (-6.0, 0.0, 2.0)],
+                         ids=["big-input-strong-forget", "small-input-fast-forget"])
+def test_tensor_core_backward_extreme_gates(gates):
+    """Tensor-core backward (bf16, 128-token chunks) with gate statistics far
+    from the workloads': i_pre ~ N(mu, 1) with mu = 4 (inputs that dominate the
+    stabiliser inside a chunk) or -6, f_pre ~ U(lo, hi) reaching strong
+    forgetting (f~ = -3: f = 0.05 per token)."""
+    mu, lo, hi = gates
+    w = WORKLOADS["mid"].replace(name="bw_gates", B=1, NH=3, T=384, DK=128, DV=256,
+                                 chunk_size=128, dtype="bf16", gate_mode="exp",
+                                 init_state=True, i_mean=mu, f_low=lo, f_high=hi)
+    x = make_inputs(w, seed=31)
+    g = torch.Generator().manual_seed(32)
+    dH = torch.randn((w.B, w.NH, w.T, w.DV), generator=g).to(w.torch_dtype)
+    ref = ob.gradients(x, dH, w.gate_mode)
+    d = parity.to_dev(x)
+    got = api.mlstm_bw(d["Q"], d["K"], d["V"], d["i_pre"], d["f_pre"], dH.cuda(), d["C0"],
+                       d["n0"], d["m0"], chunk_size=w.chunk_size, gate_mode=w.gate_mode)
+    torch.cuda.synchronize()
+    assert api.last_device_error() == _lib.OK
+    errs = _errors(ref, got)
+    bad = {k: v for k, v in errs.items() if not v <= TOL["bf16"]}
+    assert not bad, f"{gates}: {errs}"
 
 
 def test_backward_chunk_size_invariance():
