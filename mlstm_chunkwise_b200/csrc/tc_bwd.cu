@@ -427,9 +427,10 @@ struct RevCfg {
   static constexpr uint32_t kBBytes = NT * 128;
   static constexpr uint32_t kStageBytes = kTileBytes + kBBytes;
   static constexpr int kStages = NT == 256 ? 2 : 3;
-  static constexpr uint32_t kOffBar = kStages * kStageBytes;
-  static constexpr uint32_t kOffSlot = kOffBar + 8 * 8;
+  static constexpr uint32_t kOffBar = kStages * kStageBytes;  // full, empty, acc, master
+  static constexpr uint32_t kOffSlot = kOffBar + 8 * (2 * kStages + 2);
   static constexpr uint32_t kSmem = kOffSlot + 16 + 1024;
+  static_assert(kSmem <= 227 * 1024, "shared memory");
   static constexpr int kCols = NT / 2;  // columns per epilogue thread
 };
 
