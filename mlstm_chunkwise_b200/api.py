@@ -140,7 +140,9 @@ def mlstm_bw(Q, K, V, i_pre, f_pre, dH, C0=None, n0=None, m0=None, *, chunk_size
 
     Inputs as ``mlstm_fw``.  Returns a dict with dQ, dK, dV (input dtype),
     di_pre, df_pre [B,NH,T] and, when an initial state is given, dC0, dn0,
-    dm0 (float32).
+    dm0 (float32).  bf16 inputs with d_qk of 128 or 256 (a d_v the tensor-core
+    forward takes, T >= 128) run on the tensor cores in 128-token chunks,
+    whatever ``chunk_size`` is; everything else on fp32 CUDA-core kernels.
     """
     B, NH, T, DK, DV, dev, dt = _check_common(Q, K, V, i_pre, f_pre)
     _check_state(C0, n0, m0, B, NH, DK, DV, dev)
