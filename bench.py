@@ -17,6 +17,10 @@ the fp64 CPU oracle timed on a bounded sample of the same workload.
 
 ``--impl reference`` times that oracle alone on the host cores (the only
 other place this script runs it), on the same workload and metric.
+
+``--op step | bw | train`` measure, on one GPU, the single-token step, the
+backward pass (forward recomputed inside it) and a whole training step
+(forward + backward through the autograd Function) instead.
 """
 from __future__ import annotations
 
@@ -800,6 +804,81 @@ def run_bw(args):
     return 0
 
 
+# ----------------------------------------------------------------------------
+# training step: forward + backward through the autograd Function
+# ----------------------------------------------------------------------------
+TRAIN_METRIC = "mLSTM training step tokens/s (forward + backward through torch.autograd)"
+
+
+def run_train(args):
+    """One training step of the layer: mlstm_chunkwise forward, a loss
+    sum(H * G) with a fixed G, and loss.backward() into every input's .grad
+    (the backward recomputes the forward from the inputs).  Timed with CUDA
+    events around whole steps on one GPU."""
+    import torch
+
+    from mlstm_chunkwise_b200 import _lib, api
+    from mlstm_chunkwise_b200 import build as libbuild
+    from mlstm_chunkwise_b200.inputs import make_inputs
+
+    if libbuild.needs_build():
+        libbuild.build()
+    if int(os.environ.get("WORLD_SIZE", "1")) != 1 or args.gpus != 1:
+        raise SystemExit("--op train runs on one GPU")
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    w = pick_workload(args.workload)
+    if args.batch:
+        w = w.replace(name=f"{w.name}_B{args.batch}", B=args.batch)
+    x = make_inputs(w, seed=rank_seed(w, 0))
+    leaves = {k: v.to(dev).requires_grad_(True) for k, v in x.items() if v is not None}
+    G = torch.randn((w.B, w.NH, w.T, w.DV), generator=torch.Generator().manual_seed(7)).to(
+        w.torch_dtype).to(dev)
+
+    def step():
+        for v in leaves.values():
+            v.grad = None
+        H, _ = api.mlstm_chunkwise(leaves["Q"], leaves["K"], leaves["V"], leaves["i_pre"],
+                                   leaves["f_pre"], leaves.get("C0"), leaves.get("n0"),
+                                   leaves.get("m0"), chunk_size=w.chunk_size,
+                                   gate_mode=w.gate_mode)
+        H.backward(G)
+
+    warm = max(3, args.warmup)
+    for _ in range(warm):
+        step()
+    torch.cuda.synchronize()
+    lib = _lib.lib()
+    sampler = ClockSampler(0)
+    sampler.start()
+    stream = torch.cuda.current_stream(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    launches0 = lib.mlstm_kernel_launches()
+    t_host0 = time.perf_counter()
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    t_host1 = time.perf_counter()
+    launches = lib.mlstm_kernel_launches() - launches0
+    sampler.stop()
+    st = api.last_device_error(dev)
+    if st != _lib.OK:
+        raise SystemExit(f"device error in the timed region: {_lib.status_string(st)}")
+    ms = e0.elapsed_time(e1) / args.steps
+    line = {
+        "metric": TRAIN_METRIC, "value": w.B * w.T / (ms / 1e3), "unit": "tokens/s",
+        "n_gpus": 1, "steps": args.steps, "warmup": warm, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
+        "data": "synthetic", "config": workload_config(w, "mlstm_chunkwise (fw + bw)"),
+        "roofline": None, "gpu_launches": int(launches), "e2e": None,
+        "clocks": sampler.summary(t_host0, t_host1),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -814,9 +893,9 @@ def main():
                     help="skip the host-buffer end-to-end loop (profiling runs)")
     ap.add_argument("--batch", type=int, default=0,
                     help="override the workload's batch size (smaller profiling captures)")
-    ap.add_argument("--op", default="fw", choices=["fw", "step", "bw"],
+    ap.add_argument("--op", default="fw", choices=["fw", "step", "bw", "train"],
                     help="fw: the forward pass (default); step: the single-token step; "
-                         "bw: the backward pass")
+                         "bw: the backward pass; train: forward + backward through autograd")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -824,6 +903,8 @@ def main():
         return run_reference(args)
     if args.op == "step":
         return run_step(args)
+    if args.op == "train":
+        return run_train(args)
     if args.op == "bw":
         return run_bw(args)
     return run_ours(args)
