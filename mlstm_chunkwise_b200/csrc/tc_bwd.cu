@@ -250,8 +250,14 @@ tc_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     const float m_out = a.g.mchk[(long)bh * (NC + 1) + k + 1];
     const float acol_r = a.g.acol[(long)bh * tpad + t];  // -inf on padding
     const float mu = fmaxf(m_in, a.g.amax[(long)bh * tpad + t]);
+    // per-column vector of the chunk in shared memory: the squares' column
+    // weights acol_s; dq's n_k, dk's g~_{k+1} over this CTA's NT columns
     if constexpr (kJob == kSquares) {
       vec[r] = acol_r;
+      named_bar_sync(1, 128);
+    } else if constexpr (kJob == kDQ || kJob == kDK) {
+      if (r < NT)
+        vec[r] = kJob == kDQ ? a.n_states[bhk * DK + n0 + r] : a.g_states[bhk1 * DK + n0 + r];
       named_bar_sync(1, 128);
     }
     const bool ok = mbar_wait(bar_acc, 0, p, 4);
@@ -288,11 +294,9 @@ tc_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       } else {
         const int D = kJob == kDV ? DV : DK;
         float rs, alpha = 0.f, s1, s2;
-        const float* beta = nullptr;
         if constexpr (kJob == kDQ) {
           rs = expf(m_in - mu);
           alpha = valid ? a.dA[(long)bh * T + t] : 0.f;
-          beta = a.n_states + bhk * DK;
           s1 = p.key_scale;
           s2 = 1.f;
         } else {
@@ -300,7 +304,6 @@ tc_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
           rs = expf(gk + acol_r - m_out);  // w_s, 0 on padding
           if constexpr (kJob == kDK) {
             alpha = 1.f;
-            beta = a.g_states + bhk1 * DK;
             s1 = p.key_scale;
             s2 = p.key_scale;
           } else {
@@ -312,6 +315,13 @@ tc_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         const long orow = ((long)bh * T + t) * D + n0;
 #pragma unroll 1
         for (int c = 0; c < NT / 32; ++c) {
+          // this row's q or k for the dot product, loaded ahead of the TMEM reads
+          uint4 xv[4];
+          if (kJob != kDV && valid) {
+            const uint4* xs = reinterpret_cast<const uint4*>(a.X + orow + c * 32);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) xv[u] = xs[u];
+          }
           uint32_t v1[32], v2[32];
           tmem_ld32(trow + c * 32, v1);
           tmem_ld32(trow + 128 + c * 32, v2);
@@ -320,7 +330,7 @@ tc_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             float x2 = __uint_as_float(v2[j]);
-            if (kJob != kDV) x2 = fmaf(alpha, beta[n0 + c * 32 + j], x2);
+            if (kJob != kDV) x2 = fmaf(alpha, vec[c * 32 + j], x2);
             // dq: s acc1 + rs (acc2 + da n);  dk: s (acc1 + w (acc2 + g~));  dv: acc1 + s w acc2
             o[j] = kJob == kDK ? s1 * fmaf(rs, x2, __uint_as_float(v1[j]))
                                : fmaf(s1, __uint_as_float(v1[j]), s2 * rs * x2);
@@ -334,11 +344,9 @@ tc_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                                   pack_bf16x2(o[8 * u + 4], o[8 * u + 5]),
                                   pack_bf16x2(o[8 * u + 6], o[8 * u + 7]));
             if constexpr (kJob != kDV) {
-              const uint4* xs = reinterpret_cast<const uint4*>(a.X + orow + c * 32);
 #pragma unroll
               for (int u = 0; u < 4; ++u) {
-                const uint4 xv = xs[u];
-                const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+                const uint32_t xw[4] = {xv[u].x, xv[u].y, xv[u].z, xv[u].w};
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                   const float2 f = __bfloat1622float2(
