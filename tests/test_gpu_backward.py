@@ -96,6 +96,51 @@ def test_tensor_core_backward_extreme_gates(gates):
     assert not bad, f"{gates}: {errs}"
 
 
+@pytest.mark.parametrize("name", ["xlstm7b", "sigmoid_long"])
+def test_backward_full_size_sampled_heads(name):
+    """The full workload shape through mlstm_bw (the launch configuration
+    `bench.py --op bw` times), with the upstream gradient nonzero only on the
+    first T1 tokens of two heads (the first and the last).  The loss then sees
+    nothing else, so those heads' gradients on their first T1 tokens (and of
+    their initial state) equal the oracle's on the truncated sequences, and
+    every other gradient is exactly zero: later tokens, and every other head."""
+    w = WORKLOADS[name]
+    T1 = 384
+    x = make_inputs(w)
+    heads = [(0, 0), (w.B - 1, w.NH - 1)]
+    g = torch.Generator().manual_seed(41)
+    dH = torch.zeros((w.B, w.NH, w.T, w.DV), dtype=w.torch_dtype)
+    for b, h in heads:
+        dH[b, h, :T1] = torch.randn((T1, w.DV), generator=g).to(w.torch_dtype)
+    d = parity.to_dev(x)
+    got = api.mlstm_bw(d["Q"], d["K"], d["V"], d["i_pre"], d["f_pre"], dH.cuda(), d["C0"],
+                       d["n0"], d["m0"], chunk_size=w.chunk_size, gate_mode=w.gate_mode)
+    torch.cuda.synchronize()
+    assert api.last_device_error() == _lib.OK
+    del d
+    # the oracle on the sampled heads' first T1 tokens
+    xs = parity.slice_heads(x, heads)
+    per_token = ("Q", "K", "V", "i_pre", "f_pre")
+    xt = {k: (None if v is None else (v[:, :, :T1].contiguous() if k in per_token else v))
+          for k, v in xs.items()}
+    dHt = torch.stack([dH[b, h, :T1] for b, h in heads], 0).unsqueeze(0)
+    ref = ob.gradients(xt, dHt, w.gate_mode)
+    errs = {}
+    for k in ("dQ", "dK", "dV", "di_pre", "df_pre"):
+        t = got[k]
+        sampled = torch.stack([t[b, h, :T1] for b, h in heads], 0).unsqueeze(0)
+        errs[k] = parity.worst_rel(sampled.double().cpu().numpy(), ref[k].numpy())
+        for b, h in heads:
+            assert not t[b, h, T1:].any(), f"{k}: gradient after the last token of the loss"
+        assert not t[0, 1].any() and not t[w.B - 1, 0].any(), f"{k}: gradient on a head outside the loss"
+    if "dC0" in got:
+        for k in ("dC0", "dn0"):
+            sampled = torch.stack([got[k][b, h] for b, h in heads], 0).unsqueeze(0)
+            errs[k] = parity.worst_rel(sampled.double().cpu().numpy(), ref[k].numpy())
+    bad = {k: v for k, v in errs.items() if not v <= TOL[w.dtype]}
+    assert not bad, f"{name}: {errs}"
+
+
 def test_backward_chunk_size_invariance():
     """The gradients do not depend on the chunk size (64, 128, 256)."""
     outs = []
