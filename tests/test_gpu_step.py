@@ -133,3 +133,24 @@ def test_step_rejects_bad_arguments_before_launching():
                         C.data_ptr(), n.data_ptr(), g.data_ptr(), v.data_ptr(), B, NH, 2048, DV,
                         _lib.DT_BF16, _lib.GATE_EXP, None)
     assert st == _lib.ERR_UNSUPPORTED
+
+
+def test_step_full_size_sampled_heads():
+    """The 7B-shaped decode batch that `bench.py --op step` times (B=8, NH=8,
+    256 x 512 states, bf16 tokens): one step from a random state, two heads
+    (the first and the last) recomputed by the oracle."""
+    B, NH, DK, DV = 8, 8, 256, 512
+    C, n, m = _state(B, NH, DK, DV, 51)
+    q, k, v, i_pre, f_pre = _token(B, NH, DK, DV, torch.bfloat16, 52)
+    Cd, nd, md = C.cuda(), n.cuda(), m.cuda()
+    h = api.mlstm_step(q.cuda(), k.cuda(), v.cuda(), i_pre.cuda(), f_pre.cuda(), Cd, nd, md)
+    _check_ok()
+    heads = [(0, 0), (B - 1, NH - 1)]
+    x = {"Q": q[:, :, None], "K": k[:, :, None], "V": v[:, :, None],
+         "i_pre": i_pre[:, :, None], "f_pre": f_pre[:, :, None], "C0": C, "n0": n, "m0": m}
+    ref = parity.oracle_run(x, "exp", heads=heads)
+    tol = parity.TOL["bf16"]
+    assert parity.worst_rel(parity.pick(h, heads), ref["H"][:, :, 0]) < tol
+    assert parity.worst_rel(parity.pick(Cd, heads), ref["C_T"]) < tol
+    assert parity.worst_rel(parity.pick(nd, heads), ref["n_T"]) < tol
+    assert parity.m_err(parity.pick(md, heads), ref["m_T"]) < 1e-5
