@@ -34,6 +34,8 @@ CASES = [
     (1, 2, 130, 128, 128, 128, "bf16", "exp", True),    # a 2-token last chunk
     (2, 1, 100, 128, 128, 128, "bf16", "exp", True),    # shorter than a chunk: fp32 kernels
     (1, 2, 300, 256, 256, 512, "bf16", "sigmoid", True),  # d_qk 256 x d_v 256, ragged
+    (1, 1, 256, 128, 1024, 256, "bf16", "exp", True),   # widest d_v: 16 column blocks per row
+    (1, 2, 260, 256, 128, 128, "bf16", "exp", False),   # d_qk 256 x d_v 128
 ]
 
 
