@@ -410,40 +410,48 @@ tc_bwd_gvec_kernel(Problem p, Gates g, const __nv_bfloat16* __restrict__ Q,
 }
 
 // Reverse recurrence on tcgen05: one CTA per (b, h) and 128 x NT tile of
-// the [d_qk, d_v] gradient state (NT = 256 where d_v allows, else 128),
-// walking the chunks from the last,
+// the [d_qk, d_v] gradient state, walking the chunks from the last,
 //
-//   G~_k = e^{g_k + m_k - m_{k+1}} G~_{k+1} + Q_k^T dUr_k,   G~_NC = 0,
+//   G~_k = e^{g_k + m_k - m_{k+1}} G~_{k+1} + U_k,   U_k = Q_k^T dUr_k,   G~_NC = 0
 //
-// with the running G~ as a TMEM accumulator (dUr: du~ with rows scaled by
-// e^{m_k - mu_t}).  Per chunk the epilogue warps read G~_{k+1} 32 columns at
-// a time, store it as the bf16 operand copy Gb (block layout of
-// cb_block_row, index bh (NC + 1) + k + 1) and write it back times the
-// decay; the chunk's two MMAs then accumulate onto it.  G~_0 also goes to
-// dC0 in fp32.  The chunk
-// steps are sequential, so each CTA takes a wide tile and eight epilogue
-// warps (two per TMEM lane quadrant, each half of the columns) to spread the
-// fixed cost of a step (the TMEM round trip and the MMA hand-off) over more
-// of the state.  The CTAs of the first column tile carry g~ along (one row
-// per thread of the first column half) from the increments u.
+// (dUr: du~ with rows scaled by e^{m_k - mu_t}).  The chunk updates U_k do not
+// depend on the recurrence, so the MMA warp computes them ahead into two
+// alternating TMEM accumulators; the running G~ lives in the registers of the
+// epilogue threads (eight warps, two per TMEM lane quadrant, each thread one
+// state row and half of the tile's columns).  Per chunk an epilogue thread
+// stores G~_{k+1} as the bf16 operand copy Gb (block layout of cb_block_row,
+// index bh (NC + 1) + k + 1), then waits for U_k, folds it in and releases the
+// accumulator; the MMAs of the next chunks run meanwhile.  G~_0 also goes to
+// dC0 in fp32.  The CTAs of the first column tile carry g~ along (one row per
+// thread of the first column half) from the increments u.
+// The bf16 copy of a step goes out through shared memory: in the block
+// layout the tile's rows of one 64-column block are 16 KB in a row of the
+// global array, so the epilogue threads write their rows into a staging copy
+// of the two blocks and one thread issues two bulk stores (stores from each
+// thread straight to its own row would half-fill a 32-byte sector per 16-byte
+// store, twice the bytes on the way to L2).  Two staging buffers alternate.
 // Roles (320 threads): warp 0 producer, warp 1 TMEM owner and MMA issuer,
-// warps 2..9 epilogue; ring of 64-token stages (A = Q^T 16 KB, B = dUr
-// NT x 128 bytes), 96 KB in all, two CTAs per SM.
+// warps 2..9 epilogue; ring of four 64-token stages (A = Q^T 16 KB, B = dUr
+// 16 KB), one CTA per SM.
 constexpr int kRevThreads = 320;
 template <int NT>
 struct RevCfg {
+  static_assert(NT == 128, "one 64-column block per epilogue column half");
   static constexpr uint32_t kBBytes = NT * 128;
   static constexpr uint32_t kStageBytes = kTileBytes + kBBytes;
-  static constexpr int kStages = NT == 256 ? 2 : 3;
-  static constexpr uint32_t kOffBar = kStages * kStageBytes;  // full, empty, acc, master
-  static constexpr uint32_t kOffSlot = kOffBar + 8 * (2 * kStages + 2);
+  static constexpr int kStages = 4;
+  static constexpr uint32_t kStgBytes = 128 * NT * 2;  // bf16 tile, two 16 KB blocks
+  static constexpr uint32_t kOffStg = kStages * kStageBytes;  // two staging buffers
+  static constexpr uint32_t kOffBar = kOffStg + 2 * kStgBytes;  // full, empty, u_full[2], u_empty[2]
+  static constexpr uint32_t kOffSlot = kOffBar + 8 * (2 * kStages + 4);
   static constexpr uint32_t kSmem = kOffSlot + 16 + 1024;
   static_assert(kSmem <= 227 * 1024, "shared memory");
-  static constexpr int kCols = NT / 2;  // columns per epilogue thread
+  static constexpr int kCols = NT / 2;   // columns per epilogue thread
+  static constexpr uint32_t kTmemCols = 2 * NT;
 };
 
 template <int NT>
-__global__ void __launch_bounds__(kRevThreads, 2)
+__global__ void __launch_bounds__(kRevThreads, 1)
 tc_bwd_rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_dur,
                   Problem p, Gates g, const float* __restrict__ u, __nv_bfloat16* __restrict__ Gb,
                   float* __restrict__ g_states, float* __restrict__ dC0) {
@@ -454,7 +462,7 @@ tc_bwd_rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                                              ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
   const uint32_t bar_full = sbase + R::kOffBar, bar_empty = bar_full + 8 * kSt;
-  const uint32_t bar_acc = bar_full + 16 * kSt, bar_master = bar_acc + 8;
+  const uint32_t bar_ufull = bar_full + 16 * kSt, bar_uempty = bar_ufull + 16;
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + R::kOffSlot);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -468,12 +476,14 @@ tc_bwd_rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       mbar_init(bar_full + 8 * i, 1);
       mbar_init(bar_empty + 8 * i, 1);
     }
-    mbar_init(bar_acc, 1);
-    mbar_init(bar_master, kRevThreads - 64);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar_ufull + 8 * b, 1);
+      mbar_init(bar_uempty + 8 * b, kRevThreads - 64);
+    }
     fence_barrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32((const void*)tmem_slot), NT);
+    tmem_alloc(smem_u32((const void*)tmem_slot), R::kTmemCols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -510,8 +520,9 @@ tc_bwd_rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       constexpr uint32_t idesc = idesc_bf16(128, NT, 1, 1);
       bool ok = true;
       for (int kk = 0; kk < NC && ok; ++kk) {
-        // the epilogue has scaled the running state by this chunk's decay
-        ok = mbar_wait(bar_master, kk & 1, p, 8);
+        const int buf = kk & 1;
+        // the epilogue has folded in the update that last used this accumulator
+        if (kk >= 2) ok = mbar_wait(bar_uempty + 8 * buf, ((kk - 2) >> 1) & 1, p, 8);
         if (!ok) break;
         tc_fence_after();
         for (int h = 0; h < 2 && ok; ++h) {
@@ -522,15 +533,15 @@ tc_bwd_rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
           const uint32_t sa = sbase + (uint32_t)s * R::kStageBytes, sb = sa + kTileBytes;
 #pragma unroll
           for (int q = 0; q < 4; ++q)
-            mma_bf16_ss(tmem, sdesc_sw128(sa + q * 2048, 8192, 1024),
-                        sdesc_sw128(sb + q * 2048, 8192, 1024), idesc,
-                        (kk == 0 && h == 0 && q == 0) ? 0u : 1u);
+            mma_bf16_ss(tmem + (uint32_t)(buf * NT), sdesc_sw128(sa + q * 2048, 8192, 1024),
+                        sdesc_sw128(sb + q * 2048, 8192, 1024), idesc, (h | q) ? 1u : 0u);
           mma_commit(bar_empty + 8 * s);
         }
-        mma_commit(bar_acc);
+        mma_commit(bar_ufull + 8 * buf);
       }
     }
   } else {
+    constexpr int kG = R::kCols / 32;  // 32-column groups per thread
     const int q4 = warp & 3, r = q4 * 32 + lane, d = m0 + r;
     const int ch = (warp - 2) >> 2;  // column half
     const int c0 = ch * R::kCols;    // first column of this thread within the tile
@@ -540,86 +551,81 @@ tc_bwd_rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     const int n_vb = DV / 64;
     const bool g_owner = n0 == 0 && ch == 0;
     float gv = 0.f;
-    // row d, tile columns c0 + c*32 .. +31 of G~ (index kidx) as bf16
-    auto store_b16 = [&](long kidx, int c, const uint32_t (&v)[32]) {
-      const int col = n0 + c0 + c * 32;
-      __nv_bfloat16* row = Gb + cb_block_row((long)bh * (NC + 1) + kidx, col / 64, d, DK, n_vb);
+    float G[R::kCols];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int j = (col % 64) / 8 + q;
-        *reinterpret_cast<uint4*>(row + ((j ^ (d & 7)) * 8)) = make_uint4(
-            pack_bf16x2(__uint_as_float(v[8 * q]), __uint_as_float(v[8 * q + 1])),
-            pack_bf16x2(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3])),
-            pack_bf16x2(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5])),
-            pack_bf16x2(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7])));
+    for (int j = 0; j < R::kCols; ++j) G[j] = 0.f;
+    const bool issuer = warp == 2 && lane == 0;
+    int n_st = 0;  // staged copies so far (selects the buffer)
+    // The running state as bf16 at index kidx: this thread's row of its
+    // column half's block into the staging buffer, then two bulk stores.
+    auto store_b16 = [&](long kidx) {
+      const uint32_t buf = (uint32_t)(n_st & 1) * R::kStgBytes;
+      if (issuer) tma_store_wait_read_1();  // the copy from this buffer two steps ago is read
+      named_bar_sync(1, kRevThreads - 64);
+      uint8_t* blk = smem + R::kOffStg + buf + (uint32_t)ch * 16384u;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const float* x = G + 8 * j;
+        *reinterpret_cast<uint4*>(blk + sw128_offset((uint32_t)r, (uint32_t)j)) =
+            make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]),
+                       pack_bf16x2(x[4], x[5]), pack_bf16x2(x[6], x[7]));
       }
+      fence_proxy_async_smem();
+      named_bar_sync(1, kRevThreads - 64);
+      if (issuer) {
+        for (int b = 0; b < 2; ++b)
+          bulk_store(Gb + cb_block_row((long)bh * (NC + 1) + kidx, n0 / 64 + b, m0, DK, n_vb),
+                     sbase + R::kOffStg + buf + (uint32_t)b * 16384u, 16384u);
+        tma_store_commit();
+      }
+      ++n_st;
     };
-    constexpr int kG = R::kCols / 32;  // 32-column groups per thread
     bool ok = true;
-    float decay = expf(gt[NC - 1] + mc[NC - 1] - mc[NC]);
     for (int kk = 0; kk < NC; ++kk) {
-      const int k = NC - 1 - kk;
-      // next chunk's decay and this chunk's g~ increment, loaded ahead of the wait
-      const float decay_next = k > 0 ? expf(gt[k - 1] + mc[k - 1] - mc[k]) : 0.f;
+      const int k = NC - 1 - kk, buf = kk & 1;
+      const float decay = expf(gt[k] + mc[k] - mc[k + 1]);
       const float uk = g_owner ? u[((long)bh * NC + k) * DK + d] : 0.f;
-      if (kk == 0) {
-        // G~_NC = 0: nothing in TMEM yet (the first MMA overwrites)
-        tc_fence_before();
-        mbar_arrive(bar_master);
-        uint32_t z[32];
-#pragma unroll
-        for (int j = 0; j < 32; ++j) z[j] = 0u;
-#pragma unroll
-        for (int c = 0; c < kG; ++c) store_b16(NC, c, z);
-      } else {
-        ok = ok && mbar_wait(bar_acc, (kk - 1) & 1, p, 10);
-        tc_fence_after();
-#pragma unroll 1
-        for (int c = 0; c < kG; ++c) {
-          uint32_t v[32];
-          tmem_ld32(trow + c * 32, v);
-          tmem_wait_ld();
-          store_b16(k + 1, c, v);  // G~_{k+1}
-#pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(decay * __uint_as_float(v[j]));
-          tmem_st32(trow + c * 32, v);
-        }
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(bar_master);
-      }
+      store_b16(k + 1);  // G~_{k+1}
       if (g_owner) {
         g_states[((long)bh * (NC + 1) + k + 1) * DK + d] = gv;
         gv = fmaf(decay, gv, uk);
       }
-      decay = decay_next;
+      ok = ok && mbar_wait(bar_ufull + 8 * buf, (kk >> 1) & 1, p, 10);
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < kG; ++c) {
+        uint32_t v[32];
+        tmem_ld32(trow + (uint32_t)(buf * NT) + c * 32, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) G[c * 32 + j] = fmaf(decay, G[c * 32 + j], __uint_as_float(v[j]));
+      }
+      tc_fence_before();
+      mbar_arrive(bar_uempty + 8 * buf);
     }
     // G~_0
-    ok = ok && mbar_wait(bar_acc, (NC - 1) & 1, p, 11);
-    tc_fence_after();
+    store_b16(0);
     if (g_owner) g_states[(long)bh * (NC + 1) * DK + d] = gv;
-#pragma unroll 1
-    for (int c = 0; c < kG; ++c) {
-      uint32_t v[32];
-      tmem_ld32(trow + c * 32, v);
-      tmem_wait_ld();
-      store_b16(0, c, v);
-      float4* dst = reinterpret_cast<float4*>(dC0 + ((long)bh * DK + d) * DV + n0 + c0 + c * 32);
+    float4* dst = reinterpret_cast<float4*>(dC0 + ((long)bh * DK + d) * DV + n0 + c0);
 #pragma unroll
-      for (int q = 0; q < 8; ++q)
-        dst[q] = make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
-                             __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3]));
-    }
+    for (int q = 0; q < R::kCols / 4; ++q)
+      dst[q] = make_float4(G[4 * q], G[4 * q + 1], G[4 * q + 2], G[4 * q + 3]);
+    if (issuer) tma_store_wait_all();  // the staged copies have landed
     (void)ok;
   }
 
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
-    if (lane == 0) mbar_wait(bar_acc, (NC - 1) & 1, p, 12);
+    // every MMA has completed: the last commit of each accumulator
+    if (lane == 0) {
+      const int last = NC - 1;
+      mbar_wait(bar_ufull + 8 * (last & 1), (last >> 1) & 1, p, 12);
+      if (NC >= 2) mbar_wait(bar_ufull + 8 * ((last - 1) & 1), ((last - 1) >> 1) & 1, p, 12);
+    }
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem, NT);
+    tmem_dealloc(tmem, R::kTmemCols);
   }
 }
 
