@@ -87,7 +87,7 @@ template <int kJob, int NT>
 __global__ void __launch_bounds__(kThreads, 2)
 tc_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_du,
-              const TcBwdArgs a) {
+              const __grid_constant__ CUtensorMap tm_out, const TcBwdArgs a) {
   static_assert(NT == 64 || NT == 128, "output tile");
   const Problem& p = a.p;
   extern __shared__ uint8_t smem_raw[];
@@ -250,6 +250,11 @@ tc_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     const float m_out = a.g.mchk[(long)bh * (NC + 1) + k + 1];
     const float acol_r = a.g.acol[(long)bh * tpad + t];  // -inf on padding
     const float mu = fmaxf(m_in, a.g.amax[(long)bh * tpad + t]);
+    // Output staging: the ring's first stage (32 KB), free once every MMA has
+    // completed; the rows of a thread go out with bulk or TMA stores (a store
+    // per thread and row would half-fill a 32-byte sector per 16 bytes).
+    uint8_t* stg = smem;
+    const bool issuer = warp == 2 && lane == 0;
     // per-column vector of the chunk in shared memory: the squares' column
     // weights acol_s; dq's n_k, dk's g~_{k+1} over this CTA's NT columns
     if constexpr (kJob == kSquares) {
@@ -283,13 +288,12 @@ tc_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             }
             w[j / 2] = pack_bf16x2(f[0], f[1]);
           }
-          __nv_bfloat16* row = a.sq + sq_row(bhk, which, c >> 1, r);
+          // into the staging copy of s-block c / 2 (the block layout of sq)
+          uint8_t* blk = stg + (c >> 1) * 16384;
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int cc = (c & 1) * 4 + u;  // 16-byte chunk of the 128-byte row
-            *reinterpret_cast<uint4*>(row + ((cc ^ (r & 7)) * 8)) =
+          for (int u = 0; u < 4; ++u)
+            *reinterpret_cast<uint4*>(blk + sw128_offset((uint32_t)r, (uint32_t)((c & 1) * 4 + u))) =
                 make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
-          }
         }
       } else {
         const int D = kJob == kDV ? DV : DK;
@@ -335,14 +339,16 @@ tc_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             o[j] = kJob == kDK ? s1 * fmaf(rs, x2, __uint_as_float(v1[j]))
                                : fmaf(s1, __uint_as_float(v1[j]), s2 * rs * x2);
           }
-          if (valid) {
-            uint4* dst = reinterpret_cast<uint4*>(a.out + orow + c * 32);
+          // into the staging box of columns (c / 2) * 64.. (the TMA store's layout)
+          uint8_t* box = stg + (c >> 1) * 16384;
 #pragma unroll
-            for (int u = 0; u < 4; ++u)
-              dst[u] = make_uint4(pack_bf16x2(o[8 * u], o[8 * u + 1]),
-                                  pack_bf16x2(o[8 * u + 2], o[8 * u + 3]),
-                                  pack_bf16x2(o[8 * u + 4], o[8 * u + 5]),
-                                  pack_bf16x2(o[8 * u + 6], o[8 * u + 7]));
+          for (int u = 0; u < 4; ++u)
+            *reinterpret_cast<uint4*>(box + sw128_offset((uint32_t)r, (uint32_t)((c & 1) * 4 + u))) =
+                make_uint4(pack_bf16x2(o[8 * u], o[8 * u + 1]),
+                           pack_bf16x2(o[8 * u + 2], o[8 * u + 3]),
+                           pack_bf16x2(o[8 * u + 4], o[8 * u + 5]),
+                           pack_bf16x2(o[8 * u + 6], o[8 * u + 7]));
+          if (valid) {
             if constexpr (kJob != kDV) {
 #pragma unroll
               for (int u = 0; u < 4; ++u) {
@@ -360,6 +366,22 @@ tc_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         }
         if (kJob != kDV && valid) atomicAdd(&a.dot[(long)bh * T + t], dot);
       }
+    }
+    // Every epilogue thread reaches this barrier whatever its wait returned;
+    // the staged tile goes out only when the issuer's wait succeeded.
+    fence_proxy_async_smem();
+    named_bar_sync(1, 128);
+    if (issuer && ok) {
+      if constexpr (kJob == kSquares) {
+        for (int b = 0; b < 2; ++b)
+          bulk_store(a.sq + sq_row(bhk, which, b, 0), sbase + (uint32_t)b * 16384u, 16384u);
+      } else {
+        // the tile's rows past T are clipped by the tensor map
+        for (int b = 0; b < NT / 64; ++b)
+          tma_store_3d(&tm_out, sbase + (uint32_t)b * 16384u, n0 + b * 64, t0, bh);
+      }
+      tma_store_commit();
+      tma_store_wait_all();  // the staged tile has landed
     }
   }
 
@@ -643,11 +665,12 @@ cudaError_t launch_rev(const CUtensorMap& mq, const CUtensorMap& mu, const Probl
 }
 
 template <int kJob, int NT>
-cudaError_t launch_job(const CUtensorMap* m, const TcBwdArgs& a, dim3 grid, cudaStream_t st) {
+cudaError_t launch_job(const CUtensorMap* m, const CUtensorMap& out, const TcBwdArgs& a, dim3 grid,
+                       cudaStream_t st) {
   auto kern = tc_bwd_kernel<kJob, NT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
   if (e != cudaSuccess) return e;
-  kern<<<grid, kThreads, kSmem, st>>>(m[0], m[1], m[2], m[3], a);
+  kern<<<grid, kThreads, kSmem, st>>>(m[0], m[1], m[2], m[3], out, a);
   return cudaGetLastError();
 }
 
@@ -696,23 +719,29 @@ cudaError_t launch_tc_bwd(const Problem& pb, const void* Q, const void* K, const
   a.Cb = Cb;
   a.Gb = Gb;
   a.sq = sq;
-  cudaError_t e = launch_job<kSquares, 128>(m, a, dim3(2, pb.NC, pb.BH), st);
+  // output maps: 64-column boxes of 128 rows (rows past T are not written)
+  CUtensorMap oq, ok_, ov;
+  if (!encode_tmap_3d(&oq, dQ, 2, pb.DK, pb.T, pb.BH, 64, 128, 128) ||
+      !encode_tmap_3d(&ok_, dK, 2, pb.DK, pb.T, pb.BH, 64, 128, 128) ||
+      !encode_tmap_3d(&ov, dV, 2, pb.DV, pb.T, pb.BH, 64, 128, 128))
+    return cudaErrorInvalidValue;
+  cudaError_t e = launch_job<kSquares, 128>(m, m[0], a, dim3(2, pb.NC, pb.BH), st);
   if (e != cudaSuccess) return e;
   // 128 output columns per CTA (DK and DV are multiples of 128)
   a.X = static_cast<const __nv_bfloat16*>(Q);
   a.out = static_cast<__nv_bfloat16*>(dQ);
   a.dot = qdq;
-  e = launch_job<kDQ, 128>(m, a, dim3(pb.DK / 128, pb.NC, pb.BH), st);
+  e = launch_job<kDQ, 128>(m, oq, a, dim3(pb.DK / 128, pb.NC, pb.BH), st);
   if (e != cudaSuccess) return e;
   a.X = static_cast<const __nv_bfloat16*>(K);
   a.out = static_cast<__nv_bfloat16*>(dK);
   a.dot = kdk;
-  e = launch_job<kDK, 128>(m, a, dim3(pb.DK / 128, pb.NC, pb.BH), st);
+  e = launch_job<kDK, 128>(m, ok_, a, dim3(pb.DK / 128, pb.NC, pb.BH), st);
   if (e != cudaSuccess) return e;
   a.X = nullptr;
   a.out = static_cast<__nv_bfloat16*>(dV);
   a.dot = nullptr;
-  return launch_job<kDV, 128>(m, a, dim3(pb.DV / 128, pb.NC, pb.BH), st);
+  return launch_job<kDV, 128>(m, ov, a, dim3(pb.DV / 128, pb.NC, pb.BH), st);
 }
 
 }  // namespace mlstm
