@@ -184,6 +184,40 @@ mlstm_status mlstm_bw(const void* Q, const void* K, const void* V, const float* 
                       int chunk_size, mlstm_dtype dtype, mlstm_gate_mode gate_mode,
                       void* workspace, size_t workspace_bytes, mlstm_stream_t stream);
 
+/* Training pair ("Tiled Flash Linear Attention: More Efficient Linear RNN and
+ * xLSTM Kernels": the forward's per-token normaliser and stabiliser outputs
+ * serve the backward).  mlstm_fw_train is the forward pass of mlstm_fw (same
+ * arguments and outputs, no chunk size) that also keeps, in a caller buffer
+ * `saved`, what the backward needs: the bf16 chunk states and fp32 n states
+ * entering every 128-token chunk and, per token, the signed denominator
+ * copysign(max(|n.q|, e^{-m}), n.q) and the stabiliser m.  mlstm_bw_saved is
+ * mlstm_bw (same gradients) that takes `saved` and the forward's H instead of
+ * recomputing the forward.  Both run in 128-token chunks on the tensor cores
+ * and exist only for the shapes of the tensor-core backward: bf16 inputs,
+ * DK of 128 or 256, DV of 128 or a multiple of 256 up to 1024, T >= 128
+ * (else MLSTM_ERR_UNSUPPORTED, from mlstm_train_sizes first).
+ * mlstm_train_sizes: bytes of `saved` and of each call's workspace.
+ * Buffers 16-byte aligned; C0/n0/m0 and C_T/n_T/m_T each all given or all
+ * null; `saved` must not change between the two calls.  mlstm_fw_train: 4 or
+ * 5 launches; mlstm_bw_saved: 10; asynchronous on `stream`.  Errors as
+ * mlstm_fw. */
+mlstm_status mlstm_train_sizes(int B, int NH, int T, int DK, int DV, mlstm_dtype dtype,
+                               size_t* saved_bytes, size_t* fw_workspace_bytes,
+                               size_t* bw_workspace_bytes);
+mlstm_status mlstm_fw_train(const void* Q, const void* K, const void* V, const float* i_pre,
+                            const float* f_pre, const float* C0, const float* n0, const float* m0,
+                            void* H, float* C_T, float* n_T, float* m_T, void* saved,
+                            size_t saved_bytes, int B, int NH, int T, int DK, int DV,
+                            mlstm_dtype dtype, mlstm_gate_mode gate_mode, void* workspace,
+                            size_t workspace_bytes, mlstm_stream_t stream);
+mlstm_status mlstm_bw_saved(const void* Q, const void* K, const void* V, const float* i_pre,
+                            const float* f_pre, const float* C0, const float* n0, const float* m0,
+                            const void* H, const void* saved, size_t saved_bytes, const void* dH,
+                            void* dQ, void* dK, void* dV, float* di_pre, float* df_pre,
+                            float* dC0, float* dn0, float* dm0, int B, int NH, int T, int DK,
+                            int DV, mlstm_dtype dtype, mlstm_gate_mode gate_mode,
+                            void* workspace, size_t workspace_bytes, mlstm_stream_t stream);
+
 /* Single-token step (decode), the recurrence of mlstm_fw for T = 1: advances
  * the state of every (b, h) by one token in place and writes that token's
  * output ("xLSTM: the NX-AI repository behind the extended LSTM
@@ -243,8 +277,9 @@ typedef enum {
   MLSTM_KERNEL_TC_PARALLEL = 4,   /* tensor-core intra-chunk TFLA kernel       */
   MLSTM_KERNEL_TC_FUSED = 5,      /* tensor-core fused kernel                  */
   MLSTM_KERNEL_STEP = 6,          /* single-token step (1 or 2 launches)       */
-  MLSTM_KERNEL_BW = 7,            /* backward pass (10 to 13 launches per call) */
-  MLSTM_KERNEL_COUNT = 8
+  MLSTM_KERNEL_BW = 7,            /* backward pass (10 to 14 launches per call) */
+  MLSTM_KERNEL_FW_TRAIN = 8,      /* training forward (4 or 5 launches)        */
+  MLSTM_KERNEL_COUNT = 9
 } mlstm_kernel_id;
 
 /* Total number of kernels this library has enqueued since it was loaded. */

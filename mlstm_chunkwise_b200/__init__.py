@@ -7,5 +7,6 @@ The computation runs in ``libmlstm_fw.so`` (hand-written CUDA kernels; see
 synthetic inputs (``inputs.py``).
 """
 from .api import (MlstmError, substep_workspace_size, last_device_error, mlstm_bw,  # noqa: F401
-                  mlstm_chunkwise, mlstm_fw, mlstm_fw_chunk_states, mlstm_fw_parallel, mlstm_step,
-                  set_watchdog, workspace_size)
+                  mlstm_bw_saved, mlstm_chunkwise, mlstm_fw, mlstm_fw_chunk_states,
+                  mlstm_fw_parallel, mlstm_fw_train, mlstm_step, set_watchdog, train_sizes,
+                  workspace_size)

@@ -16,7 +16,7 @@ ERR_SCRATCH_TOO_SMALL = 6
 DT_F32, DT_BF16 = 0, 1
 GATE_EXP, GATE_SIGMOID = 0, 1
 ALGO_AUTO, ALGO_SIMT, ALGO_TC, ALGO_TC_FUSED = 0, 1, 2, 3
-KERNEL_COUNT = 8
+KERNEL_COUNT = 9
 
 _vp = ctypes.c_void_p
 _i = ctypes.c_int
@@ -34,6 +34,9 @@ SIGNATURES = {
     "mlstm_fw_static_scratch_capacity": (_sz, []),
     "mlstm_bw_workspace_size": (_i, [_i] * 7 + [ctypes.POINTER(_sz)]),
     "mlstm_bw": (_i, [_vp] * 17 + [_i] * 8 + [_vp, _sz, _vp]),
+    "mlstm_train_sizes": (_i, [_i] * 6 + [ctypes.POINTER(_sz)] * 3),
+    "mlstm_fw_train": (_i, [_vp] * 13 + [_sz] + [_i] * 7 + [_vp, _sz, _vp]),
+    "mlstm_bw_saved": (_i, [_vp] * 10 + [_sz] + [_vp] * 9 + [_i] * 7 + [_vp, _sz, _vp]),
     "mlstm_step": (_i, [_vp] * 9 + [_i] * 6 + [_vp]),
     "mlstm_last_device_error": (_i, [_vp]),
     "mlstm_last_device_error_word": (ctypes.c_uint32, []),

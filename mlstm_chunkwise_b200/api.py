@@ -165,6 +165,70 @@ def mlstm_bw(Q, K, V, i_pre, f_pre, dH, C0=None, n0=None, m0=None, *, chunk_size
     return out
 
 
+def train_sizes(B, NH, T, DK, DV, dtype=torch.bfloat16):
+    """Bytes of the saved buffer and of the two calls' workspaces of the
+    training pair, or None when the shape has no training path (it needs the
+    tensor-core backward: bf16, d_qk 128 or 256, d_v 128 or a multiple of 256
+    up to 1024, T >= 128)."""
+    sv, fw, bw = ctypes.c_size_t(0), ctypes.c_size_t(0), ctypes.c_size_t(0)
+    st = _lib.lib().mlstm_train_sizes(B, NH, T, DK, DV, _DT[dtype], ctypes.byref(sv),
+                                      ctypes.byref(fw), ctypes.byref(bw))
+    if st == _lib.ERR_UNSUPPORTED:
+        return None
+    _lib.check(st, "mlstm_train_sizes")
+    return int(sv.value), int(fw.value), int(bw.value)
+
+
+def mlstm_fw_train(Q, K, V, i_pre, f_pre, C0=None, n0=None, m0=None, *, gate_mode: str = "exp"):
+    """The forward pass of ``mlstm_fw`` (128-token chunks on the tensor cores)
+    that also keeps what ``mlstm_bw_saved`` needs.  Returns ``(H, (C_T, n_T,
+    m_T), saved)``; ``saved`` is an opaque uint8 tensor.  Raises
+    ``MlstmError`` (unsupported) outside the shapes of ``train_sizes``."""
+    B, NH, T, DK, DV, dev, dt = _check_common(Q, K, V, i_pre, f_pre)
+    _check_state(C0, n0, m0, B, NH, DK, DV, dev)
+    sizes = train_sizes(B, NH, T, DK, DV, dt)
+    if sizes is None:
+        raise MlstmError(_lib.ERR_UNSUPPORTED, "mlstm_fw_train")
+    sv_bytes, fw_bytes, _ = sizes
+    H = torch.empty((B, NH, T, DV), dtype=dt, device=dev)
+    C_T = torch.empty((B, NH, DK, DV), dtype=torch.float32, device=dev)
+    n_T = torch.empty((B, NH, DK), dtype=torch.float32, device=dev)
+    m_T = torch.empty((B, NH), dtype=torch.float32, device=dev)
+    saved = torch.empty(sv_bytes, dtype=torch.uint8, device=dev)
+    ws = torch.empty(max(fw_bytes, 1), dtype=torch.uint8, device=dev)
+    _lib.check(_lib.lib().mlstm_fw_train(
+        _ptr(Q), _ptr(K), _ptr(V), _ptr(i_pre), _ptr(f_pre), _ptr(C0), _ptr(n0), _ptr(m0),
+        _ptr(H), _ptr(C_T), _ptr(n_T), _ptr(m_T), _ptr(saved), saved.numel(), B, NH, T, DK, DV,
+        _DT[dt], _GATE[gate_mode], _ptr(ws), ws.numel(), _stream(dev)), "mlstm_fw_train")
+    return H, (C_T, n_T, m_T), saved
+
+
+def mlstm_bw_saved(Q, K, V, i_pre, f_pre, H, saved, dH, C0=None, n0=None, m0=None, *,
+                   gate_mode: str = "exp"):
+    """``mlstm_bw`` from the output and the saved buffer of ``mlstm_fw_train``
+    (same inputs) instead of a recomputed forward.  Returns the same dict."""
+    B, NH, T, DK, DV, dev, dt = _check_common(Q, K, V, i_pre, f_pre)
+    _check_state(C0, n0, m0, B, NH, DK, DV, dev)
+    _check_tensor("H", H, dt, (B, NH, T, DV), dev)
+    _check_tensor("dH", dH, dt, (B, NH, T, DV), dev)
+    sizes = train_sizes(B, NH, T, DK, DV, dt)
+    if sizes is None:
+        raise MlstmError(_lib.ERR_UNSUPPORTED, "mlstm_bw_saved")
+    _, _, bw_bytes = sizes
+    out = {"dQ": torch.empty_like(Q), "dK": torch.empty_like(K), "dV": torch.empty_like(V),
+           "di_pre": torch.empty_like(i_pre), "df_pre": torch.empty_like(f_pre)}
+    if C0 is not None:
+        out.update(dC0=torch.empty_like(C0), dn0=torch.empty_like(n0), dm0=torch.empty_like(m0))
+    ws = torch.empty(max(bw_bytes, 1), dtype=torch.uint8, device=dev)
+    _lib.check(_lib.lib().mlstm_bw_saved(
+        _ptr(Q), _ptr(K), _ptr(V), _ptr(i_pre), _ptr(f_pre), _ptr(C0), _ptr(n0), _ptr(m0),
+        _ptr(H), _ptr(saved), saved.numel(), _ptr(dH), _ptr(out["dQ"]), _ptr(out["dK"]),
+        _ptr(out["dV"]), _ptr(out["di_pre"]), _ptr(out["df_pre"]), _ptr(out.get("dC0")),
+        _ptr(out.get("dn0")), _ptr(out.get("dm0")), B, NH, T, DK, DV, _DT[dt],
+        _GATE[gate_mode], _ptr(ws), ws.numel(), _stream(dev)), "mlstm_bw_saved")
+    return out
+
+
 def mlstm_step(q, k, v, i_pre, f_pre, C, n, m, *, gate_mode: str = "exp", h=None):
     """One token of the recurrence for every (b, h), in place on the state.
 
@@ -263,37 +327,60 @@ def watchdog_selftest(device=None) -> None:
 
 
 class _MlstmChunkwise(torch.autograd.Function):
-    """Differentiable mLSTM: the forward is ``mlstm_fw``, the backward
-    ``mlstm_bw`` (which recomputes what it needs from the inputs).  Gradients
+    """Differentiable mLSTM.  Where the training pair exists (``train_sizes``)
+    and ``recompute`` is off, the forward is ``mlstm_fw_train`` and the
+    backward ``mlstm_bw_saved`` (about 1 GB kept per 7B-shaped call, no
+    recomputation); otherwise the forward is ``mlstm_fw`` and the backward
+    ``mlstm_bw``, which recomputes what it needs from the inputs.  Gradients
     flow from H only; the returned final state carries none."""
 
     @staticmethod
-    def forward(ctx, Q, K, V, i_pre, f_pre, C0, n0, m0, chunk_size, gate_mode, algo):
-        H, (C_T, n_T, m_T) = mlstm_fw(Q, K, V, i_pre, f_pre, C0, n0, m0, chunk_size=chunk_size,
-                                      gate_mode=gate_mode, algo=algo)
-        ctx.save_for_backward(Q, K, V, i_pre, f_pre, C0, n0, m0)
-        ctx.cfg = (chunk_size, gate_mode)
+    def forward(ctx, Q, K, V, i_pre, f_pre, C0, n0, m0, chunk_size, gate_mode, algo, recompute):
+        saved = None
+        if not recompute and algo == "auto" and Q.is_cuda and Q.dtype in _DT and \
+                train_sizes(Q.shape[0], Q.shape[1], Q.shape[2], Q.shape[3], V.shape[-1],
+                            Q.dtype) is not None:
+            H, (C_T, n_T, m_T), saved = mlstm_fw_train(Q, K, V, i_pre, f_pre, C0, n0, m0,
+                                                       gate_mode=gate_mode)
+        else:
+            H, (C_T, n_T, m_T) = mlstm_fw(Q, K, V, i_pre, f_pre, C0, n0, m0,
+                                          chunk_size=chunk_size, gate_mode=gate_mode, algo=algo)
+        if saved is not None:
+            ctx.save_for_backward(Q, K, V, i_pre, f_pre, C0, n0, m0, H, saved)
+        else:
+            ctx.save_for_backward(Q, K, V, i_pre, f_pre, C0, n0, m0)
+        ctx.cfg = (chunk_size, gate_mode, saved is not None)
         ctx.mark_non_differentiable(C_T, n_T, m_T)
         return H, C_T, n_T, m_T
 
     @staticmethod
     def backward(ctx, dH, dC_T, dn_T, dm_T):
-        Q, K, V, i_pre, f_pre, C0, n0, m0 = ctx.saved_tensors
-        chunk_size, gate_mode = ctx.cfg
-        g = mlstm_bw(Q, K, V, i_pre, f_pre, dH.contiguous(), C0, n0, m0, chunk_size=chunk_size,
-                     gate_mode=gate_mode)
+        chunk_size, gate_mode, kept = ctx.cfg
+        if kept:
+            Q, K, V, i_pre, f_pre, C0, n0, m0, H, saved = ctx.saved_tensors
+            g = mlstm_bw_saved(Q, K, V, i_pre, f_pre, H, saved, dH.contiguous(), C0, n0, m0,
+                               gate_mode=gate_mode)
+        else:
+            Q, K, V, i_pre, f_pre, C0, n0, m0 = ctx.saved_tensors
+            g = mlstm_bw(Q, K, V, i_pre, f_pre, dH.contiguous(), C0, n0, m0,
+                         chunk_size=chunk_size, gate_mode=gate_mode)
         return (g["dQ"], g["dK"], g["dV"], g["di_pre"], g["df_pre"], g.get("dC0"), g.get("dn0"),
-                g.get("dm0"), None, None, None)
+                g.get("dm0"), None, None, None, None)
 
 
 def mlstm_chunkwise(Q, K, V, i_pre, f_pre, C0=None, n0=None, m0=None, *, chunk_size: int = 64,
-                    gate_mode: str = "exp", algo: str = "auto"):
-    """mLSTM forward pass that autograd can differentiate (through ``mlstm_bw``).
+                    gate_mode: str = "exp", algo: str = "auto", recompute: bool = False):
+    """mLSTM forward pass that autograd can differentiate.
 
     Same arguments and shapes as ``mlstm_fw``; returns ``(H, (C_T, n_T, m_T))``.
     The gradient of a loss on H reaches Q, K, V, both gate pre-activations and
     the initial state; the final state is returned without a gradient path.
+    Where the training pair exists (bf16, d_qk 128 or 256, T >= 128; see
+    ``train_sizes``) the forward keeps the chunk states and per-token
+    normalisers for the backward (128-token chunks, whatever ``chunk_size``
+    says); ``recompute=True`` keeps nothing and recomputes them in the
+    backward instead (less memory, a slower backward).
     """
     H, C_T, n_T, m_T = _MlstmChunkwise.apply(Q, K, V, i_pre, f_pre, C0, n0, m0, chunk_size,
-                                             gate_mode, algo)
+                                             gate_mode, algo, recompute)
     return H, (C_T, n_T, m_T)

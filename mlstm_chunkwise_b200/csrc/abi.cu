@@ -11,6 +11,7 @@
 
 #include "common.cuh"
 #include "tc.h"
+#include "tc_bwd.h"
 
 namespace mlstm {
 namespace {
@@ -254,6 +255,7 @@ const char* mlstm_kernel_name(int id) {
     case MLSTM_KERNEL_TC_FUSED: return "tc_fused";
     case MLSTM_KERNEL_STEP: return "step";
     case MLSTM_KERNEL_BW: return "bw";
+    case MLSTM_KERNEL_FW_TRAIN: return "fw_train";
   }
   return "unknown";
 }
@@ -504,6 +506,82 @@ mlstm_status mlstm_bw(const void* Q, const void* K, const void* V, const float* 
   return from_cuda(launch_family(MLSTM_KERNEL_BW, bwd_launches(p, dtype), st, [&] {
     return launch_backward(p, dtype, Q, K, V, i_pre, f_pre, C0, n0, m0, dH, dQ, dK, dV, di_pre,
                            df_pre, dC0, dn0, dm0, workspace, st);
+  }));
+}
+
+mlstm_status mlstm_train_sizes(int B, int NH, int T, int DK, int DV, mlstm_dtype dtype,
+                               size_t* saved_bytes, size_t* fw_workspace_bytes,
+                               size_t* bw_workspace_bytes) {
+  if (!saved_bytes || !fw_workspace_bytes || !bw_workspace_bytes ||
+      !valid_enums(dtype, MLSTM_GATE_EXP, MLSTM_ALGO_AUTO))
+    return MLSTM_ERR_INVALID_ARG;
+  mlstm_status s = check_sizes(B, NH, T, DK, DV, 128);
+  if (s != MLSTM_OK) return s;
+  const Problem p = make_problem(B, NH, T, DK, DV, 128, MLSTM_GATE_EXP);
+  if (!train_supported(p, dtype)) return MLSTM_ERR_UNSUPPORTED;
+  *saved_bytes = train_saved_bytes(p);
+  *fw_workspace_bytes = fw_train_workspace_bytes(p);
+  *bw_workspace_bytes = bw_saved_workspace_bytes(p);
+  return MLSTM_OK;
+}
+
+mlstm_status mlstm_fw_train(const void* Q, const void* K, const void* V, const float* i_pre,
+                            const float* f_pre, const float* C0, const float* n0, const float* m0,
+                            void* H, float* C_T, float* n_T, float* m_T, void* saved,
+                            size_t saved_bytes, int B, int NH, int T, int DK, int DV,
+                            mlstm_dtype dtype, mlstm_gate_mode gate_mode, void* workspace,
+                            size_t workspace_bytes, mlstm_stream_t stream) {
+  if (!valid_enums(dtype, gate_mode, MLSTM_ALGO_AUTO)) return MLSTM_ERR_INVALID_ARG;
+  mlstm_status s = check_sizes(B, NH, T, DK, DV, 128);
+  if (s != MLSTM_OK) return s;
+  Problem p = make_problem(B, NH, T, DK, DV, 128, gate_mode);
+  if (!train_supported(p, dtype)) return MLSTM_ERR_UNSUPPORTED;
+  if (!Q || !K || !V || !i_pre || !f_pre || !H || !saved || !workspace)
+    return MLSTM_ERR_INVALID_ARG;
+  if (!((C0 && n0 && m0) || (!C0 && !n0 && !m0))) return MLSTM_ERR_INVALID_ARG;
+  if (!((C_T && n_T && m_T) || (!C_T && !n_T && !m_T))) return MLSTM_ERR_INVALID_ARG;
+  const void* ptrs[] = {Q, K, V, i_pre, f_pre, C0, n0, m0, H, C_T, n_T, m_T, saved, workspace};
+  for (const void* q : ptrs)
+    if (!aligned16(q)) return MLSTM_ERR_INVALID_ARG;
+  if (saved_bytes < train_saved_bytes(p) || workspace_bytes < fw_train_workspace_bytes(p))
+    return MLSTM_ERR_INVALID_ARG;
+  p.err = error_word_ptr();
+  if (!p.err) return MLSTM_ERR_CUDA;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  return from_cuda(launch_family(MLSTM_KERNEL_FW_TRAIN, fw_train_launches(p), st, [&] {
+    return launch_fw_train(p, Q, K, V, i_pre, f_pre, C0, n0, m0, H, C_T, n_T, m_T, saved,
+                           workspace, st);
+  }));
+}
+
+mlstm_status mlstm_bw_saved(const void* Q, const void* K, const void* V, const float* i_pre,
+                            const float* f_pre, const float* C0, const float* n0, const float* m0,
+                            const void* H, const void* saved, size_t saved_bytes, const void* dH,
+                            void* dQ, void* dK, void* dV, float* di_pre, float* df_pre,
+                            float* dC0, float* dn0, float* dm0, int B, int NH, int T, int DK,
+                            int DV, mlstm_dtype dtype, mlstm_gate_mode gate_mode,
+                            void* workspace, size_t workspace_bytes, mlstm_stream_t stream) {
+  if (!valid_enums(dtype, gate_mode, MLSTM_ALGO_AUTO)) return MLSTM_ERR_INVALID_ARG;
+  mlstm_status s = check_sizes(B, NH, T, DK, DV, 128);
+  if (s != MLSTM_OK) return s;
+  Problem p = make_problem(B, NH, T, DK, DV, 128, gate_mode);
+  if (!train_supported(p, dtype)) return MLSTM_ERR_UNSUPPORTED;
+  if (!((C0 && n0 && m0) || (!C0 && !n0 && !m0))) return MLSTM_ERR_INVALID_ARG;
+  if (!Q || !K || !V || !i_pre || !f_pre || !H || !saved || !dH || !dQ || !dK || !dV ||
+      !di_pre || !df_pre || !workspace)
+    return MLSTM_ERR_INVALID_ARG;
+  const void* ptrs[] = {Q,  K,  V,      i_pre,  f_pre, C0,  n0,  m0,  H,        saved,
+                        dH, dQ, dK,     dV,     di_pre, df_pre, dC0, dn0, dm0, workspace};
+  for (const void* q : ptrs)
+    if (!aligned16(q)) return MLSTM_ERR_INVALID_ARG;
+  if (saved_bytes < train_saved_bytes(p) || workspace_bytes < bw_saved_workspace_bytes(p))
+    return MLSTM_ERR_INVALID_ARG;
+  p.err = error_word_ptr();
+  if (!p.err) return MLSTM_ERR_CUDA;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  return from_cuda(launch_family(MLSTM_KERNEL_BW, bw_saved_launches(p), st, [&] {
+    return launch_bw_saved(p, Q, K, V, i_pre, f_pre, C0, n0, m0, H, saved, dH, dQ, dK, dV,
+                           di_pre, df_pre, dC0, dn0, dm0, workspace, st);
   }));
 }
 

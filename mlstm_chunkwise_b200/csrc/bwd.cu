@@ -695,11 +695,14 @@ bool tc_backward(const Problem& p, mlstm_dtype dt) {
 constexpr size_t kAlign = 256;
 inline size_t al(size_t b) { return (b + kAlign - 1) / kAlign * kAlign; }
 
-size_t carve(const Problem& p_in, mlstm_dtype dt, char* base, BwdWs* w) {
+// saved: the tensor-core backward given the training forward's saved buffers
+// (no room for the recomputed forward: chunk states, h, denominators).
+size_t carve(const Problem& p_in, mlstm_dtype dt, char* base, BwdWs* w, bool saved = false) {
   const bool tcb = tc_backward(p_in, dt);
   const Problem p = tcb ? tc_bwd_problem(p_in) : p_in;
   const size_t BH = p.BH, T = p.T, NC = p.NC, tpad = NC * p.L, DK = p.DK, DV = p.DV;
   const bool tc = tcb || tc_recompute(p, dt);
+  const bool rec = !(tcb && saved);  // room for the recomputed forward
   size_t off = 0;
   auto take = [&](size_t n) -> float* {
     float* ptr = base ? reinterpret_cast<float*>(base + off) : nullptr;
@@ -720,13 +723,13 @@ size_t carve(const Problem& p_in, mlstm_dtype dt, char* base, BwdWs* w) {
   BwdWs x = {};
   x.g = g;
   x.C_states = tcb ? nullptr : take(BH * NC * DK * DV);
-  x.n_states = take(BH * NC * DK);
+  x.n_states = rec ? take(BH * NC * DK) : nullptr;
   x.H32 = tc ? nullptr : take(BH * T * DV);
-  x.Cb = tc ? take16(BH * NC * DK * DV) : nullptr;
-  x.H16 = tc ? take16(BH * T * DV) : nullptr;
-  x.seg = tc ? take(tc_states_segment_floats(p)) : nullptr;
-  x.den = take(BH * T);
-  x.mr = take(BH * T);
+  x.Cb = tc && rec ? take16(BH * NC * DK * DV) : nullptr;
+  x.H16 = tc && rec ? take16(BH * T * DV) : nullptr;
+  x.seg = tc && rec ? take(tc_states_segment_floats(p)) : nullptr;
+  x.den = rec ? take(BH * T) : nullptr;
+  x.mr = rec ? take(BH * T) : nullptr;
   x.dU = tcb ? nullptr : take(BH * T * DV);
   x.dA = take(BH * T);
   x.G_states = tcb ? nullptr : take(BH * (NC + 1) * DK * DV);
@@ -752,28 +755,19 @@ size_t carve(const Problem& p_in, mlstm_dtype dt, char* base, BwdWs* w) {
 // and row-scaled), the reverse states (per-chunk updates on the tensor cores,
 // then a reverse scan), the squares and dq, dk, dv (tc_bwd.cu), and the gate
 // gradients.
-cudaError_t launch_bwd_tc(const Problem& p_in, const void* Q, const void* K, const void* V,
-                          const float* i_pre, const float* f_pre, const float* C0,
-                          const float* n0, const float* m0, const void* dH, void* dQ, void* dK,
-                          void* dV, float* di, float* df, float* dC0, float* dn0, float* dm0,
-                          void* ws, cudaStream_t st) {
-  const Problem p = tc_bwd_problem(p_in);
-  BwdWs w;
-  carve(p_in, MLSTM_DT_BF16, static_cast<char*>(ws), &w);
-  cudaError_t e = launch_gates(p, i_pre, f_pre, m0, w.g, st);
-  if (e != cudaSuccess) return e;
-  e = launch_tc_states(p, K, V, C0, n0, w.g, nullptr, w.Cb, w.n_states, nullptr, nullptr, nullptr,
-                       w.seg, st);
-  if (e != cudaSuccess) return e;
-  Problem ps = p;
-  ps.signed_den = 1;  // the forward outputs keep the sign of the denominator
-  e = launch_tc_parallel(ps, Q, K, V, w.g, w.Cb, w.n_states, w.H16, w.den, w.mr, st);
-  if (e != cudaSuccess) return e;
+// The gradients of the tensor-core backward from the forward's chunk states
+// (bf16 operand copy Cb, fp32 n_states), h (bf16), signed denominators and
+// per-token stabilisers, all at 128-token chunks.
+cudaError_t bwd_tc_grads(const Problem& p, BwdWs& w, const void* Q, const void* K, const void* V,
+                         const float* i_pre, const float* f_pre, const float* C0, const float* n0,
+                         const __nv_bfloat16* Cb, const float* n_states, const __nv_bfloat16* H,
+                         const float* den, const float* mr, const void* dH, void* dQ, void* dK,
+                         void* dV, float* di, float* df, float* dC0, float* dn0, float* dm0,
+                         cudaStream_t st) {
   const long toks = (long)p.BH * p.T;
   bwd_prep_kernel<__nv_bfloat16, __nv_bfloat16><<<(unsigned)((toks + 7) / 8), kThr, 0, st>>>(
-      p, static_cast<const __nv_bfloat16*>(dH), w.H16, w.den, w.mr, nullptr, w.dA, w.dU16,
-      w.dUr16, w.g);
-  e = cudaGetLastError();
+      p, static_cast<const __nv_bfloat16*>(dH), H, den, mr, nullptr, w.dA, w.dU16, w.dUr16, w.g);
+  cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   e = launch_tc_bwd_states(p, Q, w.dUr16, w.g, w.dA, w.uvec, w.Gb, w.g_states, w.dC0, st);
   if (e != cudaSuccess) return e;
@@ -784,8 +778,8 @@ cudaError_t launch_bwd_tc(const Problem& p_in, const void* Q, const void* K, con
   if (e != cudaSuccess) return e;
   e = cudaMemsetAsync(w.kdk, 0, sizeof(float) * toks, st);
   if (e != cudaSuccess) return e;
-  e = launch_tc_bwd(p, Q, K, V, w.dU16, w.g, w.dA, w.n_states, w.g_states, w.Cb, w.Gb, w.sq, dQ,
-                    dK, dV, w.qdq, w.kdk, st);
+  e = launch_tc_bwd(p, Q, K, V, w.dU16, w.g, w.dA, n_states, w.g_states, Cb, w.Gb, w.sq, dQ, dK,
+                    dV, w.qdq, w.kdk, st);
   if (e != cudaSuccess) return e;
   bwd_gates_kernel<<<p.BH, kThr, 0, st>>>(p, i_pre, f_pre, w.qdq, w.kdk, di, df, C0, n0, w.dC0,
                                           w.dn0, dm0);
@@ -799,6 +793,43 @@ cudaError_t launch_bwd_tc(const Problem& p_in, const void* Q, const void* K, con
   if (dn0)
     e = cudaMemcpyAsync(dn0, w.dn0, sizeof(float) * p.BH * p.DK, cudaMemcpyDeviceToDevice, st);
   return e;
+}
+
+// The forward on the tensor cores at 128-token chunks, keeping what the
+// gradients need: chunk states (Cb, n_states), h in H, signed denominators
+// and stabilisers (den, mr); the final state when C_T is given.
+cudaError_t fw_tc_keep(const Problem& p, Gates g, float* seg, const void* Q, const void* K,
+                       const void* V, const float* i_pre, const float* f_pre, const float* C0,
+                       const float* n0, const float* m0, __nv_bfloat16* Cb, float* n_states,
+                       void* H, float* den, float* mr, float* C_T, float* n_T, float* m_T,
+                       cudaStream_t st) {
+  cudaError_t e = launch_gates(p, i_pre, f_pre, m0, g, st);
+  if (e != cudaSuccess) return e;
+  e = launch_tc_states(p, K, V, C0, n0, g, nullptr, Cb, n_states, C_T, n_T, m_T, seg, st);
+  if (e != cudaSuccess) return e;
+  Problem ps = p;
+  ps.signed_den = 1;  // the outputs keep the sign of the denominator
+  return launch_tc_parallel(ps, Q, K, V, g, Cb, n_states, H, den, mr, st);
+}
+
+// The backward on the tensor cores (bf16, 128-token chunks): the forward
+// recomputed on the tensor cores (gates, chunk states as the bf16 operand
+// copy, h and the signed denominator), the per-token pass (du~ in bf16, plain
+// and row-scaled), the reverse states (g~ increments, then the recurrence),
+// the squares and dq, dk, dv (tc_bwd.cu), and the gate gradients.
+cudaError_t launch_bwd_tc(const Problem& p_in, const void* Q, const void* K, const void* V,
+                          const float* i_pre, const float* f_pre, const float* C0,
+                          const float* n0, const float* m0, const void* dH, void* dQ, void* dK,
+                          void* dV, float* di, float* df, float* dC0, float* dn0, float* dm0,
+                          void* ws, cudaStream_t st) {
+  const Problem p = tc_bwd_problem(p_in);
+  BwdWs w;
+  carve(p_in, MLSTM_DT_BF16, static_cast<char*>(ws), &w);
+  cudaError_t e = fw_tc_keep(p, w.g, w.seg, Q, K, V, i_pre, f_pre, C0, n0, m0, w.Cb, w.n_states,
+                             w.H16, w.den, w.mr, nullptr, nullptr, nullptr, st);
+  if (e != cudaSuccess) return e;
+  return bwd_tc_grads(p, w, Q, K, V, i_pre, f_pre, C0, n0, w.Cb, w.n_states, w.H16, w.den, w.mr,
+                      dH, dQ, dK, dV, di, df, dC0, dn0, dm0, st);
 }
 
 template <typename TIn>
@@ -938,6 +969,103 @@ cudaError_t launch_backward(const Problem& p, mlstm_dtype dt, const void* Q, con
                                        di, df, dC0, dn0, dm0, ws, st);
   return launch_bwd_t<float>(p, dt, Q, K, V, i_pre, f_pre, C0, n0, m0, dH, dQ, dK, dV, di, df,
                              dC0, dn0, dm0, ws, st);
+}
+
+
+// ---------------------------------------------------------------------------
+// Training pair: the forward that keeps what the tensor-core backward needs,
+// and that backward without the recomputation.
+// ---------------------------------------------------------------------------
+namespace {
+
+struct Saved {
+  __nv_bfloat16* Cb;
+  float *n_states, *den, *mr;
+};
+
+// Saved buffer: the bf16 chunk states and n states entering every 128-token
+// chunk, then per token the signed denominator and the stabiliser.
+size_t saved_carve(const Problem& p_in, char* base, Saved* out) {
+  const Problem p = tc_bwd_problem(p_in);
+  const size_t BH = p.BH, T = p.T, NC = p.NC, DK = p.DK, DV = p.DV;
+  size_t off = 0;
+  auto take = [&](size_t bytes) -> char* {
+    char* ptr = base ? base + off : nullptr;
+    off += al(bytes);
+    return ptr;
+  };
+  Saved x;
+  x.Cb = reinterpret_cast<__nv_bfloat16*>(take(BH * NC * DK * DV * 2));
+  x.n_states = reinterpret_cast<float*>(take(BH * NC * DK * 4));
+  x.den = reinterpret_cast<float*>(take(BH * T * 4));
+  x.mr = reinterpret_cast<float*>(take(BH * T * 4));
+  if (out) *out = x;
+  return off;
+}
+
+// Training forward workspace: the gates and the segment end states.
+size_t fw_train_carve(const Problem& p_in, char* base, Gates* g, float** seg) {
+  const Problem p = tc_bwd_problem(p_in);
+  const size_t BH = p.BH, NC = p.NC, tpad = NC * p.L;
+  size_t off = 0;
+  auto take = [&](size_t n) -> float* {
+    float* ptr = base ? reinterpret_cast<float*>(base + off) : nullptr;
+    off += al(n * sizeof(float));
+    return ptr;
+  };
+  Gates x;
+  x.bcum = take(BH * tpad);
+  x.acol = take(BH * tpad);
+  x.amax = take(BH * tpad);
+  x.gtot = take(BH * NC);
+  x.mchk = take(BH * (NC + 1));
+  float* sg = take(tc_states_segment_floats(p));
+  if (g) *g = x;
+  if (seg) *seg = sg;
+  return off;
+}
+
+}  // namespace
+
+bool train_supported(const Problem& p, mlstm_dtype dt) { return tc_backward(p, dt); }
+size_t train_saved_bytes(const Problem& p) { return saved_carve(p, nullptr, nullptr); }
+size_t fw_train_workspace_bytes(const Problem& p) { return fw_train_carve(p, nullptr, nullptr, nullptr); }
+size_t bw_saved_workspace_bytes(const Problem& p) {
+  return carve(p, MLSTM_DT_BF16, nullptr, nullptr, true);
+}
+int fw_train_launches(const Problem& p) { return 2 + tc_states_launches(tc_bwd_problem(p)) + 1; }
+int bw_saved_launches(const Problem&) { return 2 + 1 + kTcBwdStateLaunches + kTcBwdLaunches + 1; }
+
+cudaError_t launch_fw_train(const Problem& p_in, const void* Q, const void* K, const void* V,
+                            const float* i_pre, const float* f_pre, const float* C0,
+                            const float* n0, const float* m0, void* H, float* C_T, float* n_T,
+                            float* m_T, void* saved, void* ws, cudaStream_t st) {
+  const Problem p = tc_bwd_problem(p_in);
+  Saved sv;
+  saved_carve(p_in, static_cast<char*>(saved), &sv);
+  Gates g;
+  float* seg = nullptr;
+  fw_train_carve(p_in, static_cast<char*>(ws), &g, &seg);
+  return fw_tc_keep(p, g, seg, Q, K, V, i_pre, f_pre, C0, n0, m0, sv.Cb, sv.n_states, H, sv.den,
+                    sv.mr, C_T, n_T, m_T, st);
+}
+
+cudaError_t launch_bw_saved(const Problem& p_in, const void* Q, const void* K, const void* V,
+                            const float* i_pre, const float* f_pre, const float* C0,
+                            const float* n0, const float* m0, const void* H, const void* saved,
+                            const void* dH, void* dQ, void* dK, void* dV, float* di, float* df,
+                            float* dC0, float* dn0, float* dm0, void* ws, cudaStream_t st) {
+  const Problem p = tc_bwd_problem(p_in);
+  Saved sv;
+  saved_carve(p_in, static_cast<char*>(const_cast<void*>(saved)), &sv);
+  BwdWs w;
+  carve(p_in, MLSTM_DT_BF16, static_cast<char*>(ws), &w, true);
+  // the same gates as the training forward (a function of the gate inputs)
+  cudaError_t e = launch_gates(p, i_pre, f_pre, m0, w.g, st);
+  if (e != cudaSuccess) return e;
+  return bwd_tc_grads(p, w, Q, K, V, i_pre, f_pre, C0, n0, sv.Cb, sv.n_states,
+                      static_cast<const __nv_bfloat16*>(H), sv.den, sv.mr, dH, dQ, dK, dV, di, df,
+                      dC0, dn0, dm0, st);
 }
 
 }  // namespace mlstm

@@ -29,4 +29,25 @@ cudaError_t launch_tc_bwd_states(const Problem& pb, const void* Q, const __nv_bf
                                  float* g_states, float* dC0, cudaStream_t st);
 constexpr int kTcBwdStateLaunches = 2;
 
+// Training pair (bwd.cu), for the shapes of the tensor-core backward
+// (train_supported): a forward at 128-token chunks that keeps, in a caller
+// buffer of train_saved_bytes, the bf16 chunk states, the n states and per
+// token the signed denominator and the stabiliser; and the backward that
+// takes that buffer and the forward's H instead of recomputing them.
+bool train_supported(const Problem& p, mlstm_dtype dt);
+size_t train_saved_bytes(const Problem& p);
+size_t fw_train_workspace_bytes(const Problem& p);
+size_t bw_saved_workspace_bytes(const Problem& p);
+int fw_train_launches(const Problem& p);
+int bw_saved_launches(const Problem& p);
+cudaError_t launch_fw_train(const Problem& p, const void* Q, const void* K, const void* V,
+                            const float* i_pre, const float* f_pre, const float* C0,
+                            const float* n0, const float* m0, void* H, float* C_T, float* n_T,
+                            float* m_T, void* saved, void* ws, cudaStream_t st);
+cudaError_t launch_bw_saved(const Problem& p, const void* Q, const void* K, const void* V,
+                            const float* i_pre, const float* f_pre, const float* C0,
+                            const float* n0, const float* m0, const void* H, const void* saved,
+                            const void* dH, void* dQ, void* dK, void* dV, float* di, float* df,
+                            float* dC0, float* dn0, float* dm0, void* ws, cudaStream_t st);
+
 }  // namespace mlstm

@@ -148,3 +148,54 @@ def test_python_binding_refuses_cpu_tensors():
     g = torch.zeros(1, 1, 64)
     with pytest.raises(ValueError, match="CUDA tensor"):
         mlstm_fw(x, x, x, g, g)
+
+
+def train_sizes_raw(B=1, NH=2, T=256, DK=128, DV=128, dt=_lib.DT_BF16):
+    sv, fw, bw = ctypes.c_size_t(0), ctypes.c_size_t(0), ctypes.c_size_t(0)
+    st = _lib.lib().mlstm_train_sizes(B, NH, T, DK, DV, dt, ctypes.byref(sv), ctypes.byref(fw),
+                                      ctypes.byref(bw))
+    return st, sv.value, fw.value, bw.value
+
+
+def test_train_sizes(L):
+    """The saved buffer holds the bf16 chunk states and fp32 n states of every
+    128-token chunk plus two floats per token (256-byte aligned pieces)."""
+    st, sv, fw, bw = train_sizes_raw(B=2, NH=3, T=300, DK=256, DV=512)
+    assert st == _lib.OK
+    BH, NC, T = 6, 3, 300
+    al = lambda b: (b + 255) // 256 * 256  # noqa: E731
+    assert sv == al(BH * NC * 256 * 512 * 2) + al(BH * NC * 256 * 4) + 2 * al(BH * T * 4)
+    assert fw > 0 and bw > 0
+    # no training path: fp32, d_qk 64, fewer than 128 tokens
+    assert train_sizes_raw(dt=_lib.DT_F32)[0] == _lib.ERR_UNSUPPORTED
+    assert train_sizes_raw(DK=64, DV=64)[0] == _lib.ERR_UNSUPPORTED
+    assert train_sizes_raw(T=127)[0] == _lib.ERR_UNSUPPORTED
+
+
+def test_train_pair_rejects_before_launch(L):
+    """Too small a saved buffer or workspace, unaligned or missing pointers,
+    and unsupported shapes return before any CUDA call (fake aligned pointers)."""
+    st, sv, fw, bw = train_sizes_raw()
+    assert st == _lib.OK
+    P = ctypes.c_void_p(0x10000)
+    U = ctypes.c_void_p(0x10008)  # not 16-byte aligned
+
+    def fw_call(saved_bytes=sv, ws_bytes=fw, q=P, dt=_lib.DT_BF16, DK=128):
+        return L.mlstm_fw_train(q, P, P, P, P, None, None, None, P, None, None, None, P,
+                                saved_bytes, 1, 2, 256, DK, 128, dt, _lib.GATE_EXP, P, ws_bytes,
+                                None)
+
+    def bw_call(saved_bytes=sv, ws_bytes=bw, h=P):
+        return L.mlstm_bw_saved(P, P, P, P, P, None, None, None, h, P, saved_bytes, P, P, P, P,
+                                P, P, None, None, None, 1, 2, 256, 128, 128, _lib.DT_BF16,
+                                _lib.GATE_EXP, P, ws_bytes, None)
+
+    assert fw_call(saved_bytes=sv - 1) == _lib.ERR_INVALID_ARG
+    assert fw_call(ws_bytes=fw - 1) == _lib.ERR_INVALID_ARG
+    assert fw_call(q=U) == _lib.ERR_INVALID_ARG
+    assert fw_call(q=None) == _lib.ERR_INVALID_ARG
+    assert fw_call(dt=_lib.DT_F32) == _lib.ERR_UNSUPPORTED
+    assert fw_call(DK=64) == _lib.ERR_UNSUPPORTED
+    assert bw_call(saved_bytes=sv - 1) == _lib.ERR_INVALID_ARG
+    assert bw_call(ws_bytes=bw - 1) == _lib.ERR_INVALID_ARG
+    assert bw_call(h=None) == _lib.ERR_INVALID_ARG
