@@ -21,10 +21,11 @@
 //
 // The reverse states G~_k = e^{g_k + m_k - m_{k+1}} G~_{k+1} + Q_k^T dUr_k
 // (dUr: a bf16 copy of du~ whose rows carry e^{m_k - mu_t}) run in
-// tc_bwd_rev_kernel: a CTA per 128 x 256 (or 128) tile of the state keeps the running
-// G~ in TMEM and walks the chunks from the last, writing every G~_k as the
-// bf16 operand copy (and G~_0 in fp32: the gradient of the initial state);
-// g~ follows from the per-chunk sums of e^{m_k - mu_t} da~_t q_t.
+// tc_bwd_rev_kernel: a CTA per 128 x 128 tile of the state walks the chunks
+// from the last, the chunk updates computed ahead on the tensor cores and the
+// running G~ in registers, writing every G~_k as the bf16 operand copy (and
+// G~_0 in fp32: the gradient of the initial state); g~ follows from the
+// per-chunk sums of e^{m_k - mu_t} da~_t q_t.
 //
 // Launches: one for both squares (dP and Sg, written as bf16 in the block
 // layout of cb_block_row, so that the gradient kernels can read them as K- or
@@ -36,9 +37,10 @@
 //
 // Roles (192 threads): warp 0 producer (TMA and bulk copies through a
 // 3-stage ring of 32 KB stages), warp 1 TMEM owner and MMA issuer, warps 2..5
-// the epilogue (TMEM lane = chunk row).  About 100 KB of shared memory and 256
-// TMEM columns per CTA: two CTAs share an SM, so one's epilogue overlaps the
-// other's loads.
+// the epilogue (TMEM lane = chunk row), which stages its output tile in the
+// ring's first stage (idle once every MMA has completed) for bulk / TMA
+// stores.  About 100 KB of shared memory and 256 TMEM columns per CTA: two
+// CTAs share an SM, so one's epilogue overlaps the other's loads.
 #include <cuda.h>
 
 #include "tc.h"
