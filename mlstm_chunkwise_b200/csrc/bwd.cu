@@ -65,40 +65,77 @@ __device__ __forceinline__ float ld(const TIn* base, long idx, bool ok) {
   return ok ? to_float(base[idx]) : 0.f;
 }
 
+// Two floats as one packed bf16 pair (round to nearest even).
+__device__ __forceinline__ uint32_t tc_pack_bf16x2(float lo, float hi) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
 // ---------------------------------------------------------------------------
-// du~ [BH, T, DV] (fp32 when dU is set; in bf16 for the tensor-core
-// gradients when dU16 is set, and with rows scaled by e^{m_k - mu_t} when dUr16
-// is set) and da~ [BH, T]: one warp per token.
+// du~ [BH, T, DV] (fp32) and da~ [BH, T]: one warp per token.
 // ---------------------------------------------------------------------------
 // den_s holds copysign(max(|a|, e^{-m}), a) of the forward (signed_den mode).
 template <typename TIn, typename TH>
 __global__ void __launch_bounds__(kThr)
 bwd_prep_kernel(Problem p, const TIn* __restrict__ dH, const TH* __restrict__ Hf,
                 const float* __restrict__ den_s, const float* __restrict__ mr,
-                float* __restrict__ dU, float* __restrict__ dA,
-                __nv_bfloat16* __restrict__ dU16 = nullptr,
-                __nv_bfloat16* __restrict__ dUr16 = nullptr, Gates gt = {}) {
+                float* __restrict__ dU, float* __restrict__ dA) {
   const long tok = (long)blockIdx.x * (kThr / 32) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (tok >= (long)p.BH * p.T) return;
   const float ds = den_s[tok];
   const float inv = 1.f / fabsf(ds);
-  float r = 0.f;  // e^{m_k - mu_t}, the row factor of the reverse-state update
-  if (dUr16) {
-    const long bh = tok / p.T, t = tok % p.T;
-    const float m_in = gt.mchk[bh * (p.NC + 1) + t / p.L];
-    r = expf(m_in - fmaxf(m_in, gt.amax[bh * (long)p.NC * p.L + t]));
-  }
   float dot = 0.f;
   for (int c = lane; c < p.DV; c += 32) {
     const float g = to_float(dH[tok * p.DV + c]);
-    if (dU) dU[tok * p.DV + c] = g * inv;
-    if (dU16) dU16[tok * p.DV + c] = __float2bfloat16_rn(g * inv);
-    if (dUr16) dUr16[tok * p.DV + c] = __float2bfloat16_rn(r * g * inv);
+    dU[tok * p.DV + c] = g * inv;
     dot = fmaf(g, to_float(Hf[tok * p.DV + c]), dot);
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+  if (lane == 0) {
+    const bool on_n = fabsf(ds) > expf(-mr[tok]);  // the max picked |n.q|
+    dA[tok] = on_n ? -dot * inv * (ds >= 0.f ? 1.f : -1.f) : 0.f;
+  }
+}
+
+// The tensor-core path's per-token pass (bf16 dH and h, d_v a multiple of
+// 8): du~ in bf16, plain and with the row factor e^{m_k - mu_t}, and da~.  One
+// warp per token, each lane 8 consecutive values per step (16-byte accesses).
+__global__ void __launch_bounds__(kThr)
+bwd_prep_tc_kernel(Problem p, const __nv_bfloat16* __restrict__ dH,
+                   const __nv_bfloat16* __restrict__ Hf, const float* __restrict__ den_s,
+                   const float* __restrict__ mr, Gates gt, float* __restrict__ dA,
+                   __nv_bfloat16* __restrict__ dU16, __nv_bfloat16* __restrict__ dUr16) {
+  const long tok = (long)blockIdx.x * (kThr / 32) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (tok >= (long)p.BH * p.T) return;
+  const float ds = den_s[tok];
+  const float inv = 1.f / fabsf(ds);
+  const long bh = tok / p.T, t = tok % p.T;
+  const float m_in = gt.mchk[bh * (p.NC + 1) + t / p.L];
+  const float r = expf(m_in - fmaxf(m_in, gt.amax[bh * (long)p.NC * p.L + t]));
+  const uint4* g4 = reinterpret_cast<const uint4*>(dH + tok * p.DV);
+  const uint4* h4 = reinterpret_cast<const uint4*>(Hf + tok * p.DV);
+  uint4* u4 = reinterpret_cast<uint4*>(dU16 + tok * p.DV);
+  uint4* ur4 = reinterpret_cast<uint4*>(dUr16 + tok * p.DV);
+  float dot = 0.f;
+  for (int c = lane; c < p.DV / 8; c += 32) {
+    const uint4 gv = g4[c], hv = h4[c];
+    const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w}, hw[4] = {hv.x, hv.y, hv.z, hv.w};
+    uint32_t uw[4], urw[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 g = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&gw[e]));
+      const float2 h = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&hw[e]));
+      dot = fmaf(g.x, h.x, fmaf(g.y, h.y, dot));
+      uw[e] = tc_pack_bf16x2(g.x * inv, g.y * inv);
+      urw[e] = tc_pack_bf16x2(r * g.x * inv, r * g.y * inv);
+    }
+    u4[c] = make_uint4(uw[0], uw[1], uw[2], uw[3]);
+    ur4[c] = make_uint4(urw[0], urw[1], urw[2], urw[3]);
+  }
+  dot = warp_sum(dot);
   if (lane == 0) {
     const bool on_n = fabsf(ds) > expf(-mr[tok]);  // the max picked |n.q|
     dA[tok] = on_n ? -dot * inv * (ds >= 0.f ? 1.f : -1.f) : 0.f;
@@ -765,8 +802,8 @@ cudaError_t bwd_tc_grads(const Problem& p, BwdWs& w, const void* Q, const void* 
                          void* dV, float* di, float* df, float* dC0, float* dn0, float* dm0,
                          cudaStream_t st) {
   const long toks = (long)p.BH * p.T;
-  bwd_prep_kernel<__nv_bfloat16, __nv_bfloat16><<<(unsigned)((toks + 7) / 8), kThr, 0, st>>>(
-      p, static_cast<const __nv_bfloat16*>(dH), H, den, mr, nullptr, w.dA, w.dU16, w.dUr16, w.g);
+  bwd_prep_tc_kernel<<<(unsigned)((toks + 7) / 8), kThr, 0, st>>>(
+      p, static_cast<const __nv_bfloat16*>(dH), H, den, mr, w.g, w.dA, w.dU16, w.dUr16);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   e = launch_tc_bwd_states(p, Q, w.dUr16, w.g, w.dA, w.uvec, w.Gb, w.g_states, w.dC0, st);
