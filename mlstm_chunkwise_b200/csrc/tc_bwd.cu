@@ -90,7 +90,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 tc_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_du,
               const __grid_constant__ CUtensorMap tm_out, const TcBwdArgs a) {
-  static_assert(NT == 64 || NT == 128, "output tile");
+  static_assert(NT == 128, "output tiles of 128 columns (d_qk and d_v are multiples of 128)");
   const Problem& p = a.p;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
