@@ -95,3 +95,31 @@ def test_train_pair_unsupported_shapes():
         api.mlstm_fw_train(d["Q"].float(), d["K"].float(), d["V"].float(), d["i_pre"],
                            d["f_pre"])
     assert e.value.status == _lib.ERR_UNSUPPORTED
+
+
+def test_train_pair_full_size():
+    """The 7B-shaped batch (B=8, NH=8, T=8192, 256 x 512 heads) through the pair:
+    H and the final state of two heads against the oracle, and the saved
+    backward against the recomputing one over the whole batch (bit for bit on
+    dQ, dK, dV; the gate gradients up to summation order)."""
+    w = WORKLOADS["xlstm7b"]
+    x = make_inputs(w)
+    d = parity.to_dev(x)
+    dH = torch.randn((w.B, w.NH, w.T, w.DV), generator=torch.Generator().manual_seed(81),
+                     dtype=torch.float32).to(torch.bfloat16).cuda()
+    H, fin, saved = api.mlstm_fw_train(d["Q"], d["K"], d["V"], d["i_pre"], d["f_pre"],
+                                       gate_mode=w.gate_mode)
+    g_saved = api.mlstm_bw_saved(d["Q"], d["K"], d["V"], d["i_pre"], d["f_pre"], H, saved, dH,
+                                 gate_mode=w.gate_mode)
+    del saved
+    g_rec = api.mlstm_bw(d["Q"], d["K"], d["V"], d["i_pre"], d["f_pre"], dH,
+                         chunk_size=w.chunk_size, gate_mode=w.gate_mode)
+    torch.cuda.synchronize()
+    assert api.last_device_error() == _lib.OK
+    for k in ("dQ", "dK", "dV"):
+        assert torch.equal(g_saved[k], g_rec[k]), k
+    for k in ("di_pre", "df_pre"):
+        torch.testing.assert_close(g_saved[k], g_rec[k], rtol=1e-4, atol=1e-5)
+    heads = [(0, 0), (w.B - 1, w.NH - 1)]
+    ref = parity.oracle_run(x, w.gate_mode, heads=heads)
+    parity.compare(H, fin, ref, parity.TOL[w.dtype], heads=heads, label="fw_train/full")
