@@ -130,7 +130,7 @@ MEASURED_TRAFFIC = {
     ("tc_states", "xlstm7b"): {
         "bytes": 1.326e9, "profile": "profiles/tc_unfused_xlstm7b.md",
         "sources": ["tc_states.cu", "tc_ptx.cuh", "tc.h", "common.cuh"],
-        "sha1": "64f549befc01d79047227790c36aa26b5ebd9b82"},
+        "sha1": "80a7f9648cf41451a6ddc8bc3d98b992bee86cc3"},
 }
 
 

@@ -28,6 +28,13 @@
 // and tc_states_fixup_kernel adds that term, with the states C_{k0} entering
 // each segment obtained by a short scan over the segments' end states.
 //
+// For d_qk = 128 and value tiles of at most 128 columns the running state
+// fits the workers' registers (a row and half of the tile's columns each, 64
+// values at most): there the MMAs write each chunk's update U_k into one of
+// two TMEM buffers, and per chunk the workers store the state from registers,
+// then fold in the update, C_{k+1} = decay C_k + U_k, and release the buffer,
+// so the MMAs of the next chunk wait for no decay of a TMEM master.
+//
 // Roles (320 threads): warp 0 TMA producer, warp 1 TMEM owner + MMA issuer,
 // warps 2..9 workers: per chunk, the store and decay of the master state; per
 // stage, one pass that computes its token weights, accumulates the n-vector
@@ -78,7 +85,12 @@ struct SCfg {
   static constexpr uint32_t kBytes = kOffSlot + 16;
   static constexpr uint32_t kSmem = kBytes + 1024;
   static_assert(kSmem <= 227 * 1024, "shared memory");
-  static constexpr uint32_t kTmemCols = (kHalves * DVT) < 32 ? 32 : kHalves * DVT;
+  // d_qk = 128 with value tiles of at most 128 columns: the running state
+  // lives in the workers' registers (64 values a thread at most) and the MMAs
+  // write each chunk's update into one of two TMEM buffers (see the workers).
+  static constexpr bool kReg = DK == 128 && DVT <= 128;
+  static constexpr uint32_t kTmemCols =
+      kReg ? 2 * DVT : ((kHalves * DVT) < 32 ? 32 : kHalves * DVT);
 };
 
 struct SBars {
@@ -174,7 +186,31 @@ tc_states_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
       constexpr uint32_t idesc = idesc_bf16(128, DVT, 1, 1);
       bool ok = true;
       int n = 0;
-      for (int k = 0; k < nk && ok; ++k) {
+      if constexpr (S::kReg) {
+        // chunk k's update U_k into buffer k mod 2, once the workers have
+        // folded U_{k-2} (the release of that buffer)
+        for (int k = 0; k < nk && ok; ++k) {
+          const int buf = k & 1;
+          if (k >= 2) ok = mbar_wait(bar.master(buf), ((k - 2) >> 1) & 1, p, 2);
+          if (!ok) break;
+          tc_fence_after();
+          for (int j = 0; j < stages_per_chunk && ok; ++j, ++n) {
+            const int s = n % S::kStages;
+            ok = mbar_wait(bar.kready(s), (n / S::kStages) & 1, p, 3);
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t st = sbase + S::kOffStage + (uint32_t)s * S::kStageBytes;
+#pragma unroll
+            for (int kk = 0; kk < kStageTok / 16; ++kk)
+              mma_bf16_ss(tmem + (uint32_t)(buf * DVT), sdesc_sw128(st + kk * 2048, 8192, 1024),
+                          sdesc_sw128(st + S::kKBytes + kk * 2048, 8192, 1024), idesc,
+                          (j | kk) ? 1u : 0u);
+            mma_commit(bar.empty(s));
+          }
+          mma_commit(bar.chunk(buf));
+        }
+      }
+      for (int k = 0; k < nk && ok && !S::kReg; ++k) {
         for (int j = 0; j < stages_per_chunk && ok; ++j, ++n) {
           const int s = n % S::kStages;
           ok = mbar_wait(bar.kready(s), (n / S::kStages) & 1, p, 3);
@@ -228,8 +264,15 @@ tc_states_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
     float part[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // n partials, this chunk
     bool ok = true;
 
+    // kReg: the running state, row r and this worker's column half
+    float creg[S::kReg ? kColsPer : 1];
+    if constexpr (S::kReg) {
+#pragma unroll
+      for (int j = 0; j < kColsPer; ++j)
+        creg[j] = (C0 && seg == 0) ? C0[((long)bh * DK + r) * DV + dv0 + ch * kColsPer + j] : 0.f;
+    }
     // master <- C0 (or zero): row r of each half, this worker's column half
-    for (int hf = 0; hf < S::kHalves; ++hf) {
+    for (int hf = 0; hf < S::kHalves && !S::kReg; ++hf) {
       const int dk = hf * 128 + r;
       for (int c = 0; c < kColsPer; c += 32) {
         const int col = ch * kColsPer + c;
@@ -332,10 +375,17 @@ tc_states_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
     };
 
     int n = 0;
+    // the chunk's gate scalars, loaded one chunk ahead (they open every
+    // iteration's dependence chain)
+    float nx_m_in = mchk[k0], nx_m_out = mchk[k0 + 1], nx_gk = g.gtot[(long)bh * NC + k0];
     for (int k = k0; k < k1 && ok; ++k) {
       if (k > k0) fold_n();  // chunk k - 1's partials: every worker has passed its stages
-      const float m_in = mchk[k], m_out = mchk[k + 1];
-      const float gk = g.gtot[(long)bh * NC + k];
+      const float m_in = nx_m_in, m_out = nx_m_out, gk = nx_gk;
+      if (k + 1 < k1) {
+        nx_m_in = m_out;
+        nx_m_out = mchk[k + 2];
+        nx_gk = g.gtot[(long)bh * NC + k + 1];
+      }
       const float decay = expf(gk + m_in - m_out);
       if (n_mine) n_states[((long)bh * NC + k) * DK + wt] = nval;
       nval *= decay;
@@ -344,6 +394,58 @@ tc_states_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
       stage_pass(n++, gk, m_out);
       named_bar_sync(1, kWorkers);  // the n-partial reads are done: store tiles free
 
+      if constexpr (S::kReg) {
+        // The state entering chunk k is in registers: store it (this warp's
+        // tiles, as below), weight the rest of the chunk's stages, then fold in
+        // the chunk's update, C_{k+1} = decay C_k + U_k, and release its buffer.
+        const int dk0 = q * 32;
+        if (Cb) {
+          for (int c = 0; c < kColsPer; c += 64) {
+            const int col = ch * kColsPer + c;
+            if (lane == 0) tma_store_wait_read_all();  // the previous tile has been read
+            __syncwarp();
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const float* x = creg + c + 8 * j;
+              *reinterpret_cast<uint4*>(stg + lane * 128 + ((j ^ (lane & 7)) << 4)) =
+                  make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]),
+                             pack_bf16x2(x[4], x[5]), pack_bf16x2(x[6], x[7]));
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              bulk_store(Cb + cb_block_row((long)bh * NC + k, (dv0 + col) / 64, dk0, DK, DV / 64),
+                         stg_u, 4096);
+              tma_store_commit();
+            }
+          }
+        } else if (C_states) {
+          for (int c = 0; c < kColsPer; c += 32) {
+            const int col = ch * kColsPer + c;
+            uint32_t v[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(creg[c + j]);
+            store_tile(&tm_cs, *reinterpret_cast<const uint32_t(*)[16]>(v), dv0 + col, dk0,
+                       bh * NC + k);
+            store_tile(&tm_cs, *reinterpret_cast<const uint32_t(*)[16]>(v + 16), dv0 + col + 16,
+                       dk0, bh * NC + k);
+          }
+        }
+        for (int j = 1; j < stages_per_chunk && ok; ++j) stage_pass(n++, gk, m_out);
+        const int kl = k - k0, buf = kl & 1;
+        ok = ok && mbar_wait(bar.chunk(buf), (kl >> 1) & 1, p, 4);
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < kColsPer; c += 32) {
+          uint32_t v[32];
+          tmem_ld32(trow + (uint32_t)(buf * DVT + ch * kColsPer + c), v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) creg[c + j] = fmaf(decay, creg[c + j], __uint_as_float(v[j]));
+        }
+        tc_fence_before();
+        mbar_arrive(bar.master(buf));
+      } else {
       // The state entering chunk k, half by half (row halves of d_qk): store it
       // (from this warp's tiles), then decay it in place.  Half hf waits only
       // for its own MMAs of chunk k - 1 and releases itself to the MMAs of
@@ -410,9 +512,12 @@ tc_states_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
       }
 
       for (int j = 1; j < stages_per_chunk && ok; ++j) stage_pass(n++, gk, m_out);
+      }
     }
-    // final state (fold the last chunk's n partials first)
-    for (int hf = 0; hf < S::kHalves && ok; ++hf) ok = mbar_wait(bar.chunk(hf), (nk - 1) & 1, p, 6);
+    // final state (fold the last chunk's n partials first); kReg: the last
+    // fold has already waited for the last update
+    for (int hf = 0; hf < S::kHalves && ok && !S::kReg; ++hf)
+      ok = mbar_wait(bar.chunk(hf), (nk - 1) & 1, p, 6);
     tc_fence_after();
     fold_n();
     // The last segment's end state is C_T (local when segmented: the fix-up
@@ -424,8 +529,13 @@ tc_states_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         for (int c = 0; c < kColsPer; c += 32) {
           const int col = ch * kColsPer + c;
           uint32_t v[32];
-          tmem_ld32(trow + hf * DVT + col, v);
-          tmem_wait_ld();
+          if constexpr (S::kReg) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(creg[c + j]);
+          } else {
+            tmem_ld32(trow + hf * DVT + col, v);
+            tmem_wait_ld();
+          }
           float* row_dst =
               last_seg ? C_T + ((long)bh * DK + dk) * DV + dv0 + col
                        : seg_C + ((((long)bh * gridDim.x + blockIdx.x) * (n_seg - 1) + seg) * DK + dk) *
