@@ -744,9 +744,21 @@ def run_bw(args):
     dH = torch.randn((w.B, w.NH, w.T, w.DV), generator=g).to(w.torch_dtype).to(dev)
     B, NH, T, DK, DV, L = w.B, w.NH, w.T, w.DK, w.DV, w.chunk_size
 
+    saved = None
+    if args.saved:
+        # the training pair's backward: the training forward once, untimed
+        if api.train_sizes(B, NH, T, DK, DV, w.torch_dtype) is None:
+            raise SystemExit("--saved: this shape has no training pair")
+        H, _, saved = api.mlstm_fw_train(d["Q"], d["K"], d["V"], d["i_pre"], d["f_pre"],
+                                         d["C0"], d["n0"], d["m0"], gate_mode=w.gate_mode)
+
     def step():
-        api.mlstm_bw(d["Q"], d["K"], d["V"], d["i_pre"], d["f_pre"], dH, d["C0"], d["n0"],
-                     d["m0"], chunk_size=L, gate_mode=w.gate_mode)
+        if saved is not None:
+            api.mlstm_bw_saved(d["Q"], d["K"], d["V"], d["i_pre"], d["f_pre"], H, saved, dH,
+                               d["C0"], d["n0"], d["m0"], gate_mode=w.gate_mode)
+        else:
+            api.mlstm_bw(d["Q"], d["K"], d["V"], d["i_pre"], d["f_pre"], dH, d["C0"], d["n0"],
+                         d["m0"], chunk_size=L, gate_mode=w.gate_mode)
 
     warm = max(3, args.warmup)
     for _ in range(warm):
@@ -777,11 +789,14 @@ def run_bw(args):
              and T >= 128)
     Lb = 128 if tc_bw else L
     fph = flops_per_head(T, DK, DV, Lb)
-    fw_flops = B * NH * (fph["states"] + fph["inter"] + fph["intra"])
+    # the saved backward recomputes nothing: its FLOPs are the gradient kernels'
+    fw_flops = 0.0 if saved is not None else B * NH * (fph["states"] + fph["inter"] + fph["intra"])
     bw_flops = B * NH * bw_flops_per_head(T, DK, DV, Lb)
     achieved = (fw_flops + bw_flops) / (ms / 1e3) / 1e12
     if tc_bw:
-        algo, bound, peak = "bw (tensor cores, 128-token chunks)", "tensor", peaks["bf16_tflops"]
+        algo = ("bw from the training pair's saved buffer" if saved is not None
+                else "bw (tensor cores, 128-token chunks)")
+        bound, peak = "tensor", peaks["bf16_tflops"]
         peak_source = f"bf16_tflops (of {peak_src})"
     else:
         algo, bound = "bw (fp32 CUDA-core kernels)", "alu"
@@ -893,6 +908,8 @@ def main():
                     help="skip the host-buffer end-to-end loop (profiling runs)")
     ap.add_argument("--batch", type=int, default=0,
                     help="override the workload's batch size (smaller profiling captures)")
+    ap.add_argument("--saved", action="store_true",
+                    help="with --op bw: time mlstm_bw_saved (the training pair's backward)")
     ap.add_argument("--op", default="fw", choices=["fw", "step", "bw", "train"],
                     help="fw: the forward pass (default); step: the single-token step; "
                          "bw: the backward pass; train: forward + backward through autograd")
