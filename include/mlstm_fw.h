@@ -313,9 +313,11 @@ const char* mlstm_kernel_name(int id);
  * problem whose mlstm_fw_workspace_size() is larger returns
  * MLSTM_ERR_SCRATCH_TOO_SMALL and launches nothing.  All calls share the one
  * array, so calls that overlap on the GPU (other streams or host threads)
- * race and must be serialised by the caller.  The first call on a device looks
- * up the array's address with that device current; make it before any stream
- * capture.  Other errors are those of mlstm_fw(). */
+ * race and must be serialised by the caller.  The first call in a CUDA context
+ * looks up the array's address with that context current and caches it for
+ * that context; make it before any stream capture.  After a cudaDeviceReset
+ * (which ends the context) the next call looks the address up again.  Other
+ * errors are those of mlstm_fw(). */
 mlstm_status mlstm_fw_static_scratch(const void* Q, const void* K, const void* V,
                                      const float* i_pre, const float* f_pre, const float* C0,
                                      const float* n0, const float* m0, void* H, float* C_T,

@@ -10,6 +10,7 @@
 #include <vector>
 
 #include "common.cuh"
+#include "device_address.h"
 #include "tc.h"
 #include "tc_bwd.h"
 
@@ -26,19 +27,12 @@ constexpr size_t kAlign = 256;
 inline size_t round_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// Largest device count this library keeps a cached error-word address for.
-constexpr int kMaxDevices = 64;
-uint32_t* g_err_ptr[kMaxDevices] = {};
-
+// Address of g_error_word in the current context (nullptr if it cannot be
+// looked up).
+DeviceAddressCache g_err_cache;
 uint32_t* error_word_ptr() {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-  if (!g_err_ptr[dev]) {
-    void* ptr = nullptr;
-    if (cudaGetSymbolAddress(&ptr, g_error_word) != cudaSuccess) return nullptr;
-    g_err_ptr[dev] = static_cast<uint32_t*>(ptr);
-  }
-  return g_err_ptr[dev];
+  return static_cast<uint32_t*>(cached_device_address(
+      g_err_cache, [](void** p) { return cudaGetSymbolAddress(p, g_error_word); }));
 }
 
 mlstm_status check_sizes(int B, int NH, int T, int DK, int DV, int L) {
@@ -93,7 +87,7 @@ Layout layout_for(const Problem& p, mlstm_algo a, Mode mode) {
   Layout l{};
   const size_t BH = (size_t)p.BH, tpad = (size_t)p.NC * p.L;
   l.gates_bytes = 3 * round_up(BH * tpad * sizeof(float)) + round_up(BH * p.NC * sizeof(float)) +
-                  round_up(BH * (p.NC + 1) * sizeof(float));
+                  round_up(BH * (p.NC + 1) * sizeof(float)) + 4 * round_up(BH * p.NC * 4);
   const size_t n_bytes = round_up(BH * p.NC * (size_t)p.DK * sizeof(float));
   if (mode == Mode::kFull && a == MLSTM_ALGO_SIMT)
     l.states_bytes = round_up(BH * p.NC * (size_t)p.DK * p.DV * sizeof(float)) + n_bytes;
@@ -108,7 +102,10 @@ Layout layout_for(const Problem& p, mlstm_algo a, Mode mode) {
 }
 
 // Carves the gate arrays out of `ws`; returns the first byte after them.
-char* carve_gates(const Problem& p, char* ws, Gates* g, float* mchk_override) {
+// `dominance`: the gate kernels also mark the chunks whose entering state one
+// token dominates (used by the tensor-core paths that hand states on in bf16).
+char* carve_gates(const Problem& p, char* ws, Gates* g, float* mchk_override,
+                  bool dominance = false) {
   const size_t BH = (size_t)p.BH, tpad = (size_t)p.NC * p.L;
   g->bcum = reinterpret_cast<float*>(ws);
   ws += round_up(BH * tpad * sizeof(float));
@@ -120,6 +117,14 @@ char* carve_gates(const Problem& p, char* ws, Gates* g, float* mchk_override) {
   ws += round_up(BH * p.NC * sizeof(float));
   g->mchk = mchk_override ? mchk_override : reinterpret_cast<float*>(ws);
   ws += round_up(BH * (p.NC + 1) * sizeof(float));
+  g->csum = dominance ? reinterpret_cast<float*>(ws) : nullptr;
+  ws += round_up(BH * p.NC * 4);
+  g->cidx = dominance ? reinterpret_cast<int*>(ws) : nullptr;
+  ws += round_up(BH * p.NC * 4);
+  g->dom = dominance ? reinterpret_cast<int*>(ws) : nullptr;
+  ws += round_up(BH * p.NC * 4);
+  g->mdom = dominance ? reinterpret_cast<float*>(ws) : nullptr;
+  ws += round_up(BH * p.NC * 4);
   return ws;
 }
 
@@ -338,7 +343,7 @@ mlstm_status mlstm_fw(const void* Q, const void* K, const void* V, const float* 
 
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   Gates g;
-  char* rest = carve_gates(p, static_cast<char*>(workspace), &g, nullptr);
+  char* rest = carve_gates(p, static_cast<char*>(workspace), &g, nullptr, a != MLSTM_ALGO_SIMT);
   s = from_cuda(launch_family(MLSTM_KERNEL_GATES, gate_launches(p), st,
                               [&] { return launch_gates(p, i_pre, f_pre, m0, g, st); }));
   if (s != MLSTM_OK) return s;
@@ -444,14 +449,15 @@ mlstm_status mlstm_fw_parallel(const void* Q, const void* K, const void* V, cons
   if (!p.err) return MLSTM_ERR_CUDA;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   Gates g;
-  char* rest = carve_gates(p, static_cast<char*>(workspace), &g, nullptr);
+  char* rest = carve_gates(p, static_cast<char*>(workspace), &g, nullptr, a == MLSTM_ALGO_TC);
   s = from_cuda(launch_family(MLSTM_KERNEL_GATES, gate_launches(p), st,
                               [&] { return launch_gates(p, i_pre, f_pre, m0, g, st); }));
   if (s != MLSTM_OK) return s;
   if (a == MLSTM_ALGO_TC) {
     __nv_bfloat16* Cb = reinterpret_cast<__nv_bfloat16*>(rest);
     s = from_cuda(launch_family(MLSTM_KERNEL_TC_PARALLEL, 1, st, [&] {
-      cudaError_t e = launch_states_to_operand(C_states, Cb, (long)p.BH * p.NC, DK, DV, st);
+      cudaError_t e = launch_states_to_operand(C_states, Cb, (long)p.BH * p.NC, DK, DV, st,
+                                               n_states, V, g.dom, p);
       if (e != cudaSuccess) return e;
       return launch_tc_parallel(p, Q, K, V, g, Cb, n_states, H, n_out, m_out, st);
     }));

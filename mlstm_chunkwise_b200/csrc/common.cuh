@@ -42,12 +42,27 @@ struct Problem {
 //   amax [BH, NC*L]  running max of acol inside the chunk (prefix max)
 //   gtot [BH, NC]    chunk total of log forget gates (= bcum at the chunk end)
 //   mchk [BH, NC+1]  state stabiliser entering chunk k (k = NC: final m)
+// Dominance of the state entering each chunk (forward paths only; null
+// elsewhere):
+//   csum [BH, NC]    sum_s e^{acol_s - amax_{L-1}} over the chunk's tokens
+//   cidx [BH, NC]    index (within the chunk) of the chunk's largest acol
+//   dom  [BH, NC]    the token t* (0 <= t* < T) that holds more than half of
+//                    the total gate weight of the state entering chunk k, or
+//                    -1.  Such a state is close to rank one, C_k ~ n_k v_{t*}^T,
+//                    and the tensor-core paths then hand it on as
+//                    R_k = C_k - n*_k v_{t*}^T (see tc.h).
+//   mdom [BH, NC]    the log-weight of the largest term of that state (t*'s
+//                    when dom >= 0), in the unstabilised frame
 struct Gates {
-  float* bcum;
-  float* acol;
-  float* amax;
-  float* gtot;
-  float* mchk;
+  float* bcum = nullptr;
+  float* acol = nullptr;
+  float* amax = nullptr;
+  float* gtot = nullptr;
+  float* mchk = nullptr;
+  float* csum = nullptr;
+  int* cidx = nullptr;
+  int* dom = nullptr;
+  float* mdom = nullptr;
 };
 
 __device__ __forceinline__ float to_float(float x) { return x; }

@@ -17,6 +17,17 @@
 // Kernel 1 (gates_chunk_kernel): one CTA per (chunk, b*h); block-wide scans.
 // Kernel 2 (gates_state_kernel): one warp per b*h; warp scan of the (max,+)
 // maps over chunks.
+//
+// Dominance (when g.dom is given).  The state entering chunk k is a sum of
+// per-token terms with log-weights lw_j = li_j + (sum of lf after j), plus the
+// initial state with log-weight m0 + (sum of lf) when one is given.  Let M_k
+// be the largest of them (the same (max,+) recurrence as m, started from m0
+// with an initial state and from -inf without one, and carrying the index of
+// the token that attains it) and z_k = sum_j e^{lw_j - M_k} >= 1 (an affine
+// recurrence over chunks, z_{k+1} = e^{g_k + M_k - M_{k+1}} z_k +
+// e^{g_k + amax_{L-1} - M_{k+1}} csum_k).  When z_k < 2 one term holds more than
+// half of the weight: then dom_k is that token (or -1 if it is the initial
+// state).
 #include <math.h>
 
 #include "common.cuh"
@@ -117,6 +128,51 @@ gates_chunk_kernel(Problem p, const float* __restrict__ i_pre, const float* __re
       if (r == L - 1) g.gtot[(long)bh * p.NC + k] = lcum[e];
     }
   }
+  if (!g.dom) return;
+  // The chunk's largest column log-weight (the inclusive max at its end), the
+  // first token that attains it, and sum_s e^{acol_s - max}.
+  __shared__ float cmax_s;
+  __shared__ float sum_s[kGateThreads / 32];
+  __shared__ int idx_s[kGateThreads / 32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int e = 0; e < kMaxPerThread; ++e) {
+    if (e >= per) break;
+    if (first + e == L - 1) cmax_s = fmaxf(li[e], moff);  // amax is a running max
+  }
+  __syncthreads();
+  const float cmax = cmax_s;
+  float sum = 0.f;
+  int idx = L;
+#pragma unroll
+  for (int e = 0; e < kMaxPerThread; ++e) {
+    if (e >= per) break;
+    const int r = first + e;
+    if (r < L) {
+      sum += expf(acol[e] - cmax);  // -inf (padding) -> 0
+      if (acol[e] == cmax && r < idx) idx = r;
+    }
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) {
+    sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    idx = min(idx, __shfl_xor_sync(0xffffffffu, idx, o));
+  }
+  if (lane == 0) {
+    sum_s[warp] = sum;
+    idx_s[warp] = idx;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float tot = 0.f;
+    int best = L;
+    for (int w = 0; w < kGateThreads / 32; ++w) {
+      tot += sum_s[w];
+      best = min(best, idx_s[w]);
+    }
+    g.csum[(long)bh * p.NC + k] = tot;
+    g.cidx[(long)bh * p.NC + k] = best < L ? best : 0;
+  }
 }
 
 // One warp per (b, h): m_{k+1} = max(m_k + g_k, c_k) with c_k = g_k + amax at
@@ -149,6 +205,76 @@ __global__ void gates_state_kernel(Problem p, const float* __restrict__ m0, Gate
     const float m = fmaxf(carry + G, C);
     if (k < p.NC) mchk[k + 1] = m;
     carry = __shfl_sync(0xffffffffu, m, 31);
+  }
+  if (!g.dom) return;
+
+  // Dominance: M_k with the index of the term that attains it (-1: the
+  // initial state), then z_k.  dom_0 = -1: the state entering the first chunk
+  // is the initial state alone (or zero).
+  int* dom = g.dom + (long)bh * p.NC;
+  float* mdom = g.mdom + (long)bh * p.NC;
+  if (lane == 0 && p.NC > 0) {
+    dom[0] = -1;
+    mdom[0] = m0 ? m0[bh] : -INFINITY;
+  }
+  float cM = m0 ? m0[bh] : -INFINITY, cz = m0 ? 1.f : 0.f;
+  int cI = -1;
+  for (int k0 = 0; k0 < p.NC; k0 += 32) {
+    const int k = k0 + lane;
+    float gk = 0.f, G = 0.f, C = -INFINITY, amx = -INFINITY, cs = 0.f;
+    int I = -1;
+    if (k < p.NC) {
+      gk = G = g.gtot[(long)bh * p.NC + k];
+      amx = g.amax[(long)bh * tpad + (long)k * p.L + p.L - 1];
+      C = G + amx;
+      I = k * p.L + g.cidx[(long)bh * p.NC + k];
+      cs = g.csum[(long)bh * p.NC + k];
+    }
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const float Ge = __shfl_up_sync(0xffffffffu, G, o);
+      const float Ce = __shfl_up_sync(0xffffffffu, C, o);
+      const int Ie = __shfl_up_sync(0xffffffffu, I, o);
+      if (lane >= o) {
+        if (Ce + G > C) {
+          C = Ce + G;
+          I = Ie;
+        }
+        G = G + Ge;
+      }
+    }
+    // M_{k+1} and its index; M_k is the previous lane's (or the carry)
+    float Mo = C;
+    int Io = I;
+    if (cM + G >= C) {
+      Mo = cM + G;
+      Io = cI;
+    }
+    float Mi = __shfl_up_sync(0xffffffffu, Mo, 1);
+    if (lane == 0) Mi = cM;
+    // z_{k+1} = a z_k + b, scanned as affine maps
+    float a = 1.f, b = 0.f;
+    if (k < p.NC) {
+      a = Mi == -INFINITY ? 0.f : expf(gk + Mi - Mo);
+      b = expf(gk + amx - Mo) * cs;
+    }
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const float ae = __shfl_up_sync(0xffffffffu, a, o);
+      const float be = __shfl_up_sync(0xffffffffu, b, o);
+      if (lane >= o) {
+        b = fmaf(a, be, b);
+        a = a * ae;
+      }
+    }
+    const float z = fmaf(a, cz, b);
+    if (k + 1 < p.NC) {
+      dom[k + 1] = (z < 2.f) ? Io : -1;
+      mdom[k + 1] = Mo;
+    }
+    cM = __shfl_sync(0xffffffffu, Mo, 31);
+    cI = __shfl_sync(0xffffffffu, Io, 31);
+    cz = __shfl_sync(0xffffffffu, z, 31);
   }
 }
 

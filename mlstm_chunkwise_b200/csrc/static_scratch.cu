@@ -16,40 +16,32 @@
 //  * all calls share the one array: calls that overlap on the GPU (other
 //    streams, other host threads) race with each other and must be serialised
 //    by the caller;
-//  * the first call on a device looks up the array's device address (with
-//    that device current) and caches it; make that first call before any
-//    stream capture.
+//  * the first call in a CUDA context looks up the array's device address
+//    (with that context current) and caches it for that context; make that
+//    first call before any stream capture.  A cudaDeviceReset ends the
+//    context, and the next call looks the address up again in the new one.
 // The array keeps whatever the last call left in it.  Nothing needs clearing:
 // every scratch byte a call reads was written earlier in the same call.
 #include <cuda_runtime.h>
 #include <stdint.h>
 
-#include <mutex>
-
+#include "device_address.h"
 #include "mlstm_fw.h"
 
 namespace {
 
 constexpr size_t kStaticScratchBytes = size_t(16) << 20;
-constexpr int kMaxScratchDevices = 64;
 
 static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
 
-std::mutex g_scratch_mu;
-void* g_scratch_ptr[kMaxScratchDevices] = {};
+mlstm::DeviceAddressCache g_scratch_cache;
 
-// Device address of g_static_scratch on the current device (looked up once per
-// device); nullptr if the lookup fails.
+// Device address of g_static_scratch in the current context (looked up once
+// per context); nullptr, with the runtime's error cleared, if the lookup
+// fails.
 void* scratch_address() {
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxScratchDevices) return nullptr;
-  std::lock_guard<std::mutex> lk(g_scratch_mu);
-  if (!g_scratch_ptr[dev]) {
-    void* ptr = nullptr;
-    if (cudaGetSymbolAddress(&ptr, g_static_scratch) != cudaSuccess || !ptr) return nullptr;
-    g_scratch_ptr[dev] = ptr;
-  }
-  return g_scratch_ptr[dev];
+  return mlstm::cached_device_address(
+      g_scratch_cache, [](void** p) { return cudaGetSymbolAddress(p, g_static_scratch); });
 }
 
 }  // namespace

@@ -17,7 +17,10 @@
 // The fp32 master state C lives in TMEM for the whole sequence of a head; the
 // Q~ C_k MMA reads a bf16 copy of it that the row threads write into shared
 // memory once per chunk (together with the decay of the master).  The n
-// vector is carried in shared memory by the row threads.
+// vector is carried in shared memory by the row threads.  For a chunk whose
+// entering state one token t* dominates (g.dom), the copy holds C_k - n*_k
+// v_{t*}^T, the denominator uses n*_k and the epilogue adds (n*_k^T q~) v_{t*}
+// in fp32 (n* = n - d, d the rounding residual of t*'s weighted key; tc.h).
 //
 // Roles (352 threads): warp 0 TMA producer; warp 1 TMEM owner and MMA issuer;
 // warp 2 stores H (a TMA store per chunk, then it releases the Q buffer the
@@ -61,10 +64,12 @@ struct FCfg {
   static constexpr uint32_t kOffC = kOffV + kVBufs * kVBytes;
   static constexpr uint32_t kOffRedN = kOffC + kCBytes;                  // float[kRG][kDK]
   static constexpr uint32_t kOffN = kOffRedN + kRG * kDK * 4;            // float[kDK]
+  static constexpr uint32_t kOffNPrev = kOffN + kDK * 4;                 // float[kDK]: n_k
+  static constexpr uint32_t kOffDStar = kOffNPrev + kDK * 4;             // float[kDK]: d_k
   // per chunk (2 buffers) and key column: acol, e^{acol - c}, the weight w
-  static constexpr uint32_t kOffAcol = kOffN + kDK * 4;                  // float[2][3][kL]
-  static constexpr uint32_t kOffRed = kOffAcol + 2 * 3 * kL * 4;         // float[256]
-  static constexpr uint32_t kOffBar = kOffRed + 256 * 4;
+  static constexpr uint32_t kOffAcol = kOffDStar + kDK * 4;              // float[2][3][kL]
+  static constexpr uint32_t kOffRed = kOffAcol + 2 * 3 * kL * 4;         // float2[256]
+  static constexpr uint32_t kOffBar = kOffRed + 256 * 8;
   static constexpr uint32_t kOffTmemSlot = kOffBar + 256;
   static constexpr uint32_t kBytes = kOffTmemSlot + 16;
   static constexpr uint32_t kSmem = kBytes + 1024;
@@ -104,7 +109,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 tc_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_h,
                 Problem p, Gates g, const float* __restrict__ C0, const float* __restrict__ n0,
-                float* __restrict__ C_T, float* __restrict__ n_T, float* __restrict__ m_T) {
+                float* __restrict__ C_T, float* __restrict__ n_T, float* __restrict__ m_T,
+                const __nv_bfloat16* __restrict__ Vraw, const __nv_bfloat16* __restrict__ Kraw) {
   using F = FCfg<DV>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -113,8 +119,10 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   const FBars bar{sbase + F::kOffBar};
   float* redn_s = reinterpret_cast<float*>(smem + F::kOffRedN);
   float* n_s = reinterpret_cast<float*>(smem + F::kOffN);
+  float* nprev_s = reinterpret_cast<float*>(smem + F::kOffNPrev);
+  float* dstar_s = reinterpret_cast<float*>(smem + F::kOffDStar);
   float* acol_s = reinterpret_cast<float*>(smem + F::kOffAcol);
-  float* red_s = reinterpret_cast<float*>(smem + F::kOffRed);
+  float2* red_s = reinterpret_cast<float2*>(smem + F::kOffRed);
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + F::kOffTmemSlot);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -324,11 +332,13 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     struct Rows {
       float m_in, m_out, mu, bc, gk, decay, rowf;
       bool sep;
+      int bh, td;  // td: dominant token of the chunk's entering state, or -1
     };
     // Gate values of a chunk, loaded two chunks ahead of their use (the
     // loads stay in flight while the chunk in between is processed).
     struct Raw {
       float m_in, m_out, amax, bc, gk, acol, amax0, amax_last;
+      int bh, k, td;
     };
     auto load_raw = [&](const FChunk& c) -> Raw {
       Raw v;
@@ -341,6 +351,9 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       v.acol = rt < kL ? g.acol[base + rt] : 0.f;
       v.amax0 = g.amax[base];
       v.amax_last = g.amax[base + kL - 1];
+      v.bh = c.bh;
+      v.k = c.k;
+      v.td = g.dom ? g.dom[(long)c.bh * NC + c.k] : -1;
       return v;
     };
     auto finish = [&](const Raw& w, int buf) -> Rows {
@@ -351,6 +364,11 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       v.bc = w.bc;
       v.gk = w.gk;
       v.decay = expf(w.gk + w.m_in - w.m_out);
+      v.bh = w.bh;
+      v.td = w.td;
+      // dominated chunk: d = the rounding residual of t*'s weighted key, per
+      // d_qk column (read after the barrier that precedes prep)
+      if (w.td >= 0 && rt < kDK) dstar_s[rt] = dom_residual(g, p, w.bh, w.k, w.td, rt, Kraw);
       const float cmax = w.amax_last;               // max over the chunk (amax is a running max)
       const float mu0 = fmaxf(w.m_in, w.amax0);     // the smallest mu_r of the chunk
       v.sep = (cmax - mu0) <= 60.f;
@@ -395,23 +413,32 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     // memory as bf16 (MN-major, 128-byte swizzle), then the decay of the
     // master in place.  Called once every MMA of the previous chunk has
     // completed (its Q~.C read the old copy; its update wrote the master).
-    auto copy_and_decay = [&](float decay) {
+    auto copy_and_decay = [&](const Rows& rv) {
+      const float decay = rv.decay;
       const int sl = r >> 6, rr = r & 63;
       uint8_t* crow = smem + F::kOffC + sl * (DV / 64) * 8192 + rr * 128;
+      // a dominated state leaves as C - n v_{t*}^T (n_k: kept by prep)
+      const __nv_bfloat16* vstar =
+          rv.td >= 0 ? Vraw + ((long)rv.bh * p.T + rv.td) * DV + h * kHalfV : nullptr;
+      const float nrow = vstar ? dstar_s[r] - nprev_s[r] : 0.f;  // -(n - d)
       for (int c = 0; c < kHalfV; c += 32) {
         uint32_t v[32];
         tmem_ld32(trow + kColC + h * kHalfV + c, v);
         tmem_wait_ld();
+        uint32_t x[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) x[e] = v[e];
+        if (vstar) add_rank1_32(x, nrow, vstar + c);
         const int col0 = h * kHalfV + c;  // first d_v column of these 32
         uint8_t* blk = crow + (col0 >> 6) * 8192;
         const int ch0 = (col0 & 63) >> 3;
 #pragma unroll
         for (int e = 0; e < 4; ++e)
           *reinterpret_cast<uint4*>(blk + (((ch0 + e) ^ (rr & 7)) << 4)) = make_uint4(
-              pack_bf16x2(__uint_as_float(v[8 * e]), __uint_as_float(v[8 * e + 1])),
-              pack_bf16x2(__uint_as_float(v[8 * e + 2]), __uint_as_float(v[8 * e + 3])),
-              pack_bf16x2(__uint_as_float(v[8 * e + 4]), __uint_as_float(v[8 * e + 5])),
-              pack_bf16x2(__uint_as_float(v[8 * e + 6]), __uint_as_float(v[8 * e + 7])));
+              pack_bf16x2(__uint_as_float(x[8 * e]), __uint_as_float(x[8 * e + 1])),
+              pack_bf16x2(__uint_as_float(x[8 * e + 2]), __uint_as_float(x[8 * e + 3])),
+              pack_bf16x2(__uint_as_float(x[8 * e + 4]), __uint_as_float(x[8 * e + 5])),
+              pack_bf16x2(__uint_as_float(x[8 * e + 6]), __uint_as_float(x[8 * e + 7])));
 #pragma unroll
         for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * decay);
         tmem_st32(trow + kColC + h * kHalfV + c, v);
@@ -420,9 +447,9 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     };
     // Everything of chunk j that needs S(j) but not the MMAs of chunk j - 1:
     // den_inter from the unscaled Q and n_j, P into TMEM, the scaled Q~ and
-    // the weighted K in place, and n_{j+1}.  Returns this half's partial
-    // denominator.
-    auto prep = [&](int j, const Rows& rv) -> float {
+    // the weighted K in place, and n_{j+1} (n_j moves to nprev_s).  Returns
+    // this half's partial denominator and its inter-chunk part q_r . n_j.
+    auto prep = [&](int j, const Rows& rv) -> float2 {
       const int b = j & 1;
       uint8_t* qbuf = smem + F::kOffQ + b * F::kQBytes;
       uint8_t* kbuf = smem + F::kOffK + b * F::kKBytes;
@@ -445,7 +472,11 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u);
 #pragma unroll
           for (int e = 0; e < 4; e += 2) {
-            const float4 nv = *reinterpret_cast<const float4*>(n_s + h * 64 + c * 8 + 2 * e);
+            float4 nv = *reinterpret_cast<const float4*>(n_s + h * 64 + c * 8 + 2 * e);
+            if (rv.td >= 0) {  // n* = n - d
+              const float4 dv = *reinterpret_cast<const float4*>(dstar_s + h * 64 + c * 8 + 2 * e);
+              nv = make_float4(nv.x - dv.x, nv.y - dv.y, nv.z - dv.z, nv.w - dv.w);
+            }
             const float2 fa = __bfloat1622float2(h2[e]);
             const float2 fb = __bfloat1622float2(h2[e + 1]);
             dn = fmaf(fa.x, nv.x, dn);
@@ -535,20 +566,22 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         float acc = 0.f;
 #pragma unroll
         for (int i = 0; i < F::kRG; ++i) acc += redn_s[i * kDK + rt];
+        nprev_s[rt] = n_s[rt];               // n_j, for the operand copy of C_j
         n_s[rt] = rv.decay * n_s[rt] + acc;  // n_{j+1}
       }
       fence_proxy_async_smem();  // Q~ and w K for the MMAs
       named_bar_sync(1, 256);  // n_{j+1} visible; redn_s free
-      return den;
+      return make_float2(den, dn);
     };
 
     // Epilogue of chunk j: the row's denominator from both halves, then
     // O / den as bf16 through the chunk's (now free) Q buffer and TMA stores.
-    auto epilogue = [&](int j, const FChunk& c, const Rows& rv, float den_part) {
+    auto epilogue = [&](int j, const FChunk& c, const Rows& rv, float2 den_part) {
       const int b = j & 1;
       red_s[rt] = den_part;
       named_bar_sync(1, 256);
-      const float den = den_part + red_s[rt ^ 128];
+      const float2 other = red_s[rt ^ 128];
+      const float den = den_part.x + other.x;
       const float denom = fmaxf(fabsf(den), expf(-(rv.bc + rv.mu)));
       const float inv = 1.f / denom;
       ok = ok && mbar_wait(bar.o_full(), j & 1, p, 9);  // Q~.C(j) done: Q(j) free
@@ -557,6 +590,12 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       tmem_ld32(trow + kColO + h * kHalfV, v0);
       if (kHalfV >= 64) tmem_ld32(trow + kColO + h * kHalfV + 32, v1);
       tmem_wait_ld();
+      if (rv.td >= 0) {  // a dominated chunk's rank-one part, (n_j^T q~_r) v_{t*}
+        const float c1 = expf(rv.m_in - rv.mu) * (den_part.y + other.y);
+        const __nv_bfloat16* vstar = Vraw + ((long)c.bh * p.T + rv.td) * DV + h * kHalfV;
+        add_rank1_32(v0, c1, vstar);
+        if (kHalfV >= 64) add_rank1_32(v1, c1, vstar + 32);
+      }
       uint8_t* stg = smem + F::kOffQ + b * F::kQBytes;  // [DV / 64 boxes][128 rows][128 B]
       const int col0 = h * kHalfV;
       uint8_t* box = stg + (col0 >> 6) * 16384;
@@ -592,8 +631,8 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       Rows cur = finish(pending, 0);
       if (total > 1) pending = load_raw(chunk_at(1, NC));
       named_bar_sync(1, 256);  // acol, n visible
-      float den_cur = prep(0, cur);
-      copy_and_decay(cur.decay);
+      float2 den_cur = prep(0, cur);
+      copy_and_decay(cur);
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(bar.ready());
@@ -601,7 +640,7 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const FChunk c = chunk_at(j, NC);
         const bool last_of_head = (c.k == NC - 1);
         Rows nxt = cur;
-        float den_nxt = 0.f;
+        float2 den_nxt = make_float2(0.f, 0.f);
         FChunk cn{};
         if (j + 1 < total) {
           cn = chunk_at(j + 1, NC);
@@ -626,7 +665,7 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if (last_of_head) write_final(c.bh);
         if (j + 1 < total) {
           if (last_of_head) init_master(cn.bh);  // master <- C0 of the next head
-          copy_and_decay(nxt.decay);
+          copy_and_decay(nxt);
           fence_proxy_async_smem();
           tc_fence_before();
           mbar_arrive(bar.ready());
@@ -665,7 +704,9 @@ cudaError_t launch_fused_t(const Problem& p, const void* Q, const void* K, const
   e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return e;
   const int grid = p.BH < sms ? p.BH : sms;
-  kern<<<grid, kThreads, F::kSmem, st>>>(tq, tk, tv, th, p, g, C0, n0, C_T, n_T, m_T);
+  kern<<<grid, kThreads, F::kSmem, st>>>(tq, tk, tv, th, p, g, C0, n0, C_T, n_T, m_T,
+                                         static_cast<const __nv_bfloat16*>(V),
+                                         static_cast<const __nv_bfloat16*>(K));
   return cudaGetLastError();
 }
 

@@ -74,7 +74,7 @@ struct Cfg {
   static constexpr uint32_t kKSlabBytes = kKT * 128;           // 128 rows x 64 bf16
   static constexpr uint32_t kMNSlabBytes = (DVT / 64) * 8192;  // 64 rows x DVT bf16
   static constexpr uint32_t kStageBytes = kKSlabBytes > kMNSlabBytes ? kKSlabBytes : kMNSlabBytes;
-  static constexpr uint32_t kMiscBytes = 2 * kMaxL * 4 + 2 * DK * 4 + 256 * 4 + 512;
+  static constexpr uint32_t kMiscBytes = 2 * kMaxL * 4 + 2 * DK * 4 + 256 * 8 + 512;
   static constexpr uint32_t kBudget = 227 * 1024 - 1024;  // minus alignment slack
   static constexpr int kStagesFit = (int)((kBudget - kQBytes - kMiscBytes) / kStageBytes);
   static constexpr int kStages = kStagesFit > 12 ? 12 : kStagesFit;
@@ -83,8 +83,8 @@ struct Cfg {
   static constexpr uint32_t kOffStage = kOffQ + kQBytes;
   static constexpr uint32_t kOffAcol = kOffStage + kStages * kStageBytes;  // float[2][kMaxL]
   static constexpr uint32_t kOffN = kOffAcol + 2 * kMaxL * 4;  // float[2][DK]
-  static constexpr uint32_t kOffRed = kOffN + 2 * DK * 4;      // float[256]
-  static constexpr uint32_t kOffBar = kOffRed + 256 * 4;       // barriers
+  static constexpr uint32_t kOffRed = kOffN + 2 * DK * 4;      // float2[256]
+  static constexpr uint32_t kOffBar = kOffRed + 256 * 8;       // barriers
   static constexpr uint32_t kOffTmemSlot = kOffBar + 368;
   static constexpr uint32_t kBytes = kOffTmemSlot + 16;
   static constexpr uint32_t kSmem = kBytes + 1024;  // slack for 1024-byte alignment
@@ -146,7 +146,8 @@ tc_parallel_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                    const __grid_constant__ CUtensorMap tm_v, const __nv_bfloat16* __restrict__ Cb,
                    Problem p, Gates g, const float* __restrict__ n_states,
                    __nv_bfloat16* __restrict__ H, float* __restrict__ n_out,
-                   float* __restrict__ m_out, int n_items) {
+                   float* __restrict__ m_out, int n_items,
+                   const __nv_bfloat16* __restrict__ Vraw) {
   using C = Cfg<DK, DVT>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -155,7 +156,7 @@ tc_parallel_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   const Bars bar{sbase + C::kOffBar};
   float* acol_s = reinterpret_cast<float*>(smem + C::kOffAcol);
   float* n_s = reinterpret_cast<float*>(smem + C::kOffN);
-  float* red_s = reinterpret_cast<float*>(smem + C::kOffRed);
+  float2* red_s = reinterpret_cast<float2*>(smem + C::kOffRed);
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + C::kOffTmemSlot);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -371,6 +372,7 @@ tc_parallel_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     struct RowVals {
       float m_in, amax, bc, c;
       bool sep;
+      int td;  // dominant token of the chunk's entering state, or -1
     };
     auto fetch_rows = [&](const Item& x) -> RowVals {
       RowVals v;
@@ -380,6 +382,7 @@ tc_parallel_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       v.bc = g.bcum[base + x.t0 + r];
       v.c = g.amax[base + x.t0 + kQT - 1];
       v.sep = v.c - fmaxf(v.m_in, g.amax[base + x.t0]) <= 60.f;  // uniform over the CTA
+      v.td = g.dom ? g.dom[(long)x.bh * p.NC + x.k] : -1;
       return v;
     };
     auto fetch_cols = [&](const Item& x, int buf, const RowVals& v) {
@@ -391,7 +394,7 @@ tc_parallel_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       }
       for (int j = rt; j < DK; j += 256) nn[j] = n_states[((long)x.bh * p.NC + x.k) * DK + j];
     };
-    RowVals nx{0.f, 0.f, 0.f, 0.f, false};
+    RowVals nx{0.f, 0.f, 0.f, 0.f, false, -1};
     if (blockIdx.x < n_items) {
       const Item x0 = decode_item(blockIdx.x, p, n_dv, n_q);
       nx = fetch_rows(x0);
@@ -516,10 +519,15 @@ tc_parallel_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         fetch_cols(xn, (n + 1) & 1, nx);
       }
 
-      // Epilogue: combine the two halves' denominators, h = O / max(|den|, e^{-m_r}).
-      red_s[rt] = den;
+      // Epilogue: combine the two halves' denominators, h = O / max(|den|, e^{-m_r}),
+      // with a dominated chunk's rank-one part (n_k^T q~_r) v_{t*} added in fp32.
+      red_s[rt] = make_float2(den, dn);
       named_bar_sync(1, 256);
-      den += red_s[rt ^ 128];
+      const float2 other = red_s[rt ^ 128];
+      den += other.x;
+      const float c1 = f_inter * (dn + other.y);
+      const __nv_bfloat16* vstar =
+          rv.td >= 0 ? Vraw + ((long)x.bh * p.T + rv.td) * p.DV + x.dv0 : nullptr;
       ok = ok && mbar_wait(bar.o_full(n % C::kOBufs), (n / C::kOBufs) & 1, p, 12);
       tc_fence_after();
       const float mr = bc + mu;
@@ -531,6 +539,10 @@ tc_parallel_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
           tmem_ld32(trow + colO + c, v0);
           if (kHalfO >= 64) tmem_ld32(trow + colO + c + 32, v1);
           tmem_wait_ld();
+          if (vstar) {
+            add_rank1_32(v0, c1, vstar + c);
+            if (kHalfO >= 64) add_rank1_32(v1, c1, vstar + c + 32);
+          }
           if (t < p.T) {
             uint32_t pk[16];
 #pragma unroll
@@ -592,7 +604,8 @@ cudaError_t launch_parallel_t(const Problem& p, const void* Q, const void* K, co
   if (items > (1L << 30)) return cudaErrorInvalidValue;
   const int grid = (int)(items < sms ? items : sms);
   kern<<<grid, kThreads, C::kSmem, st>>>(tq, tk, tv, Cb, p, g, n_states,
-                                         static_cast<__nv_bfloat16*>(H), n_out, m_out, (int)items);
+                                         static_cast<__nv_bfloat16*>(H), n_out, m_out, (int)items,
+                                         static_cast<const __nv_bfloat16*>(V));
   return cudaGetLastError();
 }
 

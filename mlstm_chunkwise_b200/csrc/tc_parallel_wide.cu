@@ -79,7 +79,7 @@ struct WCfg {
   static_assert(kKSlabBytes <= kStageBytes && kMNSlabBytes <= kStageBytes, "stage size");
   static constexpr uint32_t kOutBytes = kQT * DVT * 2;  // output staging tile
   static constexpr uint32_t kMiscBytes =
-      2 * kPSlots * kKT * 4 + 2 * kChunks * DK * 4 + 256 * 4 + 512;
+      2 * kPSlots * kKT * 4 + 2 * kChunks * DK * 4 + 256 * 8 + 512;
   static constexpr uint32_t kBudget = 227 * 1024 - 1024;
   static constexpr int kStagesFit =
       (int)((kBudget - kQBytes - kOutBytes - kMiscBytes) / kStageBytes);
@@ -90,8 +90,8 @@ struct WCfg {
   static constexpr uint32_t kOffStage = kOffOut + kOutBytes;
   static constexpr uint32_t kOffAcol = kOffStage + kStages * kStageBytes;  // float[2][256]
   static constexpr uint32_t kOffN = kOffAcol + 2 * kPSlots * kKT * 4;  // float[2][kChunks][DK]
-  static constexpr uint32_t kOffRed = kOffN + 2 * kChunks * DK * 4;    // float[256]
-  static constexpr uint32_t kOffBar = kOffRed + 256 * 4;
+  static constexpr uint32_t kOffRed = kOffN + 2 * kChunks * DK * 4;    // float2[256]
+  static constexpr uint32_t kOffBar = kOffRed + 256 * 8;
   static constexpr uint32_t kOffTmemSlot = kOffBar + 384;
   static constexpr uint32_t kBytes = kOffTmemSlot + 16;
   static constexpr uint32_t kSmem = kBytes + 1024;
@@ -150,7 +150,8 @@ tc_parallel_wide_kernel(const __grid_constant__ CUtensorMap tm_q,
                         const __nv_bfloat16* __restrict__ Cb,
                         const __grid_constant__ CUtensorMap tm_h, Problem p, Gates g,
                         const float* __restrict__ n_states,
-                        float* __restrict__ n_out, float* __restrict__ m_out, int n_items) {
+                        float* __restrict__ n_out, float* __restrict__ m_out, int n_items,
+                        const __nv_bfloat16* __restrict__ Vraw) {
   using C = WCfg<DK, DVT, kPair>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -159,7 +160,7 @@ tc_parallel_wide_kernel(const __grid_constant__ CUtensorMap tm_q,
   const WBars bar{sbase + C::kOffBar};
   float* acol_s = reinterpret_cast<float*>(smem + C::kOffAcol);
   float* n_s = reinterpret_cast<float*>(smem + C::kOffN);
-  float* red_s = reinterpret_cast<float*>(smem + C::kOffRed);
+  float2* red_s = reinterpret_cast<float2*>(smem + C::kOffRed);
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + C::kOffTmemSlot);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -352,11 +353,12 @@ tc_parallel_wide_kernel(const __grid_constant__ CUtensorMap tm_q,
     auto chunk_of = [&](const WItem& x, int part) {
       return x.k + part < p.NC ? x.k + part : p.NC - 1;
     };
-    auto fetch_rows = [&](const WItem& x, float& m_in, float& amax, float& bc) {
+    auto fetch_rows = [&](const WItem& x, float& m_in, float& amax, float& bc, int& td) {
       const int t = x.t0 + r;
       m_in = g.mchk[(long)x.bh * (p.NC + 1) + chunk_of(x, rchunk)];
       amax = g.amax[(long)x.bh * tpad + t];
       bc = g.bcum[(long)x.bh * tpad + t];
+      td = g.dom ? g.dom[(long)x.bh * p.NC + chunk_of(x, rchunk)] : -1;
     };
     auto fetch_cols = [&](const WItem& x, int buf) {
       float* ac = acol_s + buf * kPSlots * kKT;
@@ -367,9 +369,10 @@ tc_parallel_wide_kernel(const __grid_constant__ CUtensorMap tm_q,
         nn[j] = n_states[((long)x.bh * p.NC + chunk_of(x, j / DK)) * DK + j % DK];
     };
     float nx_m_in = 0.f, nx_amax = 0.f, nx_bc = 0.f;
+    int nx_td = -1;
     if (blockIdx.x < n_items) {
       const WItem x0 = decode_witem(blockIdx.x, p, n_q);
-      fetch_rows(x0, nx_m_in, nx_amax, nx_bc);
+      fetch_rows(x0, nx_m_in, nx_amax, nx_bc, nx_td);
       fetch_cols(x0, 0);
     }
     int n = 0;
@@ -377,6 +380,7 @@ tc_parallel_wide_kernel(const __grid_constant__ CUtensorMap tm_q,
       const WItem x = decode_witem(it, p, n_q);
       const int t = x.t0 + r;
       const float m_in = nx_m_in, amax = nx_amax, bc = nx_bc;
+      const int td = nx_td;  // warp-uniform (kPair: rows of one chunk per warp)
       const float* ac = acol_s + (n & 1) * kPSlots * kKT;
       const float* nn = n_s + ((n & 1) * C::kChunks + rchunk) * DK;
       const float mu = fmaxf(m_in, amax);
@@ -468,14 +472,19 @@ tc_parallel_wide_kernel(const __grid_constant__ CUtensorMap tm_q,
       const int it_next = item_at(n + 1);
       if (it_next < n_items) {
         const WItem xn = decode_witem(it_next, p, n_q);
-        fetch_rows(xn, nx_m_in, nx_amax, nx_bc);
+        fetch_rows(xn, nx_m_in, nx_amax, nx_bc, nx_td);
         fetch_cols(xn, (n + 1) & 1);
       }
 
-      // Both halves' partial denominators -> the row's denominator.
-      red_s[rt] = den;
+      // Both halves' partial denominators (and inter-chunk parts) -> the row's.
+      red_s[rt] = make_float2(den, dn);
       named_bar_sync(1, 256);
-      den += red_s[rt ^ 128];
+      const float2 other = red_s[rt ^ 128];
+      den += other.x;
+      // a dominated chunk's rank-one part, (n_k^T q~_r) v_{t*}, added in fp32
+      const float c1 = f_inter * (dn + other.y);
+      const __nv_bfloat16* vstar =
+          td >= 0 ? Vraw + ((long)x.bh * p.T + td) * p.DV + h * kHalfO : nullptr;
       const float mr = bc + mu;
       const float denom = fmaxf(fabsf(den), expf(-mr));
       const float inv = 1.f / denom;
@@ -495,6 +504,10 @@ tc_parallel_wide_kernel(const __grid_constant__ CUtensorMap tm_q,
           tmem_ld32(trow + colO, v0);
           if (kHalfO >= 64) tmem_ld32(trow + colO + 32, v1);
           tmem_wait_ld();
+          if (vstar) {
+            add_rank1_32(v0, c1, vstar + d * DVT);
+            if (kHalfO >= 64) add_rank1_32(v1, c1, vstar + d * DVT + 32);
+          }
           // this half's columns: box (h * kHalfO) / 64, 16-byte chunks from cb
           uint8_t* box = smem + C::kOffOut + ((h * kHalfO) >> 6) * 16384;
           const int cb = ((h * kHalfO) & 63) >> 3;
@@ -562,7 +575,7 @@ cudaError_t launch_wide_t(const Problem& p, const void* Q, const void* K, const 
   if (items > (1L << 30)) return cudaErrorInvalidValue;
   const int grid = (int)(items < sms ? items : sms);
   kern<<<grid, kThreads, C::kSmem, st>>>(tq, tk, tv, Cb, th, p, g, n_states, n_out, m_out,
-                                         (int)items);
+                                         (int)items, static_cast<const __nv_bfloat16*>(V));
   return cudaGetLastError();
 }
 

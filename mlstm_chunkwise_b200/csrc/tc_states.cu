@@ -35,6 +35,16 @@
 // then fold in the update, C_{k+1} = decay C_k + U_k, and release the buffer,
 // so the MMAs of the next chunk wait for no decay of a TMEM master.
 //
+// Dominated states (g.dom[k] = t* >= 0, bf16 operand copy only): one token
+// holds most of the state entering chunk k, so C_k ~ n_k v_{t*}^T and the
+// output kernels' h = C^T q / |n^T q| would divide the independent bf16
+// rounding of C by a small n^T q.  The copy then holds R_k = C_k - n*_k
+// v_{t*}^T (fp32 subtraction, then rounding), n_states holds n*_k, and the
+// output kernels add (n*_k^T q) v_{t*} back in fp32; n*_k = n_k - d_k, d_k the
+// rounding residual of t*'s weighted key (dom_residual in tc.h).  Segments
+// after the first subtract their local n; the fix-up adds the carried-in part
+// the same way (the split is linear in (C, n)) and then d_k.
+//
 // Roles (320 threads): warp 0 TMA producer, warp 1 TMEM owner + MMA issuer,
 // warps 2..9 workers: per chunk, the store and decay of the master state; per
 // stage, one pass that computes its token weights, accumulates the n-vector
@@ -73,7 +83,7 @@ struct SCfg {
   // reuses the same bytes (it never overlaps a state store).
   static constexpr uint32_t kStgBytes = 8 * 2 * 2048;
   static_assert(kRedBytes <= kStgBytes, "n partials must fit in the store tiles");
-  static constexpr uint32_t kBudget = 227 * 1024 - 1024 - 512 - kStgBytes;
+  static constexpr uint32_t kBudget = 227 * 1024 - 1024 - 512 - DK * 4 - kStgBytes;
   static constexpr int kStagesFit = (int)(kBudget / kStageBytes);
   static constexpr int kStages = kStagesFit > 8 ? 8 : kStagesFit;
   static_assert(kStages >= 2, "ring too shallow");
@@ -82,7 +92,8 @@ struct SCfg {
   static_assert(kOffStg % 1024 == 0, "store tiles must sit on a swizzle-atom boundary");
   static constexpr uint32_t kOffBar = kOffStg + kStgBytes;
   static constexpr uint32_t kOffSlot = kOffBar + 8 * 32;
-  static constexpr uint32_t kBytes = kOffSlot + 16;
+  static constexpr uint32_t kOffNs = kOffSlot + 16;  // float[DK]: n entering the chunk
+  static constexpr uint32_t kBytes = kOffNs + DK * 4;
   static constexpr uint32_t kSmem = kBytes + 1024;
   static_assert(kSmem <= 227 * 1024, "shared memory");
   // d_qk = 128 with value tiles of at most 128 columns: the running state
@@ -105,13 +116,26 @@ struct SBars {
   __device__ __forceinline__ uint32_t done() const { return a + 224; }
 };
 
+// x[e] -= n * v[e] for 8 consecutive value columns (v: bf16, 16-byte aligned).
+__device__ __forceinline__ void deflate8(float (&x)[8], float n, const __nv_bfloat16* v) {
+  const uint4 u = __ldg(reinterpret_cast<const uint4*>(v));
+  const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float2 f = __bfloat1622float2(h2[e]);
+    x[2 * e] = fmaf(-n, f.x, x[2 * e]);
+    x[2 * e + 1] = fmaf(-n, f.y, x[2 * e + 1]);
+  }
+}
+
 template <int DK, int DVT>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_states_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                  const __grid_constant__ CUtensorMap tm_cs, Problem p, Gates g, const float* __restrict__ C0, const float* __restrict__ n0,
                  float* __restrict__ C_states, __nv_bfloat16* __restrict__ Cb,
                  float* __restrict__ n_states, float* __restrict__ C_T, float* __restrict__ n_T,
-                 float* __restrict__ m_T, float* __restrict__ seg_C, float* __restrict__ seg_n) {
+                 float* __restrict__ m_T, float* __restrict__ seg_C, float* __restrict__ seg_n,
+                 const __nv_bfloat16* __restrict__ Vraw, const __nv_bfloat16* __restrict__ Kraw) {
   using S = SCfg<DK, DVT>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -120,6 +144,7 @@ tc_states_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
   const SBars bar{sbase + S::kOffBar};
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + S::kOffSlot);
   float* red_s = reinterpret_cast<float*>(smem + S::kOffStg);  // aliases the store tiles
+  float* n_s = reinterpret_cast<float*>(smem + S::kOffNs);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int dv0 = blockIdx.x * DVT, bh = blockIdx.y;
@@ -254,8 +279,10 @@ tc_states_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
     uint8_t* stg = smem + S::kOffStg + (warp - 2) * 4096;
     const uint32_t stg_u = sbase + S::kOffStg + (uint32_t)(warp - 2) * 4096u;
     int n_st = 0;  // state stores issued by this warp (selects the tile)
-    // n-vector: worker wt owns dk column wt (DK <= 256) for the running n.
-    const bool n_mine = n_owner && wt < DK;
+    // n-vector: worker wt owns dk column wt (DK <= 256) for the running n
+    // (every CTA carries it; the first value tile's CTA writes it out).
+    const bool n_mine = wt < DK;
+    const bool n_write = n_owner && n_mine;
     float nval = (n_mine && n0 && seg == 0) ? n0[(long)bh * DK + wt] : 0.f;
     // Stage pass mapping: 16-byte column chunk cc (8 dk columns) of token rows
     // rg * kRowsPer .. + kRowsPer - 1.
@@ -288,9 +315,9 @@ tc_states_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
 
     // Adds this chunk's n partials into the running n (all workers take part).
     // red_s spans several warps' store tiles, so every warp's stores must have
-    // read them first (n_owner is uniform over the CTA, so are the barriers).
+    // read them first.
     auto fold_n = [&]() {
-      if (n_owner) {
+      {
         if (lane == 0) tma_store_wait_read_all();
         named_bar_sync(1, kWorkers);
 #pragma unroll
@@ -387,7 +414,15 @@ tc_states_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         nx_gk = g.gtot[(long)bh * NC + k + 1];
       }
       const float decay = expf(gk + m_in - m_out);
-      if (n_mine) n_states[((long)bh * NC + k) * DK + wt] = nval;
+      // dominated state: the operand copy leaves as C - n* v_{t*}^T, n* = n - d
+      // (the first segment; later ones get d from the fix-up)
+      const int tdom = (Cb && g.dom) ? g.dom[(long)bh * NC + k] : -1;
+      const __nv_bfloat16* vstar =
+          tdom >= 0 ? Vraw + ((long)bh * p.T + tdom) * DV + dv0 : nullptr;
+      float nout = nval;
+      if (tdom >= 0 && seg == 0 && n_mine) nout -= dom_residual(g, p, bh, k, tdom, wt, Kraw);
+      if (n_write) n_states[((long)bh * NC + k) * DK + wt] = nout;
+      if (n_mine) n_s[wt] = nout;  // read by the boundary pass after the barrier below
       nval *= decay;
 
       // The first stage of chunk k needs nothing from the MMAs.
@@ -404,9 +439,13 @@ tc_states_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
             const int col = ch * kColsPer + c;
             if (lane == 0) tma_store_wait_read_all();  // the previous tile has been read
             __syncwarp();
+            const float nrow = vstar ? n_s[dk0 + lane] : 0.f;
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
-              const float* x = creg + c + 8 * j;
+              float x[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) x[e] = creg[c + 8 * j + e];
+              if (vstar) deflate8(x, nrow, vstar + col + 8 * j);
               *reinterpret_cast<uint4*>(stg + lane * 128 + ((j ^ (lane & 7)) << 4)) =
                   make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]),
                              pack_bf16x2(x[4], x[5]), pack_bf16x2(x[6], x[7]));
@@ -463,19 +502,22 @@ tc_states_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
             const int col = ch * kColsPer + c;
             if (lane == 0) tma_store_wait_read_all();  // the previous tile has been read
             __syncwarp();
+            const float nrow = vstar ? n_s[dk0 + lane] : 0.f;
 #pragma unroll 1
             for (int hh = 0; hh < 2; ++hh) {
               uint32_t v[32];
               tmem_ld32(trow + hf * DVT + col + 32 * hh, v);
               tmem_wait_ld();
 #pragma unroll
-              for (int j = 0; j < 4; ++j)
+              for (int j = 0; j < 4; ++j) {
+                float x[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) x[e] = __uint_as_float(v[8 * j + e]);
+                if (vstar) deflate8(x, nrow, vstar + col + 32 * hh + 8 * j);
                 *reinterpret_cast<uint4*>(stg + lane * 128 + (((4 * hh + j) ^ (lane & 7)) << 4)) =
-                    make_uint4(
-                        pack_bf16x2(__uint_as_float(v[8 * j]), __uint_as_float(v[8 * j + 1])),
-                        pack_bf16x2(__uint_as_float(v[8 * j + 2]), __uint_as_float(v[8 * j + 3])),
-                        pack_bf16x2(__uint_as_float(v[8 * j + 4]), __uint_as_float(v[8 * j + 5])),
-                        pack_bf16x2(__uint_as_float(v[8 * j + 6]), __uint_as_float(v[8 * j + 7])));
+                    make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]),
+                               pack_bf16x2(x[4], x[5]), pack_bf16x2(x[6], x[7]));
+              }
 #pragma unroll
               for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * decay);
               tmem_st32(trow + hf * DVT + col + 32 * hh, v);
@@ -548,8 +590,8 @@ tc_states_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         }
       }
     }
-    if (n_mine && last_seg && n_T) n_T[(long)bh * DK + wt] = nval;
-    if (n_mine && !last_seg) seg_n[((long)bh * (n_seg - 1) + seg) * DK + wt] = nval;
+    if (n_write && last_seg && n_T) n_T[(long)bh * DK + wt] = nval;
+    if (n_write && !last_seg) seg_n[((long)bh * (n_seg - 1) + seg) * DK + wt] = nval;
     if (m_T && last_seg && blockIdx.x == 0 && wt == 0) m_T[bh] = mchk[NC];
     if (lane == 0) tma_store_wait_all();  // the state stores have landed
   }
@@ -571,13 +613,17 @@ tc_states_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
 //   a_k = e^{sum of e_j, j in [k0, k)},   e_j = g_j + m_j - m_{j+1} <= 0,
 // the same per-chunk decay factors the recurrence applies.  kOperand: the
 // states are the bf16 operand copy (block layout of cb_block_row), else fp32
-// [b h k][DK][DV].
+// [b h k][DK][DV].  For a dominated chunk (dom[k] = t* >= 0) the copy holds
+// C - n* v_{t*}^T and n_states n*, n* = n - d: the terms added are
+// a_k (C_{k0} - n_{k0} v_{t*}^T) + d v_{t*}^T and a_k n_{k0} - d.
 template <bool kOperand>
 __global__ void __launch_bounds__(256)
 tc_states_fixup_kernel(Problem p, Gates g, int DVT, const float* __restrict__ seg_C,
                        const float* __restrict__ seg_n, float* __restrict__ C_states,
                        __nv_bfloat16* __restrict__ Cb, float* __restrict__ n_states,
-                       float* __restrict__ C_T, float* __restrict__ n_T) {
+                       float* __restrict__ C_T, float* __restrict__ n_T,
+                       const __nv_bfloat16* __restrict__ Vraw,
+                       const __nv_bfloat16* __restrict__ Kraw) {
   const int DK = p.DK, DV = p.DV, NC = p.NC;
   const int bh = blockIdx.y, seg = blockIdx.z + 1, n_seg = gridDim.z + 1;
   const int ncs = (NC + n_seg - 1) / n_seg;
@@ -619,7 +665,7 @@ tc_states_fixup_kernel(Problem p, Gates g, int DVT, const float* __restrict__ se
     const float ev[8] = {e0.x, e0.y, e0.z, e0.w, e1.x, e1.y, e1.z, e1.w};
 #pragma unroll
     for (int i = 0; i < 8; ++i) cs[i] = fmaf(A, cs[i], ev[i]);
-    if (n_thread) ns = fmaf(A, ns, seg_n[((long)bh * (n_seg - 1) + s) * DK + dk]);
+    ns = fmaf(A, ns, seg_n[((long)bh * (n_seg - 1) + s) * DK + dk]);
   }
 
   const int k0 = seg * ncs, k1 = min(k0 + ncs, NC);
@@ -658,12 +704,24 @@ tc_states_fixup_kernel(Problem p, Gates g, int DVT, const float* __restrict__ se
 #pragma unroll
         for (int u = 0; u < kB; ++u) {
           if (c0 + u < nb) {
+            float add[8], res[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              add[i] = cs[i];
+              res[i] = 0.f;
+            }
+            const int td = g.dom ? g.dom[(long)bh * NC + kb + c0 + u] : -1;
+            if (td >= 0) {
+              const __nv_bfloat16* vs = Vraw + ((long)bh * p.T + td) * DV + col;
+              deflate8(add, ns, vs);
+              deflate8(res, -dom_residual(g, p, bh, kb + c0 + u, td, dk, Kraw), vs);
+            }
             __nv_bfloat162* h2 = reinterpret_cast<__nv_bfloat162*>(&v[u]);
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               const float2 f = __bfloat1622float2(h2[e]);
-              h2[e] = __floats2bfloat162_rn(fmaf(a[u], cs[2 * e], f.x),
-                                            fmaf(a[u], cs[2 * e + 1], f.y));
+              h2[e] = __floats2bfloat162_rn(fmaf(a[u], add[2 * e], f.x) + res[2 * e],
+                                            fmaf(a[u], add[2 * e + 1], f.y) + res[2 * e + 1]);
             }
             *reinterpret_cast<uint4*>(ptr[u]) = v[u];
           }
@@ -692,8 +750,14 @@ tc_states_fixup_kernel(Problem p, Gates g, int DVT, const float* __restrict__ se
       }
       if (n_thread) {
 #pragma unroll
-        for (int u = 0; u < kB; ++u)
-          if (c0 + u < nb) n_states[((long)bh * NC + kb + c0 + u) * DK + dk] += a[u] * ns;
+        for (int u = 0; u < kB; ++u) {
+          if (c0 + u < nb) {
+            const int kc = kb + c0 + u;
+            const int td = (kOperand && g.dom) ? g.dom[(long)bh * NC + kc] : -1;
+            const float d = td >= 0 ? dom_residual(g, p, bh, kc, td, dk, Kraw) : 0.f;
+            n_states[((long)bh * NC + kc) * DK + dk] += a[u] * ns - d;
+          }
+        }
       }
     }
   }
@@ -739,17 +803,22 @@ cudaError_t launch_states_t(const Problem& p, const void* K, const void* V, cons
   float* seg_C = seg_ws;
   float* seg_n = n_seg > 1 ? seg_ws + (size_t)p.BH * (n_seg - 1) * p.DK * p.DV : nullptr;
   dim3 grid(p.DV / DVT, p.BH, n_seg);
-  kern<<<grid, kThreads, S::kSmem, st>>>(tk, tv, tcs, p, g, C0, n0, C_states, Cb, n_states, C_T,
-                                         n_T, m_T, seg_C, seg_n);
+  // the dominance marks apply to the bf16 operand copy only
+  Gates gk = g;
+  if (!Cb) gk.dom = nullptr;
+  const __nv_bfloat16* Vraw = static_cast<const __nv_bfloat16*>(V);
+  const __nv_bfloat16* Kraw = static_cast<const __nv_bfloat16*>(K);
+  kern<<<grid, kThreads, S::kSmem, st>>>(tk, tv, tcs, p, gk, C0, n0, C_states, Cb, n_states, C_T,
+                                         n_T, m_T, seg_C, seg_n, Vraw, Kraw);
   e = cudaGetLastError();
   if (e != cudaSuccess || n_seg == 1) return e;
   dim3 fgrid(p.DK * p.DV / 8 / 256, p.BH, n_seg - 1);
   if (Cb)
-    tc_states_fixup_kernel<true><<<fgrid, 256, 0, st>>>(p, g, DVT, seg_C, seg_n, C_states, Cb,
-                                                        n_states, C_T, n_T);
+    tc_states_fixup_kernel<true><<<fgrid, 256, 0, st>>>(p, gk, DVT, seg_C, seg_n, C_states, Cb,
+                                                        n_states, C_T, n_T, Vraw, Kraw);
   else
-    tc_states_fixup_kernel<false><<<fgrid, 256, 0, st>>>(p, g, DVT, seg_C, seg_n, C_states, Cb,
-                                                         n_states, C_T, n_T);
+    tc_states_fixup_kernel<false><<<fgrid, 256, 0, st>>>(p, gk, DVT, seg_C, seg_n, C_states, Cb,
+                                                         n_states, C_T, n_T, Vraw, Kraw);
   return cudaGetLastError();
 }
 

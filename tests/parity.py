@@ -77,3 +77,18 @@ def compare(H, final, ref: dict, tol: float, heads=None, label="") -> dict:
     bad = {k: v for k, v in errs.items() if not (v <= tol)}
     assert not bad, f"{label}: errors above {tol}: {bad} (all: {errs})"
     return errs
+
+
+def worst_row_rel(x: np.ndarray, y: np.ndarray, floor: float = 1e-3) -> float:
+    """Worst per-token-row relative error of x against y ([B, NH, T, D]).
+
+    Each output row h_t is compared with its own size: max_j |x - y| divided by
+    max(max_j |y|, floor * max|y| of its (b, h) slice), so that rows whose exact
+    value is near zero do not divide by (almost) nothing.  This shows errors on
+    individual rows that the normwise slice metric averages away."""
+    d = np.abs(x - y).max(axis=-1)
+    rmax = np.abs(y).max(axis=-1)
+    smax = np.abs(y).max(axis=(-1, -2), keepdims=True)[..., 0]
+    den = np.maximum(rmax, floor * smax)
+    den = np.where(den > 0, den, 1.0)
+    return float((d / den).max()) if d.size else 0.0

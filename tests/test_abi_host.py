@@ -59,7 +59,10 @@ def test_workspace_size_formula(L):
     B, NH, T, DK, DV, Lc = 2, 3, 256, 64, 64, 64
     NC = T // Lc
     r = lambda x: (x + 255) // 256 * 256  # noqa: E731
-    gates = 3 * r(B * NH * NC * Lc * 4) + r(B * NH * NC * 4) + r(B * NH * (NC + 1) * 4)
+    # per-token bcum/acol/amax, per-chunk g, m (NC + 1), and per-chunk weight
+    # sum, argmax, dominant token and its log-weight
+    gates = 3 * r(B * NH * NC * Lc * 4) + r(B * NH * NC * 4) + r(B * NH * (NC + 1) * 4) + \
+        4 * r(B * NH * NC * 4)
     states = r(B * NH * NC * DK * DV * 4) + r(B * NH * NC * DK * 4)
     assert n == gates + states
     # ragged T rounds the chunk count up
