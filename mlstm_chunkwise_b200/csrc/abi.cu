@@ -87,7 +87,8 @@ Layout layout_for(const Problem& p, mlstm_algo a, Mode mode) {
   Layout l{};
   const size_t BH = (size_t)p.BH, tpad = (size_t)p.NC * p.L;
   l.gates_bytes = 3 * round_up(BH * tpad * sizeof(float)) + round_up(BH * p.NC * sizeof(float)) +
-                  round_up(BH * (p.NC + 1) * sizeof(float)) + 4 * round_up(BH * p.NC * 4);
+                  round_up(BH * (p.NC + 1) * sizeof(float)) + 4 * round_up(BH * p.NC * 4) +
+                  round_up(BH * 4);
   const size_t n_bytes = round_up(BH * p.NC * (size_t)p.DK * sizeof(float));
   if (mode == Mode::kFull && a == MLSTM_ALGO_SIMT)
     l.states_bytes = round_up(BH * p.NC * (size_t)p.DK * p.DV * sizeof(float)) + n_bytes;
@@ -125,6 +126,8 @@ char* carve_gates(const Problem& p, char* ws, Gates* g, float* mchk_override,
   ws += round_up(BH * p.NC * 4);
   g->mdom = dominance ? reinterpret_cast<float*>(ws) : nullptr;
   ws += round_up(BH * p.NC * 4);
+  g->hdom = dominance ? reinterpret_cast<int*>(ws) : nullptr;
+  ws += round_up(BH * 4);
   return ws;
 }
 

@@ -53,6 +53,7 @@ struct Problem {
 //                    R_k = C_k - n*_k v_{t*}^T (see tc.h).
 //   mdom [BH, NC]    the log-weight of the largest term of that state (t*'s
 //                    when dom >= 0), in the unstabilised frame
+//   hdom [BH]        1 if some chunk of the (b, h) has dom >= 0, else 0
 struct Gates {
   float* bcum = nullptr;
   float* acol = nullptr;
@@ -63,6 +64,7 @@ struct Gates {
   int* cidx = nullptr;
   int* dom = nullptr;
   float* mdom = nullptr;
+  int* hdom = nullptr;  // [BH]: 1 if any chunk of the (b, h) has dom >= 0
 };
 
 __device__ __forceinline__ float to_float(float x) { return x; }

@@ -14,7 +14,13 @@
 // Tokens past T in a ragged last chunk get lf = 0 and li = -inf: they neither
 // decay the state nor contribute to it.
 //
-// Kernel 1 (gates_chunk_kernel): one CTA per (chunk, b*h); block-wide scans.
+// Kernel 1: gates_chunk_kernel, one CTA per (chunk, b*h) with block-wide
+// scans (the backward pass and every call without the dominance marks use
+// it; with the marks, chunks of more than 128 tokens); gates_chunk_warp_kernel,
+// one warp per (chunk, b*h) with warp scans (the forward tensor-core paths at
+// chunks of at most 128 tokens, where a CTA per chunk leaves most threads
+// idle).  Both write the same arrays; with the marks, also the per-chunk
+// dominance statistics below.
 // Kernel 2 (gates_state_kernel): one warp per b*h; warp scan of the (max,+)
 // maps over chunks.
 //
@@ -38,6 +44,7 @@ namespace {
 
 constexpr int kGateThreads = 256;
 constexpr int kMaxPerThread = 16;  // chunk sizes up to 4096
+constexpr int kChunksPerBlock = kGateThreads / 32;  // warp-per-chunk kernel
 
 template <bool kMax>
 __device__ __forceinline__ float combine(float a, float b) {
@@ -75,6 +82,7 @@ __device__ float block_exclusive_scan(float v, float identity, float* smem) {
   return r;
 }
 
+template <bool kDominance>
 __global__ void __launch_bounds__(kGateThreads)
 gates_chunk_kernel(Problem p, const float* __restrict__ i_pre, const float* __restrict__ f_pre,
                    Gates g) {
@@ -128,108 +136,168 @@ gates_chunk_kernel(Problem p, const float* __restrict__ i_pre, const float* __re
       if (r == L - 1) g.gtot[(long)bh * p.NC + k] = lcum[e];
     }
   }
-  if (!g.dom) return;
-  // The chunk's largest column log-weight (the inclusive max at its end), the
-  // first token that attains it, and sum_s e^{acol_s - max}.
-  __shared__ float cmax_s;
-  __shared__ float sum_s[kGateThreads / 32];
-  __shared__ int idx_s[kGateThreads / 32];
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if constexpr (kDominance) {
+    // The max scan left the inclusive warp totals in smem[32..]: the last is
+    // the chunk's largest acol.  Then sum_s e^{acol_s - max} and the first
+    // token attaining the max, by a block reduction.
+    __shared__ float sum_s[kGateThreads / 32];
+    __shared__ int idx_s[kGateThreads / 32];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const float cmax = smem[32 + kGateThreads / 32 - 1];
+    float sum = 0.f;
+    int idx = L;
 #pragma unroll
-  for (int e = 0; e < kMaxPerThread; ++e) {
-    if (e >= per) break;
-    if (first + e == L - 1) cmax_s = fmaxf(li[e], moff);  // amax is a running max
-  }
-  __syncthreads();
-  const float cmax = cmax_s;
-  float sum = 0.f;
-  int idx = L;
+    for (int e = 0; e < kMaxPerThread; ++e) {
+      if (e >= per) break;
+      const int r = first + e;
+      if (r < L) {
+        sum += expf(acol[e] - cmax);  // -inf (padding) -> 0
+        if (acol[e] == cmax && r < idx) idx = r;
+      }
+    }
 #pragma unroll
-  for (int e = 0; e < kMaxPerThread; ++e) {
-    if (e >= per) break;
-    const int r = first + e;
-    if (r < L) {
-      sum += expf(acol[e] - cmax);  // -inf (padding) -> 0
-      if (acol[e] == cmax && r < idx) idx = r;
+    for (int o = 16; o; o >>= 1) {
+      sum += __shfl_xor_sync(0xffffffffu, sum, o);
+      idx = min(idx, __shfl_xor_sync(0xffffffffu, idx, o));
+    }
+    if (lane == 0) {
+      sum_s[warp] = sum;
+      idx_s[warp] = idx;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      float tot = 0.f;
+      int best = L;
+      for (int w = 0; w < kGateThreads / 32; ++w) {
+        tot += sum_s[w];
+        best = min(best, idx_s[w]);
+      }
+      g.csum[(long)bh * p.NC + k] = tot;
+      g.cidx[(long)bh * p.NC + k] = best < L ? best : 0;
     }
   }
+}
+
+// One warp per (chunk, b*h), 32 tokens per round: warp scans of lf (sum) and
+// acol (max) carried from round to round.  The sum runs in fp64, so bcum and
+// acol are the fp32 roundings of the exact partial sums.  It also keeps,
+// online, the chunk's largest acol, sum_s e^{acol_s - max} (rescaled when the
+// max grows) and the first token that attains the max.
+__global__ void __launch_bounds__(kGateThreads)
+gates_chunk_warp_kernel(Problem p, const float* __restrict__ i_pre, const float* __restrict__ f_pre,
+                        Gates g) {
+  const int lane = threadIdx.x & 31;
+  const long cid = (long)blockIdx.x * kChunksPerBlock + (threadIdx.x >> 5);
+  if (cid >= (long)p.BH * p.NC) return;
+  const int bh = (int)(cid / p.NC), k = (int)(cid % p.NC);
+  const int L = p.L;
+  const long tpad = (long)p.NC * L;
+  const long base = (long)bh * tpad + (long)k * L;
+  const bool dominance = g.dom != nullptr;
+  double run_b = 0.0;
+  float run_m = -INFINITY;
+  float dmax = -INFINITY, dsum = 0.f;
+  int didx = 0;
+  for (int r0 = 0; r0 < L; r0 += 32) {
+    const int r = r0 + lane;
+    const long t = (long)k * L + r;
+    float lf = 0.f, li = -INFINITY;
+    if (t < p.T) {
+      lf = logsigmoidf(f_pre[(long)bh * p.T + t]);
+      const float x = i_pre[(long)bh * p.T + t];
+      li = p.gate_sigmoid ? logsigmoidf(x) : x;
+    }
+    double bd = lf;
 #pragma unroll
-  for (int o = 16; o; o >>= 1) {
-    sum += __shfl_xor_sync(0xffffffffu, sum, o);
-    idx = min(idx, __shfl_xor_sync(0xffffffffu, idx, o));
+    for (int o = 1; o < 32; o <<= 1) {
+      const double y = __shfl_up_sync(0xffffffffu, bd, o);
+      if (lane >= o) bd += y;
+    }
+    bd += run_b;
+    run_b = __shfl_sync(0xffffffffu, bd, 31);
+    const float b = (float)bd;
+    const float a = (float)((double)li - bd);  // -inf on padding
+    float am = a;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const float y = __shfl_up_sync(0xffffffffu, am, o);
+      if (lane >= o) am = fmaxf(am, y);
+    }
+    am = fmaxf(am, run_m);
+    run_m = __shfl_sync(0xffffffffu, am, 31);
+    g.bcum[base + r] = b;
+    g.acol[base + r] = a;
+    g.amax[base + r] = am;
+    if (dominance) {
+      float e = expf(a - run_m);  // -inf (padding) -> 0; run_m is finite from round 0 on
+#pragma unroll
+      for (int o = 16; o; o >>= 1) e += __shfl_xor_sync(0xffffffffu, e, o);
+      dsum = dsum * expf(dmax - run_m) + e;  // dmax = -inf at first: 0 * 0
+      const unsigned hit = __ballot_sync(0xffffffffu, a == run_m);
+      if (run_m > dmax && hit) didx = r0 + __ffs(hit) - 1;
+      dmax = run_m;
+    }
   }
   if (lane == 0) {
-    sum_s[warp] = sum;
-    idx_s[warp] = idx;
-  }
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    float tot = 0.f;
-    int best = L;
-    for (int w = 0; w < kGateThreads / 32; ++w) {
-      tot += sum_s[w];
-      best = min(best, idx_s[w]);
+    g.gtot[(long)bh * p.NC + k] = (float)run_b;
+    if (dominance) {
+      g.csum[(long)bh * p.NC + k] = dsum;
+      g.cidx[(long)bh * p.NC + k] = didx;
     }
-    g.csum[(long)bh * p.NC + k] = tot;
-    g.cidx[(long)bh * p.NC + k] = best < L ? best : 0;
   }
 }
 
 // One warp per (b, h): m_{k+1} = max(m_k + g_k, c_k) with c_k = g_k + amax at
 // the chunk end.  The maps x -> max(x + G, C) compose associatively:
-// (later o earlier) has G = G_l + G_e and C = max(C_e + G_l, C_l).
+// (later o earlier) has G = G_l + G_e and C = max(C_e + G_l, C_l).  The same
+// prefix maps give M (another starting value) and, with the index of the term
+// that attains C carried along, the dominant token.  Chunks go in groups of
+// 32 (one per lane); the next group's loads are issued before this group's
+// scans.
 __global__ void gates_state_kernel(Problem p, const float* __restrict__ m0, Gates g) {
   const int lane = threadIdx.x & 31;
   const int bh = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (bh >= p.BH) return;
+  const bool dominance = g.dom != nullptr;
   float carry = m0 ? m0[bh] : 0.f;
   float* mchk = g.mchk + (long)bh * (p.NC + 1);
   if (lane == 0) mchk[0] = carry;
   const long tpad = (long)p.NC * p.L;
-  for (int k0 = 0; k0 < p.NC; k0 += 32) {
-    const int k = k0 + lane;
-    float G = 0.f, C = -INFINITY;  // identity map
-    if (k < p.NC) {
-      G = g.gtot[(long)bh * p.NC + k];
-      C = G + g.amax[(long)bh * tpad + (long)k * p.L + p.L - 1];
-    }
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const float Ge = __shfl_up_sync(0xffffffffu, G, o);
-      const float Ce = __shfl_up_sync(0xffffffffu, C, o);
-      if (lane >= o) {
-        C = fmaxf(Ce + G, C);
-        G = G + Ge;
-      }
-    }
-    const float m = fmaxf(carry + G, C);
-    if (k < p.NC) mchk[k + 1] = m;
-    carry = __shfl_sync(0xffffffffu, m, 31);
-  }
-  if (!g.dom) return;
-
-  // Dominance: M_k with the index of the term that attains it (-1: the
-  // initial state), then z_k.  dom_0 = -1: the state entering the first chunk
-  // is the initial state alone (or zero).
-  int* dom = g.dom + (long)bh * p.NC;
-  float* mdom = g.mdom + (long)bh * p.NC;
-  if (lane == 0 && p.NC > 0) {
-    dom[0] = -1;
-    mdom[0] = m0 ? m0[bh] : -INFINITY;
-  }
+  // dominance carries: M (-inf without an initial state), its index (-1: the
+  // initial state), and z
   float cM = m0 ? m0[bh] : -INFINITY, cz = m0 ? 1.f : 0.f;
   int cI = -1;
+  int* dom = dominance ? g.dom + (long)bh * p.NC : nullptr;
+  bool any = false;
+  float* mdom = dominance ? g.mdom + (long)bh * p.NC : nullptr;
+  if (dominance && lane == 0 && p.NC > 0) {
+    dom[0] = -1;
+    mdom[0] = cM;
+  }
+  auto load = [&](int k, float& gk, float& amx, int& ci, float& cs) {
+    gk = 0.f;
+    amx = -INFINITY;
+    ci = 0;
+    cs = 0.f;
+    if (k < p.NC) {
+      gk = g.gtot[(long)bh * p.NC + k];
+      amx = g.amax[(long)bh * tpad + (long)k * p.L + p.L - 1];
+      if (dominance) {
+        ci = g.cidx[(long)bh * p.NC + k];
+        cs = g.csum[(long)bh * p.NC + k];
+      }
+    }
+  };
+  float n_gk, n_amx, n_cs;
+  int n_ci;
+  load(lane, n_gk, n_amx, n_ci, n_cs);
   for (int k0 = 0; k0 < p.NC; k0 += 32) {
     const int k = k0 + lane;
-    float gk = 0.f, G = 0.f, C = -INFINITY, amx = -INFINITY, cs = 0.f;
-    int I = -1;
-    if (k < p.NC) {
-      gk = G = g.gtot[(long)bh * p.NC + k];
-      amx = g.amax[(long)bh * tpad + (long)k * p.L + p.L - 1];
-      C = G + amx;
-      I = k * p.L + g.cidx[(long)bh * p.NC + k];
-      cs = g.csum[(long)bh * p.NC + k];
-    }
+    const float gk = n_gk, amx = n_amx, cs = n_cs;
+    const int ci = n_ci;
+    if (k0 + 32 < p.NC) load(k + 32, n_gk, n_amx, n_ci, n_cs);
+    float G = gk, C = k < p.NC ? gk + amx : -INFINITY;  // identity map past NC
+    int I = k * p.L + ci;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const float Ge = __shfl_up_sync(0xffffffffu, G, o);
@@ -243,6 +311,11 @@ __global__ void gates_state_kernel(Problem p, const float* __restrict__ m0, Gate
         G = G + Ge;
       }
     }
+    const float m = fmaxf(carry + G, C);
+    if (k < p.NC) mchk[k + 1] = m;
+    carry = __shfl_sync(0xffffffffu, m, 31);
+    if (!dominance) continue;
+
     // M_{k+1} and its index; M_k is the previous lane's (or the carry)
     float Mo = C;
     int Io = I;
@@ -272,19 +345,33 @@ __global__ void gates_state_kernel(Problem p, const float* __restrict__ m0, Gate
       dom[k + 1] = (z < 2.f) ? Io : -1;
       mdom[k + 1] = Mo;
     }
+    any = any || __any_sync(0xffffffffu, k + 1 < p.NC && z < 2.f && Io >= 0);
     cM = __shfl_sync(0xffffffffu, Mo, 31);
     cI = __shfl_sync(0xffffffffu, Io, 31);
     cz = __shfl_sync(0xffffffffu, z, 31);
   }
+  if (dominance && lane == 0) g.hdom[bh] = any ? 1 : 0;
 }
 
 }  // namespace
 
 cudaError_t launch_gates(const Problem& p, const float* i_pre, const float* f_pre,
                          const float* m0, Gates g, cudaStream_t st) {
-  if (p.NC > 0) {
+  if (p.NC > 0 && g.dom && p.L > 128) {
     dim3 grid(p.NC, p.BH);
-    gates_chunk_kernel<<<grid, kGateThreads, 0, st>>>(p, i_pre, f_pre, g);
+    gates_chunk_kernel<true><<<grid, kGateThreads, 0, st>>>(p, i_pre, f_pre, g);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  } else if (p.NC > 0 && g.dom) {
+    const long chunks = (long)p.BH * p.NC;
+    const long blocks = (chunks + kChunksPerBlock - 1) / kChunksPerBlock;
+    if (blocks > 0x7fffffffL) return cudaErrorInvalidValue;
+    gates_chunk_warp_kernel<<<(unsigned)blocks, kGateThreads, 0, st>>>(p, i_pre, f_pre, g);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  } else if (p.NC > 0) {
+    dim3 grid(p.NC, p.BH);
+    gates_chunk_kernel<false><<<grid, kGateThreads, 0, st>>>(p, i_pre, f_pre, g);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }

@@ -66,8 +66,9 @@ struct FCfg {
   static constexpr uint32_t kOffN = kOffRedN + kRG * kDK * 4;            // float[kDK]
   static constexpr uint32_t kOffNPrev = kOffN + kDK * 4;                 // float[kDK]: n_k
   static constexpr uint32_t kOffDStar = kOffNPrev + kDK * 4;             // float[kDK]: d_k
+  static constexpr uint32_t kOffNStar = kOffDStar + kDK * 4;             // float[kDK]: n_k - d_k
   // per chunk (2 buffers) and key column: acol, e^{acol - c}, the weight w
-  static constexpr uint32_t kOffAcol = kOffDStar + kDK * 4;              // float[2][3][kL]
+  static constexpr uint32_t kOffAcol = kOffNStar + kDK * 4;              // float[2][3][kL]
   static constexpr uint32_t kOffRed = kOffAcol + 2 * 3 * kL * 4;         // float2[256]
   static constexpr uint32_t kOffBar = kOffRed + 256 * 8;
   static constexpr uint32_t kOffTmemSlot = kOffBar + 256;
@@ -121,6 +122,7 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   float* n_s = reinterpret_cast<float*>(smem + F::kOffN);
   float* nprev_s = reinterpret_cast<float*>(smem + F::kOffNPrev);
   float* dstar_s = reinterpret_cast<float*>(smem + F::kOffDStar);
+  float* nstar_s = reinterpret_cast<float*>(smem + F::kOffNStar);
   float* acol_s = reinterpret_cast<float*>(smem + F::kOffAcol);
   float2* red_s = reinterpret_cast<float2*>(smem + F::kOffRed);
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + F::kOffTmemSlot);
@@ -425,20 +427,30 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         uint32_t v[32];
         tmem_ld32(trow + kColC + h * kHalfV + c, v);
         tmem_wait_ld();
-        uint32_t x[32];
-#pragma unroll
-        for (int e = 0; e < 32; ++e) x[e] = v[e];
-        if (vstar) add_rank1_32(x, nrow, vstar + c);
         const int col0 = h * kHalfV + c;  // first d_v column of these 32
         uint8_t* blk = crow + (col0 >> 6) * 8192;
         const int ch0 = (col0 & 63) >> 3;
+        if (vstar) {
+          uint32_t x[32];
 #pragma unroll
-        for (int e = 0; e < 4; ++e)
-          *reinterpret_cast<uint4*>(blk + (((ch0 + e) ^ (rr & 7)) << 4)) = make_uint4(
-              pack_bf16x2(__uint_as_float(x[8 * e]), __uint_as_float(x[8 * e + 1])),
-              pack_bf16x2(__uint_as_float(x[8 * e + 2]), __uint_as_float(x[8 * e + 3])),
-              pack_bf16x2(__uint_as_float(x[8 * e + 4]), __uint_as_float(x[8 * e + 5])),
-              pack_bf16x2(__uint_as_float(x[8 * e + 6]), __uint_as_float(x[8 * e + 7])));
+          for (int e = 0; e < 32; ++e) x[e] = v[e];
+          add_rank1_32(x, nrow, vstar + c);
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            *reinterpret_cast<uint4*>(blk + (((ch0 + e) ^ (rr & 7)) << 4)) = make_uint4(
+                pack_bf16x2(__uint_as_float(x[8 * e]), __uint_as_float(x[8 * e + 1])),
+                pack_bf16x2(__uint_as_float(x[8 * e + 2]), __uint_as_float(x[8 * e + 3])),
+                pack_bf16x2(__uint_as_float(x[8 * e + 4]), __uint_as_float(x[8 * e + 5])),
+                pack_bf16x2(__uint_as_float(x[8 * e + 6]), __uint_as_float(x[8 * e + 7])));
+        } else {
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            *reinterpret_cast<uint4*>(blk + (((ch0 + e) ^ (rr & 7)) << 4)) = make_uint4(
+                pack_bf16x2(__uint_as_float(v[8 * e]), __uint_as_float(v[8 * e + 1])),
+                pack_bf16x2(__uint_as_float(v[8 * e + 2]), __uint_as_float(v[8 * e + 3])),
+                pack_bf16x2(__uint_as_float(v[8 * e + 4]), __uint_as_float(v[8 * e + 5])),
+                pack_bf16x2(__uint_as_float(v[8 * e + 6]), __uint_as_float(v[8 * e + 7])));
+        }
 #pragma unroll
         for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * decay);
         tmem_st32(trow + kColC + h * kHalfV + c, v);
@@ -462,7 +474,14 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       // a buffer completes once per load; the next load of the buffer needs
       // this chunk's Q released, after this wait.)
       ok = ok && mbar_wait(bar.q_full(b), (j >> 1) & 1, p, 8);
-      // den_inter over this half's 64 dk columns (slab h of Q)
+      // den_inter over this half's 64 dk columns (slab h of Q); a dominated
+      // chunk uses n* = n - d
+      const float* nvec = n_s;
+      if (rv.td >= 0) {
+        if (rt < kDK) nstar_s[rt] = n_s[rt] - dstar_s[rt];
+        named_bar_sync(1, 256);
+        nvec = nstar_s;
+      }
       float dn = 0.f;
       {
         const uint8_t* slab = qbuf + h * 16384;
@@ -472,11 +491,7 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u);
 #pragma unroll
           for (int e = 0; e < 4; e += 2) {
-            float4 nv = *reinterpret_cast<const float4*>(n_s + h * 64 + c * 8 + 2 * e);
-            if (rv.td >= 0) {  // n* = n - d
-              const float4 dv = *reinterpret_cast<const float4*>(dstar_s + h * 64 + c * 8 + 2 * e);
-              nv = make_float4(nv.x - dv.x, nv.y - dv.y, nv.z - dv.z, nv.w - dv.w);
-            }
+            const float4 nv = *reinterpret_cast<const float4*>(nvec + h * 64 + c * 8 + 2 * e);
             const float2 fa = __bfloat1622float2(h2[e]);
             const float2 fb = __bfloat1622float2(h2[e + 1]);
             dn = fmaf(fa.x, nv.x, dn);

@@ -279,9 +279,12 @@ tc_states_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
     uint8_t* stg = smem + S::kOffStg + (warp - 2) * 4096;
     const uint32_t stg_u = sbase + S::kOffStg + (uint32_t)(warp - 2) * 4096u;
     int n_st = 0;  // state stores issued by this warp (selects the tile)
-    // n-vector: worker wt owns dk column wt (DK <= 256) for the running n
-    // (every CTA carries it; the first value tile's CTA writes it out).
-    const bool n_mine = wt < DK;
+    // n-vector: worker wt owns dk column wt (DK <= 256) for the running n.
+    // The first value tile's CTA carries it and writes it out; the others
+    // carry it only when the (b, h) has dominated chunks (their operand copy
+    // then needs n).  need_n is uniform over the CTA, so are fold_n's barriers.
+    const bool need_n = n_owner || (Cb && g.hdom && g.hdom[bh] != 0);
+    const bool n_mine = need_n && wt < DK;
     const bool n_write = n_owner && n_mine;
     float nval = (n_mine && n0 && seg == 0) ? n0[(long)bh * DK + wt] : 0.f;
     // Stage pass mapping: 16-byte column chunk cc (8 dk columns) of token rows
@@ -317,7 +320,7 @@ tc_states_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
     // red_s spans several warps' store tiles, so every warp's stores must have
     // read them first.
     auto fold_n = [&]() {
-      {
+      if (need_n) {
         if (lane == 0) tma_store_wait_read_all();
         named_bar_sync(1, kWorkers);
 #pragma unroll
@@ -405,18 +408,20 @@ tc_states_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
     // the chunk's gate scalars, loaded one chunk ahead (they open every
     // iteration's dependence chain)
     float nx_m_in = mchk[k0], nx_m_out = mchk[k0 + 1], nx_gk = g.gtot[(long)bh * NC + k0];
+    int nx_dom = g.dom ? g.dom[(long)bh * NC + k0] : -1;
     for (int k = k0; k < k1 && ok; ++k) {
       if (k > k0) fold_n();  // chunk k - 1's partials: every worker has passed its stages
       const float m_in = nx_m_in, m_out = nx_m_out, gk = nx_gk;
+      // dominated state: the operand copy leaves as C - n* v_{t*}^T, n* = n - d
+      // (the first segment; later ones get d from the fix-up)
+      const int tdom = Cb ? nx_dom : -1;
       if (k + 1 < k1) {
         nx_m_in = m_out;
         nx_m_out = mchk[k + 2];
         nx_gk = g.gtot[(long)bh * NC + k + 1];
+        if (g.dom) nx_dom = g.dom[(long)bh * NC + k + 1];
       }
       const float decay = expf(gk + m_in - m_out);
-      // dominated state: the operand copy leaves as C - n* v_{t*}^T, n* = n - d
-      // (the first segment; later ones get d from the fix-up)
-      const int tdom = (Cb && g.dom) ? g.dom[(long)bh * NC + k] : -1;
       const __nv_bfloat16* vstar =
           tdom >= 0 ? Vraw + ((long)bh * p.T + tdom) * DV + dv0 : nullptr;
       float nout = nval;
@@ -439,16 +444,26 @@ tc_states_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
             const int col = ch * kColsPer + c;
             if (lane == 0) tma_store_wait_read_all();  // the previous tile has been read
             __syncwarp();
-            const float nrow = vstar ? n_s[dk0 + lane] : 0.f;
+            if (vstar) {  // dominated: C - n* v_{t*}^T
+              const float nrow = n_s[dk0 + lane];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              float x[8];
+              for (int j = 0; j < 8; ++j) {
+                float x[8];
 #pragma unroll
-              for (int e = 0; e < 8; ++e) x[e] = creg[c + 8 * j + e];
-              if (vstar) deflate8(x, nrow, vstar + col + 8 * j);
-              *reinterpret_cast<uint4*>(stg + lane * 128 + ((j ^ (lane & 7)) << 4)) =
-                  make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]),
-                             pack_bf16x2(x[4], x[5]), pack_bf16x2(x[6], x[7]));
+                for (int e = 0; e < 8; ++e) x[e] = creg[c + 8 * j + e];
+                deflate8(x, nrow, vstar + col + 8 * j);
+                *reinterpret_cast<uint4*>(stg + lane * 128 + ((j ^ (lane & 7)) << 4)) =
+                    make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]),
+                               pack_bf16x2(x[4], x[5]), pack_bf16x2(x[6], x[7]));
+              }
+            } else {
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                const float* x = creg + c + 8 * j;
+                *reinterpret_cast<uint4*>(stg + lane * 128 + ((j ^ (lane & 7)) << 4)) =
+                    make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]),
+                               pack_bf16x2(x[4], x[5]), pack_bf16x2(x[6], x[7]));
+              }
             }
             fence_proxy_async_smem();
             __syncwarp();
@@ -502,21 +517,33 @@ tc_states_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
             const int col = ch * kColsPer + c;
             if (lane == 0) tma_store_wait_read_all();  // the previous tile has been read
             __syncwarp();
-            const float nrow = vstar ? n_s[dk0 + lane] : 0.f;
 #pragma unroll 1
             for (int hh = 0; hh < 2; ++hh) {
               uint32_t v[32];
               tmem_ld32(trow + hf * DVT + col + 32 * hh, v);
               tmem_wait_ld();
+              if (vstar) {  // dominated: C - n* v_{t*}^T
+                const float nrow = n_s[dk0 + lane];
 #pragma unroll
-              for (int j = 0; j < 4; ++j) {
-                float x[8];
+                for (int j = 0; j < 4; ++j) {
+                  float x[8];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) x[e] = __uint_as_float(v[8 * j + e]);
-                if (vstar) deflate8(x, nrow, vstar + col + 32 * hh + 8 * j);
-                *reinterpret_cast<uint4*>(stg + lane * 128 + (((4 * hh + j) ^ (lane & 7)) << 4)) =
-                    make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]),
-                               pack_bf16x2(x[4], x[5]), pack_bf16x2(x[6], x[7]));
+                  for (int e = 0; e < 8; ++e) x[e] = __uint_as_float(v[8 * j + e]);
+                  deflate8(x, nrow, vstar + col + 32 * hh + 8 * j);
+                  *reinterpret_cast<uint4*>(stg + lane * 128 +
+                                            (((4 * hh + j) ^ (lane & 7)) << 4)) =
+                      make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]),
+                                 pack_bf16x2(x[4], x[5]), pack_bf16x2(x[6], x[7]));
+                }
+              } else {
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                  *reinterpret_cast<uint4*>(stg + lane * 128 +
+                                            (((4 * hh + j) ^ (lane & 7)) << 4)) = make_uint4(
+                      pack_bf16x2(__uint_as_float(v[8 * j]), __uint_as_float(v[8 * j + 1])),
+                      pack_bf16x2(__uint_as_float(v[8 * j + 2]), __uint_as_float(v[8 * j + 3])),
+                      pack_bf16x2(__uint_as_float(v[8 * j + 4]), __uint_as_float(v[8 * j + 5])),
+                      pack_bf16x2(__uint_as_float(v[8 * j + 6]), __uint_as_float(v[8 * j + 7])));
               }
 #pragma unroll
               for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * decay);
@@ -640,6 +667,8 @@ tc_states_fixup_kernel(Problem p, Gates g, int DVT, const float* __restrict__ se
     col = (t % (DV / 8)) * 8;
   }
   const bool n_thread = col == 0;  // one thread per state row carries n
+  // with dominated chunks every thread needs its row's carried-in n
+  const bool dominated = kOperand && g.hdom && g.hdom[bh] != 0;
   const float* gt = g.gtot + (long)bh * NC;
   const float* mc = g.mchk + (long)bh * (NC + 1);
   auto e_of = [&](int k) { return gt[k] + mc[k] - mc[k + 1]; };
@@ -665,7 +694,7 @@ tc_states_fixup_kernel(Problem p, Gates g, int DVT, const float* __restrict__ se
     const float ev[8] = {e0.x, e0.y, e0.z, e0.w, e1.x, e1.y, e1.z, e1.w};
 #pragma unroll
     for (int i = 0; i < 8; ++i) cs[i] = fmaf(A, cs[i], ev[i]);
-    ns = fmaf(A, ns, seg_n[((long)bh * (n_seg - 1) + s) * DK + dk]);
+    if (n_thread || dominated) ns = fmaf(A, ns, seg_n[((long)bh * (n_seg - 1) + s) * DK + dk]);
   }
 
   const int k0 = seg * ncs, k1 = min(k0 + ncs, NC);
@@ -683,14 +712,24 @@ tc_states_fixup_kernel(Problem p, Gates g, int DVT, const float* __restrict__ se
     float exc = __shfl_up_sync(0xffffffffu, inc, 1);
     if (lane == 0) exc = 0.f;
     const float a_lane = expf(lg + exc);
+    const int td_lane = (dominated && kl < k1) ? g.dom[(long)bh * NC + kl] : -1;
+    const bool any_td = dominated && __any_sync(0xffffffffu, td_lane >= 0);
     lg += __shfl_sync(0xffffffffu, inc, 31);
     const int nb = min(32, k1 - kb);
     for (int c0 = 0; c0 < nb; c0 += 4) {
       // four chunks at a time: loads first, so that they overlap
       constexpr int kB = 4;
       float a[kB];
+      int tds[kB];
 #pragma unroll
-      for (int u = 0; u < kB; ++u) a[u] = __shfl_sync(0xffffffffu, a_lane, (c0 + u) & 31);
+      for (int u = 0; u < kB; ++u) {
+        a[u] = __shfl_sync(0xffffffffu, a_lane, (c0 + u) & 31);
+        tds[u] = -1;
+      }
+      if (any_td) {
+#pragma unroll
+        for (int u = 0; u < kB; ++u) tds[u] = __shfl_sync(0xffffffffu, td_lane, (c0 + u) & 31);
+      }
       if (kOperand) {
         uint4 v[kB];
         __nv_bfloat16* ptr[kB];
@@ -704,24 +743,31 @@ tc_states_fixup_kernel(Problem p, Gates g, int DVT, const float* __restrict__ se
 #pragma unroll
         for (int u = 0; u < kB; ++u) {
           if (c0 + u < nb) {
-            float add[8], res[8];
+            __nv_bfloat162* h2 = reinterpret_cast<__nv_bfloat162*>(&v[u]);
+            if (any_td && tds[u] >= 0) {
+              const int td = tds[u];
+              float add[8], res[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              add[i] = cs[i];
-              res[i] = 0.f;
-            }
-            const int td = g.dom ? g.dom[(long)bh * NC + kb + c0 + u] : -1;
-            if (td >= 0) {
+              for (int i = 0; i < 8; ++i) {
+                add[i] = cs[i];
+                res[i] = 0.f;
+              }
               const __nv_bfloat16* vs = Vraw + ((long)bh * p.T + td) * DV + col;
               deflate8(add, ns, vs);
               deflate8(res, -dom_residual(g, p, bh, kb + c0 + u, td, dk, Kraw), vs);
-            }
-            __nv_bfloat162* h2 = reinterpret_cast<__nv_bfloat162*>(&v[u]);
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float2 f = __bfloat1622float2(h2[e]);
-              h2[e] = __floats2bfloat162_rn(fmaf(a[u], add[2 * e], f.x) + res[2 * e],
-                                            fmaf(a[u], add[2 * e + 1], f.y) + res[2 * e + 1]);
+              for (int e = 0; e < 4; ++e) {
+                const float2 f = __bfloat1622float2(h2[e]);
+                h2[e] = __floats2bfloat162_rn(fmaf(a[u], add[2 * e], f.x) + res[2 * e],
+                                              fmaf(a[u], add[2 * e + 1], f.y) + res[2 * e + 1]);
+              }
+            } else {
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float2 f = __bfloat1622float2(h2[e]);
+                h2[e] = __floats2bfloat162_rn(fmaf(a[u], cs[2 * e], f.x),
+                                              fmaf(a[u], cs[2 * e + 1], f.y));
+              }
             }
             *reinterpret_cast<uint4*>(ptr[u]) = v[u];
           }
@@ -753,7 +799,7 @@ tc_states_fixup_kernel(Problem p, Gates g, int DVT, const float* __restrict__ se
         for (int u = 0; u < kB; ++u) {
           if (c0 + u < nb) {
             const int kc = kb + c0 + u;
-            const int td = (kOperand && g.dom) ? g.dom[(long)bh * NC + kc] : -1;
+            const int td = tds[u];
             const float d = td >= 0 ? dom_residual(g, p, bh, kc, td, dk, Kraw) : 0.f;
             n_states[((long)bh * NC + kc) * DK + dk] += a[u] * ns - d;
           }

@@ -60,17 +60,17 @@ def test_workspace_size_formula(L):
     NC = T // Lc
     r = lambda x: (x + 255) // 256 * 256  # noqa: E731
     # per-token bcum/acol/amax, per-chunk g, m (NC + 1), and per-chunk weight
-    # sum, argmax, dominant token and its log-weight
+    # sum, argmax, dominant token and its log-weight, and a per-head flag
     gates = 3 * r(B * NH * NC * Lc * 4) + r(B * NH * NC * 4) + r(B * NH * (NC + 1) * 4) + \
-        4 * r(B * NH * NC * 4)
+        4 * r(B * NH * NC * 4) + r(B * NH * 4)
     states = r(B * NH * NC * DK * DV * 4) + r(B * NH * NC * DK * 4)
     assert n == gates + states
     # ragged T rounds the chunk count up
     st, n2 = ws(T=200)
     assert st == _lib.OK and n2 == n
-    # empty sequence needs only the stabiliser slot per head
+    # empty sequence needs only the stabiliser slot and the flag per head
     st, n0 = ws(T=0)
-    assert st == _lib.OK and n0 == r(B * NH * 4)
+    assert st == _lib.OK and n0 == 2 * r(B * NH * 4)
 
 
 @pytest.mark.parametrize("kw,expect", [
