@@ -59,7 +59,7 @@ def test_roofline_bound_follows_intensity(bench):
 
 def test_measured_traffic_is_dropped_when_the_sources_change(bench, monkeypatch):
     files = ["tc_parallel_wide.cu", "tc_ptx.cuh"]
-    entry = {"bytes": 1.0e9, "profile": "p", "sources": files,
+    entry = {"bytes": 1.0e9, "sources": files,
              "sha1": bench.sources_sha1(files)}
     monkeypatch.setitem(bench.MEASURED_TRAFFIC, ("tc_parallel", "probe"), entry)
     assert bench.measured_traffic("tc_parallel", "probe") == 1.0e9
@@ -69,12 +69,32 @@ def test_measured_traffic_is_dropped_when_the_sources_change(bench, monkeypatch)
     assert bench.measured_traffic("tc_parallel", "no-such-workload") is None
 
 
-def test_recorded_traffic_entries_name_existing_profiles_and_sources(bench):
+def test_recorded_traffic_entries_name_existing_sources(bench):
     for (fam, workload), e in bench.MEASURED_TRAFFIC.items():
-        assert os.path.exists(os.path.join(ROOT, e["profile"])), e["profile"]
         for f in e["sources"]:
             assert os.path.exists(os.path.join(ROOT, "mlstm_chunkwise_b200", "csrc", f)), f
-        assert len(e["sha1"]) == 40
+        assert len(e["sha1"]) == 40 and e["bytes"] > 0
+
+
+def test_roofline_uses_the_methods_bytes(bench):
+    """At the 7B shape the output kernel's method bytes are Q, K, V read and H
+    written (1.617 GB); its own bytes add the bf16 chunk states, n and gates."""
+    s = SHAPE_7B
+    mb = bench.method_bytes("tc_parallel", s["B"], s["NH"], s["T"], s["DK"], s["DV"], 2, False)
+    BH = s["B"] * s["NH"]
+    assert mb == BH * s["T"] * (2 * s["DK"] + 2 * s["DV"]) * 2
+    kb = bench.kernel_bytes("tc_parallel", s["B"], s["NH"], s["T"], s["DK"], s["DV"], s["L"], 2)
+    assert kb > mb
+    peaks = {"hbm_gbs": 6550.4, "bf16_tflops": 1646.3, "bf16_tflops_sustained": 1387.9}
+    fph = bench.flops_per_head(s["T"], s["DK"], s["DV"], s["L"])
+    flops = BH * (fph["inter"] + fph["intra"])
+    roof = bench.roofline("tc_parallel", 0.5, flops,
+                          (s["B"], s["NH"], s["T"], s["DK"], s["DV"], s["L"], 2), peaks,
+                          "measured", False, "none")
+    assert roof["bound"] == "hbm"
+    assert abs(roof["frac"] - mb / 0.5e-3 / 1e9 / 6550.4) < 1e-12
+    assert roof["frac_hbm_kernel_bytes"] > roof["frac"]
+    assert abs(roof["frac_tensor"] - flops / 0.5e-3 / 1e12 / 1646.3) < 1e-12
 
 
 def test_chunk_state_bytes_by_path(bench):
