@@ -8,6 +8,9 @@ The arithmetic lives in ``mlstm_oracle.c`` (plain C, fp64, token-by-token
 recurrence; see its header for the formula and the passages it follows).  This
 module only compiles that file with gcc and marshals numpy arrays into it.
 
+The sigmoid-input-gate variant with reduced computation (no stabiliser, no
+normaliser) is a separate function written from its plain definition.
+
 Parity pins (all in ``tests/test_oracle_pins.py``): the quadratic parallel form,
 chunk-size invariance of an independent chunkwise derivation, the single-token
 closed form, memory hold, the reduction to causal normalised linear attention,
@@ -52,6 +55,8 @@ def open_library(path: str):
         [dp] * 8 + [ctypes.c_int] * 6 + [dp] * 6 + [ctypes.c_int] + [dp] * 3
     )
     lib.mlstm_oracle_num_threads.restype = ctypes.c_int
+    lib.mlstm_oracle_sigmoid_plain.restype = ctypes.c_int
+    lib.mlstm_oracle_sigmoid_plain.argtypes = [dp] * 8 + [ctypes.c_int] * 5 + [dp] * 3
     return lib
 
 
@@ -128,3 +133,27 @@ def mlstm_recurrent(Q, K, V, i_pre, f_pre, C0=None, n0=None, m0=None,
     if rc != 0:
         raise ValueError("mlstm_oracle_recurrent rejected its arguments")
     return out
+
+
+def mlstm_sigmoid_plain(Q, K, V, i_pre, f_pre, C0=None, n0=None, m0=None, lib=None) -> dict:
+    """The sigmoid-input-gate variant with reduced computation, from its plain
+    definition (unstabilised, no normaliser; see ``mlstm_oracle_sigmoid_plain``
+    in ``mlstm_oracle.c``): h_t = C_t^T q_t with
+    C_t = sigmoid(f~_t) C_{t-1} + sigmoid(i~_t) (s k_t) v_t^T.
+
+    Returns H [B,NH,T,DV] and the unstabilised final state C_T [B,NH,DK,DV],
+    n_T [B,NH,DK] (frame m = 0)."""
+    lib = _load() if lib is None else lib
+    Q, K, V, i_pre, f_pre = (_f64(a) for a in (Q, K, V, i_pre, f_pre))
+    C0, n0, m0 = _f64(C0), _f64(n0), _f64(m0)
+    B, NH, T, DK = Q.shape
+    DV = V.shape[-1]
+    H = np.zeros((B, NH, T, DV))
+    C_T = np.zeros((B, NH, DK, DV))
+    n_T = np.zeros((B, NH, DK))
+    rc = lib.mlstm_oracle_sigmoid_plain(
+        _ptr(Q), _ptr(K), _ptr(V), _ptr(i_pre), _ptr(f_pre), _ptr(C0), _ptr(n0), _ptr(m0),
+        B, NH, T, DK, DV, _ptr(H), _ptr(C_T), _ptr(n_T))
+    if rc != 0:
+        raise RuntimeError("mlstm_oracle_sigmoid_plain failed")
+    return dict(H=H, C_T=C_T, n_T=n_T)

@@ -152,6 +152,79 @@ int mlstm_oracle_recurrent(const double* Q, const double* K, const double* V,
   return bad ? -1 : 0;
 }
 
+/*
+ * The sigmoid-input-gate variant with reduced computation.  "Tiled Flash
+ * Linear Attention: More Efficient Linear RNN and xLSTM Kernels" (abstract)
+ * introduces an mLSTM variant with a sigmoid input gate that needs less
+ * computation; the page does not define it further.  Reading: with both gates
+ * sigmoids every gate value lies in (0, 1), the memory cannot grow without
+ * bound, and the variant drops the max-state stabiliser and the normaliser:
+ *
+ *   C_t = sigmoid(f~_t) C_{t-1} + sigmoid(i~_t) (s k_t) v_t^T
+ *   h_t = C_t^T q_t                           (no normaliser, no division)
+ *
+ * This is that definition written out, token by token, in fp64, with no
+ * stabiliser.  n_t = sigmoid(f~_t) n_{t-1} + sigmoid(i~_t) (s k_t) is carried
+ * only so that the final state can be compared with the other modes' (it
+ * does not enter h).  The initial state (C0, n0) is given in the frame m0, as
+ * in the other modes: the recurrence starts from e^{m0} C0 and e^{m0} n0.
+ * The final state is returned unstabilised (the frame m = 0).
+ *
+ * Inputs as mlstm_oracle_recurrent; outputs H [B, NH, T, DV] and, where not
+ * NULL, C_T [B, NH, DK, DV] and n_T [B, NH, DK].
+ */
+static double oracle_sigmoid(double x) {
+  if (x >= 0.0) return 1.0 / (1.0 + exp(-x));
+  const double e = exp(x);
+  return e / (1.0 + e);
+}
+
+int mlstm_oracle_sigmoid_plain(const double* Q, const double* K, const double* V,
+                               const double* i_pre, const double* f_pre, const double* C0,
+                               const double* n0, const double* m0, int B, int NH, int T, int DK,
+                               int DV, double* H, double* C_T, double* n_T) {
+  if (B < 1 || NH < 1 || T < 0 || DK < 1 || DV < 1 || !H) return -1;
+  if (!((C0 && n0 && m0) || (!C0 && !n0 && !m0))) return -1;
+  const double s = 1.0 / sqrt((double)DK);
+  const long BH = (long)B * NH;
+  int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+  for (long bh = 0; bh < BH; ++bh) {
+    double* C = (double*)calloc((size_t)DK * DV, sizeof(double));
+    double* n = (double*)calloc((size_t)DK, sizeof(double));
+    if (!C || !n) {
+      bad = 1;
+      free(C); free(n);
+      continue;
+    }
+    if (C0) {
+      const double sc = exp(m0[bh]);
+      for (long a = 0; a < (long)DK * DV; ++a) C[a] = sc * C0[bh * DK * DV + a];
+      for (int a = 0; a < DK; ++a) n[a] = sc * n0[bh * DK + a];
+    }
+    for (int t = 0; t < T; ++t) {
+      const double f = oracle_sigmoid(f_pre[bh * T + t]);
+      const double ig = oracle_sigmoid(i_pre[bh * T + t]);
+      const double* k = K + ((long)bh * T + t) * DK;
+      const double* v = V + ((long)bh * T + t) * DV;
+      const double* q = Q + ((long)bh * T + t) * DK;
+      for (int a = 0; a < DK; ++a) {
+        const double wk = ig * s * k[a];
+        for (int j = 0; j < DV; ++j) C[a * DV + j] = f * C[a * DV + j] + wk * v[j];
+        n[a] = f * n[a] + wk;
+      }
+      double* h = H + ((long)bh * T + t) * DV;
+      for (int j = 0; j < DV; ++j) h[j] = 0.0;
+      for (int a = 0; a < DK; ++a)
+        for (int j = 0; j < DV; ++j) h[j] += C[a * DV + j] * q[a];
+    }
+    if (C_T) memcpy(C_T + bh * DK * DV, C, sizeof(double) * (size_t)DK * DV);
+    if (n_T) memcpy(n_T + bh * DK, n, sizeof(double) * (size_t)DK);
+    free(C); free(n);
+  }
+  return bad ? -1 : 0;
+}
+
 /* Number of OpenMP threads a parallel region of this library uses. */
 int mlstm_oracle_num_threads(void) {
 #ifdef _OPENMP

@@ -30,6 +30,8 @@ import os
 
 import numpy as np
 
+import oracle
+
 GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden",
                       "hand_derived_sequences.json")
 
@@ -333,3 +335,88 @@ def pin_snapshots(run):
 
 ALL_PINS = [pin_quadratic, pin_chunkwise, pin_single_token, pin_memory_hold,
             pin_linear_attention, pin_golden, pin_invariants, pin_snapshots]
+
+
+# ----------------------------------------------------------------------------
+# the sigmoid-input-gate variant with reduced computation (no stabiliser, no
+# normaliser): h_t = C_t^T q_t, C_t = sig(f~_t) C_{t-1} + sig(i~_t) (s k_t) v_t^T
+# ----------------------------------------------------------------------------
+
+def quadratic_form_sigmoid_plain(Q, K, V, i_pre, f_pre, C0=None, n0=None, m0=None):
+    """Fully parallel form of the variant, per (b, h): with F_t = sum_{l<=t}
+    log sig(f~_l), token j enters the read-out at t with weight
+    sig(i~_j) exp(F_t - F_j) (j <= t) and the initial state with
+    exp(F_t + m0); H = ((s Q K^T) o W) V + exp(F + m0) (Q C0).  The final state
+    is the same sum at t = T."""
+    B, NH, T, DK = Q.shape
+    DV = V.shape[-1]
+    s = 1.0 / math.sqrt(DK)
+    H = np.zeros((B, NH, T, DV))
+    C_T = np.zeros((B, NH, DK, DV))
+    n_T = np.zeros((B, NH, DK))
+    for b in range(B):
+        for h in range(NH):
+            lf = logsigmoid(f_pre[b, h])
+            li = logsigmoid(i_pre[b, h])
+            F = np.cumsum(lf)
+            causal = np.tril(np.ones((T, T), dtype=bool))
+            W = np.where(causal, np.exp(F[:, None] - F[None, :] + li[None, :]), 0.0)
+            H[b, h] = (W * (s * Q[b, h] @ K[b, h].T)) @ V[b, h]
+            wT = np.exp(F[-1] - F + li) if T else np.zeros(0)
+            C_T[b, h] = (K[b, h] * (s * wT)[:, None]).T @ V[b, h]
+            n_T[b, h] = (K[b, h] * (s * wT)[:, None]).sum(axis=0)
+            if C0 is not None:
+                g = np.exp(F + float(m0[b, h]))
+                H[b, h] += g[:, None] * (Q[b, h] @ C0[b, h])
+                gT = math.exp((F[-1] if T else 0.0) + float(m0[b, h]))
+                C_T[b, h] += gT * C0[b, h]
+                n_T[b, h] += gT * n0[b, h]
+    return dict(H=H, C_T=C_T, n_T=n_T)
+
+
+def pin_sig_quadratic(run_plain):
+    for init in (False, True):
+        c = rand_case(31, T=40, init_state=init)
+        o = run_plain(**c)
+        r = quadratic_form_sigmoid_plain(**c)
+        assert rel_err(o["H"], r["H"]) < TOL, "plain sigmoid H vs quadratic form"
+        assert rel_err(o["C_T"], r["C_T"]) < TOL, "plain sigmoid C_T vs quadratic form"
+        assert rel_err(o["n_T"], r["n_T"]) < TOL, "plain sigmoid n_T vs quadratic form"
+
+
+def pin_sig_single_token(run_plain):
+    """T = 1 from a zero state: h = sig(i~) s (k.q) v."""
+    c = rand_case(32, T=1, DK=5, DV=3)
+    o = run_plain(**c)
+    q, k, v = c["Q"][0, :, 0], c["K"][0, :, 0], c["V"][0, :, 0]
+    ig = 1.0 / (1.0 + np.exp(-c["i_pre"][0, :, 0]))
+    want = (ig * (q * k).sum(-1) / math.sqrt(5))[:, None] * v
+    assert rel_err(o["H"][0, :, 0], want) < TOL, "plain sigmoid single token"
+
+
+def pin_sig_memory_hold(run_plain):
+    """sig(f~) = 1 and sig(i~) = 0 (f~ = +1e4, i~ = -1e4): h_t = e^{m0} C0^T q_t."""
+    c = rand_case(33, T=12, init_state=True)
+    c["f_pre"] = np.full_like(c["f_pre"], 1e4)
+    c["i_pre"] = np.full_like(c["i_pre"], -1e4)
+    o = run_plain(**c)
+    want = np.exp(c["m0"])[:, :, None, None] * np.einsum("bhtk,bhkv->bhtv", c["Q"], c["C0"])
+    assert rel_err(o["H"], want) < TOL, "plain sigmoid memory hold"
+
+
+def pin_sig_against_stabilised(run_plain):
+    """The variant's state is the sigmoid mode's state in the frame m = 0, and
+    its output is that mode's h times its denominator and e^{m}: the two oracle
+    functions (different code) must agree on both."""
+    c = rand_case(34, T=36, init_state=True)
+    o = run_plain(**c)
+    st = oracle.mlstm_recurrent(**c, gate_mode="sigmoid")
+    e = np.exp(st["m_T"])
+    assert rel_err(o["C_T"], e[:, :, None, None] * st["C_T"]) < TOL, "plain vs stabilised C_T"
+    assert rel_err(o["n_T"], e[:, :, None] * st["n_T"]) < TOL, "plain vs stabilised n_T"
+    scale = np.exp(st["m"]) * st["den"]
+    assert rel_err(o["H"], st["H"] * scale[..., None]) < TOL, "plain vs stabilised H"
+
+
+SIG_PLAIN_PINS = [pin_sig_quadratic, pin_sig_single_token, pin_sig_memory_hold,
+                  pin_sig_against_stabilised]

@@ -61,3 +61,40 @@ def test_mutant_fails_a_pin(name, tmpdir_str):
         except (AssertionError, ValueError, FloatingPointError):
             caught.append(pin.__name__)
     assert caught, f"mutant {name} passes every pin"
+
+
+# Mutants of the sigmoid-input-gate variant's oracle function (plain
+# definition, no stabiliser, no normaliser); caught by pins.SIG_PLAIN_PINS.
+SIG_MUTANTS = {
+    "plain_input_gate_raw": ("const double ig = oracle_sigmoid(i_pre[bh * T + t]);",
+                             "const double ig = i_pre[bh * T + t];"),
+    "plain_no_forget": ("C[a * DV + j] = f * C[a * DV + j] + wk * v[j];",
+                        "C[a * DV + j] = C[a * DV + j] + wk * v[j];"),
+    "plain_missing_key_scale": ("const double wk = ig * s * k[a];",
+                                "const double wk = ig * k[a];"),
+    "plain_initial_frame_ignored": ("const double sc = exp(m0[bh]);", "const double sc = 1.0;"),
+    "plain_sigmoid_sign": ("if (x >= 0.0) return 1.0 / (1.0 + exp(-x));",
+                           "if (x >= 0.0) return 1.0 / (1.0 + exp(x));"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(SIG_MUTANTS))
+def test_sigmoid_plain_mutant_fails_a_pin(name, tmpdir_str):
+    old, new = SIG_MUTANTS[name]
+    src = open(SRC).read()
+    assert src.count(old) == 1, f"mutation anchor for {name} not found exactly once"
+    path_c = os.path.join(tmpdir_str, f"{name}.c")
+    path_so = os.path.join(tmpdir_str, f"lib{name}.so")
+    with open(path_c, "w") as fh:
+        fh.write(src.replace(old, new))
+    subprocess.run(["gcc", "-O2", "-fPIC", "-shared", "-fopenmp", "-std=c99", path_c, "-o",
+                    path_so, "-lm"], check=True)
+    lib = oracle.open_library(path_so)
+    run = functools.partial(oracle.mlstm_sigmoid_plain, lib=lib)
+    caught = []
+    for pin in pins.SIG_PLAIN_PINS:
+        try:
+            pin(run)
+        except (AssertionError, ValueError, FloatingPointError):
+            caught.append(pin.__name__)
+    assert caught, f"mutant {name} passes every pin"

@@ -48,3 +48,8 @@ def test_bf16_inputs_up_cast_exactly():
     c = {k: x[k].double().numpy() for k in ("Q", "K", "V", "i_pre", "f_pre")}
     r = pins.quadratic_form(**c)
     assert pins.rel_err(o["H"], r["H"]) < 1e-10
+
+
+@pytest.mark.parametrize("pin", pins.SIG_PLAIN_PINS, ids=lambda p: p.__name__)
+def test_sigmoid_plain_oracle_pin(pin):
+    pin(oracle.mlstm_sigmoid_plain)
