@@ -306,6 +306,16 @@ class ClockSampler:
 # ----------------------------------------------------------------------------
 # CPU baseline: the fp64 oracle on a bounded sample of the workload
 # ----------------------------------------------------------------------------
+def oracle_forward(oracle, c, gate_mode):
+    """The oracle's forward pass for one input dict (the sigmoid variant without
+    normaliser has a function of its own)."""
+    if gate_mode == "sigmoid_plain":
+        return oracle.mlstm_sigmoid_plain(c["Q"], c["K"], c["V"], c["i_pre"], c["f_pre"],
+                                          c["C0"], c["n0"], c["m0"])
+    return oracle.mlstm_recurrent(c["Q"], c["K"], c["V"], c["i_pre"], c["f_pre"], c["C0"],
+                                  c["n0"], c["m0"], gate_mode=gate_mode)
+
+
 def oracle_sample(w, x, target_s=15.0):
     """Time the oracle on a leading block of heads x tokens of the workload,
     sized from a short calibration run to take about `target_s` seconds.
@@ -327,8 +337,7 @@ def oracle_sample(w, x, target_s=15.0):
     def timed(heads, tokens):
         c = sub(heads, tokens)
         t0 = time.perf_counter()
-        oracle.mlstm_recurrent(c["Q"], c["K"], c["V"], c["i_pre"], c["f_pre"], c["C0"], c["n0"],
-                               c["m0"], gate_mode=w.gate_mode)
+        oracle_forward(oracle, c, w.gate_mode)
         return time.perf_counter() - t0
 
     h_cal = min(BH, cores)
@@ -392,8 +401,7 @@ def run_reference(args):
         c[k] = None if x[k] is None else torch.stack([x[k][b, h] for b, h in sel]).unsqueeze(0)
 
     def step():
-        oracle.mlstm_recurrent(c["Q"], c["K"], c["V"], c["i_pre"], c["f_pre"], c["C0"], c["n0"],
-                               c["m0"], gate_mode=w.gate_mode)
+        oracle_forward(oracle, c, w.gate_mode)
 
     for _ in range(args.warmup):
         step()

@@ -70,7 +70,29 @@ typedef enum {
 
 typedef enum { MLSTM_DT_F32 = 0, MLSTM_DT_BF16 = 1 } mlstm_dtype;
 
-typedef enum { MLSTM_GATE_EXP = 0, MLSTM_GATE_SIGMOID = 1 } mlstm_gate_mode;
+/* Gate activations.
+ *   EXP             log i = i~ (exponential input gate)
+ *   SIGMOID         log i = logsigmoid(i~)
+ *   SIGMOID_PLAIN   the sigmoid-input-gate variant with reduced computation
+ *                   ("Tiled Flash Linear Attention: More Efficient Linear RNN
+ *                   and xLSTM Kernels", abstract).  Read as: with both gates
+ *                   sigmoids every gate value lies in (0, 1), so the output
+ *                   needs no normaliser and no stabiliser,
+ *                     h_t = C_t^T q_t  with the unstabilised
+ *                     C_t = sig(f~_t) C_{t-1} + sig(i~_t) (s k_t) v_t^T.
+ *                   The kernels still carry the stabiliser internally (a
+ *                   choice of frame that h does not depend on); what the
+ *                   variant removes is the normaliser's reductions and the
+ *                   division.  The returned final state is the SIGMOID mode's
+ *                   (C_T, n_T in the frame m_T: the unstabilised state is
+ *                   e^{m_T} C_T).  Forward, chunk-state, parallel and step
+ *                   calls only: the backward and training calls return
+ *                   MLSTM_ERR_UNSUPPORTED. */
+typedef enum {
+  MLSTM_GATE_EXP = 0,
+  MLSTM_GATE_SIGMOID = 1,
+  MLSTM_GATE_SIGMOID_PLAIN = 2
+} mlstm_gate_mode;
 
 /* Which kernels compute the path.
  *   AUTO      TC_FUSED where it is supported and there are at least 592
@@ -137,7 +159,8 @@ mlstm_status mlstm_fw_chunk_states(const void* K, const void* V, const float* i_
 
 /* Parallel half: H from Q, K, V, the gates and the chunk states produced by
  * mlstm_fw_chunk_states (same m0 and gates).  Optional per-token outputs:
- *   n_out [B, NH, T] = max(|n_t^T q_t|, e^{-m_t}) (the denominator), and
+ *   n_out [B, NH, T] = max(|n_t^T q_t|, e^{-m_t}) (the denominator; e^{-m_t}
+ *   for MLSTM_GATE_SIGMOID_PLAIN), and
  *   m_out [B, NH, T] = m_t.  Algorithm SIMT or TC (AUTO picks). */
 mlstm_status mlstm_fw_parallel(const void* Q, const void* K, const void* V, const float* i_pre,
                                const float* f_pre, const float* m0, const float* C_states,
@@ -229,7 +252,8 @@ mlstm_status mlstm_bw_saved(const void* Q, const void* K, const void* V, const f
  *   C [B, NH, DK, DV], n [B, NH, DK], m [B, NH] fp32: the state before the
  *   token on entry, after it on return (a zero state is C = n = 0, m = 0).
  *   m' = max(logsigmoid(f~) + m, li), C' = fa C + ia (s k) v^T,
- *   n' = fa n + ia s k, h = C'^T q / max(|n'^T q|, e^{-m'}), s = 1/sqrt(DK).
+ *   n' = fa n + ia s k, h = C'^T q / max(|n'^T q|, e^{-m'}), s = 1/sqrt(DK)
+ *   (MLSTM_GATE_SIGMOID_PLAIN: h = e^{m'} C'^T q).
  * Sizes: B, NH >= 1, DK, DV in [1, 1024].  No workspace; asynchronous on
  * `stream`: one launch (a thread-block cluster per head), or two when d_v is
  * not a multiple of 4 and above 256 (a head then spans more column tiles

@@ -14,7 +14,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmlstm_fw
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_DEVICE = range(6)
 ERR_SCRATCH_TOO_SMALL = 6
 DT_F32, DT_BF16 = 0, 1
-GATE_EXP, GATE_SIGMOID = 0, 1
+GATE_EXP, GATE_SIGMOID, GATE_SIGMOID_PLAIN = 0, 1, 2
 ALGO_AUTO, ALGO_SIMT, ALGO_TC, ALGO_TC_FUSED = 0, 1, 2, 3
 KERNEL_COUNT = 9
 

@@ -15,7 +15,8 @@ from . import _lib
 from ._lib import MlstmError  # noqa: F401  (re-export)
 
 _DT = {torch.float32: _lib.DT_F32, torch.bfloat16: _lib.DT_BF16}
-_GATE = {"exp": _lib.GATE_EXP, "sigmoid": _lib.GATE_SIGMOID}
+_GATE = {"exp": _lib.GATE_EXP, "sigmoid": _lib.GATE_SIGMOID,
+         "sigmoid_plain": _lib.GATE_SIGMOID_PLAIN}
 _ALGO = {"auto": _lib.ALGO_AUTO, "simt": _lib.ALGO_SIMT, "tc": _lib.ALGO_TC,
          "tc_fused": _lib.ALGO_TC_FUSED}
 

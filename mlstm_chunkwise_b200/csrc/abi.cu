@@ -54,7 +54,8 @@ Problem make_problem(int B, int NH, int T, int DK, int DV, int L, mlstm_gate_mod
   p.L = L;
   p.NC = (T + L - 1) / L;
   p.BH = B * NH;
-  p.gate_sigmoid = gm == MLSTM_GATE_SIGMOID;
+  p.gate_sigmoid = gm == MLSTM_GATE_SIGMOID || gm == MLSTM_GATE_SIGMOID_PLAIN;
+  p.no_norm = gm == MLSTM_GATE_SIGMOID_PLAIN;
   p.key_scale = (float)(1.0 / sqrt((double)DK));
   p.signed_den = 0;
   p.err = nullptr;
@@ -133,7 +134,7 @@ char* carve_gates(const Problem& p, char* ws, Gates* g, float* mchk_override,
 
 bool valid_enums(mlstm_dtype dt, mlstm_gate_mode gm, mlstm_algo algo) {
   return (dt == MLSTM_DT_F32 || dt == MLSTM_DT_BF16) &&
-         (gm == MLSTM_GATE_EXP || gm == MLSTM_GATE_SIGMOID) &&
+         (gm == MLSTM_GATE_EXP || gm == MLSTM_GATE_SIGMOID || gm == MLSTM_GATE_SIGMOID_PLAIN) &&
          (algo == MLSTM_ALGO_AUTO || algo == MLSTM_ALGO_SIMT || algo == MLSTM_ALGO_TC ||
           algo == MLSTM_ALGO_TC_FUSED);
 }
@@ -489,6 +490,7 @@ mlstm_status mlstm_bw(const void* Q, const void* K, const void* V, const float* 
   if (!valid_enums(dtype, gate_mode, MLSTM_ALGO_AUTO)) return MLSTM_ERR_INVALID_ARG;
   mlstm_status s = check_sizes(B, NH, T, DK, DV, chunk_size);
   if (s != MLSTM_OK) return s;
+  if (gate_mode == MLSTM_GATE_SIGMOID_PLAIN) return MLSTM_ERR_UNSUPPORTED;
   if (!((C0 && n0 && m0) || (!C0 && !n0 && !m0))) return MLSTM_ERR_INVALID_ARG;
   if (T > 0 && (!Q || !K || !V || !i_pre || !f_pre || !dH || !dQ || !dK || !dV || !di_pre ||
                 !df_pre))
@@ -544,7 +546,7 @@ mlstm_status mlstm_fw_train(const void* Q, const void* K, const void* V, const f
   mlstm_status s = check_sizes(B, NH, T, DK, DV, 128);
   if (s != MLSTM_OK) return s;
   Problem p = make_problem(B, NH, T, DK, DV, 128, gate_mode);
-  if (!train_supported(p, dtype)) return MLSTM_ERR_UNSUPPORTED;
+  if (!train_supported(p, dtype) || p.no_norm) return MLSTM_ERR_UNSUPPORTED;
   if (!Q || !K || !V || !i_pre || !f_pre || !H || !saved || !workspace)
     return MLSTM_ERR_INVALID_ARG;
   if (!((C0 && n0 && m0) || (!C0 && !n0 && !m0))) return MLSTM_ERR_INVALID_ARG;
@@ -574,7 +576,7 @@ mlstm_status mlstm_bw_saved(const void* Q, const void* K, const void* V, const f
   mlstm_status s = check_sizes(B, NH, T, DK, DV, 128);
   if (s != MLSTM_OK) return s;
   Problem p = make_problem(B, NH, T, DK, DV, 128, gate_mode);
-  if (!train_supported(p, dtype)) return MLSTM_ERR_UNSUPPORTED;
+  if (!train_supported(p, dtype) || p.no_norm) return MLSTM_ERR_UNSUPPORTED;
   if (!((C0 && n0 && m0) || (!C0 && !n0 && !m0))) return MLSTM_ERR_INVALID_ARG;
   if (!Q || !K || !V || !i_pre || !f_pre || !H || !saved || !dH || !dQ || !dK || !dV ||
       !di_pre || !df_pre || !workspace)

@@ -30,6 +30,7 @@ struct Problem {
   int NC;                   // number of chunks = ceil(T / L)
   int BH;                   // B * NH
   int gate_sigmoid;         // 0: log i = i_pre; 1: log i = logsigmoid(i_pre)
+  int no_norm;              // sigmoid variant without normaliser: h = e^{m} O (else O / max(|den|, e^{-m}))
   float key_scale;          // 1 / sqrt(DK)
   int signed_den;           // output kernels: n_out = copysign(max(|den|, e^{-m}), den)
   uint32_t* err;            // device error word (see raise_error)

@@ -275,8 +275,9 @@ simt_parallel_kernel(Problem p, const TIn* __restrict__ Q, const TIn* __restrict
     const long t = t0 + r;
     if (t >= T) continue;
     const float mr = bc_s[r] + mu_s[r];
-    const float denom = fmaxf(fabsf(den[i]), expf(-mr));
-    const float inv = 1.f / denom;
+    // the plain sigmoid variant has no normaliser: h = e^{m} O
+    const float denom = p.no_norm ? expf(-mr) : fmaxf(fabsf(den[i]), expf(-mr));
+    const float inv = p.no_norm ? expf(mr) : 1.f / denom;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const int c = dv0 + tx * 4 + j;

@@ -70,6 +70,8 @@ step_state_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __r
                   const float* __restrict__ i_pre, const float* __restrict__ f_pre,
                   float* __restrict__ C, float* __restrict__ n, float* __restrict__ m,
                   T* __restrict__ h, int DK, int DV, int sig, float key_scale, int cluster_nm) {
+  // sig: 0 exponential input gate, 1 sigmoid, 2 the sigmoid variant without
+  // normaliser (same state update as 1)
   constexpr int kCols = 32 * kVec;       // value columns per block
   extern __shared__ float sh[];
   float* sk = sh;                        // s k   [DK]
@@ -157,14 +159,15 @@ step_state_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __r
     kq_all += dots[2 * w + 1];
   }
   const float den = gt.fa * nq_all + gt.ia * kq_all;  // n'.q
-  const float denom = fmaxf(fabsf(den), expf(-gt.m_new));
+  // sig == 2: the plain sigmoid variant, h = e^{m'} C'^T q (no normaliser)
+  const float scale = sig == 2 ? expf(gt.m_new) : 1.f / fmaxf(fabsf(den), expf(-gt.m_new));
   for (int j = threadIdx.x; j < kCols; j += blockDim.x) {
     const int cj = blockIdx.x * kCols + j;
     if (cj >= DV) break;
     float num = 0.f;
 #pragma unroll
     for (int w = 0; w < kStepWarps; ++w) num += red[w * kCols + j];
-    h[(long)bh * DV + cj] = from_float<T>(num / denom);
+    h[(long)bh * DV + cj] = from_float<T>(num * scale);
   }
 }
 
@@ -217,8 +220,8 @@ cudaError_t launch_state(const Problem& p, const void* q, const void* k, const v
   *nm_done = cluster != 0;
   return cudaLaunchKernelEx(&cfg, step_state_kernel<T, kVec>, static_cast<const T*>(q),
                             static_cast<const T*>(k), static_cast<const T*>(v), i_pre, f_pre, C, n,
-                            m, static_cast<T*>(h), p.DK, p.DV, p.gate_sigmoid, p.key_scale,
-                            cluster);
+                            m, static_cast<T*>(h), p.DK, p.DV, p.gate_sigmoid + p.no_norm,
+                            p.key_scale, cluster);
 }
 
 int step_launches(const Problem& p) {

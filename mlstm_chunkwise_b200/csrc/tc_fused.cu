@@ -597,8 +597,9 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       named_bar_sync(1, 256);
       const float2 other = red_s[rt ^ 128];
       const float den = den_part.x + other.x;
-      const float denom = fmaxf(fabsf(den), expf(-(rv.bc + rv.mu)));
-      const float inv = 1.f / denom;
+      // the plain sigmoid variant has no normaliser: h = e^{m_r} O
+      const float mr = rv.bc + rv.mu;
+      const float inv = p.no_norm ? expf(mr) : 1.f / fmaxf(fabsf(den), expf(-mr));
       ok = ok && mbar_wait(bar.o_full(), j & 1, p, 9);  // Q~.C(j) done: Q(j) free
       tc_fence_after();
       uint32_t v0[32], v1[32];

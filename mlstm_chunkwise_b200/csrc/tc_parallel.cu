@@ -531,8 +531,9 @@ tc_parallel_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       ok = ok && mbar_wait(bar.o_full(n % C::kOBufs), (n / C::kOBufs) & 1, p, 12);
       tc_fence_after();
       const float mr = bc + mu;
-      const float denom = fmaxf(fabsf(den), expf(-mr));
-      const float inv = 1.f / denom;
+      // the plain sigmoid variant has no normaliser: h = e^{m_r} O
+      const float denom = p.no_norm ? expf(-mr) : fmaxf(fabsf(den), expf(-mr));
+      const float inv = p.no_norm ? expf(mr) : 1.f / denom;
       if (ok) {
         for (int c = h * kHalfO; c < (h + 1) * kHalfO; c += 64) {
           uint32_t v0[32], v1[32];

@@ -486,8 +486,9 @@ tc_parallel_wide_kernel(const __grid_constant__ CUtensorMap tm_q,
       const __nv_bfloat16* vstar =
           td >= 0 ? Vraw + ((long)x.bh * p.T + td) * p.DV + h * kHalfO : nullptr;
       const float mr = bc + mu;
-      const float denom = fmaxf(fabsf(den), expf(-mr));
-      const float inv = 1.f / denom;
+      // the plain sigmoid variant has no normaliser: h = e^{m_r} O
+      const float denom = p.no_norm ? expf(-mr) : fmaxf(fabsf(den), expf(-mr));
+      const float inv = p.no_norm ? expf(mr) : 1.f / denom;
       if (t < p.T && h == 0) {
         if (n_out) n_out[(long)x.bh * p.T + t] = p.signed_den ? copysignf(denom, den) : denom;
         if (m_out) m_out[(long)x.bh * p.T + t] = mr;

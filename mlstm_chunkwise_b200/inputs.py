@@ -25,7 +25,7 @@ class Workload:
     DK: int
     DV: int
     dtype: str          # "f32" or "bf16": storage/compute type of Q, K, V and H
-    gate_mode: str      # "exp" or "sigmoid"
+    gate_mode: str      # "exp", "sigmoid" or "sigmoid_plain"
     chunk_size: int
     i_mean: float       # i_pre ~ N(i_mean, 1)
     f_low: float = 3.0  # f_pre ~ U(f_low, f_high)
@@ -51,6 +51,10 @@ WORKLOADS = {
     "sigmoid_long": Workload("sigmoid_long", B=2, NH=8, T=32768, DK=256, DV=512, dtype="bf16",
                              gate_mode="sigmoid", chunk_size=512, i_mean=0.0, init_state=True,
                              seed=1003),
+    # the sigmoid-input-gate variant without normaliser, on the same inputs
+    "sigmoid_long_plain": Workload("sigmoid_long_plain", B=2, NH=8, T=32768, DK=256, DV=512,
+                                   dtype="bf16", gate_mode="sigmoid_plain", chunk_size=512,
+                                   i_mean=0.0, init_state=True, seed=1003),
 }
 
 SWEEP_TOKENS = 65536
