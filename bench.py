@@ -147,8 +147,13 @@ MEASURED_TRAFFIC = {
     # 7B shape at batch 2 (16 heads, 514.3 MB per launch), scaled by the heads
     ("tc_parallel", "xlstm7b"): {
         "bytes": 4 * 514.276608e6,
-        "sources": ["tc_parallel_wide.cu", "tc_ptx.cuh", "tc.h", "common.cuh"],
+        "sources": ['tc_parallel_wide.cu', 'tc_ptx.cuh', 'tc.h', 'common.cuh'],
         "sha1": "8fab2e4c5fcf6803c6b38daf41487ce0f2462f76"},
+    # 7B shape at batch 5 (40 heads, unsegmented as at full size, 819.1 MB)
+    ("tc_states", "xlstm7b"): {
+        "bytes": 64 / 40 * 819.10784e6,
+        "sources": ['tc_states.cu', 'tc_ptx.cuh', 'tc.h', 'common.cuh'],
+        "sha1": "77d3a5f55b8bc4bb1373305efae75a31586d2365"},
 }
 
 

@@ -61,6 +61,19 @@ class MlstmError(RuntimeError):
         super().__init__(f"{where}: {status_string(status)} (status {status})")
 
 
+def open_library(path: str):
+    """Load a build of the library at ``path`` (for instance the bounds-checked
+    ``libmlstm_fw_debug.so``) with the signatures of include/mlstm_fw.h."""
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing")
+    h = ctypes.CDLL(path)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(h, name)
+        fn.restype = res
+        fn.argtypes = args
+    return h
+
+
 def lib():
     """The loaded library (loads it on first use; raises if it is missing)."""
     global _lib

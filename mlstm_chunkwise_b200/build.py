@@ -2,6 +2,11 @@
 
     python -m mlstm_chunkwise_b200.build [--force] [--debug-bounds]
 
+``--debug-bounds`` builds ``libmlstm_fw_debug.so`` instead: the same sources
+with ``-DMLSTM_DEBUG_BOUNDS=1``, whose kernels check the offsets of their
+stores and bulk copies against the buffers' extents and report a violation in
+the device error word (MLSTM_ERR_DEVICE, bit 1) instead of making the access.
+
 nvcc cross-compiles for sm_100a without a GPU.  cudart is linked statically and
 the driver API is reached through ``cudaGetDriverEntryPoint``, so the library
 loads on a machine without a CUDA driver (only calls that touch a GPU fail).
@@ -20,6 +25,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libmlstm_fw.so")
+LIB_DEBUG = os.path.join(PKG, "libmlstm_fw_debug.so")
 OBJDIR = os.path.join(ROOT, "_build")
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
@@ -37,21 +43,24 @@ def _deps():
         sorted(glob.glob(os.path.join(CSRC, "*.h"))) + sorted(glob.glob(os.path.join(INCLUDE, "*.h")))
 
 
-def needs_build() -> bool:
-    if not os.path.exists(LIB):
+def needs_build(debug_bounds: bool = False) -> bool:
+    lib = LIB_DEBUG if debug_bounds else LIB
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return any(os.path.getmtime(f) > t for f in _deps())
 
 
 def build(force: bool = False, debug_bounds: bool = False, verbose: bool = False) -> str:
-    if not force and not needs_build():
-        return LIB
-    os.makedirs(OBJDIR, exist_ok=True)
+    lib = LIB_DEBUG if debug_bounds else LIB
+    if not force and not needs_build(debug_bounds):
+        return lib
+    objdir = os.path.join(OBJDIR, "debug") if debug_bounds else OBJDIR
+    os.makedirs(objdir, exist_ok=True)
     extra = ["-DMLSTM_DEBUG_BOUNDS=1"] if debug_bounds else []
 
     def compile_one(src):
-        obj = os.path.join(OBJDIR, os.path.basename(src) + ".o")
+        obj = os.path.join(objdir, os.path.basename(src) + ".o")
         cmd = [NVCC, *ARCH, *FLAGS, *extra, "-c", src, "-o", obj]
         if verbose:
             cmd += ["-Xptxas", "-v"]
@@ -66,13 +75,13 @@ def build(force: bool = False, debug_bounds: bool = False, verbose: bool = False
         for _, err in results:
             sys.stderr.write(err)
     objs = [o for o, _ in results]
-    tmp = LIB + f".tmp{os.getpid()}"
+    tmp = lib + f".tmp{os.getpid()}"
     cmd = [NVCC, *ARCH, "-shared", "-cudart", "static", *objs, "-o", tmp]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"nvcc link failed:\n{r.stderr}")
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":

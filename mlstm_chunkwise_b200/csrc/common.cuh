@@ -22,6 +22,21 @@ __device__ __forceinline__ void raise_error(uint32_t* word, uint32_t bit) {
   if (word) atomicOr(word, bit);
 }
 
+// Debug bounds checks.  In a build with -DMLSTM_DEBUG_BOUNDS=1,
+// MLSTM_IN_BOUNDS(p, cond) sets kErrBounds in the device error word when cond
+// is false and returns cond; the caller then skips a store, or redirects a
+// load to the start of its buffer, so that every barrier still completes and
+// nothing traps.  In a normal build it is `true` and cond is not evaluated.
+__device__ __forceinline__ bool bounds_check(uint32_t* err, bool ok) {
+  if (!ok) raise_error(err, kErrBounds);
+  return ok;
+}
+#ifdef MLSTM_DEBUG_BOUNDS
+#define MLSTM_IN_BOUNDS(p, cond) ::mlstm::bounds_check((p).err, (cond))
+#else
+#define MLSTM_IN_BOUNDS(p, cond) true
+#endif
+
 // ---------------------------------------------------------------------------
 // Problem description passed by value to every kernel.
 // ---------------------------------------------------------------------------

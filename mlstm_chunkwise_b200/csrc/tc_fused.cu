@@ -304,8 +304,9 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         ok = mbar_wait(bar.stg_full(b), (j >> 1) & 1, p, 11);
         if (!ok) break;
         for (int bx = 0; bx < DV / 64; ++bx)
-          tma_store_3d(&tm_h, sbase + F::kOffQ + b * F::kQBytes + bx * 16384, bx * 64, c.k * kL,
-                       c.bh);
+          if (MLSTM_IN_BOUNDS(p, c.k < NC && c.bh < p.BH))
+            tma_store_3d(&tm_h, sbase + F::kOffQ + b * F::kQBytes + bx * 16384, bx * 64,
+                         c.k * kL, c.bh);
         tma_store_commit();
         tma_store_wait_read_all();  // the Q buffer may take chunk j + 2's Q
         mbar_arrive(bar.q_free(b));
@@ -401,7 +402,7 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         uint32_t v[32];
         tmem_ld32(trow + kColC + h * kHalfV + c, v);
         tmem_wait_ld();
-        if (C_T) {
+        if (C_T && MLSTM_IN_BOUNDS(p, bh < p.BH && h * kHalfV + c + 32 <= DV)) {
           float4* dst = reinterpret_cast<float4*>(C_T + ((long)bh * kDK + r) * DV + h * kHalfV + c);
 #pragma unroll
           for (int e = 0; e < 8; ++e)

@@ -236,11 +236,13 @@ tc_parallel_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         load_k(0);
         for (int c = 0; c < C::kSlabsK && ok; ++c) {
           const uint32_t s = next_stage(C::kMNSlabBytes);
-          for (int b = 0; b < DVT / 64; ++b)  // C_k rows [64c, 64c + 64) of block dv0 / 64 + b
-            bulk_load(sbase + C::kOffStage + s * C::kStageBytes + b * 8192,
-                      Cb + cb_block_row((long)x.bh * p.NC + x.k, x.dv0 / 64 + b, c * 64, DK,
-                                        p.DV / 64),
+          for (int b = 0; b < DVT / 64; ++b) {  // C_k rows [64c, 64c + 64) of block dv0 / 64 + b
+            const size_t off =
+                cb_block_row((long)x.bh * p.NC + x.k, x.dv0 / 64 + b, c * 64, DK, p.DV / 64);
+            const bool in = MLSTM_IN_BOUNDS(p, off + 4096 <= (size_t)p.BH * p.NC * DK * p.DV);
+            bulk_load(sbase + C::kOffStage + s * C::kStageBytes + b * 8192, Cb + (in ? off : 0),
                       8192, bar.full(s));
+          }
         }
         for (int i = 1; i < x.n_kv && ok; ++i) {
           load_k(i);
@@ -544,7 +546,7 @@ tc_parallel_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             add_rank1_32(v0, c1, vstar + c);
             if (kHalfO >= 64) add_rank1_32(v1, c1, vstar + c + 32);
           }
-          if (t < p.T) {
+          if (t < p.T && MLSTM_IN_BOUNDS(p, x.dv0 + c + 64 <= p.DV && x.bh < p.BH)) {
             uint32_t pk[16];
 #pragma unroll
             for (int j = 0; j < 32; j += 2)

@@ -239,11 +239,14 @@ tc_parallel_wide_kernel(const __grid_constant__ CUtensorMap tm_q,
           for (int c = 0; c < C::kChunks * C::kSlabsK && ok; ++c) {
             const int kc = x.k + c / C::kSlabsK < p.NC ? x.k + c / C::kSlabsK : p.NC - 1;
             const uint32_t dst = next_stage(C::kMNSlabBytes);
-            for (int b = 0; b < DVT / 64; ++b)
-              bulk_load(dst + b * 8192,
-                        Cb + cb_block_row((long)x.bh * p.NC + kc, dv0 / 64 + b,
-                                          (c % C::kSlabsK) * 64, DK, p.DV / 64),
-                        8192, bar.full((slab - 1) % C::kStages));
+            for (int b = 0; b < DVT / 64; ++b) {
+              const size_t off = cb_block_row((long)x.bh * p.NC + kc, dv0 / 64 + b,
+                                              (c % C::kSlabsK) * 64, DK, p.DV / 64);
+              const bool in = MLSTM_IN_BOUNDS(
+                  p, off + 4096 <= (size_t)p.BH * p.NC * DK * p.DV && kc >= 0);
+              bulk_load(dst + b * 8192, Cb + (in ? off : 0), 8192,
+                        bar.full((slab - 1) % C::kStages));
+            }
           }
         }
       }
@@ -537,7 +540,8 @@ tc_parallel_wide_kernel(const __grid_constant__ CUtensorMap tm_q,
         named_bar_sync(1, 256);
         if (rt == 0 && ok) {
           for (int b = 0; b < DVT / 64; ++b)
-            tma_store_3d(&tm_h, sbase + C::kOffOut + b * 16384, d * DVT + b * 64, x.t0, x.bh);
+            if (MLSTM_IN_BOUNDS(p, d * DVT + b * 64 + 64 <= p.DV && x.t0 < p.T && x.bh < p.BH))
+              tma_store_3d(&tm_h, sbase + C::kOffOut + b * 16384, d * DVT + b * 64, x.t0, x.bh);
           tma_store_commit();
         }
       }

@@ -398,7 +398,9 @@ tc_states_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) {
-        tma_store_3d(map, stg_u + t, x, y, z);
+        if (MLSTM_IN_BOUNDS(p, x >= 0 && x + 16 <= DV && y >= 0 && y + 32 <= DK &&
+                                   z >= 0 && z < p.BH * NC))
+          tma_store_3d(map, stg_u + t, x, y, z);
         tma_store_commit();
       }
       ++n_st;
@@ -426,7 +428,8 @@ tc_states_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
           tdom >= 0 ? Vraw + ((long)bh * p.T + tdom) * DV + dv0 : nullptr;
       float nout = nval;
       if (tdom >= 0 && seg == 0 && n_mine) nout -= dom_residual(g, p, bh, k, tdom, wt, Kraw);
-      if (n_write) n_states[((long)bh * NC + k) * DK + wt] = nout;
+      if (n_write && MLSTM_IN_BOUNDS(p, (long)bh * NC + k < (long)p.BH * NC))
+        n_states[((long)bh * NC + k) * DK + wt] = nout;
       if (n_mine) n_s[wt] = nout;  // read by the boundary pass after the barrier below
       nval *= decay;
 
@@ -468,8 +471,9 @@ tc_states_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
-              bulk_store(Cb + cb_block_row((long)bh * NC + k, (dv0 + col) / 64, dk0, DK, DV / 64),
-                         stg_u, 4096);
+              const size_t off = cb_block_row((long)bh * NC + k, (dv0 + col) / 64, dk0, DK, DV / 64);
+              if (MLSTM_IN_BOUNDS(p, off + 2048 <= (size_t)p.BH * NC * DK * DV))
+                bulk_store(Cb + off, stg_u, 4096);
               tma_store_commit();
             }
           }
@@ -552,8 +556,9 @@ tc_states_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
-              bulk_store(Cb + cb_block_row((long)bh * NC + k, (dv0 + col) / 64, dk0, DK, DV / 64),
-                         stg_u, 4096);
+              const size_t off = cb_block_row((long)bh * NC + k, (dv0 + col) / 64, dk0, DK, DV / 64);
+              if (MLSTM_IN_BOUNDS(p, off + 2048 <= (size_t)p.BH * NC * DK * DV))
+                bulk_store(Cb + off, stg_u, 4096);
               tma_store_commit();
             }
           }
@@ -610,6 +615,7 @@ tc_states_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                        : seg_C + ((((long)bh * gridDim.x + blockIdx.x) * (n_seg - 1) + seg) * DK + dk) *
                                      DVT + col;
           float4* dst = reinterpret_cast<float4*>(row_dst);
+          if (!MLSTM_IN_BOUNDS(p, dv0 + col + 32 <= DV && dk < DK)) continue;
 #pragma unroll
           for (int j = 0; j < 8; ++j)
             dst[j] = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
@@ -736,13 +742,15 @@ tc_states_fixup_kernel(Problem p, Gates g, int DVT, const float* __restrict__ se
 #pragma unroll
         for (int u = 0; u < kB; ++u) {
           if (c0 + u < nb) {
-            ptr[u] = Cb + cb_block_row((long)bh * NC + kb + c0 + u, vb, dk, DK, DV / 64) + jp * 8;
-            v[u] = *reinterpret_cast<const uint4*>(ptr[u]);
+            const size_t off = cb_block_row((long)bh * NC + kb + c0 + u, vb, dk, DK, DV / 64) + jp * 8;
+            // out of bounds (debug builds): neither read nor written back
+            ptr[u] = MLSTM_IN_BOUNDS(p, off + 8 <= (size_t)p.BH * NC * DK * DV) ? Cb + off : nullptr;
+            if (ptr[u]) v[u] = *reinterpret_cast<const uint4*>(ptr[u]);
           }
         }
 #pragma unroll
         for (int u = 0; u < kB; ++u) {
-          if (c0 + u < nb) {
+          if (c0 + u < nb && ptr[u]) {
             __nv_bfloat162* h2 = reinterpret_cast<__nv_bfloat162*>(&v[u]);
             if (any_td && tds[u] >= 0) {
               const int td = tds[u];
