@@ -91,8 +91,13 @@ def test_workload_full_size_sampled_heads(name):
     assert torch.isfinite(H).all()
 
 
-@pytest.mark.parametrize("T,L", [(1024, 256), (65536, 256), (1024, 64), (65536, 64)])
+@pytest.mark.parametrize("T,L", [(1024, 256), (65536, 256), (1024, 64), (65536, 64), (1024, 128),
+                                 (4096, 1024)])
 def test_sweep_full_size_sampled_heads(T, L):
+    """Full-size sweep points in the bench's launch configuration (AUTO): the
+    fused kernel at T = 1024, L = 128 (1024 heads), the wide output kernel with
+    pairs of 64-token chunks, the long-chunk kernel, and the segmented state
+    kernel at 16 heads."""
     w = sweep_workload(T, L)
     x = make_inputs(w)
     H, fin = run(w, x, "auto")
