@@ -37,13 +37,20 @@
 // [64h, 64h + 64) writes 32 packed columns at 32h), once the P.V MMA that read
 // that buffer two tiles earlier has completed.  The P.V MMAs take their A
 // operand from TMEM, so the gating of key tile i + 1 overlaps the P.V MMA of
-// tile i and no MMA waits for another to complete.  Shared
-// memory: the Q tile (DK/64 swizzled slabs), a ring of slabs as deep as the
-// remaining space allows (at DK = 256: 9 stages of 16 KB for value tiles of up
-// to 128 columns, 4 of 32 KB for 256), the per-item column weights and n_k.
-// MMA order per item: S_0, Q.C, { S_i, P_{i-1}.V_{i-1} }, P_last.V_last.  The
-// row threads gate S_0 while Q.C runs, then rescale Q.C to the row frame
-// before releasing P_0, so P_0.V_0 accumulates on the rescaled term.
+// tile i and no MMA waits for another to complete.  With a single O buffer
+// (value tiles of 256 columns) the epilogue stages each row's packed bf16
+// output in the idle P buffers and releases O before its global stores, so the
+// next item's inter-chunk MMAs overlap them.  Shared memory: the Q tile (DK/64
+// swizzled slabs; two Q buffers at DK <= 128, so the next item's Q loads while
+// this one runs), a ring of slabs as deep as the remaining space allows (at
+// DK = 256: 9 stages of 16 KB for value tiles of up to 128 columns, 4 of 32 KB
+// for 256, where two 16 KB K slabs share a stage), the per-item column weights
+// and n_k.
+// MMA order per item: S_0, Q.C, { S_i, P_{i-1}.V_{i-1} }, P_last.V_last.  When
+// the tile works in one frame (see the row threads) P_0 is released as soon as
+// it is written; otherwise the row threads gate S_0 while Q.C runs and rescale
+// Q.C to the row frame before releasing P_0, so P_0.V_0 accumulates on the
+// rescaled term.
 #include <cuda.h>
 
 #include "tc.h"
@@ -71,21 +78,29 @@ struct Cfg {
   static constexpr int kOBufs = DVT <= 128 ? 2 : 1;
   static constexpr int kSlabsK = DK / 64;
   static constexpr uint32_t kQBytes = kQT * DK * 2;
+  // Two Q buffers where they cost at most two ring stages (d_qk <= 128): the
+  // next item's Q and first slabs then load while this item still runs.
+  static constexpr int kQBufs = DK <= 128 ? 2 : 1;
   static constexpr uint32_t kKSlabBytes = kKT * 128;           // 128 rows x 64 bf16
   static constexpr uint32_t kMNSlabBytes = (DVT / 64) * 8192;  // 64 rows x DVT bf16
   static constexpr uint32_t kStageBytes = kKSlabBytes > kMNSlabBytes ? kKSlabBytes : kMNSlabBytes;
+  // K slabs per ring stage (two when a stage is sized for 256-column slabs)
+  static constexpr int kKPer =
+      (int)(kStageBytes / kKSlabBytes) < kSlabsK ? (int)(kStageBytes / kKSlabBytes) : kSlabsK;
+  static_assert(kSlabsK % kKPer == 0, "K slabs fill whole stages");
   static constexpr uint32_t kMiscBytes = 2 * kMaxL * 4 + 2 * DK * 4 + 256 * 8 + 512;
   static constexpr uint32_t kBudget = 227 * 1024 - 1024;  // minus alignment slack
-  static constexpr int kStagesFit = (int)((kBudget - kQBytes - kMiscBytes) / kStageBytes);
+  static constexpr int kStagesFit =
+      (int)((kBudget - kQBufs * kQBytes - kMiscBytes) / kStageBytes);
   static constexpr int kStages = kStagesFit > 12 ? 12 : kStagesFit;
   static_assert(kStages >= 3, "ring too shallow");
   static constexpr uint32_t kOffQ = 0;
-  static constexpr uint32_t kOffStage = kOffQ + kQBytes;
+  static constexpr uint32_t kOffStage = kOffQ + kQBufs * kQBytes;
   static constexpr uint32_t kOffAcol = kOffStage + kStages * kStageBytes;  // float[2][kMaxL]
   static constexpr uint32_t kOffN = kOffAcol + 2 * kMaxL * 4;  // float[2][DK]
   static constexpr uint32_t kOffRed = kOffN + 2 * DK * 4;      // float2[256]
   static constexpr uint32_t kOffBar = kOffRed + 256 * 8;       // barriers
-  static constexpr uint32_t kOffTmemSlot = kOffBar + 368;
+  static constexpr uint32_t kOffTmemSlot = kOffBar + 384;
   static constexpr uint32_t kBytes = kOffTmemSlot + 16;
   static constexpr uint32_t kSmem = kBytes + 1024;  // slack for 1024-byte alignment
   static_assert(kSmem <= 227 * 1024, "shared memory");
@@ -97,8 +112,9 @@ struct Bars {
   uint32_t a;
   __device__ __forceinline__ uint32_t full(int i) const { return a + 8 * i; }
   __device__ __forceinline__ uint32_t empty(int i) const { return a + 128 + 8 * i; }
-  __device__ __forceinline__ uint32_t q_full() const { return a + 256; }
-  __device__ __forceinline__ uint32_t q_empty() const { return a + 264; }
+  // per Q buffer: loaded; read by every MMA and row thread that needs it
+  __device__ __forceinline__ uint32_t q_full(int b) const { return b ? a + 368 : a + 256; }
+  __device__ __forceinline__ uint32_t q_empty(int b) const { return b ? a + 376 : a + 264; }
   // the S tile landed / was read; per P buffer: P written, P.V read it
   __device__ __forceinline__ uint32_t s_full() const { return a + 272; }
   __device__ __forceinline__ uint32_t s_empty() const { return a + 280; }
@@ -169,8 +185,10 @@ tc_parallel_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       mbar_init(bar.full(i), 1);
       mbar_init(bar.empty(i), 1);
     }
-    mbar_init(bar.q_full(), 1);
-    mbar_init(bar.q_empty(), 1 + 256);  // MMA commit + the row threads' reads of Q
+    for (int b = 0; b < C::kQBufs; ++b) {
+      mbar_init(bar.q_full(b), 1);
+      mbar_init(bar.q_empty(b), 1 + 256);  // MMA commit + the row threads' reads of Q
+    }
     mbar_init(bar.s_full(), 1);
     mbar_init(bar.s_empty(), 256);
     for (int i = 0; i < 2; ++i) {
@@ -211,10 +229,11 @@ tc_parallel_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       for (int it = item_at(0); it < n_items && ok; it = item_at(n + 1), ++n) {
         const Item x = decode_item(it, p, n_dv, n_q);
         auto load_k = [&](int i) {
-          for (int c = 0; c < C::kSlabsK && ok; ++c) {
-            const uint32_t s = next_stage(C::kKSlabBytes);
-            tma_load_3d(sbase + C::kOffStage + s * C::kStageBytes, &tm_k, c * 64, x.c0 + i * kKT,
-                        x.bh, bar.full(s));
+          for (int c = 0; c < C::kSlabsK && ok; c += C::kKPer) {
+            const uint32_t s = next_stage(C::kKPer * C::kKSlabBytes);
+            for (int e = 0; e < C::kKPer; ++e)
+              tma_load_3d(sbase + C::kOffStage + s * C::kStageBytes + e * C::kKSlabBytes, &tm_k,
+                          (c + e) * 64, x.c0 + i * kKT, x.bh, bar.full(s));
           }
         };
         auto load_v = [&](int i) {
@@ -228,11 +247,13 @@ tc_parallel_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         // Q before any ring slab of this item: the MMA consumes nothing of the
         // item until Q has landed, so a ring slab issued first could wait for
         // a stage that only frees after Q arrives.
-        if (n > 0) ok = mbar_wait(bar.q_empty(), (n - 1) & 1, p, 2);
+        const int qb = n % C::kQBufs;
+        if (n >= C::kQBufs) ok = mbar_wait(bar.q_empty(qb), ((n / C::kQBufs) - 1) & 1, p, 2);
         if (!ok) break;
-        mbar_expect_tx(bar.q_full(), C::kQBytes);
+        mbar_expect_tx(bar.q_full(qb), C::kQBytes);
         for (int c = 0; c < C::kSlabsK; ++c)
-          tma_load_3d(sbase + C::kOffQ + c * 16384, &tm_q, c * 64, x.t0, x.bh, bar.q_full());
+          tma_load_3d(sbase + C::kOffQ + qb * C::kQBytes + c * 16384, &tm_q, c * 64, x.t0, x.bh,
+                      bar.q_full(qb));
         load_k(0);
         for (int c = 0; c < C::kSlabsK && ok; ++c) {
           const uint32_t s = next_stage(C::kMNSlabBytes);
@@ -253,7 +274,8 @@ tc_parallel_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       // Drain: every issued load must have landed before the CTA may exit.
       for (int q = (slab > C::kStages ? slab - C::kStages : 0); q < slab; ++q)
         mbar_wait(bar.full(q % C::kStages), (q / C::kStages) & 1, p, 13);
-      if (n > 0) mbar_wait(bar.q_full(), (n - 1) & 1, p, 14);
+      for (int m = (n > C::kQBufs ? n - C::kQBufs : 0); m < n; ++m)
+        mbar_wait(bar.q_full(m % C::kQBufs), (m / C::kQBufs) & 1, p, 14);
     }
   } else if (warp == 1) {
     // ---------------------------- MMA issuer ------------------------------
@@ -263,6 +285,7 @@ tc_parallel_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       bool ok = true;
       int slab = 0;   // ring position
       int tile = 0;   // S tiles issued so far (all items)
+      uint32_t qoff = C::kOffQ;  // the current item's Q buffer
       auto take = [&]() -> uint32_t {
         const int s = slab % C::kStages, u = slab / C::kStages;
         ok = ok && mbar_wait(bar.full(s), u & 1, p, 5);
@@ -275,15 +298,17 @@ tc_parallel_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         if (tile >= 1) ok = ok && mbar_wait(bar.s_empty(), (tile - 1) & 1, p, 4);
         tc_fence_after();
         const uint32_t d = tmem + kColS;
-        for (int c = 0; c < C::kSlabsK; ++c) {
+        for (int c = 0; c < C::kSlabsK; c += C::kKPer) {
           const uint32_t s = take();
           if (!ok) return;
-          const uint32_t a0 = sbase + C::kOffQ + c * 16384;
-          const uint32_t b0 = sbase + C::kOffStage + s * C::kStageBytes;
+          for (int e = 0; e < C::kKPer; ++e) {
+            const uint32_t a0 = sbase + qoff + (c + e) * 16384;
+            const uint32_t b0 = sbase + C::kOffStage + s * C::kStageBytes + e * C::kKSlabBytes;
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_bf16_ss(d, sdesc_sw128(a0 + kk * 32, 16, 1024), sdesc_sw128(b0 + kk * 32, 16, 1024),
-                        idS, (c | kk) != 0);
+            for (int kk = 0; kk < 4; ++kk)
+              mma_bf16_ss(d, sdesc_sw128(a0 + kk * 32, 16, 1024),
+                          sdesc_sw128(b0 + kk * 32, 16, 1024), idS, (c | e | kk) != 0);
+          }
           mma_commit(bar.empty(s));
         }
         mma_commit(bar.s_full());
@@ -311,7 +336,9 @@ tc_parallel_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       int n = 0;
       for (int it = item_at(0); it < n_items && ok; it = item_at(n + 1), ++n) {
         const Item x = decode_item(it, p, n_dv, n_q);
-        ok = mbar_wait(bar.q_full(), n & 1, p, 3);
+        const int qb = n % C::kQBufs;
+        qoff = C::kOffQ + qb * C::kQBytes;
+        ok = mbar_wait(bar.q_full(qb), (n / C::kQBufs) & 1, p, 3);
         const int j0 = tile;  // this item's S_0
         if (ok) mma_s();
         // O buffers alternate between items (when there are two): the epilogue
@@ -323,7 +350,7 @@ tc_parallel_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         for (int c = 0; c < C::kSlabsK && ok; ++c) {  // inter-chunk term Q.C_k
           const uint32_t s = take();
           if (!ok) break;
-          const uint32_t a0 = sbase + C::kOffQ + c * 16384;
+          const uint32_t a0 = sbase + qoff + c * 16384;
           const uint32_t b0 = sbase + C::kOffStage + s * C::kStageBytes;
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
@@ -338,7 +365,7 @@ tc_parallel_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
           if (ok) mma_pv(j0 + i - 1);
         }
         if (!ok) break;
-        mma_commit(bar.q_empty());  // every MMA that reads Q has been issued
+        mma_commit(bar.q_empty(qb));  // every MMA that reads Q has been issued
         mma_pv(j0 + x.n_kv - 1);
         if (!ok) break;
         mma_commit(bar.o_full(ob));
@@ -364,15 +391,24 @@ tc_parallel_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     int tile = 0;
     int n = 0;
 
-    // Per-item values, fetched one item ahead.  The exponent of P splits as
-    //   e^{acol_s - mu_r} = e^{acol_s - c} e^{c - mu_r},
-    // c = the largest column weight of the item's keys (amax of its last row,
-    // amax being a running maximum), so the column factor is at most 1.  When
-    // the row factor stays below e^60 for every row of the tile (sep), P costs
-    // two multiplies per element; otherwise the column data holds acol log2(e)
-    // and each element takes its own exponential.
+    // Per-item values, fetched one item ahead.  Every row's terms may be
+    // scaled by a common factor, so when the exponents allow it (sep) the
+    // whole tile works in one frame F instead of each row's mu_r:
+    //   F = m_k, or the largest column weight c (amax of the tile's last row,
+    //   amax being a running maximum) when no state enters the chunk (m_k =
+    //   -inf), and
+    //   P_rs = s (q_r.k_s) e^{acol_s - F},
+    //   O_r  = e^{m_k - F} C_k^T q_r + sum_s P_rs v_s,   e^{m_k - F} = 1 or 0,
+    //   h_r  = O_r / max(|den_r|, e^{-(bcum_r + F)}),
+    // the row frame times e^{mu_r - F}.  Then P takes one column factor per
+    // key (two lanes per packed multiply) and the inter-chunk term needs no
+    // rescaling.  sep requires the column factors within e^60 of 1 (c - F, and
+    // with F = c the first row's amax no lower than c - 60) and the floor's
+    // exponent within +-80 over the tile's rows; otherwise every row keeps its
+    // own frame, each element takes its own exponential (the column data holds
+    // acol log2(e)) and the inter-chunk term is rescaled by e^{m_k - mu_r}.
     struct RowVals {
-      float m_in, amax, bc, c;
+      float m_in, amax, bc, c, F;
       bool sep;
       int td;  // dominant token of the chunk's entering state, or -1
     };
@@ -383,7 +419,13 @@ tc_parallel_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       v.amax = g.amax[base + x.t0 + r];
       v.bc = g.bcum[base + x.t0 + r];
       v.c = g.amax[base + x.t0 + kQT - 1];
-      v.sep = v.c - fmaxf(v.m_in, g.amax[base + x.t0]) <= 60.f;  // uniform over the CTA
+      // uniform over the CTA: the same loads in every thread
+      const bool fresh = v.m_in == -INFINITY;
+      v.F = fresh ? v.c : v.m_in;
+      const float spread = fresh ? v.c - g.amax[base + x.t0] : v.c - v.m_in;
+      const float fl_hi = -g.bcum[base + x.t0 + kQT - 1] - v.F;  // bcum falls along the chunk
+      const float fl_lo = -g.bcum[base + x.t0] - v.F;
+      v.sep = spread <= 60.f && fl_hi <= 80.f && fl_lo >= -80.f;
       v.td = g.dom ? g.dom[(long)x.bh * p.NC + x.k] : -1;
       return v;
     };
@@ -392,11 +434,11 @@ tc_parallel_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       float* nn = n_s + buf * DK;
       for (int j = rt; j < x.n_kv * kKT; j += 256) {
         const float a = g.acol[(long)x.bh * tpad + x.c0 + j];
-        ac[j] = v.sep ? expf(a - v.c) : a * 1.4426950408889634f;  // -inf -> 0 / -inf
+        ac[j] = v.sep ? ks * expf(a - v.F) : a * 1.4426950408889634f;  // -inf -> 0 / -inf
       }
       for (int j = rt; j < DK; j += 256) nn[j] = n_states[((long)x.bh * p.NC + x.k) * DK + j];
     };
-    RowVals nx{0.f, 0.f, 0.f, 0.f, false, -1};
+    RowVals nx{0.f, 0.f, 0.f, 0.f, 0.f, false, -1};
     if (blockIdx.x < n_items) {
       const Item x0 = decode_item(blockIdx.x, p, n_dv, n_q);
       nx = fetch_rows(x0);
@@ -410,17 +452,21 @@ tc_parallel_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       const float* ac = acol_s + (n & 1) * kMaxL;
       const uint32_t colO = (uint32_t)(n % C::kOBufs) * 128u;
       const float* nn = n_s + (n & 1) * DK;
-      const float mu = fmaxf(rv.m_in, rv.amax);
+      const float mu = fmaxf(rv.m_in, rv.amax);  // the row's own frame
+      const float fr = rv.sep ? rv.F : mu;        // the frame this tile works in
       const float mu2 = mu * 1.4426950408889634f;
-      const float f_inter = expf(rv.m_in - mu);
-      const float rowf = rv.sep ? ks * expf(rv.c - mu) : 0.f;
+      const float f_inter = expf(rv.m_in - fr);   // with sep: 1, or 0 with no entering state
+      // The inter-chunk term is rescaled unless its factor is 1 (an m_k of
+      // -inf still multiplies it by 0: a C0 given with m0 = -inf weighs nothing).
+      const bool rescale = !rv.sep || rv.m_in == -INFINITY;
       named_bar_sync(1, 256);  // this item's column data is in shared memory
 
       // Partial den_inter = q_r . n_k over this half's slabs; then release Q.
-      ok = mbar_wait(bar.q_full(), n & 1, p, 8);
+      const int qb = n % C::kQBufs;
+      ok = mbar_wait(bar.q_full(qb), (n / C::kQBufs) & 1, p, 8);
       float dn = 0.f;
       for (int c = h * kSlabsPerHalf; c < C::kSlabsK && c < (h + 1) * kSlabsPerHalf && ok; ++c) {
-        const uint8_t* slab_ptr = smem + C::kOffQ + c * 16384;
+        const uint8_t* slab_ptr = smem + C::kOffQ + qb * C::kQBytes + c * 16384;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           const uint4 v = *reinterpret_cast<const uint4*>(slab_ptr + sw128_offset(r, j));
@@ -433,7 +479,7 @@ tc_parallel_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
           }
         }
       }
-      mbar_arrive(bar.q_empty());
+      mbar_arrive(bar.q_empty(qb));
       float den = f_inter * dn;
 
       // Gated P tiles into the two TMEM P buffers (tile i into buffer i mod
@@ -457,17 +503,34 @@ tc_parallel_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
           mbar_arrive(bar.s_empty());  // S is in registers: the next S may land
           uint32_t pk[32];
           const float* acl = ac + i * kKT + h * 64;
-          if (rv.sep) {
+          if (rv.sep && !diag) {
+            uint64_t rs2 = 0;  // two fp32 partial sums, +0
+#pragma unroll
+            for (int j = 0; j < 64; j += 2) {
+              const float2 cf = *reinterpret_cast<const float2*>(acl + j);
+              const uint64_t pp = mul_f32x2(
+                  f32x2(__uint_as_float(v[j]), __uint_as_float(v[j + 1])), f32x2(cf.x, cf.y));
+              rs2 = add_f32x2(rs2, pp);
+              const float2 pf = f32x2_split(pp);
+              pk[j >> 1] = pack_bf16x2(pf.x, pf.y);
+            }
+            const float2 r2 = f32x2_split(rs2);
+            rs = r2.x + r2.y;
+          } else if (rv.sep) {
+            uint64_t rs2 = 0;
 #pragma unroll
             for (int j = 0; j < 64; j += 2) {
               const int s0 = h * 64 + j;  // key/value index within the tile
-              float pa = __uint_as_float(v[j]) * acl[j] * rowf;
-              float pb = __uint_as_float(v[j + 1]) * acl[j + 1] * rowf;
-              if (diag && s0 > r) pa = 0.f;
-              if (diag && s0 + 1 > r) pb = 0.f;
-              rs += pa + pb;
-              pk[j >> 1] = pack_bf16x2(pa, pb);
+              const float2 cf = *reinterpret_cast<const float2*>(acl + j);
+              float2 pf = f32x2_split(mul_f32x2(
+                  f32x2(__uint_as_float(v[j]), __uint_as_float(v[j + 1])), f32x2(cf.x, cf.y)));
+              if (s0 > r) pf.x = 0.f;
+              if (s0 + 1 > r) pf.y = 0.f;
+              rs2 = add_f32x2(rs2, f32x2(pf.x, pf.y));
+              pk[j >> 1] = pack_bf16x2(pf.x, pf.y);
             }
+            const float2 r2 = f32x2_split(rs2);
+            rs = r2.x + r2.y;
           } else {
 #pragma unroll
             for (int j = 0; j < 64; j += 2) {
@@ -486,7 +549,14 @@ tc_parallel_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
           tmem_st32(trow + pcol, pk);
         }
         den += rs;
-        if (i == 0) {
+        if (!rescale && i == (x.n_kv > 1 ? 1 : 0)) {
+          // Nothing to rescale, but the wait keeps this barrier's phases in
+          // step: before P_1 (or the only P) is released, the MMA issuer
+          // cannot have reached the next item's inter-chunk term.
+          ok = ok && mbar_wait(bar.inter_done(), n & 1, p, 9);
+          tc_fence_after();
+        }
+        if (rescale && i == 0) {
           ok = ok && mbar_wait(bar.inter_done(), n & 1, p, 9);
           tc_fence_after();
           if (ok) {
@@ -532,47 +602,97 @@ tc_parallel_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
           rv.td >= 0 ? Vraw + ((long)x.bh * p.T + rv.td) * p.DV + x.dv0 : nullptr;
       ok = ok && mbar_wait(bar.o_full(n % C::kOBufs), (n / C::kOBufs) & 1, p, 12);
       tc_fence_after();
-      const float mr = bc + mu;
+      const float mr = bc + fr;  // the floor's exponent in the tile's frame
       // the plain sigmoid variant has no normaliser: h = e^{m_r} O
       const float denom = p.no_norm ? expf(-mr) : fmaxf(fabsf(den), expf(-mr));
       const float inv = p.no_norm ? expf(mr) : 1.f / denom;
-      if (ok) {
-        for (int c = h * kHalfO; c < (h + 1) * kHalfO; c += 64) {
-          uint32_t v0[32], v1[32];
-          tmem_ld32(trow + colO + c, v0);
-          if (kHalfO >= 64) tmem_ld32(trow + colO + c + 32, v1);
-          tmem_wait_ld();
-          if (vstar) {
-            add_rank1_32(v0, c1, vstar + c);
-            if (kHalfO >= 64) add_rank1_32(v1, c1, vstar + c + 32);
-          }
-          if (t < p.T && MLSTM_IN_BOUNDS(p, x.dv0 + c + 64 <= p.DV && x.bh < p.BH)) {
-            uint32_t pk[16];
+      if constexpr (C::kOBufs == 1) {
+        // One O buffer: this half's rows go as packed bf16 into its P buffer
+        // (free: every P.V of the item has completed, and the next item's P is
+        // written only after the row threads' barrier at its start), O is
+        // released, and the global stores then read the staged rows, so the
+        // next item's inter-chunk MMAs overlap them.
+        const uint32_t stg = trow + (h ? kColP1 : kColP0);
+        if (ok) {
+#pragma unroll
+          for (int c = 0; c < kHalfO; c += 32) {
+            const int col = h * kHalfO + c;
+            uint32_t v0[32], pk[16];
+            tmem_ld32(trow + colO + col, v0);
+            tmem_wait_ld();
+            if (vstar) add_rank1_32(v0, c1, vstar + col);
 #pragma unroll
             for (int j = 0; j < 32; j += 2)
               pk[j >> 1] =
                   pack_bf16x2(__uint_as_float(v0[j]) * inv, __uint_as_float(v0[j + 1]) * inv);
-            uint4* dst = reinterpret_cast<uint4*>(H + ((long)x.bh * p.T + t) * p.DV + x.dv0 + c);
+            tmem_st16(stg + c / 2, pk);
+          }
+          tmem_wait_st();
+        }
+        tc_fence_before();
+        mbar_arrive(bar.o_empty(0));
+        if (ok) {
+          // every lane reads (tcgen05.ld is warp-wide); rows past T store nothing
+          const bool st = t < p.T &&
+                          MLSTM_IN_BOUNDS(p, x.dv0 + (h + 1) * kHalfO <= p.DV && x.bh < p.BH);
+          uint4* dst =
+              reinterpret_cast<uint4*>(H + ((long)x.bh * p.T + t) * p.DV + x.dv0 + h * kHalfO);
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-              dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
-            if (kHalfO >= 64) {
+          for (int c = 0; c < kHalfO / 2; c += 32) {
+            uint32_t pk[32];
+            tmem_ld32(stg + c, pk);
+            tmem_wait_ld();
+            if (st) {
 #pragma unroll
-              for (int j = 0; j < 32; j += 2)
-                pk[j >> 1] =
-                    pack_bf16x2(__uint_as_float(v1[j]) * inv, __uint_as_float(v1[j + 1]) * inv);
-#pragma unroll
-              for (int j = 0; j < 4; ++j)
-                dst[4 + j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+              for (int j = 0; j < 8; ++j)
+                dst[c / 4 + j] =
+                    make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
             }
           }
         }
+      } else {
+        if (ok) {
+          for (int c = h * kHalfO; c < (h + 1) * kHalfO; c += 64) {
+            uint32_t v0[32], v1[32];
+            tmem_ld32(trow + colO + c, v0);
+            if (kHalfO >= 64) tmem_ld32(trow + colO + c + 32, v1);
+            tmem_wait_ld();
+            if (vstar) {
+              add_rank1_32(v0, c1, vstar + c);
+              if (kHalfO >= 64) add_rank1_32(v1, c1, vstar + c + 32);
+            }
+            if (t < p.T && MLSTM_IN_BOUNDS(p, x.dv0 + c + (kHalfO >= 64 ? 64 : 32) <= p.DV &&
+                                                  x.bh < p.BH)) {
+              uint32_t pk[16];
+#pragma unroll
+              for (int j = 0; j < 32; j += 2)
+                pk[j >> 1] =
+                    pack_bf16x2(__uint_as_float(v0[j]) * inv, __uint_as_float(v0[j + 1]) * inv);
+              uint4* dst =
+                  reinterpret_cast<uint4*>(H + ((long)x.bh * p.T + t) * p.DV + x.dv0 + c);
+#pragma unroll
+              for (int j = 0; j < 4; ++j)
+                dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+              if (kHalfO >= 64) {
+#pragma unroll
+                for (int j = 0; j < 32; j += 2)
+                  pk[j >> 1] = pack_bf16x2(__uint_as_float(v1[j]) * inv,
+                                           __uint_as_float(v1[j + 1]) * inv);
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                  dst[4 + j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+              }
+            }
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(bar.o_empty(n % C::kOBufs));
       }
-      tc_fence_before();
-      mbar_arrive(bar.o_empty(n % C::kOBufs));
       if (t < p.T && x.dv0 == 0 && h == 0) {
-        if (n_out) n_out[(long)x.bh * p.T + t] = p.signed_den ? copysignf(denom, den) : denom;
-        if (m_out) m_out[(long)x.bh * p.T + t] = mr;
+        // per-token outputs in the row frame mu_r
+        const float dr = rv.sep ? denom * expf(fr - mu) : denom;
+        if (n_out) n_out[(long)x.bh * p.T + t] = p.signed_den ? copysignf(dr, den) : dr;
+        if (m_out) m_out[(long)x.bh * p.T + t] = bc + mu;
       }
     }
   }

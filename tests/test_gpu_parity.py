@@ -196,17 +196,33 @@ def test_chunk_states_against_oracle_snapshots(algo):
                    tol, label="chunk states final")
 
 
+PER_TOKEN_SHAPES = {
+    "mid_L128": dict(base="mid", T=768),
+    # the long-chunk kernel: chunk 0 without an entering state, then m_k frames
+    "d128_L512": dict(base="mid", T=1536, chunk_size=512),
+    # one O buffer per item (value tiles of 256 columns), sigmoid gate, C0 given
+    "d256x512_L512": dict(base="sigmoid_long", T=1536),
+}
+
+
+@pytest.mark.parametrize("shape", list(PER_TOKEN_SHAPES))
 @pytest.mark.parametrize("algo", ["simt", "tc"])
-def test_parallel_per_token_outputs(algo):
-    w = scaled(WORKLOADS["mid"], B=1, NH=2, T=768)
+def test_parallel_per_token_outputs(algo, shape):
+    """mlstm_fw_parallel's per-token normaliser and stabiliser (the row frame
+    of the chunkwise form) against the oracle's."""
+    kw = dict(PER_TOKEN_SHAPES[shape])
+    w = scaled(WORKLOADS[kw.pop("base")], B=1, NH=2, **kw)
     if not supported(w, algo):
         pytest.skip(f"{algo} unsupported")
     x = make_inputs(w)
     d = parity.to_dev(x)
     C_s, n_s, m_s, _ = api.mlstm_fw_chunk_states(d["K"], d["V"], d["i_pre"], d["f_pre"],
-                                                 chunk_size=w.chunk_size, algo=algo)
+                                                 d["C0"], d["n0"], d["m0"],
+                                                 chunk_size=w.chunk_size, gate_mode=w.gate_mode,
+                                                 algo=algo)
     H, n_out, m_out = api.mlstm_fw_parallel(d["Q"], d["K"], d["V"], d["i_pre"], d["f_pre"], C_s,
-                                            n_s, chunk_size=w.chunk_size, algo=algo)
+                                            n_s, d["m0"], chunk_size=w.chunk_size,
+                                            gate_mode=w.gate_mode, algo=algo)
     ref = parity.oracle_run(x, w.gate_mode)
     tol = parity.TOL[w.dtype]
     assert parity.worst_rel(H.double().cpu().numpy(), ref["H"]) < tol
