@@ -604,7 +604,8 @@ tc_parallel_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       tc_fence_after();
       const float mr = bc + fr;  // the floor's exponent in the tile's frame
       // the plain sigmoid variant has no normaliser: h = e^{m_r} O
-      const float denom = p.no_norm ? expf(-mr) : fmaxf(fabsf(den), expf(-mr));
+      const float floor_f = expf(-mr);
+      const float denom = p.no_norm ? floor_f : fmaxf(fabsf(den), floor_f);
       const float inv = p.no_norm ? expf(mr) : 1.f / denom;
       if constexpr (C::kOBufs == 1) {
         // One O buffer: this half's rows go as packed bf16 into its P buffer
@@ -690,7 +691,11 @@ tc_parallel_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       }
       if (t < p.T && x.dv0 == 0 && h == 0) {
         // per-token outputs in the row frame mu_r
-        const float dr = rv.sep ? denom * expf(fr - mu) : denom;
+        // (where the floor is picked, the row frame's floor itself, so that
+        // a comparison with e^{-m_r} tells the two cases apart exactly)
+        const float dr = !rv.sep ? denom
+                         : (p.no_norm || !(fabsf(den) > floor_f)) ? expf(-(bc + mu))
+                                                                  : fabsf(den) * expf(fr - mu);
         if (n_out) n_out[(long)x.bh * p.T + t] = p.signed_den ? copysignf(dr, den) : dr;
         if (m_out) m_out[(long)x.bh * p.T + t] = bc + mu;
       }

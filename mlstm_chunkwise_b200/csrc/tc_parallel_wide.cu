@@ -47,6 +47,10 @@
 // P_0.V_0[:, d] [, P_1.V_1[:, d]], (first tile: wait for the scaled Q),
 // Q~.C_k[:, d].  S_i of the next item waits until the last P_i.V_i MMA of
 // this one has completed; the Q~.C_k MMAs issued after it hide that wait.
+// When the exponents of a tile allow one frame for all its rows (tile_frame:
+// the entering state's m_k, as in the long-chunk kernel) Q needs no scaling,
+// and each value tile issues Q.C_k[:, d] first: the inter-chunk MMAs of the
+// first value tile run while the row threads still gate S.
 #include <cuda.h>
 
 #include "tc.h"
@@ -128,6 +132,21 @@ __device__ __forceinline__ WItem decode_witem(int it, const Problem& p, int n_q)
   x.c0 = x.k * p.L;
   x.n_kv = (x.t0 - x.c0) / kKT + 1;
   return x;
+}
+
+// Whether the item's tile works in the frame F = m_k (see the row threads),
+// from the same loads and arithmetic in the MMA issuer and the row threads.
+// Never with two chunks per tile (kPair) or without an entering state.
+template <bool kPair>
+__device__ __forceinline__ bool tile_frame(const Gates& g, const Problem& p, const WItem& x,
+                                           long tpad) {
+  if (kPair) return false;
+  const long base = (long)x.bh * tpad;
+  const float m_in = g.mchk[(long)x.bh * (p.NC + 1) + x.k];
+  const float c = g.amax[base + x.t0 + kQT - 1];  // amax is a running maximum
+  const float hi = -g.bcum[base + x.t0 + kQT - 1] - m_in;  // bcum falls along the chunk
+  const float lo = -g.bcum[base + x.t0] - m_in;
+  return m_in != -INFINITY && c - m_in <= 60.f && hi <= 80.f && lo >= -80.f;
 }
 
 // The k-th item of this CTA.  Items alternate between the first and the
@@ -224,8 +243,10 @@ tc_parallel_wide_kernel(const __grid_constant__ CUtensorMap tm_q,
             tma_load_3d(dst, &tm_k, c * 64, x.c0 + i * kKT, x.bh,
                         bar.full((slab - 1) % C::kStages));
           }
-        for (int d = 0; d < n_dv && ok; ++d) {
-          const int dv0 = d * DVT;
+        // per value tile: the V slabs of the P.V terms and the C_k slabs of the
+        // inter-chunk term, in the order the MMA issuer takes them
+        const bool frame = tile_frame<kPair>(g, p, x, tpad);
+        auto load_v = [&](int dv0) {
           for (int i = 0; i < x.n_kv && ok; ++i)
             for (int v = 0; v < 2 && ok; ++v) {
               const uint32_t dst = next_stage(C::kMNSlabBytes);
@@ -233,9 +254,11 @@ tc_parallel_wide_kernel(const __grid_constant__ CUtensorMap tm_q,
                 tma_load_3d(dst + b * 8192, &tm_v, dv0 + b * 64, x.c0 + i * kKT + v * 64, x.bh,
                             bar.full((slab - 1) % C::kStages));
             }
-          // C_k rows [64c, 64c + 64) (kPair: then those of chunk k + 1, or of
-          // chunk k again past the last chunk, where the zero half of the
-          // stacked Q~ operand meets them)
+        };
+        // C_k rows [64c, 64c + 64) (kPair: then those of chunk k + 1, or of
+        // chunk k again past the last chunk, where the zero half of the
+        // stacked Q~ operand meets them)
+        auto load_c = [&](int dv0) {
           for (int c = 0; c < C::kChunks * C::kSlabsK && ok; ++c) {
             const int kc = x.k + c / C::kSlabsK < p.NC ? x.k + c / C::kSlabsK : p.NC - 1;
             const uint32_t dst = next_stage(C::kMNSlabBytes);
@@ -247,6 +270,15 @@ tc_parallel_wide_kernel(const __grid_constant__ CUtensorMap tm_q,
               bulk_load(dst + b * 8192, Cb + (in ? off : 0), 8192,
                         bar.full((slab - 1) % C::kStages));
             }
+          }
+        };
+        for (int d = 0; d < n_dv && ok; ++d) {
+          if (frame) {
+            load_c(d * DVT);
+            load_v(d * DVT);
+          } else {
+            load_v(d * DVT);
+            load_c(d * DVT);
           }
         }
       }
@@ -272,6 +304,7 @@ tc_parallel_wide_kernel(const __grid_constant__ CUtensorMap tm_q,
       int n = 0;
       for (int it = item_at(0); it < n_items && ok; it = item_at(n + 1), ++n) {
         const WItem x = decode_witem(it, p, n_q);
+        const bool frame = tile_frame<kPair>(g, p, x, tpad);  // used after the S MMAs
         ok = mbar_wait(bar.q_full(), n & 1, p, 3);
         for (int i = 0; i < x.n_kv && ok; ++i) {  // S_i
           const int fills = i ? sc1 : sc0;
@@ -297,37 +330,54 @@ tc_parallel_wide_kernel(const __grid_constant__ CUtensorMap tm_q,
           const uint32_t dO = tmem + (uint32_t)ob * 128u;
           if (dcount >= 2) ok = ok && mbar_wait(bar.o_empty(ob), ((dcount >> 1) - 1) & 1, p, 6);
           tc_fence_after();
-          for (int i = 0; i < x.n_kv && ok; ++i) {  // P_i . V_i[:, d], A from TMEM
-            if (d == 0) ok = mbar_wait(bar.p_full(i), ((i ? sc1 : sc0) - 1) & 1, p, 8);
-            tc_fence_after();
-            const uint32_t aP = tmem + (i ? kColS1 : kColS0);
-            for (int v = 0; v < 2 && ok; ++v) {
+          // P_i . V_i[:, d] (A from TMEM); the first MMA into O initialises it
+          auto mma_pv = [&](bool init) {
+            for (int i = 0; i < x.n_kv && ok; ++i) {
+              if (d == 0) ok = mbar_wait(bar.p_full(i), ((i ? sc1 : sc0) - 1) & 1, p, 8);
+              tc_fence_after();
+              const uint32_t aP = tmem + (i ? kColS1 : kColS0);
+              for (int v = 0; v < 2 && ok; ++v) {
+                const uint32_t s = take();
+                if (!ok) break;
+                const uint32_t b0 = sbase + C::kOffStage + s * C::kStageBytes;
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                  mma_bf16_ts(dO, aP + (uint32_t)v * kColPHalf + (uint32_t)kk * 8u,
+                              sdesc_sw128(b0 + kk * 2048, 8192, 1024), idO,
+                              !init || (i | v | kk) != 0);
+                mma_commit(bar.empty(s));
+              }
+              if (d == n_dv - 1) mma_commit(bar.pv_done(i));
+            }
+          };
+          // Q~ . C_k[:, d]
+          auto mma_qc = [&](bool init) {
+            for (int c = 0; c < C::kChunks * C::kSlabsK && ok; ++c) {
               const uint32_t s = take();
               if (!ok) break;
+              const uint32_t a0 = sbase + C::kOffQ + c * 16384;
               const uint32_t b0 = sbase + C::kOffStage + s * C::kStageBytes;
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk)
-                mma_bf16_ts(dO, aP + (uint32_t)v * kColPHalf + (uint32_t)kk * 8u,
-                            sdesc_sw128(b0 + kk * 2048, 8192, 1024), idO, (i | v | kk) != 0);
+                mma_bf16_ss(dO, sdesc_sw128(a0 + kk * 32, 16, 1024),
+                            sdesc_sw128(b0 + kk * 2048, 8192, 1024), idO,
+                            !init || (c | kk) != 0);
               mma_commit(bar.empty(s));
             }
-            if (d == n_dv - 1) mma_commit(bar.pv_done(i));
-          }
-          if (!ok) break;
-          if (d == 0) {
-            ok = mbar_wait(bar.q_scaled(), n & 1, p, 7);  // Q rows scaled in place
-            tc_fence_after();
-          }
-          for (int c = 0; c < C::kChunks * C::kSlabsK && ok; ++c) {  // Q~ . C_k[:, d]
-            const uint32_t s = take();
+          };
+          if (frame) {
+            // one frame for the tile: Q is used as loaded, so the inter-chunk
+            // term goes first and waits for no row thread
+            mma_qc(true);
+            mma_pv(false);
+          } else {
+            mma_pv(true);
             if (!ok) break;
-            const uint32_t a0 = sbase + C::kOffQ + c * 16384;
-            const uint32_t b0 = sbase + C::kOffStage + s * C::kStageBytes;
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              mma_bf16_ss(dO, sdesc_sw128(a0 + kk * 32, 16, 1024),
-                          sdesc_sw128(b0 + kk * 2048, 8192, 1024), idO, 1);
-            mma_commit(bar.empty(s));
+            if (d == 0) {
+              ok = mbar_wait(bar.q_scaled(), n & 1, p, 7);  // Q rows scaled in place
+              tc_fence_after();
+            }
+            mma_qc(false);
           }
           if (!ok) break;
           if (d == n_dv - 1) mma_commit(bar.q_empty());  // last reader of Q issued
@@ -363,20 +413,30 @@ tc_parallel_wide_kernel(const __grid_constant__ CUtensorMap tm_q,
       bc = g.bcum[(long)x.bh * tpad + t];
       td = g.dom ? g.dom[(long)x.bh * p.NC + chunk_of(x, rchunk)] : -1;
     };
-    auto fetch_cols = [&](const WItem& x, int buf) {
+    // One frame for the tile (tile_frame): every row's terms scaled by
+    // e^{mu_r - m_k}, so P_rs = s (q_r.k_s) e^{acol_s - m_k} takes one column
+    // factor per key, the inter-chunk term needs no scaling of Q (factor 1)
+    // and h_r = O_r / max(|den_r|, e^{-(bcum_r + m_k)}).  Otherwise each row
+    // works in its own frame mu_r = max(m_k, amax_r): the column data holds
+    // acol log2(e), each element takes its own exponential and Q is scaled.
+    auto fetch_cols = [&](const WItem& x, int buf, bool frame, float F) {
       float* ac = acol_s + buf * kPSlots * kKT;
       float* nn = n_s + buf * C::kChunks * DK;
-      for (int j = rt; j < x.n_kv * kKT; j += 256)
-        ac[j] = g.acol[(long)x.bh * tpad + x.c0 + j] * 1.4426950408889634f;
+      for (int j = rt; j < x.n_kv * kKT; j += 256) {
+        const float a = g.acol[(long)x.bh * tpad + x.c0 + j];
+        ac[j] = frame ? ks * expf(a - F) : a * 1.4426950408889634f;  // -inf -> 0 / -inf
+      }
       for (int j = rt; j < C::kChunks * DK; j += 256)
         nn[j] = n_states[((long)x.bh * p.NC + chunk_of(x, j / DK)) * DK + j % DK];
     };
     float nx_m_in = 0.f, nx_amax = 0.f, nx_bc = 0.f;
     int nx_td = -1;
+    bool nx_frame = false;
     if (blockIdx.x < n_items) {
       const WItem x0 = decode_witem(blockIdx.x, p, n_q);
       fetch_rows(x0, nx_m_in, nx_amax, nx_bc, nx_td);
-      fetch_cols(x0, 0);
+      nx_frame = tile_frame<kPair>(g, p, x0, tpad);
+      fetch_cols(x0, 0, nx_frame, nx_m_in);
     }
     int n = 0;
     for (int it = item_at(0); it < n_items && ok; it = item_at(n + 1), ++n) {
@@ -384,11 +444,13 @@ tc_parallel_wide_kernel(const __grid_constant__ CUtensorMap tm_q,
       const int t = x.t0 + r;
       const float m_in = nx_m_in, amax = nx_amax, bc = nx_bc;
       const int td = nx_td;  // warp-uniform (kPair: rows of one chunk per warp)
+      const bool frame = nx_frame;  // uniform over the CTA
       const float* ac = acol_s + (n & 1) * kPSlots * kKT;
       const float* nn = n_s + ((n & 1) * C::kChunks + rchunk) * DK;
-      const float mu = fmaxf(m_in, amax);
+      const float mu = fmaxf(m_in, amax);  // the row's own frame
+      const float fr = frame ? m_in : mu;  // the frame this tile works in
       const float mu2 = mu * 1.4426950408889634f;
-      const float f_inter = expf(m_in - mu);
+      const float f_inter = expf(m_in - fr);  // 1 with one frame
       named_bar_sync(1, 256);
 
       // Partial den_inter = q_r . n_k over this half's slabs; then release Q.
@@ -425,16 +487,33 @@ tc_parallel_wide_kernel(const __grid_constant__ CUtensorMap tm_q,
           tmem_wait_ld();
           uint32_t pk[32];
           const float* acl = ac + i * kKT + h * 64;
+          if (frame) {
+            uint64_t rs2 = 0;  // two fp32 partial sums, +0
 #pragma unroll
-          for (int j = 0; j < 64; j += 2) {
-            const int s0 = h * 64 + j;
-            float pa = __uint_as_float(v[j]) * ks * ex2_approx(acl[j] - mu2);
-            float pb = __uint_as_float(v[j + 1]) * ks * ex2_approx(acl[j + 1] - mu2);
-            if (diag && s0 > r) pa = 0.f;
-            if (diag && s0 + 1 > r) pb = 0.f;
-            if (kPair && ((s0 ^ r) & 64)) pa = pb = 0.f;  // key and query in different chunks
-            rs += pa + pb;
-            pk[j >> 1] = pack_bf16x2(pa, pb);
+            for (int j = 0; j < 64; j += 2) {
+              const int s0 = h * 64 + j;
+              const float2 cf = *reinterpret_cast<const float2*>(acl + j);
+              float2 pf = f32x2_split(mul_f32x2(
+                  f32x2(__uint_as_float(v[j]), __uint_as_float(v[j + 1])), f32x2(cf.x, cf.y)));
+              if (diag && s0 > r) pf.x = 0.f;
+              if (diag && s0 + 1 > r) pf.y = 0.f;
+              rs2 = add_f32x2(rs2, f32x2(pf.x, pf.y));
+              pk[j >> 1] = pack_bf16x2(pf.x, pf.y);
+            }
+            const float2 r2 = f32x2_split(rs2);
+            rs = r2.x + r2.y;
+          } else {
+#pragma unroll
+            for (int j = 0; j < 64; j += 2) {
+              const int s0 = h * 64 + j;
+              float pa = __uint_as_float(v[j]) * ks * ex2_approx(acl[j] - mu2);
+              float pb = __uint_as_float(v[j + 1]) * ks * ex2_approx(acl[j + 1] - mu2);
+              if (diag && s0 > r) pa = 0.f;
+              if (diag && s0 + 1 > r) pb = 0.f;
+              if (kPair && ((s0 ^ r) & 64)) pa = pb = 0.f;  // key and query in different chunks
+              rs += pa + pb;
+              pk[j >> 1] = pack_bf16x2(pa, pb);
+            }
           }
           tmem_st32(trow + scol, pk);
           tmem_wait_st();
@@ -448,8 +527,9 @@ tc_parallel_wide_kernel(const __grid_constant__ CUtensorMap tm_q,
       // Every S MMA of this item has completed (the waits above): scale this
       // half of the Q row by e^{m_k - mu_r} in place for the inter-chunk MMAs
       // (kPair: into the row's chunk half of the stacked operand, zeros into
-      // the other half).
-      if (ok) {
+      // the other half).  With one frame Q stays as loaded (its inter-chunk
+      // MMAs may already be running); the arrival below still marks the item.
+      if (ok && !frame) {
         for (int c = h * kSlabsPerHalf; c < C::kSlabsK && c < (h + 1) * kSlabsPerHalf; ++c) {
           uint8_t* slab_ptr = smem + C::kOffQ + c * 16384;
           uint8_t* dst_ptr = slab_ptr + rchunk * C::kSlabsK * 16384;
@@ -476,7 +556,8 @@ tc_parallel_wide_kernel(const __grid_constant__ CUtensorMap tm_q,
       if (it_next < n_items) {
         const WItem xn = decode_witem(it_next, p, n_q);
         fetch_rows(xn, nx_m_in, nx_amax, nx_bc, nx_td);
-        fetch_cols(xn, (n + 1) & 1);
+        nx_frame = tile_frame<kPair>(g, p, xn, tpad);
+        fetch_cols(xn, (n + 1) & 1, nx_frame, nx_m_in);
       }
 
       // Both halves' partial denominators (and inter-chunk parts) -> the row's.
@@ -488,13 +569,19 @@ tc_parallel_wide_kernel(const __grid_constant__ CUtensorMap tm_q,
       const float c1 = f_inter * (dn + other.y);
       const __nv_bfloat16* vstar =
           td >= 0 ? Vraw + ((long)x.bh * p.T + td) * p.DV + h * kHalfO : nullptr;
-      const float mr = bc + mu;
+      const float mr = bc + fr;  // the floor's exponent in the tile's frame
       // the plain sigmoid variant has no normaliser: h = e^{m_r} O
-      const float denom = p.no_norm ? expf(-mr) : fmaxf(fabsf(den), expf(-mr));
+      const float floor_f = expf(-mr);
+      const float denom = p.no_norm ? floor_f : fmaxf(fabsf(den), floor_f);
       const float inv = p.no_norm ? expf(mr) : 1.f / denom;
-      if (t < p.T && h == 0) {
-        if (n_out) n_out[(long)x.bh * p.T + t] = p.signed_den ? copysignf(denom, den) : denom;
-        if (m_out) m_out[(long)x.bh * p.T + t] = mr;
+      if (t < p.T && h == 0) {  // per-token outputs in the row frame mu_r
+        // (where the floor is picked, the row frame's floor itself, so that
+        // a comparison with e^{-m_r} tells the two cases apart exactly)
+        const float dr = !frame ? denom
+                         : (p.no_norm || !(fabsf(den) > floor_f)) ? expf(-(bc + mu))
+                                                                  : fabsf(den) * expf(fr - mu);
+        if (n_out) n_out[(long)x.bh * p.T + t] = p.signed_den ? copysignf(dr, den) : dr;
+        if (m_out) m_out[(long)x.bh * p.T + t] = bc + mu;
       }
 
       for (int d = 0; d < n_dv; ++d, ++dcount) {
