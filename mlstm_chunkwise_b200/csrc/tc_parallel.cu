@@ -385,6 +385,10 @@ tc_parallel_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     const int h = rt >> 7;               // column half
     const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16);
     const float ks = p.key_scale;
+    // H rows go out in 32-byte stores where H allows it (row and tile starts
+    // are then 32-byte aligned too: DV and every column offset are multiples
+    // of 32 elements)
+    const bool v8 = (reinterpret_cast<uintptr_t>(H) & 31) == 0;
     constexpr int kHalfO = DVT / 2;
     constexpr int kSlabsPerHalf = (C::kSlabsK + 1) / 2;
     bool ok = true;
@@ -636,17 +640,20 @@ tc_parallel_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
           // every lane reads (tcgen05.ld is warp-wide); rows past T store nothing
           const bool st = t < p.T &&
                           MLSTM_IN_BOUNDS(p, x.dv0 + (h + 1) * kHalfO <= p.DV && x.bh < p.BH);
-          uint4* dst =
-              reinterpret_cast<uint4*>(H + ((long)x.bh * p.T + t) * p.DV + x.dv0 + h * kHalfO);
+          uint32_t* dst =
+              reinterpret_cast<uint32_t*>(H + ((long)x.bh * p.T + t) * p.DV + x.dv0 + h * kHalfO);
 #pragma unroll
           for (int c = 0; c < kHalfO / 2; c += 32) {
             uint32_t pk[32];
             tmem_ld32(stg + c, pk);
             tmem_wait_ld();
-            if (st) {
+            if (st && v8) {  // whole 32-byte sectors
+#pragma unroll
+              for (int j = 0; j < 4; ++j) st_global_v8(dst + c + 8 * j, pk + 8 * j);
+            } else if (st) {
 #pragma unroll
               for (int j = 0; j < 8; ++j)
-                dst[c / 4 + j] =
+                reinterpret_cast<uint4*>(dst + c)[j] =
                     make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
             }
           }
@@ -671,17 +678,28 @@ tc_parallel_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     pack_bf16x2(__uint_as_float(v0[j]) * inv, __uint_as_float(v0[j + 1]) * inv);
               uint4* dst =
                   reinterpret_cast<uint4*>(H + ((long)x.bh * p.T + t) * p.DV + x.dv0 + c);
+              if (v8) {
+                st_global_v8(dst, pk);
+                st_global_v8(dst + 2, pk + 8);
+              } else {
 #pragma unroll
-              for (int j = 0; j < 4; ++j)
-                dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+                for (int j = 0; j < 4; ++j)
+                  dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+              }
               if (kHalfO >= 64) {
 #pragma unroll
                 for (int j = 0; j < 32; j += 2)
                   pk[j >> 1] = pack_bf16x2(__uint_as_float(v1[j]) * inv,
                                            __uint_as_float(v1[j + 1]) * inv);
+                if (v8) {
+                  st_global_v8(dst + 4, pk);
+                  st_global_v8(dst + 6, pk + 8);
+                } else {
 #pragma unroll
-                for (int j = 0; j < 4; ++j)
-                  dst[4 + j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+                  for (int j = 0; j < 4; ++j)
+                    dst[4 + j] =
+                        make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+                }
               }
             }
           }
