@@ -144,16 +144,21 @@ def method_bytes(fam, B, NH, T, DK, DV, elem, init_state):
 # dram__bytes_write.sum), valid only while the kernel's sources are unchanged:
 # the entry records a SHA-1 over those files and is ignored when it differs.
 MEASURED_TRAFFIC = {
-    # 7B shape at batch 2 (16 heads, 514.3 MB per launch), scaled by the heads
+    # 7B shape at batch 2 (16 heads, 514.1 MB per launch), scaled by the heads
     ("tc_parallel", "xlstm7b"): {
-        "bytes": 4 * 514.276608e6,
+        "bytes": 4 * 514.113024e6,
         "sources": ['tc_parallel_wide.cu', 'tc_ptx.cuh', 'tc.h', 'common.cuh'],
-        "sha1": "8fab2e4c5fcf6803c6b38daf41487ce0f2462f76"},
-    # 7B shape at batch 5 (40 heads, unsegmented as at full size, 819.1 MB)
+        "sha1": "d77ddeaa1058f329306d4f3a8ee9e25d506f9280"},
+    # 7B shape at batch 5 (40 heads, unsegmented as at full size, 819.9 MB)
     ("tc_states", "xlstm7b"): {
-        "bytes": 64 / 40 * 819.10784e6,
+        "bytes": 64 / 40 * 819.934208e6,
         "sources": ['tc_states.cu', 'tc_ptx.cuh', 'tc.h', 'common.cuh'],
-        "sha1": "77d3a5f55b8bc4bb1373305efae75a31586d2365"},
+        "sha1": "2c1f6db9734982d4cf1ed79d073bf79bb235b0a6"},
+    # sigmoid_long at batch 1 (8 heads, the long-chunk kernel, 916.6 MB)
+    ("tc_parallel", "sigmoid_long"): {
+        "bytes": 2 * 916.586496e6,
+        "sources": ['tc_parallel.cu', 'tc_ptx.cuh', 'tc.h', 'common.cuh'],
+        "sha1": "71537485f494a037f68ab3f7aa374448d029ac74"},
 }
 
 
