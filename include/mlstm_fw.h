@@ -95,8 +95,8 @@ typedef enum {
 } mlstm_gate_mode;
 
 /* Which kernels compute the path.
- *   AUTO      TC_FUSED where it is supported and there are at least 592
- *             (b, h) pairs (4 per SM of a 148-SM B200), else TC where it is
+ *   AUTO      TC_FUSED where it is supported and there are at least 74
+ *             (b, h) pairs (half the SMs of a 148-SM B200), else TC where it is
  *             supported, else SIMT.  A fixed rule, so workspace sizes computed
  *             for AUTO always match the algorithm the call picks.
  *   SIMT      fp32 CUDA-core kernels (the only choice for fp32 inputs).

@@ -143,12 +143,16 @@ bool valid_enums(mlstm_dtype dt, mlstm_gate_mode gm, mlstm_algo algo) {
 mlstm_status resolve_algo(const Problem& p, mlstm_dtype dt, mlstm_algo req, bool allow_fused,
                           mlstm_algo* out) {
   if (req == MLSTM_ALGO_AUTO) {
-    // The fused kernel walks each head's chunks in order on one SM, so it
-    // wins only with several heads per SM (measured: 1024 heads of 8 chunks
-    // faster than the unfused path, 256 heads slower).  The threshold is a
-    // constant (4 heads per SM of a 148-SM B200) so that the workspace size
-    // computed on the host always matches the algorithm a call picks.
-    constexpr int kFusedMinHeads = 4 * 148;
+    // The fused kernel walks each head's chunks in order on one SM: a chunk
+    // there costs about 5 us of one SM against about 9-11 us of SM time on the
+    // unfused path, so it wins once its waves of 148 heads are at least half
+    // full.  Below 74 heads the unfused state kernel also splits each head's
+    // sequence into segments and wins (measured at d = 128, chunks of 128:
+    // fused faster at 96, 128, 160, 192, 256 and 1024 heads, slower at 64).
+    // The threshold is a constant of the shape (half of a 148-SM B200) so
+    // that the workspace size computed on the host always matches the
+    // algorithm a call picks.
+    constexpr int kFusedMinHeads = 148 / 2;
     if (dt == MLSTM_DT_BF16 && p.T > 0 && allow_fused && tc_fused_supported(p) &&
         p.BH >= kFusedMinHeads) {
       *out = MLSTM_ALGO_TC_FUSED;

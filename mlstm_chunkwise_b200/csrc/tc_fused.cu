@@ -328,19 +328,29 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const int rg = rt / (kDK / 8);
     bool ok = true;
 
-    // Per-chunk row values.  When sep is set the exponent of P splits into a
-    // column factor e^{acol_s - c} (c = the chunk's largest acol, factor
-    // <= 1) and a row factor e^{c - mu_r} that stays below e^60, so P costs
-    // two multiplies per element instead of an exponential.
+    // Per-chunk row values.  Every term of a row may be scaled by a common
+    // factor, so when the exponents allow it (frame) the whole chunk works in
+    // one frame F = m_k (or, with no entering state, c = the chunk's largest
+    // acol): P_rs = s S_rs e^{acol_s - F} is one column factor per key, the
+    // inter-chunk factor e^{m_k - F} is 1 (Q is used as loaded) or 0, and
+    // h_r = O_r / max(|den_r|, e^{-(bcum_r + F)}).  frame needs c - F <= 60
+    // (with F = c, the first row's amax no lower than c - 60) and the floor's
+    // exponent within +-80 over the chunk.  Otherwise, when sep is set, the
+    // exponent of P splits into a column factor e^{acol_s - c} (<= 1) and a
+    // row factor e^{c - mu_r} below e^60 (two multiplies per element); else
+    // each element takes its own exponential.  Without frame the rows use
+    // their own mu_r and Q is scaled by e^{m_k - mu_r}.
     struct Rows {
       float m_in, m_out, mu, bc, gk, decay, rowf;
-      bool sep;
+      float fr;       // the frame of this row: F, or mu_r
+      float f_inter;  // e^{m_k - fr}
+      bool sep, frame, scaleq;
       int bh, td;  // td: dominant token of the chunk's entering state, or -1
     };
     // Gate values of a chunk, loaded two chunks ahead of their use (the
     // loads stay in flight while the chunk in between is processed).
     struct Raw {
-      float m_in, m_out, amax, bc, gk, acol, amax0, amax_last;
+      float m_in, m_out, amax, bc, gk, acol, amax0, amax_last, bc0, bc_last;
       int bh, k, td;
     };
     auto load_raw = [&](const FChunk& c) -> Raw {
@@ -354,6 +364,8 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       v.acol = rt < kL ? g.acol[base + rt] : 0.f;
       v.amax0 = g.amax[base];
       v.amax_last = g.amax[base + kL - 1];
+      v.bc0 = g.bcum[base];
+      v.bc_last = g.bcum[base + kL - 1];  // bcum falls along the chunk
       v.bh = c.bh;
       v.k = c.k;
       v.td = g.dom ? g.dom[(long)c.bh * NC + c.k] : -1;
@@ -374,13 +386,23 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       if (w.td >= 0 && rt < kDK) dstar_s[rt] = dom_residual(g, p, w.bh, w.k, w.td, rt, Kraw);
       const float cmax = w.amax_last;               // max over the chunk (amax is a running max)
       const float mu0 = fmaxf(w.m_in, w.amax0);     // the smallest mu_r of the chunk
-      v.sep = (cmax - mu0) <= 60.f;
+      // one frame for the chunk (uniform: the same loads in every thread)
+      const bool fresh = w.m_in == -INFINITY;
+      const float F = fresh ? cmax : w.m_in;
+      const float spread = fresh ? cmax - w.amax0 : cmax - w.m_in;
+      v.frame = spread <= 60.f && -w.bc_last - F <= 80.f && -w.bc0 - F >= -80.f;
+      v.sep = !v.frame && (cmax - mu0) <= 60.f;
       v.rowf = v.sep ? ks * expf(cmax - v.mu) : 0.f;
+      v.fr = v.frame ? F : v.mu;
+      v.f_inter = expf(w.m_in - v.fr);
+      // Q is scaled unless its factor is 1 (with no entering state it is 0:
+      // a C0 given with m0 = -inf weighs nothing)
+      v.scaleq = !v.frame || fresh;
       if (rt < kL) {
         float* col = acol_s + buf * 3 * kL;
         col[rt] = w.acol;
-        col[kL + rt] = expf(w.acol - cmax);                         // -inf -> 0
-        col[2 * kL + rt] = ks * expf(w.gk + w.acol - w.m_out);      // -inf -> 0
+        col[kL + rt] = v.frame ? ks * expf(w.acol - F) : expf(w.acol - cmax);  // -inf -> 0
+        col[2 * kL + rt] = ks * expf(w.gk + w.acol - w.m_out);              // -inf -> 0
       }
       return v;
     };
@@ -467,9 +489,9 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       uint8_t* qbuf = smem + F::kOffQ + b * F::kQBytes;
       uint8_t* kbuf = smem + F::kOffK + b * F::kKBytes;
       const float* ac = acol_s + b * 3 * kL;   // acol
-      const float* cf = ac + kL;                // e^{acol - c}
+      const float* cf = ac + kL;                // s e^{acol - F} (frame) or e^{acol - c}
       const float* wc = ac + 2 * kL;            // s e^{g + acol - m_out}
-      const float f_inter = expf(rv.m_in - rv.mu);
+      const float f_inter = rv.f_inter;
       const float mu2 = rv.mu * kLog2e;
       // den_inter needs Q(j) and n_j only: it overlaps the S MMA.  (q_full of
       // a buffer completes once per load; the next load of the buffer needs
@@ -517,6 +539,22 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           tmem_ld32(trow + scol + hp * 32, v);
           tmem_wait_ld();
           uint32_t pk[16];
+          if (rv.frame) {
+            uint64_t rs2 = 0;  // two fp32 partial sums, +0
+#pragma unroll
+            for (int e = 0; e < 32; e += 2) {
+              const int s0 = h * 64 + hp * 32 + e;
+              const float2 c2 = *reinterpret_cast<const float2*>(cf + s0);
+              float2 pf = f32x2_split(mul_f32x2(
+                  f32x2(__uint_as_float(v[e]), __uint_as_float(v[e + 1])), f32x2(c2.x, c2.y)));
+              if (s0 > r) pf.x = 0.f;
+              if (s0 + 1 > r) pf.y = 0.f;
+              rs2 = add_f32x2(rs2, f32x2(pf.x, pf.y));
+              pk[e >> 1] = pack_bf16x2(pf.x, pf.y);
+            }
+            const float2 r2 = f32x2_split(rs2);
+            rs += r2.x + r2.y;
+          } else {
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
             const int s0 = h * 64 + hp * 32 + e;
@@ -533,12 +571,13 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             rs += pa + pb;
             pk[e >> 1] = pack_bf16x2(pa, pb);
           }
+          }
           tmem_st16(trow + scol + hp * 16, pk);
         }
         den += rs;
       }
-      // Q~ = e^{m_k - mu_r} q_r in place (slab h)
-      {
+      // Q~ = e^{m_k - mu_r} q_r in place (slab h); with one frame Q stays
+      if (rv.scaleq) {
         uint8_t* slab = qbuf + h * 16384;
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
@@ -599,7 +638,7 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const float2 other = red_s[rt ^ 128];
       const float den = den_part.x + other.x;
       // the plain sigmoid variant has no normaliser: h = e^{m_r} O
-      const float mr = rv.bc + rv.mu;
+      const float mr = rv.bc + rv.fr;  // the floor's exponent in the chunk's frame
       const float inv = p.no_norm ? expf(mr) : 1.f / fmaxf(fabsf(den), expf(-mr));
       ok = ok && mbar_wait(bar.o_full(), j & 1, p, 9);  // Q~.C(j) done: Q(j) free
       tc_fence_after();
@@ -608,7 +647,7 @@ tc_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       if (kHalfV >= 64) tmem_ld32(trow + kColO + h * kHalfV + 32, v1);
       tmem_wait_ld();
       if (rv.td >= 0) {  // a dominated chunk's rank-one part, (n_j^T q~_r) v_{t*}
-        const float c1 = expf(rv.m_in - rv.mu) * (den_part.y + other.y);
+        const float c1 = rv.f_inter * (den_part.y + other.y);
         const __nv_bfloat16* vstar = Vraw + ((long)c.bh * p.T + rv.td) * DV + h * kHalfV;
         add_rank1_32(v0, c1, vstar);
         if (kHalfV >= 64) add_rank1_32(v1, c1, vstar + 32);
