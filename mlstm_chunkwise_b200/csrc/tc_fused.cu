@@ -14,6 +14,9 @@
 //   C_{k+1} = e^{g_k + m_k - m_{k+1}} C_k + (w K_k)^T V_k,  w_s = s e^{g_k + acol_s - m_{k+1}}
 //   n_{k+1} = the same with V -> 1 (fp32, from the unrounded products w_s k_s)
 //
+// (Where the gates allow, a chunk uses one frame F for all rows instead of
+// mu_r -- F = m_k, so Q~ = Q -- see the row values below.)
+//
 // The fp32 master state C lives in TMEM for the whole sequence of a head; the
 // Q~ C_k MMA reads a bf16 copy of it that the row threads write into shared
 // memory once per chunk (together with the decay of the master).  The n
