@@ -202,3 +202,22 @@ def test_train_pair_rejects_before_launch(L):
     assert bw_call(saved_bytes=sv - 1) == _lib.ERR_INVALID_ARG
     assert bw_call(ws_bytes=bw - 1) == _lib.ERR_INVALID_ARG
     assert bw_call(h=None) == _lib.ERR_INVALID_ARG
+
+
+def test_auto_picks_fused_from_half_the_sms(L):
+    """AUTO takes the fused kernel from 74 (b, h) pairs up (half of a 148-SM
+    B200) where it supports the shape, else the unfused tensor-core path; the
+    rule depends on the shape alone, so the workspace AUTO asks for is that of
+    the algorithm it runs (checked here without a GPU, through the sizes)."""
+    kw = dict(T=1024, DK=128, DV=128, L=128, dt=_lib.DT_BF16)
+    for NH, expect in ((73, _lib.ALGO_TC), (74, _lib.ALGO_TC_FUSED), (600, _lib.ALGO_TC_FUSED)):
+        st_a, n_auto = ws(B=1, NH=NH, algo=_lib.ALGO_AUTO, **kw)
+        st_e, n_exp = ws(B=1, NH=NH, algo=expect, **kw)
+        st_o, n_other = ws(B=1, NH=NH, algo=_lib.ALGO_TC_FUSED + _lib.ALGO_TC - expect, **kw)
+        assert st_a == st_e == st_o == _lib.OK
+        assert n_other != n_exp, "the two paths need different workspaces"
+        assert n_auto == n_exp, (NH, n_auto, n_exp)
+    # shapes the fused kernel does not take stay unfused at any head count
+    st_a, n_auto = ws(B=1, NH=600, T=1024, DK=128, DV=128, L=256, algo=_lib.ALGO_AUTO)
+    st_t, n_tc = ws(B=1, NH=600, T=1024, DK=128, DV=128, L=256, algo=_lib.ALGO_TC)
+    assert st_a == st_t == _lib.OK and n_auto == n_tc
