@@ -578,8 +578,10 @@ def run_ours(args):
     # on two copy streams (the link is full duplex) into double-buffered device
     # buffers, so step i's inputs travel while step i - 1 computes and step
     # i - 2's outputs travel back; the timed region spans the first input copy
-    # to the last output copy.
-    e2e_steps = max(1, min(args.steps, 10))
+    # to the last output copy.  At least 30 steps (up to 60) when --steps
+    # allows, so that the pipeline's fill (the first copy in) and drain (the
+    # last copy out) are spread over a run closer to steady streaming.
+    e2e_steps = max(1, min(max(args.steps, 30), 60)) if args.steps >= 3 else max(1, args.steps)
     e2e_ms = float("nan")
     h2d = d2h = 0
     if not args.no_e2e:
